@@ -1,0 +1,321 @@
+"""Pins of the CPU oracle to things other than itself.
+
+The pages print no worked numeric example of the layer, so the oracle is pinned by
+(a) the hand-stepped tie rule of the routing scan printed on www.mhpq.cn/news/563172 §3.2
+(tests/golden/topk_tie_rule.txt), (b) closed forms (k = 2 weights are a logistic of the
+logit gap; k = E weights are the textbook softmax), (c) library routines on special cases
+(float64 matmul for the router, float64 torch SwiGLU for E = k = 1, a stable sort for the
+grouping permutation), (d) a brute-force dense "run every expert on every token, then mask"
+restatement of the whole layer, and (e) invariants (k distinct experts per token, weights
+non-negative summing to one, the permutation a bijection matching the histogram).
+Each is chosen so that a dropped term, a wrong sign or index, or a transposed operand in
+the oracle fails at least one of them.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+import torch.nn.functional as F
+
+import inputgen
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ------------------------------------------------------------------------- helpers
+
+
+def _f64(t):
+    return t.to(torch.float64).numpy()
+
+
+def _ref_select(logits, k):
+    """Brute force: sort every row by (value descending, index ascending)."""
+    T, E = logits.shape
+    out = np.empty((T, k), dtype=np.int64)
+    for t in range(T):
+        order = np.lexsort((np.arange(E), -logits[t].astype(np.float64)))
+        out[t] = order[:k]
+    return out
+
+
+def _expert_mats(p, e):
+    """W1, W3, W2 of expert e as float64 numpy (int8 dequantised as float32 s*q)."""
+    wl = p.wl
+    d, f = wl.d, wl.f
+    base = e * p.expert_stride
+    raw = p.expert_w[base: base + 3 * f * d]
+    if wl.wdt == inputgen.I8:
+        s = p.expert_scales[e * (2 * f + d):(e + 1) * (2 * f + d)]
+        q = raw.to(torch.float32)
+        w1 = (s[:f, None] * q[: f * d].view(f, d))
+        w3 = (s[f:2 * f, None] * q[f * d: 2 * f * d].view(f, d))
+        w2 = (s[2 * f:, None] * q[2 * f * d:].view(d, f))
+    else:
+        w1 = raw[: f * d].view(f, d)
+        w3 = raw[f * d: 2 * f * d].view(f, d)
+        w2 = raw[2 * f * d:].view(d, f)
+    return _f64(w1), _f64(w3), _f64(w2)
+
+
+def _swiglu(x, w1, w3, w2):
+    g = x @ w1.T
+    u = x @ w3.T
+    return (g / (1.0 + np.exp(-g)) * u) @ w2.T
+
+
+def _dense_layer(p):
+    """Every expert on every token, combined through a masked [T, E] weight matrix."""
+    wl = p.wl
+    x = _f64(p.x)
+    wr = _f64(p.router_w)
+    logits = x @ wr.T
+    if p.router_b is not None:
+        logits = logits + _f64(p.router_b)
+    sel = _ref_select(logits.astype(np.float32), wl.k)
+    mask = np.zeros((wl.T, wl.E))
+    for t in range(wl.T):
+        ls = logits[t, sel[t]]
+        mask[t, sel[t]] = np.exp(ls - ls.max()) / np.exp(ls - ls.max()).sum()
+    y = np.zeros((wl.T, wl.d))
+    for e in range(wl.E):
+        y += mask[:, e:e + 1] * _swiglu(x, *_expert_mats(p, e))
+    if wl.fs:
+        fs, d = wl.fs, wl.d
+        sw = p.shared_w
+        y += _swiglu(x, _f64(sw[: fs * d].view(fs, d)), _f64(sw[fs * d: 2 * fs * d].view(fs, d)),
+                     _f64(sw[2 * fs * d:].view(d, fs)))
+    return y, sel, mask
+
+
+def _rel_err(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return np.abs(a - b).max() / max(np.abs(b).max(), 1e-30)
+
+
+# ------------------------------------------------------------------------- top-k
+
+
+def test_topk_tie_rule_golden():
+    with open(os.path.join(GOLDEN, "topk_tie_rule.txt")) as fh:
+        rows = [l.strip() for l in fh if l.strip() and not l.startswith("#")]
+    for row in rows:
+        lhs, rhs = row.split("|")
+        logits = torch.tensor([[float(v) for v in lhs.split()]], dtype=torch.float32)
+        want = [int(v) for v in rhs.split()]
+        idx, _, _ = oracle.topk(logits, 2)
+        assert idx[0].tolist() == want, row
+
+
+@pytest.mark.parametrize("E,k", [(8, 2), (16, 4), (128, 8), (5, 5), (64, 1)])
+def test_topk_brute_force_with_ties(E, k):
+    T = 257
+    v = inputgen.fill_normal(torch.empty(T * E), 0, 40 + E, 1.0)
+    logits = (torch.round(v * 4) / 4).view(T, E)  # coarse grid: many exact ties
+    idx, _, gap = oracle.topk(logits, k)
+    assert np.array_equal(idx.numpy(), _ref_select(logits.numpy(), k))
+    # each token has k distinct experts
+    for t in range(T):
+        assert len(set(idx[t].tolist())) == k
+    if k < E:
+        srt = -np.sort(-logits.numpy(), axis=1)
+        assert np.allclose(gap.numpy(), srt[:, k - 1] - srt[:, k])
+
+
+# ------------------------------------------------------------------------- weights
+
+
+def test_weights_k_equals_E_is_textbook_softmax():
+    T, E = 33, 6
+    logits = inputgen.fill_normal(torch.empty(T * E), 1, 5, 2.0).view(T, E)
+    idx, w, _ = oracle.topk(logits, E)
+    sm = scipy.special.softmax(logits.numpy().astype(np.float64), axis=1)
+    assert np.allclose(w.numpy(), np.take_along_axis(sm, idx.numpy().astype(np.int64), 1), rtol=1e-6, atol=0)
+
+
+def test_weights_k2_closed_form_logistic():
+    T, E = 100, 8
+    logits = inputgen.fill_normal(torch.empty(T * E), 2, 6, 1.5).view(T, E)
+    idx, w, _ = oracle.topk(logits, 2)
+    l = logits.numpy().astype(np.float64)
+    l0 = l[np.arange(T), idx[:, 0].numpy()]
+    l1 = l[np.arange(T), idx[:, 1].numpy()]
+    assert np.allclose(w[:, 0].numpy(), 1.0 / (1.0 + np.exp(l1 - l0)), rtol=1e-6, atol=0)
+    assert np.allclose(w[:, 1].numpy(), 1.0 / (1.0 + np.exp(l0 - l1)), rtol=1e-6, atol=0)
+
+
+def test_weights_k1_is_one_and_invariants():
+    T, E = 50, 16
+    logits = inputgen.fill_normal(torch.empty(T * E), 3, 7, 3.0).view(T, E)
+    _, w1, _ = oracle.topk(logits, 1)
+    assert torch.all(w1 == 1.0)
+    for k in (2, 3, 8):
+        _, w, _ = oracle.topk(logits, k)
+        assert torch.all(w >= 0)
+        assert torch.all((w.double().sum(1) - 1).abs() <= 1e-6)
+        assert torch.all(w[:, :-1] >= w[:, 1:])  # slot order follows the logits
+
+
+def test_weights_for_other_selection_matches_softmax_subset():
+    T, E, k = 20, 8, 3
+    logits = inputgen.fill_normal(torch.empty(T * E), 4, 8, 1.0).view(T, E)
+    idx = torch.tensor([[(t + j * 3) % E for j in range(k)] for t in range(T)], dtype=torch.int32)
+    w = oracle.weights_for(logits, idx)
+    l = logits.numpy().astype(np.float64)
+    for t in range(T):
+        sub = scipy.special.softmax(l[t, idx[t].numpy()])
+        assert np.allclose(w[t].numpy(), sub, rtol=1e-6, atol=0)
+
+
+# ------------------------------------------------------------------------- router
+
+
+@pytest.mark.parametrize("act", [inputgen.F32, inputgen.BF16])
+def test_router_logits_vs_float64_matmul(act):
+    wl = inputgen.custom("r", T=37, d=96, E=12, k=2, f=8, act=act, wdt=act)
+    p = inputgen.make_problem(wl, seed=1)
+    b = inputgen.fill_normal(torch.empty(12), 1, 77, 0.3)
+    got = oracle.router_logits(p.x, p.router_w, b)
+    want = _f64(p.x) @ _f64(p.router_w).T + _f64(b)
+    assert got.shape == (37, 12)
+    assert _rel_err(got.numpy(), want) < 1e-6
+    # without bias
+    got0 = oracle.router_logits(p.x, p.router_w, None)
+    assert _rel_err(got0.numpy(), _f64(p.x) @ _f64(p.router_w).T) < 1e-6
+
+
+# ------------------------------------------------------------------------- grouping
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 4, 2), (300, 8, 2), (129, 128, 4), (64, 3, 3)])
+def test_group_is_stable_counting_sort(T, E, k):
+    logits = inputgen.fill_normal(torch.empty(T * E), 5, T + E, 1.0).view(T, E)
+    idx, _, _ = oracle.topk(logits, k)
+    counts, offsets, src, dst = oracle.group(idx, E)
+    flat = idx.numpy().reshape(-1).astype(np.int64)
+    assert np.array_equal(counts.numpy(), np.bincount(flat, minlength=E))
+    assert offsets[0] == 0 and offsets[-1] == T * k
+    assert np.all(np.diff(offsets.numpy()) == counts.numpy())
+    # a stable sort of the flattened (t, j) assignments by expert gives the same rows
+    perm = np.argsort(flat, kind="stable")
+    assert np.array_equal(src.numpy(), perm // k)
+    # dst is the inverse permutation and lands inside the right expert's range
+    assert np.array_equal(np.sort(dst.numpy().reshape(-1)), np.arange(T * k))
+    for t in range(T):
+        for j in range(k):
+            r = int(dst[t, j])
+            e = int(idx[t, j])
+            assert src[r] == t and offsets[e] <= r < offsets[e + 1]
+    # each token appears exactly k times
+    assert np.array_equal(np.bincount(src.numpy(), minlength=T), np.full(T, k))
+
+
+# ------------------------------------------------------------------------- expert FFN / layer
+
+
+@pytest.mark.parametrize("act", [inputgen.F32, inputgen.BF16])
+def test_single_expert_is_dense_swiglu(act):
+    # E = 1, k = 1: the layer is one dense SwiGLU FFN (torch float64, F.silu)
+    wl = inputgen.custom("dense", T=9, d=48, E=1, k=1, f=80, act=act, wdt=act)
+    p = inputgen.make_problem(wl, seed=2)
+    out = oracle.moe_forward(p.x, p.router_w, p.router_b, 1, p.expert_w, p.expert_stride, wl.f)
+    assert torch.all(out["w"] == 1.0) and torch.all(out["idx"] == 0)
+    x = p.x.to(torch.float64)
+    w = p.expert_w.to(torch.float64)
+    f, d = wl.f, wl.d
+    w1, w3, w2 = w[: f * d].view(f, d), w[f * d: 2 * f * d].view(f, d), w[2 * f * d: 3 * f * d].view(d, f)
+    want = (F.silu(x @ w1.T) * (x @ w3.T)) @ w2.T
+    assert _rel_err(out["y"].numpy(), want.numpy()) < 2e-6
+
+
+@pytest.mark.parametrize("case", ["f32", "bf16", "bf16_shared", "bf16_bias", "i8"])
+def test_layer_equals_brute_force_dense(case):
+    kw = dict(T=23, d=64, E=6, k=2, f=96)
+    if case == "f32":
+        wl = inputgen.custom(case, act=inputgen.F32, wdt=inputgen.F32, **kw)
+    elif case == "bf16":
+        wl = inputgen.custom(case, **kw)
+    elif case == "bf16_shared":
+        wl = inputgen.custom(case, fs=40, **dict(kw, k=3))
+    elif case == "bf16_bias":
+        wl = inputgen.custom(case, bias=((1, 2.0), (4, -1.0)), **kw)
+    else:
+        wl = inputgen.custom(case, act=inputgen.BF16, wdt=inputgen.I8, **kw)
+    p = inputgen.make_problem(wl, seed=3)
+    out = oracle.moe_forward(p.x, p.router_w, p.router_b, wl.k, p.expert_w, p.expert_stride, wl.f,
+                             p.expert_scales, p.shared_w, wl.fs)
+    y, sel, mask = _dense_layer(p)
+    assert np.array_equal(out["idx"].numpy(), sel)
+    assert _rel_err(out["y"].numpy(), y) < 2e-6
+    # the sampled path agrees bit for bit with the whole-layer path
+    toks = [0, 5, 22, 11]
+    ys = oracle.combine(p.x, out["idx"], out["w"], p.expert_w, p.expert_stride, wl.f, p.expert_scales,
+                        p.shared_w, wl.fs, toks)
+    assert torch.equal(ys, out["y"][toks])
+
+
+def test_int8_dequant_identity():
+    # the oracle on (s, q) equals the oracle on float32 weights s[o] * q[o][i]
+    wl = inputgen.custom("i8", T=11, d=32, E=3, k=2, f=48, act=inputgen.BF16, wdt=inputgen.I8)
+    p = inputgen.make_problem(wl, seed=4)
+    f, d = wl.f, wl.d
+    deq = torch.zeros(3 * p.expert_stride, dtype=torch.float32)
+    for e in range(3):
+        s = p.expert_scales[e * (2 * f + d):(e + 1) * (2 * f + d)]
+        q = p.expert_w[e * p.expert_stride: e * p.expert_stride + 3 * f * d].to(torch.float32)
+        rows = torch.cat([s[:f].repeat_interleave(d), s[f:2 * f].repeat_interleave(d), s[2 * f:].repeat_interleave(f)])
+        deq[e * p.expert_stride: e * p.expert_stride + 3 * f * d] = rows * q
+    a = oracle.moe_forward(p.x, p.router_w, None, 2, p.expert_w, p.expert_stride, f, p.expert_scales)
+    b = oracle.moe_forward(p.x, p.router_w, None, 2, deq, p.expert_stride, f)
+    assert torch.equal(a["y"], b["y"])
+
+
+def test_tiny_f32_workload_float64_restatement():
+    # the full 64-token fp32 workload against an independent float64 torch restatement
+    wl = inputgen.WORKLOADS["tiny_f32"]
+    p = inputgen.make_problem(wl, seed=0)
+    out = oracle.problem_forward(p)
+    y, sel, _ = _dense_layer(p)
+    assert np.array_equal(out["idx"].numpy(), sel)
+    assert _rel_err(out["y"].numpy(), y) < 2e-6
+
+
+def test_empty_and_nonfinite():
+    wl = inputgen.custom("z", T=0, d=16, E=4, k=2, f=16)
+    p = inputgen.make_problem(wl, seed=0)
+    out = oracle.moe_forward(p.x, p.router_w, None, 2, p.expert_w, p.expert_stride, 16)
+    assert out["y"].numel() == 0
+    wl = inputgen.custom("nf", T=3, d=16, E=4, k=2, f=16, act=inputgen.F32, wdt=inputgen.F32)
+    p = inputgen.make_problem(wl, seed=0)
+    p.x[1, 3] = float("nan")
+    with pytest.raises(RuntimeError):
+        oracle.moe_forward(p.x, p.router_w, None, 2, p.expert_w, p.expert_stride, 16)
+
+
+def test_bad_arguments_rejected():
+    logits = torch.zeros(2, 4)
+    with pytest.raises(RuntimeError):
+        oracle.topk(logits, 5)  # k > E
+    with pytest.raises(RuntimeError):
+        oracle.group(torch.tensor([[0, 7]], dtype=torch.int32), 4)  # expert id out of range
+
+
+@pytest.mark.slow
+def test_skewed_workload_histogram():
+    # +4 bias on experts 0/1 concentrates almost every assignment there; the variant with
+    # -30 on experts 12..15 leaves those four experts with exactly zero rows.
+    for name in ("skewed_bf16", "skewed_empty_bf16"):
+        wl = inputgen.WORKLOADS[name]
+        p = inputgen.make_problem(wl, seed=0)
+        logits = oracle.router_logits(p.x, p.router_w, p.router_b)
+        idx, _, _ = oracle.topk(logits, wl.k)
+        counts, _, _, _ = oracle.group(idx, wl.E)
+        frac01 = (counts[0] + counts[1]).item() / (wl.T * wl.k)
+        assert frac01 > 0.9
+        if name == "skewed_empty_bf16":
+            assert counts[12:].sum().item() == 0
