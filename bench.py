@@ -1,0 +1,353 @@
+#!/usr/bin/env python3
+"""Benchmark: MoE-layer forward tokens/s and fraction of roofline on B200.
+
+One step = one call of colibri_moe_forward over one batch (all stages: Gate, Scatter,
+Expert Compute, Gather).  Default workload: the Mixtral-shaped prefill layer (T=4096,
+d_model=4096, 8 experts, top-2, SwiGLU d_ff=14336, bf16).  Inputs are seeded synthetic
+tensors (random-init weights); the 2.8 GB of expert weights streamed per step is far larger
+than L2, so no explicit flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl colibri|reference]
+
+With --gpus N > 1 (launched by torch.distributed.run) every rank runs an independent replica
+of the workload on its own GPU (weak scaling; the layer has no exchange step when tokens
+are data-parallel); timing is the max over ranks.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/sec (prefill & decode) and % of roofline on 1 B200"
+DEFAULT_WORKLOAD = "mixtral_prefill_bf16"
+KERNELS_PER_STEP_BASE = 7  # router, count, scan, scatter, gate/up, down, combine
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="colibri", choices=["colibri", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-sample-tokens", type=int, default=None,
+                    help="tokens of the CPU-baseline sample (default sized for ~10-30 s)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args()
+    a.warmup = max(a.warmup, 3)
+    return a
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            pk = json.load(fh)
+        return dict(hbm=pk["hbm_gbs"], bf16=pk["bf16_tflops"], bf16_sus=pk.get("bf16_tflops_sustained"),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+def work(wl, counts):
+    """Algorithmic work of one call: only the k chosen experts per token, plus the shared expert."""
+    rows = wl.T * wl.k
+    d, f, fs = wl.d, wl.f, wl.fs
+    wsize = {0: 4, 1: 2, 2: 1}[wl.wdt]
+    touched = sum(1 for c in counts if c > 0)
+    flops_gateup = 2.0 * rows * d * 2 * f + 2.0 * wl.T * d * 2 * fs
+    flops_down = 2.0 * rows * f * d + 2.0 * wl.T * fs * d
+    flops_router = 2.0 * wl.T * d * wl.E
+    w13_bytes = touched * 2 * f * d * wsize + (2 * fs * d * wsize if fs else 0)
+    w2_bytes = touched * d * f * wsize + (fs * d * wsize if fs else 0)
+    scale_bytes = touched * (2 * f + d) * 4 if wl.wdt == 2 else 0
+    return dict(flops_gateup=flops_gateup, flops_down=flops_down, flops_router=flops_router,
+                flops=flops_gateup + flops_down + flops_router, w13_bytes=w13_bytes, w2_bytes=w2_bytes,
+                scale_bytes=scale_bytes, touched=touched)
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle sampling every 200 ms during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.samples = []
+        if self.proc is None:
+            return False
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append(parts)
+        return False
+
+    def summary(self):
+        s = getattr(self, "samples", [])
+        if not s:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+
+        sm = [num(p[1]) for p in s if num(p[1]) is not None]
+        mx = [num(p[2]) for p in s if num(p[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for p in s for n, v in zip(names, p[5:9]) if v.strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(s)}
+
+
+def cpu_baseline(p, n_tokens, seed_tokens=None):
+    """The oracle, as it stands, on a bounded sample: routing for every token, the expert FFN
+    and combine for n_tokens tokens spread over the batch; tokens/s extrapolated per token."""
+    import oracle
+    from inputgen import sample_tokens
+
+    wl = p.wl
+    t0 = time.perf_counter()
+    logits = oracle.router_logits(p.x, p.router_w, p.router_b)
+    idx, w, _ = oracle.topk(logits, wl.k)
+    oracle.group(idx, wl.E)
+    t_route = time.perf_counter() - t0
+    toks = seed_tokens or sample_tokens(wl.T, n_tokens)
+    t0 = time.perf_counter()
+    oracle.combine(p.x, idx, w, p.expert_w, p.expert_stride, wl.f, p.expert_scales, p.shared_w, wl.fs, toks)
+    t_ffn = time.perf_counter() - t0
+    per_token = t_route / wl.T + t_ffn / len(toks)
+    return dict(value=1.0 / per_token, unit="tokens/s", cores=1, kind="oracle",
+                sample=f"routing (logits, top-k, grouping) of all {wl.T} tokens in {t_route:.2f} s; expert FFN + "
+                       f"combine of {len(toks)} tokens spread over the batch in {t_ffn:.2f} s; tokens/s = 1 / "
+                       f"(routing time per token + FFN time per token), single-threaded C++ oracle",
+                seconds=t_route + t_ffn)
+
+
+def default_sample(wl):
+    per_token_macs = wl.k * 3 * wl.d * wl.f + 3 * wl.d * wl.fs
+    # ~0.4 s per 3.5e8 multiply-adds on one core -> aim at ~12 s
+    return int(max(2, min(wl.T, round(12.0 / (per_token_macs / 3.5e8 * 0.4)))))
+
+
+def run_reference(a, rank, world):
+    """--impl reference: the oracle on the host cores, rank 0 only, bounded sample per step."""
+    if rank != 0:
+        return 0
+    import inputgen
+    import oracle
+
+    wl = inputgen.WORKLOADS[a.workload]
+    p = inputgen.make_problem(wl, seed=a.seed)
+    sample_tokens = inputgen.sample_tokens
+    n = max(1, min(wl.T, (a.cpu_sample_tokens or max(1, default_sample(wl) // 4))))
+    toks = sample_tokens(wl.T, n)
+    logits = oracle.router_logits(p.x, p.router_w, p.router_b)
+    idx, w, _ = oracle.topk(logits, wl.k)
+
+    def step():
+        # routing for the sampled tokens, then their FFN and combine
+        rows = p.x[toks].contiguous()
+        lg = oracle.router_logits(rows, p.router_w, p.router_b)
+        oracle.topk(lg, wl.k)
+        oracle.combine(p.x, idx, w, p.expert_w, p.expert_stride, wl.f, p.expert_scales, p.shared_w, wl.fs, toks)
+
+    for _ in range(a.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(a.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = len(toks) * a.steps / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": dt / a.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(wl),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: routing and expert FFN + combine of {len(toks)} of the {wl.T} "
+                                   f"tokens (single-threaded C++ oracle, double accumulation)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(wl):
+    cfg = {"workload": wl.name, "T": wl.T, "d_model": wl.d, "num_experts": wl.E, "top_k": wl.k, "d_ff": wl.f,
+           "act_dtype": {0: "f32", 1: "bf16"}[wl.act], "weight_dtype": {0: "f32", 1: "bf16", 2: "i8"}[wl.wdt]}
+    if wl.fs:
+        cfg["shared_d_ff"] = wl.fs
+    if wl.bias:
+        cfg["router_bias"] = {str(e): v for e, v in wl.bias}
+    return cfg
+
+
+def main():
+    a = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if a.impl == "reference":
+        return run_reference(a, rank, world)
+
+    import torch
+    import torch.distributed as dist
+
+    import inputgen
+    import sparse_expert_ffn_router_b200 as colibri
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    wl = inputgen.WORKLOADS[a.workload]
+    p = inputgen.make_problem(wl, seed=a.seed, pin=True)
+    dev = torch.device("cuda", local)
+    x = p.x.to(dev)
+    rw = p.router_w.to(dev)
+    rb = None if p.router_b is None else p.router_b.to(dev)
+    ew = p.expert_w.to(dev)
+    sc = None if p.expert_scales is None else p.expert_scales.to(dev)
+    sw = None if p.shared_w is None else p.shared_w.to(dev)
+    y = torch.empty(wl.T, wl.d, dtype=x.dtype, device=dev)
+    layer = colibri.MoELayer(wl.d, wl.f, wl.E, wl.k, wl.fs, wl.act, wl.wdt, max_tokens=wl.T, device_id=local)
+    assert layer.expert_stride == p.expert_stride
+    stream = torch.cuda.current_stream(dev)
+
+    def step(xin, yout):
+        colibri.colibri_moe_forward(layer.ctx, xin, wl.T, rw, rb, ew, sc, sw, yout, stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(a.warmup):
+        step(x, y)
+    layer.sync_status()
+    counts = torch.empty(wl.E, dtype=torch.int32, device=dev)
+    colibri.colibri_get_routing(layer.ctx, counts=counts, stream=stream)
+    counts = counts.cpu().tolist()
+    wk = work(wl, counts)
+
+    # ---- device-resident timed region
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    colibri.colibri_profile_begin(layer.ctx, a.steps)
+    barrier()
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(a.steps):
+            step(x, y)
+        ev1.record(stream)
+        barrier()
+    stage_ms, ncalls = colibri.colibri_profile_end(layer.ctx)
+    layer.sync_status()
+    ms_total = ev0.elapsed_time(ev1)
+    t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    value = world * wl.T * a.steps / (ms_max / 1e3)
+
+    # ---- end to end through the same call with host buffers (pinned x in, y out)
+    x_host = p.x.pin_memory() if not p.x.is_pinned() else p.x
+    y_host = torch.empty(wl.T, wl.d, dtype=x.dtype).pin_memory()
+    for _ in range(2):
+        step(x_host, y_host)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(a.steps):
+        step(x_host, y_host)
+    e1.record(stream)
+    barrier()
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = world * wl.T * a.steps / (float(te.item()) / 1e3)
+    row_bytes = wl.d * (4 if wl.act == 0 else 2)
+
+    # ---- roofline of the dominant kernel (per-launch averages over the timed region)
+    pk = peaks()
+    per_call = {k: v / max(ncalls, 1) for k, v in stage_ms.items()}
+    if wl.wdt == 2:
+        achieved = (wk["w13_bytes"] + wk["scale_bytes"]) / (per_call["expert_gateup"] / 1e3) / 1e9
+        roof = {"kernel": "dec_gateup_kernel (int8 weight stream, gate/up)", "bound": "hbm",
+                "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s", "frac": achieved / pk["hbm"],
+                "algorithmic_bytes_per_launch": wk["w13_bytes"] + wk["scale_bytes"]}
+    elif wl.wdt == 1:
+        achieved = wk["flops_gateup"] / (per_call["expert_gateup"] / 1e3) / 1e12
+        roof = {"kernel": "tc_ffn_kernel<gate/up> (tcgen05)", "bound": "tensor", "achieved": achieved,
+                "peak": pk["bf16"], "unit": "TFLOP/s", "frac": achieved / pk["bf16"],
+                "algorithmic_flops_per_launch": wk["flops_gateup"]}
+    else:
+        achieved = wk["flops_gateup"] / (per_call["expert_gateup"] / 1e3) / 1e12
+        roof = {"kernel": "simt_ffn_kernel<gate/up> (fp32 FMA)", "bound": "alu", "achieved": achieved,
+                "peak": 148 * 128 * 2 * 1.965, "unit": "TFLOP/s",
+                "frac": achieved / (148 * 128 * 2 * 1.965), "algorithmic_flops_per_launch": wk["flops_gateup"]}
+    roof["peak_source"] = pk["source"] + (" burst" if roof["bound"] == "tensor" else "")
+    roof["traffic"] = None
+    kernels = KERNELS_PER_STEP_BASE + (2 if (wl.fs and wl.wdt == 0) else 0)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": ms_max / a.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": {0: "f32", 1: "bf16", 2: "bf16"}[wl.act],
+        "data": "synthetic (seeded SplitMix64 + Box-Muller inputs, random-init weights)",
+        "config": dict(config_of(wl), l2="inputs larger than L2: %.2f GB of expert weights per step" %
+                       ((wk["w13_bytes"] + wk["w2_bytes"]) / 1e9), parallelism=f"replicas x{world}"),
+        "roofline": roof,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": wl.T * row_bytes,
+                "d2h_bytes_per_step": wl.T * row_bytes},
+        "gpu_launches": kernels * a.steps,
+        "clocks": clk.summary(),
+        "stage_ms_per_call": per_call,
+        "tflops_per_gpu_layer": wk["flops"] * a.steps / (ms_max / 1e3) / 1e12,
+        "routing_counts": counts,
+    }
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        n = a.cpu_sample_tokens or default_sample(wl)
+        line["cpu_baseline"] = cpu_baseline(p, n)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    layer.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

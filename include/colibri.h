@@ -1,0 +1,204 @@
+/*
+ * colibri.h -- C ABI of the B200 (sm_100a) MoE layer forward.
+ *
+ * One call runs the four stages of a sparse Mixture-of-Experts FFN layer:
+ *   Gate     router logits x . Wr^T (+ b), softmax, top-k with lowest-index tie-break
+ *   Scatter  per-expert histogram, prefix sum, stable permutation of token rows
+ *   Expert   grouped SwiGLU FFN per expert: W2_e (silu(W1_e x) * (W3_e x))
+ *   Gather   y[t] = sum_j w[t][j] * FFN_{idx[t][j]}(x_t)  (+ shared expert FFN(x_t))
+ *
+ * The method is the one the "Colibri" MoE engine pages describe:
+ *   www.0539edu.com/news/4774449  §2.2 (Gate -> Scatter -> Expert Compute -> Gather, one custom
+ *                                 kernel per stage; expert weights stored contiguously per expert)
+ *   www.hotelren.com/news/4731937 §2.1 (router logits, top-k, dispatch, k GEMMs, weighted sum),
+ *                                 §2.3 (init / infer / free C API over plain structs)
+ *   www.mhpq.cn/news/563172       §2.1 (fixed stride per expert), §3.2 (top-k scan, ties keep
+ *                                 the lower index), §4.3 (colibri_get_error)
+ *   www.pptc.cn/news/100465       §3.3 (expert_offsets over one weight buffer), §3.4 ([batch][k]
+ *                                 routing layout), §4.1 (colibri_moe_forward over device pointers)
+ *   www.trdm.cn/news/555962       §6.2 (group tokens by the expert they activate)
+ *
+ * Conventions for every entry point
+ *   - Return a colibri_status; nothing is printed unless COLIBRI_DEBUG=1 is set in the
+ *     environment.  colibri_last_error() returns a one-line reason for the last failure.
+ *   - Arguments are validated on the host before anything is launched.
+ *   - Work is enqueued on the caller's CUDA stream (passed as void*; NULL = legacy default
+ *     stream) and the call returns without synchronising, except where stated.
+ *   - The caller owns every tensor it passes.  The context owns only the workspace it
+ *     allocates in colibri_init and frees in colibri_free.
+ *   - One context serves one forward at a time: calls that overlap on the GPU (for example on
+ *     two streams) share the workspace and race.
+ *   - Not re-entrant from several host threads on one context.
+ */
+#ifndef COLIBRI_H_
+#define COLIBRI_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  COLIBRI_OK = 0,
+  COLIBRI_ERR_INVALID_ARG = -1, /* NULL pointer, size out of range, bad dtype combination    */
+  COLIBRI_ERR_ALIGNMENT = -2,   /* a tensor is not 16-byte aligned                           */
+  COLIBRI_ERR_UNSUPPORTED = -3, /* valid request the library does not implement              */
+  COLIBRI_ERR_OOM = -4,         /* workspace allocation failed in colibri_init               */
+  COLIBRI_ERR_CUDA = -5,        /* a CUDA runtime/driver call or a launch failed             */
+  COLIBRI_ERR_TIMEOUT = -6      /* a device-side wait gave up (reported by colibri_sync_status) */
+} colibri_status;
+
+typedef enum { COLIBRI_F32 = 0, COLIBRI_BF16 = 1, COLIBRI_I8 = 2 } colibri_dtype;
+
+/*
+ * Layer description, fixed for the life of a context.
+ *   d_model, d_ff   hidden size d and routed-expert FFN size f; both multiples of 64.
+ *   num_experts     E, 1..256.
+ *   top_k           k, 1..min(E, 8).
+ *   shared_d_ff     f_s of one always-on shared SwiGLU expert added with weight 1, or 0 for
+ *                   none; a multiple of 64 (www.0539edu.com/news/4774449 §2.2 names the
+ *                   shared-expert-augmented variant).
+ *   act_dtype       dtype of x, router weights and y: COLIBRI_F32 or COLIBRI_BF16.
+ *   weight_dtype    dtype of the expert weights.  Supported pairs (act, weight):
+ *                   (F32, F32)   fp32 throughout (SIMT FMA; no TF32);
+ *                   (BF16, BF16) bf16 operands, fp32 accumulation on tcgen05 tensor cores;
+ *                   (BF16, I8)   int8 weights with per-output-channel fp32 scales,
+ *                                dequantised inside the kernel (weight-streaming path).
+ *                   The shared expert is available for (F32, F32) and (BF16, BF16).
+ *   max_tokens      largest T a forward may be called with (sizes the workspace).
+ *   device_id       CUDA device the context lives on.
+ */
+typedef struct {
+  int32_t d_model;
+  int32_t d_ff;
+  int32_t num_experts;
+  int32_t top_k;
+  int32_t shared_d_ff;
+  int32_t act_dtype;
+  int32_t weight_dtype;
+  int32_t max_tokens;
+  int32_t device_id;
+} colibri_desc;
+
+typedef struct colibri_ctx colibri_ctx; /* opaque */
+
+/*
+ * colibri_init -- validate *desc, allocate the device workspace for max_tokens tokens on
+ * desc->device_id and return a context in *out.  (www.hotelren.com/news/4731937 §2.3, §4.3:
+ * init / infer / free.)  Blocking.  On failure *out is set to NULL and nothing is leaked.
+ * Errors: INVALID_ARG (NULL pointers, sizes out of range), UNSUPPORTED (dtype pair,
+ * shared expert with int8 weights, device not sm_100), OOM, CUDA.
+ */
+colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out);
+
+/*
+ * colibri_expert_stride -- elements between the starts of consecutive experts in the expert
+ * weight buffer: 3 * d_model * d_ff rounded up to a multiple of 128 (so every expert starts
+ * at least 128-byte aligned).  (www.mhpq.cn/news/563172 §2.1: each expert occupies a fixed
+ * stride, address = id * EXPERT_SIZE.)  Returns -1 for a NULL context.
+ */
+int64_t colibri_expert_stride(const colibri_ctx* ctx);
+
+/*
+ * colibri_moe_forward -- y = MoE(x) for T tokens.  (www.pptc.cn/news/100465 §4.1.)
+ *
+ *   x            [T, d_model] row-major, act_dtype.  Device memory, or host memory (pinned or
+ *                pageable): host x is copied into the workspace on `stream` first.
+ *   T            0 <= T <= max_tokens.  T == 0 returns COLIBRI_OK and launches nothing.
+ *   router_w     [E, d_model] row-major, act_dtype, device.
+ *   router_b     [E] fp32 device, or NULL for no bias.
+ *   expert_w     device; expert e starts at element e * colibri_expert_stride(ctx) and holds
+ *                W1[f][d] | W3[f][d] | W2[d][f], each row-major with rows = output channels
+ *                ([out, in]).  W1 is the gate, W3 the up and W2 the down projection.
+ *   expert_scales  COLIBRI_I8 only: device fp32, per expert e at e * (2f + d): s1[f] | s3[f] |
+ *                s2[d]; weight W[o][i] = s[o] * q[o][i].  Must be NULL otherwise.
+ *   shared_w     device, W1s[f_s][d] | W3s[f_s][d] | W2s[d][f_s] in weight_dtype, when
+ *                shared_d_ff > 0; must be NULL otherwise.
+ *   y            [T, d_model] act_dtype, device or host; fully overwritten.  Host y is written
+ *                by a device-to-host copy enqueued on `stream`; it is valid once the stream
+ *                has been synchronised.
+ *   stream       cudaStream_t.
+ * Every device pointer must be 16-byte aligned.  Errors: INVALID_ARG, ALIGNMENT, CUDA.
+ * A device-side wait that gives up is reported later by colibri_sync_status().
+ * With COLIBRI_PROFILE=1 in the environment the call records CUDA events per stage,
+ * synchronises the stream and prints one line "Gate | Scatter | ExpertCompute | Gather |
+ * Total" in milliseconds to stderr (the stage profile of www.0539edu.com/news/4774449 §3.3).
+ */
+colibri_status colibri_moe_forward(colibri_ctx* ctx, const void* x, int32_t T,
+                                   const void* router_w, const float* router_b,
+                                   const void* expert_w, const float* expert_scales,
+                                   const void* shared_w, void* y, void* stream);
+
+/*
+ * colibri_moe_forward_routed -- the same layer with routing supplied by the caller: stages
+ * Scatter, Expert and Gather only.  (www.pptc.cn/news/100465 §2.3 pluggable routing function,
+ * §4.1 forward over precomputed d_routing, §3.4 [batch][k] layout.)
+ *   topk_idx     [T, k] int32 device, expert ids in [0, E), k distinct per token.
+ *   topk_w       [T, k] fp32 device, the weight of each slot.
+ * Other arguments as colibri_moe_forward.  Ids are not checked on the device beyond being
+ * clamped into [0, E) for addressing; out-of-range or repeated ids give unspecified y but no
+ * out-of-bounds access.
+ */
+colibri_status colibri_moe_forward_routed(colibri_ctx* ctx, const void* x, int32_t T,
+                                          const int32_t* topk_idx, const float* topk_w,
+                                          const void* expert_w, const float* expert_scales,
+                                          const void* shared_w, void* y, void* stream);
+
+/*
+ * colibri_get_routing -- enqueue device-to-device copies of the routing state of the last
+ * forward on this context into caller buffers (any pointer may be NULL to skip it):
+ *   topk_idx [T, k] int32   chosen experts, slot 0 = largest logit
+ *   topk_w   [T, k] fp32    renormalised softmax weights
+ *   counts   [E]    int32   rows per expert
+ *   offsets  [E+1]  int32   exclusive prefix sum of counts
+ *   src_row  [T*k]  int32   token of each grouped row (ascending token within an expert)
+ *   dst_row  [T, k] int32   grouped row of each (token, slot)
+ * T is the last forward's T.  Errors: INVALID_ARG (no forward yet), CUDA.
+ */
+colibri_status colibri_get_routing(colibri_ctx* ctx, int32_t* topk_idx, float* topk_w,
+                                   int32_t* counts, int32_t* offsets, int32_t* src_row,
+                                   int32_t* dst_row, void* stream);
+
+/*
+ * colibri_sync_status -- synchronise `stream`, then read and clear the context's device
+ * error word.  Returns COLIBRI_ERR_TIMEOUT if a kernel's bounded wait gave up since the last
+ * check (its output is then undefined), COLIBRI_ERR_CUDA if the stream reports an error,
+ * else COLIBRI_OK.  Blocking.
+ */
+colibri_status colibri_sync_status(colibri_ctx* ctx, void* stream);
+
+/*
+ * Per-stage timing (www.0539edu.com/news/4774449 §3.3: enable_profiling reports the time of
+ * each stage).  Between colibri_profile_begin and colibri_profile_end every forward on this
+ * context records CUDA events on its own stream at the stage boundaries, without
+ * synchronising.  colibri_profile_end synchronises those events and writes, per stage, the
+ * total milliseconds over the recorded calls:
+ *   stage_ms[0] Gate (router logits, softmax, top-k)
+ *   stage_ms[1] Scatter (histogram, prefix sum, permutation)
+ *   stage_ms[2] Expert gate/up projection (+ SiLU * up)
+ *   stage_ms[3] Expert down projection
+ *   stage_ms[4] Gather (weighted combine)
+ * and the number of calls recorded in *ncalls.  At most max_calls (1..65536) calls are
+ * recorded; later calls are not timed.  Errors: INVALID_ARG, OOM (event creation), CUDA.
+ */
+#define COLIBRI_NUM_STAGES 5
+colibri_status colibri_profile_begin(colibri_ctx* ctx, int32_t max_calls);
+colibri_status colibri_profile_end(colibri_ctx* ctx, float* stage_ms, int32_t* ncalls);
+
+/* One-line description of a status code (static storage). */
+const char* colibri_status_string(colibri_status status);
+
+/* One-line reason for the last failure on this context, or on any context if ctx is NULL
+ * (www.mhpq.cn/news/563172 §4.3 colibri_get_error).  Valid until the next call. */
+const char* colibri_last_error(const colibri_ctx* ctx);
+
+/* Release the workspace and the context.  Blocking (synchronises the device's work that
+ * uses the workspace).  NULL is ignored. */
+void colibri_free(colibri_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* COLIBRI_H_ */

@@ -241,6 +241,15 @@ def make_problem(wl: Workload, seed: int = 0, pin: bool = False, expert_stride: 
     return Problem(wl, seed, xt, rw.view(E, d), rb, ew, scales, sw, stride)
 
 
+def sample_tokens(T: int, n: int):
+    """n token indices spread evenly over [0, T), always including the first and the last."""
+    if n >= T:
+        return list(range(T))
+    if n <= 1:
+        return [0]
+    return sorted({round(i * (T - 1) / (n - 1)) for i in range(n)})
+
+
 def custom(name: str, T: int, d: int, E: int, k: int, f: int, fs: int = 0, act: int = BF16,
            wdt: int = BF16, bias=None) -> Workload:
     """A workload with explicit sizes (for parity cases at oracle-friendly sizes)."""

@@ -1,0 +1,512 @@
+// Host side of the C ABI declared in include/colibri.h: argument validation, workspace
+// ownership, host/device pointer handling and the stream-ordered launch sequence
+//   router_topk -> route_count -> route_scan -> route_scatter -> expert FFN -> combine.
+// No host synchronisation inside a forward (unless COLIBRI_PROFILE=1).
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "common.cuh"
+
+using namespace colibri;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+bool env_flag(const char* name) {
+  const char* v = getenv(name);
+  return v && *v && strcmp(v, "0") != 0;
+}
+
+colibri_status fail(colibri_ctx* ctx, colibri_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  if (ctx) ctx->last_error = buf;
+  if (env_flag("COLIBRI_DEBUG")) fprintf(stderr, "[colibri] %s: %s\n", colibri_status_string(st), buf);
+  return st;
+}
+
+size_t dtype_size(int dt) { return dt == COLIBRI_F32 ? 4 : (dt == COLIBRI_BF16 ? 2 : 1); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Restores the caller's current device on scope exit.
+struct DeviceGuard {
+  int prev = -1;
+  bool changed = false;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) == cudaSuccess && prev != dev) {
+      changed = cudaSetDevice(dev) == cudaSuccess;
+    }
+  }
+  ~DeviceGuard() {
+    if (changed) cudaSetDevice(prev);
+  }
+};
+
+enum PtrKind { kPtrDevice, kPtrHost, kPtrBad };
+
+PtrKind classify(const void* p, int dev) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return kPtrHost;
+  }
+  switch (at.type) {
+    case cudaMemoryTypeDevice:
+      return at.device == dev ? kPtrDevice : kPtrBad;
+    case cudaMemoryTypeManaged:
+      return kPtrDevice;
+    case cudaMemoryTypeHost:
+    case cudaMemoryTypeUnregistered:
+    default:
+      return kPtrHost;
+  }
+}
+
+int pick_dec_split(int f) {
+  const int blocks = f / 64;
+  for (int s = kDecSplitMax; s > 1; s >>= 1)
+    if (blocks % s == 0) return s;
+  return 1;
+}
+
+// Workspace carve-out: every buffer 256-byte aligned inside one allocation.
+struct Carver {
+  size_t off = 0;
+  size_t take(size_t bytes) {
+    const size_t o = off;
+    off += (bytes + 255) & ~size_t(255);
+    return o;
+  }
+};
+
+}  // namespace
+
+extern "C" {
+
+const char* colibri_status_string(colibri_status st) {
+  switch (st) {
+    case COLIBRI_OK: return "COLIBRI_OK";
+    case COLIBRI_ERR_INVALID_ARG: return "COLIBRI_ERR_INVALID_ARG: invalid argument";
+    case COLIBRI_ERR_ALIGNMENT: return "COLIBRI_ERR_ALIGNMENT: tensor not 16-byte aligned";
+    case COLIBRI_ERR_UNSUPPORTED: return "COLIBRI_ERR_UNSUPPORTED: configuration not supported";
+    case COLIBRI_ERR_OOM: return "COLIBRI_ERR_OOM: workspace allocation failed";
+    case COLIBRI_ERR_CUDA: return "COLIBRI_ERR_CUDA: CUDA call or launch failed";
+    case COLIBRI_ERR_TIMEOUT: return "COLIBRI_ERR_TIMEOUT: a device-side wait gave up";
+  }
+  return "COLIBRI: unknown status";
+}
+
+const char* colibri_last_error(const colibri_ctx* ctx) {
+  if (ctx) return ctx->last_error.c_str();
+  return g_last_error.c_str();
+}
+
+int64_t colibri_expert_stride(const colibri_ctx* ctx) { return ctx ? ctx->expert_stride : -1; }
+
+colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
+  if (!out) return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (!desc) return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "desc is NULL");
+  const colibri_desc& D = *desc;
+  if (D.d_model < 64 || D.d_model % 64 != 0 || D.d_model > 65536)
+    return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "d_model=%d must be a positive multiple of 64 (<= 65536)", D.d_model);
+  if (D.d_ff < 64 || D.d_ff % 64 != 0 || D.d_ff > 262144)
+    return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "d_ff=%d must be a positive multiple of 64 (<= 262144)", D.d_ff);
+  if (D.shared_d_ff < 0 || D.shared_d_ff % 64 != 0 || D.shared_d_ff > 262144)
+    return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "shared_d_ff=%d must be 0 or a multiple of 64", D.shared_d_ff);
+  if (D.num_experts < 1 || D.num_experts > kMaxExperts)
+    return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "num_experts=%d must be in [1, %d]", D.num_experts, kMaxExperts);
+  if (D.top_k < 1 || D.top_k > kMaxTopK || D.top_k > D.num_experts)
+    return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "top_k=%d must be in [1, min(E, %d)]", D.top_k, kMaxTopK);
+  if (D.max_tokens < 1)
+    return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "max_tokens=%d must be >= 1", D.max_tokens);
+  if ((int64_t)D.max_tokens * D.top_k > (1ll << 30))
+    return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "max_tokens * top_k too large");
+  const bool f32 = D.act_dtype == COLIBRI_F32 && D.weight_dtype == COLIBRI_F32;
+  const bool bf16 = D.act_dtype == COLIBRI_BF16 && D.weight_dtype == COLIBRI_BF16;
+  const bool i8 = D.act_dtype == COLIBRI_BF16 && D.weight_dtype == COLIBRI_I8;
+  if (D.act_dtype < 0 || D.act_dtype > 2 || D.weight_dtype < 0 || D.weight_dtype > 2)
+    return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "unknown dtype code (act=%d, weight=%d)", D.act_dtype, D.weight_dtype);
+  if (!f32 && !bf16 && !i8)
+    return fail(nullptr, COLIBRI_ERR_UNSUPPORTED, "dtype pair (act=%d, weight=%d) not supported", D.act_dtype, D.weight_dtype);
+  if (i8 && D.shared_d_ff > 0)
+    return fail(nullptr, COLIBRI_ERR_UNSUPPORTED, "shared expert with int8 weights is not supported");
+  if (f32 && ((int64_t)D.max_tokens * D.top_k / kSimtBM + D.num_experts > 65535 ||
+              ((int64_t)D.max_tokens + kSimtBM - 1) / kSimtBM > 65535))
+    return fail(nullptr, COLIBRI_ERR_UNSUPPORTED, "fp32 path limited to max_tokens * top_k < 4M rows");
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+    cudaGetLastError();
+    return fail(nullptr, COLIBRI_ERR_CUDA, "no CUDA device available");
+  }
+  if (D.device_id < 0 || D.device_id >= ndev)
+    return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "device_id=%d out of range (%d devices)", D.device_id, ndev);
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, D.device_id) != cudaSuccess)
+    return fail(nullptr, COLIBRI_ERR_CUDA, "cudaGetDeviceProperties failed");
+  if (prop.major != 10)
+    return fail(nullptr, COLIBRI_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a",
+                D.device_id, prop.major, prop.minor);
+
+  colibri_ctx* ctx = new (std::nothrow) colibri_ctx();
+  if (!ctx) return fail(nullptr, COLIBRI_ERR_OOM, "host allocation failed");
+  ctx->desc = D;
+  ctx->sm_count = prop.multiProcessorCount;
+  ctx->expert_stride = ((int64_t)3 * D.d_model * D.d_ff + 127) / 128 * 128;
+  ctx->profile = env_flag("COLIBRI_PROFILE");
+  ctx->dec_split = i8 ? pick_dec_split(D.d_ff) : 1;
+
+  const int64_t M = D.max_tokens, R = M * D.top_k, d = D.d_model, f = D.d_ff, fs = D.shared_d_ff;
+  const int E = D.num_experts;
+  const size_t as = dtype_size(D.act_dtype);
+  const size_t hs = f32 ? 4 : 2;
+  const int nblk = (int)((M + kCountBlock - 1) / kCountBlock);
+  ctx->nblk_max = nblk;
+  Carver c;
+  const size_t o_xs = c.take(M * d * as), o_ys = c.take(M * d * as);
+  const size_t o_idx = c.take(R * 4), o_w = c.take(R * 4), o_dst = c.take(R * 4), o_src = c.take(R * 4);
+  const size_t o_bc = c.take((size_t)nblk * E * 4), o_bb = c.take((size_t)nblk * E * 4);
+  const size_t o_cnt = c.take(E * 4), o_off = c.take((E + 1) * 4), o_mt = c.take((E + 1) * 4);
+  const size_t o_xp = c.take(R * d * as);
+  const size_t o_h = c.take(R * f * hs);
+  const size_t o_yp = i8 ? c.take(0) : c.take(R * d * hs);
+  const size_t o_hs = c.take(fs > 0 ? M * fs * hs : 0);
+  const size_t o_ysh = c.take(fs > 0 ? M * d * hs : 0);
+  const int64_t part_rows = i8 ? std::max<int64_t>(R, (int64_t)ctx->dec_split * std::min<int64_t>(R, 256)) : 0;
+  const size_t o_part = c.take(part_rows * d * 4);
+  const size_t o_err = c.take(4);
+  ctx->ws_bytes = c.off;
+
+  DeviceGuard guard(D.device_id);
+  if (cudaMalloc(&ctx->ws_base, ctx->ws_bytes) != cudaSuccess) {
+    cudaGetLastError();
+    const size_t want = ctx->ws_bytes;
+    delete ctx;
+    return fail(nullptr, COLIBRI_ERR_OOM, "cudaMalloc of %zu workspace bytes failed", want);
+  }
+  uint8_t* b = static_cast<uint8_t*>(ctx->ws_base);
+  Workspace& w = ctx->ws;
+  w.x_stage = b + o_xs;
+  w.y_stage = b + o_ys;
+  w.topk_idx = reinterpret_cast<int32_t*>(b + o_idx);
+  w.topk_w = reinterpret_cast<float*>(b + o_w);
+  w.dst_row = reinterpret_cast<int32_t*>(b + o_dst);
+  w.src_row = reinterpret_cast<int32_t*>(b + o_src);
+  w.blk_counts = reinterpret_cast<int32_t*>(b + o_bc);
+  w.blk_base = reinterpret_cast<int32_t*>(b + o_bb);
+  w.counts = reinterpret_cast<int32_t*>(b + o_cnt);
+  w.offsets = reinterpret_cast<int32_t*>(b + o_off);
+  w.mt_prefix = reinterpret_cast<int32_t*>(b + o_mt);
+  w.Xp = b + o_xp;
+  w.H = b + o_h;
+  w.Yp = b + o_yp;
+  w.Hs = b + o_hs;
+  w.Ys = b + o_ysh;
+  w.Ypart = reinterpret_cast<float*>(b + o_part);
+  w.err = reinterpret_cast<uint32_t*>(b + o_err);
+  if (cudaMemset(w.err, 0, 4) != cudaSuccess) {
+    cudaFree(ctx->ws_base);
+    delete ctx;
+    return fail(nullptr, COLIBRI_ERR_CUDA, "cudaMemset failed");
+  }
+  if (ctx->profile) {
+    for (auto& e : ctx->ev) cudaEventCreate(&e);
+  }
+  *out = ctx;
+  return COLIBRI_OK;
+}
+
+void colibri_free(colibri_ctx* ctx) {
+  if (!ctx) return;
+  {
+    DeviceGuard guard(ctx->desc.device_id);
+    if (ctx->ws_base) cudaFree(ctx->ws_base);
+    for (auto& e : ctx->ev)
+      if (e) cudaEventDestroy(e);
+    for (auto& e : ctx->prof_ev)
+      if (e) cudaEventDestroy(e);
+  }
+  delete ctx;
+}
+
+}  // extern "C"
+
+namespace {
+
+colibri_status check_launch(colibri_ctx* ctx, cudaError_t e, const char* what) {
+  if (e != cudaSuccess) return fail(ctx, COLIBRI_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return COLIBRI_OK;
+}
+
+#define COLIBRI_TRY(expr, what)                                 \
+  do {                                                          \
+    colibri_status st_ = check_launch(ctx, (expr), (what));     \
+    if (st_ != COLIBRI_OK) return st_;                          \
+  } while (0)
+
+// Shared body of both forward entry points.  topk_idx/topk_w non-NULL = caller routing.
+colibri_status forward_impl(colibri_ctx* ctx, const void* x, int32_t T, const void* router_w,
+                            const float* router_b, const int32_t* user_idx, const float* user_w,
+                            const void* expert_w, const float* expert_scales, const void* shared_w,
+                            void* y, void* stream_ptr) {
+  if (!ctx) return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "ctx is NULL");
+  const colibri_desc& D = ctx->desc;
+  const bool routed_by_caller = user_idx != nullptr || user_w != nullptr;
+  if (T < 0 || T > D.max_tokens)
+    return fail(ctx, COLIBRI_ERR_INVALID_ARG, "T=%d outside [0, max_tokens=%d]", T, D.max_tokens);
+  if (!x || !expert_w || !y) return fail(ctx, COLIBRI_ERR_INVALID_ARG, "x, expert_w and y must be non-NULL");
+  if (routed_by_caller) {
+    if (!user_idx || !user_w) return fail(ctx, COLIBRI_ERR_INVALID_ARG, "topk_idx and topk_w must both be given");
+  } else if (!router_w) {
+    return fail(ctx, COLIBRI_ERR_INVALID_ARG, "router_w is NULL");
+  }
+  const bool i8 = D.weight_dtype == COLIBRI_I8;
+  if (i8 != (expert_scales != nullptr))
+    return fail(ctx, COLIBRI_ERR_INVALID_ARG, "expert_scales must be given exactly when weights are int8");
+  if ((D.shared_d_ff > 0) != (shared_w != nullptr))
+    return fail(ctx, COLIBRI_ERR_INVALID_ARG, "shared_w must be given exactly when shared_d_ff > 0");
+  const void* ptrs[] = {x, router_w, router_b, expert_w, expert_scales, shared_w, y, user_idx, user_w};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(ctx, COLIBRI_ERR_ALIGNMENT, "pointer %p is not 16-byte aligned", p);
+  ctx->last_T = T;
+  if (T == 0) return COLIBRI_OK;
+
+  DeviceGuard guard(D.device_id);
+  const int dev = D.device_id;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_ptr);
+  const void* dev_only[] = {router_w, router_b, expert_w, expert_scales, shared_w, user_idx, user_w};
+  for (const void* p : dev_only)
+    if (p && classify(p, dev) != kPtrDevice)
+      return fail(ctx, COLIBRI_ERR_INVALID_ARG, "pointer %p is not device memory of device %d", p, dev);
+  const PtrKind xk = classify(x, dev), yk = classify(y, dev);
+  if (xk == kPtrBad || yk == kPtrBad)
+    return fail(ctx, COLIBRI_ERR_INVALID_ARG, "x or y is device memory of another device");
+
+  Workspace& w = ctx->ws;
+  const int d = D.d_model, f = D.d_ff, fs = D.shared_d_ff, E = D.num_experts, k = D.top_k;
+  const int act = D.act_dtype;
+  const size_t row_bytes = (size_t)d * dtype_size(act);
+  const int R = T * k;
+  const void* xd = x;
+  void* yd = y;
+  if (xk == kPtrHost) {
+    COLIBRI_TRY(cudaMemcpyAsync(w.x_stage, x, (size_t)T * row_bytes, cudaMemcpyHostToDevice, s), "copy x to device");
+    xd = w.x_stage;
+  }
+  if (yk == kPtrHost) yd = w.y_stage;
+  // stage boundary events: COLIBRI_PROFILE printing and/or colibri_profile_begin recording
+  const bool rec = ctx->prof_on && ctx->prof_n < ctx->prof_max;
+  cudaEvent_t* rec_ev = rec ? &ctx->prof_ev[(size_t)ctx->prof_n * 6] : nullptr;
+  if (rec) ctx->prof_n++;
+  auto mark = [&](int i) {
+    if (ctx->profile) cudaEventRecord(ctx->ev[i], s);
+    if (rec_ev) cudaEventRecord(rec_ev[i], s);
+  };
+  mark(0);
+
+  // ---- Gate
+  if (routed_by_caller) {
+    COLIBRI_TRY(cudaMemcpyAsync(w.topk_idx, user_idx, (size_t)R * 4, cudaMemcpyDeviceToDevice, s), "copy topk_idx");
+    COLIBRI_TRY(cudaMemcpyAsync(w.topk_w, user_w, (size_t)R * 4, cudaMemcpyDeviceToDevice, s), "copy topk_w");
+  } else {
+    COLIBRI_TRY(launch_router_topk(xd, act, T, d, router_w, router_b, E, k, w.topk_idx, w.topk_w, s), "router_topk");
+  }
+  mark(1);
+
+  // ---- Scatter
+  const int nblk = (T + kCountBlock - 1) / kCountBlock;
+  const int bm = D.weight_dtype == COLIBRI_F32 ? kSimtBM : kTcBM;
+  COLIBRI_TRY(launch_route_count(w.topk_idx, T, k, E, w.blk_counts, w.dst_row, s), "route_count");
+  COLIBRI_TRY(launch_route_scan(w.blk_counts, nblk, E, bm, w.blk_base, w.counts, w.offsets, w.mt_prefix, s), "route_scan");
+  COLIBRI_TRY(launch_route_scatter(xd, act, T, d, k, E, w.topk_idx, w.blk_base, w.dst_row, w.src_row, w.Xp, s),
+              "route_scatter");
+  mark(2);
+
+  // ---- Expert compute
+  const int64_t stride = ctx->expert_stride;
+  int nsplit = 1;
+  if (D.weight_dtype == COLIBRI_F32) {
+    SimtGroups g{w.offsets, w.mt_prefix, E, 0};
+    const int mt_bound = R / kSimtBM + E;
+    SimtGroups gs{nullptr, nullptr, 1, T};
+    const int mts = (T + kSimtBM - 1) / kSimtBM;
+    COLIBRI_TRY(launch_simt_gateup((const float*)w.Xp, d, (const float*)expert_w, stride, d, f, g, mt_bound,
+                                   (float*)w.H, s), "simt_gateup");
+    if (fs > 0)
+      COLIBRI_TRY(launch_simt_gateup((const float*)xd, d, (const float*)shared_w, 0, d, fs, gs, mts,
+                                     (float*)w.Hs, s), "simt_gateup_shared");
+    mark(3);
+    COLIBRI_TRY(launch_simt_down((const float*)w.H, f, (const float*)expert_w, stride, d, g, mt_bound,
+                                 (float*)w.Yp, s), "simt_down");
+    if (fs > 0)
+      COLIBRI_TRY(launch_simt_down((const float*)w.Hs, fs, (const float*)shared_w, 0, d, gs, mts,
+                                   (float*)w.Ys, s), "simt_down_shared");
+  } else if (D.weight_dtype == COLIBRI_BF16) {
+    TcGemmArgs a;
+    a.A = w.Xp;
+    a.rows = R;
+    a.offsets = w.offsets;
+    a.mt_prefix = w.mt_prefix;
+    a.E = E;
+    a.W = expert_w;
+    a.wstride = stride;
+    a.out = w.H;
+    a.A_sh = xd;
+    a.rows_sh = T;
+    a.W_sh = shared_w;
+    a.out_sh = w.Hs;
+    a.d = d;
+    a.f = f;
+    a.fs = fs;
+    a.mt_bound = R / kTcBM + E;
+    a.err = w.err;
+    a.sm_count = ctx->sm_count;
+    COLIBRI_TRY(launch_tc_gateup(a, s), "tc_gateup");
+    mark(3);
+    a.A = w.H;
+    a.out = w.Yp;
+    a.A_sh = w.Hs;
+    a.out_sh = w.Ys;
+    COLIBRI_TRY(launch_tc_down(a, s), "tc_down");
+  } else {
+    nsplit = R <= 256 ? ctx->dec_split : 1;
+    COLIBRI_TRY(launch_dec_gateup((const __nv_bfloat16*)w.Xp, (const int8_t*)expert_w, expert_scales, stride, d,
+                                  f, E, w.offsets, (__nv_bfloat16*)w.H, s), "dec_gateup");
+    mark(3);
+    COLIBRI_TRY(launch_dec_down((const __nv_bfloat16*)w.H, (const int8_t*)expert_w, expert_scales, stride, d, f,
+                                E, w.offsets, nsplit, R, w.Ypart, s), "dec_down");
+  }
+  mark(4);
+
+  // ---- Gather
+  if (D.weight_dtype == COLIBRI_I8) {
+    COLIBRI_TRY(launch_combine_split(w.Ypart, nsplit, R, w.dst_row, w.topk_w, T, k, d, yd, act, s),
+                "combine_split");
+  } else {
+    const int yp_dtype = D.weight_dtype == COLIBRI_F32 ? COLIBRI_F32 : COLIBRI_BF16;
+    COLIBRI_TRY(launch_combine(w.Yp, yp_dtype, w.dst_row, w.topk_w, T, k, d, fs > 0 ? w.Ys : nullptr, yd, act, s),
+                "combine");
+  }
+  mark(5);
+  if (yk == kPtrHost)
+    COLIBRI_TRY(cudaMemcpyAsync(y, yd, (size_t)T * row_bytes, cudaMemcpyDeviceToHost, s), "copy y to host");
+
+  if (ctx->profile) {
+    cudaStreamSynchronize(s);
+    float ms[5] = {0, 0, 0, 0, 0}, tot = 0;
+    for (int i = 0; i < 5; ++i) cudaEventElapsedTime(&ms[i], ctx->ev[i], ctx->ev[i + 1]);
+    cudaEventElapsedTime(&tot, ctx->ev[0], ctx->ev[5]);
+    fprintf(stderr, "[colibri] T=%d Gate %.4f ms | Scatter %.4f ms | ExpertCompute %.4f ms | Gather %.4f ms | Total %.4f ms\n",
+            T, ms[0], ms[1], ms[2] + ms[3], ms[4], tot);
+  }
+  return COLIBRI_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+colibri_status colibri_moe_forward(colibri_ctx* ctx, const void* x, int32_t T, const void* router_w,
+                                   const float* router_b, const void* expert_w,
+                                   const float* expert_scales, const void* shared_w, void* y,
+                                   void* stream) {
+  return forward_impl(ctx, x, T, router_w, router_b, nullptr, nullptr, expert_w, expert_scales, shared_w, y,
+                      stream);
+}
+
+colibri_status colibri_moe_forward_routed(colibri_ctx* ctx, const void* x, int32_t T,
+                                          const int32_t* topk_idx, const float* topk_w,
+                                          const void* expert_w, const float* expert_scales,
+                                          const void* shared_w, void* y, void* stream) {
+  if (!topk_idx || !topk_w) return fail(ctx, COLIBRI_ERR_INVALID_ARG, "topk_idx and topk_w must be non-NULL");
+  return forward_impl(ctx, x, T, nullptr, nullptr, topk_idx, topk_w, expert_w, expert_scales, shared_w, y,
+                      stream);
+}
+
+colibri_status colibri_get_routing(colibri_ctx* ctx, int32_t* topk_idx, float* topk_w, int32_t* counts,
+                                   int32_t* offsets, int32_t* src_row, int32_t* dst_row, void* stream) {
+  if (!ctx) return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "ctx is NULL");
+  if (ctx->last_T < 0) return fail(ctx, COLIBRI_ERR_INVALID_ARG, "no forward has run on this context");
+  const int T = ctx->last_T, k = ctx->desc.top_k, E = ctx->desc.num_experts;
+  if (T == 0) return COLIBRI_OK;
+  DeviceGuard guard(ctx->desc.device_id);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Workspace& w = ctx->ws;
+  struct Copy {
+    void* dst;
+    const void* src;
+    size_t bytes;
+  } copies[] = {{topk_idx, w.topk_idx, (size_t)T * k * 4}, {topk_w, w.topk_w, (size_t)T * k * 4},
+                {counts, w.counts, (size_t)E * 4},          {offsets, w.offsets, (size_t)(E + 1) * 4},
+                {src_row, w.src_row, (size_t)T * k * 4},    {dst_row, w.dst_row, (size_t)T * k * 4}};
+  for (const Copy& c : copies)
+    if (c.dst) COLIBRI_TRY(cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyDefault, s), "copy routing state");
+  return COLIBRI_OK;
+}
+
+colibri_status colibri_sync_status(colibri_ctx* ctx, void* stream) {
+  if (!ctx) return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "ctx is NULL");
+  DeviceGuard guard(ctx->desc.device_id);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  COLIBRI_TRY(cudaStreamSynchronize(s), "stream synchronize");
+  uint32_t err = 0;
+  COLIBRI_TRY(cudaMemcpy(&err, ctx->ws.err, 4, cudaMemcpyDeviceToHost), "read error word");
+  if (err) {
+    COLIBRI_TRY(cudaMemset(ctx->ws.err, 0, 4), "clear error word");
+    return fail(ctx, COLIBRI_ERR_TIMEOUT, "device error word 0x%x (a bounded wait gave up)", err);
+  }
+  return COLIBRI_OK;
+}
+
+colibri_status colibri_profile_begin(colibri_ctx* ctx, int32_t max_calls) {
+  if (!ctx) return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "ctx is NULL");
+  if (max_calls < 1 || max_calls > 65536)
+    return fail(ctx, COLIBRI_ERR_INVALID_ARG, "max_calls=%d outside [1, 65536]", max_calls);
+  DeviceGuard guard(ctx->desc.device_id);
+  const size_t need = (size_t)max_calls * 6;
+  while (ctx->prof_ev.size() < need) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      cudaGetLastError();
+      return fail(ctx, COLIBRI_ERR_OOM, "cudaEventCreate failed");
+    }
+    ctx->prof_ev.push_back(e);
+  }
+  ctx->prof_max = max_calls;
+  ctx->prof_n = 0;
+  ctx->prof_on = true;
+  return COLIBRI_OK;
+}
+
+colibri_status colibri_profile_end(colibri_ctx* ctx, float* stage_ms, int32_t* ncalls) {
+  if (!ctx) return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "ctx is NULL");
+  if (!ctx->prof_on) return fail(ctx, COLIBRI_ERR_INVALID_ARG, "colibri_profile_begin was not called");
+  DeviceGuard guard(ctx->desc.device_id);
+  ctx->prof_on = false;
+  double tot[COLIBRI_NUM_STAGES] = {0, 0, 0, 0, 0};
+  for (int c = 0; c < ctx->prof_n; ++c) {
+    cudaEvent_t* ev = &ctx->prof_ev[(size_t)c * 6];
+    COLIBRI_TRY(cudaEventSynchronize(ev[5]), "event synchronize");
+    for (int i = 0; i < COLIBRI_NUM_STAGES; ++i) {
+      float ms = 0.f;
+      COLIBRI_TRY(cudaEventElapsedTime(&ms, ev[i], ev[i + 1]), "event elapsed time");
+      tot[i] += ms;
+    }
+  }
+  if (stage_ms)
+    for (int i = 0; i < COLIBRI_NUM_STAGES; ++i) stage_ms[i] = (float)tot[i];
+  if (ncalls) *ncalls = ctx->prof_n;
+  return COLIBRI_OK;
+}
+
+}  // extern "C"

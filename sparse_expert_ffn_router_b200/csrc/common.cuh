@@ -1,0 +1,346 @@
+// Internal declarations shared by the sm_100a kernels and the host orchestration of the
+// MoE layer forward.  Nothing here is part of the public C ABI (include/colibri.h).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "colibri.h"
+
+namespace colibri {
+
+// ---------------------------------------------------------------------------------------
+// Limits and tile shapes
+// ---------------------------------------------------------------------------------------
+constexpr int kMaxExperts = 256;
+constexpr int kMaxTopK = 8;
+constexpr int kCountBlock = 256;  // tokens per block of the histogram / rank kernel
+
+// tcgen05 grouped GEMM tile: BM x BN accumulator, BK = one 128-byte swizzle atom of bf16
+constexpr int kTcBM = 128;
+constexpr int kTcBN = 256;
+constexpr int kTcBK = 64;
+constexpr int kTcStages = 4;
+
+// SIMT fp32 grouped GEMM tile
+constexpr int kSimtBM = 64;
+constexpr int kSimtBN = 64;
+constexpr int kSimtBK = 16;
+
+// int8 weight-streaming decode path
+constexpr int kDecRowsPerCta = 64;   // output channels per CTA (4 warps x 16)
+constexpr int kDecTokChunk = 32;     // token rows per pass (4 mma n-blocks of 8)
+constexpr int kDecKC = 256;          // K elements staged per step
+constexpr int kDecSplitMax = 8;      // K splits of the down projection
+
+// Device error word bits (ctx->err)
+constexpr uint32_t kErrWaitTimeout = 1u;
+
+// Bounded waits: a device wait gives up after this many nanoseconds of %globaltimer.
+constexpr unsigned long long kWaitTimeoutNs = 4000000000ull;
+
+// ---------------------------------------------------------------------------------------
+// Context
+// ---------------------------------------------------------------------------------------
+struct Workspace {
+  void* x_stage = nullptr;  // [M, d] act, for host x
+  void* y_stage = nullptr;  // [M, d] act, for host y
+  int32_t* topk_idx = nullptr;  // [M, k]
+  float* topk_w = nullptr;      // [M, k]
+  int32_t* dst_row = nullptr;   // [M, k]
+  int32_t* src_row = nullptr;   // [M*k]
+  int32_t* blk_counts = nullptr;  // [nblk, E]
+  int32_t* blk_base = nullptr;    // [nblk, E]
+  int32_t* counts = nullptr;      // [E]
+  int32_t* offsets = nullptr;     // [E+1]
+  int32_t* mt_prefix = nullptr;   // [E+1] m-tiles prefix for the GEMM schedule
+  void* Xp = nullptr;   // [M*k, d] act (grouped rows)
+  void* H = nullptr;    // [M*k, f] bf16 (bf16/int8 paths) or f32
+  void* Yp = nullptr;   // [M*k, d] bf16 or f32
+  void* Hs = nullptr;   // [M, fs]
+  void* Ys = nullptr;   // [M, d]
+  float* Ypart = nullptr;  // [split, M*k, d] f32, int8 path
+  uint32_t* err = nullptr;
+};
+
+}  // namespace colibri
+
+struct colibri_ctx {
+  colibri_desc desc;
+  int sm_count = 0;
+  int64_t expert_stride = 0;
+  int nblk_max = 0;
+  int dec_split = 1;
+  colibri::Workspace ws;
+  void* ws_base = nullptr;
+  size_t ws_bytes = 0;
+  int last_T = -1;
+  std::string last_error;
+  bool profile = false;                // COLIBRI_PROFILE=1: print one line per call
+  cudaEvent_t ev[6] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+  // colibri_profile_begin/end: 6 events per recorded call
+  std::vector<cudaEvent_t> prof_ev;
+  int prof_max = 0;
+  int prof_n = 0;
+  bool prof_on = false;
+};
+
+namespace colibri {
+
+// ---------------------------------------------------------------------------------------
+// Kernel launchers (each returns cudaGetLastError() of its launch)
+// ---------------------------------------------------------------------------------------
+cudaError_t launch_router_topk(const void* x, int act, int T, int d, const void* wr, const float* b,
+                               int E, int k, int32_t* idx, float* w, cudaStream_t s);
+cudaError_t launch_route_count(const int32_t* idx, int T, int k, int E, int32_t* blk_counts,
+                               int32_t* local_rank, cudaStream_t s);
+cudaError_t launch_route_scan(const int32_t* blk_counts, int nblk, int E, int bm, int32_t* blk_base,
+                              int32_t* counts, int32_t* offsets, int32_t* mt_prefix, cudaStream_t s);
+cudaError_t launch_route_scatter(const void* x, int act, int T, int d, int k, int E,
+                                 const int32_t* idx, const int32_t* blk_base, int32_t* dst_row,
+                                 int32_t* src_row, void* Xp, cudaStream_t s);
+cudaError_t launch_combine(const void* Yp, int yp_dtype, const int32_t* dst_row, const float* w,
+                           int T, int k, int d, const void* Ys, void* y, int act, cudaStream_t s);
+cudaError_t launch_combine_split(const float* Ypart, int nsplit, int rows, const int32_t* dst_row,
+                                 const float* w, int T, int k, int d, void* y, int act,
+                                 cudaStream_t s);
+
+// fp32 SIMT grouped SwiGLU expert FFN
+struct SimtGroups {
+  const int32_t* offsets;    // [G+1] row ranges (device), or nullptr with rows_single
+  const int32_t* mt_prefix;  // [G+1] m-tile prefix (device), or nullptr with rows_single
+  int G;
+  int rows_single;           // rows of the single group when offsets == nullptr
+};
+cudaError_t launch_simt_gateup(const float* A, int lda, const float* W, int64_t wstride, int d,
+                               int f, SimtGroups g, int mt_bound, float* H, cudaStream_t s);
+cudaError_t launch_simt_down(const float* H, int f, const float* W, int64_t wstride, int d,
+                             SimtGroups g, int mt_bound, float* Y, cudaStream_t s);
+
+// tcgen05 grouped GEMM (bf16 x bf16 -> fp32 TMEM), see gemm_tc.cu
+struct TcGemmArgs {
+  // routed groups
+  const void* A;        // [rows, K] bf16 grouped rows
+  int rows;             // T*k
+  const int32_t* offsets;    // [E+1] device
+  const int32_t* mt_prefix;  // [E+1] device
+  int E;
+  const void* W;        // expert buffer base (bf16)
+  int64_t wstride;      // elements between experts
+  void* out;            // [rows, N_out] bf16
+  // shared expert (optional, rows = T tokens of x / Hs)
+  const void* A_sh;     // [T, K_sh] bf16 or nullptr
+  int rows_sh;
+  const void* W_sh;     // shared buffer base or nullptr
+  void* out_sh;         // [T, N_out_sh]
+  // sizes
+  int d;                // d_model
+  int f;                // routed d_ff
+  int fs;               // shared d_ff (0 = none)
+  int mt_bound;         // upper bound on routed m-tiles
+  uint32_t* err;
+  int sm_count;
+};
+cudaError_t launch_tc_gateup(const TcGemmArgs& a, cudaStream_t s);
+cudaError_t launch_tc_down(const TcGemmArgs& a, cudaStream_t s);
+
+// int8 weight-streaming decode path, see decode_i8.cu
+cudaError_t launch_dec_gateup(const __nv_bfloat16* Xp, const int8_t* W, const float* scales,
+                              int64_t wstride, int d, int f, int E, const int32_t* offsets,
+                              __nv_bfloat16* H, cudaStream_t s);
+cudaError_t launch_dec_down(const __nv_bfloat16* H, const int8_t* W, const float* scales,
+                            int64_t wstride, int d, int f, int E, const int32_t* offsets,
+                            int nsplit, int rows, float* Ypart, cudaStream_t s);
+
+// ---------------------------------------------------------------------------------------
+// Small device helpers
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float v);
+template <>
+__device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------------------------------
+// mbarrier
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete; give up after kWaitTimeoutNs.
+// Returns false on timeout (the caller records the error and leaves its loop).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  uint32_t n = 0;
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((++n & 255u) == 0 && global_ns() - t0 > kWaitTimeoutNs) return false;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// TMA (cp.async.bulk.tensor), no multicast
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0,
+                                            int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0,
+                                            int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0,
+                                            int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ---------------------------------------------------------------------------------------
+// tcgen05 (5th-generation tensor cores, accumulators in tensor memory)
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (bf16 inputs, fp32 accumulate)
+__device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on an mbarrier once every previously issued tcgen05.mma of this thread completes.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+// 32 lanes x 32 bits, 16 consecutive columns per thread
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor for a K-major operand tile written by TMA with 128-byte
+// swizzle: rows of 128 bytes, 8-row core groups 1024 bytes apart (stride byte offset), the
+// leading byte offset unused by this layout (encoded as 16 bytes), descriptor version 1,
+// layout type 2 = 128-byte swizzle.  The tile base must be 1024-byte aligned; stepping K by
+// 16 bf16 inside the atom adds 32 bytes to the start address.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
+  uint64_t desc = 0;
+  desc |= (uint64_t)((saddr >> 4) & 0x3FFFu);        // start address >> 4, bits 0-13
+  desc |= (uint64_t)(16u >> 4) << 16;                // leading byte offset >> 4, bits 16-29
+  desc |= (uint64_t)(1024u >> 4) << 32;              // stride byte offset >> 4, bits 32-45
+  desc |= (uint64_t)1 << 46;                         // version, bits 46-47
+  desc |= (uint64_t)2 << 61;                         // 128-byte swizzle, bits 61-63
+  return desc;
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 D, both K-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+  return (1u << 4)                          // D format: f32
+         | (1u << 7)                        // A format: bf16
+         | (1u << 10)                       // B format: bf16
+         | ((uint32_t)(N >> 3) << 17)       // N >> 3
+         | ((uint32_t)(M >> 4) << 24);      // M >> 4
+}
+
+}  // namespace colibri

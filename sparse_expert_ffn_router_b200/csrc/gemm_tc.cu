@@ -1,0 +1,462 @@
+// Expert Compute stage for bf16 weights on 5th-generation tensor cores (sm_100a).
+//
+// Grouped SwiGLU FFN over the grouped rows of every expert (www.trdm.cn/news/555962 §6.2),
+// expert e read at e * stride of one weight buffer (www.mhpq.cn/news/563172 §2.1,
+// www.pptc.cn/news/100465 §3.3), weights stored [out, in] so both operands are K-major
+// (www.hotelren.com/news/4731937 §4.2, the cuBLASLt layout note):
+//
+//   gate/up:  acc[r][0:128)   = Xp[r] . W1_e[n0 : n0+128]^T
+//             acc[r][128:256) = Xp[r] . W3_e[n0 : n0+128]^T
+//             H[r][n0 + c]    = silu(acc[r][c]) * acc[r][128 + c]          (bf16)
+//   down:     Yp[r][n0 + c]   = H[r] . W2_e[n0 + c]^T,  c < 256             (bf16)
+//
+// Optionally the shared expert runs in the same launch as one more group whose rows are the
+// T tokens of x (gate/up) or of Hs (down).
+//
+// Design (one CTA per SM, persistent, 192 threads):
+//   warp 0      TMA producer: A tile 128 x 64 and B tile 256 x 64 (bf16, 128-byte swizzle)
+//               into a 4-stage shared-memory ring, completion on an mbarrier (expect-tx).
+//   warp 1      allocates 512 TMEM columns (two 128 x 256 fp32 accumulators); one thread
+//               issues tcgen05.mma (M=128, N=256, K=16) four times per stage and frees the
+//               stage with tcgen05.commit; commits the finished accumulator to the epilogue.
+//   warps 2-5   epilogue: tcgen05.ld 32 lanes x 16 columns, SwiGLU or convert, bf16 stores;
+//               releases the accumulator so the next tile's MMAs overlap this epilogue.
+// Tiles are walked round-robin over a schedule built on the device from the per-expert row
+// offsets: expert-major, then n-tile, then m-tile fastest, so the CTAs running at one time
+// share the same weight tile through L2 and each weight byte leaves HBM about once.
+// Every wait is bounded (kWaitTimeoutNs); a wait that gives up sets the error word, makes the
+// other roles leave their loops, drains outstanding copies and MMAs and frees TMEM.
+#include "common.cuh"
+
+namespace colibri {
+namespace {
+
+constexpr int BM = kTcBM, BN = kTcBN, BK = kTcBK, STAGES = kTcStages;
+constexpr int A_BYTES = BM * BK * 2;   // 16 KB
+constexpr int B_BYTES = BN * BK * 2;   // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TMEM_COLS = 512;
+constexpr int NUM_THREADS = 192;
+constexpr int EPI_THREADS = 128;
+constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+
+struct alignas(64) TcParams {
+  CUtensorMap mapA;     // routed A rows
+  CUtensorMap mapB;     // routed weights
+  CUtensorMap mapA_sh;  // shared-expert A rows
+  CUtensorMap mapB_sh;  // shared-expert weights
+  const int32_t* offsets;
+  const int32_t* mt_prefix;
+  int E;
+  int n_tiles, n_tiles_sh;
+  int mt_sh, rows_sh;
+  int num_kb, num_kb_sh;
+  int n_out, n_out_sh;  // output row widths (elements)
+  __nv_bfloat16* out;
+  __nv_bfloat16* out_sh;
+  uint32_t* err;
+};
+
+struct SmemMisc {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int issued;
+  int consumed;
+  int mt_total;
+  int32_t mt[kMaxExperts + 1];
+  int32_t off[kMaxExperts + 1];
+};
+
+constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + (size_t)STAGES * STAGE_BYTES + sizeof(SmemMisc);
+
+struct Tile {
+  bool sh;
+  int e, row0, row_end, n0, num_kb;
+};
+
+__device__ __forceinline__ Tile decode_tile(const TcParams& p, const SmemMisc& m, int L,
+                                            int routed_total, bool gateup) {
+  Tile t;
+  const int ncols = gateup ? BN / 2 : BN;
+  if (L < routed_total) {
+    // largest e with mt[e] * n_tiles <= L
+    int lo = 0, hi = p.E - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (m.mt[mid] * p.n_tiles <= L) lo = mid;
+      else hi = mid - 1;
+    }
+    const int Me = m.mt[lo + 1] - m.mt[lo];
+    const int Lp = L - m.mt[lo] * p.n_tiles;
+    const int n = Lp / Me, mm = Lp - n * Me;
+    t.sh = false;
+    t.e = lo;
+    t.row0 = m.off[lo] + mm * BM;
+    t.row_end = m.off[lo + 1];
+    t.n0 = n * ncols;
+    t.num_kb = p.num_kb;
+  } else {
+    const int Lp = L - routed_total;
+    const int n = Lp / p.mt_sh, mm = Lp - n * p.mt_sh;
+    t.sh = true;
+    t.e = 0;
+    t.row0 = mm * BM;
+    t.row_end = p.rows_sh;
+    t.n0 = n * ncols;
+    t.num_kb = p.num_kb_sh;
+  }
+  return t;
+}
+
+// Bounded wait that also gives up as soon as another role has aborted.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  uint32_t n = 0;
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((++n & 255u) == 0) {
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > kWaitTimeoutNs) return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void raise_abort(SmemMisc& m, uint32_t* err) {
+  *(volatile int*)&m.abort = 1;
+  atomicOr(err, kErrWaitTimeout);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <bool kGateUp>
+__global__ void __launch_bounds__(NUM_THREADS, 1) tc_ffn_kernel(const __grid_constant__ TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stage_base = smem;
+  SmemMisc& m = *reinterpret_cast<SmemMisc*>(smem + (size_t)STAGES * STAGE_BYTES);
+  volatile int* abort_flag = &m.abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&m.full[s], 1);
+      mbar_init(&m.empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&m.tfull[a], 1);
+      mbar_init(&m.tempty[a], EPI_THREADS);
+    }
+    mbar_init(&m.drain, 1);
+    m.abort = 0;
+    m.issued = 0;
+    m.consumed = 0;
+    mbar_fence_init();
+    tma_prefetch_desc(&p.mapA);
+    tma_prefetch_desc(&p.mapB);
+    if (p.mt_sh > 0) {
+      tma_prefetch_desc(&p.mapA_sh);
+      tma_prefetch_desc(&p.mapB_sh);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(&m.tmem_base, TMEM_COLS);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  for (int i = threadIdx.x; i <= p.E; i += NUM_THREADS) {
+    m.mt[i] = p.mt_prefix[i];
+    m.off[i] = p.offsets[i];
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = m.tmem_base;
+  const int routed_total = m.mt[p.E] * p.n_tiles;
+  const int total = routed_total + p.mt_sh * p.n_tiles_sh;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int issued = 0;
+      for (int L = blockIdx.x; L < total; L += gridDim.x) {
+        const Tile t = decode_tile(p, m, L, routed_total, kGateUp);
+        const CUtensorMap* mA = t.sh ? &p.mapA_sh : &p.mapA;
+        const CUtensorMap* mB = t.sh ? &p.mapB_sh : &p.mapB;
+        bool ok = true;
+        for (int kb = 0; kb < t.num_kb; ++kb) {
+          if (!wait_or_abort(&m.empty[s], ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sA = stage_base + (size_t)s * STAGE_BYTES;
+          uint8_t* sB = sA + A_BYTES;
+          mbar_arrive_expect_tx(&m.full[s], STAGE_BYTES);
+          const int kx = kb * BK;
+          tma_load_2d(sA, mA, &m.full[s], kx, t.row0);
+          if (kGateUp) {
+            if (t.sh) {
+              tma_load_3d(sB, mB, &m.full[s], kx, t.n0, 0);
+              tma_load_3d(sB + B_BYTES / 2, mB, &m.full[s], kx, t.n0, 1);
+            } else {
+              tma_load_4d(sB, mB, &m.full[s], kx, t.n0, 0, t.e);
+              tma_load_4d(sB + B_BYTES / 2, mB, &m.full[s], kx, t.n0, 1, t.e);
+            }
+          } else {
+            if (t.sh) tma_load_2d(sB, mB, &m.full[s], kx, t.n0);
+            else tma_load_3d(sB, mB, &m.full[s], kx, t.n0, t.e);
+          }
+          ++issued;
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) {
+          raise_abort(m, p.err);
+          break;
+        }
+      }
+      m.issued = issued;
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int it = 0, consumed = 0;
+      bool ok = true;
+      for (int L = blockIdx.x; L < total && ok; L += gridDim.x, ++it) {
+        const Tile t = decode_tile(p, m, L, routed_total, kGateUp);
+        const int a = it & 1;
+        const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+        if (!wait_or_abort(&m.tempty[a], aph ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(a * BN);
+        for (int kb = 0; kb < t.num_kb; ++kb) {
+          if (!wait_or_abort(&m.full[s], ph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sA = smem_u32(stage_base + (size_t)s * STAGE_BYTES);
+          const uint32_t sB = sA + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = smem_desc_sw128(sA + kk * 32);
+            const uint64_t bd = smem_desc_sw128(sB + kk * 32);
+            tc_mma_f16(d_tmem, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+          }
+          tc_commit(&m.empty[s]);
+          ++consumed;
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&m.tfull[a]);
+      }
+      if (!ok) raise_abort(m, p.err);
+      m.consumed = consumed;
+      // drain: wait until every MMA issued by this thread has completed
+      tc_commit(&m.drain);
+      mbar_wait_bounded(&m.drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------- epilogue (warps 2..5)
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int it = 0;
+    for (int L = blockIdx.x; L < total; L += gridDim.x, ++it) {
+      const Tile t = decode_tile(p, m, L, routed_total, kGateUp);
+      const int a = it & 1;
+      const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+      const bool got = wait_or_abort(&m.tfull[a], aph, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) {
+        if (lane == 0) raise_abort(m, p.err);
+        break;
+      }
+      tc_fence_after();
+      const int row = t.row0 + q * 32 + lane;
+      const bool valid = row < t.row_end;
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * BN);
+      __nv_bfloat16* out = t.sh ? p.out_sh : p.out;
+      const int n_out = t.sh ? p.n_out_sh : p.n_out;
+      if (kGateUp) {
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 16) {
+          float g[16], u[16];
+          tmem_ld16(tb + c, g);
+          tmem_ld16(tb + BN / 2 + c, u);
+          tmem_ld_wait();
+          if (valid && t.n0 + c < n_out) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              pk[i] = pack_bf16x2(silu_mul(g[2 * i], u[2 * i]), silu_mul(g[2 * i + 1], u[2 * i + 1]));
+            uint4* dst = reinterpret_cast<uint4*>(out + (size_t)row * n_out + t.n0 + c);
+            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+          float v[16];
+          tmem_ld16(tb + c, v);
+          tmem_ld_wait();
+          if (valid && t.n0 + c < n_out) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+            uint4* dst = reinterpret_cast<uint4*>(out + (size_t)row * n_out + t.n0 + c);
+            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&m.tempty[a]);
+    }
+  }
+
+  __syncthreads();
+  if (threadIdx.x == 0 && m.abort) {
+    // copies issued but never consumed: wait (bounded) until they land before exiting
+    for (int i = m.consumed; i < m.issued; ++i)
+      mbar_wait_bounded(&m.full[i % STAGES], (uint32_t)(i / STAGES) & 1u);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// bf16 tensor map with a 64-element (128-byte) inner box and 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+              const uint64_t* strides_bytes, const uint32_t* box) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t gd[5], gs[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
+                         gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <bool kGateUp>
+cudaError_t launch_tc(const TcGemmArgs& a, cudaStream_t s) {
+  TcParams p;
+  memset(&p, 0, sizeof(p));
+  const uint64_t d = a.d, f = a.f, fs = a.fs;
+  const uint64_t S = (uint64_t)a.wstride * 2;  // bytes between experts
+  bool ok = true;
+  if (kGateUp) {
+    // A: grouped rows Xp [rows, d]
+    { uint64_t dims[2] = {d, (uint64_t)a.rows}, st[1] = {d * 2}; uint32_t box[2] = {BK, BM};
+      ok &= make_map(&p.mapA, a.A, 2, dims, st, box); }
+    // B: W1|W3 of every expert as [d, f, 2, E]
+    { uint64_t dims[4] = {d, f, 2, (uint64_t)a.E}, st[3] = {d * 2, f * d * 2, S};
+      uint32_t box[4] = {BK, BN / 2, 1, 1};
+      ok &= make_map(&p.mapB, a.W, 4, dims, st, box); }
+    if (a.fs > 0) {
+      { uint64_t dims[2] = {d, (uint64_t)a.rows_sh}, st[1] = {d * 2}; uint32_t box[2] = {BK, BM};
+        ok &= make_map(&p.mapA_sh, a.A_sh, 2, dims, st, box); }
+      { uint64_t dims[3] = {d, fs, 2}, st[2] = {d * 2, fs * d * 2}; uint32_t box[3] = {BK, BN / 2, 1};
+        ok &= make_map(&p.mapB_sh, a.W_sh, 3, dims, st, box); }
+    }
+    p.n_tiles = (int)((f + BN / 2 - 1) / (BN / 2));
+    p.n_tiles_sh = a.fs > 0 ? (int)((fs + BN / 2 - 1) / (BN / 2)) : 0;
+    p.num_kb = (int)((d + BK - 1) / BK);
+    p.num_kb_sh = p.num_kb;
+    p.n_out = (int)f;
+    p.n_out_sh = (int)fs;
+  } else {
+    // A: H [rows, f]
+    { uint64_t dims[2] = {f, (uint64_t)a.rows}, st[1] = {f * 2}; uint32_t box[2] = {BK, BM};
+      ok &= make_map(&p.mapA, a.A, 2, dims, st, box); }
+    // B: W2 of every expert as [f, d, E], starting 2*f*d elements into the expert
+    { uint64_t dims[3] = {f, d, (uint64_t)a.E}, st[2] = {f * 2, S}; uint32_t box[3] = {BK, BN, 1};
+      ok &= make_map(&p.mapB, (const __nv_bfloat16*)a.W + 2 * f * d, 3, dims, st, box); }
+    if (a.fs > 0) {
+      { uint64_t dims[2] = {fs, (uint64_t)a.rows_sh}, st[1] = {fs * 2}; uint32_t box[2] = {BK, BM};
+        ok &= make_map(&p.mapA_sh, a.A_sh, 2, dims, st, box); }
+      { uint64_t dims[2] = {fs, d}, st[1] = {fs * 2}; uint32_t box[2] = {BK, BN};
+        ok &= make_map(&p.mapB_sh, (const __nv_bfloat16*)a.W_sh + 2 * fs * d, 2, dims, st, box); }
+    }
+    p.n_tiles = (int)((d + BN - 1) / BN);
+    p.n_tiles_sh = a.fs > 0 ? p.n_tiles : 0;
+    p.num_kb = (int)((f + BK - 1) / BK);
+    p.num_kb_sh = a.fs > 0 ? (int)((fs + BK - 1) / BK) : 0;
+    p.n_out = (int)d;
+    p.n_out_sh = (int)d;
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  p.offsets = a.offsets;
+  p.mt_prefix = a.mt_prefix;
+  p.E = a.E;
+  p.mt_sh = a.fs > 0 ? (a.rows_sh + BM - 1) / BM : 0;
+  p.rows_sh = a.rows_sh;
+  p.out = (__nv_bfloat16*)a.out;
+  p.out_sh = (__nv_bfloat16*)a.out_sh;
+  p.err = a.err;
+  const long long bound = (long long)a.mt_bound * p.n_tiles + (long long)p.mt_sh * p.n_tiles_sh;
+  int grid = a.sm_count;
+  if (bound < grid) grid = (int)bound;
+  if (grid <= 0) return cudaSuccess;
+  auto kern = tc_ffn_kernel<kGateUp>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_tc_gateup(const TcGemmArgs& a, cudaStream_t s) { return launch_tc<true>(a, s); }
+cudaError_t launch_tc_down(const TcGemmArgs& a, cudaStream_t s) { return launch_tc<false>(a, s); }
+
+}  // namespace colibri

@@ -1,0 +1,173 @@
+// Scatter stage: per-expert histogram, prefix sum and the stable permutation that groups
+// token rows by expert (www.trdm.cn/news/555962 §6.2: batch together the tokens that activate
+// the same expert; www.pptc.cn/news/100465 §3.3: expert offsets as a running sum;
+// www.hotelren.com/news/4731937 §2.3 dispatch_kernel).
+//
+// Row order inside an expert is ascending token index.  It is made deterministic without
+// relying on atomic ordering:
+//   route_count    one CTA per 256 tokens; each warp builds, per expert, the bit mask of its
+//                  32 lanes (tokens) that chose that expert; a token's rank among the earlier
+//                  tokens of its warp is popc(mask & lanes_below); warps are then prefixed in
+//                  order, giving the rank inside the 256-token block and the block's counts.
+//   route_scan     one CTA: per expert, exclusive prefix over blocks; counts; offsets[E+1];
+//                  and the m-tile prefix the grouped GEMM schedules from.
+//   route_scatter  one warp per token: final row = offsets[e] + block base + rank; writes
+//                  src_row / dst_row and copies the token's row into each of its k grouped
+//                  rows with 16-byte vector loads and stores.
+#include "common.cuh"
+
+namespace colibri {
+namespace {
+
+__global__ void __launch_bounds__(kCountBlock) route_count_kernel(const int32_t* __restrict__ idx,
+                                                                  int T, int k, int E,
+                                                                  int32_t* __restrict__ blk_counts,
+                                                                  int32_t* __restrict__ local_rank) {
+  extern __shared__ uint32_t masks[];  // [warps][E]
+  constexpr int W = kCountBlock / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kCountBlock + threadIdx.x;
+  uint32_t* m = masks + warp * E;
+  for (int e = lane; e < E; e += 32) m[e] = 0u;
+  __syncwarp();
+  int ids[kMaxTopK];
+  int rank[kMaxTopK];
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) {
+    ids[j] = 0;
+    rank[j] = 0;
+    if (j < k && t < T) {
+      int e = idx[(size_t)t * k + j];
+      e = min(max(e, 0), E - 1);
+      ids[j] = e;
+      atomicOr(&m[e], 1u << lane);
+    }
+  }
+  __syncwarp();
+  const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j)
+    if (j < k && t < T) rank[j] = __popc(m[ids[j]] & below);
+  __syncthreads();
+  // per expert: exclusive prefix over the warps of this block (masks become bases)
+  for (int e = threadIdx.x; e < E; e += kCountBlock) {
+    int run = 0;
+#pragma unroll
+    for (int w = 0; w < W; ++w) {
+      const int c = __popc(masks[w * E + e]);
+      masks[w * E + e] = (uint32_t)run;
+      run += c;
+    }
+    blk_counts[(size_t)blockIdx.x * E + e] = run;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j)
+    if (j < k && t < T) local_rank[(size_t)t * k + j] = (int)m[ids[j]] + rank[j];
+}
+
+__global__ void __launch_bounds__(256) route_scan_kernel(const int32_t* __restrict__ blk_counts,
+                                                         int nblk, int E, int bm,
+                                                         int32_t* __restrict__ blk_base,
+                                                         int32_t* __restrict__ counts,
+                                                         int32_t* __restrict__ offsets,
+                                                         int32_t* __restrict__ mt_prefix) {
+  __shared__ int tot[kMaxExperts];
+  __shared__ int off[kMaxExperts + 1];
+  __shared__ int mts[kMaxExperts + 1];
+  const int e = threadIdx.x;
+  if (e < E) {
+    int run = 0;
+    for (int b = 0; b < nblk; ++b) {
+      const int c = blk_counts[(size_t)b * E + e];
+      blk_base[(size_t)b * E + e] = run;
+      run += c;
+    }
+    tot[e] = run;
+    counts[e] = run;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int o = 0, mt = 0;
+    for (int q = 0; q < E; ++q) {
+      off[q] = o;
+      mts[q] = mt;
+      o += tot[q];
+      mt += (tot[q] + bm - 1) / bm;
+    }
+    off[E] = o;
+    mts[E] = mt;
+  }
+  __syncthreads();
+  for (int q = threadIdx.x; q <= E; q += blockDim.x) {
+    offsets[q] = off[q];
+    mt_prefix[q] = mts[q];
+  }
+  if (e < E) {
+    const int base = off[e];
+    for (int b = 0; b < nblk; ++b) blk_base[(size_t)b * E + e] += base;
+  }
+}
+
+template <typename Tv>
+__global__ void __launch_bounds__(256) route_scatter_kernel(
+    const Tv* __restrict__ x, int T, int vec_per_row, int k, int E, const int32_t* __restrict__ idx,
+    const int32_t* __restrict__ blk_base, int32_t* __restrict__ dst_row,
+    int32_t* __restrict__ src_row, Tv* __restrict__ Xp) {
+  const int lane = threadIdx.x & 31;
+  const int warps_total = gridDim.x * (blockDim.x >> 5);
+  for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps_total) {
+    int r = 0;
+    if (lane < k) {
+      int e = idx[(size_t)t * k + lane];
+      e = min(max(e, 0), E - 1);
+      r = blk_base[(size_t)(t / kCountBlock) * E + e] + dst_row[(size_t)t * k + lane];
+      dst_row[(size_t)t * k + lane] = r;
+      src_row[r] = t;
+    }
+    int rows[kMaxTopK];
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) rows[j] = __shfl_sync(0xffffffffu, r, j);
+    const Tv* src = x + (size_t)t * vec_per_row;
+    for (int v = lane; v < vec_per_row; v += 32) {
+      const Tv val = __ldg(src + v);
+#pragma unroll
+      for (int j = 0; j < kMaxTopK; ++j)
+        if (j < k) Xp[(size_t)rows[j] * vec_per_row + v] = val;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_route_count(const int32_t* idx, int T, int k, int E, int32_t* blk_counts,
+                               int32_t* local_rank, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  const int nblk = (T + kCountBlock - 1) / kCountBlock;
+  const size_t smem = sizeof(uint32_t) * (kCountBlock / 32) * E;
+  route_count_kernel<<<nblk, kCountBlock, smem, s>>>(idx, T, k, E, blk_counts, local_rank);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_scan(const int32_t* blk_counts, int nblk, int E, int bm, int32_t* blk_base,
+                              int32_t* counts, int32_t* offsets, int32_t* mt_prefix,
+                              cudaStream_t s) {
+  route_scan_kernel<<<1, 256, 0, s>>>(blk_counts, nblk, E, bm, blk_base, counts, offsets, mt_prefix);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_scatter(const void* x, int act, int T, int d, int k, int E,
+                                 const int32_t* idx, const int32_t* blk_base, int32_t* dst_row,
+                                 int32_t* src_row, void* Xp, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  const int esize = (act == COLIBRI_BF16) ? 2 : 4;
+  const int vec = d * esize / 16;  // d is a multiple of 64, rows are whole 16-byte vectors
+  const int warps_per_cta = 8;
+  int grid = (T + warps_per_cta - 1) / warps_per_cta;
+  if (grid > 4096) grid = 4096;
+  route_scatter_kernel<uint4><<<grid, warps_per_cta * 32, 0, s>>>(
+      (const uint4*)x, T, vec, k, E, idx, blk_base, dst_row, src_row, (uint4*)Xp);
+  return cudaGetLastError();
+}
+
+}  // namespace colibri

@@ -1,0 +1,171 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle, element by element.
+
+Small cases are sized so the oracle finishes in seconds while the GPU kernels still cover
+several tiles and ragged tails (rows per expert not a multiple of 128, d_ff not a multiple
+of the 128-column gate/up tile, d not a multiple of the 256-column down tile, empty experts,
+k = 1 and k = E, more than 32 decode tokens on one expert).  The full-size workloads run in
+the launch configuration the benchmark times, with routing compared on every token and the
+layer output on a sample of tokens.
+"""
+import numpy as np
+import pytest
+import torch
+
+import inputgen
+import oracle
+import sparse_expert_ffn_router_b200 as colibri
+from tests import gpu_harness as H
+
+pytestmark = pytest.mark.gpu
+
+BF16, F32, I8 = inputgen.BF16, inputgen.F32, inputgen.I8
+
+SMALL = {
+    # several m-tiles per expert with a ragged tail; f and d both leave partial n-tiles
+    "bf16_ragged": inputgen.custom("bf16_ragged", T=700, d=320, E=4, k=2, f=448),
+    # 16 experts top-4 with a shared expert (the fine-grained layout at small size)
+    "bf16_shared": inputgen.custom("bf16_shared", T=513, d=256, E=16, k=4, f=192, fs=320),
+    # biased router: two hot experts and four experts with exactly zero rows
+    "bf16_empty": inputgen.custom("bf16_empty", T=257, d=128, E=8, k=2, f=256,
+                                  bias=((0, 3.0), (1, 3.0), (4, -30.0), (5, -30.0), (6, -30.0), (7, -30.0))),
+    "bf16_k1_E1": inputgen.custom("bf16_k1_E1", T=130, d=192, E=1, k=1, f=128),
+    "bf16_kE": inputgen.custom("bf16_kE", T=65, d=128, E=8, k=8, f=64),
+    "bf16_T1": inputgen.custom("bf16_T1", T=1, d=256, E=8, k=2, f=256),
+    "f32_tiny": inputgen.WORKLOADS["tiny_f32"],
+    "f32_shared": inputgen.custom("f32_shared", T=100, d=128, E=4, k=2, f=192, fs=64, act=F32, wdt=F32),
+    "i8_small": inputgen.custom("i8_small", T=5, d=256, E=4, k=2, f=512, act=BF16, wdt=I8),
+    # more than 32 tokens on one expert: the decode kernels loop over token chunks
+    "i8_many": inputgen.custom("i8_many", T=80, d=128, E=2, k=1, f=192, act=BF16, wdt=I8),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_parity(name):
+    wl = SMALL[name]
+    p = inputgen.make_problem(wl, seed=0)
+    res = H.parity(p)
+    if name == "bf16_empty":
+        assert res["counts"][4:].sum().item() == 0
+
+
+def test_empty_batch_launches_nothing():
+    wl = SMALL["bf16_ragged"]
+    layer = H.make_layer(wl, max_tokens=16)
+    p = inputgen.make_problem(inputgen.custom("z", T=4, d=wl.d, E=wl.E, k=wl.k, f=wl.f), seed=0)
+    t = H.to_device(p)
+    y = torch.full((4, wl.d), 7.0, dtype=torch.bfloat16, device="cuda")
+    colibri.colibri_moe_forward(layer.ctx, t["x"], 0, t["router_w"], None, t["expert_w"], None, None, y)
+    layer.sync_status()
+    assert torch.all(y == 7.0)
+    layer.close()
+
+
+def test_T_above_max_tokens_is_rejected():
+    wl = SMALL["bf16_T1"]
+    layer = H.make_layer(wl, max_tokens=1)
+    p = inputgen.make_problem(inputgen.custom("two", T=2, d=wl.d, E=wl.E, k=wl.k, f=wl.f), seed=0)
+    t = H.to_device(p)
+    y = torch.empty(2, wl.d, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(colibri.ColibriError) as ei:
+        colibri.colibri_moe_forward(layer.ctx, t["x"], 2, t["router_w"], None, t["expert_w"], None, None, y)
+    assert ei.value.status == -1
+    layer.close()
+
+
+def test_misaligned_and_host_weight_pointers_are_rejected():
+    wl = SMALL["bf16_T1"]
+    layer = H.make_layer(wl)
+    p = inputgen.make_problem(wl, seed=0)
+    t = H.to_device(p)
+    y = torch.empty(1, wl.d, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(colibri.ColibriError) as ei:
+        colibri.colibri_moe_forward(layer.ctx, t["x"].data_ptr() + 2, 1, t["router_w"], None, t["expert_w"],
+                                    None, None, y)
+    assert ei.value.status == -2
+    with pytest.raises(colibri.ColibriError) as ei:  # weights on the host are refused
+        colibri.colibri_moe_forward(layer.ctx, t["x"], 1, t["router_w"], None, p.expert_w, None, None, y)
+    assert ei.value.status == -1
+    with pytest.raises(colibri.ColibriError) as ei:  # scales given for bf16 weights
+        colibri.colibri_moe_forward(layer.ctx, t["x"], 1, t["router_w"], None, t["expert_w"], t["router_w"],
+                                    None, y)
+    assert ei.value.status == -1
+    layer.close()
+
+
+def test_host_x_and_y_match_device_run():
+    wl = SMALL["bf16_shared"]
+    p = inputgen.make_problem(wl, seed=1)
+    layer = H.make_layer(wl)
+    t = H.to_device(p)
+    y_dev = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device="cuda")
+    layer.forward(t["x"], t["router_w"], t["router_b"], t["expert_w"], y_dev, shared_w=t["shared_w"])
+    x_host = p.x.pin_memory()
+    y_host = torch.empty(wl.T, wl.d, dtype=torch.bfloat16).pin_memory()
+    layer.forward(x_host, t["router_w"], t["router_b"], t["expert_w"], y_host, shared_w=t["shared_w"])
+    torch.cuda.synchronize()
+    layer.sync_status()
+    assert torch.equal(y_host, y_dev.cpu())
+    # pageable host memory as well
+    y_page = torch.empty(wl.T, wl.d, dtype=torch.bfloat16)
+    layer.forward(p.x, t["router_w"], t["router_b"], t["expert_w"], y_page, shared_w=t["shared_w"])
+    torch.cuda.synchronize()
+    assert torch.equal(y_page, y_dev.cpu())
+    layer.close()
+
+
+def test_repeated_calls_are_deterministic():
+    wl = SMALL["bf16_ragged"]
+    p = inputgen.make_problem(wl, seed=2)
+    layer = H.make_layer(wl)
+    t = H.to_device(p)
+    outs = []
+    for _ in range(3):
+        outs.append(H.run_gpu(p, layer=layer, dev_inputs=t))
+    for o in outs[1:]:
+        for k in ("y", "idx", "w", "counts", "offsets", "src_row", "dst_row"):
+            assert torch.equal(o[k], outs[0][k]), k
+    layer.close()
+
+
+@pytest.mark.parametrize("name", ["bf16_ragged", "f32_tiny", "i8_small", "bf16_shared"])
+def test_forward_routed_matches_oracle_routing(name):
+    wl = SMALL[name]
+    p = inputgen.make_problem(wl, seed=3)
+    ref = oracle.problem_forward(p)
+    gpu = H.run_gpu(p, routed=(ref["idx"], ref["w"]))
+    assert torch.equal(gpu["idx"], ref["idx"]) and torch.equal(gpu["counts"], ref["counts"])
+    assert torch.equal(gpu["src_row"], ref["src_row"])
+    H.check_y(p, gpu["y"], ref["y"])
+
+
+def test_smaller_T_on_a_larger_context():
+    wl = SMALL["bf16_shared"]
+    layer = H.make_layer(wl, max_tokens=2048)
+    for T in (1, 31, 257):
+        p = inputgen.make_problem(inputgen.custom("sub", T=T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, fs=wl.fs), seed=T)
+        H.parity(p, layer=layer)
+    layer.close()
+
+
+# ------------------------------------------------------------------------- full-size workloads
+
+FULL = [
+    ("mixtral_prefill_bf16", 24),
+    ("fine_grained_shared_bf16", 48),
+    ("skewed_bf16", 24),
+    ("skewed_empty_bf16", 24),
+    ("decode_int8_T1", None),
+    ("decode_int8_T8", None),
+    ("decode_int8_T32", 12),
+]
+
+
+@pytest.mark.parametrize("name,n_sample", FULL)
+def test_full_size_workload(name, n_sample):
+    wl = inputgen.WORKLOADS[name]
+    p = inputgen.make_problem(wl, seed=0)
+    toks = None if n_sample is None else H.sample_tokens(wl.T, n_sample)
+    res = H.parity(p, tokens=toks)
+    if name == "skewed_empty_bf16":
+        assert res["counts"][12:].sum().item() == 0
+    print(f"{name}: rel err {res['rel_err']:.3e}, near-tie tokens {res['near_ties']}")
