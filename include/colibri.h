@@ -186,6 +186,32 @@ colibri_status colibri_sync_status(colibri_ctx* ctx, void* stream);
 colibri_status colibri_profile_begin(colibri_ctx* ctx, int32_t max_calls);
 colibri_status colibri_profile_end(colibri_ctx* ctx, float* stage_ms, int32_t* ncalls);
 
+/*
+ * colibri_route_noalloc -- the Gate and Scatter stages alone (router logits, fp32 softmax,
+ * top-k, per-expert histogram, prefix sum and the stable grouping of token rows), with no
+ * context and no device allocation of any kind.  The pages have no counterpart of this call;
+ * it exists for callers that cannot call cudaMalloc, such as an engine whose device memory is
+ * reserved up front by its own allocator (an extra allocation would fail or fragment it) or a
+ * latency-critical loop that must not pay cudaMalloc's implicit synchronisation.
+ *   x [T, d_model] act_dtype (COLIBRI_F32 or COLIBRI_BF16), router_w [E, d_model] act_dtype,
+ *   router_b [E] fp32 or NULL; outputs topk_idx/topk_w/dst_row [T, k], counts [E],
+ *   offsets [E+1], src_row [T*k] and Xp [T*k, d_model] (x's rows grouped by expert, act_dtype),
+ *   with the meanings of colibri_get_routing.  All buffers are caller-owned device memory of the
+ *   current device, 16-byte aligned.  Work is enqueued on `stream`.
+ * Limits: d_model a multiple of 64, 1 <= E <= 256, 1 <= k <= min(E, 8), and
+ * ceil(T / 256) * E <= 32768 (the size of the built-in scratch array); larger sizes are
+ * rejected with COLIBRI_ERR_INVALID_ARG before anything is launched.  T == 0 launches nothing.
+ * The scratch is one file-scope device array (about 257 KB, held by every GPU that loads the
+ * library until exit).  The first call on each device looks up its address and should come
+ * before any stream capture.  All calls share the array: calls that overlap on the GPU race.
+ * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED, CUDA; reason via colibri_last_error(NULL).
+ */
+colibri_status colibri_route_noalloc(const void* x, int32_t act_dtype, int32_t T, int32_t d_model,
+                                     const void* router_w, const float* router_b,
+                                     int32_t num_experts, int32_t top_k, int32_t* topk_idx,
+                                     float* topk_w, int32_t* counts, int32_t* offsets,
+                                     int32_t* src_row, int32_t* dst_row, void* Xp, void* stream);
+
 /* One-line description of a status code (static storage). */
 const char* colibri_status_string(colibri_status status);
 

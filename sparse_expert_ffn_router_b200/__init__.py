@@ -38,6 +38,7 @@ EXPORTS = (
     "colibri_sync_status",
     "colibri_profile_begin",
     "colibri_profile_end",
+    "colibri_route_noalloc",
     "colibri_status_string",
     "colibri_last_error",
     "colibri_free",
@@ -93,6 +94,8 @@ def load() -> ctypes.CDLL:
     lib.colibri_profile_begin.restype = ctypes.c_int
     lib.colibri_profile_end.argtypes = [vp, vp, vp]
     lib.colibri_profile_end.restype = ctypes.c_int
+    lib.colibri_route_noalloc.argtypes = [vp, i32, i32, i32, vp, vp, i32, i32] + [vp] * 8
+    lib.colibri_route_noalloc.restype = ctypes.c_int
     lib.colibri_status_string.argtypes = [ctypes.c_int]
     lib.colibri_status_string.restype = ctypes.c_char_p
     lib.colibri_last_error.argtypes = [vp]
@@ -188,6 +191,16 @@ def colibri_profile_end(ctx: int):
     n = ctypes.c_int32()
     _check(load().colibri_profile_end(ctx, ms, ctypes.byref(n)), "colibri_profile_end", ctx)
     return dict(zip(STAGE_NAMES, [float(v) for v in ms])), int(n.value)
+
+
+def colibri_route_noalloc(x, act_dtype: int, T: int, d_model: int, router_w, router_b, num_experts: int,
+                          top_k: int, topk_idx, topk_w, counts, offsets, src_row, dst_row, Xp, stream=None) -> None:
+    """Gate + Scatter without a context or any device allocation (see include/colibri.h)."""
+    _check(load().colibri_route_noalloc(_addr(x), act_dtype, T, d_model, _addr(router_w), _addr(router_b),
+                                        num_experts, top_k, _addr(topk_idx), _addr(topk_w), _addr(counts),
+                                        _addr(offsets), _addr(src_row), _addr(dst_row), _addr(Xp),
+                                        _stream(stream)),
+           "colibri_route_noalloc")
 
 
 def colibri_free(ctx: int) -> None:

@@ -91,6 +91,14 @@ struct Carver {
 
 }  // namespace
 
+namespace colibri {
+// Records the reason of a failure of a context-free entry point (read by colibri_last_error(NULL)).
+void record_error(const char* msg) {
+  g_last_error = msg;
+  if (env_flag("COLIBRI_DEBUG")) fprintf(stderr, "[colibri] %s\n", msg);
+}
+}  // namespace colibri
+
 extern "C" {
 
 const char* colibri_status_string(colibri_status st) {
