@@ -36,7 +36,7 @@ KERNELS_PER_STEP_BASE = 7  # router, count, scan, scatter, gate/up, down, combin
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="colibri", choices=["colibri", "reference"])
@@ -77,58 +77,74 @@ def work(wl, counts):
 
 
 class ClockSampler:
-    """nvidia-smi clocks/throttle sampling every 200 ms during the timed region."""
+    """Samples the SM clock and clock-event reasons through NVML (read-only queries) every
+    20 ms on a background thread during the timed region."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
+    def __init__(self, pci_bus_id: str):
+        self.pci = pci_bus_id
+        self.samples = []
+        self.max_mhz = None
+        self.error = None
 
     def __enter__(self):
+        import threading
+
+        self.stop = threading.Event()
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(self.pci.encode() if isinstance(self.pci, str) else self.pci)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.sample()
+        except Exception as exc:  # NVML missing or unreadable: report unsampled
+            self.error = repr(exc)
+            self.nv = None
+            return self
+        self.thread = threading.Thread(target=self.loop, daemon=True)
+        self.thread.start()
         return self
 
+    def sample(self):
+        nv = self.nv
+        mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+        reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        self.samples.append((mhz, reasons))
+
+    def loop(self):
+        while not self.stop.wait(0.02):
+            try:
+                self.sample()
+            except Exception:
+                break
+
     def __exit__(self, *exc):
-        self.samples = []
-        if self.proc is None:
-            return False
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        for line in out.splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                self.samples.append(parts)
+        self.stop.set()
+        if self.nv is not None:
+            self.thread.join(timeout=2)
+            try:
+                self.sample()
+            except Exception:
+                pass
         return False
 
     def summary(self):
-        s = getattr(self, "samples", [])
-        if not s:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-
-        def num(v):
-            try:
-                return float(v)
-            except ValueError:
-                return None
-
-        sm = [num(p[1]) for p in s if num(p[1]) is not None]
-        mx = [num(p[2]) for p in s if num(p[2]) is not None]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for p in s for n, v in zip(names, p[5:9]) if v.strip().lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(s)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"], "samples": 0,
+                    "error": self.error}
+        nv = self.nv
+        mhz = [m for m, _ in self.samples]
+        active = sorted({name for _, bits in self.samples for name, const in self.REASONS
+                         if bits & getattr(nv, const, 0)})
+        return {"sm_mhz": statistics.median(mhz), "sm_min_mhz": min(mhz), "sm_max_mhz": self.max_mhz,
+                "reasons": active, "samples": len(mhz), "source": "NVML, 20 ms"}
 
 
 def cpu_baseline(p, n_tokens, seed_tokens=None):
@@ -266,7 +282,9 @@ def main():
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     colibri.colibri_profile_begin(layer.ctx, a.steps)
     barrier()
-    with ClockSampler(local) as clk:
+    props = torch.cuda.get_device_properties(dev)
+    pci = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+    with ClockSampler(pci) as clk:
         ev0.record(stream)
         for _ in range(a.steps):
             step(x, y)

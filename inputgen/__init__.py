@@ -149,6 +149,10 @@ WORKLOADS = {
                                   bias=((0, 4.0), (1, 4.0), (12, -30.0), (13, -30.0), (14, -30.0),
                                         (15, -30.0)),
                                   note="skewed routing with four experts forced empty"),
+    # the Mixtral-shaped layer with 4 experts and 1024 tokens: the same kernels and tile shapes
+    # on ~1.5 GB of device memory (still far larger than L2), sized for ncu captures
+    "mixtral_prefill_bf16_small": Workload("mixtral_prefill_bf16_small", 1024, 4096, 4, 2, 14336,
+                                           note="profiling-size Mixtral-shaped layer"),
     # decode, int8 weights with per-output-channel scales
     "decode_int8_T1": Workload("decode_int8_T1", 1, 4096, 8, 2, 14336, act=BF16, wdt=I8),
     "decode_int8_T8": Workload("decode_int8_T8", 8, 4096, 8, 2, 14336, act=BF16, wdt=I8),
