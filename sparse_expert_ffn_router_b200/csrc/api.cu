@@ -79,6 +79,16 @@ int pick_dec_split(int f) {
   return 1;
 }
 
+// Pair (2-CTA) tiles for the bf16 expert GEMMs.  COLIBRI_GEMM_CTA=1 or 2 forces a mode
+// (both are exact; this only selects the tile shape).
+bool use_pair_tiles(const colibri_ctx* ctx, int avg_rows_per_expert) {
+  const char* v = getenv("COLIBRI_GEMM_CTA");
+  if (v && v[0] == '1') return false;
+  if (v && v[0] == '2') return true;
+  (void)ctx;
+  return avg_rows_per_expert >= 512;
+}
+
 // Workspace carve-out: every buffer 256-byte aligned inside one allocation.
 struct Carver {
   size_t off = 0;
@@ -333,7 +343,10 @@ colibri_status forward_impl(colibri_ctx* ctx, const void* x, int32_t T, const vo
 
   // ---- Scatter
   const int nblk = (T + kCountBlock - 1) / kCountBlock;
-  const int bm = D.weight_dtype == COLIBRI_F32 ? kSimtBM : kTcBM;
+  // bf16 weights: pair tiles (two CTAs, 256 rows) when experts average >= 512 rows, where the
+  // halved L2 traffic per unit of work outweighs the larger last tile of each expert.
+  const bool pair_tiles = D.weight_dtype == COLIBRI_BF16 && use_pair_tiles(ctx, T * k / E);
+  const int bm = D.weight_dtype == COLIBRI_F32 ? kSimtBM : (pair_tiles ? kTcPairBM : kTcBM);
   COLIBRI_TRY(launch_route_count(w.topk_idx, T, k, E, w.blk_counts, w.dst_row, s), "route_count");
   COLIBRI_TRY(launch_route_scan(w.blk_counts, nblk, E, bm, w.blk_base, w.counts, w.offsets, w.mt_prefix, s), "route_scan");
   COLIBRI_TRY(launch_route_scatter(xd, act, T, d, k, E, w.topk_idx, w.blk_base, w.dst_row, w.src_row, w.Xp, s),
@@ -376,9 +389,10 @@ colibri_status forward_impl(colibri_ctx* ctx, const void* x, int32_t T, const vo
     a.d = d;
     a.f = f;
     a.fs = fs;
-    a.mt_bound = R / kTcBM + E;
+    a.mt_bound = R / bm + E;
     a.err = w.err;
     a.sm_count = ctx->sm_count;
+    a.pair = pair_tiles;
     COLIBRI_TRY(launch_tc_gateup(a, s), "tc_gateup");
     mark(3);
     a.A = w.H;

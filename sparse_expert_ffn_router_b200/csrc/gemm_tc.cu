@@ -79,8 +79,9 @@ struct Tile {
   int e, row0, row_end, n0, num_kb;
 };
 
-__device__ __forceinline__ Tile decode_tile(const TcParams& p, const SmemMisc& m, int L,
-                                            int routed_total, bool gateup) {
+template <typename Misc>
+__device__ __forceinline__ Tile decode_tile(const TcParams& p, const Misc& m, int L, int routed_total,
+                                            bool gateup, int bm = BM) {
   Tile t;
   const int ncols = gateup ? BN / 2 : BN;
   if (L < routed_total) {
@@ -96,7 +97,7 @@ __device__ __forceinline__ Tile decode_tile(const TcParams& p, const SmemMisc& m
     const int n = Lp / Me, mm = Lp - n * Me;
     t.sh = false;
     t.e = lo;
-    t.row0 = m.off[lo] + mm * BM;
+    t.row0 = m.off[lo] + mm * bm;
     t.row_end = m.off[lo + 1];
     t.n0 = n * ncols;
     t.num_kb = p.num_kb;
@@ -105,7 +106,7 @@ __device__ __forceinline__ Tile decode_tile(const TcParams& p, const SmemMisc& m
     const int n = Lp / p.mt_sh, mm = Lp - n * p.mt_sh;
     t.sh = true;
     t.e = 0;
-    t.row0 = mm * BM;
+    t.row0 = mm * bm;
     t.row_end = p.rows_sh;
     t.n0 = n * ncols;
     t.num_kb = p.num_kb_sh;
@@ -127,7 +128,8 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
   }
 }
 
-__device__ __forceinline__ void raise_abort(SmemMisc& m, uint32_t* err) {
+template <typename Misc>
+__device__ __forceinline__ void raise_abort(Misc& m, uint32_t* err) {
   *(volatile int*)&m.abort = 1;
   atomicOr(err, kErrWaitTimeout);
 }
@@ -348,6 +350,247 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ffn_kernel(const __grid_con
   }
 }
 
+// ------------------------------------------------------------------------- pair kernel
+// The same grouped GEMM with clusters of two CTAs and tcgen05 cta_group::2: a pair computes a
+// 256 x 256 tile; each CTA loads its own 128 rows of A and its own 128 rows (N) of B (for
+// gate/up: the leader W1, the peer W3), so a stage is 32 KB and six stages fit.  The leader
+// issues the M=256 MMAs, which read both CTAs' shared memory and write 128 rows into each
+// CTA's TMEM; its commits arrive on both CTAs' barriers (multicast commit).  Both CTAs' copies
+// count on the leader's full barrier; both epilogues release the accumulator on the leader's
+// barrier.  Per 128x256x64 unit of work a CTA moves 32 KB from L2 instead of 48 KB.
+constexpr int BM2 = 256;
+constexpr int STAGES2 = kTcPairStages;
+constexpr int HALF_BYTES = 128 * BK * 2;          // 16 KB
+constexpr int STAGE2_BYTES = 2 * HALF_BYTES;      // A half + B half
+constexpr uint32_t IDESC2 = idesc_bf16_f32(BM2, BN);
+
+struct SmemMisc2 {
+  uint64_t full[STAGES2];    // used in the leader: both CTAs' copies (64 KB per phase)
+  uint64_t empty[STAGES2];   // per CTA: freed by the leader's multicast commit
+  uint64_t tfull[2];         // per CTA: accumulator ready (multicast commit)
+  uint64_t tempty[2];        // used in the leader: 8 epilogue-warp arrivals (4 local, 4 peer)
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int32_t mt[kMaxExperts + 1];
+  int32_t off[kMaxExperts + 1];
+};
+
+constexpr size_t SMEM2_BYTES = (size_t)STAGES2 * STAGE2_BYTES + sizeof(SmemMisc2);
+static_assert(SMEM2_BYTES <= 232448, "pair-tile stages exceed the shared memory of one CTA");
+
+template <bool kGateUp>
+__global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_constant__ TcParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // The 128-byte swizzle needs 1024-byte aligned stages; the dynamic shared window of a CTA
+  // starts 1024-byte aligned (both CTAs of a pair take this branch together).
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) atomicOr(p.err, kErrWaitTimeout);
+    return;
+  }
+  uint8_t* smem = smem_raw;
+  uint8_t* stage_base = smem;
+  SmemMisc2& m = *reinterpret_cast<SmemMisc2*>(smem + (size_t)STAGES2 * STAGE2_BYTES);
+  volatile int* abort_flag = &m.abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = (int)cluster_id_x(), npairs = (int)num_clusters_x();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES2; ++s) {
+      mbar_init(&m.full[s], 1);
+      mbar_init(&m.empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&m.tfull[a], 1);
+      mbar_init(&m.tempty[a], 8);
+    }
+    mbar_init(&m.drain, 1);
+    m.abort = 0;
+    mbar_fence_init();
+    tma_prefetch_desc(&p.mapA);
+    tma_prefetch_desc(&p.mapB);
+    if (p.mt_sh > 0) {
+      tma_prefetch_desc(&p.mapA_sh);
+      tma_prefetch_desc(&p.mapB_sh);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&m.tmem_base, TMEM_COLS);
+    tmem_relinquish_pair();
+    tc_fence_before();
+  }
+  for (int i = threadIdx.x; i <= p.E; i += NUM_THREADS) {
+    m.mt[i] = p.mt_prefix[i];
+    m.off[i] = p.offsets[i];
+  }
+  __syncthreads();
+  cluster_sync_all();  // the peer's barriers are initialised before any cross-CTA arrival
+  tc_fence_after();
+  const uint32_t tmem_base = m.tmem_base;
+  const int routed_total = m.mt[p.E] * p.n_tiles;
+  const int total = routed_total + p.mt_sh * p.n_tiles_sh;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- TMA producer (both CTAs)
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      for (int L = pair; L < total; L += npairs) {
+        const Tile t = decode_tile(p, m, L, routed_total, kGateUp, BM2);
+        const CUtensorMap* mA = t.sh ? &p.mapA_sh : &p.mapA;
+        const CUtensorMap* mB = t.sh ? &p.mapB_sh : &p.mapB;
+        const int arow = t.row0 + 128 * (int)rank;
+        bool ok = true;
+        for (int kb = 0; kb < t.num_kb; ++kb) {
+          if (!wait_or_abort(&m.empty[s], ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sA = stage_base + (size_t)s * STAGE2_BYTES;
+          uint8_t* sB = sA + HALF_BYTES;
+          if (rank == 0) mbar_arrive_expect_tx(&m.full[s], 2 * STAGE2_BYTES);
+          const uint32_t bar = mapa_shared(smem_u32(&m.full[s]), 0);
+          const int kx = kb * BK;
+          tma2_load_2d(sA, mA, bar, kx, arow);
+          if (kGateUp) {
+            if (t.sh) tma2_load_3d(sB, mB, bar, kx, t.n0, (int)rank);
+            else tma2_load_4d(sB, mB, bar, kx, t.n0, (int)rank, t.e);
+          } else {
+            if (t.sh) tma2_load_2d(sB, mB, bar, kx, t.n0 + 128 * (int)rank);
+            else tma2_load_3d(sB, mB, bar, kx, t.n0 + 128 * (int)rank, t.e);
+          }
+          if (++s == STAGES2) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) {
+          raise_abort(m, p.err);
+          break;
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer (leader only)
+    if (lane == 0 && rank == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int it = 0;
+      bool ok = true;
+      for (int L = pair; L < total && ok; L += npairs, ++it) {
+        const Tile t = decode_tile(p, m, L, routed_total, kGateUp, BM2);
+        const int a = it & 1;
+        const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+        if (!wait_or_abort(&m.tempty[a], aph ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(a * BN);
+        for (int kb = 0; kb < t.num_kb; ++kb) {
+          if (!wait_or_abort(&m.full[s], ph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sA = smem_u32(stage_base + (size_t)s * STAGE2_BYTES);
+          const uint32_t sB = sA + HALF_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = smem_desc_sw128(sA + kk * 32);
+            const uint64_t bd = smem_desc_sw128(sB + kk * 32);
+            tc_mma_f16_pair(d_tmem, ad, bd, IDESC2, (kb | kk) != 0 ? 1u : 0u);
+          }
+          tc_commit_pair_mc(&m.empty[s], 0x3);
+          if (++s == STAGES2) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(&m.tfull[a], 0x3);
+      }
+      if (!ok) raise_abort(m, p.err);
+      tc_commit_pair(&m.drain);
+      mbar_wait_bounded(&m.drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------- epilogue (warps 2..5, both CTAs)
+    const int q = warp & 3;
+    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&m.tempty[0]), 0);
+    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&m.tempty[1]), 0);
+    int it = 0;
+    for (int L = pair; L < total; L += npairs, ++it) {
+      const Tile t = decode_tile(p, m, L, routed_total, kGateUp, BM2);
+      const int a = it & 1;
+      const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+      const bool got = wait_or_abort(&m.tfull[a], aph, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) {
+        if (lane == 0) raise_abort(m, p.err);
+        break;
+      }
+      tc_fence_after();
+      const int row = t.row0 + 128 * (int)rank + q * 32 + lane;
+      const bool valid = row < t.row_end;
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * BN);
+      __nv_bfloat16* out = t.sh ? p.out_sh : p.out;
+      const int n_out = t.sh ? p.n_out_sh : p.n_out;
+      if (kGateUp) {
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 16) {
+          float g[16], u[16];
+          tmem_ld16(tb + c, g);
+          tmem_ld16(tb + BN / 2 + c, u);
+          tmem_ld_wait();
+          if (valid && t.n0 + c < n_out) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              pk[i] = pack_bf16x2(silu_mul(g[2 * i], u[2 * i]), silu_mul(g[2 * i + 1], u[2 * i + 1]));
+            uint4* dst = reinterpret_cast<uint4*>(out + (size_t)row * n_out + t.n0 + c);
+            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+          float v[16];
+          tmem_ld16(tb + c, v);
+          tmem_ld_wait();
+          if (valid && t.n0 + c < n_out) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+            uint4* dst = reinterpret_cast<uint4*>(out + (size_t)row * n_out + t.n0 + c);
+            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(a ? tempty_leader1 : tempty_leader0);
+    }
+  }
+
+  __syncthreads();
+  if (threadIdx.x == 0 && m.abort) {
+    // error path: give copies still in flight time to land before the CTA leaves
+    const unsigned long long t0 = global_ns();
+    while (global_ns() - t0 < 2000000ull) {
+    }
+  }
+  cluster_sync_all();  // the peer no longer reads this CTA's shared memory or arrives on it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------------- host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -389,6 +632,9 @@ bool make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims
 
 template <bool kGateUp>
 cudaError_t launch_tc(const TcGemmArgs& a, cudaStream_t s) {
+  const bool pair = a.pair;
+  const int bm = pair ? BM2 : BM;
+  const uint32_t b_rows_down = pair ? 128 : BN;
   TcParams p;
   memset(&p, 0, sizeof(p));
   const uint64_t d = a.d, f = a.f, fs = a.fs;
@@ -419,12 +665,12 @@ cudaError_t launch_tc(const TcGemmArgs& a, cudaStream_t s) {
     { uint64_t dims[2] = {f, (uint64_t)a.rows}, st[1] = {f * 2}; uint32_t box[2] = {BK, BM};
       ok &= make_map(&p.mapA, a.A, 2, dims, st, box); }
     // B: W2 of every expert as [f, d, E], starting 2*f*d elements into the expert
-    { uint64_t dims[3] = {f, d, (uint64_t)a.E}, st[2] = {f * 2, S}; uint32_t box[3] = {BK, BN, 1};
+    { uint64_t dims[3] = {f, d, (uint64_t)a.E}, st[2] = {f * 2, S}; uint32_t box[3] = {BK, b_rows_down, 1};
       ok &= make_map(&p.mapB, (const __nv_bfloat16*)a.W + 2 * f * d, 3, dims, st, box); }
     if (a.fs > 0) {
       { uint64_t dims[2] = {fs, (uint64_t)a.rows_sh}, st[1] = {fs * 2}; uint32_t box[2] = {BK, BM};
         ok &= make_map(&p.mapA_sh, a.A_sh, 2, dims, st, box); }
-      { uint64_t dims[2] = {fs, d}, st[1] = {fs * 2}; uint32_t box[2] = {BK, BN};
+      { uint64_t dims[2] = {fs, d}, st[1] = {fs * 2}; uint32_t box[2] = {BK, b_rows_down};
         ok &= make_map(&p.mapB_sh, (const __nv_bfloat16*)a.W_sh + 2 * fs * d, 2, dims, st, box); }
     }
     p.n_tiles = (int)((d + BN - 1) / BN);
@@ -438,19 +684,43 @@ cudaError_t launch_tc(const TcGemmArgs& a, cudaStream_t s) {
   p.offsets = a.offsets;
   p.mt_prefix = a.mt_prefix;
   p.E = a.E;
-  p.mt_sh = a.fs > 0 ? (a.rows_sh + BM - 1) / BM : 0;
+  p.mt_sh = a.fs > 0 ? (a.rows_sh + bm - 1) / bm : 0;
   p.rows_sh = a.rows_sh;
   p.out = (__nv_bfloat16*)a.out;
   p.out_sh = (__nv_bfloat16*)a.out_sh;
   p.err = a.err;
   const long long bound = (long long)a.mt_bound * p.n_tiles + (long long)p.mt_sh * p.n_tiles_sh;
-  int grid = a.sm_count;
-  if (bound < grid) grid = (int)bound;
-  if (grid <= 0) return cudaSuccess;
-  auto kern = tc_ffn_kernel<kGateUp>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  if (!pair) {
+    int grid = a.sm_count;
+    if (bound < grid) grid = (int)bound;
+    if (grid <= 0) return cudaSuccess;
+    auto kern = tc_ffn_kernel<kGateUp>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(p);
+    return cudaGetLastError();
+  }
+  int pairs = a.sm_count / 2;
+  if (bound < pairs) pairs = (int)bound;
+  if (pairs <= 0) return cudaSuccess;
+  auto kern = tc2_ffn_kernel<kGateUp>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM2_BYTES);
   if (e != cudaSuccess) return e;
-  kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(p);
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = SMEM2_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

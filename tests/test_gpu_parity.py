@@ -48,6 +48,26 @@ def test_small_parity(name):
         assert res["counts"][4:].sum().item() == 0
 
 
+BF16_SMALL = [n for n, w in SMALL.items() if w.wdt == BF16]
+
+
+@pytest.mark.parametrize("mode", ["1", "2"])
+@pytest.mark.parametrize("name", BF16_SMALL)
+def test_small_parity_each_tile_mode(name, mode, monkeypatch):
+    # "1": one CTA per 128-row tile; "2": clusters of two CTAs with 256-row pair tiles
+    monkeypatch.setenv("COLIBRI_GEMM_CTA", mode)
+    wl = SMALL[name]
+    H.parity(inputgen.make_problem(wl, seed=5))
+
+
+@pytest.mark.parametrize("mode", ["1", "2"])
+def test_mixtral_each_tile_mode(mode, monkeypatch):
+    monkeypatch.setenv("COLIBRI_GEMM_CTA", mode)
+    wl = inputgen.WORKLOADS["mixtral_prefill_bf16_small"]
+    p = inputgen.make_problem(wl, seed=0)
+    H.parity(p, tokens=H.sample_tokens(wl.T, 12))
+
+
 def test_empty_batch_launches_nothing():
     wl = SMALL["bf16_ragged"]
     layer = H.make_layer(wl, max_tokens=16)
