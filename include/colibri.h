@@ -121,6 +121,10 @@ int64_t colibri_expert_stride(const colibri_ctx* ctx);
  *   stream       cudaStream_t.
  * Every device pointer must be 16-byte aligned.  Errors: INVALID_ARG, ALIGNMENT, CUDA.
  * A device-side wait that gives up is reported later by colibri_sync_status().
+ * When x and y are device memory, `stream` is not the legacy default stream, no profiling is
+ * active and the stream is not itself being captured, the launch sequence is captured into a
+ * CUDA graph the first time a given argument set is seen and replayed on later calls with the
+ * same arguments (up to 8 argument sets per context; COLIBRI_GRAPHS=0 disables this).
  * With COLIBRI_PROFILE=1 in the environment the call records CUDA events per stage,
  * synchronises the stream and prints one line "Gate | Scatter | ExpertCompute | Gather |
  * Total" in milliseconds to stderr (the stage profile of www.0539edu.com/news/4774449 §3.3).

@@ -89,6 +89,8 @@ bool use_pair_tiles(const colibri_ctx* ctx, int avg_rows_per_expert) {
   return avg_rows_per_expert >= 512;
 }
 
+constexpr size_t kMaxGraphs = 8;  // captured forwards kept per context (least recently used evicted)
+
 // Workspace carve-out: every buffer 256-byte aligned inside one allocation.
 struct Carver {
   size_t off = 0;
@@ -202,6 +204,9 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   const size_t o_ysh = c.take(fs > 0 ? M * d * hs : 0);
   const int64_t part_rows = i8 ? std::max<int64_t>(R, (int64_t)ctx->dec_split * std::min<int64_t>(R, 256)) : 0;
   const size_t o_part = c.take(part_rows * d * 4);
+  const size_t plane_w = (size_t)std::max<int64_t>(d, f);
+  const size_t o_phi = c.take(i8 ? R * plane_w : 0), o_plo = c.take(i8 ? R * plane_w : 0);
+  const size_t o_psc = c.take(i8 ? R * 4 : 0);
   const size_t o_err = c.take(4);
   ctx->ws_bytes = c.off;
 
@@ -231,6 +236,9 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   w.Hs = b + o_hs;
   w.Ys = b + o_ysh;
   w.Ypart = reinterpret_cast<float*>(b + o_part);
+  w.plane_hi = reinterpret_cast<int8_t*>(b + o_phi);
+  w.plane_lo = reinterpret_cast<int8_t*>(b + o_plo);
+  w.plane_scale = reinterpret_cast<float*>(b + o_psc);
   w.err = reinterpret_cast<uint32_t*>(b + o_err);
   if (cudaMemset(w.err, 0, 4) != cudaSuccess) {
     cudaFree(ctx->ws_base);
@@ -239,6 +247,15 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   }
   if (ctx->profile) {
     for (auto& e : ctx->ev) cudaEventCreate(&e);
+  }
+  ctx->use_graphs = !(getenv("COLIBRI_GRAPHS") && strcmp(getenv("COLIBRI_GRAPHS"), "0") == 0);
+  cudaError_t ce = configure_router_kernels();
+  if (ce == cudaSuccess) ce = configure_tc_kernels();
+  if (ce != cudaSuccess) {
+    cudaGetLastError();
+    cudaFree(ctx->ws_base);
+    delete ctx;
+    return fail(nullptr, COLIBRI_ERR_CUDA, "kernel configuration failed: %s", cudaGetErrorString(ce));
   }
   *out = ctx;
   return COLIBRI_OK;
@@ -253,6 +270,7 @@ void colibri_free(colibri_ctx* ctx) {
       if (e) cudaEventDestroy(e);
     for (auto& e : ctx->prof_ev)
       if (e) cudaEventDestroy(e);
+    for (auto& g : ctx->graphs) cudaGraphExecDestroy(g.exec);
   }
   delete ctx;
 }
@@ -272,44 +290,14 @@ colibri_status check_launch(colibri_ctx* ctx, cudaError_t e, const char* what) {
     if (st_ != COLIBRI_OK) return st_;                          \
   } while (0)
 
-// Shared body of both forward entry points.  topk_idx/topk_w non-NULL = caller routing.
-colibri_status forward_impl(colibri_ctx* ctx, const void* x, int32_t T, const void* router_w,
-                            const float* router_b, const int32_t* user_idx, const float* user_w,
-                            const void* expert_w, const float* expert_scales, const void* shared_w,
-                            void* y, void* stream_ptr) {
-  if (!ctx) return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "ctx is NULL");
+// The launch sequence of one forward (stream-ordered, no host synchronisation unless
+// COLIBRI_PROFILE printing is on).
+colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int32_t T, const void* router_w,
+                               const float* router_b, const int32_t* user_idx, const float* user_w,
+                               const void* expert_w, const float* expert_scales, const void* shared_w, void* y,
+                               PtrKind yk, cudaStream_t s, bool pair_tiles) {
   const colibri_desc& D = ctx->desc;
-  const bool routed_by_caller = user_idx != nullptr || user_w != nullptr;
-  if (T < 0 || T > D.max_tokens)
-    return fail(ctx, COLIBRI_ERR_INVALID_ARG, "T=%d outside [0, max_tokens=%d]", T, D.max_tokens);
-  if (!x || !expert_w || !y) return fail(ctx, COLIBRI_ERR_INVALID_ARG, "x, expert_w and y must be non-NULL");
-  if (routed_by_caller) {
-    if (!user_idx || !user_w) return fail(ctx, COLIBRI_ERR_INVALID_ARG, "topk_idx and topk_w must both be given");
-  } else if (!router_w) {
-    return fail(ctx, COLIBRI_ERR_INVALID_ARG, "router_w is NULL");
-  }
-  const bool i8 = D.weight_dtype == COLIBRI_I8;
-  if (i8 != (expert_scales != nullptr))
-    return fail(ctx, COLIBRI_ERR_INVALID_ARG, "expert_scales must be given exactly when weights are int8");
-  if ((D.shared_d_ff > 0) != (shared_w != nullptr))
-    return fail(ctx, COLIBRI_ERR_INVALID_ARG, "shared_w must be given exactly when shared_d_ff > 0");
-  const void* ptrs[] = {x, router_w, router_b, expert_w, expert_scales, shared_w, y, user_idx, user_w};
-  for (const void* p : ptrs)
-    if (p && !aligned16(p)) return fail(ctx, COLIBRI_ERR_ALIGNMENT, "pointer %p is not 16-byte aligned", p);
-  ctx->last_T = T;
-  if (T == 0) return COLIBRI_OK;
-
-  DeviceGuard guard(D.device_id);
-  const int dev = D.device_id;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_ptr);
-  const void* dev_only[] = {router_w, router_b, expert_w, expert_scales, shared_w, user_idx, user_w};
-  for (const void* p : dev_only)
-    if (p && classify(p, dev) != kPtrDevice)
-      return fail(ctx, COLIBRI_ERR_INVALID_ARG, "pointer %p is not device memory of device %d", p, dev);
-  const PtrKind xk = classify(x, dev), yk = classify(y, dev);
-  if (xk == kPtrBad || yk == kPtrBad)
-    return fail(ctx, COLIBRI_ERR_INVALID_ARG, "x or y is device memory of another device");
-
+  const bool routed_by_caller = user_idx != nullptr;
   Workspace& w = ctx->ws;
   const int d = D.d_model, f = D.d_ff, fs = D.shared_d_ff, E = D.num_experts, k = D.top_k;
   const int act = D.act_dtype;
@@ -337,20 +325,24 @@ colibri_status forward_impl(colibri_ctx* ctx, const void* x, int32_t T, const vo
     COLIBRI_TRY(cudaMemcpyAsync(w.topk_idx, user_idx, (size_t)R * 4, cudaMemcpyDeviceToDevice, s), "copy topk_idx");
     COLIBRI_TRY(cudaMemcpyAsync(w.topk_w, user_w, (size_t)R * 4, cudaMemcpyDeviceToDevice, s), "copy topk_w");
   } else {
-    COLIBRI_TRY(launch_router_topk(xd, act, T, d, router_w, router_b, E, k, w.topk_idx, w.topk_w, s), "router_topk");
+    COLIBRI_TRY(launch_router_topk(xd, act, T, d, router_w, router_b, E, k, w.topk_idx, w.topk_w, w.err, s),
+                "router_topk");
   }
   mark(1);
 
   // ---- Scatter
   const int nblk = (T + kCountBlock - 1) / kCountBlock;
-  // bf16 weights: pair tiles (two CTAs, 256 rows) when experts average >= 512 rows, where the
-  // halved L2 traffic per unit of work outweighs the larger last tile of each expert.
-  const bool pair_tiles = D.weight_dtype == COLIBRI_BF16 && use_pair_tiles(ctx, T * k / E);
   const int bm = D.weight_dtype == COLIBRI_F32 ? kSimtBM : (pair_tiles ? kTcPairBM : kTcBM);
-  COLIBRI_TRY(launch_route_count(w.topk_idx, T, k, E, w.blk_counts, w.dst_row, s), "route_count");
-  COLIBRI_TRY(launch_route_scan(w.blk_counts, nblk, E, bm, w.blk_base, w.counts, w.offsets, w.mt_prefix, s), "route_scan");
-  COLIBRI_TRY(launch_route_scatter(xd, act, T, d, k, E, w.topk_idx, w.blk_base, w.dst_row, w.src_row, w.Xp, s),
-              "route_scatter");
+  if (T <= kFusedRouteMaxT) {
+    COLIBRI_TRY(launch_route_fused(xd, act, T, d, w.topk_idx, k, E, bm, w.counts, w.offsets, w.mt_prefix,
+                                   w.src_row, w.dst_row, w.Xp, s), "route_fused");
+  } else {
+    COLIBRI_TRY(launch_route_count(w.topk_idx, T, k, E, w.blk_counts, w.dst_row, s), "route_count");
+    COLIBRI_TRY(launch_route_scan(w.blk_counts, nblk, E, bm, w.blk_base, w.counts, w.offsets, w.mt_prefix, s),
+                "route_scan");
+    COLIBRI_TRY(launch_route_scatter(xd, act, T, d, k, E, w.topk_idx, w.blk_base, w.dst_row, w.src_row, w.Xp, s),
+                "route_scatter");
+  }
   mark(2);
 
   // ---- Expert compute
@@ -402,11 +394,15 @@ colibri_status forward_impl(colibri_ctx* ctx, const void* x, int32_t T, const vo
     COLIBRI_TRY(launch_tc_down(a, s), "tc_down");
   } else {
     nsplit = R <= 256 ? ctx->dec_split : 1;
-    COLIBRI_TRY(launch_dec_gateup((const __nv_bfloat16*)w.Xp, (const int8_t*)expert_w, expert_scales, stride, d,
-                                  f, E, w.offsets, (__nv_bfloat16*)w.H, s), "dec_gateup");
+    COLIBRI_TRY(launch_dec_split((const __nv_bfloat16*)w.Xp, R, d, w.plane_hi, w.plane_lo, w.plane_scale, s),
+                "dec_split_x");
+    COLIBRI_TRY(launch_dec_gateup(w.plane_hi, w.plane_lo, w.plane_scale, (const int8_t*)expert_w, expert_scales,
+                                  stride, d, f, E, w.offsets, (__nv_bfloat16*)w.H, T, s), "dec_gateup");
     mark(3);
-    COLIBRI_TRY(launch_dec_down((const __nv_bfloat16*)w.H, (const int8_t*)expert_w, expert_scales, stride, d, f,
-                                E, w.offsets, nsplit, R, w.Ypart, s), "dec_down");
+    COLIBRI_TRY(launch_dec_split((const __nv_bfloat16*)w.H, R, f, w.plane_hi, w.plane_lo, w.plane_scale, s),
+                "dec_split_h");
+    COLIBRI_TRY(launch_dec_down(w.plane_hi, w.plane_lo, w.plane_scale, (const int8_t*)expert_w, expert_scales,
+                                stride, d, f, E, w.offsets, nsplit, R, w.Ypart, T, s), "dec_down");
   }
   mark(4);
 
@@ -432,6 +428,105 @@ colibri_status forward_impl(colibri_ctx* ctx, const void* x, int32_t T, const vo
             T, ms[0], ms[1], ms[2] + ms[3], ms[4], tot);
   }
   return COLIBRI_OK;
+}
+
+// Shared body of both forward entry points.  topk_idx/topk_w non-NULL = caller routing.
+colibri_status forward_impl(colibri_ctx* ctx, const void* x, int32_t T, const void* router_w,
+                            const float* router_b, const int32_t* user_idx, const float* user_w,
+                            const void* expert_w, const float* expert_scales, const void* shared_w,
+                            void* y, void* stream_ptr) {
+  if (!ctx) return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "ctx is NULL");
+  const colibri_desc& D = ctx->desc;
+  const bool routed_by_caller = user_idx != nullptr || user_w != nullptr;
+  if (T < 0 || T > D.max_tokens)
+    return fail(ctx, COLIBRI_ERR_INVALID_ARG, "T=%d outside [0, max_tokens=%d]", T, D.max_tokens);
+  if (!x || !expert_w || !y) return fail(ctx, COLIBRI_ERR_INVALID_ARG, "x, expert_w and y must be non-NULL");
+  if (routed_by_caller) {
+    if (!user_idx || !user_w) return fail(ctx, COLIBRI_ERR_INVALID_ARG, "topk_idx and topk_w must both be given");
+  } else if (!router_w) {
+    return fail(ctx, COLIBRI_ERR_INVALID_ARG, "router_w is NULL");
+  }
+  const bool i8 = D.weight_dtype == COLIBRI_I8;
+  if (i8 != (expert_scales != nullptr))
+    return fail(ctx, COLIBRI_ERR_INVALID_ARG, "expert_scales must be given exactly when weights are int8");
+  if ((D.shared_d_ff > 0) != (shared_w != nullptr))
+    return fail(ctx, COLIBRI_ERR_INVALID_ARG, "shared_w must be given exactly when shared_d_ff > 0");
+  const void* ptrs[] = {x, router_w, router_b, expert_w, expert_scales, shared_w, y, user_idx, user_w};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(ctx, COLIBRI_ERR_ALIGNMENT, "pointer %p is not 16-byte aligned", p);
+  ctx->last_T = T;
+  if (T == 0) return COLIBRI_OK;
+
+  DeviceGuard guard(D.device_id);
+  const int dev = D.device_id;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_ptr);
+  const void* dev_only[] = {router_w, router_b, expert_w, expert_scales, shared_w, user_idx, user_w};
+  for (const void* p : dev_only)
+    if (p && classify(p, dev) != kPtrDevice)
+      return fail(ctx, COLIBRI_ERR_INVALID_ARG, "pointer %p is not device memory of device %d", p, dev);
+  const PtrKind xk = classify(x, dev), yk = classify(y, dev);
+  if (xk == kPtrBad || yk == kPtrBad)
+    return fail(ctx, COLIBRI_ERR_INVALID_ARG, "x or y is device memory of another device");
+  // bf16 weights: pair tiles (two CTAs, 256 rows) when experts average >= 512 rows, where the
+  // halved L2 traffic per unit of work outweighs the larger last tile of each expert.
+  const bool pair_tiles =
+      D.weight_dtype == COLIBRI_BF16 && use_pair_tiles(ctx, T * D.top_k / D.num_experts);
+
+  // Replay a captured CUDA graph of this exact call when possible: device x and y, a stream
+  // other than the legacy default stream that is not itself being captured, and no profiling.
+  const bool graphable = ctx->use_graphs && reinterpret_cast<uintptr_t>(s) > 2 && xk == kPtrDevice &&
+                         yk == kPtrDevice && !ctx->profile && !ctx->prof_on;
+  if (graphable) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) {
+      cudaGetLastError();
+      cs = cudaStreamCaptureStatusActive;
+    }
+    if (cs == cudaStreamCaptureStatusNone) {
+      const uintptr_t key[14] = {(uintptr_t)x,        (uintptr_t)T,        (uintptr_t)router_w, (uintptr_t)router_b,
+                                 (uintptr_t)user_idx, (uintptr_t)user_w,   (uintptr_t)expert_w, (uintptr_t)expert_scales,
+                                 (uintptr_t)shared_w, (uintptr_t)y,        (uintptr_t)s,        (uintptr_t)pair_tiles,
+                                 0, 0};
+      for (auto& g : ctx->graphs) {
+        if (memcmp(g.key, key, sizeof(key)) == 0) {
+          g.last_use = ++ctx->graph_clock;
+          COLIBRI_TRY(cudaGraphLaunch(g.exec, s), "graph launch");
+          return COLIBRI_OK;
+        }
+      }
+      COLIBRI_TRY(cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal), "begin capture");
+      const colibri_status st = enqueue_forward(ctx, x, xk, T, router_w, router_b, user_idx, user_w, expert_w,
+                                                expert_scales, shared_w, y, yk, s, pair_tiles);
+      cudaGraph_t graph = nullptr;
+      const cudaError_t ce = cudaStreamEndCapture(s, &graph);
+      if (st != COLIBRI_OK) {
+        if (graph) cudaGraphDestroy(graph);
+        cudaGetLastError();
+        return st;
+      }
+      if (ce != cudaSuccess) return check_launch(ctx, ce, "end capture");
+      cudaGraphExec_t exec = nullptr;
+      const cudaError_t ie = cudaGraphInstantiate(&exec, graph, 0);
+      cudaGraphDestroy(graph);
+      if (ie != cudaSuccess) return check_launch(ctx, ie, "graph instantiate");
+      if (ctx->graphs.size() >= kMaxGraphs) {
+        size_t lru = 0;
+        for (size_t i = 1; i < ctx->graphs.size(); ++i)
+          if (ctx->graphs[i].last_use < ctx->graphs[lru].last_use) lru = i;
+        cudaGraphExecDestroy(ctx->graphs[lru].exec);
+        ctx->graphs.erase(ctx->graphs.begin() + lru);
+      }
+      colibri_ctx::GraphEntry ge;
+      memcpy(ge.key, key, sizeof(key));
+      ge.exec = exec;
+      ge.last_use = ++ctx->graph_clock;
+      ctx->graphs.push_back(ge);
+      COLIBRI_TRY(cudaGraphLaunch(exec, s), "graph launch");
+      return COLIBRI_OK;
+    }
+  }
+  return enqueue_forward(ctx, x, xk, T, router_w, router_b, user_idx, user_w, expert_w, expert_scales, shared_w, y,
+                         yk, s, pair_tiles);
 }
 
 }  // namespace

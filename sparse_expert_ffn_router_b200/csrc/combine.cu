@@ -3,6 +3,8 @@
 // (www.hotelren.com/news/4731937 §2.1 step 6 and §2.3 combine_kernel; the fixed-order k-way
 // aggregation of www.pptc.cn/news/100465 §2.1, without the atomic accumulation of its §1 so
 // that the result is deterministic).  One warp per token, 16-byte vector accesses.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace colibri {
@@ -80,48 +82,41 @@ __global__ void __launch_bounds__(256) combine_kernel(const Typ* __restrict__ Yp
   }
 }
 
-// int8 path: the down projection leaves `nsplit` K-partial sums per grouped row.
+// int8 path: the down projection leaves `nsplit` K-partial sums per grouped row.  One thread
+// per (token, 8 consecutive outputs): all k x nsplit partial loads of a thread are independent,
+// so a handful of tokens is one short latency, not a serial walk.
 template <typename Tout>
 __global__ void __launch_bounds__(256) combine_split_kernel(const float* __restrict__ Ypart,
                                                             int nsplit, int rows,
                                                             const int32_t* __restrict__ dst_row,
                                                             const float* __restrict__ w, int T,
                                                             int k, int d, Tout* __restrict__ y) {
-  const int lane = threadIdx.x & 31;
-  const int warps_total = gridDim.x * (blockDim.x >> 5);
+  const int chunks = d >> 3;
   const size_t split_stride = (size_t)rows * d;
-  for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps_total) {
-    int r = 0;
-    float wj = 0.f;
-    if (lane < k) {
-      r = dst_row[(size_t)t * k + lane];
-      wj = w[(size_t)t * k + lane];
-    }
-    int rws[kMaxTopK];
-    float ws[kMaxTopK];
+  for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < (long long)T * chunks;
+       q += (long long)gridDim.x * blockDim.x) {
+    const int t = (int)(q / chunks), c = (int)(q - (long long)t * chunks) * 8;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int j = 0; j < kMaxTopK; ++j) {
-      rws[j] = __shfl_sync(0xffffffffu, r, j);
-      ws[j] = __shfl_sync(0xffffffffu, wj, j);
-    }
-    for (int c = lane * 8; c < d; c += 32 * 8) {
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (j < k) {
+        const int r = dst_row[(size_t)t * k + j];
+        const float wj = w[(size_t)t * k + j];
+        float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int j = 0; j < kMaxTopK; ++j) {
-        if (j < k) {
-          float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-          for (int sidx = 0; sidx < nsplit; ++sidx) {
+        for (int sidx = 0; sidx < kDecSplitMax; ++sidx) {
+          if (sidx < nsplit) {
             float v[8];
-            load8(Ypart + sidx * split_stride + (size_t)rws[j] * d + c, v);
+            load8(Ypart + sidx * split_stride + (size_t)r * d + c, v);
 #pragma unroll
             for (int i = 0; i < 8; ++i) part[i] += v[i];
           }
-#pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i] = fmaf(ws[j], part[i], acc[i]);
         }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(wj, part[i], acc[i]);
       }
-      store8(y + (size_t)t * d + c, acc);
     }
+    store8(y + (size_t)t * d + c, acc);
   }
 }
 
@@ -159,7 +154,9 @@ cudaError_t launch_combine_split(const float* Ypart, int nsplit, int rows, const
                                  const float* w, int T, int k, int d, void* y, int act,
                                  cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  const int grid = grid_for_tokens(T);
+  if (nsplit > kDecSplitMax) return cudaErrorInvalidValue;
+  long long threads = (long long)T * (d / 8);
+  int grid = (int)std::min<long long>((threads + 255) / 256, 8192);
   if (act == COLIBRI_BF16)
     combine_split_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(Ypart, nsplit, rows, dst_row, w, T, k,
                                                              d, (__nv_bfloat16*)y);

@@ -20,6 +20,8 @@ namespace colibri {
 constexpr int kMaxExperts = 256;
 constexpr int kMaxTopK = 8;
 constexpr int kCountBlock = 256;  // tokens per block of the histogram / rank kernel
+constexpr int kFusedRouteMaxT = 64;       // largest T routed by the single-CTA fused kernel
+constexpr int kFusedRouteThreads = 1024;  // its threads (the row copies use all of them)
 
 // tcgen05 grouped GEMM tile: BM x BN accumulator, BK = one 128-byte swizzle atom of bf16
 constexpr int kTcBM = 128;
@@ -41,9 +43,6 @@ constexpr int kSimtBN = 64;
 constexpr int kSimtBK = 16;
 
 // int8 weight-streaming decode path
-constexpr int kDecRowsPerCta = 64;   // output channels per CTA (4 warps x 16)
-constexpr int kDecTokChunk = 32;     // token rows per pass (4 mma n-blocks of 8)
-constexpr int kDecKC = 256;          // K elements staged per step
 constexpr int kDecSplitMax = 8;      // K splits of the down projection
 
 // Device error word bits (ctx->err)
@@ -73,6 +72,9 @@ struct Workspace {
   void* Hs = nullptr;   // [M, fs]
   void* Ys = nullptr;   // [M, d]
   float* Ypart = nullptr;  // [split, M*k, d] f32, int8 path
+  int8_t* plane_hi = nullptr;  // [M*k, max(d, f)] int8 activation planes, int8 path
+  int8_t* plane_lo = nullptr;
+  float* plane_scale = nullptr;  // [M*k]
   uint32_t* err = nullptr;
 };
 
@@ -96,6 +98,15 @@ struct colibri_ctx {
   int prof_max = 0;
   int prof_n = 0;
   bool prof_on = false;
+  // CUDA graphs of the launch sequence, keyed by the forward's arguments
+  struct GraphEntry {
+    uintptr_t key[14];
+    cudaGraphExec_t exec;
+    uint64_t last_use;
+  };
+  std::vector<GraphEntry> graphs;
+  uint64_t graph_clock = 0;
+  bool use_graphs = true;
 };
 
 namespace colibri {
@@ -103,8 +114,9 @@ namespace colibri {
 // ---------------------------------------------------------------------------------------
 // Kernel launchers (each returns cudaGetLastError() of its launch)
 // ---------------------------------------------------------------------------------------
+// err: the context's device error word for bounded waits that give up (may be NULL).
 cudaError_t launch_router_topk(const void* x, int act, int T, int d, const void* wr, const float* b,
-                               int E, int k, int32_t* idx, float* w, cudaStream_t s);
+                               int E, int k, int32_t* idx, float* w, uint32_t* err, cudaStream_t s);
 cudaError_t launch_route_count(const int32_t* idx, int T, int k, int E, int32_t* blk_counts,
                                int32_t* local_rank, cudaStream_t s);
 cudaError_t launch_route_scan(const int32_t* blk_counts, int nblk, int E, int bm, int32_t* blk_base,
@@ -112,6 +124,10 @@ cudaError_t launch_route_scan(const int32_t* blk_counts, int nblk, int E, int bm
 cudaError_t launch_route_scatter(const void* x, int act, int T, int d, int k, int E,
                                  const int32_t* idx, const int32_t* blk_base, int32_t* dst_row,
                                  int32_t* src_row, void* Xp, cudaStream_t s);
+// T <= kFusedRouteThreads: count + scan + scatter in one single-CTA launch
+cudaError_t launch_route_fused(const void* x, int act, int T, int d, const int32_t* idx, int k, int E, int bm,
+                               int32_t* counts, int32_t* offsets, int32_t* mt_prefix, int32_t* src_row,
+                               int32_t* dst_row, void* Xp, cudaStream_t s);
 cudaError_t launch_combine(const void* Yp, int yp_dtype, const int32_t* dst_row, const float* w,
                            int T, int k, int d, const void* Ys, void* y, int act, cudaStream_t s);
 cudaError_t launch_combine_split(const float* Ypart, int nsplit, int rows, const int32_t* dst_row,
@@ -155,16 +171,25 @@ struct TcGemmArgs {
   int sm_count;
   bool pair;            // clusters of two CTAs with 256-row pair tiles (cta_group::2)
 };
+// bf16 tensor map: 64-element (128-byte) inner box, 128-byte swizzle, zero fill out of bounds
+bool make_bf16_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                    const uint64_t* strides_bytes, const uint32_t* box);
+cudaError_t configure_tc_kernels();      // once per device, before any launch
+cudaError_t configure_router_kernels();  // once per device, before any launch
 cudaError_t launch_tc_gateup(const TcGemmArgs& a, cudaStream_t s);
 cudaError_t launch_tc_down(const TcGemmArgs& a, cudaStream_t s);
 
 // int8 weight-streaming decode path, see decode_i8.cu
-cudaError_t launch_dec_gateup(const __nv_bfloat16* Xp, const int8_t* W, const float* scales,
-                              int64_t wstride, int d, int f, int E, const int32_t* offsets,
-                              __nv_bfloat16* H, cudaStream_t s);
-cudaError_t launch_dec_down(const __nv_bfloat16* H, const int8_t* W, const float* scales,
-                            int64_t wstride, int d, int f, int E, const int32_t* offsets,
-                            int nsplit, int rows, float* Ypart, cudaStream_t s);
+// Split bf16 rows into two int8 planes with a per-row scale: x ~= a * (hi + lo / 254).
+cudaError_t launch_dec_split(const __nv_bfloat16* X, int R, int K, int8_t* hi, int8_t* lo, float* scale,
+                             cudaStream_t s);
+// max_rows_per_expert: an upper bound (T) that picks the token-block width of the kernels.
+cudaError_t launch_dec_gateup(const int8_t* Xhi, const int8_t* Xlo, const float* xscale, const int8_t* W,
+                              const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
+                              __nv_bfloat16* H, int max_rows_per_expert, cudaStream_t s);
+cudaError_t launch_dec_down(const int8_t* Hhi, const int8_t* Hlo, const float* hscale, const int8_t* W,
+                            const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
+                            int nsplit, int rows, float* Ypart, int max_rows_per_expert, cudaStream_t s);
 
 // ---------------------------------------------------------------------------------------
 // Small device helpers

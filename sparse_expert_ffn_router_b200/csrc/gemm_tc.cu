@@ -611,9 +611,12 @@ EncodeTiledFn get_encode() {
   return fn;
 }
 
-// bf16 tensor map with a 64-element (128-byte) inner box and 128-byte swizzle.
-bool make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-              const uint64_t* strides_bytes, const uint32_t* box) {
+}  // namespace
+
+// bf16 tensor map with a 64-element (128-byte) inner box and 128-byte swizzle; out-of-bounds
+// elements of a box read as zero.
+bool make_bf16_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                    const uint64_t* strides_bytes, const uint32_t* box) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return false;
   cuuint64_t gd[5], gs[4];
@@ -628,6 +631,13 @@ bool make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims
                          gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+namespace {
+
+bool make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+              const uint32_t* box) {
+  return make_bf16_tmap(map, base, rank, dims, strides_bytes, box);
 }
 
 template <bool kGateUp>
@@ -695,8 +705,6 @@ cudaError_t launch_tc(const TcGemmArgs& a, cudaStream_t s) {
     if (bound < grid) grid = (int)bound;
     if (grid <= 0) return cudaSuccess;
     auto kern = tc_ffn_kernel<kGateUp>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-    if (e != cudaSuccess) return e;
     kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(p);
     return cudaGetLastError();
   }
@@ -704,8 +712,6 @@ cudaError_t launch_tc(const TcGemmArgs& a, cudaStream_t s) {
   if (bound < pairs) pairs = (int)bound;
   if (pairs <= 0) return cudaSuccess;
   auto kern = tc2_ffn_kernel<kGateUp>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM2_BYTES);
-  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3(2 * pairs);
@@ -719,12 +725,26 @@ cudaError_t launch_tc(const TcGemmArgs& a, cudaStream_t s) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 }  // namespace
+
+// Done once per device at context creation, so that nothing in the launch path is a
+// non-stream call (the launch sequence can then be captured into a CUDA graph).
+cudaError_t configure_tc_kernels() {
+  cudaError_t e = cudaFuncSetAttribute(tc_ffn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(tc_ffn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(tc2_ffn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM2_BYTES);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(tc2_ffn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM2_BYTES);
+  if (e == cudaSuccess && !get_encode()) e = cudaErrorNotSupported;
+  return e;
+}
 
 cudaError_t launch_tc_gateup(const TcGemmArgs& a, cudaStream_t s) { return launch_tc<true>(a, s); }
 cudaError_t launch_tc_down(const TcGemmArgs& a, cudaStream_t s) { return launch_tc<false>(a, s); }

@@ -138,7 +138,95 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(
   }
 }
 
+// Small batches (T <= 64): histogram, prefix sum and scatter in one single-CTA launch.  Same
+// rank rule as the three-kernel path: a token's rank inside its expert is the number of
+// earlier tokens (warp masks, then a prefix over warps) that chose that expert.
+template <typename Tv>
+__global__ void __launch_bounds__(kFusedRouteThreads) route_fused_kernel(
+    const Tv* __restrict__ x, int T, int vec_per_row, const int32_t* __restrict__ idx, int k, int E, int bm,
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ mt_prefix,
+    int32_t* __restrict__ src_row, int32_t* __restrict__ dst_row, Tv* __restrict__ Xp) {
+  constexpr int W = kFusedRouteThreads / 32;
+  __shared__ uint32_t masks[W][kMaxExperts];
+  __shared__ int off_s[kMaxExperts + 1];
+  __shared__ int rows_s[kFusedRouteMaxT][kMaxTopK];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, t = threadIdx.x;
+  for (int e = lane; e < E; e += 32) masks[warp][e] = 0u;
+  __syncwarp();
+  int ids[kMaxTopK], rank[kMaxTopK];
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) {
+    ids[j] = 0;
+    rank[j] = 0;
+    if (j < k && t < T) {
+      ids[j] = min(max(idx[(size_t)t * k + j], 0), E - 1);
+      atomicOr(&masks[warp][ids[j]], 1u << lane);
+    }
+  }
+  __syncwarp();
+  const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j)
+    if (j < k && t < T) rank[j] = __popc(masks[warp][ids[j]] & below);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kFusedRouteThreads) {
+    int run = 0;
+#pragma unroll
+    for (int w = 0; w < W; ++w) {
+      const int c = __popc(masks[w][e]);
+      masks[w][e] = (uint32_t)run;
+      run += c;
+    }
+    off_s[e] = run;  // total for now
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int o = 0, mt = 0;
+    for (int q = 0; q < E; ++q) {
+      const int c = off_s[q];
+      counts[q] = c;
+      offsets[q] = o;
+      mt_prefix[q] = mt;
+      off_s[q] = o;
+      o += c;
+      mt += (c + bm - 1) / bm;
+    }
+    off_s[E] = o;
+    offsets[E] = o;
+    mt_prefix[E] = mt;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) {
+    if (j < k && t < T) {
+      const int r = off_s[ids[j]] + (int)masks[warp][ids[j]] + rank[j];
+      dst_row[(size_t)t * k + j] = r;
+      src_row[r] = t;
+      rows_s[t][j] = r;
+    }
+  }
+  __syncthreads();
+  // copy: the whole CTA walks (token, 16-byte vector) pairs
+  for (int q = threadIdx.x; q < T * vec_per_row; q += kFusedRouteThreads) {
+    const int tt = q / vec_per_row, v = q - tt * vec_per_row;
+    const Tv val = __ldg(x + (size_t)tt * vec_per_row + v);
+    for (int j = 0; j < k; ++j) Xp[(size_t)rows_s[tt][j] * vec_per_row + v] = val;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_route_fused(const void* x, int act, int T, int d, const int32_t* idx, int k, int E, int bm,
+                               int32_t* counts, int32_t* offsets, int32_t* mt_prefix, int32_t* src_row,
+                               int32_t* dst_row, void* Xp, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  if (T > kFusedRouteMaxT) return cudaErrorInvalidValue;
+  const int esize = (act == COLIBRI_BF16) ? 2 : 4;
+  const int vec = d * esize / 16;
+  route_fused_kernel<uint4><<<1, kFusedRouteThreads, 0, s>>>((const uint4*)x, T, vec, idx, k, E, bm, counts,
+                                                            offsets, mt_prefix, src_row, dst_row, (uint4*)Xp);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_route_count(const int32_t* idx, int T, int k, int E, int32_t* blk_counts,
                                int32_t* local_rank, cudaStream_t s) {

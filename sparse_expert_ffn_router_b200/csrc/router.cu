@@ -1,6 +1,6 @@
-// Gate stage: router logits, softmax and top-k.  bf16 activations with E <= 128 use the
-// tensor-core kernel below (the stage is bound by one read of x); fp32 activations, and more
-// than 128 experts, use the SIMT kernel.
+// Gate stage: router logits, softmax and top-k.  bf16 activations use the tcgen05 kernel at the
+// end of this file (the stage is bound by one read of x); fp32 activations use the SIMT kernel
+// (fp32 FMA, no TF32).
 //
 // logits l[t][e] = b[e] + sum_i x[t][i] * Wr[e][i]      (www.hotelren.com/news/4731937 §3.2,
 //                                                        www.0539edu.com/news/4774449 §2.1)
@@ -11,6 +11,9 @@
 // weights: softmax over all E renormalised over the k chosen, computed as
 // exp(l_j - l_0) / sum_j' exp(l_j' - l_0) in fp32.
 // Output layout [T][k] (www.pptc.cn/news/100465 §3.4).
+#include <algorithm>
+#include <cstring>
+
 #include "common.cuh"
 
 namespace colibri {
@@ -129,138 +132,236 @@ __global__ void __launch_bounds__(kRouterThreads) router_topk_simt_kernel(
 }
 
 // ---------------------------------------------------------------------------------------
-// bf16 router on the tensor cores (mma.sync m16n8k16, fp32 accumulation).  One warp owns 16
-// tokens x all E experts (NB n-blocks of 8).  For a 32-wide K block a thread (g = lane / 4,
-// c = lane % 4) loads 16 contiguous bytes [8c, 8c + 8) of token rows g and g + 8 and of expert
-// row g of every n-block; MMA k-step s in {0, 1} takes elements 8c + 4s + {0,1} as logical
-// k = 2c, 2c+1 and 8c + 4s + {2,3} as k = 2c+8, 2c+9 on both operands, so the K permutation
-// cancels in the dot product.  The CTA's 4 warps cover TM token groups x KS K-slices
-// (TM * KS = 4); K-slice partial logits are summed in fixed slice order in shared memory.
+// bf16 router on the 5th-generation tensor cores.  A CTA owns 128 tokens (the 128 TMEM lanes)
+// and all experts padded to N = 16 * ceil(E / 16) columns: one elected thread streams x and Wr
+// tiles (64-wide K blocks, 128-byte swizzle) through a 4-stage shared-memory ring with TMA and
+// issues tcgen05.mma (M=128, N, K=16) into an fp32 accumulator in TMEM; padded expert rows are
+// read as zeros and never selected.  Then every thread owns one token row: it reads that row's
+// logits from TMEM 16 columns at a time, adds the bias and keeps the k best in registers by
+// insertion with a strict ">" (so of two equal logits the lower expert index, seen first,
+// stays ahead), then writes ids and the renormalised softmax weights.  Every wait is bounded.
 // ---------------------------------------------------------------------------------------
-__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-      "{%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
+constexpr int kRtMaxStages = 16;
+constexpr int kRtABytes = 128 * 64 * 2;            // x tile: 128 tokens x 64 K
+constexpr size_t kRtRingBytes = 200 * 1024;        // shared memory given to the ring
 
-__device__ __forceinline__ uint4 ld_nc16(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
+struct alignas(64) RouterTcParams {
+  CUtensorMap mapX;  // [T, d], box {64, 128}
+  CUtensorMap mapW;  // [E, d], box {64, N}
+  const float* b;
+  int T, d, E, k, N;
+  int stages;  // ring depth: as many stages as fit in kRtRingBytes (small expert counts go deeper)
+  uint32_t stage_bytes, tmem_cols;
+  int32_t* idx;
+  float* w;
+  uint32_t* err;
+};
 
-template <int NB, int TM>
-__global__ void __launch_bounds__(128) router_topk_mma_kernel(
-    const __nv_bfloat16* __restrict__ x, int T, int d, const __nv_bfloat16* __restrict__ wr,
-    const float* __restrict__ b, int E, int k, int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
-  constexpr int KS = 4 / TM;
-  constexpr int TT = 16 * TM;
-  extern __shared__ float sm[];
-  float* part = sm;                       // [KS][TT][E]
-  float* lg = part + KS * TT * E;         // [TT][E + 1]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
-  const int tg = warp % TM, ks = warp / TM;
-  const int t0 = blockIdx.x * TT + tg * 16;
-  const int ta = min(t0 + g, T - 1), tb = min(t0 + g + 8, T - 1);
-  const bool va = t0 + g < T, vb = t0 + g + 8 < T;
-  const __nv_bfloat16* xa = x + (size_t)ta * d + 8 * c;
-  const __nv_bfloat16* xb = x + (size_t)tb * d + 8 * c;
-  const __nv_bfloat16* wrow[NB];
-  bool wv[NB];
-#pragma unroll
-  for (int nb = 0; nb < NB; ++nb) {
-    const int e = nb * 8 + g;
-    wv[nb] = e < E;
-    wrow[nb] = wr + (size_t)min(e, E - 1) * d + 8 * c;
-  }
-  float acc[NB][4];
-#pragma unroll
-  for (int nb = 0; nb < NB; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
-  const uint4 zero = make_uint4(0, 0, 0, 0);
-  const int nkb = d / 32;
-  for (int kb = ks; kb < nkb; kb += KS) {
-    const int ko = kb * 32;
-    const uint4 av = va ? ld_nc16(xa + ko) : zero;
-    const uint4 bv4 = vb ? ld_nc16(xb + ko) : zero;
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-      const uint4 wq = wv[nb] ? ld_nc16(wrow[nb] + ko) : zero;
-      mma16816(acc[nb], av.x, bv4.x, av.y, bv4.y, wq.x, wq.y);  // k-step 0
-      mma16816(acc[nb], av.z, bv4.z, av.w, bv4.w, wq.z, wq.w);  // k-step 1
+__device__ __forceinline__ bool rt_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  uint32_t n = 0;
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((++n & 255u) == 0) {
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > kWaitTimeoutNs) return false;
     }
   }
-  // C fragment: rows g / g + 8 (tokens), columns 2c, 2c + 1 (experts of the n-block)
-  float* pw = part + (size_t)ks * TT * E;
+}
+
+__global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant__ RouterTcParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {  // the 128-byte swizzle needs 1024-byte aligned tiles
+    if (threadIdx.x == 0 && p.err) atomicOr(p.err, kErrWaitTimeout);
+    return;
+  }
+  const int S = p.stages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * p.stage_bytes);
+  uint64_t* empty = full + S;
+  uint64_t* done = empty + S;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+    tma_prefetch_desc(&p.mapX);
+    tma_prefetch_desc(&p.mapW);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_holder, p.tmem_cols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int row0 = blockIdx.x * 128;
+  const int nkb = p.d / 64;
+
+  if (threadIdx.x == 0) {
+    const uint32_t idesc = idesc_bf16_f32(128, p.N);
+    const uint32_t bytes = kRtABytes + (uint32_t)p.N * 128u;
+    auto issue = [&](int kb) {
+      uint8_t* sa = smem + (size_t)(kb % S) * p.stage_bytes;
+      mbar_arrive_expect_tx(&full[kb % S], bytes);
+      tma_load_2d(sa, &p.mapX, &full[kb % S], kb * 64, row0);
+      tma_load_2d(sa + kRtABytes, &p.mapW, &full[kb % S], kb * 64, 0);
+    };
+    for (int kb = 0; kb < nkb && kb < S; ++kb) issue(kb);
+    bool ok = true;
+    for (int kb = 0; kb < nkb && ok; ++kb) {
+      const int s = kb % S;
+      const uint32_t ph = (uint32_t)(kb / S) & 1u;
+      if (!rt_wait(&full[s], ph, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t sa = smem_u32(smem + (size_t)s * p.stage_bytes);
 #pragma unroll
-  for (int nb = 0; nb < NB; ++nb) {
+      for (int kk = 0; kk < 4; ++kk)
+        tc_mma_f16(tmem, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sa + kRtABytes + kk * 32), idesc,
+                   (kb | kk) != 0 ? 1u : 0u);
+      tc_commit(&empty[s]);
+      if (kb + S < nkb) {
+        if (!rt_wait(&empty[s], ph, abort_flag)) {  // MMAs of this stage done: refill it
+          ok = false;
+          break;
+        }
+        issue(kb + S);
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      if (p.err) atomicOr(p.err, kErrWaitTimeout);
+    }
+    tc_commit(done);  // arrives once every MMA issued above has completed
+  }
+  // ------------------------------------------------------------- epilogue: one token per thread
+  const bool got = rt_wait(done, 0, abort_flag) && !*abort_flag;
+  const bool warp_ok = __all_sync(0xffffffffu, got);
+  tc_fence_after();
+  float bv[kMaxTopK];
+  int bi[kMaxTopK];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int row = tg * 16 + g + (q >> 1) * 8;
-      const int e = nb * 8 + 2 * c + (q & 1);
-      if (e < E) pw[row * E + e] = acc[nb][q];
+  for (int j = 0; j < kMaxTopK; ++j) {
+    bv[j] = -INFINITY;
+    bi[j] = 0x7fffffff;
+  }
+  if (warp_ok) {
+    const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16);
+    for (int c0 = 0; c0 < p.N; c0 += 16) {
+      float v[16];
+      tmem_ld16(tbase + c0, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int e = c0 + i;
+        if (e < p.E) {
+          float cv = v[i] + (p.b ? p.b[e] : 0.f);
+          int ci = e;
+#pragma unroll
+          for (int j = 0; j < kMaxTopK; ++j) {
+            if (j < p.k && cv > bv[j]) {
+              const float tv = bv[j];
+              const int ti = bi[j];
+              bv[j] = cv;
+              bi[j] = ci;
+              cv = tv;
+              ci = ti;
+            }
+          }
+        }
+      }
+    }
+    const int t = row0 + threadIdx.x;
+    if (t < p.T) {
+      float den = 0.f;
+#pragma unroll
+      for (int j = 0; j < kMaxTopK; ++j)
+        if (j < p.k) den += expf(bv[j] - bv[0]);
+#pragma unroll
+      for (int j = 0; j < kMaxTopK; ++j)
+        if (j < p.k) {
+          p.idx[(size_t)t * p.k + j] = bi[j];
+          p.w[(size_t)t * p.k + j] = expf(bv[j] - bv[0]) / den;
+        }
     }
   }
+  tc_fence_before();
   __syncthreads();
-  for (int i = threadIdx.x; i < TT * E; i += 128) {
-    const int row = i / E, e = i - row * E;
-    float v = b ? b[e] : 0.f;
-    float sum = 0.f;
-#pragma unroll
-    for (int s2 = 0; s2 < KS; ++s2) sum += part[(size_t)s2 * TT * E + i];
-    lg[row * (E + 1) + e] = sum + v;
-  }
-  __syncthreads();
-  for (int tt = warp; tt < TT; tt += 4) {
-    const int t = blockIdx.x * TT + tt;
-    if (t >= T) break;
-    warp_topk(lg + tt * (E + 1), E, k, lane, idx_out + (size_t)t * k, w_out + (size_t)t * k);
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, p.tmem_cols);
   }
 }
 
-template <int NB, int TM>
-cudaError_t launch_mma_router(const void* x, int T, int d, const void* wr, const float* b, int E, int k,
-                              int32_t* idx, float* w, cudaStream_t s) {
-  constexpr int KS = 4 / TM, TT = 16 * TM;
-  const size_t smem = sizeof(float) * ((size_t)KS * TT * E + (size_t)TT * (E + 1));
-  auto kern = router_topk_mma_kernel<NB, TM>;
-  if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  kern<<<(T + TT - 1) / TT, 128, smem, s>>>((const __nv_bfloat16*)x, T, d, (const __nv_bfloat16*)wr, b, E, k,
-                                            idx, w);
+constexpr size_t kRtMaxSmem = kRtRingBytes + 1024;
+
+cudaError_t launch_router_tc(const void* x, int T, int d, const void* wr, const float* b, int E, int k,
+                             int32_t* idx, float* w, uint32_t* err, cudaStream_t s) {
+  RouterTcParams p;
+  memset(&p, 0, sizeof(p));
+  p.N = (E + 15) / 16 * 16;
+  {
+    const uint64_t dims[2] = {(uint64_t)d, (uint64_t)T}, st[1] = {(uint64_t)d * 2};
+    const uint32_t box[2] = {64, 128};
+    if (!make_bf16_tmap(&p.mapX, x, 2, dims, st, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[2] = {(uint64_t)d, (uint64_t)E}, st[1] = {(uint64_t)d * 2};
+    const uint32_t box[2] = {64, (uint32_t)p.N};
+    if (!make_bf16_tmap(&p.mapW, wr, 2, dims, st, box)) return cudaErrorInvalidValue;
+  }
+  p.b = b;
+  p.T = T;
+  p.d = d;
+  p.E = E;
+  p.k = k;
+  p.stage_bytes = (uint32_t)((kRtABytes + p.N * 128 + 1023) / 1024 * 1024);
+  p.stages = (int)std::min<size_t>(kRtMaxStages, kRtRingBytes / p.stage_bytes);
+  p.tmem_cols = 32;
+  while ((int)p.tmem_cols < p.N) p.tmem_cols <<= 1;
+  p.idx = idx;
+  p.w = w;
+  p.err = err;
+  const size_t smem = (size_t)p.stages * p.stage_bytes + 1024;
+  router_tc_kernel<<<(T + 127) / 128, 128, smem, s>>>(p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
+// Largest dynamic shared memory the router kernels use (E = 256 on the SIMT kernel; 256 padded
+// experts on the tensor-core kernel), set once per device at context creation.
+cudaError_t configure_router_kernels() {
+  const int simt = (int)(sizeof(float) * ((size_t)kRouterTT * (kRouterDK + 1) + (size_t)kMaxExperts * (kRouterDK + 1) +
+                                          (size_t)kRouterTT * (kMaxExperts + 1)));
+  cudaError_t e = cudaFuncSetAttribute(router_topk_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, simt);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(router_topk_simt_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, simt);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRtMaxSmem);
+  return e;
+}
+
 cudaError_t launch_router_topk(const void* x, int act, int T, int d, const void* wr, const float* b,
-                               int E, int k, int32_t* idx, float* w, cudaStream_t s) {
+                               int E, int k, int32_t* idx, float* w, uint32_t* err, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
+  if (act == COLIBRI_BF16) return launch_router_tc(x, T, d, wr, b, E, k, idx, w, err, s);
   const size_t smem =
       sizeof(float) * ((size_t)kRouterTT * (kRouterDK + 1) + (size_t)E * (kRouterDK + 1) +
                        (size_t)kRouterTT * (E + 1));
   const dim3 grid((T + kRouterTT - 1) / kRouterTT);
-  if (act == COLIBRI_BF16 && E <= 128) {
-    // tensor-core router; token tile and K split chosen by the number of experts
-    if (E <= 8) return launch_mma_router<1, 1>(x, T, d, wr, b, E, k, idx, w, s);
-    if (E <= 16) return launch_mma_router<2, 1>(x, T, d, wr, b, E, k, idx, w, s);
-    if (E <= 32) return launch_mma_router<4, 2>(x, T, d, wr, b, E, k, idx, w, s);
-    if (E <= 64) return launch_mma_router<8, 4>(x, T, d, wr, b, E, k, idx, w, s);
-    return launch_mma_router<16, 4>(x, T, d, wr, b, E, k, idx, w, s);
-  }
-  if (act == COLIBRI_BF16) {
-    auto kern = router_topk_simt_kernel<__nv_bfloat16>;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    kern<<<grid, kRouterThreads, smem, s>>>((const __nv_bfloat16*)x, T, d,
-                                            (const __nv_bfloat16*)wr, b, E, k, idx, w);
-  } else {
-    auto kern = router_topk_simt_kernel<float>;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    kern<<<grid, kRouterThreads, smem, s>>>((const float*)x, T, d, (const float*)wr, b, E, k, idx, w);
-  }
+  router_topk_simt_kernel<float><<<grid, kRouterThreads, smem, s>>>((const float*)x, T, d, (const float*)wr, b, E,
+                                                                     k, idx, w);
   return cudaGetLastError();
 }
 

@@ -147,6 +147,82 @@ def test_repeated_calls_are_deterministic():
     layer.close()
 
 
+@pytest.mark.parametrize("name", ["bf16_shared", "f32_shared", "i8_small", "bf16_empty"])
+def test_graph_replay_matches_plain_launches(name):
+    # on a non-default stream the forward is captured into a CUDA graph once and replayed
+    wl = SMALL[name]
+    p = inputgen.make_problem(wl, seed=7)
+    layer = H.make_layer(wl)
+    t = H.to_device(p)
+    args = (t["x"], t["router_w"], t["router_b"], t["expert_w"])
+    kw = dict(expert_scales=t["expert_scales"], shared_w=t["shared_w"])
+    y0 = torch.empty(wl.T, wl.d, dtype=p.x.dtype, device="cuda")
+    layer.forward(*args, y0, **kw)  # legacy default stream: plain launches
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    ys = [torch.full_like(y0, 3.0) for _ in range(3)]
+    for y in ys:  # capture, then two replays
+        layer.forward(*args, y, stream=s, **kw)
+    s.synchronize()
+    layer.sync_status()
+    for y in ys:
+        assert torch.equal(y, y0)
+    # the replay reads the current contents of its buffers
+    x2 = inputgen.make_x(wl, seed=11).cuda()
+    t["x"].copy_(x2)
+    torch.cuda.synchronize()
+    y_plain = torch.empty_like(y0)
+    layer.forward(*args, y_plain, **kw)
+    torch.cuda.synchronize()
+    layer.forward(*args, ys[0], stream=s, **kw)
+    s.synchronize()
+    assert torch.equal(ys[0], y_plain)
+    layer.close()
+
+
+def test_graph_cache_distinguishes_token_counts():
+    wl = SMALL["bf16_shared"]
+    layer = H.make_layer(wl, max_tokens=600)
+    s = torch.cuda.Stream()
+    for T in (513, 40, 513, 7, 40):
+        p = inputgen.make_problem(inputgen.custom("g", T=T, d=wl.d, E=wl.E, k=wl.k, f=wl.f, fs=wl.fs), seed=T)
+        t = H.to_device(p)
+        y = torch.empty(T, wl.d, dtype=torch.bfloat16, device="cuda")
+        layer.forward(t["x"], t["router_w"], None, t["expert_w"], y, shared_w=t["shared_w"], stream=s)
+        s.synchronize()
+        yr = oracle.problem_forward(p, tokens=[0, T - 1])["y"]
+        H.check_y(p, y.float().cpu()[[0, T - 1]], yr)
+    layer.close()
+
+
+def test_forward_inside_a_user_cuda_graph():
+    # a caller may capture the forward into its own graph: the library then only enqueues
+    wl = SMALL["bf16_ragged"]
+    p = inputgen.make_problem(wl, seed=9)
+    layer = H.make_layer(wl)
+    t = H.to_device(p)
+    y_ref = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device="cuda")
+    layer.forward(t["x"], t["router_w"], None, t["expert_w"], y_ref)
+    torch.cuda.synchronize()
+    y = torch.zeros_like(y_ref)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # warm-up outside capture, as torch asks
+        layer.forward(t["x"], t["router_w"], None, t["expert_w"], y, stream=side)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    y.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        layer.forward(t["x"], t["router_w"], None, t["expert_w"], y, stream=torch.cuda.current_stream())
+    g.replay()
+    torch.cuda.synchronize()
+    layer.sync_status()
+    assert torch.equal(y, y_ref)
+    del g
+    layer.close()
+
+
 @pytest.mark.parametrize("name", ["bf16_ragged", "f32_tiny", "i8_small", "bf16_shared"])
 def test_forward_routed_matches_oracle_routing(name):
     wl = SMALL[name]
