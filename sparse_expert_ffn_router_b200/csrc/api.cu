@@ -72,8 +72,10 @@ PtrKind classify(const void* p, int dev) {
   }
 }
 
+// K splits of the int8 down projection: each split must cover whole 128-byte K blocks.
 int pick_dec_split(int f) {
-  const int blocks = f / 64;
+  if (f % 128 != 0) return 1;
+  const int blocks = f / 128;
   for (int s = kDecSplitMax; s > 1; s >>= 1)
     if (blocks % s == 0) return s;
   return 1;
@@ -161,6 +163,8 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
     return fail(nullptr, COLIBRI_ERR_UNSUPPORTED, "dtype pair (act=%d, weight=%d) not supported", D.act_dtype, D.weight_dtype);
   if (i8 && D.shared_d_ff > 0)
     return fail(nullptr, COLIBRI_ERR_UNSUPPORTED, "shared expert with int8 weights is not supported");
+  if (i8 && D.d_ff > kDecMaxFF)
+    return fail(nullptr, COLIBRI_ERR_UNSUPPORTED, "int8 weights support d_ff <= %d", kDecMaxFF);
   if (f32 && ((int64_t)D.max_tokens * D.top_k / kSimtBM + D.num_experts > 65535 ||
               ((int64_t)D.max_tokens + kSimtBM - 1) / kSimtBM > 65535))
     return fail(nullptr, COLIBRI_ERR_UNSUPPORTED, "fp32 path limited to max_tokens * top_k < 4M rows");
@@ -198,7 +202,8 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   const size_t o_bc = c.take((size_t)nblk * E * 4), o_bb = c.take((size_t)nblk * E * 4);
   const size_t o_cnt = c.take(E * 4), o_off = c.take((E + 1) * 4), o_mt = c.take((E + 1) * 4);
   const size_t o_xp = c.take(R * d * as);
-  const size_t o_h = c.take(R * f * hs);
+  const size_t o_h = c.take(i8 ? std::max<int64_t>(2 * R, 2 * kDecGateSplitMax * std::min<int64_t>(R, kDecGateSplitRows)) * f * 4
+                             : R * f * hs);
   const size_t o_yp = i8 ? c.take(0) : c.take(R * d * hs);
   const size_t o_hs = c.take(fs > 0 ? M * fs * hs : 0);
   const size_t o_ysh = c.take(fs > 0 ? M * d * hs : 0);
@@ -207,6 +212,9 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   const size_t plane_w = (size_t)std::max<int64_t>(d, f);
   const size_t o_phi = c.take(i8 ? R * plane_w : 0), o_plo = c.take(i8 ? R * plane_w : 0);
   const size_t o_psc = c.take(i8 ? R * 4 : 0);
+  const bool rsplit = D.act_dtype == COLIBRI_BF16 && M >= kRouterSplitMinT;
+  const size_t o_rpart = c.take(rsplit ? (size_t)kRouterMaxSplit * M * E * 4 : 0);
+  const size_t o_rtick = c.take(rsplit ? (size_t)((M + 127) / 128) * 4 : 0);
   const size_t o_err = c.take(4);
   ctx->ws_bytes = c.off;
 
@@ -240,7 +248,10 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   w.plane_lo = reinterpret_cast<int8_t*>(b + o_plo);
   w.plane_scale = reinterpret_cast<float*>(b + o_psc);
   w.err = reinterpret_cast<uint32_t*>(b + o_err);
-  if (cudaMemset(w.err, 0, 4) != cudaSuccess) {
+  w.router_part = rsplit ? reinterpret_cast<float*>(b + o_rpart) : nullptr;
+  w.router_ticket = rsplit ? reinterpret_cast<int32_t*>(b + o_rtick) : nullptr;
+  if (cudaMemset(w.err, 0, 4) != cudaSuccess ||
+      (rsplit && cudaMemset(w.router_ticket, 0, (size_t)((M + 127) / 128) * 4) != cudaSuccess)) {
     cudaFree(ctx->ws_base);
     delete ctx;
     return fail(nullptr, COLIBRI_ERR_CUDA, "cudaMemset failed");
@@ -251,6 +262,7 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   ctx->use_graphs = !(getenv("COLIBRI_GRAPHS") && strcmp(getenv("COLIBRI_GRAPHS"), "0") == 0);
   cudaError_t ce = configure_router_kernels();
   if (ce == cudaSuccess) ce = configure_tc_kernels();
+  if (ce == cudaSuccess) ce = configure_dec_kernels();
   if (ce != cudaSuccess) {
     cudaGetLastError();
     cudaFree(ctx->ws_base);
@@ -325,7 +337,8 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
     COLIBRI_TRY(cudaMemcpyAsync(w.topk_idx, user_idx, (size_t)R * 4, cudaMemcpyDeviceToDevice, s), "copy topk_idx");
     COLIBRI_TRY(cudaMemcpyAsync(w.topk_w, user_w, (size_t)R * 4, cudaMemcpyDeviceToDevice, s), "copy topk_w");
   } else {
-    COLIBRI_TRY(launch_router_topk(xd, act, T, d, router_w, router_b, E, k, w.topk_idx, w.topk_w, w.err, s),
+    COLIBRI_TRY(launch_router_topk(xd, act, T, d, router_w, router_b, E, k, w.topk_idx, w.topk_w, w.err,
+                                   w.router_part, w.router_ticket, s),
                 "router_topk");
   }
   mark(1);
@@ -393,16 +406,29 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
     a.out_sh = w.Ys;
     COLIBRI_TRY(launch_tc_down(a, s), "tc_down");
   } else {
-    nsplit = R <= 256 ? ctx->dec_split : 1;
+    // K splits of the down projection: enough work items to cover every SM a few times
+    nsplit = 1;
+    if (R <= 256) {
+      const int touched = std::min(E, R), tiles = (d + 127) / 128;
+      while (nsplit < ctx->dec_split && touched * tiles * nsplit < 4 * ctx->sm_count) nsplit <<= 1;
+    }
+    // K splits of the gate/up projection (partials summed before SiLU by the finishing kernel)
+    int gsplit = 1;
+    if (R <= kDecGateSplitRows && d % 128 == 0) {
+      const int touched = std::min(E, R), tiles = 2 * ((f + 127) / 128);
+      while (gsplit < kDecGateSplitMax && (d / 128) % (2 * gsplit) == 0 &&
+             touched * tiles * gsplit < 8 * ctx->sm_count)
+        gsplit <<= 1;
+    }
     COLIBRI_TRY(launch_dec_split((const __nv_bfloat16*)w.Xp, R, d, w.plane_hi, w.plane_lo, w.plane_scale, s),
                 "dec_split_x");
     COLIBRI_TRY(launch_dec_gateup(w.plane_hi, w.plane_lo, w.plane_scale, (const int8_t*)expert_w, expert_scales,
-                                  stride, d, f, E, w.offsets, (__nv_bfloat16*)w.H, T, s), "dec_gateup");
+                                  stride, d, f, E, w.offsets, gsplit, (float*)w.H, R, T, w.err, s), "dec_gateup");
     mark(3);
-    COLIBRI_TRY(launch_dec_split((const __nv_bfloat16*)w.H, R, f, w.plane_hi, w.plane_lo, w.plane_scale, s),
-                "dec_split_h");
+    COLIBRI_TRY(launch_dec_finish_h((const float*)w.H, gsplit, R, f, w.plane_hi, w.plane_lo, w.plane_scale, s),
+                "dec_finish_h");
     COLIBRI_TRY(launch_dec_down(w.plane_hi, w.plane_lo, w.plane_scale, (const int8_t*)expert_w, expert_scales,
-                                stride, d, f, E, w.offsets, nsplit, R, w.Ypart, T, s), "dec_down");
+                                stride, d, f, E, w.offsets, nsplit, R, w.Ypart, T, w.err, s), "dec_down");
   }
   mark(4);
 

@@ -43,7 +43,10 @@ constexpr int kSimtBN = 64;
 constexpr int kSimtBK = 16;
 
 // int8 weight-streaming decode path
-constexpr int kDecSplitMax = 8;      // K splits of the down projection
+constexpr int kDecSplitMax = 16;     // K splits of the down projection
+constexpr int kDecMaxFF = 65536;     // largest d_ff of the int8 path (one H row in shared memory)
+constexpr int kDecGateSplitMax = 4;  // K splits of the gate/up projection (small batches)
+constexpr int kDecGateSplitRows = 64;  // routed rows up to which the gate/up projection may split
 
 // Device error word bits (ctx->err)
 constexpr uint32_t kErrWaitTimeout = 1u;
@@ -67,11 +70,13 @@ struct Workspace {
   int32_t* offsets = nullptr;     // [E+1]
   int32_t* mt_prefix = nullptr;   // [E+1] m-tiles prefix for the GEMM schedule
   void* Xp = nullptr;   // [M*k, d] act (grouped rows)
-  void* H = nullptr;    // [M*k, f] bf16 (bf16/int8 paths) or f32
+  void* H = nullptr;    // [M*k, f] bf16 (bf16 path), f32 (fp32 path), [2, M*k, f] f32 gate/up partials (int8)
   void* Yp = nullptr;   // [M*k, d] bf16 or f32
   void* Hs = nullptr;   // [M, fs]
   void* Ys = nullptr;   // [M, d]
   float* Ypart = nullptr;  // [split, M*k, d] f32, int8 path
+  float* router_part = nullptr;    // [8, M, E] K-split partial logits
+  int32_t* router_ticket = nullptr;  // [ceil(M/128)] arrival counters (zero between calls)
   int8_t* plane_hi = nullptr;  // [M*k, max(d, f)] int8 activation planes, int8 path
   int8_t* plane_lo = nullptr;
   float* plane_scale = nullptr;  // [M*k]
@@ -115,8 +120,15 @@ namespace colibri {
 // Kernel launchers (each returns cudaGetLastError() of its launch)
 // ---------------------------------------------------------------------------------------
 // err: the context's device error word for bounded waits that give up (may be NULL).
+// part/ticket: [8, T, E] partial logits and [ceil(T/128)] zeroed counters for the K-split
+// router used when T >= kRouterSplitMinT (NULL: no split).
+constexpr int kRouterSmallT = 64;       // T up to which one CTA per token computes the logits
+constexpr int kRouterSplitMinT = 2048;  // T from which the tensor-core router splits K
+constexpr int kRouterMaxSplit = 8;
+int router_ksplit(int T, int d);
 cudaError_t launch_router_topk(const void* x, int act, int T, int d, const void* wr, const float* b,
-                               int E, int k, int32_t* idx, float* w, uint32_t* err, cudaStream_t s);
+                               int E, int k, int32_t* idx, float* w, uint32_t* err, float* part,
+                               int32_t* ticket, cudaStream_t s);
 cudaError_t launch_route_count(const int32_t* idx, int T, int k, int E, int32_t* blk_counts,
                                int32_t* local_rank, cudaStream_t s);
 cudaError_t launch_route_scan(const int32_t* blk_counts, int nblk, int E, int bm, int32_t* blk_base,
@@ -171,6 +183,9 @@ struct TcGemmArgs {
   int sm_count;
   bool pair;            // clusters of two CTAs with 256-row pair tiles (cta_group::2)
 };
+// Tensor map with a 128-byte inner box, 128-byte swizzle, zero fill out of bounds
+bool make_tmap(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int rank, const uint64_t* dims,
+               const uint64_t* strides_bytes, const uint32_t* box);
 // bf16 tensor map: 64-element (128-byte) inner box, 128-byte swizzle, zero fill out of bounds
 bool make_bf16_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                     const uint64_t* strides_bytes, const uint32_t* box);
@@ -183,13 +198,19 @@ cudaError_t launch_tc_down(const TcGemmArgs& a, cudaStream_t s);
 // Split bf16 rows into two int8 planes with a per-row scale: x ~= a * (hi + lo / 254).
 cudaError_t launch_dec_split(const __nv_bfloat16* X, int R, int K, int8_t* hi, int8_t* lo, float* scale,
                              cudaStream_t s);
-// max_rows_per_expert: an upper bound (T) that picks the token-block width of the kernels.
+// max_rows_per_expert: an upper bound (T) that picks the token chunk (8, 16 or 32 rows).
+cudaError_t configure_dec_kernels();  // once per device, before any launch
+// gate/up: W1 . x and W3 . x (scaled) as fp32 K-split partials GU [nsplit, 2, R, f]
 cudaError_t launch_dec_gateup(const int8_t* Xhi, const int8_t* Xlo, const float* xscale, const int8_t* W,
                               const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
-                              __nv_bfloat16* H, int max_rows_per_expert, cudaStream_t s);
+                              int nsplit, float* GU, int R, int max_rows_per_expert, uint32_t* err, cudaStream_t s);
+// H = silu(sum g) * (sum u) (bf16) from GU, split into int8 planes
+cudaError_t launch_dec_finish_h(const float* GU, int nsplit, int R, int f, int8_t* hi, int8_t* lo, float* scale,
+                                cudaStream_t s);
 cudaError_t launch_dec_down(const int8_t* Hhi, const int8_t* Hlo, const float* hscale, const int8_t* W,
                             const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
-                            int nsplit, int rows, float* Ypart, int max_rows_per_expert, cudaStream_t s);
+                            int nsplit, int R, float* Ypart, int max_rows_per_expert, uint32_t* err,
+                            cudaStream_t s);
 
 // ---------------------------------------------------------------------------------------
 // Small device helpers
@@ -458,6 +479,25 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
   desc |= (uint64_t)1 << 46;                         // version, bits 46-47
   desc |= (uint64_t)2 << 61;                         // 128-byte swizzle, bits 61-63
   return desc;
+}
+
+// Instruction descriptor, kind::i8: signed int8 A and B, s32 D, both K-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_s8_s32(int M, int N) {
+  return (2u << 4)                          // D format: s32
+         | (1u << 7)                        // A format: signed 8-bit
+         | (1u << 10)                       // B format: signed 8-bit
+         | ((uint32_t)(N >> 3) << 17)       // N >> 3
+         | ((uint32_t)(M >> 4) << 24);      // M >> 4
+}
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::i8 (int8 inputs, s32 accumulate)
+__device__ __forceinline__ void tc_mma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 D, both K-major, shape M x N.

@@ -1,8 +1,7 @@
 // Expert Compute stage for int8 weights with per-output-channel fp32 scales, dequantised in
 // the kernel (www.0539edu.com/news/4774449 §3.1 stores int8 weights with scales; the scale
 // here is per output channel).  For a handful of tokens the layer is a stream over the
-// weights of the touched experts, bound by HBM bandwidth, so the design streams each weight
-// byte once and keeps everything else off the critical path:
+// weights of the touched experts, bound by HBM bandwidth:
 //
 //   gate/up:  H[r][o]    = silu(s1[o] * sum_i q1[o][i] x[r][i]) * (s3[o] * sum_i q3[o][i] x[r][i])
 //   down:     Yp_s[r][o] = s2[o] * sum_{i in split s} q2[o][i] H[r][i]
@@ -12,56 +11,25 @@
 // planes with a per-row scale, x ~= a * (hi + lo / 254) with a = max|x| / 127 (the residual
 // after hi is at most a/2, so lo fits in [-127, 127]; the representation error is at most
 // a / 508 = max|x| / 64516 per element, far below bf16's own rounding of the result).  The dot
-// products then run on the integer tensor cores (mma.sync m16n8k32, s8 x s8 -> s32, exact
-// integer accumulation), weights as the A operand (16 output channels), tokens as n-blocks
-// of 8, and the epilogue forms s[o] * a * (acc_hi + acc_lo / 254) in fp32.
+// products then run on the 5th-generation tensor cores as kind::i8 MMAs with exact int32
+// accumulation in TMEM: A = 128 weight rows (output channels) x 128 K bytes, B = the hi plane
+// rows of up to 32 tokens stacked on their lo plane rows (N = 2 x tokens), so one MMA yields
+// both planes.  The epilogue forms s[o] * a * (acc_hi + acc_lo / 254) in fp32.
 //
-// Work decomposition: every warp is independent (no shared memory, no CTA barrier).  A work
-// item is (touched expert, 16 output channels, K range); a persistent grid of warps walks the
-// items of the experts that received rows only.  Per 256-wide K block a thread issues all of its
-// 16-byte weight loads (ld.global.nc.L1::no_allocate, streamed once) before using any of them;
-// activation planes are read through L1, where the warps of an SM working on the same expert
-// share them.  The down projection is split over K into `nsplit` fp32 partial sums (summed in
-// fixed order by the combine) so that a single token still spreads over every SM.
-//
-// Fragment bookkeeping: for each 64-wide K block a thread (g = lane/4, c = lane%4) loads 16
-// consecutive weight bytes [16c, 16c + 16) of rows g and g + 8.  MMA k-step s (0, 1) uses bytes
-// [16c + 8s, 16c + 8s + 8): the first four as logical k = 4c..4c+3 and the last four as
-// k = 16+4c..16+4c+3.  The activation fragment of the same step is read from the same physical
-// positions, so the permutation of K inside the block is the same on both operands and the
-// dot product is unchanged.
+// The stream kernel is persistent, one CTA per SM: warp 0 issues TMA copies of weight tiles
+// (128-byte swizzle) and plane tiles into a ring of ~200 KB, warp 1 issues the MMAs, warps 2-5
+// run the epilogue from double-buffered accumulators.  Work items (touched expert, 128-row tile
+// of output channels, K split, 8/16/32-token chunk) are built on the device from the row
+// offsets, so experts that received no rows cost nothing.  The down projection is split over K
+// into fp32 partial sums (summed in fixed order by the combine) to spread one token over every
+// SM.  Every wait is bounded.
 #include <algorithm>
+#include <cstring>
 
 #include "common.cuh"
 
 namespace colibri {
 namespace {
-
-constexpr int kWarpsPerCta = 8;
-constexpr int KB = 256;  // K elements per streamed block (4 sub-blocks of 64)
-
-__device__ __forceinline__ uint4 ldg_stream(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
-__device__ __forceinline__ uint2 ldg_cached8(const void* p) {
-  uint2 v;
-  asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
-  return v;
-}
-
-__device__ __forceinline__ void mma_s8_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                             uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-      "{%0, %1, %2, %3};"
-      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 
 // One warp per row: a = max|x| / 127, hi = rint(x / a), lo = rint((x - a * hi) * 254 / a).
 __global__ void __launch_bounds__(256) dec_split_rows_kernel(const __nv_bfloat16* __restrict__ X, int R, int K,
@@ -105,183 +73,355 @@ __global__ void __launch_bounds__(256) dec_split_rows_kernel(const __nv_bfloat16
   }
 }
 
-// Map a work-item index onto (touched expert, item within that expert).  Experts that received
-// no rows own no items.  Returns false when the index is past the last item.
-__device__ __forceinline__ bool item_of(const int32_t* __restrict__ offsets, int E, int items_per_expert,
-                                        int item, int& e, int& local) {
-  int base = 0;
-  for (int q = 0; q < E; ++q) {
-    if (offsets[q + 1] - offsets[q] <= 0) continue;
-    if (item < base + items_per_expert) {
-      e = q;
-      local = item - base;
-      return true;
+// h = silu(g) * u from the gate/up partials, rounded to bf16 (as the bf16 path stores H), then
+// split into int8 planes like dec_split_rows.  One CTA per row; the row is kept in shared memory.
+constexpr int kFinishThreads = 256;
+constexpr int kFinishMaxSmem = 2 * kDecMaxFF;  // one bf16 row of H
+__global__ void __launch_bounds__(kFinishThreads) dec_finish_h_kernel(const float* __restrict__ GU, int nsplit, int R,
+                                                                      int f, int8_t* __restrict__ hi,
+                                                                      int8_t* __restrict__ lo,
+                                                                      float* __restrict__ scale) {
+  extern __shared__ __nv_bfloat16 hrow[];  // [f]
+  __shared__ float red[kFinishThreads / 32];
+  const int r = blockIdx.x;
+  const size_t plane = (size_t)R * f;
+  float mx = 0.f;
+  for (int j = threadIdx.x; j < f; j += kFinishThreads) {
+    float g = 0.f, u = 0.f;
+    for (int sp = 0; sp < nsplit; ++sp) {  // K-split partials, summed in split order
+      g += GU[(2 * sp) * plane + (size_t)r * f + j];
+      u += GU[(2 * sp + 1) * plane + (size_t)r * f + j];
     }
-    base += items_per_expert;
+    const __nv_bfloat16 h = __float2bfloat16_rn(silu_mul(g, u));
+    hrow[j] = h;
+    mx = fmaxf(mx, fabsf(__bfloat162float(h)));
   }
-  return false;
+#pragma unroll
+  for (int off = 16; off; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  mx = 0.f;
+#pragma unroll
+  for (int w = 0; w < kFinishThreads / 32; ++w) mx = fmaxf(mx, red[w]);
+  const float a = mx > 0.f ? mx / 127.f : 1.f;
+  const float inv_a = 1.f / a;
+  if (threadIdx.x == 0) scale[r] = a;
+  for (int j = threadIdx.x; j < f; j += kFinishThreads) {
+    const float xv = __bfloat162float(hrow[j]);
+    const float qh = fminf(fmaxf(rintf(xv * inv_a), -127.f), 127.f);
+    const float res = fmaf(-a, qh, xv);
+    const float ql = fminf(fmaxf(rintf(res * inv_a * 254.f), -127.f), 127.f);
+    hi[(size_t)r * f + j] = (int8_t)qh;
+    lo[(size_t)r * f + j] = (int8_t)ql;
+  }
 }
 
-// One warp: 16 weight rows [o0, o0 + 16) of NMAT matrices (row m of matrix `mat` at
-// wbase[mat] + m * ldw bytes) times token rows [r0, r0 + ntok) of the split activation planes
-// (`ldx` bytes per row), over K range [kbeg, kend); NT n-blocks of 8 tokens.  acc[m][n][p][4]
-// receives the s32 C fragments of plane p (0 = hi, 1 = lo).
-template <int NMAT, int NT>
-__device__ __forceinline__ void warp_stream(const int8_t* const (&wbase)[NMAT], int ldw,
-                                            const int8_t* __restrict__ Xhi, const int8_t* __restrict__ Xlo, int ldx,
-                                            int r0, int ntok, int kbeg, int kend, int lane,
-                                            int (&acc)[NMAT][NT][2][4]) {
-  const int g = lane >> 2, c = lane & 3;
-  const int8_t* wrow_g[NMAT];
-  const int8_t* wrow_g8[NMAT];
-#pragma unroll
-  for (int m = 0; m < NMAT; ++m) {
-    wrow_g[m] = wbase[m] + (size_t)g * ldw;
-    wrow_g8[m] = wbase[m] + (size_t)(g + 8) * ldw;
+// ------------------------------------------------------------------------- stream kernel
+constexpr int kDsThreads = 192;
+constexpr int kDsTmemCols = 256;
+constexpr size_t kDsRingBytes = 200 * 1024;
+constexpr int kDsMaxStages = 12;
+
+struct alignas(64) DecStreamParams {
+  CUtensorMap mapW;   // int8 weights: gate/up {d, f, 2, E} (W1, W3); down {f, d, E} (W2)
+  CUtensorMap mapHi;  // int8 activation planes {K, R}
+  CUtensorMap mapLo;
+  const float* wscale;      // expert scales base (per expert: s1[f] | s3[f] | s2[d])
+  const float* rscale;      // plane row scales [R]
+  const int32_t* offsets;   // [E+1]
+  int E, d, f;
+  int out_rows;             // f (gate/up) or d (down)
+  int K, nsplit, kspan;     // kspan: K range of one split (a multiple of 128 unless nsplit == 1)
+  int nt8;                  // tokens per chunk (8, 16 or 32); MMA N = 2 * nt8
+  int R;                    // rows of the planes (T * k)
+  uint32_t stage_bytes;
+  int stages;
+  float* GU;                // gate/up output: [nsplit, 2, R, f] fp32 partials (W1 . x, W3 . x, scaled)
+  float* Ypart;             // down output [nsplit, R, d]
+  uint32_t* err;
+};
+
+struct DecItem {
+  int e, mat, tile, split, chunk, row0, ntok;
+};
+
+// Items of one touched expert: (matrix: W1 and W3 for gate/up, W2 for down) x 128-row tiles x
+// K splits x token chunks, tile fastest.
+template <bool kGateUp>
+__device__ __forceinline__ bool dec_item(const DecStreamParams& p, const int32_t* touched, const int32_t* item_prefix,
+                                         int ntouched, int L, DecItem& it) {
+  if (L >= item_prefix[ntouched]) return false;
+  int lo = 0, hi = ntouched - 1;  // largest ti with item_prefix[ti] <= L
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (item_prefix[mid] <= L) lo = mid;
+    else hi = mid - 1;
   }
-  size_t xoff[NT];
-  bool xv[NT];
-#pragma unroll
-  for (int n = 0; n < NT; ++n) {
-    const int t = n * 8 + g;
-    xv[n] = t < ntok;
-    xoff[n] = (size_t)(r0 + (xv[n] ? t : 0)) * ldx + 16 * c;
+  const int e = touched[lo];
+  const int tiles = (p.out_rows + 127) / 128;
+  int local = L - item_prefix[lo];
+  it.e = e;
+  it.tile = local % tiles;
+  local /= tiles;
+  if (kGateUp) {
+    it.mat = local & 1;
+    local >>= 1;
+  } else {
+    it.mat = 0;
   }
-  for (int k0 = kbeg; k0 < kend; k0 += KB) {
-    const int nsub = min(4, (kend - k0) >> 6);
-    uint4 wl[4][NMAT], wh[4][NMAT];
+  it.split = local % p.nsplit;
+  it.chunk = local / p.nsplit;
+  const int base = p.offsets[e], cnt = p.offsets[e + 1] - base;
+  it.row0 = base + it.chunk * p.nt8;
+  it.ntok = min(p.nt8, cnt - it.chunk * p.nt8);
+  return true;
+}
+
+__device__ __forceinline__ bool ds_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  uint32_t n = 0;
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((++n & 255u) == 0) {
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > kWaitTimeoutNs) return false;
+    }
+  }
+}
+
+template <bool kGateUp>
+__global__ void __launch_bounds__(kDsThreads, 1) dec_stream_kernel(const __grid_constant__ DecStreamParams p) {
+  constexpr int NMAT = 1;  // one weight tile per item (W1 and W3 tiles of gate/up are separate items)
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) atomicOr(p.err, kErrWaitTimeout);
+    return;
+  }
+  const int S = p.stages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * p.stage_bytes);
+  uint64_t* empty = full + S;
+  uint64_t* tfull = empty + S;    // [2]
+  uint64_t* tempty = tfull + 2;   // [2]
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int32_t* ntouched_s = reinterpret_cast<int32_t*>(tmem_holder + 2);
+  int32_t* issued_s = ntouched_s + 1;   // copies issued / stages consumed, for the error path
+  int32_t* consumed_s = ntouched_s + 2;
+  int32_t* touched = ntouched_s + 3;             // [E]
+  int32_t* item_prefix = touched + kMaxExperts;  // [E + 1]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *issued_s = 0;
+    *consumed_s = 0;
+    mbar_fence_init();
+    tma_prefetch_desc(&p.mapW);
+    tma_prefetch_desc(&p.mapHi);
+    tma_prefetch_desc(&p.mapLo);
+    // touched experts and the prefix of their work items
+    const int tiles = (p.out_rows + 127) / 128;
+    int n = 0, acc = 0;
+    for (int e = 0; e < p.E; ++e) {
+      const int cnt = p.offsets[e + 1] - p.offsets[e];
+      if (cnt <= 0) continue;
+      touched[n] = e;
+      item_prefix[n] = acc;
+      acc += tiles * (kGateUp ? 2 : 1) * p.nsplit * ((cnt + p.nt8 - 1) / p.nt8);
+      ++n;
+    }
+    item_prefix[n] = acc;
+    *ntouched_s = n;
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, kDsTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int ntouched = *ntouched_s;
+  const int N = 2 * p.nt8;
+  const uint32_t a_bytes = 128u * 128u;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      const uint32_t tx = NMAT * a_bytes + (uint32_t)N * 128u;
+      int issued = 0;
+      bool ok = true;
+      DecItem it;
+      for (int L = blockIdx.x; ok && dec_item<kGateUp>(p, touched, item_prefix, ntouched, L, it); L += gridDim.x) {
+        const int kbeg = it.split * p.kspan, kend = min(p.K, kbeg + p.kspan);
+        for (int kx = kbeg; kx < kend; kx += 128) {
+          if (!ds_wait(&empty[s], ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + (size_t)s * p.stage_bytes;
+          mbar_arrive_expect_tx(&full[s], tx);
+          if (kGateUp) tma_load_4d(st, &p.mapW, &full[s], kx, it.tile * 128, it.mat, it.e);
+          else tma_load_3d(st, &p.mapW, &full[s], kx, it.tile * 128, it.e);
+          uint8_t* sb = st + NMAT * a_bytes;
+          tma_load_2d(sb, &p.mapHi, &full[s], kx, it.row0);
+          tma_load_2d(sb + p.nt8 * 128, &p.mapLo, &full[s], kx, it.row0);
+          ++issued;
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        atomicOr(p.err, kErrWaitTimeout);
+      }
+      *issued_s = issued;
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_s8_s32(128, N);
+      int s = 0;
+      uint32_t ph = 0;
+      int iter = 0, consumed = 0;
+      bool ok = true;
+      DecItem it;
+      for (int L = blockIdx.x; ok && dec_item<kGateUp>(p, touched, item_prefix, ntouched, L, it);
+           L += gridDim.x, ++iter) {
+        const int a = iter & 1;
+        const uint32_t aph = (uint32_t)(iter >> 1) & 1u;
+        if (!ds_wait(&tempty[a], aph ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dbase = tmem + (uint32_t)(a * NMAT * N);
+        const int kbeg = it.split * p.kspan, kend = min(p.K, kbeg + p.kspan);
+        bool first = true;
+        for (int kx = kbeg; kx < kend; kx += 128) {
+          if (!ds_wait(&full[s], ph, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = smem_u32(smem + (size_t)s * p.stage_bytes);
+          const uint32_t sb = st + NMAT * a_bytes;
 #pragma unroll
-    for (int sub = 0; sub < 4; ++sub) {
-      if (sub < nsub) {
+          for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m)
+              tc_mma_i8(dbase + (uint32_t)(m * N), smem_desc_sw128(st + m * a_bytes + kk * 32),
+                        smem_desc_sw128(sb + kk * 32), idesc, (first && kk == 0) ? 0u : 1u);
+          }
+          first = false;
+          tc_commit(&empty[s]);
+          ++consumed;
+          if (++s == S) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&tfull[a]);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        atomicOr(p.err, kErrWaitTimeout);
+      }
+      *consumed_s = consumed;
+      tc_commit(drain);
+      mbar_wait_bounded(drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------- epilogue (warps 2..5)
+    const int q = warp & 3;
+    int iter = 0;
+    DecItem it;
+    for (int L = blockIdx.x; dec_item<kGateUp>(p, touched, item_prefix, ntouched, L, it); L += gridDim.x, ++iter) {
+      const int a = iter & 1;
+      const uint32_t aph = (uint32_t)(iter >> 1) & 1u;
+      const bool got = ds_wait(&tfull[a], aph, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const int o = it.tile * 128 + q * 32 + lane;
+      const bool vo = o < p.out_rows;
+      const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * NMAT * N);
+      const float* es = p.wscale + (size_t)it.e * (2 * p.f + p.d);
+      const float sc = vo ? es[(kGateUp ? it.mat * p.f : 2 * p.f) + o] : 0.f;
+      // columns [0, nt8) hold the hi plane, [nt8, 2 nt8) the lo plane of the same tokens
+      for (int j = 0; j < p.nt8; j += (p.nt8 == 8 ? 8 : 16)) {
+        float hi[NMAT][16], lo[NMAT][16];
 #pragma unroll
         for (int m = 0; m < NMAT; ++m) {
-          wl[sub][m] = ldg_stream(wrow_g[m] + k0 + sub * 64 + 16 * c);
-          wh[sub][m] = ldg_stream(wrow_g8[m] + k0 + sub * 64 + 16 * c);
-        }
-      }
-    }
+          if (p.nt8 == 8) {  // one load: columns 0-7 hi, 8-15 lo
+            float v[16];
+            tmem_ld16(tb + m * N, v);
+            tmem_ld_wait();
 #pragma unroll
-    for (int sub = 0; sub < 4; ++sub) {
-      if (sub >= nsub) break;
-      const int kx = k0 + sub * 64;
+            for (int i = 0; i < 8; ++i) {
+              hi[m][i] = (float)__float_as_int(v[i]);
+              lo[m][i] = (float)__float_as_int(v[8 + i]);
+            }
+          } else {
+            float vh[16], vl[16];
+            tmem_ld16(tb + m * N + j, vh);
+            tmem_ld16(tb + m * N + p.nt8 + j, vl);
+            tmem_ld_wait();
 #pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        uint4 xh = make_uint4(0u, 0u, 0u, 0u), xl = make_uint4(0u, 0u, 0u, 0u);
-        if (xv[n]) {
-          xh = *reinterpret_cast<const uint4*>(Xhi + xoff[n] + kx);
-          xl = *reinterpret_cast<const uint4*>(Xlo + xoff[n] + kx);
-        }
-#pragma unroll
-        for (int st = 0; st < 2; ++st) {
-          const uint32_t bh0 = st ? xh.z : xh.x, bh1 = st ? xh.w : xh.y;
-          const uint32_t bl0 = st ? xl.z : xl.x, bl1 = st ? xl.w : xl.y;
-#pragma unroll
-          for (int m = 0; m < NMAT; ++m) {
-            const uint32_t a0 = st ? wl[sub][m].z : wl[sub][m].x, a2 = st ? wl[sub][m].w : wl[sub][m].y;
-            const uint32_t a1 = st ? wh[sub][m].z : wh[sub][m].x, a3 = st ? wh[sub][m].w : wh[sub][m].y;
-            mma_s8_16832(acc[m][n][0], a0, a1, a2, a3, bh0, bh1);
-            mma_s8_16832(acc[m][n][1], a0, a1, a2, a3, bl0, bl1);
+            for (int i = 0; i < 16; ++i) {
+              hi[m][i] = (float)__float_as_int(vh[i]);
+              lo[m][i] = (float)__float_as_int(vl[i]);
+            }
           }
         }
+        const int width = p.nt8 == 8 ? 8 : 16;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int t = j + i;
+          if (i >= width || t >= it.ntok || !vo) continue;
+          const int row = it.row0 + t;
+          const float v = sc * p.rscale[row] * (hi[0][i] + lo[0][i] * (1.0f / 254.0f));
+          if (kGateUp) p.GU[(((size_t)it.split * 2 + it.mat) * p.R + row) * p.f + o] = v;
+          else p.Ypart[((size_t)it.split * p.R + row) * p.d + o] = v;
+        }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[a]);
     }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) {
+    // copies issued but never consumed: wait (bounded) until they land before the CTA exits
+    for (int i = *consumed_s; i < *issued_s; ++i) mbar_wait_bounded(&full[i % S], (uint32_t)(i / S) & 1u);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kDsTmemCols);
   }
 }
 
-// s32 accumulators of the two planes -> fp32 dot product in units of the row scale a
-__device__ __forceinline__ float planes(const int (&hl)[2][4], int q) {
-  return (float)hl[0][q] + (float)hl[1][q] * (1.0f / 254.0f);
-}
+int dec_nt8(int max_rows_per_expert) { return max_rows_per_expert <= 8 ? 8 : (max_rows_per_expert <= 16 ? 16 : 32); }
 
-// One CTA of 8 warps per SM for the 16- and 32-token variants (their accumulators need the
-// registers), two per SM for the 8-token variant.
-template <int NT>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, NT == 1 ? 2 : 1) dec_gateup_kernel(
-    const int8_t* __restrict__ Xhi, const int8_t* __restrict__ Xlo, const float* __restrict__ xscale,
-    const int8_t* __restrict__ W, const float* __restrict__ scales, int64_t wstride, int d, int f, int E,
-    const int32_t* __restrict__ offsets, __nv_bfloat16* __restrict__ H) {
-  const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
-  const int warp_id = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
-  const int nwarps = gridDim.x * kWarpsPerCta;
-  const int items_per_expert = f / 16;
-  for (int item = warp_id;; item += nwarps) {
-    int e, local;
-    if (!item_of(offsets, E, items_per_expert, item, e, local)) break;
-    const int row_base = offsets[e], cnt = offsets[e + 1] - row_base;
-    const int o0 = local * 16;
-    const int8_t* base = W + (int64_t)e * wstride;
-    const int8_t* const wb[2] = {base + (size_t)o0 * d, base + (size_t)f * d + (size_t)o0 * d};
-    const float* sc = scales + (int64_t)e * (2 * f + d);
-    for (int tc0 = 0; tc0 < cnt; tc0 += NT * 8) {
-      const int ntok = min(NT * 8, cnt - tc0);
-      int acc[2][NT][2][4] = {};
-      warp_stream<2, NT>(wb, d, Xhi, Xlo, d, row_base + tc0, ntok, 0, d, lane, acc);
-#pragma unroll
-      for (int n = 0; n < NT; ++n) {
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {  // columns 2c, 2c + 1 (tokens)
-          const int tk = n * 8 + 2 * c + cc;
-          if (tk >= ntok) continue;
-          const int row = row_base + tc0 + tk;
-          const float a = xscale[row];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {  // output rows g, g + 8
-            const int o = o0 + g + 8 * h;
-            const float gv = sc[o] * a * planes(acc[0][n], 2 * h + cc);
-            const float uv = sc[f + o] * a * planes(acc[1][n], 2 * h + cc);
-            H[(size_t)row * f + o] = __float2bfloat16_rn(silu_mul(gv, uv));
-          }
-        }
-      }
-    }
-  }
-}
-
-template <int NT>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, NT == 1 ? 2 : 1) dec_down_kernel(
-    const int8_t* __restrict__ Hhi, const int8_t* __restrict__ Hlo, const float* __restrict__ hscale,
-    const int8_t* __restrict__ W, const float* __restrict__ scales, int64_t wstride, int d, int f, int E,
-    const int32_t* __restrict__ offsets, int nsplit, int rows, float* __restrict__ Ypart) {
-  const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
-  const int warp_id = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
-  const int nwarps = gridDim.x * kWarpsPerCta;
-  const int groups = d / 16;
-  const int items_per_expert = groups * nsplit;
-  const int kspan = f / nsplit;
-  for (int item = warp_id;; item += nwarps) {
-    int e, local;
-    if (!item_of(offsets, E, items_per_expert, item, e, local)) break;
-    const int split = local / groups, o0 = (local - split * groups) * 16;
-    const int row_base = offsets[e], cnt = offsets[e + 1] - row_base;
-    const int8_t* base = W + (int64_t)e * wstride + 2 * (size_t)f * d;
-    const int8_t* const wb[1] = {base + (size_t)o0 * f};
-    const float* s2 = scales + (int64_t)e * (2 * f + d) + 2 * f;
-    float* out = Ypart + (size_t)split * rows * d;
-    const int kbeg = split * kspan, kend = kbeg + kspan;
-    for (int tc0 = 0; tc0 < cnt; tc0 += NT * 8) {
-      const int ntok = min(NT * 8, cnt - tc0);
-      int acc[1][NT][2][4] = {};
-      warp_stream<1, NT>(wb, f, Hhi, Hlo, f, row_base + tc0, ntok, kbeg, kend, lane, acc);
-#pragma unroll
-      for (int n = 0; n < NT; ++n) {
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int tk = n * 8 + 2 * c + cc;
-          if (tk >= ntok) continue;
-          const int row = row_base + tc0 + tk;
-          const float a = hscale[row];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int o = o0 + g + 8 * h;
-            out[(size_t)row * d + o] = s2[o] * a * planes(acc[0][n], 2 * h + cc);
-          }
-        }
-      }
-    }
-  }
-}
-
-int persistent_ctas(int per_sm) {
+int sm_count_current() {
   static int sms = 0;
   if (!sms) {
     int dev = 0;
@@ -289,7 +429,21 @@ int persistent_ctas(int per_sm) {
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (sms <= 0) sms = 148;
   }
-  return sms * per_sm;
+  return sms;
+}
+
+template <bool kGateUp>
+cudaError_t launch_stream(DecStreamParams& p, const int8_t* hi, const int8_t* lo, int K, cudaStream_t s) {
+  constexpr int NMAT = 1;
+  const uint64_t pd[2] = {(uint64_t)K, (uint64_t)p.R}, ps[1] = {(uint64_t)K};
+  const uint32_t pb[2] = {128, (uint32_t)p.nt8};
+  if (!make_tmap(&p.mapHi, CU_TENSOR_MAP_DATA_TYPE_UINT8, hi, 2, pd, ps, pb)) return cudaErrorInvalidValue;
+  if (!make_tmap(&p.mapLo, CU_TENSOR_MAP_DATA_TYPE_UINT8, lo, 2, pd, ps, pb)) return cudaErrorInvalidValue;
+  p.stage_bytes = (uint32_t)(NMAT * 128 * 128 + 2 * p.nt8 * 128);
+  p.stages = (int)std::min<size_t>(kDsMaxStages, kDsRingBytes / p.stage_bytes);
+  const size_t smem = (size_t)p.stages * p.stage_bytes + 4096;
+  dec_stream_kernel<kGateUp><<<sm_count_current(), kDsThreads, smem, s>>>(p);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -302,35 +456,77 @@ cudaError_t launch_dec_split(const __nv_bfloat16* X, int R, int K, int8_t* hi, i
   return cudaGetLastError();
 }
 
+cudaError_t configure_dec_kernels() {
+  const int smem = (int)(kDsRingBytes + 4096);
+  cudaError_t e = cudaFuncSetAttribute(dec_stream_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(dec_stream_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(dec_finish_h_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFinishMaxSmem);
+  return e;
+}
+
 cudaError_t launch_dec_gateup(const int8_t* Xhi, const int8_t* Xlo, const float* xscale, const int8_t* W,
                               const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
-                              __nv_bfloat16* H, int max_rows_per_expert, cudaStream_t s) {
-  const int grid = persistent_ctas(max_rows_per_expert <= 8 ? 2 : 1);
-  const int threads = kWarpsPerCta * 32;
-  if (max_rows_per_expert <= 8)
-    dec_gateup_kernel<1><<<grid, threads, 0, s>>>(Xhi, Xlo, xscale, W, scales, wstride, d, f, E, offsets, H);
-  else if (max_rows_per_expert <= 16)
-    dec_gateup_kernel<2><<<grid, threads, 0, s>>>(Xhi, Xlo, xscale, W, scales, wstride, d, f, E, offsets, H);
-  else
-    dec_gateup_kernel<4><<<grid, threads, 0, s>>>(Xhi, Xlo, xscale, W, scales, wstride, d, f, E, offsets, H);
+                              int nsplit, float* GU, int R, int max_rows_per_expert, uint32_t* err, cudaStream_t s) {
+  DecStreamParams p;
+  memset(&p, 0, sizeof(p));
+  const uint64_t dims[4] = {(uint64_t)d, (uint64_t)f, 2, (uint64_t)E};
+  const uint64_t st[3] = {(uint64_t)d, (uint64_t)f * d, (uint64_t)wstride};
+  const uint32_t box[4] = {128, 128, 1, 1};
+  if (!make_tmap(&p.mapW, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, 4, dims, st, box)) return cudaErrorInvalidValue;
+  p.wscale = scales;
+  p.rscale = xscale;
+  p.offsets = offsets;
+  p.E = E;
+  p.d = d;
+  p.f = f;
+  p.out_rows = f;
+  p.K = d;
+  p.nsplit = nsplit;
+  p.kspan = d / nsplit;
+  p.nt8 = dec_nt8(max_rows_per_expert);
+  p.R = R;
+  p.GU = GU;
+  p.err = err;
+  return launch_stream<true>(p, Xhi, Xlo, d, s);
+}
+
+cudaError_t launch_dec_finish_h(const float* GU, int nsplit, int R, int f, int8_t* hi, int8_t* lo, float* scale,
+                                cudaStream_t s) {
+  if (R <= 0) return cudaSuccess;
+  const size_t smem = (size_t)f * sizeof(__nv_bfloat16);
+  if (smem > (size_t)kFinishMaxSmem) return cudaErrorInvalidValue;
+  dec_finish_h_kernel<<<R, kFinishThreads, smem, s>>>(GU, nsplit, R, f, hi, lo, scale);
   return cudaGetLastError();
 }
 
 cudaError_t launch_dec_down(const int8_t* Hhi, const int8_t* Hlo, const float* hscale, const int8_t* W,
                             const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
-                            int nsplit, int rows, float* Ypart, int max_rows_per_expert, cudaStream_t s) {
-  const int grid = persistent_ctas(max_rows_per_expert <= 8 ? 2 : 1);
-  const int threads = kWarpsPerCta * 32;
-  if (max_rows_per_expert <= 8)
-    dec_down_kernel<1><<<grid, threads, 0, s>>>(Hhi, Hlo, hscale, W, scales, wstride, d, f, E, offsets, nsplit, rows,
-                                                Ypart);
-  else if (max_rows_per_expert <= 16)
-    dec_down_kernel<2><<<grid, threads, 0, s>>>(Hhi, Hlo, hscale, W, scales, wstride, d, f, E, offsets, nsplit, rows,
-                                                Ypart);
-  else
-    dec_down_kernel<4><<<grid, threads, 0, s>>>(Hhi, Hlo, hscale, W, scales, wstride, d, f, E, offsets, nsplit, rows,
-                                                Ypart);
-  return cudaGetLastError();
+                            int nsplit, int R, float* Ypart, int max_rows_per_expert, uint32_t* err,
+                            cudaStream_t s) {
+  DecStreamParams p;
+  memset(&p, 0, sizeof(p));
+  const uint64_t dims[3] = {(uint64_t)f, (uint64_t)d, (uint64_t)E};
+  const uint64_t st[2] = {(uint64_t)f, (uint64_t)wstride};
+  const uint32_t box[3] = {128, 128, 1};
+  if (!make_tmap(&p.mapW, CU_TENSOR_MAP_DATA_TYPE_UINT8, W + 2 * (size_t)f * d, 3, dims, st, box))
+    return cudaErrorInvalidValue;
+  p.wscale = scales;
+  p.rscale = hscale;
+  p.offsets = offsets;
+  p.E = E;
+  p.d = d;
+  p.f = f;
+  p.out_rows = d;
+  p.K = f;
+  p.nsplit = nsplit;
+  p.kspan = f / nsplit;
+  p.nt8 = dec_nt8(max_rows_per_expert);
+  p.R = R;
+  p.Ypart = Ypart;
+  p.err = err;
+  return launch_stream<false>(p, Hhi, Hlo, f, s);
 }
 
 }  // namespace colibri

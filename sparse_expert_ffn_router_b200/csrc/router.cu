@@ -132,6 +132,52 @@ __global__ void __launch_bounds__(kRouterThreads) router_topk_simt_kernel(
 }
 
 // ---------------------------------------------------------------------------------------
+// Small batches (T <= 64): one CTA per token.  Warp w computes the logits of experts w, w + 8,
+// ... with its lanes splitting d (16-byte loads; the token row is read through L1) and a
+// shuffle reduction; then warp 0 selects the top-k.  Latency-bound work, so no tensor cores.
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ float dot16(const uint4& xa, const uint4& wa, float acc, const __nv_bfloat16*) {
+  const __nv_bfloat162* xh = reinterpret_cast<const __nv_bfloat162*>(&xa);
+  const __nv_bfloat162* wh = reinterpret_cast<const __nv_bfloat162*>(&wa);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 xf = __bfloat1622float2(xh[i]), wf = __bfloat1622float2(wh[i]);
+    acc = fmaf(xf.x, wf.x, acc);
+    acc = fmaf(xf.y, wf.y, acc);
+  }
+  return acc;
+}
+__device__ __forceinline__ float dot16(const uint4& xa, const uint4& wa, float acc, const float*) {
+  acc = fmaf(__uint_as_float(xa.x), __uint_as_float(wa.x), acc);
+  acc = fmaf(__uint_as_float(xa.y), __uint_as_float(wa.y), acc);
+  acc = fmaf(__uint_as_float(xa.z), __uint_as_float(wa.z), acc);
+  acc = fmaf(__uint_as_float(xa.w), __uint_as_float(wa.w), acc);
+  return acc;
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(256) router_small_kernel(const Tin* __restrict__ x, int d,
+                                                           const Tin* __restrict__ wr, const float* __restrict__ b,
+                                                           int E, int k, int32_t* __restrict__ idx_out,
+                                                           float* __restrict__ w_out) {
+  __shared__ float lg[kMaxExperts];
+  const int t = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nvec = d * (int)sizeof(Tin) / 16;
+  const uint4* xv = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+  for (int e = warp; e < E; e += 8) {
+    const uint4* wv = reinterpret_cast<const uint4*>(wr + (size_t)e * d);
+    float acc = 0.f;
+#pragma unroll 4
+    for (int v = lane; v < nvec; v += 32) acc = dot16(__ldg(xv + v), __ldg(wv + v), acc, x);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) lg[e] = acc + (b ? b[e] : 0.f);
+  }
+  __syncthreads();
+  if (warp == 0) warp_topk(lg, E, k, lane, idx_out + (size_t)t * k, w_out + (size_t)t * k);
+}
+
+// ---------------------------------------------------------------------------------------
 // bf16 router on the 5th-generation tensor cores.  A CTA owns 128 tokens (the 128 TMEM lanes)
 // and all experts padded to N = 16 * ceil(E / 16) columns: one elected thread streams x and Wr
 // tiles (64-wide K blocks, 128-byte swizzle) through a 4-stage shared-memory ring with TMA and
@@ -150,6 +196,9 @@ struct alignas(64) RouterTcParams {
   CUtensorMap mapW;  // [E, d], box {64, N}
   const float* b;
   int T, d, E, k, N;
+  int ksplit;        // CTAs per 128-token tile, each over d / ksplit (gridDim.y)
+  float* part;       // [ksplit, E, T] partial logits (ksplit > 1; token-contiguous, so stores coalesce)
+  int32_t* ticket;   // [tiles] arrival counters, zero between calls (ksplit > 1)
   int stages;  // ring depth: as many stages as fit in kRtRingBytes (small expert counts go deeper)
   uint32_t stage_bytes, tmem_cols;
   int32_t* idx;
@@ -203,20 +252,35 @@ __global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const int row0 = blockIdx.x * 128;
-  const int nkb = p.d / 64;
+  const int kspan = p.d / p.ksplit;               // a multiple of 64
+  const int kb0 = blockIdx.y * (kspan / 64);
+  const int nkb = kspan / 64;
 
+  const uint32_t bytes = kRtABytes + (uint32_t)p.N * 128u;
   if (threadIdx.x == 0) {
-    const uint32_t idesc = idesc_bf16_f32(128, p.N);
-    const uint32_t bytes = kRtABytes + (uint32_t)p.N * 128u;
-    auto issue = [&](int kb) {
-      uint8_t* sa = smem + (size_t)(kb % S) * p.stage_bytes;
-      mbar_arrive_expect_tx(&full[kb % S], bytes);
-      tma_load_2d(sa, &p.mapX, &full[kb % S], kb * 64, row0);
-      tma_load_2d(sa + kRtABytes, &p.mapW, &full[kb % S], kb * 64, 0);
-    };
-    for (int kb = 0; kb < nkb && kb < S; ++kb) issue(kb);
+    // ------------------------------------------------------------- TMA producer (warp 0)
     bool ok = true;
-    for (int kb = 0; kb < nkb && ok; ++kb) {
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % S;
+      const uint32_t ph = (uint32_t)(kb / S) & 1u;
+      if (!rt_wait(&empty[s], ph ^ 1u, abort_flag)) {
+        ok = false;
+        break;
+      }
+      uint8_t* sa = smem + (size_t)s * p.stage_bytes;
+      mbar_arrive_expect_tx(&full[s], bytes);
+      tma_load_2d(sa, &p.mapX, &full[s], (kb0 + kb) * 64, row0);
+      tma_load_2d(sa + kRtABytes, &p.mapW, &full[s], (kb0 + kb) * 64, 0);
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      if (p.err) atomicOr(p.err, kErrWaitTimeout);
+    }
+  } else if (threadIdx.x == 32) {
+    // ------------------------------------------------------------- MMA issuer (warp 1)
+    const uint32_t idesc = idesc_bf16_f32(128, p.N);
+    bool ok = true;
+    for (int kb = 0; kb < nkb; ++kb) {
       const int s = kb % S;
       const uint32_t ph = (uint32_t)(kb / S) & 1u;
       if (!rt_wait(&full[s], ph, abort_flag)) {
@@ -229,14 +293,7 @@ __global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant
       for (int kk = 0; kk < 4; ++kk)
         tc_mma_f16(tmem, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sa + kRtABytes + kk * 32), idesc,
                    (kb | kk) != 0 ? 1u : 0u);
-      tc_commit(&empty[s]);
-      if (kb + S < nkb) {
-        if (!rt_wait(&empty[s], ph, abort_flag)) {  // MMAs of this stage done: refill it
-          ok = false;
-          break;
-        }
-        issue(kb + S);
-      }
+      tc_commit(&empty[s]);  // frees the stage once these MMAs have read it
     }
     if (!ok) {
       *abort_flag = 1;
@@ -255,12 +312,46 @@ __global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant
     bv[j] = -INFINITY;
     bi[j] = 0x7fffffff;
   }
-  if (warp_ok) {
-    const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16);
+  __shared__ int last_cta;
+  const int t = row0 + threadIdx.x;
+  const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16);
+  bool select = warp_ok;
+  if (p.ksplit > 1) {
+    // write this K slice's logits, then the last CTA of the tile sums the slices in order
+    if (warp_ok) {
+      for (int c0 = 0; c0 < p.N; c0 += 16) {
+        float v[16];
+        tmem_ld16(tbase + c0, v);
+        tmem_ld_wait();
+        if (t < p.T)
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (c0 + i < p.E) p.part[((size_t)blockIdx.y * p.E + c0 + i) * p.T + t] = v[i];
+      }
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last_cta = (atomicAdd(&p.ticket[blockIdx.x], 1) == p.ksplit - 1);
+    __syncthreads();
+    select = __all_sync(0xffffffffu, warp_ok) && last_cta;
+    if (last_cta && threadIdx.x == 0) p.ticket[blockIdx.x] = 0;  // ready for the next call
+    __threadfence();
+  }
+  if (select) {
     for (int c0 = 0; c0 < p.N; c0 += 16) {
       float v[16];
-      tmem_ld16(tbase + c0, v);
-      tmem_ld_wait();
+      if (p.ksplit == 1) {
+        tmem_ld16(tbase + c0, v);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float acc = 0.f;
+          if (t < p.T && c0 + i < p.E)
+            for (int sp = 0; sp < p.ksplit; ++sp) acc += __ldcg(&p.part[((size_t)sp * p.E + c0 + i) * p.T + t]);
+          v[i] = acc;
+        }
+      }
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int e = c0 + i;
@@ -281,7 +372,6 @@ __global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant
         }
       }
     }
-    const int t = row0 + threadIdx.x;
     if (t < p.T) {
       float den = 0.f;
 #pragma unroll
@@ -306,10 +396,14 @@ __global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant
 constexpr size_t kRtMaxSmem = kRtRingBytes + 1024;
 
 cudaError_t launch_router_tc(const void* x, int T, int d, const void* wr, const float* b, int E, int k,
-                             int32_t* idx, float* w, uint32_t* err, cudaStream_t s) {
+                             int32_t* idx, float* w, uint32_t* err, int ksplit, float* part, int32_t* ticket,
+                             cudaStream_t s) {
   RouterTcParams p;
   memset(&p, 0, sizeof(p));
   p.N = (E + 15) / 16 * 16;
+  p.ksplit = ksplit;
+  p.part = part;
+  p.ticket = ticket;
   {
     const uint64_t dims[2] = {(uint64_t)d, (uint64_t)T}, st[1] = {(uint64_t)d * 2};
     const uint32_t box[2] = {64, 128};
@@ -333,7 +427,7 @@ cudaError_t launch_router_tc(const void* x, int T, int d, const void* wr, const 
   p.w = w;
   p.err = err;
   const size_t smem = (size_t)p.stages * p.stage_bytes + 1024;
-  router_tc_kernel<<<(T + 127) / 128, 128, smem, s>>>(p);
+  router_tc_kernel<<<dim3((T + 127) / 128, ksplit), 128, smem, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -352,10 +446,30 @@ cudaError_t configure_router_kernels() {
   return e;
 }
 
+int router_ksplit(int T, int d) {
+  if (T < kRouterSplitMinT) return 1;
+  const int tiles = (T + 127) / 128;
+  int ks = 1;
+  while (ks < 8 && tiles * ks * 2 <= 160 && (d / 64) % (2 * ks) == 0) ks <<= 1;
+  return ks;
+}
+
 cudaError_t launch_router_topk(const void* x, int act, int T, int d, const void* wr, const float* b,
-                               int E, int k, int32_t* idx, float* w, uint32_t* err, cudaStream_t s) {
+                               int E, int k, int32_t* idx, float* w, uint32_t* err, float* part,
+                               int32_t* ticket, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  if (act == COLIBRI_BF16) return launch_router_tc(x, T, d, wr, b, E, k, idx, w, err, s);
+  if (T <= kRouterSmallT) {
+    if (act == COLIBRI_BF16)
+      router_small_kernel<__nv_bfloat16><<<T, 256, 0, s>>>((const __nv_bfloat16*)x, d, (const __nv_bfloat16*)wr, b,
+                                                           E, k, idx, w);
+    else
+      router_small_kernel<float><<<T, 256, 0, s>>>((const float*)x, d, (const float*)wr, b, E, k, idx, w);
+    return cudaGetLastError();
+  }
+  if (act == COLIBRI_BF16) {
+    const int ks = (part && ticket) ? router_ksplit(T, d) : 1;
+    return launch_router_tc(x, T, d, wr, b, E, k, idx, w, err, ks, part, ticket, s);
+  }
   const size_t smem =
       sizeof(float) * ((size_t)kRouterTT * (kRouterDK + 1) + (size_t)E * (kRouterDK + 1) +
                        (size_t)kRouterTT * (E + 1));
