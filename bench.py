@@ -30,7 +30,23 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/sec (prefill & decode) and % of roofline on 1 B200"
 DEFAULT_WORKLOAD = "mixtral_prefill_bf16"
-KERNELS_PER_STEP_BASE = 7  # router, count, scan, scatter, gate/up, down, combine
+# T up to which the Scatter stage is one fused launch (histogram, prefix sum and scatter)
+FUSED_ROUTE_MAX_T = 64
+
+
+def kernels_per_step(wl):
+    """Kernels one forward launches, following the library's launch sequence."""
+    n = 1                                            # Gate: router + top-k
+    n += 1 if wl.T <= FUSED_ROUTE_MAX_T else 3       # Scatter: fused, or count + scan + scatter
+    if wl.wdt == 0:
+        n += 2 + (2 if wl.fs else 0)                 # fp32: gate/up + down (+ the shared expert's)
+    elif wl.wdt == 1:
+        n += 2                                       # bf16: gate/up + down (shared expert inside)
+    else:
+        n += 3                                       # int8: gate/up stream, finish H, down stream
+    return n + 1                                     # Gather
+
+
 # fp32 FMA peak: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (the unit counts and clock of the part)
 FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
@@ -222,6 +238,22 @@ def run_reference(a, rank, world):
     return 0
 
 
+def max_over_ranks(ms, world, device):
+    """The largest of the ranks' times: each rank times its own replica on its own device."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, tokens_per_step, steps, ms):
+    """Whole-job tokens/s: every rank processed `steps` batches of `tokens_per_step` in `ms`."""
+    return world * tokens_per_step * steps / (ms / 1e3)
+
+
 def config_of(wl):
     cfg = {"workload": wl.name, "T": wl.T, "d_model": wl.d, "num_experts": wl.E, "top_k": wl.k, "d_ff": wl.f,
            "act_dtype": {0: "f32", 1: "bf16"}[wl.act], "weight_dtype": {0: "f32", 1: "bf16", 2: "i8"}[wl.wdt]}
@@ -307,28 +339,50 @@ def main():
     barrier()
     stage_ms, ncalls = colibri.colibri_profile_end(layer.ctx)
     layer.sync_status()
-    t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
-    value = world * wl.T * a.steps / (ms_max / 1e3)
+    ms_max = max_over_ranks(ms_total, world, dev)
+    value = job_throughput(world, wl.T, a.steps, ms_max)
 
-    # ---- end to end through the same call with host buffers (pinned x in, y out)
+    # ---- end to end through the same call with host buffers (pinned x in, y out).  Every step
+    # copies its x from pinned host memory and its y back inside the call.  Serial: one context
+    # on one stream.  Pipelined (the reported e2e value): two contexts on two streams taking
+    # alternate steps, so one step's copies overlap the other's kernels, as a serving loop
+    # would run it.
     x_host = p.x.pin_memory() if not p.x.is_pinned() else p.x
-    y_host = torch.empty(wl.T, wl.d, dtype=x.dtype).pin_memory()
+    y_hosts = [torch.empty(wl.T, wl.d, dtype=x.dtype).pin_memory() for _ in range(2)]
     for _ in range(2):
-        step(x_host, y_host)
+        step(x_host, y_hosts[0])
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(a.steps):
-        step(x_host, y_host)
+        step(x_host, y_hosts[0])
     e1.record(stream)
     barrier()
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = world * wl.T * a.steps / (float(te.item()) / 1e3)
+    e2e_serial = job_throughput(world, wl.T, a.steps, max_over_ranks(e0.elapsed_time(e1), world, dev))
+
+    layer2 = colibri.MoELayer(wl.d, wl.f, wl.E, wl.k, wl.fs, wl.act, wl.wdt, max_tokens=wl.T, device_id=local)
+    stream2 = torch.cuda.Stream(device=dev)
+    ctxs, streams = (layer.ctx, layer2.ctx), (stream, stream2)
+
+    def e2e_step(i):
+        colibri.colibri_moe_forward(ctxs[i & 1], x_host, wl.T, rw, rb, ew, sc, sw, y_hosts[i & 1], streams[i & 1])
+
+    for i in range(4):
+        e2e_step(i)
+    barrier()
+    f0, f1, fj = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+                  torch.cuda.Event())
+    f0.record(stream)
+    stream2.wait_event(f0)
+    for i in range(a.steps):
+        e2e_step(i)
+    fj.record(stream2)
+    stream.wait_event(fj)
+    f1.record(stream)
+    barrier()
+    layer2.sync_status()
+    layer2.close()
+    e2e_value = job_throughput(world, wl.T, a.steps, max_over_ranks(f0.elapsed_time(f1), world, dev))
     row_bytes = wl.d * (4 if wl.act == 0 else 2)
 
     # ---- roofline of the dominant kernel (per-launch averages over the timed region)
@@ -336,12 +390,16 @@ def main():
     per_call = {k: v / max(ncalls, 1) for k, v in stage_ms.items()}
     if wl.wdt == 2:
         achieved = (wk["w13_bytes"] + wk["scale_bytes"]) / (per_call["expert_gateup"] / 1e3) / 1e9
-        roof = {"kernel": "dec_gateup_kernel (int8 weight stream, gate/up)", "bound": "hbm",
+        roof = {"kernel": "dec_stream_kernel<gate/up> (tcgen05 kind::i8 weight stream)", "bound": "hbm",
                 "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s", "frac": achieved / pk["hbm"],
                 "algorithmic_bytes_per_launch": wk["w13_bytes"] + wk["scale_bytes"]}
     elif wl.wdt == 1:
         achieved = wk["flops_gateup"] / (per_call["expert_gateup"] / 1e3) / 1e12
-        roof = {"kernel": "tc_ffn_kernel<gate/up> (tcgen05)", "bound": "tensor", "achieved": achieved,
+        pair = os.environ.get("COLIBRI_GEMM_CTA", "") == "2" or (
+            os.environ.get("COLIBRI_GEMM_CTA", "") != "1" and wl.T * wl.k // wl.E >= 512)
+        name = ("tc2_ffn_kernel<gate/up> (tcgen05, 2-CTA pair tiles)" if pair
+                else "tc_ffn_kernel<gate/up> (tcgen05)")
+        roof = {"kernel": name, "bound": "tensor", "achieved": achieved,
                 "peak": pk["bf16"], "unit": "TFLOP/s", "frac": achieved / pk["bf16"],
                 "algorithmic_flops_per_launch": wk["flops_gateup"]}
     else:
@@ -352,7 +410,7 @@ def main():
     roof["peak_source"] = pk["source"] + (" burst" if roof["bound"] == "tensor" else "")
     roof["traffic"] = None
     roof["timing"] = "kernel stage events averaged over the profiling region's calls"
-    kernels = KERNELS_PER_STEP_BASE + (2 if (wl.fs and wl.wdt == 0) else 0)
+    kernels = kernels_per_step(wl)
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
@@ -363,7 +421,9 @@ def main():
                        ((wk["w13_bytes"] + wk["w2_bytes"]) / 1e9), parallelism=f"replicas x{world}"),
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": wl.T * row_bytes,
-                "d2h_bytes_per_step": wl.T * row_bytes},
+                "d2h_bytes_per_step": wl.T * row_bytes, "serial_value": e2e_serial,
+                "how": "colibri_moe_forward with pinned host x and y (copies inside the call, every step); "
+                       "value: two contexts on two streams taking alternate steps; serial_value: one stream"},
         "gpu_launches": kernels * a.steps,
         "clocks": clk.summary(),
         "stage_ms_per_call": per_call,

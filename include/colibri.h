@@ -216,6 +216,17 @@ colibri_status colibri_route_noalloc(const void* x, int32_t act_dtype, int32_t T
                                      float* topk_w, int32_t* counts, int32_t* offsets,
                                      int32_t* src_row, int32_t* dst_row, void* Xp, void* stream);
 
+/*
+ * Failure-detection self test (no counterpart on the pages; it exercises the error reporting of
+ * www.mhpq.cn/news/563172 §4.3).  Enqueues on `stream` one kernel whose single thread waits on a
+ * device barrier that nothing ever completes, giving up after `timeout_us` microseconds
+ * (1..1000000) exactly as a stalled pipeline wait of the forward kernels gives up after 4 s: it
+ * sets the context's device error word and returns.  Nothing faults or hangs; the next
+ * colibri_sync_status() on that stream returns COLIBRI_ERR_TIMEOUT and clears the word, and the
+ * context stays usable.  Errors: INVALID_ARG (NULL ctx, timeout out of range), CUDA.
+ */
+colibri_status colibri_selftest_wait_timeout(colibri_ctx* ctx, int32_t timeout_us, void* stream);
+
 /* One-line description of a status code (static storage). */
 const char* colibri_status_string(colibri_status status);
 

@@ -153,6 +153,10 @@ WORKLOADS = {
     # on ~1.5 GB of device memory (still far larger than L2), sized for ncu captures
     "mixtral_prefill_bf16_small": Workload("mixtral_prefill_bf16_small", 1024, 4096, 4, 2, 14336,
                                            note="profiling-size Mixtral-shaped layer"),
+    # routing-dominated layer for profiling the router: 16384 tokens (x = 134 MB, larger than
+    # L2) over 8 experts with a tiny d_ff, ~0.2 GB on the device
+    "router_profile_bf16": Workload("router_profile_bf16", 16384, 4096, 8, 2, 64,
+                                    note="router profiling case"),
     # decode, int8 weights with per-output-channel scales
     "decode_int8_T1": Workload("decode_int8_T1", 1, 4096, 8, 2, 14336, act=BF16, wdt=I8),
     "decode_int8_T8": Workload("decode_int8_T8", 8, 4096, 8, 2, 14336, act=BF16, wdt=I8),

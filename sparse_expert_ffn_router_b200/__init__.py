@@ -39,6 +39,7 @@ EXPORTS = (
     "colibri_profile_begin",
     "colibri_profile_end",
     "colibri_route_noalloc",
+    "colibri_selftest_wait_timeout",
     "colibri_status_string",
     "colibri_last_error",
     "colibri_free",
@@ -96,6 +97,8 @@ def load() -> ctypes.CDLL:
     lib.colibri_profile_end.restype = ctypes.c_int
     lib.colibri_route_noalloc.argtypes = [vp, i32, i32, i32, vp, vp, i32, i32] + [vp] * 8
     lib.colibri_route_noalloc.restype = ctypes.c_int
+    lib.colibri_selftest_wait_timeout.argtypes = [vp, i32, vp]
+    lib.colibri_selftest_wait_timeout.restype = ctypes.c_int
     lib.colibri_status_string.argtypes = [ctypes.c_int]
     lib.colibri_status_string.restype = ctypes.c_char_p
     lib.colibri_last_error.argtypes = [vp]
@@ -175,6 +178,11 @@ def colibri_get_routing(ctx: int, topk_idx=None, topk_w=None, counts=None, offse
 
 def colibri_sync_status(ctx: int, stream=None) -> None:
     _check(load().colibri_sync_status(ctx, _stream(stream)), "colibri_sync_status", ctx)
+
+
+def colibri_selftest_wait_timeout(ctx: int, timeout_us: int, stream=None) -> None:
+    _check(load().colibri_selftest_wait_timeout(ctx, timeout_us, _stream(stream)),
+           "colibri_selftest_wait_timeout", ctx)
 
 
 NUM_STAGES = 5

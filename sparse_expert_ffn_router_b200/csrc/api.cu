@@ -111,6 +111,8 @@ void record_error(const char* msg) {
   g_last_error = msg;
   if (env_flag("COLIBRI_DEBUG")) fprintf(stderr, "[colibri] %s\n", msg);
 }
+// Records the reason of a failure on a context (or on no context) and returns `st`.
+colibri_status report(colibri_ctx* ctx, colibri_status st, const char* msg) { return fail(ctx, st, "%s", msg); }
 }  // namespace colibri
 
 extern "C" {
@@ -201,7 +203,7 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   const size_t o_idx = c.take(R * 4), o_w = c.take(R * 4), o_dst = c.take(R * 4), o_src = c.take(R * 4);
   const size_t o_bc = c.take((size_t)nblk * E * 4), o_bb = c.take((size_t)nblk * E * 4);
   const size_t o_cnt = c.take(E * 4), o_off = c.take((E + 1) * 4), o_mt = c.take((E + 1) * 4);
-  const size_t o_xp = c.take(R * d * as);
+  const size_t o_xp = c.take(i8 ? 0 : R * d * as);  // int8 weights read the row planes instead
   const size_t o_h = c.take(i8 ? std::max<int64_t>(2 * R, 2 * kDecGateSplitMax * std::min<int64_t>(R, kDecGateSplitRows)) * f * 4
                              : R * f * hs);
   const size_t o_yp = i8 ? c.take(0) : c.take(R * d * hs);
@@ -211,7 +213,7 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   const size_t o_part = c.take(part_rows * d * 4);
   const size_t plane_w = (size_t)std::max<int64_t>(d, f);
   const size_t o_phi = c.take(i8 ? R * plane_w : 0), o_plo = c.take(i8 ? R * plane_w : 0);
-  const size_t o_psc = c.take(i8 ? R * 4 : 0);
+  const size_t o_psc = c.take(i8 ? part_rows * 4 : 0);  // per (down K split, row) scales of the H planes
   const bool rsplit = D.act_dtype == COLIBRI_BF16 && M >= kRouterSplitMinT;
   const size_t o_rpart = c.take(rsplit ? (size_t)kRouterMaxSplit * M * E * 4 : 0);
   const size_t o_rtick = c.take(rsplit ? (size_t)((M + 127) / 128) * 4 : 0);
@@ -260,6 +262,7 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
     for (auto& e : ctx->ev) cudaEventCreate(&e);
   }
   ctx->use_graphs = !(getenv("COLIBRI_GRAPHS") && strcmp(getenv("COLIBRI_GRAPHS"), "0") == 0);
+  ctx->use_pdl = !(getenv("COLIBRI_PDL") && strcmp(getenv("COLIBRI_PDL"), "0") == 0);
   cudaError_t ce = configure_router_kernels();
   if (ce == cudaSuccess) ce = configure_tc_kernels();
   if (ce == cudaSuccess) ce = configure_dec_kernels();
@@ -317,8 +320,12 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
   const int R = T * k;
   const void* xd = x;
   void* yd = y;
+  // Kernels after the first may overlap their predecessor's tail (not while stage events are
+  // recorded between them: the events would then not bound the stages).
+  LaunchScope launch_scope(ctx->use_pdl && !ctx->profile && !ctx->prof_on);
   if (xk == kPtrHost) {
     COLIBRI_TRY(cudaMemcpyAsync(w.x_stage, x, (size_t)T * row_bytes, cudaMemcpyHostToDevice, s), "copy x to device");
+    launch_chain_break();
     xd = w.x_stage;
   }
   if (yk == kPtrHost) yd = w.y_stage;
@@ -336,6 +343,7 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
   if (routed_by_caller) {
     COLIBRI_TRY(cudaMemcpyAsync(w.topk_idx, user_idx, (size_t)R * 4, cudaMemcpyDeviceToDevice, s), "copy topk_idx");
     COLIBRI_TRY(cudaMemcpyAsync(w.topk_w, user_w, (size_t)R * 4, cudaMemcpyDeviceToDevice, s), "copy topk_w");
+    launch_chain_break();
   } else {
     COLIBRI_TRY(launch_router_topk(xd, act, T, d, router_w, router_b, E, k, w.topk_idx, w.topk_w, w.err,
                                    w.router_part, w.router_ticket, s),
@@ -346,15 +354,17 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
   // ---- Scatter
   const int nblk = (T + kCountBlock - 1) / kCountBlock;
   const int bm = D.weight_dtype == COLIBRI_F32 ? kSimtBM : (pair_tiles ? kTcPairBM : kTcBM);
+  const RowPlanes xplanes{w.plane_hi, w.plane_lo, w.plane_scale};
+  const RowPlanes* planes = D.weight_dtype == COLIBRI_I8 ? &xplanes : nullptr;
   if (T <= kFusedRouteMaxT) {
     COLIBRI_TRY(launch_route_fused(xd, act, T, d, w.topk_idx, k, E, bm, w.counts, w.offsets, w.mt_prefix,
-                                   w.src_row, w.dst_row, w.Xp, s), "route_fused");
+                                   w.src_row, w.dst_row, w.Xp, planes, s), "route_fused");
   } else {
     COLIBRI_TRY(launch_route_count(w.topk_idx, T, k, E, w.blk_counts, w.dst_row, s), "route_count");
     COLIBRI_TRY(launch_route_scan(w.blk_counts, nblk, E, bm, w.blk_base, w.counts, w.offsets, w.mt_prefix, s),
                 "route_scan");
-    COLIBRI_TRY(launch_route_scatter(xd, act, T, d, k, E, w.topk_idx, w.blk_base, w.dst_row, w.src_row, w.Xp, s),
-                "route_scatter");
+    COLIBRI_TRY(launch_route_scatter(xd, act, T, d, k, E, w.topk_idx, w.blk_base, w.dst_row, w.src_row, w.Xp,
+                                     planes, s), "route_scatter");
   }
   mark(2);
 
@@ -420,13 +430,11 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
              touched * tiles * gsplit < 8 * ctx->sm_count)
         gsplit <<= 1;
     }
-    COLIBRI_TRY(launch_dec_split((const __nv_bfloat16*)w.Xp, R, d, w.plane_hi, w.plane_lo, w.plane_scale, s),
-                "dec_split_x");
     COLIBRI_TRY(launch_dec_gateup(w.plane_hi, w.plane_lo, w.plane_scale, (const int8_t*)expert_w, expert_scales,
                                   stride, d, f, E, w.offsets, gsplit, (float*)w.H, R, T, w.err, s), "dec_gateup");
     mark(3);
-    COLIBRI_TRY(launch_dec_finish_h((const float*)w.H, gsplit, R, f, w.plane_hi, w.plane_lo, w.plane_scale, s),
-                "dec_finish_h");
+    COLIBRI_TRY(launch_dec_finish_h((const float*)w.H, gsplit, R, f, nsplit, w.plane_hi, w.plane_lo, w.plane_scale,
+                                    s), "dec_finish_h");
     COLIBRI_TRY(launch_dec_down(w.plane_hi, w.plane_lo, w.plane_scale, (const int8_t*)expert_w, expert_scales,
                                 stride, d, f, E, w.offsets, nsplit, R, w.Ypart, T, w.err, s), "dec_down");
   }

@@ -44,6 +44,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const Typ* __restrict__ Yp
                                                       const float* __restrict__ w, int T, int k,
                                                       int d, const Typ* __restrict__ Ys,
                                                       Tout* __restrict__ y) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int warps_total = gridDim.x * (blockDim.x >> 5);
   for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps_total) {
@@ -60,6 +62,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const Typ* __restrict__ Yp
       rows[j] = __shfl_sync(0xffffffffu, r, j);
       ws[j] = __shfl_sync(0xffffffffu, wj, j);
     }
+#pragma unroll 2
     for (int c = lane * 8; c < d; c += 32 * 8) {
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -83,40 +86,63 @@ __global__ void __launch_bounds__(256) combine_kernel(const Typ* __restrict__ Yp
 }
 
 // int8 path: the down projection leaves `nsplit` K-partial sums per grouped row.  One thread
-// per (token, 8 consecutive outputs): all k x nsplit partial loads of a thread are independent,
-// so a handful of tokens is one short latency, not a serial walk.
+// per (token, 4 consecutive outputs).  A slot's partials are loaded 8 at a time before they are
+// summed (in split order), so a handful of tokens costs a few memory round trips, not one per
+// partial.
+__device__ __forceinline__ float4 ld4(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
+__device__ __forceinline__ void add4(float4& a, const float4& b) {
+  a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+}
+__device__ __forceinline__ void store4(float* p, const float4& v) { *reinterpret_cast<float4*>(p) = v; }
+__device__ __forceinline__ void store4(__nv_bfloat16* p, const float4& v) {
+  const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+  uint2 q;
+  q.x = *reinterpret_cast<const uint32_t*>(&a);
+  q.y = *reinterpret_cast<const uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(p) = q;
+}
+
 template <typename Tout>
 __global__ void __launch_bounds__(256) combine_split_kernel(const float* __restrict__ Ypart,
                                                             int nsplit, int rows,
                                                             const int32_t* __restrict__ dst_row,
                                                             const float* __restrict__ w, int T,
                                                             int k, int d, Tout* __restrict__ y) {
-  const int chunks = d >> 3;
-  const size_t split_stride = (size_t)rows * d;
+  pdl_trigger();
+  pdl_wait();
+  const int chunks = d >> 2;
+  const size_t ss = (size_t)rows * d;
   for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < (long long)T * chunks;
        q += (long long)gridDim.x * blockDim.x) {
-    const int t = (int)(q / chunks), c = (int)(q - (long long)t * chunks) * 8;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const int t = (int)(q / chunks), c = (int)(q - (long long)t * chunks) * 4;
+    int rs[kMaxTopK];
+    float ws[kMaxTopK];
 #pragma unroll
     for (int j = 0; j < kMaxTopK; ++j) {
-      if (j < k) {
-        const int r = dst_row[(size_t)t * k + j];
-        const float wj = w[(size_t)t * k + j];
-        float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int sidx = 0; sidx < kDecSplitMax; ++sidx) {
-          if (sidx < nsplit) {
-            float v[8];
-            load8(Ypart + sidx * split_stride + (size_t)r * d + c, v);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) part[i] += v[i];
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = fmaf(wj, part[i], acc[i]);
-      }
+      rs[j] = j < k ? dst_row[(size_t)t * k + j] : 0;
+      ws[j] = j < k ? w[(size_t)t * k + j] : 0.f;
     }
-    store8(y + (size_t)t * d + c, acc);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      if (j >= k) break;
+      const float* base = Ypart + (size_t)rs[j] * d + c;
+      float4 part = make_float4(0.f, 0.f, 0.f, 0.f);
+      int sp = 0;
+      for (; sp + 8 <= nsplit; sp += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = ld4(base + (size_t)(sp + i) * ss);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) add4(part, v[i]);
+      }
+      for (; sp < nsplit; ++sp) add4(part, ld4(base + (size_t)sp * ss));
+      acc.x = fmaf(ws[j], part.x, acc.x);
+      acc.y = fmaf(ws[j], part.y, acc.y);
+      acc.z = fmaf(ws[j], part.z, acc.z);
+      acc.w = fmaf(ws[j], part.w, acc.w);
+    }
+    store4(y + (size_t)t * d + c, acc);
   }
 }
 
@@ -130,24 +156,22 @@ int grid_for_tokens(int T) {
 cudaError_t launch_combine(const void* Yp, int yp_dtype, const int32_t* dst_row, const float* w,
                            int T, int k, int d, const void* Ys, void* y, int act, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  const int grid = grid_for_tokens(T);
+  const dim3 grid(grid_for_tokens(T)), block(256);
   if (yp_dtype == COLIBRI_BF16) {
+    const __nv_bfloat16* yp = (const __nv_bfloat16*)Yp;
+    const __nv_bfloat16* ys = (const __nv_bfloat16*)Ys;
     if (act == COLIBRI_BF16)
-      combine_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, 256, 0, s>>>(
-          (const __nv_bfloat16*)Yp, dst_row, w, T, k, d, (const __nv_bfloat16*)Ys,
-          (__nv_bfloat16*)y);
-    else
-      combine_kernel<float, __nv_bfloat16><<<grid, 256, 0, s>>>(
-          (const __nv_bfloat16*)Yp, dst_row, w, T, k, d, (const __nv_bfloat16*)Ys, (float*)y);
-  } else {
-    if (act == COLIBRI_BF16)
-      combine_kernel<__nv_bfloat16, float><<<grid, 256, 0, s>>>(
-          (const float*)Yp, dst_row, w, T, k, d, (const float*)Ys, (__nv_bfloat16*)y);
-    else
-      combine_kernel<float, float><<<grid, 256, 0, s>>>((const float*)Yp, dst_row, w, T, k, d,
-                                                        (const float*)Ys, (float*)y);
+      return launch_kernel(combine_kernel<__nv_bfloat16, __nv_bfloat16>, grid, block, 0, s, 1, yp, dst_row, w, T, k,
+                           d, ys, (__nv_bfloat16*)y);
+    return launch_kernel(combine_kernel<float, __nv_bfloat16>, grid, block, 0, s, 1, yp, dst_row, w, T, k, d, ys,
+                         (float*)y);
   }
-  return cudaGetLastError();
+  const float* yp = (const float*)Yp;
+  const float* ys = (const float*)Ys;
+  if (act == COLIBRI_BF16)
+    return launch_kernel(combine_kernel<__nv_bfloat16, float>, grid, block, 0, s, 1, yp, dst_row, w, T, k, d, ys,
+                         (__nv_bfloat16*)y);
+  return launch_kernel(combine_kernel<float, float>, grid, block, 0, s, 1, yp, dst_row, w, T, k, d, ys, (float*)y);
 }
 
 cudaError_t launch_combine_split(const float* Ypart, int nsplit, int rows, const int32_t* dst_row,
@@ -155,15 +179,13 @@ cudaError_t launch_combine_split(const float* Ypart, int nsplit, int rows, const
                                  cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
   if (nsplit > kDecSplitMax) return cudaErrorInvalidValue;
-  long long threads = (long long)T * (d / 8);
-  int grid = (int)std::min<long long>((threads + 255) / 256, 8192);
+  long long threads = (long long)T * (d / 4);
+  const dim3 grid((unsigned)std::min<long long>((threads + 255) / 256, 8192)), block(256);
   if (act == COLIBRI_BF16)
-    combine_split_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(Ypart, nsplit, rows, dst_row, w, T, k,
-                                                             d, (__nv_bfloat16*)y);
-  else
-    combine_split_kernel<float><<<grid, 256, 0, s>>>(Ypart, nsplit, rows, dst_row, w, T, k, d,
-                                                     (float*)y);
-  return cudaGetLastError();
+    return launch_kernel(combine_split_kernel<__nv_bfloat16>, grid, block, 0, s, 1, Ypart, nsplit, rows, dst_row, w,
+                         T, k, d, (__nv_bfloat16*)y);
+  return launch_kernel(combine_split_kernel<float>, grid, block, 0, s, 1, Ypart, nsplit, rows, dst_row, w, T, k, d,
+                       (float*)y);
 }
 
 }  // namespace colibri

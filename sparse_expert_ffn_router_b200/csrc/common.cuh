@@ -112,9 +112,68 @@ struct colibri_ctx {
   std::vector<GraphEntry> graphs;
   uint64_t graph_clock = 0;
   bool use_graphs = true;
+  bool use_pdl = true;  // programmatic dependent launch between the kernels of a forward
 };
 
 namespace colibri {
+
+// ---------------------------------------------------------------------------------------
+// Launches.  Every kernel goes through launch_kernel().  Inside a LaunchScope that enables it,
+// each launch after the first of the scope uses programmatic dependent launch: its CTAs may be
+// scheduled while the previous kernel still runs, so they do their set-up (barriers, TMEM,
+// descriptor prefetch) in its shadow.  Every kernel therefore calls pdl_wait() before it reads
+// anything an earlier launch wrote, on every path (so that a kernel never completes before its
+// predecessor), and pdl_trigger() to let its successor be scheduled; both are no-ops for a
+// launch without the attribute.  A copy or memset between two launches breaks the chain
+// (launch_chain_break): the launch after it is an ordinary one.
+// ---------------------------------------------------------------------------------------
+namespace detail {
+inline thread_local bool tl_pdl = false;   // launches of the current scope may overlap
+inline thread_local int tl_chain = 0;      // launches since the scope began or the chain broke
+}  // namespace detail
+struct LaunchScope {
+  explicit LaunchScope(bool pdl) {
+    detail::tl_pdl = pdl;
+    detail::tl_chain = 0;
+  }
+  ~LaunchScope() {
+    detail::tl_pdl = false;
+    detail::tl_chain = 0;
+  }
+};
+inline void launch_chain_break() { detail::tl_chain = 0; }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                          unsigned cluster_x, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (detail::tl_pdl && detail::tl_chain > 0) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  ++detail::tl_chain;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------------------
 // Kernel launchers (each returns cudaGetLastError() of its launch)
@@ -133,13 +192,21 @@ cudaError_t launch_route_count(const int32_t* idx, int T, int k, int E, int32_t*
                                int32_t* local_rank, cudaStream_t s);
 cudaError_t launch_route_scan(const int32_t* blk_counts, int nblk, int E, int bm, int32_t* blk_base,
                               int32_t* counts, int32_t* offsets, int32_t* mt_prefix, cudaStream_t s);
+// Grouped rows go to Xp (a copy of the token row), or -- when `planes` is given (bf16 input,
+// int8 weights) -- to the int8 planes of the token row instead: planes->hi/lo [R, d] and the
+// per-row scale planes->scale [R] (x ~= scale * (hi + lo / 254)); Xp is then not written.
+struct RowPlanes {
+  int8_t* hi;
+  int8_t* lo;
+  float* scale;
+};
 cudaError_t launch_route_scatter(const void* x, int act, int T, int d, int k, int E,
                                  const int32_t* idx, const int32_t* blk_base, int32_t* dst_row,
-                                 int32_t* src_row, void* Xp, cudaStream_t s);
-// T <= kFusedRouteThreads: count + scan + scatter in one single-CTA launch
+                                 int32_t* src_row, void* Xp, const RowPlanes* planes, cudaStream_t s);
+// T <= kFusedRouteMaxT: count + scan + scatter in one single-CTA launch
 cudaError_t launch_route_fused(const void* x, int act, int T, int d, const int32_t* idx, int k, int E, int bm,
                                int32_t* counts, int32_t* offsets, int32_t* mt_prefix, int32_t* src_row,
-                               int32_t* dst_row, void* Xp, cudaStream_t s);
+                               int32_t* dst_row, void* Xp, const RowPlanes* planes, cudaStream_t s);
 cudaError_t launch_combine(const void* Yp, int yp_dtype, const int32_t* dst_row, const float* w,
                            int T, int k, int d, const void* Ys, void* y, int act, cudaStream_t s);
 cudaError_t launch_combine_split(const float* Ypart, int nsplit, int rows, const int32_t* dst_row,
@@ -194,19 +261,17 @@ cudaError_t configure_router_kernels();  // once per device, before any launch
 cudaError_t launch_tc_gateup(const TcGemmArgs& a, cudaStream_t s);
 cudaError_t launch_tc_down(const TcGemmArgs& a, cudaStream_t s);
 
-// int8 weight-streaming decode path, see decode_i8.cu
-// Split bf16 rows into two int8 planes with a per-row scale: x ~= a * (hi + lo / 254).
-cudaError_t launch_dec_split(const __nv_bfloat16* X, int R, int K, int8_t* hi, int8_t* lo, float* scale,
-                             cudaStream_t s);
+// int8 weight-streaming decode path, see decode_i8.cu (the x planes come from the scatter)
 // max_rows_per_expert: an upper bound (T) that picks the token chunk (8, 16 or 32 rows).
 cudaError_t configure_dec_kernels();  // once per device, before any launch
 // gate/up: W1 . x and W3 . x (scaled) as fp32 K-split partials GU [nsplit, 2, R, f]
 cudaError_t launch_dec_gateup(const int8_t* Xhi, const int8_t* Xlo, const float* xscale, const int8_t* W,
                               const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
                               int nsplit, float* GU, int R, int max_rows_per_expert, uint32_t* err, cudaStream_t s);
-// H = silu(sum g) * (sum u) (bf16) from GU, split into int8 planes
-cudaError_t launch_dec_finish_h(const float* GU, int nsplit, int R, int f, int8_t* hi, int8_t* lo, float* scale,
-                                cudaStream_t s);
+// H = silu(sum g) * (sum u) (bf16) from the gsplit partials GU, split into int8 planes with one
+// scale per (down K split, row): scale[ds * R + r] covers H[r][ds * f / dsplit, (ds + 1) * f / dsplit).
+cudaError_t launch_dec_finish_h(const float* GU, int gsplit, int R, int f, int dsplit, int8_t* hi, int8_t* lo,
+                                float* scale, cudaStream_t s);
 cudaError_t launch_dec_down(const int8_t* Hhi, const int8_t* Hlo, const float* hscale, const int8_t* W,
                             const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
                             int nsplit, int R, float* Ypart, int max_rows_per_expert, uint32_t* err,
@@ -216,6 +281,17 @@ cudaError_t launch_dec_down(const int8_t* Hhi, const int8_t* Hlo, const float* h
 // Small device helpers
 // ---------------------------------------------------------------------------------------
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+
+// Two int8 planes of a value, given the row scale a and 1/a: hi = rint(x / a), lo = rint((x - a hi)
+// * 254 / a), both clamped to [-127, 127], so that x ~= a * (hi + lo / 254).
+__device__ __forceinline__ void split_planes(float x, float a, float inv_a, int& qh, int& ql) {
+  const float h = fminf(fmaxf(rintf(x * inv_a), -127.f), 127.f);
+  const float l = fminf(fmaxf(rintf(fmaf(-a, h, x) * inv_a * 254.f), -127.f), 127.f);
+  qh = (int)h;
+  ql = (int)l;
+}
+// Plane scale of a row from its largest magnitude (an all-zero row gets 1).
+__device__ __forceinline__ float plane_scale(float maxabs) { return maxabs > 0.f ? maxabs / 127.f : 1.f; }
 
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }

@@ -7,10 +7,12 @@
 //   down:     Yp_s[r][o] = s2[o] * sum_{i in split s} q2[o][i] H[r][i]
 //
 // W[o][i] = s[o] q[o][i], so the weight scale factors out of each dot product exactly.  The
-// weights are never converted: each activation row (bf16) is first split, once, into two int8
-// planes with a per-row scale, x ~= a * (hi + lo / 254) with a = max|x| / 127 (the residual
-// after hi is at most a/2, so lo fits in [-127, 127]; the representation error is at most
-// a / 508 = max|x| / 64516 per element, far below bf16's own rounding of the result).  The dot
+// weights are never converted: each activation row (bf16) is split, once, into two int8 planes
+// with a scale, x ~= a * (hi + lo / 254) with a = max|x| / 127 (the residual after hi is at most
+// a/2, so lo fits in [-127, 127]; the representation error is at most a / 508 = max|x| / 64516
+// per element, far below bf16's own rounding of the result).  The token rows x are split by the
+// scatter as they are grouped (one scale per row); H is split by dec_finish_h with one scale
+// per (row, K range of one down-projection split), the range that one accumulator covers.  The dot
 // products then run on the 5th-generation tensor cores as kind::i8 MMAs with exact int32
 // accumulation in TMEM: A = 128 weight rows (output channels) x 128 K bytes, B = the hi plane
 // rows of up to 32 tokens stacked on their lo plane rows (N = 2 x tokens), so one MMA yields
@@ -31,70 +33,45 @@
 namespace colibri {
 namespace {
 
-// One warp per row: a = max|x| / 127, hi = rint(x / a), lo = rint((x - a * hi) * 254 / a).
-__global__ void __launch_bounds__(256) dec_split_rows_kernel(const __nv_bfloat16* __restrict__ X, int R, int K,
-                                                             int8_t* __restrict__ hi, int8_t* __restrict__ lo,
-                                                             float* __restrict__ scale) {
-  const int lane = threadIdx.x & 31;
-  const int nw = gridDim.x * (blockDim.x >> 5);
-  for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < R; r += nw) {
-    const uint4* src = reinterpret_cast<const uint4*>(X + (size_t)r * K);
-    float mx = 0.f;
-    for (int v = lane; v < K / 8; v += 32) {
-      const uint4 q = src[v];
-      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f2 = __bfloat1622float2(h[i]);
-        mx = fmaxf(mx, fmaxf(fabsf(f2.x), fabsf(f2.y)));
-      }
-    }
-#pragma unroll
-    for (int off = 16; off; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    const float a = mx > 0.f ? mx / 127.f : 1.f;
-    const float inv_a = 1.f / a;
-    if (lane == 0) scale[r] = a;
-    for (int v = lane; v < K / 8; v += 32) {
-      const uint4 q = src[v];
-      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
-      uint32_t hw[2] = {0u, 0u}, lw[2] = {0u, 0u};
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float xv = __bfloat162float(i & 1 ? h[i >> 1].y : h[i >> 1].x);
-        const float qh = fminf(fmaxf(rintf(xv * inv_a), -127.f), 127.f);
-        const float res = fmaf(-a, qh, xv);
-        const float ql = fminf(fmaxf(rintf(res * inv_a * 254.f), -127.f), 127.f);
-        hw[i >> 2] |= ((uint32_t)((int)qh) & 0xffu) << (8 * (i & 3));
-        lw[i >> 2] |= ((uint32_t)((int)ql) & 0xffu) << (8 * (i & 3));
-      }
-      reinterpret_cast<uint2*>(hi + (size_t)r * K)[v] = make_uint2(hw[0], hw[1]);
-      reinterpret_cast<uint2*>(lo + (size_t)r * K)[v] = make_uint2(lw[0], lw[1]);
-    }
-  }
-}
-
-// h = silu(g) * u from the gate/up partials, rounded to bf16 (as the bf16 path stores H), then
-// split into int8 planes like dec_split_rows.  One CTA per row; the row is kept in shared memory.
+// h = silu(g) * u from the gate/up partials (summed in split order), rounded to bf16 as the bf16
+// path stores H, then split into int8 planes.  One CTA per (row, K range of one down split): the
+// down projection accumulates each split separately, so each split may carry its own plane
+// scale and no reduction crosses CTAs.  The range's bf16 values wait in shared memory between
+// the max and the split.
 constexpr int kFinishThreads = 256;
 constexpr int kFinishMaxSmem = 2 * kDecMaxFF;  // one bf16 row of H
-__global__ void __launch_bounds__(kFinishThreads) dec_finish_h_kernel(const float* __restrict__ GU, int nsplit, int R,
-                                                                      int f, int8_t* __restrict__ hi,
+__global__ void __launch_bounds__(kFinishThreads) dec_finish_h_kernel(const float* __restrict__ GU, int gsplit, int R,
+                                                                      int f, int dsplit, int8_t* __restrict__ hi,
                                                                       int8_t* __restrict__ lo,
                                                                       float* __restrict__ scale) {
-  extern __shared__ __nv_bfloat16 hrow[];  // [f]
+  pdl_trigger();
+  pdl_wait();
+  extern __shared__ __align__(16) uint8_t hseg_raw[];  // [span] bf16
+  __nv_bfloat16* hseg = reinterpret_cast<__nv_bfloat16*>(hseg_raw);
   __shared__ float red[kFinishThreads / 32];
-  const int r = blockIdx.x;
+  const int r = blockIdx.x / dsplit, ds = blockIdx.x - r * dsplit;
+  const int span = f / dsplit, k0 = ds * span;
   const size_t plane = (size_t)R * f;
+  const float* g0 = GU + (size_t)r * f + k0;
   float mx = 0.f;
-  for (int j = threadIdx.x; j < f; j += kFinishThreads) {
-    float g = 0.f, u = 0.f;
-    for (int sp = 0; sp < nsplit; ++sp) {  // K-split partials, summed in split order
-      g += GU[(2 * sp) * plane + (size_t)r * f + j];
-      u += GU[(2 * sp + 1) * plane + (size_t)r * f + j];
+  for (int j = threadIdx.x * 4; j < span; j += kFinishThreads * 4) {
+    float4 g = __ldg(reinterpret_cast<const float4*>(g0 + j));
+    float4 u = __ldg(reinterpret_cast<const float4*>(g0 + plane + j));
+#pragma unroll 3
+    for (int sp = 1; sp < gsplit; ++sp) {
+      const float4 gs = __ldg(reinterpret_cast<const float4*>(g0 + (size_t)(2 * sp) * plane + j));
+      const float4 us = __ldg(reinterpret_cast<const float4*>(g0 + (size_t)(2 * sp + 1) * plane + j));
+      g.x += gs.x; g.y += gs.y; g.z += gs.z; g.w += gs.w;
+      u.x += us.x; u.y += us.y; u.z += us.z; u.w += us.w;
     }
-    const __nv_bfloat16 h = __float2bfloat16_rn(silu_mul(g, u));
-    hrow[j] = h;
-    mx = fmaxf(mx, fabsf(__bfloat162float(h)));
+    const __nv_bfloat162 h01 = __floats2bfloat162_rn(silu_mul(g.x, u.x), silu_mul(g.y, u.y));
+    const __nv_bfloat162 h23 = __floats2bfloat162_rn(silu_mul(g.z, u.z), silu_mul(g.w, u.w));
+    uint2 pk;
+    pk.x = (uint32_t)__bfloat16_as_ushort(h01.x) | ((uint32_t)__bfloat16_as_ushort(h01.y) << 16);
+    pk.y = (uint32_t)__bfloat16_as_ushort(h23.x) | ((uint32_t)__bfloat16_as_ushort(h23.y) << 16);
+    *reinterpret_cast<uint2*>(hseg + j) = pk;
+    const float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
+    mx = fmaxf(mx, fmaxf(fmaxf(fabsf(f01.x), fabsf(f01.y)), fmaxf(fabsf(f23.x), fabsf(f23.y))));
   }
 #pragma unroll
   for (int off = 16; off; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
@@ -103,16 +80,27 @@ __global__ void __launch_bounds__(kFinishThreads) dec_finish_h_kernel(const floa
   mx = 0.f;
 #pragma unroll
   for (int w = 0; w < kFinishThreads / 32; ++w) mx = fmaxf(mx, red[w]);
-  const float a = mx > 0.f ? mx / 127.f : 1.f;
-  const float inv_a = 1.f / a;
-  if (threadIdx.x == 0) scale[r] = a;
-  for (int j = threadIdx.x; j < f; j += kFinishThreads) {
-    const float xv = __bfloat162float(hrow[j]);
-    const float qh = fminf(fmaxf(rintf(xv * inv_a), -127.f), 127.f);
-    const float res = fmaf(-a, qh, xv);
-    const float ql = fminf(fmaxf(rintf(res * inv_a * 254.f), -127.f), 127.f);
-    hi[(size_t)r * f + j] = (int8_t)qh;
-    lo[(size_t)r * f + j] = (int8_t)ql;
+  const float a = plane_scale(mx), inv_a = __frcp_rn(a);  // correctly rounded 1 / a
+  if (threadIdx.x == 0) scale[(size_t)ds * R + r] = a;
+  int8_t* hrow = hi + (size_t)r * f + k0;
+  int8_t* lrow = lo + (size_t)r * f + k0;
+  for (int j = threadIdx.x * 4; j < span; j += kFinishThreads * 4) {
+    const uint2 pk = *reinterpret_cast<const uint2*>(hseg + j);
+    const float2 f01 = make_float2(__bfloat162float(__ushort_as_bfloat16((unsigned short)(pk.x & 0xffffu))),
+                                   __bfloat162float(__ushort_as_bfloat16((unsigned short)(pk.x >> 16))));
+    const float2 f23 = make_float2(__bfloat162float(__ushort_as_bfloat16((unsigned short)(pk.y & 0xffffu))),
+                                   __bfloat162float(__ushort_as_bfloat16((unsigned short)(pk.y >> 16))));
+    int qh0, ql0, qh1, ql1, qh2, ql2, qh3, ql3;
+    split_planes(f01.x, a, inv_a, qh0, ql0);
+    split_planes(f01.y, a, inv_a, qh1, ql1);
+    split_planes(f23.x, a, inv_a, qh2, ql2);
+    split_planes(f23.y, a, inv_a, qh3, ql3);
+    const uint32_t hw = ((uint32_t)qh0 & 0xffu) | (((uint32_t)qh1 & 0xffu) << 8) | (((uint32_t)qh2 & 0xffu) << 16) |
+                        ((uint32_t)qh3 << 24);
+    const uint32_t lw = ((uint32_t)ql0 & 0xffu) | (((uint32_t)ql1 & 0xffu) << 8) | (((uint32_t)ql2 & 0xffu) << 16) |
+                        ((uint32_t)ql3 << 24);
+    *reinterpret_cast<uint32_t*>(hrow + j) = hw;
+    *reinterpret_cast<uint32_t*>(lrow + j) = lw;
   }
 }
 
@@ -127,7 +115,8 @@ struct alignas(64) DecStreamParams {
   CUtensorMap mapHi;  // int8 activation planes {K, R}
   CUtensorMap mapLo;
   const float* wscale;      // expert scales base (per expert: s1[f] | s3[f] | s2[d])
-  const float* rscale;      // plane row scales [R]
+  const float* rscale;      // plane scales: rscale[split * rscale_split_stride + row]
+  int rscale_split_stride;  // 0: one scale per row (x planes); R: one per (K split, row) (H planes)
   const int32_t* offsets;   // [E+1]
   int E, d, f;
   int out_rows;             // f (gate/up) or d (down)
@@ -195,6 +184,7 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_stream_kernel(const __grid_
   constexpr int NMAT = 1;  // one weight tile per item (W1 and W3 tiles of gate/up are separate items)
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {
+    pdl_wait();
     if (threadIdx.x == 0) atomicOr(p.err, kErrWaitTimeout);
     return;
   }
@@ -230,6 +220,17 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_stream_kernel(const __grid_
     tma_prefetch_desc(&p.mapW);
     tma_prefetch_desc(&p.mapHi);
     tma_prefetch_desc(&p.mapLo);
+  }
+  // Everything below may read what earlier kernels wrote.  TMEM is allocated only after the
+  // wait too: the previous kernel has then released its own columns, so two kernels of the
+  // chain never hold TMEM on one SM at the same time.
+  pdl_wait();
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, kDsTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (threadIdx.x == 0) {
     // touched experts and the prefix of their work items
     const int tiles = (p.out_rows + 127) / 128;
     int n = 0, acc = 0;
@@ -243,11 +244,6 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_stream_kernel(const __grid_
     }
     item_prefix[n] = acc;
     *ntouched_s = n;
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_holder, kDsTmemCols);
-    tmem_relinquish();
-    tc_fence_before();
   }
   __syncthreads();
   tc_fence_after();
@@ -266,8 +262,15 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_stream_kernel(const __grid_
       bool ok = true;
       DecItem it;
       for (int L = blockIdx.x; ok && dec_item<kGateUp>(p, touched, item_prefix, ntouched, L, it); L += gridDim.x) {
+        // The item's K blocks start at a rotated block (item index mod block count): items in
+        // flight at the same time then read different column offsets of their weight rows, which
+        // spreads the requests over the DRAM channels instead of hitting the same address bits
+        // everywhere.  The accumulation is exact int32, so the block order does not matter.
         const int kbeg = it.split * p.kspan, kend = min(p.K, kbeg + p.kspan);
-        for (int kx = kbeg; kx < kend; kx += 128) {
+        const int nkb = (kend - kbeg + 127) / 128;
+        int kb = L % nkb;
+        for (int i = 0; i < nkb; ++i, kb = (kb + 1 == nkb) ? 0 : kb + 1) {
+          const int kx = kbeg + kb * 128;
           if (!ds_wait(&empty[s], ph ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -292,6 +295,7 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_stream_kernel(const __grid_
       }
       *issued_s = issued;
     }
+    pdl_trigger();  // every copy of this CTA is issued: let the next kernel be scheduled
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
@@ -397,7 +401,8 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_stream_kernel(const __grid_
           const int t = j + i;
           if (i >= width || t >= it.ntok || !vo) continue;
           const int row = it.row0 + t;
-          const float v = sc * p.rscale[row] * (hi[0][i] + lo[0][i] * (1.0f / 254.0f));
+          const float v = sc * p.rscale[(size_t)it.split * p.rscale_split_stride + row] *
+                          (hi[0][i] + lo[0][i] * (1.0f / 254.0f));
           if (kGateUp) p.GU[(((size_t)it.split * 2 + it.mat) * p.R + row) * p.f + o] = v;
           else p.Ypart[((size_t)it.split * p.R + row) * p.d + o] = v;
         }
@@ -442,19 +447,10 @@ cudaError_t launch_stream(DecStreamParams& p, const int8_t* hi, const int8_t* lo
   p.stage_bytes = (uint32_t)(NMAT * 128 * 128 + 2 * p.nt8 * 128);
   p.stages = (int)std::min<size_t>(kDsMaxStages, kDsRingBytes / p.stage_bytes);
   const size_t smem = (size_t)p.stages * p.stage_bytes + 4096;
-  dec_stream_kernel<kGateUp><<<sm_count_current(), kDsThreads, smem, s>>>(p);
-  return cudaGetLastError();
+  return launch_kernel(dec_stream_kernel<kGateUp>, dim3(sm_count_current()), dim3(kDsThreads), smem, s, 1, p);
 }
 
 }  // namespace
-
-cudaError_t launch_dec_split(const __nv_bfloat16* X, int R, int K, int8_t* hi, int8_t* lo, float* scale,
-                             cudaStream_t s) {
-  if (R <= 0) return cudaSuccess;
-  const int grid = std::min((R + 7) / 8, 4096);
-  dec_split_rows_kernel<<<grid, 256, 0, s>>>(X, R, K, hi, lo, scale);
-  return cudaGetLastError();
-}
 
 cudaError_t configure_dec_kernels() {
   const int smem = (int)(kDsRingBytes + 4096);
@@ -492,13 +488,14 @@ cudaError_t launch_dec_gateup(const int8_t* Xhi, const int8_t* Xlo, const float*
   return launch_stream<true>(p, Xhi, Xlo, d, s);
 }
 
-cudaError_t launch_dec_finish_h(const float* GU, int nsplit, int R, int f, int8_t* hi, int8_t* lo, float* scale,
-                                cudaStream_t s) {
+cudaError_t launch_dec_finish_h(const float* GU, int gsplit, int R, int f, int dsplit, int8_t* hi, int8_t* lo,
+                                float* scale, cudaStream_t s) {
   if (R <= 0) return cudaSuccess;
-  const size_t smem = (size_t)f * sizeof(__nv_bfloat16);
+  if (dsplit < 1 || f % dsplit != 0 || (f / dsplit) % 4 != 0) return cudaErrorInvalidValue;
+  const size_t smem = (size_t)(f / dsplit) * sizeof(__nv_bfloat16);
   if (smem > (size_t)kFinishMaxSmem) return cudaErrorInvalidValue;
-  dec_finish_h_kernel<<<R, kFinishThreads, smem, s>>>(GU, nsplit, R, f, hi, lo, scale);
-  return cudaGetLastError();
+  return launch_kernel(dec_finish_h_kernel, dim3((unsigned)((size_t)R * dsplit)), dim3(kFinishThreads), smem, s, 1, GU,
+                       gsplit, R, f, dsplit, hi, lo, scale);
 }
 
 cudaError_t launch_dec_down(const int8_t* Hhi, const int8_t* Hlo, const float* hscale, const int8_t* W,
@@ -514,6 +511,7 @@ cudaError_t launch_dec_down(const int8_t* Hhi, const int8_t* Hlo, const float* h
     return cudaErrorInvalidValue;
   p.wscale = scales;
   p.rscale = hscale;
+  p.rscale_split_stride = R;
   p.offsets = offsets;
   p.E = E;
   p.d = d;

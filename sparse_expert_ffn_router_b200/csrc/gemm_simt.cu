@@ -43,6 +43,8 @@ __global__ void __launch_bounds__(256) simt_ffn_kernel(const float* __restrict__
                                                        int64_t wstride, int d, int f,
                                                        SimtGroups groups,
                                                        float* __restrict__ out, int ldo, int N) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ __align__(16) float As[BK][BM + 4];
   __shared__ __align__(16) float Bs[BK][BN + 4];
   __shared__ __align__(16) float Cs[kGateUp ? BK : 1][BN + 4];
@@ -115,16 +117,14 @@ cudaError_t launch_simt_gateup(const float* A, int lda, const float* W, int64_t 
                                int f, SimtGroups g, int mt_bound, float* H, cudaStream_t s) {
   if (mt_bound <= 0) return cudaSuccess;
   const dim3 grid((f + BN - 1) / BN, mt_bound);
-  simt_ffn_kernel<true><<<grid, 256, 0, s>>>(A, lda, d, W, wstride, d, f, g, H, f, f);
-  return cudaGetLastError();
+  return launch_kernel(simt_ffn_kernel<true>, grid, dim3(256), 0, s, 1, A, lda, d, W, wstride, d, f, g, H, f, f);
 }
 
 cudaError_t launch_simt_down(const float* H, int f, const float* W, int64_t wstride, int d,
                              SimtGroups g, int mt_bound, float* Y, cudaStream_t s) {
   if (mt_bound <= 0) return cudaSuccess;
   const dim3 grid((d + BN - 1) / BN, mt_bound);
-  simt_ffn_kernel<false><<<grid, 256, 0, s>>>(H, f, f, W, wstride, d, f, g, Y, d, d);
-  return cudaGetLastError();
+  return launch_kernel(simt_ffn_kernel<false>, grid, dim3(256), 0, s, 1, H, f, f, W, wstride, d, f, g, Y, d, d);
 }
 
 }  // namespace colibri

@@ -23,7 +23,8 @@
 //               releases the accumulator so the next tile's MMAs overlap this epilogue.
 // Tiles are walked round-robin over a schedule built on the device from the per-expert row
 // offsets: expert-major, then n-tile, then m-tile fastest, so the CTAs running at one time
-// share the same weight tile through L2 and each weight byte leaves HBM about once.
+// share the same weight tile through L2 and each weight byte leaves HBM about once; tiles of
+// experts with a single m-tile (weight streaming) are interleaved with the others.
 // Every wait is bounded (kWaitTimeoutNs); a wait that gives up sets the error word, makes the
 // other roles leave their loops, drains outstanding copies and MMAs and frees TMEM.
 #include "common.cuh"
@@ -70,6 +71,8 @@ struct SmemMisc {
   int mt_total;
   int32_t mt[kMaxExperts + 1];
   int32_t off[kMaxExperts + 1];
+  int32_t hv[kMaxExperts + 1];  // m-tile prefix over experts with >= 2 m-tiles (compute-bound tiles)
+  int32_t lt[kMaxExperts + 1];  // prefix over experts with exactly 1 m-tile (weight-streaming tiles)
 };
 
 constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + (size_t)STAGES * STAGE_BYTES + sizeof(SmemMisc);
@@ -79,21 +82,76 @@ struct Tile {
   int e, row0, row_end, n0, num_kb;
 };
 
+// Routed tiles come in two classes.  An expert with two or more m-tiles reuses each weight tile
+// across its m-tiles (compute-bound); an expert with a single m-tile streams its weights once
+// (bound by HBM).  When both classes exist (skewed routing) their tiles are interleaved in
+// proportion, so that at any time some CTAs compute while others stream weights, instead of a
+// compute-bound phase followed by a bandwidth-bound one.  Within a class the order is
+// expert-major, then n-tile, then m-tile fastest (CTAs running together share a weight tile).
+template <typename Misc>
+__device__ void build_class_prefix(Misc& m, int E) {  // one full warp
+  const int lane = threadIdx.x & 31;
+  const int C = (E + 31) / 32;
+  const int e0 = min(E, lane * C), e1 = min(E, e0 + C);
+  int sh = 0, sl = 0;
+  for (int e = e0; e < e1; ++e) {
+    const int Me = m.mt[e + 1] - m.mt[e];
+    sh += Me >= 2 ? Me : 0;
+    sl += Me == 1 ? 1 : 0;
+  }
+  int ih = sh, il = sl;  // inclusive warp prefix
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int a = __shfl_up_sync(0xffffffffu, ih, o), b = __shfl_up_sync(0xffffffffu, il, o);
+    if (lane >= o) {
+      ih += a;
+      il += b;
+    }
+  }
+  int ph = ih - sh, pl = il - sl;
+  for (int e = e0; e < e1; ++e) {
+    m.hv[e] = ph;
+    m.lt[e] = pl;
+    const int Me = m.mt[e + 1] - m.mt[e];
+    ph += Me >= 2 ? Me : 0;
+    pl += Me == 1 ? 1 : 0;
+  }
+  if (lane == 31) {
+    m.hv[E] = ih;
+    m.lt[E] = il;
+  }
+}
+
+// largest e in [0, E) with pre[e] * n_tiles <= L
+__device__ __forceinline__ int find_group(const int32_t* pre, int E, int n_tiles, int L) {
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pre[mid] * n_tiles <= L) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
 template <typename Misc>
 __device__ __forceinline__ Tile decode_tile(const TcParams& p, const Misc& m, int L, int routed_total,
                                             bool gateup, int bm = BM) {
   Tile t;
   const int ncols = gateup ? BN / 2 : BN;
   if (L < routed_total) {
-    // largest e with mt[e] * n_tiles <= L
-    int lo = 0, hi = p.E - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (m.mt[mid] * p.n_tiles <= L) lo = mid;
-      else hi = mid - 1;
+    const int nA = m.hv[p.E] * p.n_tiles, nB = m.lt[p.E] * p.n_tiles;
+    const int32_t* pre = m.mt;
+    int idx = L;
+    if (nA > 0 && nB > 0) {
+      const long long tot = (long long)nA + nB;
+      const int b = (int)((long long)L * nB / tot);
+      const bool light = (int)((long long)(L + 1) * nB / tot) > b;
+      pre = light ? m.lt : m.hv;
+      idx = light ? b : L - b;
     }
+    const int lo = find_group(pre, p.E, p.n_tiles, idx);
     const int Me = m.mt[lo + 1] - m.mt[lo];
-    const int Lp = L - m.mt[lo] * p.n_tiles;
+    const int Lp = idx - pre[lo] * p.n_tiles;
     const int n = Lp / Me, mm = Lp - n * Me;
     t.sh = false;
     t.e = lo;
@@ -170,6 +228,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ffn_kernel(const __grid_con
       tma_prefetch_desc(&p.mapB_sh);
     }
   }
+  pdl_wait();  // below: reads of earlier kernels' output; TMEM once the previous kernel released its own
   if (warp == 1) {
     tmem_alloc(&m.tmem_base, TMEM_COLS);
     tmem_relinquish();
@@ -179,6 +238,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ffn_kernel(const __grid_con
     m.mt[i] = p.mt_prefix[i];
     m.off[i] = p.offsets[i];
   }
+  __syncthreads();
+  if (warp == 0) build_class_prefix(m, p.E);
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = m.tmem_base;
@@ -231,6 +292,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ffn_kernel(const __grid_con
       }
       m.issued = issued;
     }
+    pdl_trigger();  // every copy of this CTA is issued: let the next kernel be scheduled
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
@@ -374,6 +436,8 @@ struct SmemMisc2 {
   int abort;
   int32_t mt[kMaxExperts + 1];
   int32_t off[kMaxExperts + 1];
+  int32_t hv[kMaxExperts + 1];
+  int32_t lt[kMaxExperts + 1];
 };
 
 constexpr size_t SMEM2_BYTES = (size_t)STAGES2 * STAGE2_BYTES + sizeof(SmemMisc2);
@@ -385,6 +449,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
   // The 128-byte swizzle needs 1024-byte aligned stages; the dynamic shared window of a CTA
   // starts 1024-byte aligned (both CTAs of a pair take this branch together).
   if (smem_u32(smem_raw) & 1023u) {
+    pdl_wait();
     if (threadIdx.x == 0) atomicOr(p.err, kErrWaitTimeout);
     return;
   }
@@ -415,6 +480,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
       tma_prefetch_desc(&p.mapB_sh);
     }
   }
+  pdl_wait();  // below: reads of earlier kernels' output; TMEM once the previous kernel released its own
   if (warp == 1) {
     tmem_alloc_pair(&m.tmem_base, TMEM_COLS);
     tmem_relinquish_pair();
@@ -424,6 +490,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
     m.mt[i] = p.mt_prefix[i];
     m.off[i] = p.offsets[i];
   }
+  __syncthreads();
+  if (warp == 0) build_class_prefix(m, p.E);
   __syncthreads();
   cluster_sync_all();  // the peer's barriers are initialised before any cross-CTA arrival
   tc_fence_after();
@@ -471,6 +539,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
         }
       }
     }
+    pdl_trigger();  // every copy of this CTA is issued: let the next kernel be scheduled
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer (leader only)
@@ -709,30 +778,12 @@ cudaError_t launch_tc(const TcGemmArgs& a, cudaStream_t s) {
     int grid = a.sm_count;
     if (bound < grid) grid = (int)bound;
     if (grid <= 0) return cudaSuccess;
-    auto kern = tc_ffn_kernel<kGateUp>;
-    kern<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(p);
-    return cudaGetLastError();
+    return launch_kernel(tc_ffn_kernel<kGateUp>, dim3(grid), dim3(NUM_THREADS), SMEM_BYTES, s, 1, p);
   }
   int pairs = a.sm_count / 2;
   if (bound < pairs) pairs = (int)bound;
   if (pairs <= 0) return cudaSuccess;
-  auto kern = tc2_ffn_kernel<kGateUp>;
-  cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3(2 * pairs);
-  cfg.blockDim = dim3(NUM_THREADS);
-  cfg.dynamicSmemBytes = SMEM2_BYTES;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  return launch_kernel(tc2_ffn_kernel<kGateUp>, dim3(2 * pairs), dim3(NUM_THREADS), SMEM2_BYTES, s, 2, p);
 }
 
 }  // namespace

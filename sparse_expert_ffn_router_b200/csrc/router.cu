@@ -86,6 +86,8 @@ template <typename Tin>
 __global__ void __launch_bounds__(kRouterThreads) router_topk_simt_kernel(
     const Tin* __restrict__ x, int T, int d, const Tin* __restrict__ wr, const float* __restrict__ b,
     int E, int k, int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ float sm[];
   constexpr int P = kRouterDK + 1;
   float* xs = sm;                        // [TT][P]
@@ -155,23 +157,51 @@ __device__ __forceinline__ float dot16(const uint4& xa, const uint4& wa, float a
   return acc;
 }
 
+// Small batches: one CTA per token.  Every thread takes the same 16-byte slices of x and of 8
+// expert rows at a time, so each thread has 9 independent loads per slice in flight; the 8
+// partial dot products are reduced per warp by shuffles and then over the 8 warps in a fixed
+// order (deterministic).
 template <typename Tin>
 __global__ void __launch_bounds__(256) router_small_kernel(const Tin* __restrict__ x, int d,
                                                            const Tin* __restrict__ wr, const float* __restrict__ b,
                                                            int E, int k, int32_t* __restrict__ idx_out,
                                                            float* __restrict__ w_out) {
+  pdl_trigger();
+  pdl_wait();
+  constexpr int kWarps = 8, kChunk = 8;
+  __shared__ float part[kWarps][kMaxExperts];
   __shared__ float lg[kMaxExperts];
   const int t = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nvec = d * (int)sizeof(Tin) / 16;
   const uint4* xv = reinterpret_cast<const uint4*>(x + (size_t)t * d);
-  for (int e = warp; e < E; e += 8) {
-    const uint4* wv = reinterpret_cast<const uint4*>(wr + (size_t)e * d);
-    float acc = 0.f;
-#pragma unroll 4
-    for (int v = lane; v < nvec; v += 32) acc = dot16(__ldg(xv + v), __ldg(wv + v), acc, x);
+  for (int e0 = 0; e0 < E; e0 += kChunk) {
+    float acc[kChunk];
 #pragma unroll
-    for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) lg[e] = acc + (b ? b[e] : 0.f);
+    for (int i = 0; i < kChunk; ++i) acc[i] = 0.f;
+#pragma unroll 2
+    for (int v = threadIdx.x; v < nvec; v += kWarps * 32) {
+      const uint4 xq = __ldg(xv + v);
+#pragma unroll
+      for (int i = 0; i < kChunk; ++i)
+        if (e0 + i < E) acc[i] = dot16(xq, __ldg(reinterpret_cast<const uint4*>(wr + (size_t)(e0 + i) * d) + v), acc[i], x);
+    }
+#pragma unroll
+    for (int i = 0; i < kChunk; ++i) {
+#pragma unroll
+      for (int off = 16; off; off >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int i = 0; i < kChunk; ++i)
+        if (e0 + i < E) part[warp][e0 + i] = acc[i];
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kWarps * 32) {
+    float sum = part[0][e];
+#pragma unroll
+    for (int wi = 1; wi < kWarps; ++wi) sum += part[wi][e];
+    lg[e] = sum + (b ? b[e] : 0.f);
   }
   __syncthreads();
   if (warp == 0) warp_topk(lg, E, k, lane, idx_out + (size_t)t * k, w_out + (size_t)t * k);
@@ -222,6 +252,7 @@ __device__ __forceinline__ bool rt_wait(uint64_t* bar, uint32_t parity, volatile
 __global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant__ RouterTcParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {  // the 128-byte swizzle needs 1024-byte aligned tiles
+    pdl_wait();
     if (threadIdx.x == 0 && p.err) atomicOr(p.err, kErrWaitTimeout);
     return;
   }
@@ -231,6 +262,8 @@ __global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant
   uint64_t* done = empty + S;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int* issued_s = const_cast<int*>(abort_flag) + 1;  // copies issued / stages consumed (error path)
+  int* consumed_s = issued_s + 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -239,10 +272,13 @@ __global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant
     }
     mbar_init(done, 1);
     *abort_flag = 0;
+    *issued_s = 0;
+    *consumed_s = 0;
     mbar_fence_init();
     tma_prefetch_desc(&p.mapX);
     tma_prefetch_desc(&p.mapW);
   }
+  pdl_wait();  // below: reads of earlier kernels' output; TMEM once the previous kernel released its own
   if (warp == 0) {
     tmem_alloc(tmem_holder, p.tmem_cols);
     tmem_relinquish();
@@ -257,49 +293,63 @@ __global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant
   const int nkb = kspan / 64;
 
   const uint32_t bytes = kRtABytes + (uint32_t)p.N * 128u;
-  if (threadIdx.x == 0) {
-    // ------------------------------------------------------------- TMA producer (warp 0)
-    bool ok = true;
-    for (int kb = 0; kb < nkb; ++kb) {
-      const int s = kb % S;
-      const uint32_t ph = (uint32_t)(kb / S) & 1u;
-      if (!rt_wait(&empty[s], ph ^ 1u, abort_flag)) {
-        ok = false;
-        break;
+  // The CTAs of a launch start their K walk at different blocks (rotated by the tile index), so
+  // the x rows read at one time do not all sit at the same column offset, which would put every
+  // request on the same DRAM channels.  (This fixes, per tile, the order of the fp32 sum.)
+  const int kb_rot = blockIdx.x % nkb;
+  if (warp == 0) {
+    if (lane == 0) {
+      // ----------------------------------------------------------- TMA producer
+      bool ok = true;
+      for (int i = 0; i < nkb; ++i) {
+        const int kb = (kb_rot + i) % nkb;
+        const int s = i % S;
+        const uint32_t ph = (uint32_t)(i / S) & 1u;
+        if (!rt_wait(&empty[s], ph ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint8_t* sa = smem + (size_t)s * p.stage_bytes;
+        mbar_arrive_expect_tx(&full[s], bytes);
+        tma_load_2d(sa, &p.mapX, &full[s], (kb0 + kb) * 64, row0);
+        tma_load_2d(sa + kRtABytes, &p.mapW, &full[s], (kb0 + kb) * 64, 0);
+        *issued_s = i + 1;
       }
-      uint8_t* sa = smem + (size_t)s * p.stage_bytes;
-      mbar_arrive_expect_tx(&full[s], bytes);
-      tma_load_2d(sa, &p.mapX, &full[s], (kb0 + kb) * 64, row0);
-      tma_load_2d(sa + kRtABytes, &p.mapW, &full[s], (kb0 + kb) * 64, 0);
-    }
-    if (!ok) {
-      *abort_flag = 1;
-      if (p.err) atomicOr(p.err, kErrWaitTimeout);
-    }
-  } else if (threadIdx.x == 32) {
-    // ------------------------------------------------------------- MMA issuer (warp 1)
-    const uint32_t idesc = idesc_bf16_f32(128, p.N);
-    bool ok = true;
-    for (int kb = 0; kb < nkb; ++kb) {
-      const int s = kb % S;
-      const uint32_t ph = (uint32_t)(kb / S) & 1u;
-      if (!rt_wait(&full[s], ph, abort_flag)) {
-        ok = false;
-        break;
+      if (!ok) {
+        *abort_flag = 1;
+        if (p.err) atomicOr(p.err, kErrWaitTimeout);
       }
-      tc_fence_after();
-      const uint32_t sa = smem_u32(smem + (size_t)s * p.stage_bytes);
+    }
+    pdl_trigger();  // every copy of this CTA is issued: let the next kernel be scheduled
+    __syncwarp();  // the other lanes wait here, not in a spin beside the producer
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ----------------------------------------------------------- MMA issuer
+      const uint32_t idesc = idesc_bf16_f32(128, p.N);
+      bool ok = true;
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % S;
+        const uint32_t ph = (uint32_t)(i / S) & 1u;
+        if (!rt_wait(&full[s], ph, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + (size_t)s * p.stage_bytes);
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        tc_mma_f16(tmem, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sa + kRtABytes + kk * 32), idesc,
-                   (kb | kk) != 0 ? 1u : 0u);
-      tc_commit(&empty[s]);  // frees the stage once these MMAs have read it
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_f16(tmem, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sa + kRtABytes + kk * 32), idesc,
+                     (i | kk) != 0 ? 1u : 0u);
+        tc_commit(&empty[s]);  // frees the stage once these MMAs have read it
+        *consumed_s = i + 1;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        if (p.err) atomicOr(p.err, kErrWaitTimeout);
+      }
+      tc_commit(done);  // arrives once every MMA issued above has completed
     }
-    if (!ok) {
-      *abort_flag = 1;
-      if (p.err) atomicOr(p.err, kErrWaitTimeout);
-    }
-    tc_commit(done);  // arrives once every MMA issued above has completed
+    __syncwarp();
   }
   // ------------------------------------------------------------- epilogue: one token per thread
   const bool got = rt_wait(done, 0, abort_flag) && !*abort_flag;
@@ -387,6 +437,11 @@ __global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant
   }
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) {
+    // copies issued but never consumed: wait (bounded) until they land before the CTA exits
+    for (int i = *consumed_s; i < *issued_s; ++i) mbar_wait_bounded(&full[i % S], (uint32_t)(i / S) & 1u);
+  }
+  __syncthreads();
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, p.tmem_cols);
@@ -427,8 +482,7 @@ cudaError_t launch_router_tc(const void* x, int T, int d, const void* wr, const 
   p.w = w;
   p.err = err;
   const size_t smem = (size_t)p.stages * p.stage_bytes + 1024;
-  router_tc_kernel<<<dim3((T + 127) / 128, ksplit), 128, smem, s>>>(p);
-  return cudaGetLastError();
+  return launch_kernel(router_tc_kernel, dim3((T + 127) / 128, ksplit), dim3(128), smem, s, 1, p);
 }
 
 }  // namespace
@@ -460,11 +514,10 @@ cudaError_t launch_router_topk(const void* x, int act, int T, int d, const void*
   if (T <= 0) return cudaSuccess;
   if (T <= kRouterSmallT) {
     if (act == COLIBRI_BF16)
-      router_small_kernel<__nv_bfloat16><<<T, 256, 0, s>>>((const __nv_bfloat16*)x, d, (const __nv_bfloat16*)wr, b,
-                                                           E, k, idx, w);
-    else
-      router_small_kernel<float><<<T, 256, 0, s>>>((const float*)x, d, (const float*)wr, b, E, k, idx, w);
-    return cudaGetLastError();
+      return launch_kernel(router_small_kernel<__nv_bfloat16>, dim3(T), dim3(256), 0, s, 1, (const __nv_bfloat16*)x, d,
+                           (const __nv_bfloat16*)wr, b, E, k, idx, w);
+    return launch_kernel(router_small_kernel<float>, dim3(T), dim3(256), 0, s, 1, (const float*)x, d,
+                         (const float*)wr, b, E, k, idx, w);
   }
   if (act == COLIBRI_BF16) {
     const int ks = (part && ticket) ? router_ksplit(T, d) : 1;
@@ -474,9 +527,8 @@ cudaError_t launch_router_topk(const void* x, int act, int T, int d, const void*
       sizeof(float) * ((size_t)kRouterTT * (kRouterDK + 1) + (size_t)E * (kRouterDK + 1) +
                        (size_t)kRouterTT * (E + 1));
   const dim3 grid((T + kRouterTT - 1) / kRouterTT);
-  router_topk_simt_kernel<float><<<grid, kRouterThreads, smem, s>>>((const float*)x, T, d, (const float*)wr, b, E,
-                                                                     k, idx, w);
-  return cudaGetLastError();
+  return launch_kernel(router_topk_simt_kernel<float>, grid, dim3(kRouterThreads), smem, s, 1, (const float*)x, T, d,
+                       (const float*)wr, b, E, k, idx, w);
 }
 
 }  // namespace colibri

@@ -180,6 +180,32 @@ def test_graph_replay_matches_plain_launches(name):
     layer.close()
 
 
+@pytest.mark.parametrize("name", ["bf16_shared", "bf16_T1", "f32_shared", "i8_small", "i8_many"])
+def test_overlapped_launches_match_serial_launches(name, monkeypatch):
+    # programmatic dependent launch (the default) only lets a kernel start its set-up early:
+    # the results must be bit-identical to strictly serialised launches
+    wl = SMALL[name]
+    p = inputgen.make_problem(wl, seed=13)
+    t = H.to_device(p)
+    args = (t["x"], t["router_w"], t["router_b"], t["expert_w"])
+    kw = dict(expert_scales=t["expert_scales"], shared_w=t["shared_w"])
+    outs = []
+    for pdl in ("0", "1"):
+        monkeypatch.setenv("COLIBRI_PDL", pdl)
+        layer = H.make_layer(wl)
+        s = torch.cuda.Stream()
+        for on_stream in (False, True):  # plain launches, then a captured graph
+            y = torch.full((wl.T, wl.d), 5.0, dtype=p.x.dtype, device="cuda")
+            layer.forward(*args, y, stream=s if on_stream else None, **kw)
+            torch.cuda.synchronize()
+            outs.append(y)
+        layer.sync_status()
+        layer.close()
+    for y in outs[1:]:
+        assert torch.equal(y, outs[0])
+    H.parity(p)  # and the overlapped launches against the oracle
+
+
 def test_graph_cache_distinguishes_token_counts():
     wl = SMALL["bf16_shared"]
     layer = H.make_layer(wl, max_tokens=600)
