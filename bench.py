@@ -42,8 +42,10 @@ def kernels_per_step(wl):
         n += 2 + (2 if wl.fs else 0)                 # fp32: gate/up + down (+ the shared expert's)
     elif wl.wdt == 1:
         n += 2                                       # bf16: gate/up + down (shared expert inside)
-    else:
+    elif os.environ.get("COLIBRI_DEC_FUSED", "1") == "0":
         n += 3                                       # int8: gate/up stream, finish H, down stream
+    else:
+        return n + 1                                 # int8: one fused launch, the combine inside
     return n + 1                                     # Gather
 
 
@@ -389,16 +391,26 @@ def main():
     pk = peaks()
     per_call = {k: v / max(ncalls, 1) for k, v in stage_ms.items()}
     if wl.wdt == 2:
-        achieved = (wk["w13_bytes"] + wk["scale_bytes"]) / (per_call["expert_gateup"] / 1e3) / 1e9
-        roof = {"kernel": "dec_stream_kernel<gate/up> (tcgen05 kind::i8 weight stream)", "bound": "hbm",
-                "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s", "frac": achieved / pk["hbm"],
-                "algorithmic_bytes_per_launch": wk["w13_bytes"] + wk["scale_bytes"]}
+        # the expert stage and the combine: one fused launch (or, with COLIBRI_DEC_FUSED=0, the
+        # gate/up stream, H planes, down stream and combine launches), all touched weights
+        wbytes = wk["w13_bytes"] + wk["w2_bytes"] + wk["scale_bytes"]
+        ms_exp = per_call["expert_gateup"] + per_call["expert_down"] + per_call["gather"]
+        achieved = wbytes / (ms_exp / 1e3) / 1e9
+        fused = os.environ.get("COLIBRI_DEC_FUSED", "1") != "0"
+        roof = {"kernel": ("dec_fused_kernel (one cooperative launch: tcgen05 kind::i8 gate/up stream, H planes, "
+                           "down stream, combine)") if fused else
+                ("dec_stream_kernel<gate/up> + dec_finish_h_kernel + dec_stream_kernel<down> + "
+                 "combine_split_kernel (tcgen05 kind::i8 weight streams)"),
+                "bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s", "frac": achieved / pk["hbm"],
+                "algorithmic_bytes_per_launch": wbytes}
     elif wl.wdt == 1:
         achieved = wk["flops_gateup"] / (per_call["expert_gateup"] / 1e3) / 1e12
-        pair = os.environ.get("COLIBRI_GEMM_CTA", "") == "2" or (
-            os.environ.get("COLIBRI_GEMM_CTA", "") != "1" and wl.T * wl.k // wl.E >= 512)
-        name = ("tc2_ffn_kernel<gate/up> (tcgen05, 2-CTA pair tiles)" if pair
-                else "tc_ffn_kernel<gate/up> (tcgen05)")
+        mode = os.environ.get("COLIBRI_GEMM_CTA", "")[:1]
+        if mode not in ("1", "2", "s"):
+            mode = "2" if wl.T * wl.k // wl.E >= 512 else "s"
+        name = {"1": "tc_ffn_kernel<gate/up> (tcgen05, 128x256 tiles)",
+                "2": "tc2_ffn_kernel<gate/up> (tcgen05, 2-CTA 256x256 pair tiles)",
+                "s": "tcs_ffn_kernel<gate/up> (tcgen05, weights x 16..256 token rows)"}[mode]
         roof = {"kernel": name, "bound": "tensor", "achieved": achieved,
                 "peak": pk["bf16"], "unit": "TFLOP/s", "frac": achieved / pk["bf16"],
                 "algorithmic_flops_per_launch": wk["flops_gateup"]}

@@ -81,14 +81,18 @@ int pick_dec_split(int f) {
   return 1;
 }
 
-// Pair (2-CTA) tiles for the bf16 expert GEMMs.  COLIBRI_GEMM_CTA=1 or 2 forces a mode
-// (both are exact; this only selects the tile shape).
-bool use_pair_tiles(const colibri_ctx* ctx, int avg_rows_per_expert) {
+// Tile shape of the bf16 expert GEMMs: 0 = one CTA, 128 rows x 256 columns; 1 = pairs of CTAs
+// (cta_group::2), 256 x 256; 2 = swapped operands, 128 channels x 16..256 rows.  Pair tiles when
+// experts average >= 512 rows (the halved L2 traffic outweighs the larger last tile of each
+// expert), else swapped tiles (little row padding for small or uneven groups).
+// COLIBRI_GEMM_CTA=1, 2 or s forces a mode (all are exact; this only selects the tiling).
+enum GemmMode { kGemmOne = 0, kGemmPair = 1, kGemmSwap = 2 };
+int gemm_mode(int avg_rows_per_expert) {
   const char* v = getenv("COLIBRI_GEMM_CTA");
-  if (v && v[0] == '1') return false;
-  if (v && v[0] == '2') return true;
-  (void)ctx;
-  return avg_rows_per_expert >= 512;
+  if (v && v[0] == '1') return kGemmOne;
+  if (v && v[0] == '2') return kGemmPair;
+  if (v && v[0] == 's') return kGemmSwap;
+  return avg_rows_per_expert >= 512 ? kGemmPair : kGemmSwap;
 }
 
 constexpr size_t kMaxGraphs = 8;  // captured forwards kept per context (least recently used evicted)
@@ -218,6 +222,7 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   const size_t o_rpart = c.take(rsplit ? (size_t)kRouterMaxSplit * M * E * 4 : 0);
   const size_t o_rtick = c.take(rsplit ? (size_t)((M + 127) / 128) * 4 : 0);
   const size_t o_err = c.take(4);
+  const size_t o_gbar = c.take(i8 ? 16 : 0);
   ctx->ws_bytes = c.off;
 
   DeviceGuard guard(D.device_id);
@@ -250,10 +255,12 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   w.plane_lo = reinterpret_cast<int8_t*>(b + o_plo);
   w.plane_scale = reinterpret_cast<float*>(b + o_psc);
   w.err = reinterpret_cast<uint32_t*>(b + o_err);
+  w.grid_bar = i8 ? reinterpret_cast<int32_t*>(b + o_gbar) : nullptr;
   w.router_part = rsplit ? reinterpret_cast<float*>(b + o_rpart) : nullptr;
   w.router_ticket = rsplit ? reinterpret_cast<int32_t*>(b + o_rtick) : nullptr;
   if (cudaMemset(w.err, 0, 4) != cudaSuccess ||
-      (rsplit && cudaMemset(w.router_ticket, 0, (size_t)((M + 127) / 128) * 4) != cudaSuccess)) {
+      (rsplit && cudaMemset(w.router_ticket, 0, (size_t)((M + 127) / 128) * 4) != cudaSuccess) ||
+      (i8 && cudaMemset(w.grid_bar, 0, 16) != cudaSuccess)) {
     cudaFree(ctx->ws_base);
     delete ctx;
     return fail(nullptr, COLIBRI_ERR_CUDA, "cudaMemset failed");
@@ -262,9 +269,13 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
     for (auto& e : ctx->ev) cudaEventCreate(&e);
   }
   ctx->use_graphs = !(getenv("COLIBRI_GRAPHS") && strcmp(getenv("COLIBRI_GRAPHS"), "0") == 0);
-  ctx->use_pdl = !(getenv("COLIBRI_PDL") && strcmp(getenv("COLIBRI_PDL"), "0") == 0);
+  // Programmatic dependent launch measured slower on the small-batch decode chain and neutral on
+  // prefill, so it is opt-in (COLIBRI_PDL=1).
+  ctx->use_pdl = env_flag("COLIBRI_PDL");
+  ctx->dec_fused = !(getenv("COLIBRI_DEC_FUSED") && strcmp(getenv("COLIBRI_DEC_FUSED"), "0") == 0);
   cudaError_t ce = configure_router_kernels();
   if (ce == cudaSuccess) ce = configure_tc_kernels();
+  if (ce == cudaSuccess) ce = configure_tcs_kernels();
   if (ce == cudaSuccess) ce = configure_dec_kernels();
   if (ce != cudaSuccess) {
     cudaGetLastError();
@@ -310,7 +321,7 @@ colibri_status check_launch(colibri_ctx* ctx, cudaError_t e, const char* what) {
 colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int32_t T, const void* router_w,
                                const float* router_b, const int32_t* user_idx, const float* user_w,
                                const void* expert_w, const float* expert_scales, const void* shared_w, void* y,
-                               PtrKind yk, cudaStream_t s, bool pair_tiles) {
+                               PtrKind yk, cudaStream_t s, int gemm) {
   const colibri_desc& D = ctx->desc;
   const bool routed_by_caller = user_idx != nullptr;
   Workspace& w = ctx->ws;
@@ -353,7 +364,7 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
 
   // ---- Scatter
   const int nblk = (T + kCountBlock - 1) / kCountBlock;
-  const int bm = D.weight_dtype == COLIBRI_F32 ? kSimtBM : (pair_tiles ? kTcPairBM : kTcBM);
+  const int bm = D.weight_dtype == COLIBRI_F32 ? kSimtBM : (gemm == kGemmPair ? kTcPairBM : kTcBM);
   const RowPlanes xplanes{w.plane_hi, w.plane_lo, w.plane_scale};
   const RowPlanes* planes = D.weight_dtype == COLIBRI_I8 ? &xplanes : nullptr;
   if (T <= kFusedRouteMaxT) {
@@ -363,8 +374,8 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
     COLIBRI_TRY(launch_route_count(w.topk_idx, T, k, E, w.blk_counts, w.dst_row, s), "route_count");
     COLIBRI_TRY(launch_route_scan(w.blk_counts, nblk, E, bm, w.blk_base, w.counts, w.offsets, w.mt_prefix, s),
                 "route_scan");
-    COLIBRI_TRY(launch_route_scatter(xd, act, T, d, k, E, w.topk_idx, w.blk_base, w.dst_row, w.src_row, w.Xp,
-                                     planes, s), "route_scatter");
+    COLIBRI_TRY(launch_route_scatter(xd, act, T, d, k, E, w.topk_idx, w.blk_base, w.offsets, w.dst_row, w.src_row,
+                                     w.Xp, planes, s), "route_scatter");
   }
   mark(2);
 
@@ -407,14 +418,16 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
     a.mt_bound = R / bm + E;
     a.err = w.err;
     a.sm_count = ctx->sm_count;
-    a.pair = pair_tiles;
-    COLIBRI_TRY(launch_tc_gateup(a, s), "tc_gateup");
+    a.pair = gemm == kGemmPair;
+    if (gemm == kGemmSwap) COLIBRI_TRY(launch_tcs_gateup(a, s), "tcs_gateup");
+    else COLIBRI_TRY(launch_tc_gateup(a, s), "tc_gateup");
     mark(3);
     a.A = w.H;
     a.out = w.Yp;
     a.A_sh = w.Hs;
     a.out_sh = w.Ys;
-    COLIBRI_TRY(launch_tc_down(a, s), "tc_down");
+    if (gemm == kGemmSwap) COLIBRI_TRY(launch_tcs_down(a, s), "tcs_down");
+    else COLIBRI_TRY(launch_tc_down(a, s), "tc_down");
   } else {
     // K splits of the down projection: enough work items to cover every SM a few times
     nsplit = 1;
@@ -430,18 +443,48 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
              touched * tiles * gsplit < 8 * ctx->sm_count)
         gsplit <<= 1;
     }
-    COLIBRI_TRY(launch_dec_gateup(w.plane_hi, w.plane_lo, w.plane_scale, (const int8_t*)expert_w, expert_scales,
-                                  stride, d, f, E, w.offsets, gsplit, (float*)w.H, R, T, w.err, s), "dec_gateup");
-    mark(3);
-    COLIBRI_TRY(launch_dec_finish_h((const float*)w.H, gsplit, R, f, nsplit, w.plane_hi, w.plane_lo, w.plane_scale,
-                                    s), "dec_finish_h");
-    COLIBRI_TRY(launch_dec_down(w.plane_hi, w.plane_lo, w.plane_scale, (const int8_t*)expert_w, expert_scales,
-                                stride, d, f, E, w.offsets, nsplit, R, w.Ypart, T, w.err, s), "dec_down");
+    if (ctx->dec_fused) {
+      // one cooperative launch for gate/up, H, down and the combine (stages 3-5 are empty)
+      DecFusedArgs fa;
+      fa.planes_hi = w.plane_hi;
+      fa.planes_lo = w.plane_lo;
+      fa.planes_scale = w.plane_scale;
+      fa.W = (const int8_t*)expert_w;
+      fa.scales = expert_scales;
+      fa.wstride = stride;
+      fa.d = d;
+      fa.f = f;
+      fa.E = E;
+      fa.T = T;
+      fa.k = k;
+      fa.offsets = w.offsets;
+      fa.dst_row = w.dst_row;
+      fa.topk_w = w.topk_w;
+      fa.gsplit = gsplit;
+      fa.dsplit = nsplit;
+      fa.GU = (float*)w.H;
+      fa.Ypart = w.Ypart;
+      fa.y = (__nv_bfloat16*)yd;
+      fa.bar = w.grid_bar;
+      fa.err = w.err;
+      COLIBRI_TRY(launch_dec_fused(fa, s), "dec_fused");
+      mark(3);
+    } else {
+      COLIBRI_TRY(launch_dec_gateup(w.plane_hi, w.plane_lo, w.plane_scale, (const int8_t*)expert_w, expert_scales,
+                                    stride, d, f, E, w.offsets, gsplit, (float*)w.H, R, T, w.err, s), "dec_gateup");
+      mark(3);
+      COLIBRI_TRY(launch_dec_finish_h((const float*)w.H, gsplit, R, f, nsplit, w.plane_hi, w.plane_lo,
+                                      w.plane_scale, s), "dec_finish_h");
+      COLIBRI_TRY(launch_dec_down(w.plane_hi, w.plane_lo, w.plane_scale, (const int8_t*)expert_w, expert_scales,
+                                  stride, d, f, E, w.offsets, nsplit, R, w.Ypart, T, w.err, s), "dec_down");
+    }
   }
   mark(4);
 
   // ---- Gather
-  if (D.weight_dtype == COLIBRI_I8) {
+  if (D.weight_dtype == COLIBRI_I8 && ctx->dec_fused) {
+    // done inside the fused kernel
+  } else if (D.weight_dtype == COLIBRI_I8) {
     COLIBRI_TRY(launch_combine_split(w.Ypart, nsplit, R, w.dst_row, w.topk_w, T, k, d, yd, act, s),
                 "combine_split");
   } else {
@@ -501,10 +544,8 @@ colibri_status forward_impl(colibri_ctx* ctx, const void* x, int32_t T, const vo
   const PtrKind xk = classify(x, dev), yk = classify(y, dev);
   if (xk == kPtrBad || yk == kPtrBad)
     return fail(ctx, COLIBRI_ERR_INVALID_ARG, "x or y is device memory of another device");
-  // bf16 weights: pair tiles (two CTAs, 256 rows) when experts average >= 512 rows, where the
-  // halved L2 traffic per unit of work outweighs the larger last tile of each expert.
-  const bool pair_tiles =
-      D.weight_dtype == COLIBRI_BF16 && use_pair_tiles(ctx, T * D.top_k / D.num_experts);
+  // bf16 weights: the tiling of the expert GEMMs (see gemm_mode)
+  const int gemm = D.weight_dtype == COLIBRI_BF16 ? gemm_mode(T * D.top_k / D.num_experts) : kGemmOne;
 
   // Replay a captured CUDA graph of this exact call when possible: device x and y, a stream
   // other than the legacy default stream that is not itself being captured, and no profiling.
@@ -519,7 +560,7 @@ colibri_status forward_impl(colibri_ctx* ctx, const void* x, int32_t T, const vo
     if (cs == cudaStreamCaptureStatusNone) {
       const uintptr_t key[14] = {(uintptr_t)x,        (uintptr_t)T,        (uintptr_t)router_w, (uintptr_t)router_b,
                                  (uintptr_t)user_idx, (uintptr_t)user_w,   (uintptr_t)expert_w, (uintptr_t)expert_scales,
-                                 (uintptr_t)shared_w, (uintptr_t)y,        (uintptr_t)s,        (uintptr_t)pair_tiles,
+                                 (uintptr_t)shared_w, (uintptr_t)y,        (uintptr_t)s,        (uintptr_t)gemm,
                                  0, 0};
       for (auto& g : ctx->graphs) {
         if (memcmp(g.key, key, sizeof(key)) == 0) {
@@ -530,7 +571,7 @@ colibri_status forward_impl(colibri_ctx* ctx, const void* x, int32_t T, const vo
       }
       COLIBRI_TRY(cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal), "begin capture");
       const colibri_status st = enqueue_forward(ctx, x, xk, T, router_w, router_b, user_idx, user_w, expert_w,
-                                                expert_scales, shared_w, y, yk, s, pair_tiles);
+                                                expert_scales, shared_w, y, yk, s, gemm);
       cudaGraph_t graph = nullptr;
       const cudaError_t ce = cudaStreamEndCapture(s, &graph);
       if (st != COLIBRI_OK) {
@@ -560,7 +601,7 @@ colibri_status forward_impl(colibri_ctx* ctx, const void* x, int32_t T, const vo
     }
   }
   return enqueue_forward(ctx, x, xk, T, router_w, router_b, user_idx, user_w, expert_w, expert_scales, shared_w, y,
-                         yk, s, pair_tiles);
+                         yk, s, gemm);
 }
 
 }  // namespace

@@ -2,7 +2,7 @@
 // summed in slot order j = 0..k-1 in fp32 and rounded once to the activation dtype
 // (www.hotelren.com/news/4731937 §2.1 step 6 and §2.3 combine_kernel; the fixed-order k-way
 // aggregation of www.pptc.cn/news/100465 §2.1, without the atomic accumulation of its §1 so
-// that the result is deterministic).  One warp per token, 16-byte vector accesses.
+// that the result is deterministic).  16-byte vector accesses.
 #include <algorithm>
 
 #include "common.cuh"
@@ -38,6 +38,8 @@ __device__ __forceinline__ void store8(float* p, const float (&v)[8]) {
   reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
 
+// One thread per (token, 8 consecutive outputs): the k slot loads of a thread are independent,
+// and a warp covers 512 contiguous bytes of each row it reads or writes.
 template <typename Tout, typename Typ>
 __global__ void __launch_bounds__(256) combine_kernel(const Typ* __restrict__ Yp,
                                                       const int32_t* __restrict__ dst_row,
@@ -46,42 +48,34 @@ __global__ void __launch_bounds__(256) combine_kernel(const Typ* __restrict__ Yp
                                                       Tout* __restrict__ y) {
   pdl_trigger();
   pdl_wait();
-  const int lane = threadIdx.x & 31;
-  const int warps_total = gridDim.x * (blockDim.x >> 5);
-  for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps_total) {
-    int r = 0;
-    float wj = 0.f;
-    if (lane < k) {
-      r = dst_row[(size_t)t * k + lane];
-      wj = w[(size_t)t * k + lane];
-    }
+  const int chunks = d >> 3;
+  for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < (long long)T * chunks;
+       q += (long long)gridDim.x * blockDim.x) {
+    const int t = (int)(q / chunks), c = (int)(q - (long long)t * chunks) * 8;
     int rows[kMaxTopK];
     float ws[kMaxTopK];
 #pragma unroll
     for (int j = 0; j < kMaxTopK; ++j) {
-      rows[j] = __shfl_sync(0xffffffffu, r, j);
-      ws[j] = __shfl_sync(0xffffffffu, wj, j);
+      rows[j] = j < k ? dst_row[(size_t)t * k + j] : 0;
+      ws[j] = j < k ? w[(size_t)t * k + j] : 0.f;
     }
-#pragma unroll 2
-    for (int c = lane * 8; c < d; c += 32 * 8) {
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int j = 0; j < kMaxTopK; ++j) {
-        if (j < k) {
-          float v[8];
-          load8(Yp + (size_t)rows[j] * d + c, v);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i] = fmaf(ws[j], v[i], acc[i]);
-        }
-      }
-      if (Ys) {
+    for (int j = 0; j < kMaxTopK; ++j) {
+      if (j < k) {
         float v[8];
-        load8(Ys + (size_t)t * d + c, v);
+        load8(Yp + (size_t)rows[j] * d + c, v);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] += v[i];
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(ws[j], v[i], acc[i]);
       }
-      store8(y + (size_t)t * d + c, acc);
     }
+    if (Ys) {
+      float v[8];
+      load8(Ys + (size_t)t * d + c, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] += v[i];
+    }
+    store8(y + (size_t)t * d + c, acc);
   }
 }
 
@@ -146,9 +140,9 @@ __global__ void __launch_bounds__(256) combine_split_kernel(const float* __restr
   }
 }
 
-int grid_for_tokens(int T) {
-  int g = (T + 7) / 8;
-  return g > 8192 ? 8192 : g;
+int grid_for_rows(int T, int d) {
+  const long long threads = (long long)T * (d / 8);
+  return (int)std::min<long long>((threads + 255) / 256, 16384);
 }
 
 }  // namespace
@@ -156,7 +150,7 @@ int grid_for_tokens(int T) {
 cudaError_t launch_combine(const void* Yp, int yp_dtype, const int32_t* dst_row, const float* w,
                            int T, int k, int d, const void* Ys, void* y, int act, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  const dim3 grid(grid_for_tokens(T)), block(256);
+  const dim3 grid(grid_for_rows(T, d)), block(256);
   if (yp_dtype == COLIBRI_BF16) {
     const __nv_bfloat16* yp = (const __nv_bfloat16*)Yp;
     const __nv_bfloat16* ys = (const __nv_bfloat16*)Ys;

@@ -77,6 +77,7 @@ struct Workspace {
   float* Ypart = nullptr;  // [split, M*k, d] f32, int8 path
   float* router_part = nullptr;    // [8, M, E] K-split partial logits
   int32_t* router_ticket = nullptr;  // [ceil(M/128)] arrival counters (zero between calls)
+  int32_t* grid_bar = nullptr;       // [4] grid-barrier counters of the fused int8 kernel (zero between calls)
   int8_t* plane_hi = nullptr;  // [M*k, max(d, f)] int8 activation planes, int8 path
   int8_t* plane_lo = nullptr;
   float* plane_scale = nullptr;  // [M*k]
@@ -112,7 +113,8 @@ struct colibri_ctx {
   std::vector<GraphEntry> graphs;
   uint64_t graph_clock = 0;
   bool use_graphs = true;
-  bool use_pdl = true;  // programmatic dependent launch between the kernels of a forward
+  bool use_pdl = false;  // programmatic dependent launch between the kernels of a forward (opt-in)
+  bool dec_fused = true;  // int8 weights: the one-launch expert stage (COLIBRI_DEC_FUSED=0: four launches)
 };
 
 namespace colibri {
@@ -200,9 +202,11 @@ struct RowPlanes {
   int8_t* lo;
   float* scale;
 };
+// blk_base: per (block, expert) exclusive prefix of the block counts (without offsets[e])
 cudaError_t launch_route_scatter(const void* x, int act, int T, int d, int k, int E,
-                                 const int32_t* idx, const int32_t* blk_base, int32_t* dst_row,
-                                 int32_t* src_row, void* Xp, const RowPlanes* planes, cudaStream_t s);
+                                 const int32_t* idx, const int32_t* blk_base, const int32_t* offsets,
+                                 int32_t* dst_row, int32_t* src_row, void* Xp, const RowPlanes* planes,
+                                 cudaStream_t s);
 // T <= kFusedRouteMaxT: count + scan + scatter in one single-CTA launch
 cudaError_t launch_route_fused(const void* x, int act, int T, int d, const int32_t* idx, int k, int E, int bm,
                                int32_t* counts, int32_t* offsets, int32_t* mt_prefix, int32_t* src_row,
@@ -260,6 +264,12 @@ cudaError_t configure_tc_kernels();      // once per device, before any launch
 cudaError_t configure_router_kernels();  // once per device, before any launch
 cudaError_t launch_tc_gateup(const TcGemmArgs& a, cudaStream_t s);
 cudaError_t launch_tc_down(const TcGemmArgs& a, cudaStream_t s);
+// The same grouped GEMMs with weights on the M side and token rows on the N side (tiles of
+// 128 channels x 16..256 rows), see gemm_tcs.cu.  Reads A/rows/offsets/E/W/wstride/out, the
+// shared-expert fields, d/f/fs, err and sm_count of TcGemmArgs.
+cudaError_t configure_tcs_kernels();     // once per device, before any launch
+cudaError_t launch_tcs_gateup(const TcGemmArgs& a, cudaStream_t s);
+cudaError_t launch_tcs_down(const TcGemmArgs& a, cudaStream_t s);
 
 // int8 weight-streaming decode path, see decode_i8.cu (the x planes come from the scatter)
 // max_rows_per_expert: an upper bound (T) that picks the token chunk (8, 16 or 32 rows).
@@ -276,6 +286,27 @@ cudaError_t launch_dec_down(const int8_t* Hhi, const int8_t* Hlo, const float* h
                             const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
                             int nsplit, int R, float* Ypart, int max_rows_per_expert, uint32_t* err,
                             cudaStream_t s);
+// The whole int8 expert stage (gate/up stream, H planes, down stream, combine) in one
+// cooperative launch with grid barriers; the x planes must already be in planes_hi/lo/scale.
+struct DecFusedArgs {
+  int8_t* planes_hi;        // [R, max(d, f)]: x planes in, H planes written in place
+  int8_t* planes_lo;
+  float* planes_scale;      // x scales [R] in; H scales [dsplit, R] written
+  const int8_t* W;          // expert buffer (int8) and its per-channel scales
+  const float* scales;
+  int64_t wstride;
+  int d, f, E, T, k;
+  const int32_t* offsets;   // [E+1]
+  const int32_t* dst_row;   // [T, k]
+  const float* topk_w;      // [T, k]
+  int gsplit, dsplit;       // K splits of gate/up and of down
+  float* GU;                // [gsplit, 2, R, f]
+  float* Ypart;             // [dsplit, R, d]
+  __nv_bfloat16* y;         // [T, d]
+  int32_t* bar;             // [4] zeroed counters
+  uint32_t* err;
+};
+cudaError_t launch_dec_fused(const DecFusedArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------------------------------
 // Small device helpers

@@ -26,6 +26,7 @@
 // into fp32 partial sums (summed in fixed order by the combine) to spread one token over every
 // SM.  Every wait is bounded.
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
 
 #include "common.cuh"
@@ -104,11 +105,12 @@ __global__ void __launch_bounds__(kFinishThreads) dec_finish_h_kernel(const floa
   }
 }
 
-// ------------------------------------------------------------------------- stream kernel
+// ------------------------------------------------------------------------- stream kernels
 constexpr int kDsThreads = 192;
 constexpr int kDsTmemCols = 256;
 constexpr size_t kDsRingBytes = 200 * 1024;
 constexpr int kDsMaxStages = 12;
+constexpr int kDsMaxKbs = 4;
 
 struct alignas(64) DecStreamParams {
   CUtensorMap mapW;   // int8 weights: gate/up {d, f, 2, E} (W1, W3); down {f, d, E} (W2)
@@ -123,7 +125,8 @@ struct alignas(64) DecStreamParams {
   int K, nsplit, kspan;     // kspan: K range of one split (a multiple of 128 unless nsplit == 1)
   int nt8;                  // tokens per chunk (8, 16 or 32); MMA N = 2 * nt8
   int R;                    // rows of the planes (T * k)
-  uint32_t stage_bytes;
+  int kbs;                  // 128-byte K blocks per ring stage (1..kDsMaxKbs)
+  uint32_t stage_bytes;     // kbs x (weight tile 128 x 128 + planes 2 nt8 x 128)
   int stages;
   float* GU;                // gate/up output: [nsplit, 2, R, f] fp32 partials (W1 . x, W3 . x, scaled)
   float* Ypart;             // down output [nsplit, R, d]
@@ -179,9 +182,295 @@ __device__ __forceinline__ bool ds_wait(uint64_t* bar, uint32_t parity, volatile
   }
 }
 
+// Shared-memory control block of the stream kernels (after the ring).
+struct DsCtl {
+  uint64_t full[kDsMaxStages];
+  uint64_t empty[kDsMaxStages];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem;
+  int abort;
+  int issued;    // copies issued / stages consumed, for the error path
+  int consumed;
+  int flag;      // result of a grid-wide wait, broadcast to the epilogue warps
+  int ntouched;
+  int32_t touched[kMaxExperts];
+  int32_t pre[2][kMaxExperts + 1];  // item prefix over the touched experts: [0] gate/up, [1] down
+  int32_t defer_row[kDsMaxStages];  // fused kernel: down stages whose plane copies wait for H
+  int32_t defer_kx[kDsMaxStages][kDsMaxKbs];
+  int32_t defer_nk[kDsMaxStages];
+  int32_t defer_s[kDsMaxStages];
+  float red[4];                     // fused kernel: per-warp maxima of the H pass
+};
+constexpr size_t kDsCtlBytes = 4096;
+static_assert(sizeof(DsCtl) <= kDsCtlBytes, "stream-kernel control block");
+
+__device__ __forceinline__ void ds_abort(DsCtl& c, uint32_t* err) {
+  *(volatile int*)&c.abort = 1;
+  atomicOr(err, kErrWaitTimeout);
+}
+
+// Ring position shared by the phases a role walks through.
+struct DsRing {
+  int s = 0;
+  uint32_t ph = 0;
+  int n = 0;  // copies issued (producer) or stages consumed (MMA)
+  __device__ void advance(int S) {
+    ++n;
+    if (++s == S) {
+      s = 0;
+      ph ^= 1u;
+    }
+  }
+};
+
+// Plane copies of K block j of a stage (hi rows, then lo rows of the same tokens).
+__device__ __forceinline__ void ds_load_planes(const DecStreamParams& p, uint8_t* stage, uint64_t* full, int j, int kx,
+                                               int row0) {
+  uint8_t* sb = stage + (size_t)p.kbs * 128 * 128 + (size_t)j * (2 * p.nt8 * 128);
+  tma_load_2d(sb, &p.mapHi, full, kx, row0);
+  tma_load_2d(sb + p.nt8 * 128, &p.mapLo, full, kx, row0);
+}
+
+// Producer: every stage of one phase.  A stage carries kbs consecutive K blocks of one item, so
+// each weight row is read kbs x 128 contiguous bytes at a time.  With `defer` the plane copies of
+// the first ring-full of stages are held back (their weight copies go out at once) until
+// `ready()` returns true.
+template <bool kGateUp, typename Ready>
+__device__ bool ds_produce(const DecStreamParams& p, uint8_t* smem, DsCtl& c, int S, int pre_idx, DsRing& r,
+                           bool defer, Ready ready) {
+  const uint32_t blk_bytes = 128u * 128u + (uint32_t)(2 * p.nt8) * 128u;
+  int held = 0;
+  bool released = !defer;
+  auto release = [&]() {
+    for (int h = 0; h < held; ++h) {
+      uint8_t* st = smem + (size_t)c.defer_s[h] * p.stage_bytes;
+      for (int j = 0; j < c.defer_nk[h]; ++j)
+        ds_load_planes(p, st, &c.full[c.defer_s[h]], j, c.defer_kx[h][j], c.defer_row[h]);
+    }
+  };
+  DecItem it;
+  for (int L = blockIdx.x; dec_item<kGateUp>(p, c.touched, c.pre[pre_idx], c.ntouched, L, it); L += gridDim.x) {
+    // The item's K blocks start at a rotated block (item index mod block count): items in flight
+    // at the same time then read different column offsets of their weight rows, which spreads
+    // the requests over the DRAM channels instead of hitting the same address bits everywhere.
+    // The accumulation is exact int32, so the block order does not matter.
+    const int kbeg = it.split * p.kspan, kend = min(p.K, kbeg + p.kspan);
+    const int nkb = (kend - kbeg + 127) / 128;
+    int kb = L % nkb;
+    for (int i = 0; i < nkb; i += p.kbs) {
+      const int nk = min(p.kbs, nkb - i);
+      if (!ds_wait(&c.empty[r.s], r.ph ^ 1u, &c.abort)) return false;
+      uint8_t* st = smem + (size_t)r.s * p.stage_bytes;
+      mbar_arrive_expect_tx(&c.full[r.s], (uint32_t)nk * blk_bytes);
+      for (int j = 0; j < nk; ++j, kb = (kb + 1 == nkb) ? 0 : kb + 1) {
+        const int kx = kbeg + kb * 128;
+        uint8_t* sw = st + (size_t)j * 128 * 128;
+        if (kGateUp) tma_load_4d(sw, &p.mapW, &c.full[r.s], kx, it.tile * 128, it.mat, it.e);
+        else tma_load_3d(sw, &p.mapW, &c.full[r.s], kx, it.tile * 128, it.e);
+        if (released) ds_load_planes(p, st, &c.full[r.s], j, kx, it.row0);
+        else c.defer_kx[held][j] = kx;
+      }
+      if (!released) {
+        c.defer_row[held] = it.row0;
+        c.defer_nk[held] = nk;
+        c.defer_s[held] = r.s;
+        if (++held == S) {
+          // the held plane copies are issued even when the wait gave up, so that every issued
+          // stage completes and the error path drains quickly
+          const bool go = ready();
+          release();
+          if (!go) return false;
+          released = true;
+        }
+      }
+      c.issued = r.n + 1;
+      r.advance(S);
+    }
+  }
+  if (!released && held > 0) {
+    const bool go = ready();
+    release();
+    if (!go) return false;
+  }
+  return true;
+}
+
+// MMA issuer: every item of one phase (A = 128 weight rows, B = hi rows stacked on lo rows).
+template <bool kGateUp>
+__device__ bool ds_mma(const DecStreamParams& p, uint8_t* smem, DsCtl& c, int S, int pre_idx, DsRing& r, int& iter,
+                       uint32_t tmem) {
+  const int N = 2 * p.nt8;
+  const uint32_t idesc = idesc_s8_s32(128, N);
+  const uint32_t plane_bytes = (uint32_t)(2 * p.nt8 * 128);
+  DecItem it;
+  for (int L = blockIdx.x; dec_item<kGateUp>(p, c.touched, c.pre[pre_idx], c.ntouched, L, it);
+       L += gridDim.x, ++iter) {
+    const int a = iter & 1;
+    const uint32_t aph = (uint32_t)(iter >> 1) & 1u;
+    if (!ds_wait(&c.tempty[a], aph ^ 1u, &c.abort)) return false;
+    tc_fence_after();
+    const uint32_t dbase = tmem + (uint32_t)(a * N);
+    const int kbeg = it.split * p.kspan, kend = min(p.K, kbeg + p.kspan);
+    const int nkb = (kend - kbeg + 127) / 128;
+    bool first = true;
+    for (int i = 0; i < nkb; i += p.kbs) {
+      const int nk = min(p.kbs, nkb - i);
+      if (!ds_wait(&c.full[r.s], r.ph, &c.abort)) return false;
+      tc_fence_after();
+      const uint32_t st = smem_u32(smem + (size_t)r.s * p.stage_bytes);
+      const uint32_t sb = st + (uint32_t)p.kbs * 128u * 128u;
+      for (int j = 0; j < nk; ++j) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          tc_mma_i8(dbase, smem_desc_sw128(st + j * 128u * 128u + kk * 32),
+                    smem_desc_sw128(sb + j * plane_bytes + kk * 32), idesc, first ? 0u : 1u);
+          first = false;
+        }
+      }
+      tc_commit(&c.empty[r.s]);
+      c.consumed = r.n + 1;
+      r.advance(S);
+    }
+    tc_commit(&c.tfull[a]);
+  }
+  return true;
+}
+
+// Epilogue (warps 2..5): every item of one phase; writes the scaled fp32 partial sums.
+template <bool kGateUp>
+__device__ bool ds_epilogue(const DecStreamParams& p, DsCtl& c, int pre_idx, int& iter, uint32_t tmem, int warp,
+                            int lane) {
+  const int q = warp & 3;
+  const int N = 2 * p.nt8;
+  DecItem it;
+  for (int L = blockIdx.x; dec_item<kGateUp>(p, c.touched, c.pre[pre_idx], c.ntouched, L, it);
+       L += gridDim.x, ++iter) {
+    const int a = iter & 1;
+    const uint32_t aph = (uint32_t)(iter >> 1) & 1u;
+    const bool got = ds_wait(&c.tfull[a], aph, &c.abort);
+    if (!__all_sync(0xffffffffu, got)) return false;
+    tc_fence_after();
+    const int o = it.tile * 128 + q * 32 + lane;
+    const bool vo = o < p.out_rows;
+    const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * N);
+    const float* es = p.wscale + (size_t)it.e * (2 * p.f + p.d);
+    const float sc = vo ? es[(kGateUp ? it.mat * p.f : 2 * p.f) + o] : 0.f;
+    // columns [0, nt8) hold the hi plane, [nt8, 2 nt8) the lo plane of the same tokens
+    for (int j = 0; j < p.nt8; j += (p.nt8 == 8 ? 8 : 16)) {
+      float hi[16], lo[16];
+      if (p.nt8 == 8) {  // one load: columns 0-7 hi, 8-15 lo
+        float v[16];
+        tmem_ld16(tb, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          hi[i] = (float)__float_as_int(v[i]);
+          lo[i] = (float)__float_as_int(v[8 + i]);
+        }
+      } else {
+        float vh[16], vl[16];
+        tmem_ld16(tb + j, vh);
+        tmem_ld16(tb + p.nt8 + j, vl);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          hi[i] = (float)__float_as_int(vh[i]);
+          lo[i] = (float)__float_as_int(vl[i]);
+        }
+      }
+      const int width = p.nt8 == 8 ? 8 : 16;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int t = j + i;
+        if (i >= width || t >= it.ntok || !vo) continue;
+        const int row = it.row0 + t;
+        const float v = sc * p.rscale[(size_t)it.split * p.rscale_split_stride + row] * (hi[i] + lo[i] * (1.0f / 254.0f));
+        if (kGateUp) p.GU[(((size_t)it.split * 2 + it.mat) * p.R + row) * p.f + o] = v;
+        else p.Ypart[((size_t)it.split * p.R + row) * p.d + o] = v;
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&c.tempty[a]);
+  }
+  return true;
+}
+
+// Barriers, TMEM and the touched experts with their item prefixes.  Returns the TMEM base.
+__device__ __forceinline__ void ds_prologue(const DecStreamParams* const* phases, int nphases, uint8_t* smem, DsCtl& c,
+                                            int S) {
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&c.full[s], 1);
+      mbar_init(&c.empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&c.tfull[a], 1);
+      mbar_init(&c.tempty[a], 4);
+    }
+    mbar_init(&c.drain, 1);
+    c.abort = 0;
+    c.issued = 0;
+    c.consumed = 0;
+    c.flag = 0;
+    mbar_fence_init();
+    for (int i = 0; i < nphases; ++i) {
+      tma_prefetch_desc(&phases[i]->mapW);
+      tma_prefetch_desc(&phases[i]->mapHi);
+      tma_prefetch_desc(&phases[i]->mapLo);
+    }
+  }
+  // Everything below may read what earlier kernels wrote.  TMEM is allocated only after the
+  // wait too: the previous kernel has then released its own columns, so two kernels of the
+  // chain never hold TMEM on one SM at the same time.
+  pdl_wait();
+  if (warp == 1) {
+    tmem_alloc(&c.tmem, kDsTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  if (threadIdx.x == 0) {
+    const DecStreamParams& p0 = *phases[0];
+    int n = 0;
+    int acc[2] = {0, 0};
+    for (int e = 0; e < p0.E; ++e) {
+      const int cnt = p0.offsets[e + 1] - p0.offsets[e];
+      if (cnt <= 0) continue;
+      c.touched[n] = e;
+      for (int i = 0; i < nphases; ++i) {
+        const DecStreamParams& p = *phases[i];
+        const bool gateup = p.GU != nullptr;
+        c.pre[i][n] = acc[i];
+        acc[i] += (p.out_rows + 127) / 128 * (gateup ? 2 : 1) * p.nsplit * ((cnt + p.nt8 - 1) / p.nt8);
+      }
+      ++n;
+    }
+    for (int i = 0; i < nphases; ++i) c.pre[i][n] = acc[i];
+    c.ntouched = n;
+  }
+  __syncthreads();
+  tc_fence_after();
+}
+
+// Copies issued but never consumed (error path): wait (bounded) until they land; then free TMEM.
+__device__ __forceinline__ void ds_teardown(DsCtl& c, int S) {
+  __syncthreads();
+  if (threadIdx.x == 0 && c.abort) {
+    for (int i = c.consumed; i < c.issued; ++i)
+      if (!mbar_wait_bounded(&c.full[i % S], (uint32_t)(i / S) & 1u)) break;
+  }
+  __syncthreads();
+  if ((threadIdx.x >> 5) == 1) {
+    tc_fence_after();
+    tmem_dealloc(c.tmem, kDsTmemCols);
+  }
+}
+
 template <bool kGateUp>
 __global__ void __launch_bounds__(kDsThreads, 1) dec_stream_kernel(const __grid_constant__ DecStreamParams p) {
-  constexpr int NMAT = 1;  // one weight tile per item (W1 and W3 tiles of gate/up are separate items)
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {
     pdl_wait();
@@ -189,239 +478,272 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_stream_kernel(const __grid_
     return;
   }
   const int S = p.stages;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * p.stage_bytes);
-  uint64_t* empty = full + S;
-  uint64_t* tfull = empty + S;    // [2]
-  uint64_t* tempty = tfull + 2;   // [2]
-  uint64_t* drain = tempty + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  int32_t* ntouched_s = reinterpret_cast<int32_t*>(tmem_holder + 2);
-  int32_t* issued_s = ntouched_s + 1;   // copies issued / stages consumed, for the error path
-  int32_t* consumed_s = ntouched_s + 2;
-  int32_t* touched = ntouched_s + 3;             // [E]
-  int32_t* item_prefix = touched + kMaxExperts;  // [E + 1]
+  DsCtl& c = *reinterpret_cast<DsCtl*>(smem + (size_t)S * p.stage_bytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
-    }
-    mbar_init(drain, 1);
-    *abort_flag = 0;
-    *issued_s = 0;
-    *consumed_s = 0;
-    mbar_fence_init();
-    tma_prefetch_desc(&p.mapW);
-    tma_prefetch_desc(&p.mapHi);
-    tma_prefetch_desc(&p.mapLo);
-  }
-  // Everything below may read what earlier kernels wrote.  TMEM is allocated only after the
-  // wait too: the previous kernel has then released its own columns, so two kernels of the
-  // chain never hold TMEM on one SM at the same time.
-  pdl_wait();
-  if (warp == 1) {
-    tmem_alloc(tmem_holder, kDsTmemCols);
-    tmem_relinquish();
-    tc_fence_before();
-  }
-  if (threadIdx.x == 0) {
-    // touched experts and the prefix of their work items
-    const int tiles = (p.out_rows + 127) / 128;
-    int n = 0, acc = 0;
-    for (int e = 0; e < p.E; ++e) {
-      const int cnt = p.offsets[e + 1] - p.offsets[e];
-      if (cnt <= 0) continue;
-      touched[n] = e;
-      item_prefix[n] = acc;
-      acc += tiles * (kGateUp ? 2 : 1) * p.nsplit * ((cnt + p.nt8 - 1) / p.nt8);
-      ++n;
-    }
-    item_prefix[n] = acc;
-    *ntouched_s = n;
-  }
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
-  const int ntouched = *ntouched_s;
-  const int N = 2 * p.nt8;
-  const uint32_t a_bytes = 128u * 128u;
-
+  const DecStreamParams* phases[1] = {&p};
+  ds_prologue(phases, 1, smem, c, S);
+  const uint32_t tmem = c.tmem;
   if (warp == 0) {
-    // ------------------------------------------------------------- TMA producer
     if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0;
-      const uint32_t tx = NMAT * a_bytes + (uint32_t)N * 128u;
-      int issued = 0;
-      bool ok = true;
-      DecItem it;
-      for (int L = blockIdx.x; ok && dec_item<kGateUp>(p, touched, item_prefix, ntouched, L, it); L += gridDim.x) {
-        // The item's K blocks start at a rotated block (item index mod block count): items in
-        // flight at the same time then read different column offsets of their weight rows, which
-        // spreads the requests over the DRAM channels instead of hitting the same address bits
-        // everywhere.  The accumulation is exact int32, so the block order does not matter.
-        const int kbeg = it.split * p.kspan, kend = min(p.K, kbeg + p.kspan);
-        const int nkb = (kend - kbeg + 127) / 128;
-        int kb = L % nkb;
-        for (int i = 0; i < nkb; ++i, kb = (kb + 1 == nkb) ? 0 : kb + 1) {
-          const int kx = kbeg + kb * 128;
-          if (!ds_wait(&empty[s], ph ^ 1u, abort_flag)) {
-            ok = false;
-            break;
-          }
-          uint8_t* st = smem + (size_t)s * p.stage_bytes;
-          mbar_arrive_expect_tx(&full[s], tx);
-          if (kGateUp) tma_load_4d(st, &p.mapW, &full[s], kx, it.tile * 128, it.mat, it.e);
-          else tma_load_3d(st, &p.mapW, &full[s], kx, it.tile * 128, it.e);
-          uint8_t* sb = st + NMAT * a_bytes;
-          tma_load_2d(sb, &p.mapHi, &full[s], kx, it.row0);
-          tma_load_2d(sb + p.nt8 * 128, &p.mapLo, &full[s], kx, it.row0);
-          ++issued;
-          if (++s == S) {
-            s = 0;
-            ph ^= 1u;
-          }
-        }
-      }
-      if (!ok) {
-        *abort_flag = 1;
-        atomicOr(p.err, kErrWaitTimeout);
-      }
-      *issued_s = issued;
+      DsRing r;
+      if (!ds_produce<kGateUp>(p, smem, c, S, 0, r, false, [] { return true; })) ds_abort(c, p.err);
     }
     pdl_trigger();  // every copy of this CTA is issued: let the next kernel be scheduled
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_s8_s32(128, N);
-      int s = 0;
-      uint32_t ph = 0;
-      int iter = 0, consumed = 0;
-      bool ok = true;
-      DecItem it;
-      for (int L = blockIdx.x; ok && dec_item<kGateUp>(p, touched, item_prefix, ntouched, L, it);
-           L += gridDim.x, ++iter) {
-        const int a = iter & 1;
-        const uint32_t aph = (uint32_t)(iter >> 1) & 1u;
-        if (!ds_wait(&tempty[a], aph ^ 1u, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t dbase = tmem + (uint32_t)(a * NMAT * N);
-        const int kbeg = it.split * p.kspan, kend = min(p.K, kbeg + p.kspan);
-        bool first = true;
-        for (int kx = kbeg; kx < kend; kx += 128) {
-          if (!ds_wait(&full[s], ph, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t st = smem_u32(smem + (size_t)s * p.stage_bytes);
-          const uint32_t sb = st + NMAT * a_bytes;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-#pragma unroll
-            for (int m = 0; m < NMAT; ++m)
-              tc_mma_i8(dbase + (uint32_t)(m * N), smem_desc_sw128(st + m * a_bytes + kk * 32),
-                        smem_desc_sw128(sb + kk * 32), idesc, (first && kk == 0) ? 0u : 1u);
-          }
-          first = false;
-          tc_commit(&empty[s]);
-          ++consumed;
-          if (++s == S) {
-            s = 0;
-            ph ^= 1u;
-          }
-        }
-        if (!ok) break;
-        tc_commit(&tfull[a]);
-      }
-      if (!ok) {
-        *abort_flag = 1;
-        atomicOr(p.err, kErrWaitTimeout);
-      }
-      *consumed_s = consumed;
-      tc_commit(drain);
-      mbar_wait_bounded(drain, 0);
+      DsRing r;
+      int iter = 0;
+      if (!ds_mma<kGateUp>(p, smem, c, S, 0, r, iter, tmem)) ds_abort(c, p.err);
+      tc_commit(&c.drain);  // wait until every MMA issued by this thread has completed
+      mbar_wait_bounded(&c.drain, 0);
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------- epilogue (warps 2..5)
-    const int q = warp & 3;
     int iter = 0;
-    DecItem it;
-    for (int L = blockIdx.x; dec_item<kGateUp>(p, touched, item_prefix, ntouched, L, it); L += gridDim.x, ++iter) {
-      const int a = iter & 1;
-      const uint32_t aph = (uint32_t)(iter >> 1) & 1u;
-      const bool got = ds_wait(&tfull[a], aph, abort_flag);
-      if (!__all_sync(0xffffffffu, got)) break;
-      tc_fence_after();
-      const int o = it.tile * 128 + q * 32 + lane;
-      const bool vo = o < p.out_rows;
-      const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * NMAT * N);
-      const float* es = p.wscale + (size_t)it.e * (2 * p.f + p.d);
-      const float sc = vo ? es[(kGateUp ? it.mat * p.f : 2 * p.f) + o] : 0.f;
-      // columns [0, nt8) hold the hi plane, [nt8, 2 nt8) the lo plane of the same tokens
-      for (int j = 0; j < p.nt8; j += (p.nt8 == 8 ? 8 : 16)) {
-        float hi[NMAT][16], lo[NMAT][16];
-#pragma unroll
-        for (int m = 0; m < NMAT; ++m) {
-          if (p.nt8 == 8) {  // one load: columns 0-7 hi, 8-15 lo
-            float v[16];
-            tmem_ld16(tb + m * N, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              hi[m][i] = (float)__float_as_int(v[i]);
-              lo[m][i] = (float)__float_as_int(v[8 + i]);
-            }
-          } else {
-            float vh[16], vl[16];
-            tmem_ld16(tb + m * N + j, vh);
-            tmem_ld16(tb + m * N + p.nt8 + j, vl);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              hi[m][i] = (float)__float_as_int(vh[i]);
-              lo[m][i] = (float)__float_as_int(vl[i]);
-            }
+    if (!ds_epilogue<kGateUp>(p, c, 0, iter, tmem, warp, lane) && lane == 0) ds_abort(c, p.err);
+  }
+  ds_teardown(c, S);
+}
+
+// ------------------------------------------------------------------------- fused decode kernel
+// The whole int8 expert stage in one cooperative launch (all CTAs resident, one per SM):
+//   phase 1  gate/up weight stream -> GU partials                 (as dec_stream_kernel<true>)
+//   barrier
+//   phase 2  H = silu(g) * u -> int8 planes (epilogue warps, one (row, down split) unit at a
+//            time; no shared-memory row buffer: the values are recomputed for the split pass),
+//            while the producer already streams the first ring-full of down weights
+//   barrier
+//   phase 3  down weight stream -> Ypart                            (as dec_stream_kernel<false>)
+//   barrier
+//   phase 4  y[t] = sum_j w[t][j] * sum_split Ypart[split][dst_row[t][j]]  (fixed order)
+// Grid barriers are arrival counters in global memory with bounded waits; the last CTA to
+// leave resets them for the next launch.  One launch replaces four, the down stream starts
+// with a full ring, and no kernel boundary separates the phases.
+struct alignas(64) DecFusedParams {
+  DecStreamParams gu;       // phase 1 (GU output)
+  DecStreamParams dn;       // phase 3 (Ypart output); its planes are written by phase 2
+  int8_t* hhi;              // H planes [R, f] and their scales [dsplit, R]
+  int8_t* hlo;
+  float* hscale;
+  const int32_t* dst_row;   // [T, k]
+  const float* topk_w;      // [T, k]
+  int T, k;
+  __nv_bfloat16* y;         // [T, d]
+  int32_t* bar;             // [4] arrival counters, zero between launches
+};
+
+__device__ __forceinline__ int ld_acquire(const int32_t* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+// Wait (bounded) until `*ctr` reaches `target`.
+__device__ bool grid_wait(const int32_t* ctr, int target, volatile int* abort_flag) {
+  const unsigned long long t0 = global_ns();
+  while (ld_acquire(ctr) < target) {
+    if (*abort_flag) return false;
+    if (global_ns() - t0 > kWaitTimeoutNs) return false;
+    __nanosleep(128);
+  }
+  return true;
+}
+
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_constant__ DecFusedParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int S = p.gu.stages;
+  DsCtl& c = *reinterpret_cast<DsCtl*>(smem + (size_t)S * p.gu.stage_bytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = gridDim.x;
+  const bool aligned = (smem_u32(smem) & 1023u) == 0;  // the 128-byte swizzle needs 1024-byte stages
+  const DecStreamParams* phases[2] = {&p.gu, &p.dn};
+  if (aligned) ds_prologue(phases, 2, smem, c, S);
+  const uint32_t tmem = aligned ? c.tmem : 0u;
+  if (!aligned) {
+    if (threadIdx.x == 0) {  // report, and arrive at every barrier so the other CTAs do not wait
+      atomicOr(p.gu.err, kErrWaitTimeout);
+      for (int b = 0; b < 3; ++b) atomicAdd(&p.bar[b], 1);
+    }
+  } else if (warp == 0) {
+    if (lane == 0) {
+      DsRing r;
+      bool ok = ds_produce<true>(p.gu, smem, c, S, 0, r, false, [] { return true; });
+      // down weights go out at once; their plane copies wait for phase 2 of every CTA
+      if (ok)
+        ok = ds_produce<false>(p.dn, smem, c, S, 1, r, true, [&] {
+          if (!grid_wait(&p.bar[1], G, &c.abort)) return false;
+          fence_proxy_async_global();
+          return true;
+        });
+      if (!ok) ds_abort(c, p.gu.err);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      DsRing r;
+      int iter = 0;
+      bool ok = ds_mma<true>(p.gu, smem, c, S, 0, r, iter, tmem);
+      if (ok) ok = ds_mma<false>(p.dn, smem, c, S, 1, r, iter, tmem);
+      if (!ok) ds_abort(c, p.gu.err);
+      tc_commit(&c.drain);
+      mbar_wait_bounded(&c.drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------- epilogue warps: phases 1-4
+    const int tid = threadIdx.x - 64;  // 0..127
+    int iter = 0;
+    // Grid barrier over the epilogue warps of every CTA: each CTA arrives exactly once (also
+    // after an error, so that the others are not kept waiting); the result is the same for all
+    // four warps of a CTA (false once this CTA has aborted or the wait gave up).
+    auto grid_barrier = [&](int idx) -> bool {
+      epi_sync();
+      if (tid == 0) {
+        __threadfence();
+        atomicAdd(&p.bar[idx], 1);
+        c.flag = (!c.abort && grid_wait(&p.bar[idx], G, &c.abort)) ? 1 : 0;
+        if (!c.flag && !c.abort) ds_abort(c, p.gu.err);
+      }
+      epi_sync();
+      return *(volatile int*)&c.flag != 0;
+    };
+    bool ok = ds_epilogue<true>(p.gu, c, 0, iter, tmem, warp, lane);
+    if (!__all_sync(0xffffffffu, ok) && lane == 0) ds_abort(c, p.gu.err);
+    // barrier 1: every CTA's GU partials are written
+    ok = grid_barrier(0);
+    if (ok) {
+      // phase 2: H planes, one (row, down split) unit per round
+      float* red = c.red;
+      const int R = p.gu.R, f = p.gu.f, gs = p.gu.nsplit, ds = p.dn.nsplit;
+      const size_t plane = (size_t)R * f;
+      const int span = f / ds;
+      for (int u = blockIdx.x; u < R * ds; u += G) {
+        const int r = u / ds, sp = u - r * ds, k0 = sp * span;
+        const float* g0 = p.gu.GU + (size_t)r * f + k0;
+        float mx = 0.f;
+        for (int j = tid * 4; j < span; j += 128 * 4) {
+          float4 g = __ldcg(reinterpret_cast<const float4*>(g0 + j));
+          float4 uu = __ldcg(reinterpret_cast<const float4*>(g0 + plane + j));
+          for (int s2 = 1; s2 < gs; ++s2) {
+            const float4 a = __ldcg(reinterpret_cast<const float4*>(g0 + (size_t)(2 * s2) * plane + j));
+            const float4 b = __ldcg(reinterpret_cast<const float4*>(g0 + (size_t)(2 * s2 + 1) * plane + j));
+            g.x += a.x; g.y += a.y; g.z += a.z; g.w += a.w;
+            uu.x += b.x; uu.y += b.y; uu.z += b.z; uu.w += b.w;
           }
+          const float h0 = __bfloat162float(__float2bfloat16_rn(silu_mul(g.x, uu.x)));
+          const float h1 = __bfloat162float(__float2bfloat16_rn(silu_mul(g.y, uu.y)));
+          const float h2 = __bfloat162float(__float2bfloat16_rn(silu_mul(g.z, uu.z)));
+          const float h3 = __bfloat162float(__float2bfloat16_rn(silu_mul(g.w, uu.w)));
+          mx = fmaxf(mx, fmaxf(fmaxf(fabsf(h0), fabsf(h1)), fmaxf(fabsf(h2), fabsf(h3))));
         }
-        const int width = p.nt8 == 8 ? 8 : 16;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int t = j + i;
-          if (i >= width || t >= it.ntok || !vo) continue;
-          const int row = it.row0 + t;
-          const float v = sc * p.rscale[(size_t)it.split * p.rscale_split_stride + row] *
-                          (hi[0][i] + lo[0][i] * (1.0f / 254.0f));
-          if (kGateUp) p.GU[(((size_t)it.split * 2 + it.mat) * p.R + row) * p.f + o] = v;
-          else p.Ypart[((size_t)it.split * p.R + row) * p.d + o] = v;
+        for (int off = 16; off; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        if (lane == 0) red[tid >> 5] = mx;
+        epi_sync();
+        mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+        epi_sync();  // red[] is rewritten by the next unit
+        const float a = plane_scale(mx), inv_a = __frcp_rn(a);  // correctly rounded 1 / a
+        if (tid == 0) p.hscale[(size_t)sp * R + r] = a;
+        int8_t* hrow = p.hhi + (size_t)r * f + k0;
+        int8_t* lrow = p.hlo + (size_t)r * f + k0;
+        for (int j = tid * 4; j < span; j += 128 * 4) {  // the same values again, now split
+          float4 g = __ldcg(reinterpret_cast<const float4*>(g0 + j));
+          float4 uu = __ldcg(reinterpret_cast<const float4*>(g0 + plane + j));
+          for (int s2 = 1; s2 < gs; ++s2) {
+            const float4 a2 = __ldcg(reinterpret_cast<const float4*>(g0 + (size_t)(2 * s2) * plane + j));
+            const float4 b2 = __ldcg(reinterpret_cast<const float4*>(g0 + (size_t)(2 * s2 + 1) * plane + j));
+            g.x += a2.x; g.y += a2.y; g.z += a2.z; g.w += a2.w;
+            uu.x += b2.x; uu.y += b2.y; uu.z += b2.z; uu.w += b2.w;
+          }
+          const float hv[4] = {__bfloat162float(__float2bfloat16_rn(silu_mul(g.x, uu.x))),
+                               __bfloat162float(__float2bfloat16_rn(silu_mul(g.y, uu.y))),
+                               __bfloat162float(__float2bfloat16_rn(silu_mul(g.z, uu.z))),
+                               __bfloat162float(__float2bfloat16_rn(silu_mul(g.w, uu.w)))};
+          uint32_t hw = 0u, lw = 0u;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            int qh, ql;
+            split_planes(hv[i], a, inv_a, qh, ql);
+            hw |= ((uint32_t)qh & 0xffu) << (8 * i);
+            lw |= ((uint32_t)ql & 0xffu) << (8 * i);
+          }
+          *reinterpret_cast<uint32_t*>(hrow + j) = hw;
+          *reinterpret_cast<uint32_t*>(lrow + j) = lw;
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[a]);
+      fence_proxy_async_global();  // the planes are read next by TMA copies of other CTAs
+    }
+    // barrier 2: every CTA's H planes are written (the producer waits on the same counter)
+    ok = grid_barrier(1);
+    if (ok) ok = ds_epilogue<false>(p.dn, c, 1, iter, tmem, warp, lane);
+    if (!__all_sync(0xffffffffu, ok) && lane == 0) ds_abort(c, p.gu.err);
+    // barrier 3: every CTA's down partials are written
+    ok = grid_barrier(2);
+    if (ok) {
+      // phase 4: combine, one thread per (token, 4 consecutive outputs)
+      const int d = p.dn.d, ns = p.dn.nsplit, k = p.k;
+      const size_t ss = (size_t)p.dn.R * d;
+      const int chunks = d >> 2;
+      for (long long qi = (long long)blockIdx.x * 128 + tid; qi < (long long)p.T * chunks; qi += (long long)G * 128) {
+        const int t = (int)(qi / chunks), cc = (int)(qi - (long long)t * chunks) * 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < k; ++j) {
+          const int rr = p.dst_row[(size_t)t * k + j];
+          const float wj = p.topk_w[(size_t)t * k + j];
+          const float* base = p.dn.Ypart + (size_t)rr * d + cc;
+          float4 part = make_float4(0.f, 0.f, 0.f, 0.f);
+          int sp = 0;
+          for (; sp + 4 <= ns; sp += 4) {
+            float4 v[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) v[i] = __ldcg(reinterpret_cast<const float4*>(base + (size_t)(sp + i) * ss));
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              part.x += v[i].x; part.y += v[i].y; part.z += v[i].z; part.w += v[i].w;
+            }
+          }
+          for (; sp < ns; ++sp) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(base + (size_t)sp * ss));
+            part.x += v.x; part.y += v.y; part.z += v.z; part.w += v.w;
+          }
+          acc.x = fmaf(wj, part.x, acc.x);
+          acc.y = fmaf(wj, part.y, acc.y);
+          acc.z = fmaf(wj, part.z, acc.z);
+          acc.w = fmaf(wj, part.w, acc.w);
+        }
+        const __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x, acc.y), hi2 = __floats2bfloat162_rn(acc.z, acc.w);
+        uint2 pk;
+        pk.x = (uint32_t)__bfloat16_as_ushort(lo2.x) | ((uint32_t)__bfloat16_as_ushort(lo2.y) << 16);
+        pk.y = (uint32_t)__bfloat16_as_ushort(hi2.x) | ((uint32_t)__bfloat16_as_ushort(hi2.y) << 16);
+        *reinterpret_cast<uint2*>(p.y + (size_t)t * d + cc) = pk;
+      }
     }
   }
-  __syncthreads();
-  if (threadIdx.x == 0 && *abort_flag) {
-    // copies issued but never consumed: wait (bounded) until they land before the CTA exits
-    for (int i = *consumed_s; i < *issued_s; ++i) mbar_wait_bounded(&full[i % S], (uint32_t)(i / S) & 1u);
+  if (aligned) ds_teardown(c, S);
+  else __syncthreads();
+  // exit ticket: the last CTA to leave resets the counters for the next launch
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(&p.bar[3], 1) == G - 1) {
+      p.bar[0] = 0;
+      p.bar[1] = 0;
+      p.bar[2] = 0;
+      p.bar[3] = 0;
+      __threadfence();
+    }
   }
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kDsTmemCols);
-  }
+}
+
+// K blocks per ring stage: COLIBRI_DEC_KB (1..4), default 2.
+int dec_kbs() {
+  const char* v = getenv("COLIBRI_DEC_KB");
+  const int k = v ? atoi(v) : 2;
+  return k < 1 ? 1 : (k > kDsMaxKbs ? kDsMaxKbs : k);
 }
 
 int dec_nt8(int max_rows_per_expert) { return max_rows_per_expert <= 8 ? 8 : (max_rows_per_expert <= 16 ? 16 : 32); }
@@ -437,40 +759,48 @@ int sm_count_current() {
   return sms;
 }
 
-template <bool kGateUp>
-cudaError_t launch_stream(DecStreamParams& p, const int8_t* hi, const int8_t* lo, int K, cudaStream_t s) {
-  constexpr int NMAT = 1;
+bool plane_maps(DecStreamParams& p, const int8_t* hi, const int8_t* lo, int K) {
   const uint64_t pd[2] = {(uint64_t)K, (uint64_t)p.R}, ps[1] = {(uint64_t)K};
   const uint32_t pb[2] = {128, (uint32_t)p.nt8};
-  if (!make_tmap(&p.mapHi, CU_TENSOR_MAP_DATA_TYPE_UINT8, hi, 2, pd, ps, pb)) return cudaErrorInvalidValue;
-  if (!make_tmap(&p.mapLo, CU_TENSOR_MAP_DATA_TYPE_UINT8, lo, 2, pd, ps, pb)) return cudaErrorInvalidValue;
-  p.stage_bytes = (uint32_t)(NMAT * 128 * 128 + 2 * p.nt8 * 128);
+  if (!make_tmap(&p.mapHi, CU_TENSOR_MAP_DATA_TYPE_UINT8, hi, 2, pd, ps, pb)) return false;
+  if (!make_tmap(&p.mapLo, CU_TENSOR_MAP_DATA_TYPE_UINT8, lo, 2, pd, ps, pb)) return false;
+  p.kbs = dec_kbs();
+  p.stage_bytes = (uint32_t)(p.kbs * (128 * 128 + 2 * p.nt8 * 128));
   p.stages = (int)std::min<size_t>(kDsMaxStages, kDsRingBytes / p.stage_bytes);
-  const size_t smem = (size_t)p.stages * p.stage_bytes + 4096;
+  return true;
+}
+
+template <bool kGateUp>
+cudaError_t launch_stream(const DecStreamParams& p, cudaStream_t s) {
+  const size_t smem = (size_t)p.stages * p.stage_bytes + kDsCtlBytes;
   return launch_kernel(dec_stream_kernel<kGateUp>, dim3(sm_count_current()), dim3(kDsThreads), smem, s, 1, p);
 }
 
 }  // namespace
 
 cudaError_t configure_dec_kernels() {
-  const int smem = (int)(kDsRingBytes + 4096);
+  const int smem = (int)(kDsRingBytes + kDsCtlBytes);
   cudaError_t e = cudaFuncSetAttribute(dec_stream_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(dec_stream_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(dec_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(dec_finish_h_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFinishMaxSmem);
   return e;
 }
 
-cudaError_t launch_dec_gateup(const int8_t* Xhi, const int8_t* Xlo, const float* xscale, const int8_t* W,
-                              const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
-                              int nsplit, float* GU, int R, int max_rows_per_expert, uint32_t* err, cudaStream_t s) {
-  DecStreamParams p;
+namespace {
+
+// Parameters of one stream phase (weights, planes, scales, outputs); false if a tensor map
+// cannot be encoded.
+bool dec_gateup_params(DecStreamParams& p, const int8_t* Xhi, const int8_t* Xlo, const float* xscale, const int8_t* W,
+                       const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets, int nsplit,
+                       float* GU, int R, int max_rows_per_expert, uint32_t* err) {
   memset(&p, 0, sizeof(p));
   const uint64_t dims[4] = {(uint64_t)d, (uint64_t)f, 2, (uint64_t)E};
   const uint64_t st[3] = {(uint64_t)d, (uint64_t)f * d, (uint64_t)wstride};
   const uint32_t box[4] = {128, 128, 1, 1};
-  if (!make_tmap(&p.mapW, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, 4, dims, st, box)) return cudaErrorInvalidValue;
+  if (!make_tmap(&p.mapW, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, 4, dims, st, box)) return false;
   p.wscale = scales;
   p.rscale = xscale;
   p.offsets = offsets;
@@ -485,7 +815,45 @@ cudaError_t launch_dec_gateup(const int8_t* Xhi, const int8_t* Xlo, const float*
   p.R = R;
   p.GU = GU;
   p.err = err;
-  return launch_stream<true>(p, Xhi, Xlo, d, s);
+  return plane_maps(p, Xhi, Xlo, d);
+}
+
+bool dec_down_params(DecStreamParams& p, const int8_t* Hhi, const int8_t* Hlo, const float* hscale, const int8_t* W,
+                     const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets, int nsplit,
+                     int R, float* Ypart, int max_rows_per_expert, uint32_t* err) {
+  memset(&p, 0, sizeof(p));
+  const uint64_t dims[3] = {(uint64_t)f, (uint64_t)d, (uint64_t)E};
+  const uint64_t st[2] = {(uint64_t)f, (uint64_t)wstride};
+  const uint32_t box[3] = {128, 128, 1};
+  if (!make_tmap(&p.mapW, CU_TENSOR_MAP_DATA_TYPE_UINT8, W + 2 * (size_t)f * d, 3, dims, st, box)) return false;
+  p.wscale = scales;
+  p.rscale = hscale;
+  p.rscale_split_stride = R;
+  p.offsets = offsets;
+  p.E = E;
+  p.d = d;
+  p.f = f;
+  p.out_rows = d;
+  p.K = f;
+  p.nsplit = nsplit;
+  p.kspan = f / nsplit;
+  p.nt8 = dec_nt8(max_rows_per_expert);
+  p.R = R;
+  p.Ypart = Ypart;
+  p.err = err;
+  return plane_maps(p, Hhi, Hlo, f);
+}
+
+}  // namespace
+
+cudaError_t launch_dec_gateup(const int8_t* Xhi, const int8_t* Xlo, const float* xscale, const int8_t* W,
+                              const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
+                              int nsplit, float* GU, int R, int max_rows_per_expert, uint32_t* err, cudaStream_t s) {
+  DecStreamParams p;
+  if (!dec_gateup_params(p, Xhi, Xlo, xscale, W, scales, wstride, d, f, E, offsets, nsplit, GU, R,
+                         max_rows_per_expert, err))
+    return cudaErrorInvalidValue;
+  return launch_stream<true>(p, s);
 }
 
 cudaError_t launch_dec_finish_h(const float* GU, int gsplit, int R, int f, int dsplit, int8_t* hi, int8_t* lo,
@@ -503,28 +871,47 @@ cudaError_t launch_dec_down(const int8_t* Hhi, const int8_t* Hlo, const float* h
                             int nsplit, int R, float* Ypart, int max_rows_per_expert, uint32_t* err,
                             cudaStream_t s) {
   DecStreamParams p;
-  memset(&p, 0, sizeof(p));
-  const uint64_t dims[3] = {(uint64_t)f, (uint64_t)d, (uint64_t)E};
-  const uint64_t st[2] = {(uint64_t)f, (uint64_t)wstride};
-  const uint32_t box[3] = {128, 128, 1};
-  if (!make_tmap(&p.mapW, CU_TENSOR_MAP_DATA_TYPE_UINT8, W + 2 * (size_t)f * d, 3, dims, st, box))
+  if (!dec_down_params(p, Hhi, Hlo, hscale, W, scales, wstride, d, f, E, offsets, nsplit, R, Ypart,
+                       max_rows_per_expert, err))
     return cudaErrorInvalidValue;
-  p.wscale = scales;
-  p.rscale = hscale;
-  p.rscale_split_stride = R;
-  p.offsets = offsets;
-  p.E = E;
-  p.d = d;
-  p.f = f;
-  p.out_rows = d;
-  p.K = f;
-  p.nsplit = nsplit;
-  p.kspan = f / nsplit;
-  p.nt8 = dec_nt8(max_rows_per_expert);
-  p.R = R;
-  p.Ypart = Ypart;
-  p.err = err;
-  return launch_stream<false>(p, Hhi, Hlo, f, s);
+  return launch_stream<false>(p, s);
+}
+
+cudaError_t launch_dec_fused(const DecFusedArgs& a, cudaStream_t s) {
+  if (a.T <= 0) return cudaSuccess;
+  if (a.f % a.dsplit != 0 || (a.f / a.dsplit) % 4 != 0 || a.d % 4 != 0) return cudaErrorInvalidValue;
+  DecFusedParams p;
+  memset(&p, 0, sizeof(p));
+  const int R = a.T * a.k;
+  if (!dec_gateup_params(p.gu, a.planes_hi, a.planes_lo, a.planes_scale, a.W, a.scales, a.wstride, a.d, a.f, a.E,
+                         a.offsets, a.gsplit, a.GU, R, a.T, a.err) ||
+      !dec_down_params(p.dn, a.planes_hi, a.planes_lo, a.planes_scale, a.W, a.scales, a.wstride, a.d, a.f, a.E,
+                       a.offsets, a.dsplit, R, a.Ypart, a.T, a.err))
+    return cudaErrorInvalidValue;
+  p.hhi = a.planes_hi;
+  p.hlo = a.planes_lo;
+  p.hscale = a.planes_scale;
+  p.dst_row = a.dst_row;
+  p.topk_w = a.topk_w;
+  p.T = a.T;
+  p.k = a.k;
+  p.y = a.y;
+  p.bar = a.bar;
+  const size_t smem = (size_t)p.gu.stages * p.gu.stage_bytes + kDsCtlBytes;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(sm_count_current());
+  cfg.blockDim = dim3(kDsThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: the grid barriers need it
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  launch_chain_break();  // an ordinary launch: the next one must not overlap it
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, dec_fused_kernel, p);
+  launch_chain_break();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace colibri

@@ -119,7 +119,7 @@ extern "C" colibri_status colibri_route_noalloc(const void* x, int32_t act_dtype
   if (e == cudaSuccess)
     e = launch_route_scan(blk_counts, (int)nblk, num_experts, kTcBM, blk_base, counts, offsets, mt_prefix, s);
   if (e == cudaSuccess)
-    e = launch_route_scatter(x, act_dtype, T, d_model, top_k, num_experts, topk_idx, blk_base, dst_row,
+    e = launch_route_scatter(x, act_dtype, T, d_model, top_k, num_experts, topk_idx, blk_base, offsets, dst_row,
                              src_row, Xp, nullptr, s);
   if (e != cudaSuccess) return nf_fail(COLIBRI_ERR_CUDA, cudaGetErrorString(e));
   return COLIBRI_OK;

@@ -9,8 +9,8 @@
 //                  32 lanes (tokens) that chose that expert; a token's rank among the earlier
 //                  tokens of its warp is popc(mask & lanes_below); warps are then prefixed in
 //                  order, giving the rank inside the 256-token block and the block's counts.
-//   route_scan     one CTA: per expert, exclusive prefix over blocks; counts; offsets[E+1];
-//                  and the m-tile prefix the grouped GEMM schedules from.
+//   route_scan     one CTA: per expert, exclusive prefix over blocks; counts; offsets[E+1]
+//                  and the m-tile prefix the grouped GEMM schedules from (scans over experts).
 //   route_scatter  one warp per token: final row = offsets[e] + block base + rank; writes
 //                  src_row / dst_row and copies the token's row into each of its k grouped
 //                  rows with 16-byte vector loads and stores.
@@ -134,47 +134,64 @@ __global__ void __launch_bounds__(256) route_scan_kernel(const int32_t* __restri
                                                          int32_t* __restrict__ mt_prefix) {
   pdl_trigger();
   pdl_wait();
-  __shared__ int tot[kMaxExperts];
-  __shared__ int off[kMaxExperts + 1];
-  __shared__ int mts[kMaxExperts + 1];
-  const int e = threadIdx.x;
+  __shared__ int wsum[2][8];
+  const int e = threadIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // per expert: exclusive prefix over the blocks, eight block counts in flight at a time
+  int run = 0;
   if (e < E) {
-    int run = 0;
-    for (int b = 0; b < nblk; ++b) {
+    int b = 0;
+    for (; b + 8 <= nblk; b += 8) {
+      int c[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) c[i] = blk_counts[(size_t)(b + i) * E + e];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        blk_base[(size_t)(b + i) * E + e] = run;
+        run += c[i];
+      }
+    }
+    for (; b < nblk; ++b) {
       const int c = blk_counts[(size_t)b * E + e];
       blk_base[(size_t)b * E + e] = run;
       run += c;
     }
-    tot[e] = run;
     counts[e] = run;
   }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int o = 0, mt = 0;
-    for (int q = 0; q < E; ++q) {
-      off[q] = o;
-      mts[q] = mt;
-      o += tot[q];
-      mt += (tot[q] + bm - 1) / bm;
+  // offsets[] and the m-tile prefix: exclusive scans over the experts (warp scans, then warps)
+  const int mt = (run + bm - 1) / bm;
+  int io = run, im = mt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int a = __shfl_up_sync(0xffffffffu, io, o), c = __shfl_up_sync(0xffffffffu, im, o);
+    if (lane >= o) {
+      io += a;
+      im += c;
     }
-    off[E] = o;
-    mts[E] = mt;
+  }
+  if (lane == 31) {
+    wsum[0][warp] = io;
+    wsum[1][warp] = im;
   }
   __syncthreads();
-  for (int q = threadIdx.x; q <= E; q += blockDim.x) {
-    offsets[q] = off[q];
-    mt_prefix[q] = mts[q];
+  int bo = 0, bmt = 0;
+  for (int w = 0; w < warp; ++w) {
+    bo += wsum[0][w];
+    bmt += wsum[1][w];
   }
   if (e < E) {
-    const int base = off[e];
-    for (int b = 0; b < nblk; ++b) blk_base[(size_t)b * E + e] += base;
+    offsets[e] = bo + io - run;
+    mt_prefix[e] = bmt + im - mt;
+  }
+  if (e == E - 1) {
+    offsets[E] = bo + io;
+    mt_prefix[E] = bmt + im;
   }
 }
 
 template <typename Tv>
 __global__ void __launch_bounds__(256) route_scatter_kernel(
     const Tv* __restrict__ x, int T, int vec_per_row, int k, int E, const int32_t* __restrict__ idx,
-    const int32_t* __restrict__ blk_base, int32_t* __restrict__ dst_row,
+    const int32_t* __restrict__ blk_base, const int32_t* __restrict__ offsets, int32_t* __restrict__ dst_row,
     int32_t* __restrict__ src_row, Tv* __restrict__ Xp, RowPlanes P) {
   pdl_trigger();
   pdl_wait();
@@ -185,7 +202,7 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(
     if (lane < k) {
       int e = idx[(size_t)t * k + lane];
       e = min(max(e, 0), E - 1);
-      r = blk_base[(size_t)(t / kCountBlock) * E + e] + dst_row[(size_t)t * k + lane];
+      r = offsets[e] + blk_base[(size_t)(t / kCountBlock) * E + e] + dst_row[(size_t)t * k + lane];
       dst_row[(size_t)t * k + lane] = r;
       src_row[r] = t;
     }
@@ -372,8 +389,9 @@ cudaError_t launch_route_scan(const int32_t* blk_counts, int nblk, int E, int bm
 }
 
 cudaError_t launch_route_scatter(const void* x, int act, int T, int d, int k, int E,
-                                 const int32_t* idx, const int32_t* blk_base, int32_t* dst_row,
-                                 int32_t* src_row, void* Xp, const RowPlanes* planes, cudaStream_t s) {
+                                 const int32_t* idx, const int32_t* blk_base, const int32_t* offsets,
+                                 int32_t* dst_row, int32_t* src_row, void* Xp, const RowPlanes* planes,
+                                 cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
   if (planes && act != COLIBRI_BF16) return cudaErrorInvalidValue;
   const RowPlanes P = planes ? *planes : RowPlanes{nullptr, nullptr, nullptr};
@@ -383,7 +401,7 @@ cudaError_t launch_route_scatter(const void* x, int act, int T, int d, int k, in
   int grid = (T + warps_per_cta - 1) / warps_per_cta;
   if (grid > 4096) grid = 4096;
   return launch_kernel(route_scatter_kernel<uint4>, dim3(grid), dim3(warps_per_cta * 32), 0, s, 1, (const uint4*)x,
-                       T, vec, k, E, idx, blk_base, dst_row, src_row, (uint4*)Xp, P);
+                       T, vec, k, E, idx, blk_base, offsets, dst_row, src_row, (uint4*)Xp, P);
 }
 
 }  // namespace colibri

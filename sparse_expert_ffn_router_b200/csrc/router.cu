@@ -394,12 +394,16 @@ __global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant
         tmem_ld16(tbase + c0, v);
         tmem_ld_wait();
       } else {
+        // the 16 experts' partials of one split are loaded together, then added in split order
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float acc = 0.f;
-          if (t < p.T && c0 + i < p.E)
-            for (int sp = 0; sp < p.ksplit; ++sp) acc += __ldcg(&p.part[((size_t)sp * p.E + c0 + i) * p.T + t]);
-          v[i] = acc;
+        for (int i = 0; i < 16; ++i) v[i] = 0.f;
+        for (int sp = 0; sp < p.ksplit; ++sp) {
+          float pv[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pv[i] = (t < p.T && c0 + i < p.E) ? __ldcg(&p.part[((size_t)sp * p.E + c0 + i) * p.T + t]) : 0.f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] += pv[i];
         }
       }
 #pragma unroll

@@ -51,16 +51,35 @@ def test_small_parity(name):
 BF16_SMALL = [n for n, w in SMALL.items() if w.wdt == BF16]
 
 
-@pytest.mark.parametrize("mode", ["1", "2"])
+@pytest.mark.parametrize("mode", ["1", "2", "s"])
 @pytest.mark.parametrize("name", BF16_SMALL)
 def test_small_parity_each_tile_mode(name, mode, monkeypatch):
-    # "1": one CTA per 128-row tile; "2": clusters of two CTAs with 256-row pair tiles
+    # "1": one CTA per 128-row tile; "2": clusters of two CTAs with 256-row pair tiles;
+    # "s": swapped operands, 128 weight rows x 16..256 token rows
     monkeypatch.setenv("COLIBRI_GEMM_CTA", mode)
     wl = SMALL[name]
     H.parity(inputgen.make_problem(wl, seed=5))
 
 
-@pytest.mark.parametrize("mode", ["1", "2"])
+I8_SMALL = [n for n, w in SMALL.items() if w.wdt == I8]
+
+
+@pytest.mark.parametrize("fused", ["0", "1"])
+@pytest.mark.parametrize("name", I8_SMALL)
+def test_int8_each_launch_plan(name, fused, monkeypatch):
+    # "1": gate/up, H planes, down and combine in one cooperative launch (the default);
+    # "0": the same stages as four launches
+    monkeypatch.setenv("COLIBRI_DEC_FUSED", fused)
+    wl = SMALL[name]
+    p = inputgen.make_problem(wl, seed=9)
+    layer = H.make_layer(wl)
+    t = H.to_device(p)
+    for _ in range(3):  # repeated calls: the fused kernel's grid-barrier counters reset themselves
+        H.parity(p, layer=layer, dev_inputs=t)
+    layer.close()
+
+
+@pytest.mark.parametrize("mode", ["1", "2", "s"])
 def test_mixtral_each_tile_mode(mode, monkeypatch):
     monkeypatch.setenv("COLIBRI_GEMM_CTA", mode)
     wl = inputgen.WORKLOADS["mixtral_prefill_bf16_small"]
