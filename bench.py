@@ -36,18 +36,29 @@ FUSED_ROUTE_MAX_T = 64
 
 def kernels_per_step(wl):
     """Kernels one forward launches, following the library's launch sequence."""
+    fused_int8 = wl.wdt == 2 and os.environ.get("COLIBRI_DEC_FUSED", "1") != "0"
+    if fused_int8 and wl.T <= FUSED_ROUTE_MAX_T and os.environ.get("COLIBRI_DEC_ROUTE", "0") not in ("", "0"):
+        return 1                                     # router, grouping, experts, combine: one launch
     n = 1                                            # Gate: router + top-k
     n += 1 if wl.T <= FUSED_ROUTE_MAX_T else 3       # Scatter: fused, or count + scan + scatter
+    if fused_int8:
+        return n + 1                                 # int8: one fused launch, the combine inside
     if wl.wdt == 0:
         n += 2 + (2 if wl.fs else 0)                 # fp32: gate/up + down (+ the shared expert's)
     elif wl.wdt == 1:
         n += 2                                       # bf16: gate/up + down (shared expert inside)
-    elif os.environ.get("COLIBRI_DEC_FUSED", "1") == "0":
-        n += 3                                       # int8: gate/up stream, finish H, down stream
     else:
-        return n + 1                                 # int8: one fused launch, the combine inside
+        n += 3                                       # int8: gate/up stream, finish H, down stream
     return n + 1                                     # Gather
 
+
+# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture of the
+# same kernel on the same workload (profiles/); None where no capture of the current kernel
+# exists.  Keyed by (workload, dominant-kernel tag).
+NCU_TRAFFIC = {
+    ("fine_grained_shared_bf16", "tc_ffn"): 1.007e9 + 76.5e6,   # launches_fine_grained_shared_bf16.md
+    ("decode_int8_T1", "dec_fused"): 353.3e6 + 4.8e6,           # dec_fused_decode_int8_T1.md
+}
 
 # fp32 FMA peak: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (the unit counts and clock of the part)
 FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
@@ -407,7 +418,7 @@ def main():
         achieved = wk["flops_gateup"] / (per_call["expert_gateup"] / 1e3) / 1e12
         mode = os.environ.get("COLIBRI_GEMM_CTA", "")[:1]
         if mode not in ("1", "2", "s"):
-            mode = "2" if wl.T * wl.k // wl.E >= 512 else "s"
+            mode = "2" if wl.T * wl.k // wl.E >= 512 else "1"
         name = {"1": "tc_ffn_kernel<gate/up> (tcgen05, 128x256 tiles)",
                 "2": "tc2_ffn_kernel<gate/up> (tcgen05, 2-CTA 256x256 pair tiles)",
                 "s": "tcs_ffn_kernel<gate/up> (tcgen05, weights x 16..256 token rows)"}[mode]
@@ -420,7 +431,10 @@ def main():
                 "peak": FP32_SIMT_TFLOPS, "unit": "TFLOP/s",
                 "frac": achieved / FP32_SIMT_TFLOPS, "algorithmic_flops_per_launch": wk["flops_gateup"]}
     roof["peak_source"] = pk["source"] + (" burst" if roof["bound"] == "tensor" else "")
-    roof["traffic"] = None
+    tag = {"dec_fused_kernel": "dec_fused", "tc_ffn_kernel<": "tc_ffn", "tc2_ffn_kernel<": "tc2_ffn",
+           "tcs_ffn_kernel<": "tcs_ffn"}
+    ktag = next((v for k, v in tag.items() if roof["kernel"].startswith(k)), None)
+    roof["traffic"] = NCU_TRAFFIC.get((wl.name, ktag))
     roof["timing"] = "kernel stage events averaged over the profiling region's calls"
     kernels = kernels_per_step(wl)
 

@@ -84,7 +84,8 @@ int pick_dec_split(int f) {
 // Tile shape of the bf16 expert GEMMs: 0 = one CTA, 128 rows x 256 columns; 1 = pairs of CTAs
 // (cta_group::2), 256 x 256; 2 = swapped operands, 128 channels x 16..256 rows.  Pair tiles when
 // experts average >= 512 rows (the halved L2 traffic outweighs the larger last tile of each
-// expert), else swapped tiles (little row padding for small or uneven groups).
+// expert), else one-CTA tiles.  The swapped tiles pad fewer rows but measured slower on every
+// workload, so they are only used on request.
 // COLIBRI_GEMM_CTA=1, 2 or s forces a mode (all are exact; this only selects the tiling).
 enum GemmMode { kGemmOne = 0, kGemmPair = 1, kGemmSwap = 2 };
 int gemm_mode(int avg_rows_per_expert) {
@@ -92,7 +93,7 @@ int gemm_mode(int avg_rows_per_expert) {
   if (v && v[0] == '1') return kGemmOne;
   if (v && v[0] == '2') return kGemmPair;
   if (v && v[0] == 's') return kGemmSwap;
-  return avg_rows_per_expert >= 512 ? kGemmPair : kGemmSwap;
+  return avg_rows_per_expert >= 512 ? kGemmPair : kGemmOne;
 }
 
 constexpr size_t kMaxGraphs = 8;  // captured forwards kept per context (least recently used evicted)
@@ -222,7 +223,7 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   const size_t o_rpart = c.take(rsplit ? (size_t)kRouterMaxSplit * M * E * 4 : 0);
   const size_t o_rtick = c.take(rsplit ? (size_t)((M + 127) / 128) * 4 : 0);
   const size_t o_err = c.take(4);
-  const size_t o_gbar = c.take(i8 ? 16 : 0);
+  const size_t o_gbar = c.take(i8 ? kFusedBarCount * 4 : 0);
   ctx->ws_bytes = c.off;
 
   DeviceGuard guard(D.device_id);
@@ -260,7 +261,7 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   w.router_ticket = rsplit ? reinterpret_cast<int32_t*>(b + o_rtick) : nullptr;
   if (cudaMemset(w.err, 0, 4) != cudaSuccess ||
       (rsplit && cudaMemset(w.router_ticket, 0, (size_t)((M + 127) / 128) * 4) != cudaSuccess) ||
-      (i8 && cudaMemset(w.grid_bar, 0, 16) != cudaSuccess)) {
+      (i8 && cudaMemset(w.grid_bar, 0, kFusedBarCount * 4) != cudaSuccess)) {
     cudaFree(ctx->ws_base);
     delete ctx;
     return fail(nullptr, COLIBRI_ERR_CUDA, "cudaMemset failed");
@@ -273,6 +274,7 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   // prefill, so it is opt-in (COLIBRI_PDL=1).
   ctx->use_pdl = env_flag("COLIBRI_PDL");
   ctx->dec_fused = !(getenv("COLIBRI_DEC_FUSED") && strcmp(getenv("COLIBRI_DEC_FUSED"), "0") == 0);
+  ctx->dec_route = env_flag("COLIBRI_DEC_ROUTE");
   cudaError_t ce = configure_router_kernels();
   if (ce == cudaSuccess) ce = configure_tc_kernels();
   if (ce == cudaSuccess) ce = configure_tcs_kernels();
@@ -350,12 +352,18 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
   };
   mark(0);
 
+  // int8 weights, T <= 64, on request (COLIBRI_DEC_ROUTE=1): router, top-k and grouping run as
+  // phase 0 of the fused expert launch.  Measured slower at T=1 (0.104 against 0.098 ms per step:
+  // the whole grid waits for the routing instead of streaming), so it is off by default.
+  const bool route_in_dec =
+      D.weight_dtype == COLIBRI_I8 && ctx->dec_fused && ctx->dec_route && T <= kFusedRouteMaxT;
+
   // ---- Gate
   if (routed_by_caller) {
     COLIBRI_TRY(cudaMemcpyAsync(w.topk_idx, user_idx, (size_t)R * 4, cudaMemcpyDeviceToDevice, s), "copy topk_idx");
     COLIBRI_TRY(cudaMemcpyAsync(w.topk_w, user_w, (size_t)R * 4, cudaMemcpyDeviceToDevice, s), "copy topk_w");
     launch_chain_break();
-  } else {
+  } else if (!route_in_dec) {
     COLIBRI_TRY(launch_router_topk(xd, act, T, d, router_w, router_b, E, k, w.topk_idx, w.topk_w, w.err,
                                    w.router_part, w.router_ticket, s),
                 "router_topk");
@@ -367,7 +375,9 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
   const int bm = D.weight_dtype == COLIBRI_F32 ? kSimtBM : (gemm == kGemmPair ? kTcPairBM : kTcBM);
   const RowPlanes xplanes{w.plane_hi, w.plane_lo, w.plane_scale};
   const RowPlanes* planes = D.weight_dtype == COLIBRI_I8 ? &xplanes : nullptr;
-  if (T <= kFusedRouteMaxT) {
+  if (route_in_dec) {
+    // grouping and the x planes are phase 0 of the fused expert launch
+  } else if (T <= kFusedRouteMaxT) {
     COLIBRI_TRY(launch_route_fused(xd, act, T, d, w.topk_idx, k, E, bm, w.counts, w.offsets, w.mt_prefix,
                                    w.src_row, w.dst_row, w.Xp, planes, s), "route_fused");
   } else {
@@ -467,6 +477,16 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
       fa.y = (__nv_bfloat16*)yd;
       fa.bar = w.grid_bar;
       fa.err = w.err;
+      if (route_in_dec) {
+        fa.route_in_kernel = routed_by_caller ? 2 : 1;
+        fa.x = (const __nv_bfloat16*)xd;
+        fa.router_w = (const __nv_bfloat16*)router_w;
+        fa.router_b = router_b;
+        fa.topk_idx = w.topk_idx;
+        fa.counts = w.counts;
+        fa.offsets_out = w.offsets;
+        fa.src_row = w.src_row;
+      }
       COLIBRI_TRY(launch_dec_fused(fa, s), "dec_fused");
       mark(3);
     } else {

@@ -115,6 +115,7 @@ struct colibri_ctx {
   bool use_graphs = true;
   bool use_pdl = false;  // programmatic dependent launch between the kernels of a forward (opt-in)
   bool dec_fused = true;  // int8 weights: the one-launch expert stage (COLIBRI_DEC_FUSED=0: four launches)
+  bool dec_route = false; // int8, T <= 64: routing inside that launch too (COLIBRI_DEC_ROUTE=1)
 };
 
 namespace colibri {
@@ -296,16 +297,27 @@ struct DecFusedArgs {
   const float* scales;
   int64_t wstride;
   int d, f, E, T, k;
-  const int32_t* offsets;   // [E+1]
-  const int32_t* dst_row;   // [T, k]
-  const float* topk_w;      // [T, k]
+  const int32_t* offsets;   // [E+1] (written by an earlier launch unless route_in_kernel)
+  int32_t* dst_row;         // [T, k]
+  float* topk_w;            // [T, k]
   int gsplit, dsplit;       // K splits of gate/up and of down
   float* GU;                // [gsplit, 2, R, f]
   float* Ypart;             // [dsplit, R, d]
   __nv_bfloat16* y;         // [T, d]
-  int32_t* bar;             // [4] zeroed counters
+  int32_t* bar;             // [kFusedBarCount] zeroed counters
   uint32_t* err;
+  // T <= 64: 1 = router, top-k and grouping in the same launch; 2 = grouping only (topk_idx and
+  // topk_w given); 0 = all done by earlier launches
+  int route_in_kernel = 0;
+  const __nv_bfloat16* x = nullptr;         // [T, d]
+  const __nv_bfloat16* router_w = nullptr;  // [E, d]
+  const float* router_b = nullptr;
+  int32_t* topk_idx = nullptr;              // [T, k]
+  int32_t* counts = nullptr;                // [E]
+  int32_t* offsets_out = nullptr;           // [E+1]
+  int32_t* src_row = nullptr;               // [T*k]
 };
+constexpr int kFusedBarCount = 8;
 cudaError_t launch_dec_fused(const DecFusedArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------------------------------
@@ -321,6 +333,83 @@ __device__ __forceinline__ void split_planes(float x, float a, float inv_a, int&
   qh = (int)h;
   ql = (int)l;
 }
+// One warp selects the top-k of one token whose E logits sit in shared memory.
+__device__ __forceinline__ void warp_topk(const float* lg, int E, int k, int lane, int32_t* idx_out,
+                                          float* w_out) {
+  float v[8];
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    const int e = lane + 32 * m;
+    v[m] = (e < E) ? lg[e] : -INFINITY;
+  }
+  uint32_t used = 0;
+  float sel_v[kMaxTopK];
+  int sel_e[kMaxTopK];
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) {
+    sel_v[j] = -INFINITY;
+    sel_e[j] = 0;
+    if (j < k) {
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const int e = lane + 32 * m;
+        if (e < E && !((used >> m) & 1u)) {
+          if (v[m] > bv || (v[m] == bv && e < be)) {
+            bv = v[m];
+            be = e;
+          }
+        }
+      }
+#pragma unroll
+      for (int off = 16; off; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+        if (ov > bv || (ov == bv && oe < be)) {
+          bv = ov;
+          be = oe;
+        }
+      }
+      if ((be & 31) == lane) used |= 1u << (be >> 5);
+      sel_v[j] = bv;
+      sel_e[j] = be;
+    }
+  }
+  if (lane == 0) {
+    float den = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j)
+      if (j < k) den += expf(sel_v[j] - sel_v[0]);
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j)
+      if (j < k) {
+        idx_out[j] = sel_e[j];
+        w_out[j] = expf(sel_v[j] - sel_v[0]) / den;
+      }
+  }
+}
+
+// 8 products of one 16-byte slice of x and of a router row, accumulated in order.
+__device__ __forceinline__ float dot16(const uint4& xa, const uint4& wa, float acc, const __nv_bfloat16*) {
+  const __nv_bfloat162* xh = reinterpret_cast<const __nv_bfloat162*>(&xa);
+  const __nv_bfloat162* wh = reinterpret_cast<const __nv_bfloat162*>(&wa);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 xf = __bfloat1622float2(xh[i]), wf = __bfloat1622float2(wh[i]);
+    acc = fmaf(xf.x, wf.x, acc);
+    acc = fmaf(xf.y, wf.y, acc);
+  }
+  return acc;
+}
+__device__ __forceinline__ float dot16(const uint4& xa, const uint4& wa, float acc, const float*) {
+  acc = fmaf(__uint_as_float(xa.x), __uint_as_float(wa.x), acc);
+  acc = fmaf(__uint_as_float(xa.y), __uint_as_float(wa.y), acc);
+  acc = fmaf(__uint_as_float(xa.z), __uint_as_float(wa.z), acc);
+  acc = fmaf(__uint_as_float(xa.w), __uint_as_float(wa.w), acc);
+  return acc;
+}
+
 // Plane scale of a row from its largest magnitude (an all-zero row gets 1).
 __device__ __forceinline__ float plane_scale(float maxabs) { return maxabs > 0.f ? maxabs / 127.f : 1.f; }
 

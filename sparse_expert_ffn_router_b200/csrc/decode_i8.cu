@@ -141,7 +141,7 @@ struct DecItem {
 // K splits x token chunks, tile fastest.
 template <bool kGateUp>
 __device__ __forceinline__ bool dec_item(const DecStreamParams& p, const int32_t* touched, const int32_t* item_prefix,
-                                         int ntouched, int L, DecItem& it) {
+                                         int ntouched, const int32_t* off, int L, DecItem& it) {
   if (L >= item_prefix[ntouched]) return false;
   int lo = 0, hi = ntouched - 1;  // largest ti with item_prefix[ti] <= L
   while (lo < hi) {
@@ -163,7 +163,7 @@ __device__ __forceinline__ bool dec_item(const DecStreamParams& p, const int32_t
   }
   it.split = local % p.nsplit;
   it.chunk = local / p.nsplit;
-  const int base = p.offsets[e], cnt = p.offsets[e + 1] - base;
+  const int base = off[e], cnt = off[e + 1] - base;
   it.row0 = base + it.chunk * p.nt8;
   it.ntok = min(p.nt8, cnt - it.chunk * p.nt8);
   return true;
@@ -195,6 +195,7 @@ struct DsCtl {
   int consumed;
   int flag;      // result of a grid-wide wait, broadcast to the epilogue warps
   int ntouched;
+  int32_t off[kMaxExperts + 1];     // row offsets of the experts' groups
   int32_t touched[kMaxExperts];
   int32_t pre[2][kMaxExperts + 1];  // item prefix over the touched experts: [0] gate/up, [1] down
   int32_t defer_row[kDsMaxStages];  // fused kernel: down stages whose plane copies wait for H
@@ -203,7 +204,7 @@ struct DsCtl {
   int32_t defer_s[kDsMaxStages];
   float red[4];                     // fused kernel: per-warp maxima of the H pass
 };
-constexpr size_t kDsCtlBytes = 4096;
+constexpr size_t kDsCtlBytes = 8192;
 static_assert(sizeof(DsCtl) <= kDsCtlBytes, "stream-kernel control block");
 
 __device__ __forceinline__ void ds_abort(DsCtl& c, uint32_t* err) {
@@ -251,7 +252,7 @@ __device__ bool ds_produce(const DecStreamParams& p, uint8_t* smem, DsCtl& c, in
     }
   };
   DecItem it;
-  for (int L = blockIdx.x; dec_item<kGateUp>(p, c.touched, c.pre[pre_idx], c.ntouched, L, it); L += gridDim.x) {
+  for (int L = blockIdx.x; dec_item<kGateUp>(p, c.touched, c.pre[pre_idx], c.ntouched, c.off, L, it); L += gridDim.x) {
     // The item's K blocks start at a rotated block (item index mod block count): items in flight
     // at the same time then read different column offsets of their weight rows, which spreads
     // the requests over the DRAM channels instead of hitting the same address bits everywhere.
@@ -305,7 +306,7 @@ __device__ bool ds_mma(const DecStreamParams& p, uint8_t* smem, DsCtl& c, int S,
   const uint32_t idesc = idesc_s8_s32(128, N);
   const uint32_t plane_bytes = (uint32_t)(2 * p.nt8 * 128);
   DecItem it;
-  for (int L = blockIdx.x; dec_item<kGateUp>(p, c.touched, c.pre[pre_idx], c.ntouched, L, it);
+  for (int L = blockIdx.x; dec_item<kGateUp>(p, c.touched, c.pre[pre_idx], c.ntouched, c.off, L, it);
        L += gridDim.x, ++iter) {
     const int a = iter & 1;
     const uint32_t aph = (uint32_t)(iter >> 1) & 1u;
@@ -345,7 +346,7 @@ __device__ bool ds_epilogue(const DecStreamParams& p, DsCtl& c, int pre_idx, int
   const int q = warp & 3;
   const int N = 2 * p.nt8;
   DecItem it;
-  for (int L = blockIdx.x; dec_item<kGateUp>(p, c.touched, c.pre[pre_idx], c.ntouched, L, it);
+  for (int L = blockIdx.x; dec_item<kGateUp>(p, c.touched, c.pre[pre_idx], c.ntouched, c.off, L, it);
        L += gridDim.x, ++iter) {
     const int a = iter & 1;
     const uint32_t aph = (uint32_t)(iter >> 1) & 1u;
@@ -386,7 +387,8 @@ __device__ bool ds_epilogue(const DecStreamParams& p, DsCtl& c, int pre_idx, int
         const int t = j + i;
         if (i >= width || t >= it.ntok || !vo) continue;
         const int row = it.row0 + t;
-        const float v = sc * p.rscale[(size_t)it.split * p.rscale_split_stride + row] * (hi[i] + lo[i] * (1.0f / 254.0f));
+        const float v = sc * __ldcg(p.rscale + (size_t)it.split * p.rscale_split_stride + row) *
+                        (hi[i] + lo[i] * (1.0f / 254.0f));
         if (kGateUp) p.GU[(((size_t)it.split * 2 + it.mat) * p.R + row) * p.f + o] = v;
         else p.Ypart[((size_t)it.split * p.R + row) * p.d + o] = v;
       }
@@ -398,9 +400,8 @@ __device__ bool ds_epilogue(const DecStreamParams& p, DsCtl& c, int pre_idx, int
   return true;
 }
 
-// Barriers, TMEM and the touched experts with their item prefixes.  Returns the TMEM base.
-__device__ __forceinline__ void ds_prologue(const DecStreamParams* const* phases, int nphases, uint8_t* smem, DsCtl& c,
-                                            int S) {
+// Barriers, descriptor prefetch, then (after the grid dependency wait) TMEM.
+__device__ __forceinline__ void ds_init(const DecStreamParams* const* phases, int nphases, DsCtl& c, int S) {
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -432,12 +433,21 @@ __device__ __forceinline__ void ds_prologue(const DecStreamParams* const* phases
     tmem_relinquish();
     tc_fence_before();
   }
+}
+
+// The experts' row offsets (from global memory, or already in c.off when `offsets` is NULL),
+// the touched experts and the prefix of their work items per phase.
+__device__ __forceinline__ void ds_items(const DecStreamParams* const* phases, int nphases, DsCtl& c,
+                                         const int32_t* offsets) {
+  const int E = phases[0]->E;
+  if (offsets)
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) c.off[e] = offsets[e];
+  __syncthreads();
   if (threadIdx.x == 0) {
-    const DecStreamParams& p0 = *phases[0];
     int n = 0;
     int acc[2] = {0, 0};
-    for (int e = 0; e < p0.E; ++e) {
-      const int cnt = p0.offsets[e + 1] - p0.offsets[e];
+    for (int e = 0; e < E; ++e) {
+      const int cnt = c.off[e + 1] - c.off[e];
       if (cnt <= 0) continue;
       c.touched[n] = e;
       for (int i = 0; i < nphases; ++i) {
@@ -481,7 +491,8 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_stream_kernel(const __grid_
   DsCtl& c = *reinterpret_cast<DsCtl*>(smem + (size_t)S * p.stage_bytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const DecStreamParams* phases[1] = {&p};
-  ds_prologue(phases, 1, smem, c, S);
+  ds_init(phases, 1, c, S);
+  ds_items(phases, 1, c, p.offsets);
   const uint32_t tmem = c.tmem;
   if (warp == 0) {
     if (lane == 0) {
@@ -526,12 +537,25 @@ struct alignas(64) DecFusedParams {
   int8_t* hhi;              // H planes [R, f] and their scales [dsplit, R]
   int8_t* hlo;
   float* hscale;
-  const int32_t* dst_row;   // [T, k]
-  const float* topk_w;      // [T, k]
+  int32_t* dst_row;         // [T, k]
+  float* topk_w;            // [T, k]
   int T, k;
   __nv_bfloat16* y;         // [T, d]
-  int32_t* bar;             // [4] arrival counters, zero between launches
+  int32_t* bar;             // [kFusedBars] arrival counters, zero between launches
+  // phase 0 (route_in_kernel): router, top-k, grouping and the x planes in this launch
+  int route_in_kernel;
+  const __nv_bfloat16* x;   // [T, d]
+  const __nv_bfloat16* router_w;  // [E, d]
+  const float* router_b;    // [E] or NULL
+  int32_t* topk_idx;        // [T, k]
+  int32_t* counts;          // [E]
+  int32_t* offsets;         // [E+1]
+  int32_t* src_row;         // [T*k]
+  float* xscale;            // [R] scales of the x planes (the buffer p.gu.rscale reads)
 };
+// grid-barrier counters: router done, x planes done, GU done, H done, Ypart done, exit ticket
+enum { kBarRouter = 0, kBarPlanes, kBarGU, kBarH, kBarY, kBarExit, kFusedBars };
+static_assert(kFusedBars <= kFusedBarCount, "grid-barrier counters of the fused kernel");
 
 __device__ __forceinline__ int ld_acquire(const int32_t* p) {
   int v;
@@ -554,6 +578,166 @@ __device__ bool grid_wait(const int32_t* ctr, int target, volatile int* abort_fl
 
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+// Phase 0 (T <= 64): router + top-k (one CTA per token; skipped when the caller routed), a grid
+// barrier, then in every CTA the
+// grouping of all T x k choices (ranks from per-expert token bit masks, offsets by a scan; the
+// same in every CTA, so no second exchange is needed), and for the CTA's own tokens: dst_row,
+// src_row and the int8 planes of the token row in each of its k grouped rows.  The ring memory,
+// idle until the producer starts, holds the scratch.  CTA 0 also writes counts and offsets.
+// Arrives on the planes barrier; the producer waits on it before its first plane copy.
+__device__ void fused_route(const DecFusedParams& p, uint8_t* smem, DsCtl& c) {
+  constexpr int kWarps = kDsThreads / 32;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = gridDim.x, T = p.T, k = p.k, E = p.gu.E, d = p.gu.d;
+  const int nvec = d / 8;  // 16-byte slices of a bf16 row
+  float* part = reinterpret_cast<float*>(smem);      // [kWarps][E]
+  float* lg = part + kWarps * kMaxExperts;           // [E]
+  for (int t = blockIdx.x; p.route_in_kernel == 1 && t < T; t += G) {  // 2: the caller routed
+    const uint4* xv = reinterpret_cast<const uint4*>(p.x + (size_t)t * d);
+    for (int e0 = 0; e0 < E; e0 += 8) {
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      for (int v = tid; v < nvec; v += kDsThreads) {
+        const uint4 xq = __ldg(xv + v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (e0 + i < E)
+            acc[i] = dot16(xq, __ldg(reinterpret_cast<const uint4*>(p.router_w + (size_t)(e0 + i) * d) + v), acc[i],
+                           p.x);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+#pragma unroll
+        for (int off = 16; off; off >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
+      }
+      if (lane == 0) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (e0 + i < E) part[warp * kMaxExperts + e0 + i] = acc[i];
+      }
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kDsThreads) {
+      float sum = part[e];
+      for (int w = 1; w < kWarps; ++w) sum += part[w * kMaxExperts + e];
+      lg[e] = sum + (p.router_b ? p.router_b[e] : 0.f);
+    }
+    __syncthreads();
+    if (warp == 0) warp_topk(lg, E, k, lane, p.topk_idx + (size_t)t * k, p.topk_w + (size_t)t * k);
+    __syncthreads();
+  }
+  // every token's choices are needed below
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    atomicAdd(&p.bar[kBarRouter], 1);
+    c.flag = grid_wait(&p.bar[kBarRouter], G, &c.abort) ? 1 : 0;
+    if (!c.flag) ds_abort(c, p.gu.err);
+  }
+  __syncthreads();
+  unsigned long long* mask = reinterpret_cast<unsigned long long*>(smem);  // [E] tokens choosing e
+  for (int e = tid; e < E; e += kDsThreads) mask[e] = 0ull;
+  __syncthreads();
+  if (c.flag) {
+    for (int i = tid; i < T * k; i += kDsThreads) {
+      const int e = min(max(__ldcg(p.topk_idx + i), 0), E - 1);
+      atomicOr(&mask[e], 1ull << (i / k));
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {  // offsets: exclusive scan of the counts over the experts
+    const int C = (E + 31) / 32;
+    const int e0 = min(E, lane * C), e1 = min(E, e0 + C);
+    int sum = 0;
+    for (int e = e0; e < e1; ++e) sum += __popcll(mask[e]);
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += a;
+    }
+    int run = incl - sum;
+    for (int e = e0; e < e1; ++e) {
+      const int cnt = __popcll(mask[e]);
+      c.off[e] = run;
+      if (blockIdx.x == 0) {
+        p.counts[e] = cnt;
+        p.offsets[e] = run;
+      }
+      run += cnt;
+    }
+    if (lane == 31) {
+      c.off[E] = incl;
+      if (blockIdx.x == 0) p.offsets[E] = incl;
+    }
+  }
+  __syncthreads();
+  float* red = reinterpret_cast<float*>(smem + (size_t)kMaxExperts * sizeof(unsigned long long));  // [kWarps]
+  for (int t = blockIdx.x; t < T && c.flag; t += G) {
+    int rows[kMaxTopK];
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      rows[j] = 0;
+      if (j < k) {
+        const int e = min(max(__ldcg(p.topk_idx + (size_t)t * k + j), 0), E - 1);
+        rows[j] = c.off[e] + __popcll(mask[e] & ((1ull << t) - 1ull));
+      }
+    }
+    if (tid < k) {
+      const int r = rows[tid];
+      p.dst_row[(size_t)t * k + tid] = r;
+      p.src_row[r] = t;
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(p.x + (size_t)t * d);
+    float mx = 0.f;
+    for (int v = tid; v < nvec; v += kDsThreads) {
+      const uint4 q = __ldg(src + v);
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f2 = __bfloat1622float2(h2[i]);
+        mx = fmaxf(mx, fmaxf(fabsf(f2.x), fabsf(f2.y)));
+      }
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    if (lane == 0) red[warp] = mx;
+    __syncthreads();
+    mx = red[0];
+    for (int w = 1; w < kWarps; ++w) mx = fmaxf(mx, red[w]);
+    __syncthreads();
+    const float a = plane_scale(mx), inv_a = __frcp_rn(a);  // correctly rounded 1 / a
+    if (tid < k) p.xscale[rows[tid]] = a;
+    for (int v = tid; v < nvec; v += kDsThreads) {
+      const uint4 q = __ldg(src + v);
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&q);
+      uint32_t hw[2] = {0u, 0u}, lw[2] = {0u, 0u};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f2 = __bfloat1622float2(h2[i]);
+        int qh0, ql0, qh1, ql1;
+        split_planes(f2.x, a, inv_a, qh0, ql0);
+        split_planes(f2.y, a, inv_a, qh1, ql1);
+        hw[i >> 1] |= (((uint32_t)qh0 & 0xffu) | (((uint32_t)qh1 & 0xffu) << 8)) << (16 * (i & 1));
+        lw[i >> 1] |= (((uint32_t)ql0 & 0xffu) | (((uint32_t)ql1 & 0xffu) << 8)) << (16 * (i & 1));
+      }
+#pragma unroll
+      for (int j = 0; j < kMaxTopK; ++j) {
+        if (j < k) {
+          reinterpret_cast<uint2*>(p.hhi + (size_t)rows[j] * d)[v] = make_uint2(hw[0], hw[1]);
+          reinterpret_cast<uint2*>(p.hlo + (size_t)rows[j] * d)[v] = make_uint2(lw[0], lw[1]);
+        }
+      }
+    }
+  }
+  // the planes are read next by TMA copies of other CTAs
+  fence_proxy_async_global();
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) atomicAdd(&p.bar[kBarPlanes], 1);
+}
+
 __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_constant__ DecFusedParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int S = p.gu.stages;
@@ -562,21 +746,35 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_c
   const int G = gridDim.x;
   const bool aligned = (smem_u32(smem) & 1023u) == 0;  // the 128-byte swizzle needs 1024-byte stages
   const DecStreamParams* phases[2] = {&p.gu, &p.dn};
-  if (aligned) ds_prologue(phases, 2, smem, c, S);
+  if (aligned) {
+    ds_init(phases, 2, c, S);
+    if (p.route_in_kernel) {
+      fused_route(p, smem, c);
+      ds_items(phases, 2, c, nullptr);
+    } else {
+      ds_items(phases, 2, c, p.gu.offsets);
+    }
+  }
   const uint32_t tmem = aligned ? c.tmem : 0u;
   if (!aligned) {
     if (threadIdx.x == 0) {  // report, and arrive at every barrier so the other CTAs do not wait
       atomicOr(p.gu.err, kErrWaitTimeout);
-      for (int b = 0; b < 3; ++b) atomicAdd(&p.bar[b], 1);
+      for (int b = 0; b < kBarExit; ++b) atomicAdd(&p.bar[b], 1);
     }
   } else if (warp == 0) {
     if (lane == 0) {
       DsRing r;
-      bool ok = ds_produce<true>(p.gu, smem, c, S, 0, r, false, [] { return true; });
+      // with the routing done in this launch, the gate/up weights go out at once and the plane
+      // copies wait until every CTA has written its tokens' planes
+      bool ok = ds_produce<true>(p.gu, smem, c, S, 0, r, p.route_in_kernel != 0, [&] {
+        if (!grid_wait(&p.bar[kBarPlanes], G, &c.abort)) return false;
+        fence_proxy_async_global();
+        return true;
+      });
       // down weights go out at once; their plane copies wait for phase 2 of every CTA
       if (ok)
         ok = ds_produce<false>(p.dn, smem, c, S, 1, r, true, [&] {
-          if (!grid_wait(&p.bar[1], G, &c.abort)) return false;
+          if (!grid_wait(&p.bar[kBarH], G, &c.abort)) return false;
           fence_proxy_async_global();
           return true;
         });
@@ -614,8 +812,8 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_c
     };
     bool ok = ds_epilogue<true>(p.gu, c, 0, iter, tmem, warp, lane);
     if (!__all_sync(0xffffffffu, ok) && lane == 0) ds_abort(c, p.gu.err);
-    // barrier 1: every CTA's GU partials are written
-    ok = grid_barrier(0);
+    // barrier: every CTA's GU partials are written
+    ok = grid_barrier(kBarGU);
     if (ok) {
       // phase 2: H planes, one (row, down split) unit per round
       float* red = c.red;
@@ -625,21 +823,37 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_c
       for (int u = blockIdx.x; u < R * ds; u += G) {
         const int r = u / ds, sp = u - r * ds, k0 = sp * span;
         const float* g0 = p.gu.GU + (size_t)r * f + k0;
+        // h for 4 consecutive columns: all gsplit partials are loaded before they are summed (in
+        // split order), so one pass is one memory round trip per step
+        auto hvals = [&](int j, float (&hv)[4]) {
+          float4 gv[kDecGateSplitMax], uv[kDecGateSplitMax];
+#pragma unroll
+          for (int s2 = 0; s2 < kDecGateSplitMax; ++s2) {
+            if (s2 < gs) {
+              gv[s2] = __ldcg(reinterpret_cast<const float4*>(g0 + (size_t)(2 * s2) * plane + j));
+              uv[s2] = __ldcg(reinterpret_cast<const float4*>(g0 + (size_t)(2 * s2 + 1) * plane + j));
+            }
+          }
+          float4 g = gv[0], uu = uv[0];
+#pragma unroll
+          for (int s2 = 1; s2 < kDecGateSplitMax; ++s2) {
+            if (s2 < gs) {
+              g.x += gv[s2].x; g.y += gv[s2].y; g.z += gv[s2].z; g.w += gv[s2].w;
+              uu.x += uv[s2].x; uu.y += uv[s2].y; uu.z += uv[s2].z; uu.w += uv[s2].w;
+            }
+          }
+          hv[0] = __bfloat162float(__float2bfloat16_rn(silu_mul(g.x, uu.x)));
+          hv[1] = __bfloat162float(__float2bfloat16_rn(silu_mul(g.y, uu.y)));
+          hv[2] = __bfloat162float(__float2bfloat16_rn(silu_mul(g.z, uu.z)));
+          hv[3] = __bfloat162float(__float2bfloat16_rn(silu_mul(g.w, uu.w)));
+        };
+        // two passes over the partials (max, then split): keeping the values in registers between
+        // them measured slower (the kernel's register count doubled)
         float mx = 0.f;
         for (int j = tid * 4; j < span; j += 128 * 4) {
-          float4 g = __ldcg(reinterpret_cast<const float4*>(g0 + j));
-          float4 uu = __ldcg(reinterpret_cast<const float4*>(g0 + plane + j));
-          for (int s2 = 1; s2 < gs; ++s2) {
-            const float4 a = __ldcg(reinterpret_cast<const float4*>(g0 + (size_t)(2 * s2) * plane + j));
-            const float4 b = __ldcg(reinterpret_cast<const float4*>(g0 + (size_t)(2 * s2 + 1) * plane + j));
-            g.x += a.x; g.y += a.y; g.z += a.z; g.w += a.w;
-            uu.x += b.x; uu.y += b.y; uu.z += b.z; uu.w += b.w;
-          }
-          const float h0 = __bfloat162float(__float2bfloat16_rn(silu_mul(g.x, uu.x)));
-          const float h1 = __bfloat162float(__float2bfloat16_rn(silu_mul(g.y, uu.y)));
-          const float h2 = __bfloat162float(__float2bfloat16_rn(silu_mul(g.z, uu.z)));
-          const float h3 = __bfloat162float(__float2bfloat16_rn(silu_mul(g.w, uu.w)));
-          mx = fmaxf(mx, fmaxf(fmaxf(fabsf(h0), fabsf(h1)), fmaxf(fabsf(h2), fabsf(h3))));
+          float hv[4];
+          hvals(j, hv);
+          mx = fmaxf(mx, fmaxf(fmaxf(fabsf(hv[0]), fabsf(hv[1])), fmaxf(fabsf(hv[2]), fabsf(hv[3]))));
         }
 #pragma unroll
         for (int off = 16; off; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
@@ -652,18 +866,8 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_c
         int8_t* hrow = p.hhi + (size_t)r * f + k0;
         int8_t* lrow = p.hlo + (size_t)r * f + k0;
         for (int j = tid * 4; j < span; j += 128 * 4) {  // the same values again, now split
-          float4 g = __ldcg(reinterpret_cast<const float4*>(g0 + j));
-          float4 uu = __ldcg(reinterpret_cast<const float4*>(g0 + plane + j));
-          for (int s2 = 1; s2 < gs; ++s2) {
-            const float4 a2 = __ldcg(reinterpret_cast<const float4*>(g0 + (size_t)(2 * s2) * plane + j));
-            const float4 b2 = __ldcg(reinterpret_cast<const float4*>(g0 + (size_t)(2 * s2 + 1) * plane + j));
-            g.x += a2.x; g.y += a2.y; g.z += a2.z; g.w += a2.w;
-            uu.x += b2.x; uu.y += b2.y; uu.z += b2.z; uu.w += b2.w;
-          }
-          const float hv[4] = {__bfloat162float(__float2bfloat16_rn(silu_mul(g.x, uu.x))),
-                               __bfloat162float(__float2bfloat16_rn(silu_mul(g.y, uu.y))),
-                               __bfloat162float(__float2bfloat16_rn(silu_mul(g.z, uu.z))),
-                               __bfloat162float(__float2bfloat16_rn(silu_mul(g.w, uu.w)))};
+          float hv[4];
+          hvals(j, hv);
           uint32_t hw = 0u, lw = 0u;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -678,12 +882,12 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_c
       }
       fence_proxy_async_global();  // the planes are read next by TMA copies of other CTAs
     }
-    // barrier 2: every CTA's H planes are written (the producer waits on the same counter)
-    ok = grid_barrier(1);
+    // barrier: every CTA's H planes are written (the producer waits on the same counter)
+    ok = grid_barrier(kBarH);
     if (ok) ok = ds_epilogue<false>(p.dn, c, 1, iter, tmem, warp, lane);
     if (!__all_sync(0xffffffffu, ok) && lane == 0) ds_abort(c, p.gu.err);
-    // barrier 3: every CTA's down partials are written
-    ok = grid_barrier(2);
+    // barrier: every CTA's down partials are written
+    ok = grid_barrier(kBarY);
     if (ok) {
       // phase 4: combine, one thread per (token, 4 consecutive outputs)
       const int d = p.dn.d, ns = p.dn.nsplit, k = p.k;
@@ -693,8 +897,8 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_c
         const int t = (int)(qi / chunks), cc = (int)(qi - (long long)t * chunks) * 4;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int j = 0; j < k; ++j) {
-          const int rr = p.dst_row[(size_t)t * k + j];
-          const float wj = p.topk_w[(size_t)t * k + j];
+          const int rr = __ldcg(p.dst_row + (size_t)t * k + j);
+          const float wj = __ldcg(p.topk_w + (size_t)t * k + j);
           const float* base = p.dn.Ypart + (size_t)rr * d + cc;
           float4 part = make_float4(0.f, 0.f, 0.f, 0.f);
           int sp = 0;
@@ -729,11 +933,8 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_c
   // exit ticket: the last CTA to leave resets the counters for the next launch
   if (threadIdx.x == 0) {
     __threadfence();
-    if (atomicAdd(&p.bar[3], 1) == G - 1) {
-      p.bar[0] = 0;
-      p.bar[1] = 0;
-      p.bar[2] = 0;
-      p.bar[3] = 0;
+    if (atomicAdd(&p.bar[kBarExit], 1) == G - 1) {
+      for (int b = 0; b < kFusedBars; ++b) p.bar[b] = 0;
       __threadfence();
     }
   }
@@ -897,6 +1098,18 @@ cudaError_t launch_dec_fused(const DecFusedArgs& a, cudaStream_t s) {
   p.k = a.k;
   p.y = a.y;
   p.bar = a.bar;
+  p.route_in_kernel = a.route_in_kernel;
+  p.x = a.x;
+  p.router_w = a.router_w;
+  p.router_b = a.router_b;
+  p.topk_idx = a.topk_idx;
+  p.counts = a.counts;
+  p.offsets = a.offsets_out;
+  p.src_row = a.src_row;
+  p.xscale = a.planes_scale;
+  if (a.route_in_kernel && (a.T > 64 || !a.x || !a.topk_idx || !a.counts || !a.offsets_out || !a.src_row ||
+                            (a.route_in_kernel == 1 && !a.router_w)))
+    return cudaErrorInvalidValue;
   const size_t smem = (size_t)p.gu.stages * p.gu.stage_bytes + kDsCtlBytes;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(sm_count_current());

@@ -23,62 +23,6 @@ constexpr int kRouterTT = 32;  // tokens per CTA
 constexpr int kRouterDK = 32;  // K chunk staged in shared memory
 constexpr int kRouterThreads = 256;
 
-// One warp selects the top-k of one token whose E logits sit in shared memory.
-__device__ __forceinline__ void warp_topk(const float* lg, int E, int k, int lane, int32_t* idx_out,
-                                          float* w_out) {
-  float v[8];
-#pragma unroll
-  for (int m = 0; m < 8; ++m) {
-    const int e = lane + 32 * m;
-    v[m] = (e < E) ? lg[e] : -INFINITY;
-  }
-  uint32_t used = 0;
-  float sel_v[kMaxTopK];
-  int sel_e[kMaxTopK];
-#pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j) {
-    sel_v[j] = -INFINITY;
-    sel_e[j] = 0;
-    if (j < k) {
-      float bv = -INFINITY;
-      int be = 0x7fffffff;
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const int e = lane + 32 * m;
-        if (e < E && !((used >> m) & 1u)) {
-          if (v[m] > bv || (v[m] == bv && e < be)) {
-            bv = v[m];
-            be = e;
-          }
-        }
-      }
-#pragma unroll
-      for (int off = 16; off; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-        if (ov > bv || (ov == bv && oe < be)) {
-          bv = ov;
-          be = oe;
-        }
-      }
-      if ((be & 31) == lane) used |= 1u << (be >> 5);
-      sel_v[j] = bv;
-      sel_e[j] = be;
-    }
-  }
-  if (lane == 0) {
-    float den = 0.f;
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j)
-      if (j < k) den += expf(sel_v[j] - sel_v[0]);
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j)
-      if (j < k) {
-        idx_out[j] = sel_e[j];
-        w_out[j] = expf(sel_v[j] - sel_v[0]) / den;
-      }
-  }
-}
 
 // SIMT router: 32 tokens per CTA, warp w accumulates experts w, w+8, ... for the token of
 // its lane; x and Wr chunks are staged in shared memory as fp32.
@@ -138,24 +82,6 @@ __global__ void __launch_bounds__(kRouterThreads) router_topk_simt_kernel(
 // ... with its lanes splitting d (16-byte loads; the token row is read through L1) and a
 // shuffle reduction; then warp 0 selects the top-k.  Latency-bound work, so no tensor cores.
 // ---------------------------------------------------------------------------------------
-__device__ __forceinline__ float dot16(const uint4& xa, const uint4& wa, float acc, const __nv_bfloat16*) {
-  const __nv_bfloat162* xh = reinterpret_cast<const __nv_bfloat162*>(&xa);
-  const __nv_bfloat162* wh = reinterpret_cast<const __nv_bfloat162*>(&wa);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 xf = __bfloat1622float2(xh[i]), wf = __bfloat1622float2(wh[i]);
-    acc = fmaf(xf.x, wf.x, acc);
-    acc = fmaf(xf.y, wf.y, acc);
-  }
-  return acc;
-}
-__device__ __forceinline__ float dot16(const uint4& xa, const uint4& wa, float acc, const float*) {
-  acc = fmaf(__uint_as_float(xa.x), __uint_as_float(wa.x), acc);
-  acc = fmaf(__uint_as_float(xa.y), __uint_as_float(wa.y), acc);
-  acc = fmaf(__uint_as_float(xa.z), __uint_as_float(wa.z), acc);
-  acc = fmaf(__uint_as_float(xa.w), __uint_as_float(wa.w), acc);
-  return acc;
-}
 
 // Small batches: one CTA per token.  Every thread takes the same 16-byte slices of x and of 8
 // expert rows at a time, so each thread has 9 independent loads per slice in flight; the 8
