@@ -56,7 +56,7 @@ def kernels_per_step(wl):
 # same kernel on the same workload (profiles/); None where no capture of the current kernel
 # exists.  Keyed by (workload, dominant-kernel tag).
 NCU_TRAFFIC = {
-    ("fine_grained_shared_bf16", "tc_ffn"): 1.007e9 + 76.5e6,   # launches_fine_grained_shared_bf16.md
+    ("mixtral_prefill_bf16", "tc2_ffn"): 2.943e9 + 0.230e9,     # tc2_ffn_traffic_mixtral_prefill_bf16.md
     ("decode_int8_T1", "dec_fused"): 353.3e6 + 4.8e6,           # dec_fused_decode_int8_T1.md
 }
 

@@ -82,6 +82,12 @@ struct Tile {
   int e, row0, row_end, n0, num_kb;
 };
 
+// An m-tile with at most kLightRows rows is computed with the operands swapped (one-CTA kernel):
+// the weight tile is the M side (128 rows per MMA, two MMAs for the tile's 256 weight rows) and
+// the tile's rows the N side (N = rows rounded up to 16), so a tile of a few rows costs a few
+// percent of a 128 x 256 tile of MMAs and is bound by the stream of its weights.
+constexpr int kLightRows = 64;
+
 // Routed tiles come in two classes.  An expert with two or more m-tiles reuses each weight tile
 // across its m-tiles (compute-bound); an expert with a single m-tile streams its weights once
 // (bound by HBM).  When both classes exist (skewed routing) their tiles are interleaved in
@@ -311,6 +317,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ffn_kernel(const __grid_con
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(a * BN);
+        const int rows = t.row_end - t.row0;
+        const bool light = rows <= kLightRows;
+        const uint32_t idesc_l = idesc_bf16_f32(128, (rows + 15) / 16 * 16);
         for (int kb = 0; kb < t.num_kb; ++kb) {
           if (!wait_or_abort(&m.full[s], ph, abort_flag)) {
             ok = false;
@@ -319,11 +328,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ffn_kernel(const __grid_con
           tc_fence_after();
           const uint32_t sA = smem_u32(stage_base + (size_t)s * STAGE_BYTES);
           const uint32_t sB = sA + A_BYTES;
+          if (light) {
+            // swapped: weight rows [0,128) -> columns [0,N), rows [128,256) -> columns [128,128+N)
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(sA + kk * 32);
-            const uint64_t bd = smem_desc_sw128(sB + kk * 32);
-            tc_mma_f16(d_tmem, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t xd = smem_desc_sw128(sA + kk * 32);
+              const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+              tc_mma_f16(d_tmem, smem_desc_sw128(sB + kk * 32), xd, idesc_l, acc);
+              tc_mma_f16(d_tmem + 128, smem_desc_sw128(sB + B_BYTES / 2 + kk * 32), xd, idesc_l, acc);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t ad = smem_desc_sw128(sA + kk * 32);
+              const uint64_t bd = smem_desc_sw128(sB + kk * 32);
+              tc_mma_f16(d_tmem, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+            }
           }
           tc_commit(&m.empty[s]);
           ++consumed;
@@ -361,7 +381,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ffn_kernel(const __grid_con
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * BN);
       __nv_bfloat16* out = t.sh ? p.out_sh : p.out;
       const int n_out = t.sh ? p.n_out_sh : p.n_out;
-      if (kGateUp) {
+      const int rows = t.row_end - t.row0;
+      if (rows <= kLightRows) {
+        // swapped tile: TMEM lane = weight row (output column), TMEM column = the tile's row
+        const int ch = q * 32 + lane;  // gate/up: column n0 + ch; down: n0 + ch and n0 + 128 + ch
+        for (int j0 = 0; j0 < rows; j0 += 16) {
+          float v0[16], v1[16];
+          tmem_ld16(tb + j0, v0);
+          tmem_ld16(tb + 128 + j0, v1);
+          tmem_ld_wait();
+          if (kGateUp) {
+            if (t.n0 + ch < n_out) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                if (j0 + i < rows)
+                  out[(size_t)(t.row0 + j0 + i) * n_out + t.n0 + ch] = __float2bfloat16_rn(silu_mul(v0[i], v1[i]));
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              if (j0 + i < rows) {
+                __nv_bfloat16* o = out + (size_t)(t.row0 + j0 + i) * n_out + t.n0 + ch;
+                if (t.n0 + ch < n_out) o[0] = __float2bfloat16_rn(v0[i]);
+                if (t.n0 + 128 + ch < n_out) o[128] = __float2bfloat16_rn(v1[i]);
+              }
+            }
+          }
+        }
+      } else if (kGateUp) {
 #pragma unroll 1
         for (int c = 0; c < BN / 2; c += 16) {
           float g[16], u[16];
