@@ -57,7 +57,6 @@ def kernels_per_step(wl):
 # exists.  Keyed by (workload, dominant-kernel tag).
 NCU_TRAFFIC = {
     ("mixtral_prefill_bf16", "tc2_ffn"): 2.943e9 + 0.230e9,     # tc2_ffn_traffic_mixtral_prefill_bf16.md
-    ("decode_int8_T1", "dec_fused"): 353.3e6 + 4.8e6,           # dec_fused_decode_int8_T1.md
 }
 
 # fp32 FMA peak: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (the unit counts and clock of the part)

@@ -126,6 +126,7 @@ struct alignas(64) DecStreamParams {
   int nt8;                  // tokens per chunk (8, 16 or 32); MMA N = 2 * nt8
   int R;                    // rows of the planes (T * k)
   int kbs;                  // 128-byte K blocks per ring stage (1..kDsMaxKbs)
+  int evict_first;          // weight copies with an L2 evict-first policy (read once)
   uint32_t stage_bytes;     // kbs x (weight tile 128 x 128 + planes 2 nt8 x 128)
   int stages;
   float* GU;                // gate/up output: [nsplit, 2, R, f] fp32 partials (W1 . x, W3 . x, scaled)
@@ -242,6 +243,7 @@ template <bool kGateUp, typename Ready>
 __device__ bool ds_produce(const DecStreamParams& p, uint8_t* smem, DsCtl& c, int S, int pre_idx, DsRing& r,
                            bool defer, Ready ready) {
   const uint32_t blk_bytes = 128u * 128u + (uint32_t)(2 * p.nt8) * 128u;
+  const uint64_t policy = l2_evict_first_policy();
   int held = 0;
   bool released = !defer;
   auto release = [&]() {
@@ -268,8 +270,13 @@ __device__ bool ds_produce(const DecStreamParams& p, uint8_t* smem, DsCtl& c, in
       for (int j = 0; j < nk; ++j, kb = (kb + 1 == nkb) ? 0 : kb + 1) {
         const int kx = kbeg + kb * 128;
         uint8_t* sw = st + (size_t)j * 128 * 128;
-        if (kGateUp) tma_load_4d(sw, &p.mapW, &c.full[r.s], kx, it.tile * 128, it.mat, it.e);
-        else tma_load_3d(sw, &p.mapW, &c.full[r.s], kx, it.tile * 128, it.e);
+        if (p.evict_first) {
+          if (kGateUp) tma_load_4d_hint(sw, &p.mapW, &c.full[r.s], kx, it.tile * 128, it.mat, it.e, policy);
+          else tma_load_3d_hint(sw, &p.mapW, &c.full[r.s], kx, it.tile * 128, it.e, policy);
+        } else {
+          if (kGateUp) tma_load_4d(sw, &p.mapW, &c.full[r.s], kx, it.tile * 128, it.mat, it.e);
+          else tma_load_3d(sw, &p.mapW, &c.full[r.s], kx, it.tile * 128, it.e);
+        }
         if (released) ds_load_planes(p, st, &c.full[r.s], j, kx, it.row0);
         else c.defer_kx[held][j] = kx;
       }
@@ -966,6 +973,7 @@ bool plane_maps(DecStreamParams& p, const int8_t* hi, const int8_t* lo, int K) {
   if (!make_tmap(&p.mapHi, CU_TENSOR_MAP_DATA_TYPE_UINT8, hi, 2, pd, ps, pb)) return false;
   if (!make_tmap(&p.mapLo, CU_TENSOR_MAP_DATA_TYPE_UINT8, lo, 2, pd, ps, pb)) return false;
   p.kbs = dec_kbs();
+  p.evict_first = !(getenv("COLIBRI_DEC_EVICT") && strcmp(getenv("COLIBRI_DEC_EVICT"), "0") == 0);
   p.stage_bytes = (uint32_t)(p.kbs * (128 * 128 + 2 * p.nt8 * 128));
   p.stages = (int)std::min<size_t>(kDsMaxStages, kDsRingBytes / p.stage_bytes);
   return true;

@@ -80,6 +80,7 @@ constexpr size_t SMEM_BYTES = 1024 /*align slack*/ + (size_t)STAGES * STAGE_BYTE
 struct Tile {
   bool sh;
   int e, row0, row_end, n0, num_kb;
+  int mtiles;  // m-tiles of the tile's group
 };
 
 // An m-tile with at most kLightRows rows is computed with the operands swapped (one-CTA kernel):
@@ -160,6 +161,7 @@ __device__ __forceinline__ Tile decode_tile(const TcParams& p, const Misc& m, in
     const int Lp = idx - pre[lo] * p.n_tiles;
     const int n = Lp / Me, mm = Lp - n * Me;
     t.sh = false;
+    t.mtiles = Me;
     t.e = lo;
     t.row0 = m.off[lo] + mm * bm;
     t.row_end = m.off[lo + 1];
@@ -169,6 +171,7 @@ __device__ __forceinline__ Tile decode_tile(const TcParams& p, const Misc& m, in
     const int Lp = L - routed_total;
     const int n = Lp / p.mt_sh, mm = Lp - n * p.mt_sh;
     t.sh = true;
+    t.mtiles = p.mt_sh;
     t.e = 0;
     t.row0 = mm * bm;
     t.row_end = p.rows_sh;
@@ -258,6 +261,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ffn_kernel(const __grid_con
       int s = 0;
       uint32_t ph = 0;
       int issued = 0;
+      const uint64_t evict_first = l2_evict_first_policy();
       for (int L = blockIdx.x; L < total; L += gridDim.x) {
         const Tile t = decode_tile(p, m, L, routed_total, kGateUp);
         const CUtensorMap* mA = t.sh ? &p.mapA_sh : &p.mapA;
@@ -273,16 +277,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ffn_kernel(const __grid_con
           mbar_arrive_expect_tx(&m.full[s], STAGE_BYTES);
           const int kx = kb * BK;
           tma_load_2d(sA, mA, &m.full[s], kx, t.row0);
+          // the weight tile of a group with a single (light) m-tile is read by this tile alone:
+          // evict it first from L2
+          const bool stream = t.mtiles == 1 && t.row_end - t.row0 <= kLightRows && !t.sh;
           if (kGateUp) {
             if (t.sh) {
               tma_load_3d(sB, mB, &m.full[s], kx, t.n0, 0);
               tma_load_3d(sB + B_BYTES / 2, mB, &m.full[s], kx, t.n0, 1);
+            } else if (stream) {
+              tma_load_4d_hint(sB, mB, &m.full[s], kx, t.n0, 0, t.e, evict_first);
+              tma_load_4d_hint(sB + B_BYTES / 2, mB, &m.full[s], kx, t.n0, 1, t.e, evict_first);
             } else {
               tma_load_4d(sB, mB, &m.full[s], kx, t.n0, 0, t.e);
               tma_load_4d(sB + B_BYTES / 2, mB, &m.full[s], kx, t.n0, 1, t.e);
             }
           } else {
             if (t.sh) tma_load_2d(sB, mB, &m.full[s], kx, t.n0);
+            else if (stream) tma_load_3d_hint(sB, mB, &m.full[s], kx, t.n0, t.e, evict_first);
             else tma_load_3d(sB, mB, &m.full[s], kx, t.n0, t.e);
           }
           ++issued;

@@ -33,7 +33,11 @@ SMALL = {
     "bf16_T1": inputgen.custom("bf16_T1", T=1, d=256, E=8, k=2, f=256),
     "f32_tiny": inputgen.WORKLOADS["tiny_f32"],
     "f32_shared": inputgen.custom("f32_shared", T=100, d=128, E=4, k=2, f=192, fs=64, act=F32, wdt=F32),
+    # the largest expert count and top-k the ABI accepts (E = 256, k = 8)
+    "bf16_maxE": inputgen.custom("bf16_maxE", T=300, d=128, E=256, k=8, f=128),
+    "f32_maxE": inputgen.custom("f32_maxE", T=40, d=64, E=256, k=8, f=64, act=F32, wdt=F32),
     "i8_small": inputgen.custom("i8_small", T=5, d=256, E=4, k=2, f=512, act=BF16, wdt=I8),
+    "i8_maxE": inputgen.custom("i8_maxE", T=64, d=128, E=256, k=8, f=128, act=BF16, wdt=I8),
     # more than 32 tokens on one expert: the decode kernels loop over token chunks
     "i8_many": inputgen.custom("i8_many", T=80, d=128, E=2, k=1, f=192, act=BF16, wdt=I8),
 }
