@@ -37,7 +37,7 @@ FUSED_ROUTE_MAX_T = 64
 def kernels_per_step(wl):
     """Kernels one forward launches, following the library's launch sequence."""
     fused_int8 = wl.wdt == 2 and os.environ.get("COLIBRI_DEC_FUSED", "1") != "0"
-    if fused_int8 and wl.T <= FUSED_ROUTE_MAX_T and os.environ.get("COLIBRI_DEC_ROUTE", "0") not in ("", "0"):
+    if fused_int8 and wl.T <= FUSED_ROUTE_MAX_T and os.environ.get("COLIBRI_DEC_ROUTE", "1") != "0":
         return 1                                     # router, grouping, experts, combine: one launch
     n = 1                                            # Gate: router + top-k
     n += 1 if wl.T <= FUSED_ROUTE_MAX_T else 3       # Scatter: fused, or count + scan + scatter
@@ -57,6 +57,7 @@ def kernels_per_step(wl):
 # exists.  Keyed by (workload, dominant-kernel tag).
 NCU_TRAFFIC = {
     ("mixtral_prefill_bf16", "tc2_ffn"): 2.943e9 + 0.230e9,     # tc2_ffn_traffic_mixtral_prefill_bf16.md
+    ("fine_grained_shared_bf16", "tc_ffn"): 1.0089e9 + 74.8e6,  # launches_fine_grained_shared_bf16.md
 }
 
 # fp32 FMA peak: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (the unit counts and clock of the part)

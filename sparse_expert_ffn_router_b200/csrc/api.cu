@@ -274,7 +274,7 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   // prefill, so it is opt-in (COLIBRI_PDL=1).
   ctx->use_pdl = env_flag("COLIBRI_PDL");
   ctx->dec_fused = !(getenv("COLIBRI_DEC_FUSED") && strcmp(getenv("COLIBRI_DEC_FUSED"), "0") == 0);
-  ctx->dec_route = env_flag("COLIBRI_DEC_ROUTE");
+  ctx->dec_route = !(getenv("COLIBRI_DEC_ROUTE") && strcmp(getenv("COLIBRI_DEC_ROUTE"), "0") == 0);
   cudaError_t ce = configure_router_kernels();
   if (ce == cudaSuccess) ce = configure_tc_kernels();
   if (ce == cudaSuccess) ce = configure_tcs_kernels();
@@ -352,9 +352,10 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
   };
   mark(0);
 
-  // int8 weights, T <= 64, on request (COLIBRI_DEC_ROUTE=1): router, top-k and grouping run as
-  // phase 0 of the fused expert launch.  Measured slower at T=1 (0.104 against 0.098 ms per step:
-  // the whole grid waits for the routing instead of streaming), so it is off by default.
+  // int8 weights, T <= 64: router, top-k and grouping run as phase 0 of the fused expert launch
+  // (COLIBRI_DEC_ROUTE=0: as two launches before it).  With the weight streams evicted first
+  // from L2 the router's inputs stay resident and the one launch is the faster plan (T=1: 0.0856
+  // against 0.0874 ms per step, T=8: 0.198 against 0.204 ms).
   const bool route_in_dec =
       D.weight_dtype == COLIBRI_I8 && ctx->dec_fused && ctx->dec_route && T <= kFusedRouteMaxT;
 

@@ -115,7 +115,7 @@ struct colibri_ctx {
   bool use_graphs = true;
   bool use_pdl = false;  // programmatic dependent launch between the kernels of a forward (opt-in)
   bool dec_fused = true;  // int8 weights: the one-launch expert stage (COLIBRI_DEC_FUSED=0: four launches)
-  bool dec_route = false; // int8, T <= 64: routing inside that launch too (COLIBRI_DEC_ROUTE=1)
+  bool dec_route = true;  // int8, T <= 64: routing inside that launch too (COLIBRI_DEC_ROUTE=0: not)
 };
 
 namespace colibri {
@@ -534,6 +534,20 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
       "%4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
+}
+
+// Prefetch of a tensor tile into L2 only (no shared memory, no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap* map, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
 }
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

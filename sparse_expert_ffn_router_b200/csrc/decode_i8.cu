@@ -111,6 +111,7 @@ constexpr int kDsTmemCols = 256;
 constexpr size_t kDsRingBytes = 200 * 1024;
 constexpr int kDsMaxStages = 12;
 constexpr int kDsMaxKbs = 4;
+constexpr int kDsPrefetchBlocks = 24;  // weight blocks (16 KB each) pulled into L2 while the ring waits
 
 struct alignas(64) DecStreamParams {
   CUtensorMap mapW;   // int8 weights: gate/up {d, f, 2, E} (W1, W3); down {f, d, E} (W2)
@@ -195,6 +196,7 @@ struct DsCtl {
   int issued;    // copies issued / stages consumed, for the error path
   int consumed;
   int flag;      // result of a grid-wide wait, broadcast to the epilogue warps
+  int first;     // this CTA's first work item (items first, first + gridDim.x, ...)
   int ntouched;
   int32_t off[kMaxExperts + 1];     // row offsets of the experts' groups
   int32_t touched[kMaxExperts];
@@ -246,6 +248,24 @@ __device__ bool ds_produce(const DecStreamParams& p, uint8_t* smem, DsCtl& c, in
   const uint64_t policy = l2_evict_first_policy();
   int held = 0;
   bool released = !defer;
+  // L2 prefetch of the weight blocks that follow the current position (item L, next block kb,
+  // `left` blocks left in that item), up to kDsPrefetchBlocks blocks.
+  auto prefetch_ahead = [&](int L, int kb, int left) {
+    int n = 0;
+    DecItem q;
+    for (int L2 = L; n < kDsPrefetchBlocks && dec_item<kGateUp>(p, c.touched, c.pre[pre_idx], c.ntouched, c.off, L2, q);
+         L2 += gridDim.x) {
+      const int kbeg = q.split * p.kspan, kend = min(p.K, kbeg + p.kspan);
+      const int nkb2 = (kend - kbeg + 127) / 128;
+      int b = (L2 == L) ? kb : L2 % nkb2;
+      int cnt = (L2 == L) ? left : nkb2;
+      for (; cnt > 0 && n < kDsPrefetchBlocks; --cnt, ++n, b = (b + 1 == nkb2) ? 0 : b + 1) {
+        const int kx = kbeg + b * 128;
+        if (kGateUp) tma_prefetch_l2_4d(&p.mapW, kx, q.tile * 128, q.mat, q.e);
+        else tma_prefetch_l2_3d(&p.mapW, kx, q.tile * 128, q.e);
+      }
+    }
+  };
   auto release = [&]() {
     for (int h = 0; h < held; ++h) {
       uint8_t* st = smem + (size_t)c.defer_s[h] * p.stage_bytes;
@@ -254,7 +274,7 @@ __device__ bool ds_produce(const DecStreamParams& p, uint8_t* smem, DsCtl& c, in
     }
   };
   DecItem it;
-  for (int L = blockIdx.x; dec_item<kGateUp>(p, c.touched, c.pre[pre_idx], c.ntouched, c.off, L, it); L += gridDim.x) {
+  for (int L = c.first; dec_item<kGateUp>(p, c.touched, c.pre[pre_idx], c.ntouched, c.off, L, it); L += gridDim.x) {
     // The item's K blocks start at a rotated block (item index mod block count): items in flight
     // at the same time then read different column offsets of their weight rows, which spreads
     // the requests over the DRAM channels instead of hitting the same address bits everywhere.
@@ -285,6 +305,9 @@ __device__ bool ds_produce(const DecStreamParams& p, uint8_t* smem, DsCtl& c, in
         c.defer_nk[held] = nk;
         c.defer_s[held] = r.s;
         if (++held == S) {
+          // The ring is full of weight copies and the planes are not ready yet: pull the next
+          // weight blocks of this CTA into L2 meanwhile, so the stream resumes from L2.
+          prefetch_ahead(L, kb, nkb - i - nk);
           // the held plane copies are issued even when the wait gave up, so that every issued
           // stage completes and the error path drains quickly
           const bool go = ready();
@@ -313,7 +336,7 @@ __device__ bool ds_mma(const DecStreamParams& p, uint8_t* smem, DsCtl& c, int S,
   const uint32_t idesc = idesc_s8_s32(128, N);
   const uint32_t plane_bytes = (uint32_t)(2 * p.nt8 * 128);
   DecItem it;
-  for (int L = blockIdx.x; dec_item<kGateUp>(p, c.touched, c.pre[pre_idx], c.ntouched, c.off, L, it);
+  for (int L = c.first; dec_item<kGateUp>(p, c.touched, c.pre[pre_idx], c.ntouched, c.off, L, it);
        L += gridDim.x, ++iter) {
     const int a = iter & 1;
     const uint32_t aph = (uint32_t)(iter >> 1) & 1u;
@@ -353,7 +376,7 @@ __device__ bool ds_epilogue(const DecStreamParams& p, DsCtl& c, int pre_idx, int
   const int q = warp & 3;
   const int N = 2 * p.nt8;
   DecItem it;
-  for (int L = blockIdx.x; dec_item<kGateUp>(p, c.touched, c.pre[pre_idx], c.ntouched, c.off, L, it);
+  for (int L = c.first; dec_item<kGateUp>(p, c.touched, c.pre[pre_idx], c.ntouched, c.off, L, it);
        L += gridDim.x, ++iter) {
     const int a = iter & 1;
     const uint32_t aph = (uint32_t)(iter >> 1) & 1u;
@@ -424,6 +447,7 @@ __device__ __forceinline__ void ds_init(const DecStreamParams* const* phases, in
     c.issued = 0;
     c.consumed = 0;
     c.flag = 0;
+    c.first = blockIdx.x;
     mbar_fence_init();
     for (int i = 0; i < nphases; ++i) {
       tma_prefetch_desc(&phases[i]->mapW);
@@ -594,12 +618,22 @@ __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" :::
 // Arrives on the planes barrier; the producer waits on it before its first plane copy.
 __device__ void fused_route(const DecFusedParams& p, uint8_t* smem, DsCtl& c) {
   constexpr int kWarps = kDsThreads / 32;
+  constexpr int kRedundantT = 1;  // up to this many tokens every CTA routes all of them itself
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, T = p.T, k = p.k, E = p.gu.E, d = p.gu.d;
   const int nvec = d / 8;  // 16-byte slices of a bf16 row
-  float* part = reinterpret_cast<float*>(smem);      // [kWarps][E]
-  float* lg = part + kWarps * kMaxExperts;           // [E]
-  for (int t = blockIdx.x; p.route_in_kernel == 1 && t < T; t += G) {  // 2: the caller routed
+  // scratch in the ring (idle until the producer starts)
+  float* part = reinterpret_cast<float*>(smem);                         // [kWarps][kMaxExperts]
+  float* lg = part + kWarps * kMaxExperts;                              // [kMaxExperts]
+  int32_t* s_idx = reinterpret_cast<int32_t*>(smem + 8192);             // [T * k]
+  float* s_w = reinterpret_cast<float*>(smem + 10240);                  // [T * k]
+  unsigned long long* mask = reinterpret_cast<unsigned long long*>(smem + 12288);  // [E] tokens choosing e
+  float* red = reinterpret_cast<float*>(smem + 14336);                  // [kWarps]
+  // A single token is routed by every CTA itself (the router weights are read from L2 by each
+  // CTA), which saves a grid barrier; with more tokens CTA t routes token t and a barrier
+  // follows (8 tokens routed in every CTA measured 20% slower at T=8).
+  const bool redundant = p.route_in_kernel == 1 && T <= kRedundantT;
+  for (int t = redundant ? 0 : blockIdx.x; p.route_in_kernel == 1 && t < T; t += redundant ? 1 : G) {
     const uint4* xv = reinterpret_cast<const uint4*>(p.x + (size_t)t * d);
     for (int e0 = 0; e0 < E; e0 += 8) {
       float acc[8];
@@ -631,24 +665,39 @@ __device__ void fused_route(const DecFusedParams& p, uint8_t* smem, DsCtl& c) {
       lg[e] = sum + (p.router_b ? p.router_b[e] : 0.f);
     }
     __syncthreads();
-    if (warp == 0) warp_topk(lg, E, k, lane, p.topk_idx + (size_t)t * k, p.topk_w + (size_t)t * k);
+    if (warp == 0) {
+      if (redundant) {
+        warp_topk(lg, E, k, lane, s_idx + (size_t)t * k, s_w + (size_t)t * k);
+        __syncwarp();
+        if (blockIdx.x == 0 && lane < k) {  // one CTA publishes the choices
+          p.topk_idx[(size_t)t * k + lane] = s_idx[(size_t)t * k + lane];
+          p.topk_w[(size_t)t * k + lane] = s_w[(size_t)t * k + lane];
+        }
+      } else {
+        warp_topk(lg, E, k, lane, p.topk_idx + (size_t)t * k, p.topk_w + (size_t)t * k);
+      }
+    }
     __syncthreads();
   }
-  // every token's choices are needed below
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    atomicAdd(&p.bar[kBarRouter], 1);
-    c.flag = grid_wait(&p.bar[kBarRouter], G, &c.abort) ? 1 : 0;
-    if (!c.flag) ds_abort(c, p.gu.err);
+  c.flag = 1;
+  if (p.route_in_kernel == 1 && !redundant) {
+    // every token's choices are needed below
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+      atomicAdd(&p.bar[kBarRouter], 1);
+      c.flag = grid_wait(&p.bar[kBarRouter], G, &c.abort) ? 1 : 0;
+      if (!c.flag) ds_abort(c, p.gu.err);
+    }
+    __syncthreads();
   }
-  __syncthreads();
-  unsigned long long* mask = reinterpret_cast<unsigned long long*>(smem);  // [E] tokens choosing e
+  // the choices: this CTA's own copy, or from global memory (another CTA's, or the caller's)
+  auto choice = [&](int i) { return redundant ? s_idx[i] : __ldcg(p.topk_idx + i); };
   for (int e = tid; e < E; e += kDsThreads) mask[e] = 0ull;
   __syncthreads();
   if (c.flag) {
     for (int i = tid; i < T * k; i += kDsThreads) {
-      const int e = min(max(__ldcg(p.topk_idx + i), 0), E - 1);
+      const int e = min(max(choice(i), 0), E - 1);
       atomicOr(&mask[e], 1ull << (i / k));
     }
   }
@@ -680,14 +729,13 @@ __device__ void fused_route(const DecFusedParams& p, uint8_t* smem, DsCtl& c) {
     }
   }
   __syncthreads();
-  float* red = reinterpret_cast<float*>(smem + (size_t)kMaxExperts * sizeof(unsigned long long));  // [kWarps]
   for (int t = blockIdx.x; t < T && c.flag; t += G) {
     int rows[kMaxTopK];
 #pragma unroll
     for (int j = 0; j < kMaxTopK; ++j) {
       rows[j] = 0;
       if (j < k) {
-        const int e = min(max(__ldcg(p.topk_idx + (size_t)t * k + j), 0), E - 1);
+        const int e = min(max(choice(t * k + j), 0), E - 1);
         rows[j] = c.off[e] + __popcll(mask[e] & ((1ull << t) - 1ull));
       }
     }
@@ -757,6 +805,9 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_c
     ds_init(phases, 2, c, S);
     if (p.route_in_kernel) {
       fused_route(p, smem, c);
+      // CTAs 0..T-1 also split their token's planes and start last: the items are dealt so
+      // that the CTAs that take one item more than the others are not among them
+      if (threadIdx.x == 0) c.first = (int)((blockIdx.x + gridDim.x - (unsigned)min(p.T, (int)gridDim.x)) % gridDim.x);
       ds_items(phases, 2, c, nullptr);
     } else {
       ds_items(phases, 2, c, p.gu.offsets);

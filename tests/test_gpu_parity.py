@@ -72,8 +72,8 @@ I8_SMALL = [n for n, w in SMALL.items() if w.wdt == I8]
 @pytest.mark.parametrize("name", I8_SMALL)
 def test_int8_each_launch_plan(name, fused, route, monkeypatch):
     # fused "1": gate/up, H planes, down and combine in one cooperative launch (the default);
-    # "0": the same stages as four launches.  route "1": for T <= 64 the router, top-k and
-    # grouping run inside that launch too.
+    # "0": the same stages as four launches.  route "1" (the default): for T <= 64 the router,
+    # top-k and grouping run inside that launch too.
     monkeypatch.setenv("COLIBRI_DEC_FUSED", fused)
     monkeypatch.setenv("COLIBRI_DEC_ROUTE", route)
     wl = SMALL[name]
@@ -274,11 +274,13 @@ def test_forward_inside_a_user_cuda_graph():
     layer.close()
 
 
-@pytest.mark.parametrize("name", ["bf16_ragged", "f32_tiny", "i8_small", "i8_small_route", "bf16_shared"])
+@pytest.mark.parametrize("name", ["bf16_ragged", "f32_tiny", "i8_small", "i8_small_split", "bf16_shared"])
 def test_forward_routed_matches_oracle_routing(name, monkeypatch):
-    if name.endswith("_route"):  # the grouping inside the fused int8 launch, on caller routing
-        monkeypatch.setenv("COLIBRI_DEC_ROUTE", "1")
-        name = name[: -len("_route")]
+    # "_split": the plan with separate routing launches before the fused int8 launch (the
+    # default groups inside it)
+    if name.endswith("_split"):
+        monkeypatch.setenv("COLIBRI_DEC_ROUTE", "0")
+        name = name[: -len("_split")]
     wl = SMALL[name]
     p = inputgen.make_problem(wl, seed=3)
     ref = oracle.problem_forward(p)
