@@ -51,6 +51,15 @@ typedef enum {
 
 typedef enum { COLIBRI_F32 = 0, COLIBRI_BF16 = 1, COLIBRI_I8 = 2 } colibri_dtype;
 
+/* Router variants, OR-ed into colibri_desc.router_flags (0 = the default router). */
+typedef enum {
+  COLIBRI_ROUTER_CLAMP = 1,       /* clamp every logit to [-50, 50] before selection and
+                                     weighting (www.0539edu.com/news/4774449 §5.2, the
+                                     gate-softmax clip option against overflow)              */
+  COLIBRI_ROUTER_RAW_WEIGHTS = 2  /* combine weights = the k chosen logits themselves, no
+                                     softmax (www.hotelren.com/news/4731937 §3.2)             */
+} colibri_router_flag;
+
 /*
  * Layer description, fixed for the life of a context.
  *   d_model, d_ff   hidden size d and routed-expert FFN size f; both multiples of 64.
@@ -68,6 +77,11 @@ typedef enum { COLIBRI_F32 = 0, COLIBRI_BF16 = 1, COLIBRI_I8 = 2 } colibri_dtype
  *                   The shared expert is available for (F32, F32) and (BF16, BF16).
  *   max_tokens      largest T a forward may be called with (sizes the workspace).
  *   device_id       CUDA device the context lives on.
+ *   router_flags    0, or COLIBRI_ROUTER_* bits.  Default: weights are the softmax over all E
+ *                   logits renormalised over the k chosen.  Selection (logit descending, lower
+ *                   expert index on ties) is the same for every variant, applied to the clamped
+ *                   logits when COLIBRI_ROUTER_CLAMP is set (logits above 50 then tie and go to
+ *                   the lower index).  Unknown bits: COLIBRI_ERR_INVALID_ARG.
  */
 typedef struct {
   int32_t d_model;
@@ -79,6 +93,7 @@ typedef struct {
   int32_t weight_dtype;
   int32_t max_tokens;
   int32_t device_id;
+  int32_t router_flags;
 } colibri_desc;
 
 typedef struct colibri_ctx colibri_ctx; /* opaque */
@@ -196,7 +211,8 @@ colibri_status colibri_profile_end(colibri_ctx* ctx, float* stage_ms, int32_t* n
  * context and no device allocation of any kind.  The pages have no counterpart of this call;
  * it exists for callers that cannot call cudaMalloc, such as an engine whose device memory is
  * reserved up front by its own allocator (an extra allocation would fail or fragment it) or a
- * latency-critical loop that must not pay cudaMalloc's implicit synchronisation.
+ * latency-critical loop that must not pay cudaMalloc's implicit synchronisation.  It runs the
+ * default router (router_flags = 0).
  *   x [T, d_model] act_dtype (COLIBRI_F32 or COLIBRI_BF16), router_w [E, d_model] act_dtype,
  *   router_b [E] fp32 or NULL; outputs topk_idx/topk_w/dst_row [T, k], counts [E],
  *   offsets [E+1], src_row [T*k] and Xp [T*k, d_model] (x's rows grouped by expert, act_dtype),

@@ -37,20 +37,23 @@ def _load():
             build()
         lib = ctypes.CDLL(_LIB_PATH)
         vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
-        lib.oracle_router_logits.argtypes = [vp, i32, i32, i32, vp, vp, i32, vp]
-        lib.oracle_weights_for.argtypes = [vp, i32, i32, i32, vp, vp]
-        lib.oracle_topk.argtypes = [vp, i32, i32, i32, vp, vp, vp]
+        lib.oracle_router_logits.argtypes = [vp, i32, i32, i32, vp, vp, i32, i32, vp]
+        lib.oracle_weights_for.argtypes = [vp, i32, i32, i32, vp, i32, vp]
+        lib.oracle_topk.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp]
         lib.oracle_group.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp]
         lib.oracle_expert_row.argtypes = [vp, i32, i32, i32, vp, i32, i64, i32, vp, i32, vp]
         lib.oracle_combine.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, i32, i64, i32, vp, vp,
                                        i32, vp, i32, vp]
-        lib.oracle_moe_forward.argtypes = [vp, i32, i32, i32, vp, vp, i32, i32, vp, i32, i64, i32,
+        lib.oracle_moe_forward.argtypes = [vp, i32, i32, i32, vp, vp, i32, i32, i32, vp, i32, i64, i32,
                                            vp, vp, i32] + [vp] * 8
         for n in ("oracle_router_logits", "oracle_weights_for", "oracle_topk", "oracle_group",
                   "oracle_expert_row", "oracle_combine", "oracle_moe_forward"):
             getattr(lib, n).restype = ctypes.c_int
         _lib = lib
     return _lib
+
+
+ROUTER_CLAMP, ROUTER_RAW = 1, 2  # router variants (logit clamp to [-50, 50]; raw-logit weights)
 
 
 def _ptr(t):
@@ -65,31 +68,35 @@ def _check(rc, what):
         raise RuntimeError(f"oracle {what} failed with code {rc}")
 
 
-def router_logits(x: torch.Tensor, router_w: torch.Tensor, router_b: Optional[torch.Tensor]) -> torch.Tensor:
+def router_logits(x: torch.Tensor, router_w: torch.Tensor, router_b: Optional[torch.Tensor],
+                  flags: int = 0) -> torch.Tensor:
+    """Logits [T, E] float32; ``flags`` & ROUTER_CLAMP limits them to [-50, 50]."""
     T, d = x.shape
     E = router_w.shape[0]
     out = torch.empty(T, E, dtype=torch.float32)
     _check(_load().oracle_router_logits(_ptr(x), _CODE[x.dtype], T, d, _ptr(router_w), _ptr(router_b), E,
-                                        _ptr(out)), "router_logits")
+                                        flags, _ptr(out)), "router_logits")
     return out
 
 
-def topk(logits: torch.Tensor, k: int):
-    """(idx [T,k] int32, w [T,k] f32, gap [T] f32) with the oracle's selection rule."""
+def topk(logits: torch.Tensor, k: int, flags: int = 0):
+    """(idx [T,k] int32, w [T,k] f32, gap [T] f32) with the oracle's selection rule; ``flags`` &
+    ROUTER_RAW makes the weights the chosen logits."""
     T, E = logits.shape
     idx = torch.empty(T, k, dtype=torch.int32)
     w = torch.empty(T, k, dtype=torch.float32)
     gap = torch.empty(T, dtype=torch.float32)
-    _check(_load().oracle_topk(_ptr(logits.contiguous()), T, E, k, _ptr(idx), _ptr(w), _ptr(gap)), "topk")
+    _check(_load().oracle_topk(_ptr(logits.contiguous()), T, E, k, flags, _ptr(idx), _ptr(w), _ptr(gap)),
+           "topk")
     return idx, w, gap
 
 
-def weights_for(logits: torch.Tensor, idx: torch.Tensor) -> torch.Tensor:
+def weights_for(logits: torch.Tensor, idx: torch.Tensor, flags: int = 0) -> torch.Tensor:
     T, E = logits.shape
     k = idx.shape[1]
     w = torch.empty(T, k, dtype=torch.float32)
-    _check(_load().oracle_weights_for(_ptr(logits.contiguous()), T, E, k, _ptr(idx.contiguous()), _ptr(w)),
-           "weights_for")
+    _check(_load().oracle_weights_for(_ptr(logits.contiguous()), T, E, k, _ptr(idx.contiguous()), flags,
+                                      _ptr(w)), "weights_for")
     return w
 
 
@@ -128,7 +135,7 @@ def combine(x: torch.Tensor, idx: torch.Tensor, w: torch.Tensor, expert_w: torch
     return y
 
 
-def moe_forward(x, router_w, router_b, k, expert_w, stride, f, scales=None, shared_w=None, fs=0):
+def moe_forward(x, router_w, router_b, k, expert_w, stride, f, scales=None, shared_w=None, fs=0, flags=0):
     """Whole layer on the host.  Returns a dict of every intermediate the GPU path exposes."""
     T, d = x.shape
     E = router_w.shape[0]
@@ -143,18 +150,18 @@ def moe_forward(x, router_w, router_b, k, expert_w, stride, f, scales=None, shar
         y=torch.empty(T, d, dtype=torch.float32),
     )
     rc = _load().oracle_moe_forward(
-        _ptr(x), _CODE[x.dtype], T, d, _ptr(router_w), _ptr(router_b), E, k, _ptr(expert_w),
+        _ptr(x), _CODE[x.dtype], T, d, _ptr(router_w), _ptr(router_b), E, k, flags, _ptr(expert_w),
         _CODE[expert_w.dtype], stride, f, _ptr(scales), _ptr(shared_w), fs,
         *[_ptr(out[n]) for n in ("logits", "idx", "w", "counts", "offsets", "src_row", "dst_row", "y")])
     _check(rc, "moe_forward")
     return out
 
 
-def problem_forward(p, tokens: Optional[Sequence[int]] = None):
+def problem_forward(p, tokens: Optional[Sequence[int]] = None, flags: int = 0):
     """Oracle on an ``inputgen.Problem``: routing for all tokens, y for `tokens` (default: all)."""
     wl = p.wl
-    logits = router_logits(p.x, p.router_w, p.router_b)
-    idx, w, gap = topk(logits, wl.k)
+    logits = router_logits(p.x, p.router_w, p.router_b, flags)
+    idx, w, gap = topk(logits, wl.k, flags)
     counts, offsets, src, dst = group(idx, wl.E)
     toks = list(range(wl.T)) if tokens is None else list(tokens)
     y = combine(p.x, idx, w, p.expert_w, p.expert_stride, wl.f, p.expert_scales, p.shared_w, wl.fs, toks)

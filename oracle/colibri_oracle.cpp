@@ -19,7 +19,10 @@
 //
 // Readings taken where the pages are silent or disagree:
 //   * weights are the softmax over all E logits renormalised over the k chosen, which is
-//     exp(l_j - l_0) / sum_j' exp(l_j' - l_0) over the chosen set;
+//     exp(l_j - l_0) / sum_j' exp(l_j' - l_0) over the chosen set; the raw-logit variant
+//     ([hotelren] §3.2: no softmax) takes the chosen logits themselves as the weights;
+//   * the clamp variant limits the logits to [-50, 50] before selection and weighting, so
+//     logits beyond 50 tie and the tie rule below decides;
 //   * ties in the logits go to the lower expert index;
 //   * slot 0 holds the largest logit;
 //   * the expert FFN is SwiGLU: W2 (silu(W1 x) * (W3 x)), no biases;
@@ -38,6 +41,10 @@ namespace {
 
 enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_I8 = 2 };
 enum { ORC_OK = 0, ORC_EARG = -1, ORC_ENONFINITE = -2 };
+// Router variants: clamp the logits to [-50, 50] ([0539edu] §5.2, the gate-softmax clip
+// option against overflow); use the chosen raw logits as the combine weights, no softmax
+// ([hotelren] §3.2).
+enum { ORC_ROUTER_CLAMP = 1, ORC_ROUTER_RAW = 2 };
 
 // Exact widening of one stored element to double.
 inline double widen(const void* p, int dtype, int64_t i) {
@@ -101,15 +108,18 @@ extern "C" {
 // Step 1, router logits: l[t][e] = b[e] + sum_i x[t][i] * Wr[e][i].
 // [0539edu] §2.1 (gate output of shape [batch, seq_len, num_experts], then softmax and
 // top-k); [hotelren] §3.2 (linear projection input @ router_weight + router_bias).
+// With ORC_ROUTER_CLAMP in `flags` each logit is then limited to [-50, 50] ([0539edu] §5.2).
 int oracle_router_logits(const void* x, int act, int T, int d, const void* wr, const float* b,
-                         int E, float* logits) {
+                         int E, int flags, float* logits) {
   if (T < 0 || d <= 0 || E <= 0 || (T > 0 && (!x || !wr || !logits))) return ORC_EARG;
+  if (flags & ~(ORC_ROUTER_CLAMP | ORC_ROUTER_RAW)) return ORC_EARG;
   for (int t = 0; t < T; ++t) {
     for (int e = 0; e < E; ++e) {
       double acc = 0.0;
       for (int i = 0; i < d; ++i)
         acc += widen(x, act, (int64_t)t * d + i) * widen(wr, act, (int64_t)e * d + i);
       if (b) acc += (double)b[e];
+      if (flags & ORC_ROUTER_CLAMP) acc = std::min(50.0, std::max(-50.0, acc));
       logits[(int64_t)t * E + e] = (float)acc;
       if (!std::isfinite(logits[(int64_t)t * E + e])) return ORC_ENONFINITE;
     }
@@ -120,8 +130,11 @@ int oracle_router_logits(const void* x, int act, int T, int d, const void* wr, c
 // Step 2/3 weights for a given selection: w_j = exp(l_j - l_0) / sum_j' exp(l_j' - l_0),
 // which equals the softmax over all E renormalised over the chosen k (the common
 // normaliser cancels).  [0539edu] §2.1 softmax then top-k; renormalised over the chosen k.
-int oracle_weights_for(const float* logits, int T, int E, int k, const int32_t* idx, float* w) {
+// With ORC_ROUTER_RAW in `flags`, w_j = l_j: the raw logit of each chosen expert ([hotelren]
+// §3.2 skips the softmax).
+int oracle_weights_for(const float* logits, int T, int E, int k, const int32_t* idx, int flags, float* w) {
   if (T < 0 || E <= 0 || k <= 0 || k > E) return ORC_EARG;
+  if (flags & ~(ORC_ROUTER_CLAMP | ORC_ROUTER_RAW)) return ORC_EARG;
   for (int t = 0; t < T; ++t) {
     const float* l = logits + (int64_t)t * E;
     const int32_t* id = idx + (int64_t)t * k;
@@ -129,6 +142,10 @@ int oracle_weights_for(const float* logits, int T, int E, int k, const int32_t* 
     for (int j = 0; j < k; ++j) {
       if (id[j] < 0 || id[j] >= E) return ORC_EARG;
       lmax = std::max(lmax, (double)l[id[j]]);
+    }
+    if (flags & ORC_ROUTER_RAW) {
+      for (int j = 0; j < k; ++j) w[(int64_t)t * k + j] = l[id[j]];
+      continue;
     }
     double den = 0.0;
     for (int j = 0; j < k; ++j) den += std::exp((double)l[id[j]] - lmax);
@@ -141,7 +158,7 @@ int oracle_weights_for(const float* logits, int T, int E, int k, const int32_t* 
 // first k, slot 0 = largest.  The strict ">" of the per-token scan in [mhpq] §3.2 keeps the
 // lower index on ties.  Also reports gap[t] = l_(k) - l_(k+1), the distance between the last
 // chosen and the first unchosen logit (+inf when k == E), for the near-tie protocol.
-int oracle_topk(const float* logits, int T, int E, int k, int32_t* idx, float* w, float* gap) {
+int oracle_topk(const float* logits, int T, int E, int k, int flags, int32_t* idx, float* w, float* gap) {
   if (T < 0 || E <= 0 || k <= 0 || k > E) return ORC_EARG;
   std::vector<int> order(E);
   for (int t = 0; t < T; ++t) {
@@ -153,7 +170,7 @@ int oracle_topk(const float* logits, int T, int E, int k, int32_t* idx, float* w
     for (int j = 0; j < k; ++j) idx[(int64_t)t * k + j] = order[j];
     if (gap) gap[t] = (k < E) ? (float)((double)l[order[k - 1]] - (double)l[order[k]]) : INFINITY;
   }
-  return w ? oracle_weights_for(logits, T, E, k, idx, w) : ORC_OK;
+  return w ? oracle_weights_for(logits, T, E, k, idx, flags, w) : ORC_OK;
 }
 
 // Steps 4/5, counts, offsets and the permutation that groups rows by expert.
@@ -232,7 +249,7 @@ int oracle_combine(const void* x, int act, int T, int d, int k, const int32_t* i
 
 // The whole layer: steps 1-7 for every token.  Any output pointer may be NULL except y.
 int oracle_moe_forward(const void* x, int act, int T, int d, const void* router_w,
-                       const float* router_b, int E, int k, const void* expert_w, int wdt,
+                       const float* router_b, int E, int k, int flags, const void* expert_w, int wdt,
                        int64_t stride, int f, const float* scales, const void* shared_w, int fs,
                        float* logits_out, int32_t* idx_out, float* w_out, int32_t* counts,
                        int32_t* offsets, int32_t* src_row, int32_t* dst_row, float* y) {
@@ -241,9 +258,9 @@ int oracle_moe_forward(const void* x, int act, int T, int d, const void* router_
   if (!y) return ORC_EARG;
   std::vector<float> logits((size_t)T * E), wv((size_t)T * k);
   std::vector<int32_t> iv((size_t)T * k), cnt(E), off(E + 1), src((size_t)T * k), dst((size_t)T * k);
-  int rc = oracle_router_logits(x, act, T, d, router_w, router_b, E, logits.data());
+  int rc = oracle_router_logits(x, act, T, d, router_w, router_b, E, flags, logits.data());
   if (rc) return rc;
-  rc = oracle_topk(logits.data(), T, E, k, iv.data(), wv.data(), nullptr);
+  rc = oracle_topk(logits.data(), T, E, k, flags, iv.data(), wv.data(), nullptr);
   if (rc) return rc;
   rc = oracle_group(iv.data(), T, k, E, cnt.data(), off.data(), src.data(), dst.data());
   if (rc) return rc;

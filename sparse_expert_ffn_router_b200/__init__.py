@@ -17,6 +17,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libcolibri.so")
 
 COLIBRI_F32, COLIBRI_BF16, COLIBRI_I8 = 0, 1, 2
+COLIBRI_ROUTER_CLAMP, COLIBRI_ROUTER_RAW_WEIGHTS = 1, 2
 
 STATUS = {
     0: "COLIBRI_OK",
@@ -57,6 +58,7 @@ class colibri_desc(ctypes.Structure):
         ("weight_dtype", ctypes.c_int32),
         ("max_tokens", ctypes.c_int32),
         ("device_id", ctypes.c_int32),
+        ("router_flags", ctypes.c_int32),
     ]
 
 
@@ -142,10 +144,10 @@ def colibri_last_error(ctx=None) -> str:
 
 def colibri_init(d_model: int, d_ff: int, num_experts: int, top_k: int, shared_d_ff: int = 0,
                  act_dtype: int = COLIBRI_BF16, weight_dtype: int = COLIBRI_BF16, max_tokens: int = 1,
-                 device_id: int = 0) -> int:
+                 device_id: int = 0, router_flags: int = 0) -> int:
     """Returns the opaque context handle (an address)."""
     desc = colibri_desc(d_model, d_ff, num_experts, top_k, shared_d_ff, act_dtype, weight_dtype,
-                        max_tokens, device_id)
+                        max_tokens, device_id, router_flags)
     out = ctypes.c_void_p()
     _check(load().colibri_init(ctypes.byref(desc), ctypes.byref(out)), "colibri_init")
     return out.value
@@ -220,10 +222,10 @@ class MoELayer:
     """Owns one context; forwards tensors to the C ABI (no computation in Python)."""
 
     def __init__(self, d_model, d_ff, num_experts, top_k, shared_d_ff=0, act_dtype=COLIBRI_BF16,
-                 weight_dtype=COLIBRI_BF16, max_tokens=1, device_id=0):
+                 weight_dtype=COLIBRI_BF16, max_tokens=1, device_id=0, router_flags=0):
         self.desc = dict(d_model=d_model, d_ff=d_ff, num_experts=num_experts, top_k=top_k,
                          shared_d_ff=shared_d_ff, act_dtype=act_dtype, weight_dtype=weight_dtype,
-                         max_tokens=max_tokens, device_id=device_id)
+                         max_tokens=max_tokens, device_id=device_id, router_flags=router_flags)
         self.ctx = colibri_init(**self.desc)
 
     @property

@@ -159,6 +159,8 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
     return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "top_k=%d must be in [1, min(E, %d)]", D.top_k, kMaxTopK);
   if (D.max_tokens < 1)
     return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "max_tokens=%d must be >= 1", D.max_tokens);
+  if (D.router_flags & ~(COLIBRI_ROUTER_CLAMP | COLIBRI_ROUTER_RAW_WEIGHTS))
+    return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "router_flags=0x%x has unknown bits", (unsigned)D.router_flags);
   if ((int64_t)D.max_tokens * D.top_k > (1ll << 30))
     return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "max_tokens * top_k too large");
   const bool f32 = D.act_dtype == COLIBRI_F32 && D.weight_dtype == COLIBRI_F32;
@@ -365,7 +367,7 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
     COLIBRI_TRY(cudaMemcpyAsync(w.topk_w, user_w, (size_t)R * 4, cudaMemcpyDeviceToDevice, s), "copy topk_w");
     launch_chain_break();
   } else if (!route_in_dec) {
-    COLIBRI_TRY(launch_router_topk(xd, act, T, d, router_w, router_b, E, k, w.topk_idx, w.topk_w, w.err,
+    COLIBRI_TRY(launch_router_topk(xd, act, T, d, router_w, router_b, E, k, D.router_flags, w.topk_idx, w.topk_w, w.err,
                                    w.router_part, w.router_ticket, s),
                 "router_topk");
   }
@@ -446,7 +448,8 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
       const int touched = std::min(E, R), tiles = (d + 127) / 128;
       while (nsplit < ctx->dec_split && touched * tiles * nsplit < 4 * ctx->sm_count) nsplit <<= 1;
     }
-    // K splits of the gate/up projection (partials summed before SiLU by the finishing kernel)
+    // K splits of the gate/up projection (partials summed before SiLU by the finishing kernel).
+    // Up to 4: 8 splits (64 KB items) measured slower for one token (gate/up phase 5 us longer).
     int gsplit = 1;
     if (R <= kDecGateSplitRows && d % 128 == 0) {
       const int touched = std::min(E, R), tiles = 2 * ((f + 127) / 128);
@@ -483,6 +486,7 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
         fa.x = (const __nv_bfloat16*)xd;
         fa.router_w = (const __nv_bfloat16*)router_w;
         fa.router_b = router_b;
+        fa.router_flags = D.router_flags;
         fa.topk_idx = w.topk_idx;
         fa.counts = w.counts;
         fa.offsets_out = w.offsets;
@@ -676,6 +680,9 @@ colibri_status colibri_sync_status(colibri_ctx* ctx, void* stream) {
   COLIBRI_TRY(cudaMemcpy(&err, ctx->ws.err, 4, cudaMemcpyDeviceToHost), "read error word");
   if (err) {
     COLIBRI_TRY(cudaMemset(ctx->ws.err, 0, 4), "clear error word");
+    // a wait that gave up may leave the fused kernel's grid-barrier counters out of step
+    if (ctx->ws.grid_bar)
+      COLIBRI_TRY(cudaMemset(ctx->ws.grid_bar, 0, kFusedBarCount * 4), "reset grid-barrier counters");
     return fail(ctx, COLIBRI_ERR_TIMEOUT, "device error word 0x%x (a bounded wait gave up)", err);
   }
   return COLIBRI_OK;

@@ -189,7 +189,7 @@ constexpr int kRouterSplitMinT = 2048;  // T from which the tensor-core router s
 constexpr int kRouterMaxSplit = 8;
 int router_ksplit(int T, int d);
 cudaError_t launch_router_topk(const void* x, int act, int T, int d, const void* wr, const float* b,
-                               int E, int k, int32_t* idx, float* w, uint32_t* err, float* part,
+                               int E, int k, int rflags, int32_t* idx, float* w, uint32_t* err, float* part,
                                int32_t* ticket, cudaStream_t s);
 cudaError_t launch_route_count(const int32_t* idx, int T, int k, int E, int32_t* blk_counts,
                                int32_t* local_rank, cudaStream_t s);
@@ -304,7 +304,8 @@ struct DecFusedArgs {
   float* GU;                // [gsplit, 2, R, f]
   float* Ypart;             // [dsplit, R, d]
   __nv_bfloat16* y;         // [T, d]
-  int32_t* bar;             // [kFusedBarCount] zeroed counters
+  int32_t* bar;             // [kFusedBarCount] grid-barrier counters: zero at first use, then
+                            // owned by the kernel (never reset between launches)
   uint32_t* err;
   // T <= 64: 1 = router, top-k and grouping in the same launch; 2 = grouping only (topk_idx and
   // topk_w given); 0 = all done by earlier launches
@@ -312,6 +313,7 @@ struct DecFusedArgs {
   const __nv_bfloat16* x = nullptr;         // [T, d]
   const __nv_bfloat16* router_w = nullptr;  // [E, d]
   const float* router_b = nullptr;
+  int router_flags = 0;                     // kRouterClamp | kRouterRaw
   int32_t* topk_idx = nullptr;              // [T, k]
   int32_t* counts = nullptr;                // [E]
   int32_t* offsets_out = nullptr;           // [E+1]
@@ -333,14 +335,40 @@ __device__ __forceinline__ void split_planes(float x, float a, float inv_a, int&
   qh = (int)h;
   ql = (int)l;
 }
-// One warp selects the top-k of one token whose E logits sit in shared memory.
-__device__ __forceinline__ void warp_topk(const float* lg, int E, int k, int lane, int32_t* idx_out,
+// Router variants (colibri_desc.router_flags).  kRouterClamp limits every logit to [-50, 50]
+// before selection and weighting (the gate-softmax clip option of
+// www.0539edu.com/news/4774449 §5.2); kRouterRaw makes the combine weights the chosen logits
+// themselves, with no softmax (www.hotelren.com/news/4731937 §3.2).  Selection is unchanged.
+constexpr int kRouterClamp = 1;
+constexpr int kRouterRaw = 2;
+__device__ __forceinline__ float router_clamp(float l, int flags) {
+  return (flags & kRouterClamp) ? fminf(fmaxf(l, -50.f), 50.f) : l;
+}
+// Combine weights of the k chosen logits (slot 0 the largest).
+__device__ __forceinline__ void topk_weights(const float* sel_v, int k, int flags, float* w) {
+  if (flags & kRouterRaw) {
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j)
+      if (j < k) w[j] = sel_v[j];
+    return;
+  }
+  float den = 0.f;
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j)
+    if (j < k) den += expf(sel_v[j] - sel_v[0]);
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j)
+    if (j < k) w[j] = expf(sel_v[j] - sel_v[0]) / den;
+}
+// One warp selects the top-k of one token whose E logits (bias added, not yet clamped) sit in
+// shared memory.
+__device__ __forceinline__ void warp_topk(const float* lg, int E, int k, int flags, int lane, int32_t* idx_out,
                                           float* w_out) {
   float v[8];
 #pragma unroll
   for (int m = 0; m < 8; ++m) {
     const int e = lane + 32 * m;
-    v[m] = (e < E) ? lg[e] : -INFINITY;
+    v[m] = (e < E) ? router_clamp(lg[e], flags) : -INFINITY;
   }
   uint32_t used = 0;
   float sel_v[kMaxTopK];
@@ -377,15 +405,13 @@ __device__ __forceinline__ void warp_topk(const float* lg, int E, int k, int lan
     }
   }
   if (lane == 0) {
-    float den = 0.f;
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j)
-      if (j < k) den += expf(sel_v[j] - sel_v[0]);
+    float w[kMaxTopK];
+    topk_weights(sel_v, k, flags, w);
 #pragma unroll
     for (int j = 0; j < kMaxTopK; ++j)
       if (j < k) {
         idx_out[j] = sel_e[j];
-        w_out[j] = expf(sel_v[j] - sel_v[0]) / den;
+        w_out[j] = w[j];
       }
   }
 }

@@ -196,6 +196,8 @@ struct DsCtl {
   int issued;    // copies issued / stages consumed, for the error path
   int consumed;
   int flag;      // result of a grid-wide wait, broadcast to the epilogue warps
+  int hpass;     // fused kernel: 1 once the epilogue warps passed the H barrier, -1 if it failed
+  uint32_t pbase;  // fused kernel: start of this launch's round on the planes barrier
   int first;     // this CTA's first work item (items first, first + gridDim.x, ...)
   int ntouched;
   int32_t off[kMaxExperts + 1];     // row offsets of the experts' groups
@@ -380,14 +382,15 @@ __device__ bool ds_epilogue(const DecStreamParams& p, DsCtl& c, int pre_idx, int
        L += gridDim.x, ++iter) {
     const int a = iter & 1;
     const uint32_t aph = (uint32_t)(iter >> 1) & 1u;
+    // the weight scale is an input of the call: loaded before the accumulator is waited for
+    const int o = it.tile * 128 + q * 32 + lane;
+    const bool vo = o < p.out_rows;
+    const float* es = p.wscale + (size_t)it.e * (2 * p.f + p.d);
+    const float sc = vo ? __ldg(es + (kGateUp ? it.mat * p.f : 2 * p.f) + o) : 0.f;
     const bool got = ds_wait(&c.tfull[a], aph, &c.abort);
     if (!__all_sync(0xffffffffu, got)) return false;
     tc_fence_after();
-    const int o = it.tile * 128 + q * 32 + lane;
-    const bool vo = o < p.out_rows;
     const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * N);
-    const float* es = p.wscale + (size_t)it.e * (2 * p.f + p.d);
-    const float sc = vo ? es[(kGateUp ? it.mat * p.f : 2 * p.f) + o] : 0.f;
     // columns [0, nt8) hold the hi plane, [nt8, 2 nt8) the lo plane of the same tokens
     for (int j = 0; j < p.nt8; j += (p.nt8 == 8 ? 8 : 16)) {
       float hi[16], lo[16];
@@ -447,6 +450,7 @@ __device__ __forceinline__ void ds_init(const DecStreamParams* const* phases, in
     c.issued = 0;
     c.consumed = 0;
     c.flag = 0;
+    c.hpass = 0;
     c.first = blockIdx.x;
     mbar_fence_init();
     for (int i = 0; i < nphases; ++i) {
@@ -578,14 +582,17 @@ struct alignas(64) DecFusedParams {
   const __nv_bfloat16* x;   // [T, d]
   const __nv_bfloat16* router_w;  // [E, d]
   const float* router_b;    // [E] or NULL
+  int router_flags;         // kRouterClamp | kRouterRaw
   int32_t* topk_idx;        // [T, k]
   int32_t* counts;          // [E]
   int32_t* offsets;         // [E+1]
   int32_t* src_row;         // [T*k]
   float* xscale;            // [R] scales of the x planes (the buffer p.gu.rscale reads)
 };
-// grid-barrier counters: router done, x planes done, GU done, H done, Ypart done, exit ticket
-enum { kBarRouter = 0, kBarPlanes, kBarGU, kBarH, kBarY, kBarExit, kFusedBars };
+// up to this many tokens every CTA of the fused kernel routes all of them itself
+constexpr int kRedundantT = 1;
+// grid-barrier counters: router done, x planes done, GU done, H done, Ypart done
+enum { kBarRouter = 0, kBarPlanes, kBarGU, kBarH, kBarY, kFusedBars };
 static_assert(kFusedBars <= kFusedBarCount, "grid-barrier counters of the fused kernel");
 
 __device__ __forceinline__ int ld_acquire(const int32_t* p) {
@@ -594,17 +601,54 @@ __device__ __forceinline__ int ld_acquire(const int32_t* p) {
   return v;
 }
 
+// Grid barriers are never reset.  A counter runs through [0, G * kBarLaps) (atom.inc wraps it
+// to 0), and every launch that uses it adds exactly G: each CTA arrives once, also after an
+// error.  A CTA's arrival returns the count before it; the round it belongs to started at the
+// multiple of G below that, and the barrier is passed once the counter has moved G beyond that
+// start.  The arrival (one thread, after a CTA barrier) is an acquire-release RMW, so every write
+// the CTA made before its CTA barrier is visible to a CTA that acquires the counter later.
+constexpr uint32_t kBarLaps = 1u << 16;
+__device__ __forceinline__ uint32_t bar_arrive(int32_t* ctr, int G) {  // returns the count before
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.inc.u32 %0, [%1], %2;"
+               : "=r"(old)
+               : "l"(ctr), "r"((uint32_t)G * kBarLaps - 1u)
+               : "memory");
+  return old;
+}
+__device__ __forceinline__ uint32_t bar_base(uint32_t old, int G) { return old - old % (uint32_t)G; }
+__device__ __forceinline__ bool bar_passed(const int32_t* ctr, uint32_t base, int G) {
+  const uint32_t wrap = (uint32_t)G * kBarLaps;
+  return ((uint32_t)ld_acquire(ctr) + wrap - base) % wrap >= (uint32_t)G;
+}
+
 __device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
-// Wait (bounded) until `*ctr` reaches `target`.
-__device__ bool grid_wait(const int32_t* ctr, int target, volatile int* abort_flag) {
+// A flag in shared memory passed from one role of the CTA to another.
+__device__ __forceinline__ int ld_acquire_cta(const int* p) {
+  int v;
+  asm volatile("ld.acquire.cta.shared.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_cta(int* p, int v) {
+  asm volatile("st.release.cta.shared.b32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+
+// Wait (bounded) until the round of the barrier `ctr` that started at `base` is complete.
+__device__ bool grid_wait(const int32_t* ctr, uint32_t base, int G, volatile int* abort_flag) {
   const unsigned long long t0 = global_ns();
-  while (ld_acquire(ctr) < target) {
+  while (!bar_passed(ctr, base, G)) {
     if (*abort_flag) return false;
     if (global_ns() - t0 > kWaitTimeoutNs) return false;
-    __nanosleep(128);
+    __nanosleep(64);
   }
   return true;
+}
+// Arrive and wait; the last CTA to arrive completes the round and does not wait.
+__device__ bool grid_sync(int32_t* ctr, int G, volatile int* abort_flag) {
+  const uint32_t old = bar_arrive(ctr, G), base = bar_base(old, G);
+  if (old - base == (uint32_t)G - 1u) return true;
+  return grid_wait(ctr, base, G, abort_flag);
 }
 
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
@@ -618,7 +662,6 @@ __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" :::
 // Arrives on the planes barrier; the producer waits on it before its first plane copy.
 __device__ void fused_route(const DecFusedParams& p, uint8_t* smem, DsCtl& c) {
   constexpr int kWarps = kDsThreads / 32;
-  constexpr int kRedundantT = 1;  // up to this many tokens every CTA routes all of them itself
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, T = p.T, k = p.k, E = p.gu.E, d = p.gu.d;
   const int nvec = d / 8;  // 16-byte slices of a bf16 row
@@ -635,17 +678,37 @@ __device__ void fused_route(const DecFusedParams& p, uint8_t* smem, DsCtl& c) {
   const bool redundant = p.route_in_kernel == 1 && T <= kRedundantT;
   for (int t = redundant ? 0 : blockIdx.x; p.route_in_kernel == 1 && t < T; t += redundant ? 1 : G) {
     const uint4* xv = reinterpret_cast<const uint4*>(p.x + (size_t)t * d);
+    // the bias is loaded first (it is consumed last), and every slice of x and of the 8 expert
+    // rows that a thread needs for one batch is loaded before any of them is used, so a batch
+    // costs one memory round trip (d = 4096: one batch of 3 slices x 9 rows per thread)
+    float bias[(kMaxExperts + kDsThreads - 1) / kDsThreads];
+#pragma unroll
+    for (int j = 0; j < (int)(sizeof(bias) / sizeof(float)); ++j) {
+      const int e = tid + j * kDsThreads;
+      bias[j] = (p.router_b && e < E) ? __ldg(p.router_b + e) : 0.f;
+    }
+    constexpr int kSlices = 3;
     for (int e0 = 0; e0 < E; e0 += 8) {
       float acc[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-      for (int v = tid; v < nvec; v += kDsThreads) {
-        const uint4 xq = __ldg(xv + v);
+      for (int v0 = tid; v0 < nvec; v0 += kSlices * kDsThreads) {
+        uint4 xq[kSlices], wq[kSlices][8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (e0 + i < E)
-            acc[i] = dot16(xq, __ldg(reinterpret_cast<const uint4*>(p.router_w + (size_t)(e0 + i) * d) + v), acc[i],
-                           p.x);
+        for (int u = 0; u < kSlices; ++u) {
+          const int v = v0 + u * kDsThreads;
+          xq[u] = v < nvec ? __ldg(xv + v) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            wq[u][i] = (v < nvec && e0 + i < E)
+                           ? __ldg(reinterpret_cast<const uint4*>(p.router_w + (size_t)(e0 + i) * d) + v)
+                           : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < kSlices; ++u)
+          if (v0 + u * kDsThreads < nvec)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = dot16(xq[u], wq[u][i], acc[i], p.x);
       }
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -659,22 +722,26 @@ __device__ void fused_route(const DecFusedParams& p, uint8_t* smem, DsCtl& c) {
       }
     }
     __syncthreads();
-    for (int e = tid; e < E; e += kDsThreads) {
-      float sum = part[e];
-      for (int w = 1; w < kWarps; ++w) sum += part[w * kMaxExperts + e];
-      lg[e] = sum + (p.router_b ? p.router_b[e] : 0.f);
+#pragma unroll
+    for (int j = 0; j < (int)(sizeof(bias) / sizeof(float)); ++j) {
+      const int e = tid + j * kDsThreads;
+      if (e < E) {
+        float sum = part[e];
+        for (int w = 1; w < kWarps; ++w) sum += part[w * kMaxExperts + e];
+        lg[e] = sum + bias[j];
+      }
     }
     __syncthreads();
     if (warp == 0) {
       if (redundant) {
-        warp_topk(lg, E, k, lane, s_idx + (size_t)t * k, s_w + (size_t)t * k);
+        warp_topk(lg, E, k, p.router_flags, lane, s_idx + (size_t)t * k, s_w + (size_t)t * k);
         __syncwarp();
         if (blockIdx.x == 0 && lane < k) {  // one CTA publishes the choices
           p.topk_idx[(size_t)t * k + lane] = s_idx[(size_t)t * k + lane];
           p.topk_w[(size_t)t * k + lane] = s_w[(size_t)t * k + lane];
         }
       } else {
-        warp_topk(lg, E, k, lane, p.topk_idx + (size_t)t * k, p.topk_w + (size_t)t * k);
+        warp_topk(lg, E, k, p.router_flags, lane, p.topk_idx + (size_t)t * k, p.topk_w + (size_t)t * k);
       }
     }
     __syncthreads();
@@ -682,27 +749,25 @@ __device__ void fused_route(const DecFusedParams& p, uint8_t* smem, DsCtl& c) {
   c.flag = 1;
   if (p.route_in_kernel == 1 && !redundant) {
     // every token's choices are needed below
-    __threadfence();
     __syncthreads();
     if (tid == 0) {
-      atomicAdd(&p.bar[kBarRouter], 1);
-      c.flag = grid_wait(&p.bar[kBarRouter], G, &c.abort) ? 1 : 0;
+      c.flag = grid_sync(&p.bar[kBarRouter], G, &c.abort) ? 1 : 0;
       if (!c.flag) ds_abort(c, p.gu.err);
     }
     __syncthreads();
   }
   // the choices: this CTA's own copy, or from global memory (another CTA's, or the caller's)
   auto choice = [&](int i) { return redundant ? s_idx[i] : __ldcg(p.topk_idx + i); };
-  for (int e = tid; e < E; e += kDsThreads) mask[e] = 0ull;
-  __syncthreads();
-  if (c.flag) {
-    for (int i = tid; i < T * k; i += kDsThreads) {
-      const int e = min(max(choice(i), 0), E - 1);
-      atomicOr(&mask[e], 1ull << (i / k));
+  if (warp == 0) {  // per-expert token masks, then the offsets: exclusive scan of the counts
+    for (int e = lane; e < E; e += 32) mask[e] = 0ull;
+    __syncwarp();
+    if (c.flag) {
+      for (int i = lane; i < T * k; i += 32) {
+        const int e = min(max(choice(i), 0), E - 1);
+        atomicOr(&mask[e], 1ull << (i / k));
+      }
     }
-  }
-  __syncthreads();
-  if (warp == 0) {  // offsets: exclusive scan of the counts over the experts
+    __syncwarp();
     const int C = (E + 31) / 32;
     const int e0 = min(E, lane * C), e1 = min(E, e0 + C);
     int sum = 0;
@@ -788,9 +853,8 @@ __device__ void fused_route(const DecFusedParams& p, uint8_t* smem, DsCtl& c) {
   }
   // the planes are read next by TMA copies of other CTAs
   fence_proxy_async_global();
-  __threadfence();
   __syncthreads();
-  if (tid == 0) atomicAdd(&p.bar[kBarPlanes], 1);
+  if (tid == 0) c.pbase = bar_base(bar_arrive(&p.bar[kBarPlanes], G), G);  // the producer (this thread) waits
 }
 
 __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_constant__ DecFusedParams p) {
@@ -815,9 +879,11 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_c
   }
   const uint32_t tmem = aligned ? c.tmem : 0u;
   if (!aligned) {
-    if (threadIdx.x == 0) {  // report, and arrive at every barrier so the other CTAs do not wait
+    if (threadIdx.x == 0) {  // report, and arrive at every barrier the others wait on
       atomicOr(p.gu.err, kErrWaitTimeout);
-      for (int b = 0; b < kBarExit; ++b) atomicAdd(&p.bar[b], 1);
+      if (p.route_in_kernel == 1 && p.T > kRedundantT) bar_arrive(&p.bar[kBarRouter], G);
+      if (p.route_in_kernel) bar_arrive(&p.bar[kBarPlanes], G);
+      for (int b = kBarGU; b <= kBarY; ++b) bar_arrive(&p.bar[b], G);
     }
   } else if (warp == 0) {
     if (lane == 0) {
@@ -825,14 +891,21 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_c
       // with the routing done in this launch, the gate/up weights go out at once and the plane
       // copies wait until every CTA has written its tokens' planes
       bool ok = ds_produce<true>(p.gu, smem, c, S, 0, r, p.route_in_kernel != 0, [&] {
-        if (!grid_wait(&p.bar[kBarPlanes], G, &c.abort)) return false;
+        if (!grid_wait(&p.bar[kBarPlanes], c.pbase, G, &c.abort)) return false;
         fence_proxy_async_global();
         return true;
       });
-      // down weights go out at once; their plane copies wait for phase 2 of every CTA
+      // down weights go out at once; their plane copies wait until this CTA's epilogue warps
+      // have passed the H barrier (phase 2 of every CTA done)
       if (ok)
         ok = ds_produce<false>(p.dn, smem, c, S, 1, r, true, [&] {
-          if (!grid_wait(&p.bar[kBarH], G, &c.abort)) return false;
+          const unsigned long long t0 = global_ns();
+          int v;
+          while ((v = ld_acquire_cta(&c.hpass)) == 0) {
+            if (*(volatile int*)&c.abort || global_ns() - t0 > kWaitTimeoutNs) return false;
+            __nanosleep(32);
+          }
+          if (v < 0) return false;
           fence_proxy_async_global();
           return true;
         });
@@ -860,10 +933,12 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_c
     auto grid_barrier = [&](int idx) -> bool {
       epi_sync();
       if (tid == 0) {
-        __threadfence();
-        atomicAdd(&p.bar[idx], 1);
-        c.flag = (!c.abort && grid_wait(&p.bar[idx], G, &c.abort)) ? 1 : 0;
-        if (!c.flag && !c.abort) ds_abort(c, p.gu.err);
+        const uint32_t old = bar_arrive(&p.bar[idx], G), base = bar_base(old, G);
+        const bool passed =
+            !c.abort && (old - base == (uint32_t)G - 1u || grid_wait(&p.bar[idx], base, G, &c.abort));
+        c.flag = passed ? 1 : 0;
+        if (!passed && !c.abort) ds_abort(c, p.gu.err);
+        if (idx == kBarH) st_release_cta(&c.hpass, passed ? 1 : -1);  // the producer waits on it
       }
       epi_sync();
       return *(volatile int*)&c.flag != 0;
@@ -905,13 +980,29 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_c
           hv[2] = __bfloat162float(__float2bfloat16_rn(silu_mul(g.z, uu.z)));
           hv[3] = __bfloat162float(__float2bfloat16_rn(silu_mul(g.w, uu.w)));
         };
-        // two passes over the partials (max, then split): keeping the values in registers between
-        // them measured slower (the kernel's register count doubled)
+        // A short unit (at most kHKeep steps per thread, e.g. one token's 896-column unit) keeps its
+        // h values in registers between the max and the split; a longer one makes two passes over
+        // the partials (holding every step measured slower: the kernel's register count doubled).
+        constexpr int kHKeep = 2;
+        const bool keep = span <= 128 * 4 * kHKeep;
+        float hk[kHKeep][4];
         float mx = 0.f;
-        for (int j = tid * 4; j < span; j += 128 * 4) {
-          float hv[4];
-          hvals(j, hv);
-          mx = fmaxf(mx, fmaxf(fmaxf(fabsf(hv[0]), fabsf(hv[1])), fmaxf(fabsf(hv[2]), fabsf(hv[3]))));
+        if (keep) {
+#pragma unroll
+          for (int it = 0; it < kHKeep; ++it) {
+            const int j = tid * 4 + it * 128 * 4;
+            if (j < span) {
+              hvals(j, hk[it]);
+              mx = fmaxf(mx, fmaxf(fmaxf(fabsf(hk[it][0]), fabsf(hk[it][1])), fmaxf(fabsf(hk[it][2]), fabsf(hk[it][3]))));
+            }
+            asm volatile("" ::: "memory");  // one step's partials in registers at a time
+          }
+        } else {
+          for (int j = tid * 4; j < span; j += 128 * 4) {
+            float hv[4];
+            hvals(j, hv);
+            mx = fmaxf(mx, fmaxf(fmaxf(fabsf(hv[0]), fabsf(hv[1])), fmaxf(fabsf(hv[2]), fabsf(hv[3]))));
+          }
         }
 #pragma unroll
         for (int off = 16; off; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
@@ -923,9 +1014,7 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_c
         if (tid == 0) p.hscale[(size_t)sp * R + r] = a;
         int8_t* hrow = p.hhi + (size_t)r * f + k0;
         int8_t* lrow = p.hlo + (size_t)r * f + k0;
-        for (int j = tid * 4; j < span; j += 128 * 4) {  // the same values again, now split
-          float hv[4];
-          hvals(j, hv);
+        auto put = [&](int j, const float (&hv)[4]) {
           uint32_t hw = 0u, lw = 0u;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -936,6 +1025,19 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_c
           }
           *reinterpret_cast<uint32_t*>(hrow + j) = hw;
           *reinterpret_cast<uint32_t*>(lrow + j) = lw;
+        };
+        if (keep) {
+#pragma unroll
+          for (int it = 0; it < kHKeep; ++it) {
+            const int j = tid * 4 + it * 128 * 4;
+            if (j < span) put(j, hk[it]);
+          }
+        } else {
+          for (int j = tid * 4; j < span; j += 128 * 4) {  // the same values again, now split
+            float hv[4];
+            hvals(j, hv);
+            put(j, hv);
+          }
         }
       }
       fence_proxy_async_global();  // the planes are read next by TMA copies of other CTAs
@@ -988,14 +1090,6 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_c
   }
   if (aligned) ds_teardown(c, S);
   else __syncthreads();
-  // exit ticket: the last CTA to leave resets the counters for the next launch
-  if (threadIdx.x == 0) {
-    __threadfence();
-    if (atomicAdd(&p.bar[kBarExit], 1) == G - 1) {
-      for (int b = 0; b < kFusedBars; ++b) p.bar[b] = 0;
-      __threadfence();
-    }
-  }
 }
 
 // K blocks per ring stage: COLIBRI_DEC_KB (1..4), default 2.
@@ -1161,6 +1255,7 @@ cudaError_t launch_dec_fused(const DecFusedArgs& a, cudaStream_t s) {
   p.x = a.x;
   p.router_w = a.router_w;
   p.router_b = a.router_b;
+  p.router_flags = a.router_flags;
   p.topk_idx = a.topk_idx;
   p.counts = a.counts;
   p.offsets = a.offsets_out;

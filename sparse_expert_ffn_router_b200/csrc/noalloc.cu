@@ -113,7 +113,7 @@ extern "C" colibri_status colibri_route_noalloc(const void* x, int32_t act_dtype
   int32_t* blk_base = scratch + kNoAllocMaxBlockExperts;
   int32_t* mt_prefix = scratch + 2 * kNoAllocMaxBlockExperts;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_router_topk(x, act_dtype, T, d_model, router_w, router_b, num_experts, top_k,
+  cudaError_t e = launch_router_topk(x, act_dtype, T, d_model, router_w, router_b, num_experts, top_k, 0,
                                      topk_idx, topk_w, nullptr, nullptr, nullptr, s);
   if (e == cudaSuccess) e = launch_route_count(topk_idx, T, top_k, num_experts, blk_counts, dst_row, s);
   if (e == cudaSuccess)

@@ -9,7 +9,8 @@
 // selection is made by k rounds of a warp-wide arg-max (the warp-shuffle top-k idea of
 // www.pptc.cn/news/100465 §2.1, generalised from 2 to k <= 8 and to 256 experts).
 // weights: softmax over all E renormalised over the k chosen, computed as
-// exp(l_j - l_0) / sum_j' exp(l_j' - l_0) in fp32.
+// exp(l_j - l_0) / sum_j' exp(l_j' - l_0) in fp32; or, on request, the raw chosen logits, and
+// optionally with every logit clamped to [-50, 50] first (router_clamp / topk_weights).
 // Output layout [T][k] (www.pptc.cn/news/100465 §3.4).
 #include <algorithm>
 #include <cstring>
@@ -29,7 +30,7 @@ constexpr int kRouterThreads = 256;
 template <typename Tin>
 __global__ void __launch_bounds__(kRouterThreads) router_topk_simt_kernel(
     const Tin* __restrict__ x, int T, int d, const Tin* __restrict__ wr, const float* __restrict__ b,
-    int E, int k, int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
+    int E, int k, int rflags, int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
   pdl_trigger();
   pdl_wait();
   extern __shared__ float sm[];
@@ -73,7 +74,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_topk_simt_kernel(
   for (int tt = warp; tt < kRouterTT; tt += kRouterThreads / 32) {
     const int t = t0 + tt;
     if (t >= T) break;
-    warp_topk(lg + tt * (E + 1), E, k, lane, idx_out + (size_t)t * k, w_out + (size_t)t * k);
+    warp_topk(lg + tt * (E + 1), E, k, rflags, lane, idx_out + (size_t)t * k, w_out + (size_t)t * k);
   }
 }
 
@@ -90,7 +91,8 @@ __global__ void __launch_bounds__(kRouterThreads) router_topk_simt_kernel(
 template <typename Tin>
 __global__ void __launch_bounds__(256) router_small_kernel(const Tin* __restrict__ x, int d,
                                                            const Tin* __restrict__ wr, const float* __restrict__ b,
-                                                           int E, int k, int32_t* __restrict__ idx_out,
+                                                           int E, int k, int rflags,
+                                                           int32_t* __restrict__ idx_out,
                                                            float* __restrict__ w_out) {
   pdl_trigger();
   pdl_wait();
@@ -130,7 +132,7 @@ __global__ void __launch_bounds__(256) router_small_kernel(const Tin* __restrict
     lg[e] = sum + (b ? b[e] : 0.f);
   }
   __syncthreads();
-  if (warp == 0) warp_topk(lg, E, k, lane, idx_out + (size_t)t * k, w_out + (size_t)t * k);
+  if (warp == 0) warp_topk(lg, E, k, rflags, lane, idx_out + (size_t)t * k, w_out + (size_t)t * k);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -152,6 +154,7 @@ struct alignas(64) RouterTcParams {
   CUtensorMap mapW;  // [E, d], box {64, N}
   const float* b;
   int T, d, E, k, N;
+  int rflags;        // kRouterClamp | kRouterRaw
   int ksplit;        // CTAs per 128-token tile, each over d / ksplit (gridDim.y)
   float* part;       // [ksplit, E, T] partial logits (ksplit > 1; token-contiguous, so stores coalesce)
   int32_t* ticket;   // [tiles] arrival counters, zero between calls (ksplit > 1)
@@ -336,7 +339,7 @@ __global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant
       for (int i = 0; i < 16; ++i) {
         const int e = c0 + i;
         if (e < p.E) {
-          float cv = v[i] + (p.b ? p.b[e] : 0.f);
+          float cv = router_clamp(v[i] + (p.b ? p.b[e] : 0.f), p.rflags);
           int ci = e;
 #pragma unroll
           for (int j = 0; j < kMaxTopK; ++j) {
@@ -353,15 +356,13 @@ __global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant
       }
     }
     if (t < p.T) {
-      float den = 0.f;
-#pragma unroll
-      for (int j = 0; j < kMaxTopK; ++j)
-        if (j < p.k) den += expf(bv[j] - bv[0]);
+      float wv[kMaxTopK];
+      topk_weights(bv, p.k, p.rflags, wv);
 #pragma unroll
       for (int j = 0; j < kMaxTopK; ++j)
         if (j < p.k) {
           p.idx[(size_t)t * p.k + j] = bi[j];
-          p.w[(size_t)t * p.k + j] = expf(bv[j] - bv[0]) / den;
+          p.w[(size_t)t * p.k + j] = wv[j];
         }
     }
   }
@@ -381,8 +382,8 @@ __global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant
 constexpr size_t kRtMaxSmem = kRtRingBytes + 1024;
 
 cudaError_t launch_router_tc(const void* x, int T, int d, const void* wr, const float* b, int E, int k,
-                             int32_t* idx, float* w, uint32_t* err, int ksplit, float* part, int32_t* ticket,
-                             cudaStream_t s) {
+                             int rflags, int32_t* idx, float* w, uint32_t* err, int ksplit, float* part,
+                             int32_t* ticket, cudaStream_t s) {
   RouterTcParams p;
   memset(&p, 0, sizeof(p));
   p.N = (E + 15) / 16 * 16;
@@ -404,6 +405,7 @@ cudaError_t launch_router_tc(const void* x, int T, int d, const void* wr, const 
   p.d = d;
   p.E = E;
   p.k = k;
+  p.rflags = rflags;
   p.stage_bytes = (uint32_t)((kRtABytes + p.N * 128 + 1023) / 1024 * 1024);
   p.stages = (int)std::min<size_t>(kRtMaxStages, kRtRingBytes / p.stage_bytes);
   p.tmem_cols = 32;
@@ -439,26 +441,26 @@ int router_ksplit(int T, int d) {
 }
 
 cudaError_t launch_router_topk(const void* x, int act, int T, int d, const void* wr, const float* b,
-                               int E, int k, int32_t* idx, float* w, uint32_t* err, float* part,
+                               int E, int k, int rflags, int32_t* idx, float* w, uint32_t* err, float* part,
                                int32_t* ticket, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
   if (T <= kRouterSmallT) {
     if (act == COLIBRI_BF16)
       return launch_kernel(router_small_kernel<__nv_bfloat16>, dim3(T), dim3(256), 0, s, 1, (const __nv_bfloat16*)x, d,
-                           (const __nv_bfloat16*)wr, b, E, k, idx, w);
+                           (const __nv_bfloat16*)wr, b, E, k, rflags, idx, w);
     return launch_kernel(router_small_kernel<float>, dim3(T), dim3(256), 0, s, 1, (const float*)x, d,
-                         (const float*)wr, b, E, k, idx, w);
+                         (const float*)wr, b, E, k, rflags, idx, w);
   }
   if (act == COLIBRI_BF16) {
     const int ks = (part && ticket) ? router_ksplit(T, d) : 1;
-    return launch_router_tc(x, T, d, wr, b, E, k, idx, w, err, ks, part, ticket, s);
+    return launch_router_tc(x, T, d, wr, b, E, k, rflags, idx, w, err, ks, part, ticket, s);
   }
   const size_t smem =
       sizeof(float) * ((size_t)kRouterTT * (kRouterDK + 1) + (size_t)E * (kRouterDK + 1) +
                        (size_t)kRouterTT * (E + 1));
   const dim3 grid((T + kRouterTT - 1) / kRouterTT);
   return launch_kernel(router_topk_simt_kernel<float>, grid, dim3(kRouterThreads), smem, s, 1, (const float*)x, T, d,
-                       (const float*)wr, b, E, k, idx, w);
+                       (const float*)wr, b, E, k, rflags, idx, w);
 }
 
 }  // namespace colibri

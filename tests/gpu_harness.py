@@ -36,16 +36,16 @@ def to_device(p, dev="cuda"):
         shared_w=None if p.shared_w is None else p.shared_w.to(dev))
 
 
-def make_layer(wl, max_tokens=None):
+def make_layer(wl, max_tokens=None, router_flags=0):
     return colibri.MoELayer(wl.d, wl.f, wl.E, wl.k, wl.fs, wl.act, wl.wdt,
-                            max_tokens=max_tokens or max(wl.T, 1), device_id=0)
+                            max_tokens=max_tokens or max(wl.T, 1), device_id=0, router_flags=router_flags)
 
 
-def run_gpu(p, layer=None, dev_inputs=None, routed=None):
+def run_gpu(p, layer=None, dev_inputs=None, routed=None, router_flags=0):
     """Run one forward through the C ABI; returns y (host, float32) and the routing state."""
     wl = p.wl
     own = layer is None
-    layer = layer or make_layer(wl)
+    layer = layer or make_layer(wl, router_flags=router_flags)
     assert layer.expert_stride == p.expert_stride
     t = dev_inputs or to_device(p)
     y = torch.empty(wl.T, wl.d, dtype=p.x.dtype, device="cuda")
@@ -92,8 +92,9 @@ def valid_topk_under_slack(logits_row: np.ndarray, chosen: np.ndarray, k: int) -
     return logits_row[mask].max() - logits_row[chosen].min() < NEAR_TIE
 
 
-def compare_routing(p, ref, gpu):
-    """Apply the near-tie protocol; returns (routing used for the oracle y, n_near_tie)."""
+def compare_routing(p, ref, gpu, flags=0):
+    """Apply the near-tie protocol; returns (routing used for the oracle y, n_near_tie).
+    ``flags``: the router variant both sides ran (the oracle's logits are already clamped)."""
     wl = p.wl
     logits, idx_o = ref["logits"], ref["idx"]
     near = near_tie_tokens(logits, idx_o, ref["gap"])
@@ -106,8 +107,9 @@ def compare_routing(p, ref, gpu):
         g = idx_g[t].numpy().astype(np.int64)
         assert valid_topk_under_slack(logits[t].numpy().astype(np.float64), g, wl.k), f"token {t}"
         idx_use[t] = idx_g[t]
-    w_use = oracle.weights_for(logits, idx_use)
-    assert (gpu["w"] - w_use).abs().max().item() < 2e-5, "routing weights differ"
+    w_use = oracle.weights_for(logits, idx_use, flags)
+    # softmax weights lie in [0, 1]; raw-logit weights are compared relative to their size
+    assert ((gpu["w"] - w_use).abs() <= 2e-5 * w_use.abs().clamp(min=1.0)).all(), "routing weights differ"
     counts, offsets, src, dst = oracle.group(idx_use, wl.E)
     assert torch.equal(gpu["counts"], counts)
     assert torch.equal(gpu["offsets"], offsets)
@@ -126,19 +128,20 @@ def check_y(p, y_gpu_rows, y_ref_rows, tol=None):
     return err / max(scale, 1e-30)
 
 
-def parity(p, tokens=None, layer=None, dev_inputs=None):
-    """Full protocol: routing on every token, y on `tokens` (default all)."""
+def parity(p, tokens=None, layer=None, dev_inputs=None, flags=0):
+    """Full protocol: routing on every token, y on `tokens` (default all).  ``flags`` selects
+    the router variant on both sides."""
     wl = p.wl
-    logits = oracle.router_logits(p.x, p.router_w, p.router_b)
-    idx, w, gap = oracle.topk(logits, wl.k)
+    logits = oracle.router_logits(p.x, p.router_w, p.router_b, flags)
+    idx, w, gap = oracle.topk(logits, wl.k, flags)
     ref = dict(logits=logits, idx=idx, w=w, gap=gap)
-    gpu = run_gpu(p, layer=layer, dev_inputs=dev_inputs)
-    idx_use, w_use, n_near = compare_routing(p, ref, gpu)
+    gpu = run_gpu(p, layer=layer, dev_inputs=dev_inputs, router_flags=flags)
+    idx_use, w_use, n_near = compare_routing(p, ref, gpu, flags)
     toks = list(range(wl.T)) if tokens is None else list(tokens)
     y_ref = oracle.combine(p.x, idx_use, w_use, p.expert_w, p.expert_stride, wl.f, p.expert_scales, p.shared_w,
                            wl.fs, toks)
     rel = check_y(p, gpu["y"][toks], y_ref)
-    return dict(rel_err=rel, near_ties=n_near, counts=gpu["counts"])
+    return dict(rel_err=rel, near_ties=n_near, counts=gpu["counts"], idx=gpu["idx"], ref_idx=idx)
 
 
 def sample_tokens(T: int, n: int):

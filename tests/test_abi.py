@@ -71,6 +71,8 @@ def _desc(**kw):
     (dict(act_dtype=colibri.COLIBRI_F32, weight_dtype=colibri.COLIBRI_BF16), -3),
     (dict(act_dtype=colibri.COLIBRI_I8, weight_dtype=colibri.COLIBRI_I8), -3),
     (dict(weight_dtype=colibri.COLIBRI_I8, shared_d_ff=64), -3),
+    (dict(router_flags=4), -1),        # unknown router variant bit
+    (dict(router_flags=-1), -1),
 ])
 def test_init_rejects_bad_descriptions(lib, kw, code):
     with pytest.raises(colibri.ColibriError) as ei:

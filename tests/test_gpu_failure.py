@@ -18,10 +18,14 @@ pytestmark = pytest.mark.gpu
 TIMEOUT = -6
 
 
-def test_wait_that_runs_out_is_reported_and_the_context_stays_usable():
-    wl = inputgen.custom("fail_T1", T=1, d=256, E=8, k=2, f=256)
+@pytest.mark.parametrize("wdt", [inputgen.BF16, inputgen.I8])
+def test_wait_that_runs_out_is_reported_and_the_context_stays_usable(wdt):
+    # int8: the fused kernel's grid-barrier counters have advanced before the error, and the
+    # status call resets them; the layer must still compute correctly afterwards
+    wl = inputgen.custom("fail_T1", T=1, d=256, E=8, k=2, f=256, act=inputgen.BF16, wdt=wdt)
     p = inputgen.make_problem(wl, seed=1)
     layer = H.make_layer(wl)
+    H.parity(p, layer=layer)
     s = torch.cuda.Stream()
     colibri.colibri_selftest_wait_timeout(layer.ctx, 20000, stream=s)
     with pytest.raises(colibri.ColibriError) as ei:

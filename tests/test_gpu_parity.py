@@ -85,6 +85,17 @@ def test_int8_each_launch_plan(name, fused, route, monkeypatch):
     layer.close()
 
 
+@pytest.mark.parametrize("env", [{"COLIBRI_DEC_KB": "1"}, {"COLIBRI_DEC_KB": "4"}, {"COLIBRI_DEC_EVICT": "0"},
+                                 {"COLIBRI_DEC_ROUTE": "0", "COLIBRI_DEC_KB": "3"}])
+@pytest.mark.parametrize("name", I8_SMALL)
+def test_int8_stream_settings(name, env, monkeypatch):
+    # K blocks per ring stage, the L2 policy of the weight copies and the routing plan change
+    # only how the weights are streamed, never the result
+    for key, val in env.items():
+        monkeypatch.setenv(key, val)
+    H.parity(inputgen.make_problem(SMALL[name], seed=21))
+
+
 @pytest.mark.parametrize("mode", ["1", "2", "s"])
 def test_mixtral_each_tile_mode(mode, monkeypatch):
     monkeypatch.setenv("COLIBRI_GEMM_CTA", mode)
@@ -288,6 +299,59 @@ def test_forward_routed_matches_oracle_routing(name, monkeypatch):
     assert torch.equal(gpu["idx"], ref["idx"]) and torch.equal(gpu["counts"], ref["counts"])
     assert torch.equal(gpu["src_row"], ref["src_row"])
     H.check_y(p, gpu["y"], ref["y"])
+
+
+VARIANT = {
+    # T >= 2048 bf16 tokens: the tensor-core router splits K over several CTAs per tile
+    "bf16_ksplit": inputgen.custom("bf16_ksplit", T=2048, d=256, E=8, k=2, f=64),
+    # one decode token: every CTA of the fused int8 launch routes it itself
+    "i8_T1": inputgen.custom("i8_T1", T=1, d=256, E=8, k=2, f=256, act=BF16, wdt=I8),
+}
+CLAMP, RAW = colibri.COLIBRI_ROUTER_CLAMP, colibri.COLIBRI_ROUTER_RAW_WEIGHTS
+
+
+def _robust_tokens(lraw: np.ndarray, lclamp: np.ndarray, k: int):
+    """Tokens whose clamped selection and slot order are decided exactly: no logit within 1e-4
+    of +-50 before the clamp (both sides clamp the same ones), and every gap among the k + 1
+    largest clamped logits either exactly zero (a tie at +-50, decided by the index rule) or at
+    least 1e-4."""
+    out = []
+    for t in range(lraw.shape[0]):
+        if (np.abs(np.abs(lraw[t]) - 50.0) < 1e-4).any():
+            continue
+        top = -np.sort(-lclamp[t])[: k + 1]
+        gaps = top[:-1] - top[1:]
+        if np.all((gaps == 0) | (gaps >= 1e-4)):
+            out.append(t)
+    return out
+
+
+# every router kernel: small-T (bf16, f32), tensor-core (one CTA and K-split per tile), SIMT
+# fp32, and the int8 routing inside the fused launch (one token, several tokens, and the plan
+# with separate routing launches)
+@pytest.mark.parametrize("name,flags", [
+    ("bf16_T1", CLAMP | RAW), ("bf16_ragged", CLAMP), ("bf16_ragged", RAW), ("bf16_ragged", CLAMP | RAW),
+    ("bf16_ksplit", CLAMP | RAW), ("bf16_maxE", CLAMP), ("f32_tiny", CLAMP | RAW), ("f32_shared", CLAMP | RAW),
+    ("i8_small", CLAMP | RAW), ("i8_T1", CLAMP | RAW), ("i8_small_split", CLAMP | RAW), ("i8_maxE", CLAMP)])
+def test_router_variants(name, flags, monkeypatch):
+    if name.endswith("_split"):
+        monkeypatch.setenv("COLIBRI_DEC_ROUTE", "0")
+        name = name[: -len("_split")]
+    wl = VARIANT.get(name) or SMALL[name]
+    p = inputgen.make_problem(wl, seed=11)
+    if flags & CLAMP:
+        # logits near 50 for every expert (bias 49, 49.5 or 50 plus the token's N(0, 1) part), so
+        # the clamp bites on some experts of most tokens and clamped experts tie at exactly 50
+        p.router_b = torch.tensor([49.0 + 0.5 * (e % 3) for e in range(wl.E)], dtype=torch.float32)
+    r = H.parity(p, flags=flags)
+    if flags & CLAMP:
+        lraw = oracle.router_logits(p.x, p.router_w, p.router_b).numpy()
+        lc = oracle.router_logits(p.x, p.router_w, p.router_b, CLAMP).numpy()
+        robust = _robust_tokens(lraw, lc, wl.k)
+        assert robust
+        assert torch.equal(r["idx"][robust], r["ref_idx"][robust]), "tie at 50 not resolved to the lower index"
+        ties = [t for t in robust if (lc[t] == 50.0).sum() >= 2]
+        assert ties or wl.T == 1  # the tie rule was exercised (a single token may have no tie)
 
 
 def test_smaller_T_on_a_larger_context():

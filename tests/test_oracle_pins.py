@@ -68,19 +68,26 @@ def _swiglu(x, w1, w3, w2):
     return (g / (1.0 + np.exp(-g)) * u) @ w2.T
 
 
-def _dense_layer(p):
-    """Every expert on every token, combined through a masked [T, E] weight matrix."""
+def _dense_layer(p, flags=0):
+    """Every expert on every token, combined through a masked [T, E] weight matrix.
+    ``flags``: oracle.ROUTER_CLAMP clips the logits to [-50, 50]; oracle.ROUTER_RAW uses the
+    chosen logits as the weights."""
     wl = p.wl
     x = _f64(p.x)
     wr = _f64(p.router_w)
     logits = x @ wr.T
     if p.router_b is not None:
         logits = logits + _f64(p.router_b)
+    if flags & oracle.ROUTER_CLAMP:
+        logits = np.clip(logits, -50.0, 50.0)
     sel = _ref_select(logits.astype(np.float32), wl.k)
     mask = np.zeros((wl.T, wl.E))
     for t in range(wl.T):
         ls = logits[t, sel[t]]
-        mask[t, sel[t]] = np.exp(ls - ls.max()) / np.exp(ls - ls.max()).sum()
+        if flags & oracle.ROUTER_RAW:
+            mask[t, sel[t]] = ls
+        else:
+            mask[t, sel[t]] = np.exp(ls - ls.max()) / np.exp(ls - ls.max()).sum()
     y = np.zeros((wl.T, wl.d))
     for e in range(wl.E):
         y += mask[:, e:e + 1] * _swiglu(x, *_expert_mats(p, e))
@@ -189,6 +196,62 @@ def test_router_logits_vs_float64_matmul(act):
     assert _rel_err(got0.numpy(), _f64(p.x) @ _f64(p.router_w).T) < 1e-6
 
 
+@pytest.mark.parametrize("act", [inputgen.F32, inputgen.BF16])
+def test_router_clamp_vs_clipped_float64_matmul(act):
+    # biases far outside [-50, 50] on some experts: the clamped logits are the float64 matmul
+    # clipped to [-50, 50], exactly +-50 where it bites and untouched elsewhere
+    wl = inputgen.custom("rc", T=29, d=64, E=10, k=2, f=8, act=act, wdt=act)
+    p = inputgen.make_problem(wl, seed=5)
+    b = torch.zeros(10)
+    b[2], b[7], b[9] = 80.0, -90.0, 49.5
+    got = oracle.router_logits(p.x, p.router_w, b, oracle.ROUTER_CLAMP).numpy()
+    raw = _f64(p.x) @ _f64(p.router_w).T + _f64(b)
+    assert _rel_err(got, np.clip(raw, -50.0, 50.0)) < 1e-6
+    assert np.all(got[:, 2] == 50.0) and np.all(got[:, 7] == -50.0)
+    assert np.all(got <= 50.0) and np.all(got >= -50.0)
+    # some tokens push expert 9 over 50 and some do not (both sides of the clip are exercised)
+    assert 0 < int((got[:, 9] == 50.0).sum()) < 29
+    unclipped = np.abs(raw) < 50.0
+    assert _rel_err(got[unclipped], raw[unclipped]) < 1e-6
+    assert np.array_equal(oracle.router_logits(p.x, p.router_w, b).numpy() == 50.0, np.zeros_like(got, bool))
+
+
+def test_clamp_makes_large_logits_tie_and_lower_index_wins():
+    # logits 70, 60, 55 on experts 5, 3, 1: unclamped the order is 5, 3; clamped all three are
+    # 50 and the tie rule keeps the two lowest indices, 1 then 3
+    wl = inputgen.custom("rt", T=4, d=64, E=8, k=2, f=8, act=inputgen.F32, wdt=inputgen.F32)
+    p = inputgen.make_problem(wl, seed=6)
+    x = torch.zeros_like(p.x)  # logits = bias exactly
+    b = torch.zeros(8)
+    b[5], b[3], b[1] = 70.0, 60.0, 55.0
+    l0 = oracle.router_logits(x, p.router_w, b)
+    l1 = oracle.router_logits(x, p.router_w, b, oracle.ROUTER_CLAMP)
+    i0, w0, _ = oracle.topk(l0, 2)
+    i1, w1, _ = oracle.topk(l1, 2, oracle.ROUTER_CLAMP)
+    assert i0.tolist() == [[5, 3]] * 4
+    assert i1.tolist() == [[1, 3]] * 4
+    assert torch.allclose(w0, torch.tensor([[1 / (1 + math.exp(-10)), 1 / (1 + math.exp(10))]] * 4))
+    assert torch.all(w1 == 0.5)  # equal logits, equal weights
+    _, w3, _ = oracle.topk(l1, 2, oracle.ROUTER_CLAMP | oracle.ROUTER_RAW)
+    assert torch.all(w3 == 50.0)
+
+
+@pytest.mark.parametrize("k", [1, 2, 4])
+def test_raw_weights_are_the_chosen_logits(k):
+    T, E = 40, 12
+    logits = inputgen.fill_normal(torch.empty(T * E), 9, 11, 2.0).view(T, E)
+    idx0, w0, gap0 = oracle.topk(logits, k)
+    idx, w, gap = oracle.topk(logits, k, oracle.ROUTER_RAW)
+    assert torch.equal(idx, idx0) and torch.equal(gap, gap0)  # selection unchanged
+    assert torch.equal(w, torch.gather(logits, 1, idx.long()))
+    assert torch.all(w[:, :-1] >= w[:, 1:])
+    # weights_for on an arbitrary selection agrees
+    other = torch.tensor([[(t + 5 * j) % E for j in range(k)] for t in range(T)], dtype=torch.int32)
+    assert torch.equal(oracle.weights_for(logits, other, oracle.ROUTER_RAW), torch.gather(logits, 1, other.long()))
+    with pytest.raises(RuntimeError):
+        oracle.topk(logits, k, 4)  # unknown variant bit
+
+
 # ------------------------------------------------------------------------- grouping
 
 
@@ -233,10 +296,22 @@ def test_single_expert_is_dense_swiglu(act):
     assert _rel_err(out["y"].numpy(), want.numpy()) < 2e-6
 
 
-@pytest.mark.parametrize("case", ["f32", "bf16", "bf16_shared", "bf16_bias", "i8"])
+@pytest.mark.parametrize("case", ["f32", "bf16", "bf16_shared", "bf16_bias", "i8", "bf16_clamp", "f32_raw",
+                                  "i8_clamp_raw"])
 def test_layer_equals_brute_force_dense(case):
     kw = dict(T=23, d=64, E=6, k=2, f=96)
-    if case == "f32":
+    flags = 0
+    if case == "bf16_clamp":
+        # three experts beyond 50: clamped, they tie and the two lowest indices win
+        wl = inputgen.custom(case, bias=((5, 70.0), (3, 60.0), (1, 55.0)), **kw)
+        flags = oracle.ROUTER_CLAMP
+    elif case == "f32_raw":
+        wl = inputgen.custom(case, act=inputgen.F32, wdt=inputgen.F32, **dict(kw, k=3))
+        flags = oracle.ROUTER_RAW
+    elif case == "i8_clamp_raw":
+        wl = inputgen.custom(case, act=inputgen.BF16, wdt=inputgen.I8, bias=((4, 49.5),), **kw)
+        flags = oracle.ROUTER_CLAMP | oracle.ROUTER_RAW
+    elif case == "f32":
         wl = inputgen.custom(case, act=inputgen.F32, wdt=inputgen.F32, **kw)
     elif case == "bf16":
         wl = inputgen.custom(case, **kw)
@@ -248,9 +323,14 @@ def test_layer_equals_brute_force_dense(case):
         wl = inputgen.custom(case, act=inputgen.BF16, wdt=inputgen.I8, **kw)
     p = inputgen.make_problem(wl, seed=3)
     out = oracle.moe_forward(p.x, p.router_w, p.router_b, wl.k, p.expert_w, p.expert_stride, wl.f,
-                             p.expert_scales, p.shared_w, wl.fs)
-    y, sel, mask = _dense_layer(p)
+                             p.expert_scales, p.shared_w, wl.fs, flags)
+    y, sel, mask = _dense_layer(p, flags)
     assert np.array_equal(out["idx"].numpy(), sel)
+    if case == "bf16_clamp":
+        assert out["idx"].tolist() == [[1, 3]] * wl.T
+    if case == "i8_clamp_raw":
+        assert torch.all(out["idx"][:, 0] == 4) and torch.all(out["w"][:, 0] <= 50.0)
+        assert 0 < int((out["w"][:, 0] == 50.0).sum()) < wl.T
     assert _rel_err(out["y"].numpy(), y) < 2e-6
     # the sampled path agrees bit for bit with the whole-layer path
     toks = [0, 5, 22, 11]
