@@ -111,7 +111,6 @@ constexpr int kDsTmemCols = 256;
 constexpr size_t kDsRingBytes = 200 * 1024;
 constexpr int kDsMaxStages = 12;
 constexpr int kDsMaxKbs = 4;
-constexpr int kDsPrefetchBlocks = 24;  // weight blocks (16 KB each) pulled into L2 while the ring waits
 
 struct alignas(64) DecStreamParams {
   CUtensorMap mapW;   // int8 weights: gate/up {d, f, 2, E} (W1, W3); down {f, d, E} (W2)
@@ -250,24 +249,6 @@ __device__ bool ds_produce(const DecStreamParams& p, uint8_t* smem, DsCtl& c, in
   const uint64_t policy = l2_evict_first_policy();
   int held = 0;
   bool released = !defer;
-  // L2 prefetch of the weight blocks that follow the current position (item L, next block kb,
-  // `left` blocks left in that item), up to kDsPrefetchBlocks blocks.
-  auto prefetch_ahead = [&](int L, int kb, int left) {
-    int n = 0;
-    DecItem q;
-    for (int L2 = L; n < kDsPrefetchBlocks && dec_item<kGateUp>(p, c.touched, c.pre[pre_idx], c.ntouched, c.off, L2, q);
-         L2 += gridDim.x) {
-      const int kbeg = q.split * p.kspan, kend = min(p.K, kbeg + p.kspan);
-      const int nkb2 = (kend - kbeg + 127) / 128;
-      int b = (L2 == L) ? kb : L2 % nkb2;
-      int cnt = (L2 == L) ? left : nkb2;
-      for (; cnt > 0 && n < kDsPrefetchBlocks; --cnt, ++n, b = (b + 1 == nkb2) ? 0 : b + 1) {
-        const int kx = kbeg + b * 128;
-        if (kGateUp) tma_prefetch_l2_4d(&p.mapW, kx, q.tile * 128, q.mat, q.e);
-        else tma_prefetch_l2_3d(&p.mapW, kx, q.tile * 128, q.e);
-      }
-    }
-  };
   auto release = [&]() {
     for (int h = 0; h < held; ++h) {
       uint8_t* st = smem + (size_t)c.defer_s[h] * p.stage_bytes;
@@ -307,10 +288,10 @@ __device__ bool ds_produce(const DecStreamParams& p, uint8_t* smem, DsCtl& c, in
         c.defer_nk[held] = nk;
         c.defer_s[held] = r.s;
         if (++held == S) {
-          // The ring is full of weight copies and the planes are not ready yet: pull the next
-          // weight blocks of this CTA into L2 meanwhile, so the stream resumes from L2.
-          prefetch_ahead(L, kb, nkb - i - nk);
-          // the held plane copies are issued even when the wait gave up, so that every issued
+          // The ring is full of weight copies and the planes are not ready yet.  (Pulling the
+          // next weight blocks into L2 meanwhile measured slower: the extra requests delayed the
+          // last items of the other CTAs and the grid barrier behind them.)
+          // The held plane copies are issued even when the wait gave up, so that every issued
           // stage completes and the error path drains quickly
           const bool go = ready();
           release();
