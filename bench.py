@@ -56,8 +56,8 @@ def kernels_per_step(wl):
 # same kernel on the same workload (profiles/); None where no capture of the current kernel
 # exists.  Keyed by (workload, dominant-kernel tag).
 NCU_TRAFFIC = {
-    ("mixtral_prefill_bf16", "tc2_ffn"): 2.943e9 + 0.230e9,     # tc2_ffn_traffic_mixtral_prefill_bf16.md
-    ("fine_grained_shared_bf16", "tc_ffn"): 1.0089e9 + 74.8e6,  # launches_fine_grained_shared_bf16.md
+    ("mixtral_prefill_bf16", "tc2_ffn"): 3.1173e9 + 0.2305e9,      # tc2_ffn_traffic_mixtral_prefill_bf16.md
+    ("fine_grained_shared_bf16", "tc_ffn"): 1.00698e9 + 74.0e6,   # launches_fine_grained_shared_bf16.md
 }
 
 # fp32 FMA peak: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (the unit counts and clock of the part)

@@ -51,6 +51,15 @@ typedef enum {
 
 typedef enum { COLIBRI_F32 = 0, COLIBRI_BF16 = 1, COLIBRI_I8 = 2 } colibri_dtype;
 
+/* Layout of the int8 weight scales (colibri_desc.weight_scale_mode). */
+typedef enum {
+  COLIBRI_SCALE_PER_CHANNEL = 0,  /* per expert e at e * (2f + d): s1[f] | s3[f] | s2[d] (one fp32
+                                     per output channel of W1, W3, W2)                          */
+  COLIBRI_SCALE_PER_MATRIX = 1    /* per expert e at 3 * e: s1 | s3 | s2, one fp32 per weight
+                                     matrix (www.0539edu.com/news/4774449 §3.1: a scale computed
+                                     for each expert weight matrix, symmetric int8)            */
+} colibri_scale_mode;
+
 /* Router variants, OR-ed into colibri_desc.router_flags (0 = the default router). */
 typedef enum {
   COLIBRI_ROUTER_CLAMP = 1,       /* clamp every logit to [-50, 50] before selection and
@@ -82,6 +91,9 @@ typedef enum {
  *                   expert index on ties) is the same for every variant, applied to the clamped
  *                   logits when COLIBRI_ROUTER_CLAMP is set (logits above 50 then tie and go to
  *                   the lower index).  Unknown bits: COLIBRI_ERR_INVALID_ARG.
+ *   weight_scale_mode  COLIBRI_I8 weights: COLIBRI_SCALE_PER_CHANNEL (0) or
+ *                   COLIBRI_SCALE_PER_MATRIX; must be 0 for other weight types (INVALID_ARG).
+ *                   W[o][i] = s * q[o][i] with s the channel's or the matrix's scale.
  */
 typedef struct {
   int32_t d_model;
@@ -94,6 +106,7 @@ typedef struct {
   int32_t max_tokens;
   int32_t device_id;
   int32_t router_flags;
+  int32_t weight_scale_mode;
 } colibri_desc;
 
 typedef struct colibri_ctx colibri_ctx; /* opaque */
@@ -127,7 +140,8 @@ int64_t colibri_expert_stride(const colibri_ctx* ctx);
  *                W1[f][d] | W3[f][d] | W2[d][f], each row-major with rows = output channels
  *                ([out, in]).  W1 is the gate, W3 the up and W2 the down projection.
  *   expert_scales  COLIBRI_I8 only: device fp32, per expert e at e * (2f + d): s1[f] | s3[f] |
- *                s2[d]; weight W[o][i] = s[o] * q[o][i].  Must be NULL otherwise.
+ *                s2[d]; weight W[o][i] = s[o] * q[o][i] (with COLIBRI_SCALE_PER_MATRIX: at 3 * e,
+ *                s1 | s3 | s2, W[o][i] = s * q[o][i]).  Must be NULL otherwise.
  *   shared_w     device, W1s[f_s][d] | W3s[f_s][d] | W2s[d][f_s] in weight_dtype, when
  *                shared_d_ff > 0; must be NULL otherwise.
  *   y            [T, d_model] act_dtype, device or host; fully overwritten.  Host y is written

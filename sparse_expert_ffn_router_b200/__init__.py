@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libcolibri.so")
 
 COLIBRI_F32, COLIBRI_BF16, COLIBRI_I8 = 0, 1, 2
 COLIBRI_ROUTER_CLAMP, COLIBRI_ROUTER_RAW_WEIGHTS = 1, 2
+COLIBRI_SCALE_PER_CHANNEL, COLIBRI_SCALE_PER_MATRIX = 0, 1
 
 STATUS = {
     0: "COLIBRI_OK",
@@ -59,6 +60,7 @@ class colibri_desc(ctypes.Structure):
         ("max_tokens", ctypes.c_int32),
         ("device_id", ctypes.c_int32),
         ("router_flags", ctypes.c_int32),
+        ("weight_scale_mode", ctypes.c_int32),
     ]
 
 
@@ -144,10 +146,10 @@ def colibri_last_error(ctx=None) -> str:
 
 def colibri_init(d_model: int, d_ff: int, num_experts: int, top_k: int, shared_d_ff: int = 0,
                  act_dtype: int = COLIBRI_BF16, weight_dtype: int = COLIBRI_BF16, max_tokens: int = 1,
-                 device_id: int = 0, router_flags: int = 0) -> int:
+                 device_id: int = 0, router_flags: int = 0, weight_scale_mode: int = 0) -> int:
     """Returns the opaque context handle (an address)."""
     desc = colibri_desc(d_model, d_ff, num_experts, top_k, shared_d_ff, act_dtype, weight_dtype,
-                        max_tokens, device_id, router_flags)
+                        max_tokens, device_id, router_flags, weight_scale_mode)
     out = ctypes.c_void_p()
     _check(load().colibri_init(ctypes.byref(desc), ctypes.byref(out)), "colibri_init")
     return out.value
@@ -222,10 +224,11 @@ class MoELayer:
     """Owns one context; forwards tensors to the C ABI (no computation in Python)."""
 
     def __init__(self, d_model, d_ff, num_experts, top_k, shared_d_ff=0, act_dtype=COLIBRI_BF16,
-                 weight_dtype=COLIBRI_BF16, max_tokens=1, device_id=0, router_flags=0):
+                 weight_dtype=COLIBRI_BF16, max_tokens=1, device_id=0, router_flags=0, weight_scale_mode=0):
         self.desc = dict(d_model=d_model, d_ff=d_ff, num_experts=num_experts, top_k=top_k,
                          shared_d_ff=shared_d_ff, act_dtype=act_dtype, weight_dtype=weight_dtype,
-                         max_tokens=max_tokens, device_id=device_id, router_flags=router_flags)
+                         max_tokens=max_tokens, device_id=device_id, router_flags=router_flags,
+                         weight_scale_mode=weight_scale_mode)
         self.ctx = colibri_init(**self.desc)
 
     @property

@@ -161,6 +161,8 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
     return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "max_tokens=%d must be >= 1", D.max_tokens);
   if (D.router_flags & ~(COLIBRI_ROUTER_CLAMP | COLIBRI_ROUTER_RAW_WEIGHTS))
     return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "router_flags=0x%x has unknown bits", (unsigned)D.router_flags);
+  if (D.weight_scale_mode != COLIBRI_SCALE_PER_CHANNEL && D.weight_scale_mode != COLIBRI_SCALE_PER_MATRIX)
+    return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "weight_scale_mode=%d unknown", D.weight_scale_mode);
   if ((int64_t)D.max_tokens * D.top_k > (1ll << 30))
     return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "max_tokens * top_k too large");
   const bool f32 = D.act_dtype == COLIBRI_F32 && D.weight_dtype == COLIBRI_F32;
@@ -174,6 +176,8 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
     return fail(nullptr, COLIBRI_ERR_UNSUPPORTED, "shared expert with int8 weights is not supported");
   if (i8 && D.d_ff > kDecMaxFF)
     return fail(nullptr, COLIBRI_ERR_UNSUPPORTED, "int8 weights support d_ff <= %d", kDecMaxFF);
+  if (!i8 && D.weight_scale_mode != COLIBRI_SCALE_PER_CHANNEL)
+    return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "weight_scale_mode applies to int8 weights only");
   if (f32 && ((int64_t)D.max_tokens * D.top_k / kSimtBM + D.num_experts > 65535 ||
               ((int64_t)D.max_tokens + kSimtBM - 1) / kSimtBM > 65535))
     return fail(nullptr, COLIBRI_ERR_UNSUPPORTED, "fp32 path limited to max_tokens * top_k < 4M rows");
@@ -465,6 +469,7 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
       fa.planes_scale = w.plane_scale;
       fa.W = (const int8_t*)expert_w;
       fa.scales = expert_scales;
+      fa.scale_mode = D.weight_scale_mode;
       fa.wstride = stride;
       fa.d = d;
       fa.f = f;
@@ -496,12 +501,12 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
       mark(3);
     } else {
       COLIBRI_TRY(launch_dec_gateup(w.plane_hi, w.plane_lo, w.plane_scale, (const int8_t*)expert_w, expert_scales,
-                                    stride, d, f, E, w.offsets, gsplit, (float*)w.H, R, T, w.err, s), "dec_gateup");
+                                    D.weight_scale_mode, stride, d, f, E, w.offsets, gsplit, (float*)w.H, R, T, w.err, s), "dec_gateup");
       mark(3);
       COLIBRI_TRY(launch_dec_finish_h((const float*)w.H, gsplit, R, f, nsplit, w.plane_hi, w.plane_lo,
                                       w.plane_scale, s), "dec_finish_h");
       COLIBRI_TRY(launch_dec_down(w.plane_hi, w.plane_lo, w.plane_scale, (const int8_t*)expert_w, expert_scales,
-                                  stride, d, f, E, w.offsets, nsplit, R, w.Ypart, T, w.err, s), "dec_down");
+                                  D.weight_scale_mode, stride, d, f, E, w.offsets, nsplit, R, w.Ypart, T, w.err, s), "dec_down");
     }
   }
   mark(4);

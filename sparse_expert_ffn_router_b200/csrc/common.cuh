@@ -276,17 +276,20 @@ cudaError_t launch_tcs_down(const TcGemmArgs& a, cudaStream_t s);
 // max_rows_per_expert: an upper bound (T) that picks the token chunk (8, 16 or 32 rows).
 cudaError_t configure_dec_kernels();  // once per device, before any launch
 // gate/up: W1 . x and W3 . x (scaled) as fp32 K-split partials GU [nsplit, 2, R, f]
+// scale_mode: COLIBRI_SCALE_PER_CHANNEL (scales per expert [f | f | d]) or
+// COLIBRI_SCALE_PER_MATRIX (scales [E][3]: W1, W3, W2)
 cudaError_t launch_dec_gateup(const int8_t* Xhi, const int8_t* Xlo, const float* xscale, const int8_t* W,
-                              const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
-                              int nsplit, float* GU, int R, int max_rows_per_expert, uint32_t* err, cudaStream_t s);
+                              const float* scales, int scale_mode, int64_t wstride, int d, int f, int E,
+                              const int32_t* offsets, int nsplit, float* GU, int R, int max_rows_per_expert,
+                              uint32_t* err, cudaStream_t s);
 // H = silu(sum g) * (sum u) (bf16) from the gsplit partials GU, split into int8 planes with one
 // scale per (down K split, row): scale[ds * R + r] covers H[r][ds * f / dsplit, (ds + 1) * f / dsplit).
 cudaError_t launch_dec_finish_h(const float* GU, int gsplit, int R, int f, int dsplit, int8_t* hi, int8_t* lo,
                                 float* scale, cudaStream_t s);
 cudaError_t launch_dec_down(const int8_t* Hhi, const int8_t* Hlo, const float* hscale, const int8_t* W,
-                            const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
-                            int nsplit, int R, float* Ypart, int max_rows_per_expert, uint32_t* err,
-                            cudaStream_t s);
+                            const float* scales, int scale_mode, int64_t wstride, int d, int f, int E,
+                            const int32_t* offsets, int nsplit, int R, float* Ypart, int max_rows_per_expert,
+                            uint32_t* err, cudaStream_t s);
 // The whole int8 expert stage (gate/up stream, H planes, down stream, combine) in one
 // cooperative launch with grid barriers; the x planes must already be in planes_hi/lo/scale.
 struct DecFusedArgs {
@@ -295,6 +298,7 @@ struct DecFusedArgs {
   float* planes_scale;      // x scales [R] in; H scales [dsplit, R] written
   const int8_t* W;          // expert buffer (int8) and its per-channel scales
   const float* scales;
+  int scale_mode;           // COLIBRI_SCALE_PER_CHANNEL or COLIBRI_SCALE_PER_MATRIX
   int64_t wstride;
   int d, f, E, T, k;
   const int32_t* offsets;   // [E+1] (written by an earlier launch unless route_in_kernel)

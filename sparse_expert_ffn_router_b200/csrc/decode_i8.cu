@@ -116,7 +116,8 @@ struct alignas(64) DecStreamParams {
   CUtensorMap mapW;   // int8 weights: gate/up {d, f, 2, E} (W1, W3); down {f, d, E} (W2)
   CUtensorMap mapHi;  // int8 activation planes {K, R}
   CUtensorMap mapLo;
-  const float* wscale;      // expert scales base (per expert: s1[f] | s3[f] | s2[d])
+  const float* wscale;      // expert scales: per expert s1[f] | s3[f] | s2[d], or [E][3] per matrix
+  int scale_per_matrix;     // 1: one scale per weight matrix (W1, W3, W2) of each expert
   const float* rscale;      // plane scales: rscale[split * rscale_split_stride + row]
   int rscale_split_stride;  // 0: one scale per row (x planes); R: one per (K split, row) (H planes)
   const int32_t* offsets;   // [E+1]
@@ -196,7 +197,6 @@ struct DsCtl {
   int consumed;
   int flag;      // result of a grid-wide wait, broadcast to the epilogue warps
   int hpass;     // fused kernel: 1 once the epilogue warps passed the H barrier, -1 if it failed
-  uint32_t pbase;  // fused kernel: start of this launch's round on the planes barrier
   int first;     // this CTA's first work item (items first, first + gridDim.x, ...)
   int ntouched;
   int32_t off[kMaxExperts + 1];     // row offsets of the experts' groups
@@ -366,8 +366,10 @@ __device__ bool ds_epilogue(const DecStreamParams& p, DsCtl& c, int pre_idx, int
     // the weight scale is an input of the call: loaded before the accumulator is waited for
     const int o = it.tile * 128 + q * 32 + lane;
     const bool vo = o < p.out_rows;
-    const float* es = p.wscale + (size_t)it.e * (2 * p.f + p.d);
-    const float sc = vo ? __ldg(es + (kGateUp ? it.mat * p.f : 2 * p.f) + o) : 0.f;
+    const int m = kGateUp ? it.mat : 2;  // W1, W3 or W2
+    const float* sp = p.scale_per_matrix ? p.wscale + (size_t)it.e * 3 + m
+                                         : p.wscale + (size_t)it.e * (2 * p.f + p.d) + (size_t)m * p.f + o;
+    const float sc = vo ? __ldg(sp) : 0.f;
     const bool got = ds_wait(&c.tfull[a], aph, &c.abort);
     if (!__all_sync(0xffffffffu, got)) return false;
     tc_fence_after();
@@ -640,7 +642,8 @@ __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" :::
 // same in every CTA, so no second exchange is needed), and for the CTA's own tokens: dst_row,
 // src_row and the int8 planes of the token row in each of its k grouped rows.  The ring memory,
 // idle until the producer starts, holds the scratch.  CTA 0 also writes counts and offsets.
-// Arrives on the planes barrier; the producer waits on it before its first plane copy.
+// The caller then arrives on the planes barrier; the producer waits on it before its first plane
+// copy.
 __device__ void fused_route(const DecFusedParams& p, uint8_t* smem, DsCtl& c) {
   constexpr int kWarps = kDsThreads / 32;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -832,10 +835,9 @@ __device__ void fused_route(const DecFusedParams& p, uint8_t* smem, DsCtl& c) {
       }
     }
   }
-  // the planes are read next by TMA copies of other CTAs
+  // the planes are read next by TMA copies of other CTAs; the caller arrives on the planes
+  // barrier after its next CTA barrier
   fence_proxy_async_global();
-  __syncthreads();
-  if (tid == 0) c.pbase = bar_base(bar_arrive(&p.bar[kBarPlanes], G), G);  // the producer (this thread) waits
 }
 
 __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_constant__ DecFusedParams p) {
@@ -846,6 +848,7 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_c
   const int G = gridDim.x;
   const bool aligned = (smem_u32(smem) & 1023u) == 0;  // the 128-byte swizzle needs 1024-byte stages
   const DecStreamParams* phases[2] = {&p.gu, &p.dn};
+  uint32_t planes_old = 0;  // thread 0: the planes barrier count before its arrival
   if (aligned) {
     ds_init(phases, 2, c, S);
     if (p.route_in_kernel) {
@@ -853,7 +856,10 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_c
       // CTAs 0..T-1 also split their token's planes and start last: the items are dealt so
       // that the CTAs that take one item more than the others are not among them
       if (threadIdx.x == 0) c.first = (int)((blockIdx.x + gridDim.x - (unsigned)min(p.T, (int)gridDim.x)) % gridDim.x);
-      ds_items(phases, 2, c, nullptr);
+      ds_items(phases, 2, c, nullptr);  // starts with a CTA barrier: this CTA's planes are written
+      // Arrival on the planes barrier by the producer thread itself; the count it returns is
+      // only needed when the producer waits, so the round trip overlaps its first copies.
+      if (threadIdx.x == 0) planes_old = bar_arrive(&p.bar[kBarPlanes], G);
     } else {
       ds_items(phases, 2, c, p.gu.offsets);
     }
@@ -872,7 +878,7 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_c
       // with the routing done in this launch, the gate/up weights go out at once and the plane
       // copies wait until every CTA has written its tokens' planes
       bool ok = ds_produce<true>(p.gu, smem, c, S, 0, r, p.route_in_kernel != 0, [&] {
-        if (!grid_wait(&p.bar[kBarPlanes], c.pbase, G, &c.abort)) return false;
+        if (!grid_wait(&p.bar[kBarPlanes], bar_base(planes_old, G), G, &c.abort)) return false;
         fence_proxy_async_global();
         return true;
       });
@@ -1129,14 +1135,15 @@ namespace {
 // Parameters of one stream phase (weights, planes, scales, outputs); false if a tensor map
 // cannot be encoded.
 bool dec_gateup_params(DecStreamParams& p, const int8_t* Xhi, const int8_t* Xlo, const float* xscale, const int8_t* W,
-                       const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets, int nsplit,
-                       float* GU, int R, int max_rows_per_expert, uint32_t* err) {
+                       const float* scales, int scale_mode, int64_t wstride, int d, int f, int E,
+                       const int32_t* offsets, int nsplit, float* GU, int R, int max_rows_per_expert, uint32_t* err) {
   memset(&p, 0, sizeof(p));
   const uint64_t dims[4] = {(uint64_t)d, (uint64_t)f, 2, (uint64_t)E};
   const uint64_t st[3] = {(uint64_t)d, (uint64_t)f * d, (uint64_t)wstride};
   const uint32_t box[4] = {128, 128, 1, 1};
   if (!make_tmap(&p.mapW, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, 4, dims, st, box)) return false;
   p.wscale = scales;
+  p.scale_per_matrix = scale_mode == COLIBRI_SCALE_PER_MATRIX;
   p.rscale = xscale;
   p.offsets = offsets;
   p.E = E;
@@ -1154,14 +1161,15 @@ bool dec_gateup_params(DecStreamParams& p, const int8_t* Xhi, const int8_t* Xlo,
 }
 
 bool dec_down_params(DecStreamParams& p, const int8_t* Hhi, const int8_t* Hlo, const float* hscale, const int8_t* W,
-                     const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets, int nsplit,
-                     int R, float* Ypart, int max_rows_per_expert, uint32_t* err) {
+                     const float* scales, int scale_mode, int64_t wstride, int d, int f, int E,
+                     const int32_t* offsets, int nsplit, int R, float* Ypart, int max_rows_per_expert, uint32_t* err) {
   memset(&p, 0, sizeof(p));
   const uint64_t dims[3] = {(uint64_t)f, (uint64_t)d, (uint64_t)E};
   const uint64_t st[2] = {(uint64_t)f, (uint64_t)wstride};
   const uint32_t box[3] = {128, 128, 1};
   if (!make_tmap(&p.mapW, CU_TENSOR_MAP_DATA_TYPE_UINT8, W + 2 * (size_t)f * d, 3, dims, st, box)) return false;
   p.wscale = scales;
+  p.scale_per_matrix = scale_mode == COLIBRI_SCALE_PER_MATRIX;
   p.rscale = hscale;
   p.rscale_split_stride = R;
   p.offsets = offsets;
@@ -1182,10 +1190,11 @@ bool dec_down_params(DecStreamParams& p, const int8_t* Hhi, const int8_t* Hlo, c
 }  // namespace
 
 cudaError_t launch_dec_gateup(const int8_t* Xhi, const int8_t* Xlo, const float* xscale, const int8_t* W,
-                              const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
-                              int nsplit, float* GU, int R, int max_rows_per_expert, uint32_t* err, cudaStream_t s) {
+                              const float* scales, int scale_mode, int64_t wstride, int d, int f, int E,
+                              const int32_t* offsets, int nsplit, float* GU, int R, int max_rows_per_expert,
+                              uint32_t* err, cudaStream_t s) {
   DecStreamParams p;
-  if (!dec_gateup_params(p, Xhi, Xlo, xscale, W, scales, wstride, d, f, E, offsets, nsplit, GU, R,
+  if (!dec_gateup_params(p, Xhi, Xlo, xscale, W, scales, scale_mode, wstride, d, f, E, offsets, nsplit, GU, R,
                          max_rows_per_expert, err))
     return cudaErrorInvalidValue;
   return launch_stream<true>(p, s);
@@ -1202,11 +1211,11 @@ cudaError_t launch_dec_finish_h(const float* GU, int gsplit, int R, int f, int d
 }
 
 cudaError_t launch_dec_down(const int8_t* Hhi, const int8_t* Hlo, const float* hscale, const int8_t* W,
-                            const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
-                            int nsplit, int R, float* Ypart, int max_rows_per_expert, uint32_t* err,
-                            cudaStream_t s) {
+                            const float* scales, int scale_mode, int64_t wstride, int d, int f, int E,
+                            const int32_t* offsets, int nsplit, int R, float* Ypart, int max_rows_per_expert,
+                            uint32_t* err, cudaStream_t s) {
   DecStreamParams p;
-  if (!dec_down_params(p, Hhi, Hlo, hscale, W, scales, wstride, d, f, E, offsets, nsplit, R, Ypart,
+  if (!dec_down_params(p, Hhi, Hlo, hscale, W, scales, scale_mode, wstride, d, f, E, offsets, nsplit, R, Ypart,
                        max_rows_per_expert, err))
     return cudaErrorInvalidValue;
   return launch_stream<false>(p, s);
@@ -1218,9 +1227,11 @@ cudaError_t launch_dec_fused(const DecFusedArgs& a, cudaStream_t s) {
   DecFusedParams p;
   memset(&p, 0, sizeof(p));
   const int R = a.T * a.k;
-  if (!dec_gateup_params(p.gu, a.planes_hi, a.planes_lo, a.planes_scale, a.W, a.scales, a.wstride, a.d, a.f, a.E,
+  if (!dec_gateup_params(p.gu, a.planes_hi, a.planes_lo, a.planes_scale, a.W, a.scales, a.scale_mode, a.wstride, a.d,
+                         a.f, a.E,
                          a.offsets, a.gsplit, a.GU, R, a.T, a.err) ||
-      !dec_down_params(p.dn, a.planes_hi, a.planes_lo, a.planes_scale, a.W, a.scales, a.wstride, a.d, a.f, a.E,
+      !dec_down_params(p.dn, a.planes_hi, a.planes_lo, a.planes_scale, a.W, a.scales, a.scale_mode, a.wstride, a.d,
+                       a.f, a.E,
                        a.offsets, a.dsplit, R, a.Ypart, a.T, a.err))
     return cudaErrorInvalidValue;
   p.hhi = a.planes_hi;

@@ -73,6 +73,8 @@ def _desc(**kw):
     (dict(weight_dtype=colibri.COLIBRI_I8, shared_d_ff=64), -3),
     (dict(router_flags=4), -1),        # unknown router variant bit
     (dict(router_flags=-1), -1),
+    (dict(weight_scale_mode=1), -1),   # per-matrix scales with bf16 weights
+    (dict(weight_scale_mode=2, weight_dtype=colibri.COLIBRI_I8), -1),
 ])
 def test_init_rejects_bad_descriptions(lib, kw, code):
     with pytest.raises(colibri.ColibriError) as ei:

@@ -7,6 +7,8 @@ k = 1 and k = E, more than 32 decode tokens on one expert).  The full-size workl
 the launch configuration the benchmark times, with routing compared on every token and the
 layer output on a sample of tokens.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -352,6 +354,35 @@ def test_router_variants(name, flags, monkeypatch):
         assert torch.equal(r["idx"][robust], r["ref_idx"][robust]), "tie at 50 not resolved to the lower index"
         ties = [t for t in robust if (lc[t] == 50.0).sum() >= 2]
         assert ties or wl.T == 1  # the tie rule was exercised (a single token may have no tie)
+
+
+# int8 weights with one scale per weight matrix (W1, W3, W2 of each expert) instead of one per
+# output channel: the GPU gets the [E][3] scales; the oracle gets the same scales written out per
+# channel (W[o][i] = s * q[o][i] for every o), which is what the per-matrix layout means.
+@pytest.mark.parametrize("name", ["i8_small", "i8_T1", "i8_many", "i8_small_split"])
+def test_int8_per_matrix_scales(name, monkeypatch):
+    if name.endswith("_split"):  # the four-launch plan (separate gate/up, H, down, combine)
+        monkeypatch.setenv("COLIBRI_DEC_FUSED", "0")
+        name = name[: -len("_split")]
+    wl = VARIANT.get(name) or SMALL[name]
+    p = inputgen.make_problem(wl, seed=13)
+    f, d, E = wl.f, wl.d, wl.E
+    per_channel = p.expert_scales.view(E, 2 * f + d)
+    per_matrix = torch.stack([per_channel[:, 0], per_channel[:, f], per_channel[:, 2 * f]], dim=1).contiguous()
+    written_out = torch.cat([per_matrix[:, 0:1].expand(E, f), per_matrix[:, 1:2].expand(E, f),
+                             per_matrix[:, 2:3].expand(E, d)], dim=1).contiguous().view(-1)
+    p_ref = dataclasses.replace(p, expert_scales=written_out)
+    p_gpu = dataclasses.replace(p, expert_scales=per_matrix.view(-1))
+    layer = colibri.MoELayer(wl.d, wl.f, wl.E, wl.k, wl.fs, wl.act, wl.wdt, max_tokens=wl.T,
+                             weight_scale_mode=colibri.COLIBRI_SCALE_PER_MATRIX)
+    gpu = H.run_gpu(p_gpu, layer=layer)
+    layer.close()
+    ref = oracle.problem_forward(p_ref)
+    idx_use, w_use, _ = H.compare_routing(p_ref, ref, gpu)
+    toks = list(range(wl.T))
+    y_ref = oracle.combine(p_ref.x, idx_use, w_use, p_ref.expert_w, p_ref.expert_stride, f, p_ref.expert_scales,
+                           None, 0, toks)
+    H.check_y(p_ref, gpu["y"], y_ref)
 
 
 def test_smaller_T_on_a_larger_context():
