@@ -44,6 +44,20 @@ def test_library_exports_every_declared_symbol(lib):
         assert getattr(lib, name) is not None
 
 
+def test_descriptor_layout_matches_the_header(tmp_path):
+    # the binding's ctypes struct must have the C struct's size and field offsets
+    fields = [name for name, _ in colibri.colibri_desc._fields_]
+    src = tmp_path / "layout.c"
+    body = "".join(f'  printf("%zu\\n", offsetof(colibri_desc, {n}));\n' for n in fields)
+    src.write_text('#include <stddef.h>\n#include <stdio.h>\n#include "colibri.h"\nint main(void) {\n'
+                   '  printf("%zu\\n", sizeof(colibri_desc));\n' + body + "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    assert got[0] == ctypes.sizeof(colibri.colibri_desc)
+    assert got[1:] == [getattr(colibri.colibri_desc, n).offset for n in fields]
+
+
 def test_status_strings(lib):
     for code, name in colibri.STATUS.items():
         assert colibri.colibri_status_string(code).startswith(name)
