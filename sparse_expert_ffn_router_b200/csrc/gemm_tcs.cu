@@ -36,7 +36,6 @@ constexpr int SW_EPI_THREADS = 128;
 constexpr int SW_BK = 64;                       // K elements per stage (128 bytes of bf16)
 constexpr int SW_W_BYTES = 128 * SW_BK * 2;     // 16 KB: one 128-channel weight tile
 constexpr int SW_BOX_ROWS = 16;                 // MMA N granularity; token rows of the small TMA box
-constexpr int SW_BOX_BYTES = SW_BOX_ROWS * SW_BK * 2;
 constexpr int SW_BIG_ROWS = 64;                 // token rows of the large TMA box
 constexpr int SW_STAGE_BYTES = 48 * 1024;       // gate/up: W1 + W3 + 128 rows; down: W2 + 256 rows
 constexpr int SW_STAGES = 4;
