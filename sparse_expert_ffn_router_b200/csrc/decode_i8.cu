@@ -1,7 +1,8 @@
-// Expert Compute stage for int8 weights with per-output-channel fp32 scales, dequantised in
-// the kernel (www.0539edu.com/news/4774449 §3.1 stores int8 weights with scales; the scale
-// here is per output channel).  For a handful of tokens the layer is a stream over the
-// weights of the touched experts, bound by HBM bandwidth:
+// Expert Compute stage for int8 weights with fp32 scales, dequantised in the kernel
+// (www.0539edu.com/news/4774449 §3.1 stores int8 weights with a scale per weight matrix; the
+// default here is one scale per output channel, the per-matrix layout is an option).  For a
+// handful of tokens the layer is a stream over the weights of the touched experts, bound by HBM
+// bandwidth:
 //
 //   gate/up:  H[r][o]    = silu(s1[o] * sum_i q1[o][i] x[r][i]) * (s3[o] * sum_i q3[o][i] x[r][i])
 //   down:     Yp_s[r][o] = s2[o] * sum_{i in split s} q2[o][i] H[r][i]
@@ -25,6 +26,11 @@
 // offsets, so experts that received no rows cost nothing.  The down projection is split over K
 // into fp32 partial sums (summed in fixed order by the combine) to spread one token over every
 // SM.  Every wait is bounded.
+//
+// dec_fused_kernel runs the whole stage (for up to 64 tokens also the router, top-k and the
+// grouping) as one cooperative launch whose phases are separated by grid barriers; the four
+// separate kernels (dec_stream_kernel twice, dec_finish_h_kernel, and the combine) remain as the
+// plan taken when the fused launch is turned off.
 #include <algorithm>
 #include <cstdlib>
 #include <cstring>
