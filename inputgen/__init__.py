@@ -11,8 +11,14 @@ the C ABI expects:
 * ``router_b``   [E] float32 or None
 * ``expert_w``   one buffer; expert e starts at element ``e * expert_stride`` and
                  holds W1[f, d] | W3[f, d] | W2[d, f] (rows are [out, in])
-* ``expert_scales`` (int8 weights only) per expert [f | f | d] float32
+* ``expert_scales`` int8 weights: per expert [f | f | d] float32 (one per output channel);
+                 int4 weights: per expert s1[f, d/128] | s3[f, d/128] | s2[d, f/128] float32
+                 (one per output channel and group of 128 consecutive inputs)
 * ``shared_w``   W1s[fs, d] | W3s[fs, d] | W2s[d, fs] or None
+
+int4 weights are stored packed, two per byte along the input dimension: element 2j of a row in
+the low nibble of byte j, element 2j + 1 in the high nibble, each a two's-complement 4-bit
+integer; the buffer is a uint8 tensor and ``expert_stride`` still counts elements (nibbles).
 """
 from __future__ import annotations
 
@@ -29,9 +35,10 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libinputgen.so")
 _lib = None
 
-F32, BF16, I8 = 0, 1, 2
-_TORCH_DTYPE = {F32: torch.float32, BF16: torch.bfloat16, I8: torch.int8}
-DTYPE_NAMES = {F32: "f32", BF16: "bf16", I8: "i8"}
+F32, BF16, I8, I4 = 0, 1, 2, 3
+_TORCH_DTYPE = {F32: torch.float32, BF16: torch.bfloat16, I8: torch.int8, I4: torch.uint8}
+DTYPE_NAMES = {F32: "f32", BF16: "bf16", I8: "i8", I4: "i4"}
+I4_GROUP = 128  # inputs per int4 scale group
 
 
 def build() -> str:
@@ -161,13 +168,26 @@ WORKLOADS = {
     "decode_int8_T1": Workload("decode_int8_T1", 1, 4096, 8, 2, 14336, act=BF16, wdt=I8),
     "decode_int8_T8": Workload("decode_int8_T8", 8, 4096, 8, 2, 14336, act=BF16, wdt=I8),
     "decode_int8_T32": Workload("decode_int8_T32", 32, 4096, 8, 2, 14336, act=BF16, wdt=I8),
+    # decode, int4 weights with one fp32 scale per output channel and group of 128 inputs
+    "decode_int4_T1": Workload("decode_int4_T1", 1, 4096, 8, 2, 14336, act=BF16, wdt=I4),
+    "decode_int4_T8": Workload("decode_int4_T8", 8, 4096, 8, 2, 14336, act=BF16, wdt=I4),
+    "decode_int4_T32": Workload("decode_int4_T32", 32, 4096, 8, 2, 14336, act=BF16, wdt=I4),
 }
 
 
-def expert_stride_elems(d: int, f: int) -> int:
-    """Elements between consecutive experts: 3*d*f rounded up to a multiple of 128."""
+def expert_stride_elems(d: int, f: int, wdt: int = BF16) -> int:
+    """Elements between consecutive experts: 3*d*f rounded up to a multiple of 128 (of 256 for
+    int4, so that every expert still starts on a 128-byte boundary)."""
     n = 3 * d * f
-    return (n + 127) // 128 * 128
+    m = 256 if wdt == I4 else 128
+    return (n + m - 1) // m * m
+
+
+def pack_int4(q: torch.Tensor) -> torch.Tensor:
+    """Pack int8 values in [-8, 7] two per byte: element 2j in the low nibble of byte j."""
+    assert q.dtype == torch.int8 and q.numel() % 2 == 0
+    u = (q.to(torch.int16) & 0xF).to(torch.uint8).view(-1, 2)
+    return (u[:, 0] | (u[:, 1] << 4)).contiguous()
 
 
 # tensor ids of the seeded streams
@@ -205,11 +225,15 @@ def make_problem(wl: Workload, seed: int = 0, pin: bool = False, expert_stride: 
 
     Distributions: x ~ N(0, 1); router W ~ N(0, 1/d); expert W ~ N(0, 1/d_in) with d_in = d for
     W1/W3 and f for W2 (bf16/fp32 weights); int8 weights uniform on [-127, 127] with scales
-    U(0.5, 1.5) / (127 sqrt(d_in)); router bias as the workload states (else none).
+    U(0.5, 1.5) / (127 sqrt(d_in)); int4 weights uniform on [-7, 7] with group scales
+    U(0.5, 1.5) / (7 sqrt(d_in)); router bias as the workload states (else none).
     """
     T, d, E, f, fs = wl.T, wl.d, wl.E, wl.f, wl.fs
     adt = _TORCH_DTYPE[wl.act]
-    stride = expert_stride if expert_stride is not None else expert_stride_elems(d, f)
+    stride = expert_stride if expert_stride is not None else expert_stride_elems(d, f, wl.wdt)
+    if wl.wdt == I4:
+        assert d % I4_GROUP == 0 and f % I4_GROUP == 0, "int4 weights need d and f multiples of 128"
+        assert stride % 2 == 0
     xt = make_x(wl, seed, pin) if x else None
     rw = _empty(E * d, adt, pin)
     fill_normal(rw, seed, TID_ROUTER_W, 1.0 / math.sqrt(d))
@@ -221,20 +245,34 @@ def make_problem(wl: Workload, seed: int = 0, pin: bool = False, expert_stride: 
         if pin:
             rb = rb.pin_memory()
     wdt = _TORCH_DTYPE[wl.wdt]
-    ew = _empty(E * stride, wdt, pin)
+    i4 = wl.wdt == I4
+    ew = _empty(E * stride // 2 if i4 else E * stride, wdt, pin)
     ew.zero_() if stride != 3 * d * f else None
     scales = _empty(E * (2 * f + d), torch.float32, pin) if wl.wdt == I8 else None
+    if i4:
+        scales = _empty(E * 3 * d * f // I4_GROUP, torch.float32, pin)
     for e in range(E):
         base = e * stride
         segs = ((0, f * d, d), (f * d, f * d, d), (2 * f * d, d * f, f))  # W1, W3, W2
         for m, (off, n, d_in) in enumerate(segs):
-            view = ew[base + off: base + off + n]
             tid = TID_EXPERT_BASE + 3 * e + m
+            if i4:
+                q = fill_int(torch.empty(n, dtype=torch.int8), seed, tid, -7, 7)
+                ew[(base + off) // 2: (base + off + n) // 2] = pack_int4(q)
+                continue
+            view = ew[base + off: base + off + n]
             if wl.wdt == I8:
                 fill_int(view, seed, tid, -127, 127)
             else:
                 fill_normal(view, seed, tid, 1.0 / math.sqrt(d_in))
-        if scales is not None:
+        if i4:
+            sbase = e * 3 * d * f // I4_GROUP
+            for m, (off, n, d_in) in enumerate(segs):
+                lo = 0.5 / (7.0 * math.sqrt(d_in))
+                hi = 1.5 / (7.0 * math.sqrt(d_in))
+                fill_uniform(scales[sbase + off // I4_GROUP: sbase + (off + n) // I4_GROUP], seed,
+                             TID_SCALE_BASE + 3 * e + m, lo, hi)
+        elif scales is not None:
             sbase = e * (2 * f + d)
             for m, (off, n, d_in) in enumerate(((0, f, d), (f, f, d), (2 * f, d, f))):
                 lo = 0.5 / (127.0 * math.sqrt(d_in))
@@ -242,7 +280,7 @@ def make_problem(wl: Workload, seed: int = 0, pin: bool = False, expert_stride: 
                 fill_uniform(scales[sbase + off: sbase + off + n], seed, TID_SCALE_BASE + 3 * e + m, lo, hi)
     sw = None
     if fs:
-        assert wl.wdt != I8, "shared expert is defined for bf16/fp32 weights"
+        assert wl.wdt not in (I8, I4), "shared expert is defined for bf16/fp32 weights"
         sw = _empty(3 * fs * d, wdt, pin)
         for m, (off, n, d_in) in enumerate(((0, fs * d, d), (fs * d, fs * d, d), (2 * fs * d, d * fs, fs))):
             fill_normal(sw[off: off + n], seed, TID_SHARED_BASE + m, 1.0 / math.sqrt(d_in))

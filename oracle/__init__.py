@@ -17,8 +17,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
-F32, BF16, I8 = 0, 1, 2
-_CODE = {torch.float32: F32, torch.bfloat16: BF16, torch.int8: I8}
+F32, BF16, I8, I4 = 0, 1, 2, 3
+# int4 weights travel as packed bytes (two elements per uint8)
+_CODE = {torch.float32: F32, torch.bfloat16: BF16, torch.int8: I8, torch.uint8: I4}
 
 
 def build() -> str:
@@ -46,8 +47,9 @@ def _load():
                                        i32, vp, i32, vp]
         lib.oracle_moe_forward.argtypes = [vp, i32, i32, i32, vp, vp, i32, i32, i32, vp, i32, i64, i32,
                                            vp, vp, i32] + [vp] * 8
+        lib.oracle_weight_element.argtypes = [vp, i32, i64, i64, i64, i64, vp, vp]
         for n in ("oracle_router_logits", "oracle_weights_for", "oracle_topk", "oracle_group",
-                  "oracle_expert_row", "oracle_combine", "oracle_moe_forward"):
+                  "oracle_expert_row", "oracle_combine", "oracle_moe_forward", "oracle_weight_element"):
             getattr(lib, n).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -155,6 +157,16 @@ def moe_forward(x, router_w, router_b, k, expert_w, stride, f, scales=None, shar
         *[_ptr(out[n]) for n in ("logits", "idx", "w", "counts", "offsets", "src_row", "dst_row", "y")])
     _check(rc, "moe_forward")
     return out
+
+
+def weight_element(w: torch.Tensor, base: int, cols: int, o: int, i: int,
+                   scale: Optional[torch.Tensor] = None) -> float:
+    """W[o][i] of the [rows, cols] matrix at element offset `base` of buffer `w` as the oracle
+    reads it (int8 / int4: dequantised with the matrix's scales)."""
+    out = ctypes.c_double()
+    _check(_load().oracle_weight_element(_ptr(w), _CODE[w.dtype], base, cols, o, i, _ptr(scale),
+                                         ctypes.byref(out)), "weight_element")
+    return out.value
 
 
 def problem_forward(p, tokens: Optional[Sequence[int]] = None, flags: int = 0):

@@ -6,8 +6,9 @@
 //
 // Arithmetic: inputs are widened exactly to double (float32 as is, bfloat16 by placing its
 // bits in the top half of a float32, int8 weights dequantised as the float32 product
-// s[o] * q[o][i]); every dot product and sum is accumulated in double in ascending index
-// order and rounded to float32 once.  Results are float32.
+// s[o] * q[o][i], int4 weights as the float32 product s[o][i / 128] * q[o][i]); every dot
+// product and sum is accumulated in double in ascending index order and rounded to float32
+// once.  Results are float32.
 //
 // The pages describing the method (the "Colibri" MoE engine) are cited by address and
 // section:
@@ -27,7 +28,13 @@
 //   * slot 0 holds the largest logit;
 //   * the expert FFN is SwiGLU: W2 (silu(W1 x) * (W3 x)), no biases;
 //   * within one expert, rows are in ascending token order;
-//   * the optional shared expert is a SwiGLU FFN added with weight 1.
+//   * the optional shared expert is a SwiGLU FFN added with weight 1;
+//   * int4 weights ([mhpq] §4.2: INT4 packed in INT32, group-wise quantisation with group size
+//     128; [trdm] §6.1: two 4-bit weights per byte, unpacked at compute time): element 2j of a
+//     row sits in the low nibble of byte j and element 2j + 1 in the high nibble (so the eight
+//     elements of a little-endian int32 run from its lowest nibble up), each a two's-complement
+//     value in [-8, 7]; symmetric, no zero point (the int8 quantiser of [0539edu] §3.1 has
+//     none); one fp32 scale per output row and group of 128 consecutive inputs.
 //
 // Parity pins: see tests/test_oracle_pins.py (brute force, closed forms, invariants).
 
@@ -39,7 +46,8 @@
 
 namespace {
 
-enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_I8 = 2 };
+enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_I8 = 2, ORC_I4 = 3 };
+constexpr int kI4Group = 128;  // inputs per int4 scale group
 enum { ORC_OK = 0, ORC_EARG = -1, ORC_ENONFINITE = -2 };
 // Router variants: clamp the logits to [-50, 50] ([0539edu] §5.2, the gate-softmax clip
 // option against overflow); use the chosen raw logits as the combine weights, no softmax
@@ -58,29 +66,52 @@ inline double widen(const void* p, int dtype, int64_t i) {
   return (double)((const int8_t*)p)[i];
 }
 
+// The signed 4-bit value stored at element index n of a packed int4 buffer.
+inline int int4_at(const void* w, int64_t n) {
+  const uint8_t byte = ((const uint8_t*)w)[n >> 1];
+  const int nib = (n & 1) ? (byte >> 4) : (byte & 0xF);
+  return nib >= 8 ? nib - 16 : nib;
+}
+
 // One weight matrix element W[o][i] of a [rows, cols] row-major matrix at element offset
 // `base` of the expert buffer.  For int8 storage the element is s[o] * q[o][i] rounded to
-// float32 ("per-output-channel fp32 scale, dequantised in the kernel").
+// float32 ("per-output-channel fp32 scale, dequantised in the kernel"); for int4 storage it is
+// s[o][i / 128] * q[o][i] with the matrix's scales [rows][cols / 128].
 inline double weight(const void* w, int wdt, int64_t base, int64_t cols, int64_t o, int64_t i,
                      const float* scale) {
   if (wdt == ORC_I8) {
     float deq = scale[o] * (float)((const int8_t*)w)[base + o * cols + i];
     return (double)deq;
   }
+  if (wdt == ORC_I4) {
+    float deq = scale[o * (cols / kI4Group) + i / kI4Group] * (float)int4_at(w, base + o * cols + i);
+    return (double)deq;
+  }
   return widen(w, wdt, base + o * cols + i);
 }
+
+// Scales of one expert: int8 [f | f | d] per output channel, int4 [f][d/128] | [f][d/128] |
+// [d][f/128] per output channel and input group.
+inline int64_t expert_scale_count(int wdt, int d, int f) {
+  if (wdt == ORC_I8) return 2 * (int64_t)f + d;
+  if (wdt == ORC_I4) return 3 * (int64_t)d * f / kI4Group;
+  return 0;
+}
+inline bool quantised(int wdt) { return wdt == ORC_I8 || wdt == ORC_I4; }
 
 // SwiGLU feed-forward of one input row through one expert whose three matrices start at
 // element `base` of buffer `w`: W1[f][d] (gate), W3[f][d] (up), W2[d][f] (down).
 // [hotelren] §2.1 (six steps: each chosen expert is an FFN applied to the token), SwiGLU form
-// as the workloads state.  `scales` (int8 only) holds [f | f | d] output-channel scales.
+// as the workloads state.  `scales` (int8 / int4 only) holds the expert's scales in the layout
+// of expert_scale_count.
 bool expert_ffn(const double* xrow, int d, int f, const void* w, int wdt, int64_t base,
                 const float* scales, float* yrow) {
   std::vector<float> h(f);
   const int64_t w1 = base, w3 = base + (int64_t)f * d, w2 = base + 2 * (int64_t)f * d;
+  const int64_t s3_off = wdt == ORC_I4 ? (int64_t)f * d / kI4Group : f;
   const float* s1 = scales ? scales : nullptr;
-  const float* s3 = scales ? scales + f : nullptr;
-  const float* s2 = scales ? scales + 2 * f : nullptr;
+  const float* s3 = scales ? scales + s3_off : nullptr;
+  const float* s2 = scales ? scales + 2 * s3_off : nullptr;
   for (int o = 0; o < f; ++o) {
     double g = 0.0, u = 0.0;
     for (int i = 0; i < d; ++i) {
@@ -206,7 +237,9 @@ int oracle_expert_row(const void* x, int act, int d, int t, const void* expert_w
                       int64_t stride, int f, const float* scales, int e, float* yrow) {
   std::vector<double> xr(d);
   for (int i = 0; i < d; ++i) xr[i] = widen(x, act, (int64_t)t * d + i);
-  const float* sc = (wdt == ORC_I8) ? scales + (int64_t)e * (2 * f + d) : nullptr;
+  if (quantised(wdt) && !scales) return ORC_EARG;
+  if (wdt == ORC_I4 && (d % kI4Group || f % kI4Group)) return ORC_EARG;
+  const float* sc = quantised(wdt) ? scales + (int64_t)e * expert_scale_count(wdt, d, f) : nullptr;
   return expert_ffn(xr.data(), d, f, expert_w, wdt, (int64_t)e * stride, sc, yrow) ? ORC_OK
                                                                                     : ORC_ENONFINITE;
 }
@@ -221,8 +254,9 @@ int oracle_combine(const void* x, int act, int T, int d, int k, const int32_t* i
                    const float* scales, const void* shared_w, int fs, const int32_t* tokens,
                    int ntok, float* y) {
   if (d <= 0 || k <= 0 || f <= 0 || ntok < 0) return ORC_EARG;
-  if (wdt == ORC_I8 && !scales) return ORC_EARG;
-  if (fs > 0 && (!shared_w || wdt == ORC_I8)) return ORC_EARG;
+  if (quantised(wdt) && !scales) return ORC_EARG;
+  if (wdt == ORC_I4 && (d % kI4Group || f % kI4Group)) return ORC_EARG;
+  if (fs > 0 && (!shared_w || quantised(wdt))) return ORC_EARG;
   std::vector<float> yp(d), ys(d);
   std::vector<double> xr(d);
   for (int n = 0; n < ntok; ++n) {
@@ -232,7 +266,7 @@ int oracle_combine(const void* x, int act, int T, int d, int k, const int32_t* i
     std::vector<double> acc(d, 0.0);
     for (int j = 0; j < k; ++j) {
       const int e = idx[(int64_t)t * k + j];
-      const float* sc = (wdt == ORC_I8) ? scales + (int64_t)e * (2 * f + d) : nullptr;
+      const float* sc = quantised(wdt) ? scales + (int64_t)e * expert_scale_count(wdt, d, f) : nullptr;
       if (!expert_ffn(xr.data(), d, f, expert_w, wdt, (int64_t)e * stride, sc, yp.data()))
         return ORC_ENONFINITE;
       const double wj = (double)w[(int64_t)t * k + j];
@@ -244,6 +278,18 @@ int oracle_combine(const void* x, int act, int T, int d, int k, const int32_t* i
     }
     for (int i = 0; i < d; ++i) y[(int64_t)n * d + i] = (float)acc[i];
   }
+  return ORC_OK;
+}
+
+// One dequantised weight element W[o][i] (as `weight` above) of the [rows, cols] matrix at
+// element offset `base`, with that matrix's scales; exposed so that tests can pin the storage
+// formats element by element.
+int oracle_weight_element(const void* w, int wdt, int64_t base, int64_t cols, int64_t o, int64_t i,
+                          const float* scale, double* out) {
+  if (!w || !out || cols <= 0 || o < 0 || i < 0 || i >= cols) return ORC_EARG;
+  if (quantised(wdt) && !scale) return ORC_EARG;
+  if (wdt == ORC_I4 && cols % kI4Group) return ORC_EARG;
+  *out = weight(w, wdt, base, cols, o, i, scale);
   return ORC_OK;
 }
 

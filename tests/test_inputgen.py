@@ -96,3 +96,21 @@ def test_int8_problem_scales():
     lo2, hi2 = 0.5 / (127 * math.sqrt(64)), 1.5 / (127 * math.sqrt(64))
     assert s[:, :128].min() >= lo1 and s[:, :128].max() <= hi1
     assert s[:, 128:].min() >= lo2 and s[:, 128:].max() <= hi2
+
+
+def test_int4_problem_packing_and_scales():
+    wl = inputgen.custom("i4", T=2, d=256, E=2, k=1, f=128, act=inputgen.BF16, wdt=inputgen.I4)
+    p = inputgen.make_problem(wl, seed=5)
+    assert p.expert_w.dtype == torch.uint8
+    assert p.expert_stride % 256 == 0 and p.expert_w.numel() == wl.E * p.expert_stride // 2
+    lo = (p.expert_w.to(torch.int16) & 0xF)
+    hi = (p.expert_w.to(torch.int16) >> 4)
+    for nib in (lo, hi):  # values in [-7, 7]: nibble 8 (-8) never occurs
+        assert not torch.any(nib == 8)
+    assert p.expert_scales.numel() == wl.E * 3 * wl.d * wl.f // 128
+    f, d = wl.f, wl.d
+    s = p.expert_scales.view(wl.E, -1)
+    s13 = s[:, : 2 * f * d // 128]
+    s2 = s[:, 2 * f * d // 128:]
+    assert torch.all(s13 > 0.5 / (7 * d ** 0.5) * 0.999) and torch.all(s13 < 1.5 / (7 * d ** 0.5) * 1.001)
+    assert torch.all(s2 > 0.5 / (7 * f ** 0.5) * 0.999) and torch.all(s2 < 1.5 / (7 * f ** 0.5) * 1.001)

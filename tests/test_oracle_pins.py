@@ -43,11 +43,33 @@ def _ref_select(logits, k):
     return out
 
 
-def _expert_mats(p, e):
-    """W1, W3, W2 of expert e as float64 numpy (int8 dequantised as float32 s*q)."""
+def _unpack_int4(packed: torch.Tensor) -> torch.Tensor:
+    """Packed bytes -> int8 elements (low nibble first), nibbles 8..15 read as -8..-1."""
+    b = packed.to(torch.int16)
+    q = torch.stack([b & 0xF, b >> 4], dim=-1).reshape(-1)
+    return torch.where(q >= 8, q - 16, q).to(torch.int8)
+
+
+def _int4_mats(p, e):
+    """W1, W3, W2 of an int4 expert dequantised as float32 s[o][i // 128] * q[o][i]."""
     wl = p.wl
     d, f = wl.d, wl.f
     base = e * p.expert_stride
+    q = _unpack_int4(p.expert_w[base // 2: (base + 3 * f * d) // 2]).to(torch.float32)
+    s = p.expert_scales[e * 3 * d * f // 128:(e + 1) * 3 * d * f // 128]
+    s1 = s[: f * d // 128].view(f, d // 128).repeat_interleave(128, dim=1)
+    s3 = s[f * d // 128: 2 * f * d // 128].view(f, d // 128).repeat_interleave(128, dim=1)
+    s2 = s[2 * f * d // 128:].view(d, f // 128).repeat_interleave(128, dim=1)
+    return (s1 * q[: f * d].view(f, d), s3 * q[f * d: 2 * f * d].view(f, d), s2 * q[2 * f * d:].view(d, f))
+
+
+def _expert_mats(p, e):
+    """W1, W3, W2 of expert e as float64 numpy (int8 / int4 dequantised as float32 s*q)."""
+    wl = p.wl
+    d, f = wl.d, wl.f
+    base = e * p.expert_stride
+    if wl.wdt == inputgen.I4:
+        return tuple(_f64(m) for m in _int4_mats(p, e))
     raw = p.expert_w[base: base + 3 * f * d]
     if wl.wdt == inputgen.I8:
         s = p.expert_scales[e * (2 * f + d):(e + 1) * (2 * f + d)]
@@ -297,7 +319,7 @@ def test_single_expert_is_dense_swiglu(act):
 
 
 @pytest.mark.parametrize("case", ["f32", "bf16", "bf16_shared", "bf16_bias", "i8", "bf16_clamp", "f32_raw",
-                                  "i8_clamp_raw"])
+                                  "i8_clamp_raw", "i4"])
 def test_layer_equals_brute_force_dense(case):
     kw = dict(T=23, d=64, E=6, k=2, f=96)
     flags = 0
@@ -319,6 +341,8 @@ def test_layer_equals_brute_force_dense(case):
         wl = inputgen.custom(case, fs=40, **dict(kw, k=3))
     elif case == "bf16_bias":
         wl = inputgen.custom(case, bias=((1, 2.0), (4, -1.0)), **kw)
+    elif case == "i4":  # int4 needs d and f multiples of the 128-wide scale group
+        wl = inputgen.custom(case, act=inputgen.BF16, wdt=inputgen.I4, **dict(kw, d=256, f=128))
     else:
         wl = inputgen.custom(case, act=inputgen.BF16, wdt=inputgen.I8, **kw)
     p = inputgen.make_problem(wl, seed=3)
@@ -353,6 +377,64 @@ def test_int8_dequant_identity():
     a = oracle.moe_forward(p.x, p.router_w, None, 2, p.expert_w, p.expert_stride, f, p.expert_scales)
     b = oracle.moe_forward(p.x, p.router_w, None, 2, deq, p.expert_stride, f)
     assert torch.equal(a["y"], b["y"])
+
+
+def _golden_int4():
+    rows = []
+    with open(os.path.join(GOLDEN, "int4_packing.txt")) as fh:
+        for line in fh:
+            line = line.split("#")[0].strip()
+            if line:
+                word, *vals = line.split()
+                rows.append((int(word, 16), [int(v) for v in vals]))
+    return rows
+
+
+def test_int4_packing_golden():
+    # the hand-worked words of tests/golden/int4_packing.txt, read back element by element by the
+    # oracle (one 128-element row, unit scale), and written by the generator's packer
+    rows = _golden_int4()
+    assert len(rows) >= 4
+    for word, vals in rows:
+        buf = torch.zeros(64, dtype=torch.uint8)
+        buf[:4] = torch.tensor(list(word.to_bytes(4, "little")), dtype=torch.uint8)
+        one = torch.ones(1, dtype=torch.float32)
+        got = [oracle.weight_element(buf, 0, 128, 0, i, one) for i in range(8)]
+        assert got == [float(v) for v in vals], hex(word)
+        assert all(oracle.weight_element(buf, 0, 128, 0, i, one) == 0.0 for i in range(8, 128))
+        packed = inputgen.pack_int4(torch.tensor(vals, dtype=torch.int8))
+        assert packed.tolist() == list(word.to_bytes(4, "little")), hex(word)
+        assert _unpack_int4(packed).tolist() == vals
+
+
+def test_int4_group_scales_apply_per_128_inputs():
+    # W[o][i] = s[o][i // 128] * q[o][i]: distinct scales per (row, group) show which one applies
+    rows, cols = 3, 384
+    q = torch.tensor([((o * 7 + i) % 15) - 7 for o in range(rows) for i in range(cols)], dtype=torch.int8)
+    buf = inputgen.pack_int4(q)
+    s = torch.tensor([2.0 ** -(o * 3 + g) for o in range(rows) for g in range(cols // 128)], dtype=torch.float32)
+    for o in range(rows):
+        for i in (0, 1, 127, 128, 255, 256, 383):
+            want = float(q[o * cols + i]) * 2.0 ** -(o * 3 + i // 128)
+            assert oracle.weight_element(buf, 0, cols, o, i, s) == want
+    # an offset base (the second matrix of an expert) shifts the element index, not the scales
+    assert oracle.weight_element(buf, cols, cols, 1, 5, s) == float(q[2 * cols + 5]) * 2.0 ** -(3 + 0)
+
+
+def test_int4_dequant_identity():
+    # the oracle on (s, q) equals the oracle on float32 weights s[o][i // 128] * q[o][i]
+    wl = inputgen.custom("i4", T=7, d=256, E=3, k=2, f=256, act=inputgen.BF16, wdt=inputgen.I4)
+    p = inputgen.make_problem(wl, seed=6)
+    f, d = wl.f, wl.d
+    deq = torch.zeros(3 * p.expert_stride, dtype=torch.float32)
+    for e in range(3):
+        w1, w3, w2 = _int4_mats(p, e)
+        deq[e * p.expert_stride: e * p.expert_stride + 3 * f * d] = torch.cat([w1.reshape(-1), w3.reshape(-1),
+                                                                             w2.reshape(-1)])
+    a = oracle.moe_forward(p.x, p.router_w, None, 2, p.expert_w, p.expert_stride, f, p.expert_scales)
+    b = oracle.moe_forward(p.x, p.router_w, None, 2, deq, p.expert_stride, f)
+    assert torch.equal(a["y"], b["y"])
+    assert torch.equal(a["idx"], b["idx"])
 
 
 def test_tiny_f32_workload_float64_restatement():
