@@ -12,8 +12,8 @@ the C ABI expects:
 * ``expert_w``   one buffer; expert e starts at element ``e * expert_stride`` and
                  holds W1[f, d] | W3[f, d] | W2[d, f] (rows are [out, in])
 * ``expert_scales`` int8 weights: per expert [f | f | d] float32 (one per output channel);
-                 int4 weights: per expert s1[f, d/128] | s3[f, d/128] | s2[d, f/128] float32
-                 (one per output channel and group of 128 consecutive inputs)
+                 int4 weights: per expert s1[d/128, f] | s3[d/128, f] | s2[f/128, d] float32
+                 (one per group of 128 consecutive inputs and output channel, group-major)
 * ``shared_w``   W1s[fs, d] | W3s[fs, d] | W2s[d, fs] or None
 
 int4 weights are stored packed, two per byte along the input dimension: element 2j of a row in

@@ -47,7 +47,7 @@ def _load():
                                        i32, vp, i32, vp]
         lib.oracle_moe_forward.argtypes = [vp, i32, i32, i32, vp, vp, i32, i32, i32, vp, i32, i64, i32,
                                            vp, vp, i32] + [vp] * 8
-        lib.oracle_weight_element.argtypes = [vp, i32, i64, i64, i64, i64, vp, vp]
+        lib.oracle_weight_element.argtypes = [vp, i32, i64, i64, i64, i64, i64, vp, vp]
         for n in ("oracle_router_logits", "oracle_weights_for", "oracle_topk", "oracle_group",
                   "oracle_expert_row", "oracle_combine", "oracle_moe_forward", "oracle_weight_element"):
             getattr(lib, n).restype = ctypes.c_int
@@ -159,12 +159,12 @@ def moe_forward(x, router_w, router_b, k, expert_w, stride, f, scales=None, shar
     return out
 
 
-def weight_element(w: torch.Tensor, base: int, cols: int, o: int, i: int,
+def weight_element(w: torch.Tensor, base: int, rows: int, cols: int, o: int, i: int,
                    scale: Optional[torch.Tensor] = None) -> float:
     """W[o][i] of the [rows, cols] matrix at element offset `base` of buffer `w` as the oracle
     reads it (int8 / int4: dequantised with the matrix's scales)."""
     out = ctypes.c_double()
-    _check(_load().oracle_weight_element(_ptr(w), _CODE[w.dtype], base, cols, o, i, _ptr(scale),
+    _check(_load().oracle_weight_element(_ptr(w), _CODE[w.dtype], base, rows, cols, o, i, _ptr(scale),
                                          ctypes.byref(out)), "weight_element")
     return out.value
 

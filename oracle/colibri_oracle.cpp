@@ -34,7 +34,9 @@
 //     row sits in the low nibble of byte j and element 2j + 1 in the high nibble (so the eight
 //     elements of a little-endian int32 run from its lowest nibble up), each a two's-complement
 //     value in [-8, 7]; symmetric, no zero point (the int8 quantiser of [0539edu] §3.1 has
-//     none); one fp32 scale per output row and group of 128 consecutive inputs.
+//     none); one fp32 scale per output row and group of 128 consecutive inputs, stored
+//     group-major ([cols / 128][rows] per matrix: the scales of one group's rows are adjacent;
+//     the pages do not fix this layout).
 //
 // Parity pins: see tests/test_oracle_pins.py (brute force, closed forms, invariants).
 
@@ -76,22 +78,22 @@ inline int int4_at(const void* w, int64_t n) {
 // One weight matrix element W[o][i] of a [rows, cols] row-major matrix at element offset
 // `base` of the expert buffer.  For int8 storage the element is s[o] * q[o][i] rounded to
 // float32 ("per-output-channel fp32 scale, dequantised in the kernel"); for int4 storage it is
-// s[o][i / 128] * q[o][i] with the matrix's scales [rows][cols / 128].
-inline double weight(const void* w, int wdt, int64_t base, int64_t cols, int64_t o, int64_t i,
+// s[i / 128][o] * q[o][i] with the matrix's scales [cols / 128][rows].
+inline double weight(const void* w, int wdt, int64_t base, int64_t rows, int64_t cols, int64_t o, int64_t i,
                      const float* scale) {
   if (wdt == ORC_I8) {
     float deq = scale[o] * (float)((const int8_t*)w)[base + o * cols + i];
     return (double)deq;
   }
   if (wdt == ORC_I4) {
-    float deq = scale[o * (cols / kI4Group) + i / kI4Group] * (float)int4_at(w, base + o * cols + i);
+    float deq = scale[(i / kI4Group) * rows + o] * (float)int4_at(w, base + o * cols + i);
     return (double)deq;
   }
   return widen(w, wdt, base + o * cols + i);
 }
 
-// Scales of one expert: int8 [f | f | d] per output channel, int4 [f][d/128] | [f][d/128] |
-// [d][f/128] per output channel and input group.
+// Scales of one expert: int8 [f | f | d] per output channel, int4 [d/128][f] | [d/128][f] |
+// [f/128][d] per input group and output channel.
 inline int64_t expert_scale_count(int wdt, int d, int f) {
   if (wdt == ORC_I8) return 2 * (int64_t)f + d;
   if (wdt == ORC_I4) return 3 * (int64_t)d * f / kI4Group;
@@ -115,8 +117,8 @@ bool expert_ffn(const double* xrow, int d, int f, const void* w, int wdt, int64_
   for (int o = 0; o < f; ++o) {
     double g = 0.0, u = 0.0;
     for (int i = 0; i < d; ++i) {
-      g += weight(w, wdt, w1, d, o, i, s1) * xrow[i];
-      u += weight(w, wdt, w3, d, o, i, s3) * xrow[i];
+      g += weight(w, wdt, w1, f, d, o, i, s1) * xrow[i];
+      u += weight(w, wdt, w3, f, d, o, i, s3) * xrow[i];
     }
     const double gf = (double)(float)g, uf = (double)(float)u;
     const double hv = gf / (1.0 + std::exp(-gf)) * uf;  // silu(g) * u
@@ -125,7 +127,7 @@ bool expert_ffn(const double* xrow, int d, int f, const void* w, int wdt, int64_
   }
   for (int o = 0; o < d; ++o) {
     double acc = 0.0;
-    for (int i = 0; i < f; ++i) acc += weight(w, wdt, w2, f, o, i, s2) * (double)h[i];
+    for (int i = 0; i < f; ++i) acc += weight(w, wdt, w2, d, f, o, i, s2) * (double)h[i];
     yrow[o] = (float)acc;
     if (!std::isfinite(yrow[o])) return false;
   }
@@ -284,12 +286,12 @@ int oracle_combine(const void* x, int act, int T, int d, int k, const int32_t* i
 // One dequantised weight element W[o][i] (as `weight` above) of the [rows, cols] matrix at
 // element offset `base`, with that matrix's scales; exposed so that tests can pin the storage
 // formats element by element.
-int oracle_weight_element(const void* w, int wdt, int64_t base, int64_t cols, int64_t o, int64_t i,
+int oracle_weight_element(const void* w, int wdt, int64_t base, int64_t rows, int64_t cols, int64_t o, int64_t i,
                           const float* scale, double* out) {
-  if (!w || !out || cols <= 0 || o < 0 || i < 0 || i >= cols) return ORC_EARG;
+  if (!w || !out || rows <= 0 || cols <= 0 || o < 0 || o >= rows || i < 0 || i >= cols) return ORC_EARG;
   if (quantised(wdt) && !scale) return ORC_EARG;
   if (wdt == ORC_I4 && cols % kI4Group) return ORC_EARG;
-  *out = weight(w, wdt, base, cols, o, i, scale);
+  *out = weight(w, wdt, base, rows, cols, o, i, scale);
   return ORC_OK;
 }
 

@@ -57,9 +57,10 @@ def _int4_mats(p, e):
     base = e * p.expert_stride
     q = _unpack_int4(p.expert_w[base // 2: (base + 3 * f * d) // 2]).to(torch.float32)
     s = p.expert_scales[e * 3 * d * f // 128:(e + 1) * 3 * d * f // 128]
-    s1 = s[: f * d // 128].view(f, d // 128).repeat_interleave(128, dim=1)
-    s3 = s[f * d // 128: 2 * f * d // 128].view(f, d // 128).repeat_interleave(128, dim=1)
-    s2 = s[2 * f * d // 128:].view(d, f // 128).repeat_interleave(128, dim=1)
+    # group-major scales: [inputs / 128][outputs] per matrix
+    s1 = s[: f * d // 128].view(d // 128, f).t().repeat_interleave(128, dim=1)
+    s3 = s[f * d // 128: 2 * f * d // 128].view(d // 128, f).t().repeat_interleave(128, dim=1)
+    s2 = s[2 * f * d // 128:].view(f // 128, d).t().repeat_interleave(128, dim=1)
     return (s1 * q[: f * d].view(f, d), s3 * q[f * d: 2 * f * d].view(f, d), s2 * q[2 * f * d:].view(d, f))
 
 
@@ -399,26 +400,27 @@ def test_int4_packing_golden():
         buf = torch.zeros(64, dtype=torch.uint8)
         buf[:4] = torch.tensor(list(word.to_bytes(4, "little")), dtype=torch.uint8)
         one = torch.ones(1, dtype=torch.float32)
-        got = [oracle.weight_element(buf, 0, 128, 0, i, one) for i in range(8)]
+        got = [oracle.weight_element(buf, 0, 1, 128, 0, i, one) for i in range(8)]
         assert got == [float(v) for v in vals], hex(word)
-        assert all(oracle.weight_element(buf, 0, 128, 0, i, one) == 0.0 for i in range(8, 128))
+        assert all(oracle.weight_element(buf, 0, 1, 128, 0, i, one) == 0.0 for i in range(8, 128))
         packed = inputgen.pack_int4(torch.tensor(vals, dtype=torch.int8))
         assert packed.tolist() == list(word.to_bytes(4, "little")), hex(word)
         assert _unpack_int4(packed).tolist() == vals
 
 
 def test_int4_group_scales_apply_per_128_inputs():
-    # W[o][i] = s[o][i // 128] * q[o][i]: distinct scales per (row, group) show which one applies
+    # W[o][i] = s[i // 128][o] * q[o][i] (group-major scales): distinct power-of-two scales per
+    # (group, row) show which one applies
     rows, cols = 3, 384
     q = torch.tensor([((o * 7 + i) % 15) - 7 for o in range(rows) for i in range(cols)], dtype=torch.int8)
     buf = inputgen.pack_int4(q)
-    s = torch.tensor([2.0 ** -(o * 3 + g) for o in range(rows) for g in range(cols // 128)], dtype=torch.float32)
+    s = torch.tensor([2.0 ** -(o * 3 + g) for g in range(cols // 128) for o in range(rows)], dtype=torch.float32)
     for o in range(rows):
         for i in (0, 1, 127, 128, 255, 256, 383):
             want = float(q[o * cols + i]) * 2.0 ** -(o * 3 + i // 128)
-            assert oracle.weight_element(buf, 0, cols, o, i, s) == want
+            assert oracle.weight_element(buf, 0, rows, cols, o, i, s) == want
     # an offset base (the second matrix of an expert) shifts the element index, not the scales
-    assert oracle.weight_element(buf, cols, cols, 1, 5, s) == float(q[2 * cols + 5]) * 2.0 ** -(3 + 0)
+    assert oracle.weight_element(buf, cols, 2, cols, 1, 5, s[:2]) == float(q[2 * cols + 5]) * 2.0 ** -(3 + 0)
 
 
 def test_int4_dequant_identity():
