@@ -49,7 +49,7 @@ typedef enum {
   COLIBRI_ERR_TIMEOUT = -6      /* a device-side wait gave up (reported by colibri_sync_status) */
 } colibri_status;
 
-typedef enum { COLIBRI_F32 = 0, COLIBRI_BF16 = 1, COLIBRI_I8 = 2 } colibri_dtype;
+typedef enum { COLIBRI_F32 = 0, COLIBRI_BF16 = 1, COLIBRI_I8 = 2, COLIBRI_I4 = 3 } colibri_dtype;
 
 /* Layout of the int8 weight scales (colibri_desc.weight_scale_mode). */
 typedef enum {
@@ -83,6 +83,11 @@ typedef enum {
  *                   (BF16, BF16) bf16 operands, fp32 accumulation on tcgen05 tensor cores;
  *                   (BF16, I8)   int8 weights with per-output-channel fp32 scales,
  *                                dequantised inside the kernel (weight-streaming path).
+ *                   (BF16, I4)   int4 weights, two per byte along the input dimension, with
+ *                                one fp32 scale per output channel and group of 128 inputs
+ *                                (www.mhpq.cn/news/563172 §4.2: INT4 packed in INT32, group
+ *                                size 128; www.trdm.cn/news/555962 §6.1: two 4-bit weights per
+ *                                byte); d_model and d_ff multiples of 128.
  *                   The shared expert is available for (F32, F32) and (BF16, BF16).
  *   max_tokens      largest T a forward may be called with (sizes the workspace).
  *   device_id       CUDA device the context lives on.
@@ -122,8 +127,8 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out);
 
 /*
  * colibri_expert_stride -- elements between the starts of consecutive experts in the expert
- * weight buffer: 3 * d_model * d_ff rounded up to a multiple of 128 (so every expert starts
- * at least 128-byte aligned).  (www.mhpq.cn/news/563172 §2.1: each expert occupies a fixed
+ * weight buffer: 3 * d_model * d_ff rounded up to a multiple of 128 (of 256 for int4, whose
+ * elements are half a byte), so every expert starts at least 128-byte aligned.  (www.mhpq.cn/news/563172 §2.1: each expert occupies a fixed
  * stride, address = id * EXPERT_SIZE.)  Returns -1 for a NULL context.
  */
 int64_t colibri_expert_stride(const colibri_ctx* ctx);
@@ -139,9 +144,14 @@ int64_t colibri_expert_stride(const colibri_ctx* ctx);
  *   expert_w     device; expert e starts at element e * colibri_expert_stride(ctx) and holds
  *                W1[f][d] | W3[f][d] | W2[d][f], each row-major with rows = output channels
  *                ([out, in]).  W1 is the gate, W3 the up and W2 the down projection.
- *   expert_scales  COLIBRI_I8 only: device fp32, per expert e at e * (2f + d): s1[f] | s3[f] |
+ *   expert_scales  COLIBRI_I8: device fp32, per expert e at e * (2f + d): s1[f] | s3[f] |
  *                s2[d]; weight W[o][i] = s[o] * q[o][i] (with COLIBRI_SCALE_PER_MATRIX: at 3 * e,
- *                s1 | s3 | s2, W[o][i] = s * q[o][i]).  Must be NULL otherwise.
+ *                s1 | s3 | s2, W[o][i] = s * q[o][i]).
+ *                COLIBRI_I4: device fp32, per expert e at e * 3 * d * f / 128: s1[d/128][f] |
+ *                s3[d/128][f] | s2[f/128][d] (group-major); W[o][i] = s[i / 128][o] * q[o][i],
+ *                where q[o][i] is the two's-complement nibble of element o * cols + i of the
+ *                matrix (element 2j of the buffer in the low nibble of byte j, 2j + 1 in the high
+ *                nibble; expert e starts at byte e * stride / 2).  Must be NULL for F32 / BF16.
  *   shared_w     device, W1s[f_s][d] | W3s[f_s][d] | W2s[d][f_s] in weight_dtype, when
  *                shared_d_ff > 0; must be NULL otherwise.
  *   y            [T, d_model] act_dtype, device or host; fully overwritten.  Host y is written
@@ -150,8 +160,8 @@ int64_t colibri_expert_stride(const colibri_ctx* ctx);
  *   stream       cudaStream_t.
  * Every device pointer must be 16-byte aligned.  Errors: INVALID_ARG, ALIGNMENT, CUDA.
  * A device-side wait that gives up is reported later by colibri_sync_status().
- * When x and y are device memory, `stream` is not the legacy default stream, no profiling is
- * active and the stream is not itself being captured, the launch sequence is captured into a
+ * When x and y are device memory, `stream` is not the legacy default stream, COLIBRI_PROFILE
+ * printing is off and the stream is not itself being captured, the launch sequence is captured into a
  * CUDA graph the first time a given argument set is seen and replayed on later calls with the
  * same arguments (up to 8 argument sets per context; COLIBRI_GRAPHS=0 disables this).
  * With COLIBRI_PROFILE=1 in the environment the call records CUDA events per stage,
@@ -180,7 +190,9 @@ colibri_status colibri_moe_forward_routed(colibri_ctx* ctx, const void* x, int32
 
 /*
  * colibri_get_routing -- enqueue device-to-device copies of the routing state of the last
- * forward on this context into caller buffers (any pointer may be NULL to skip it):
+ * forward on this context into caller buffers (any pointer may be NULL to skip it).  The pages
+ * have no counterpart of this call: it exposes the Gate and Scatter results (whose layouts follow
+ * www.pptc.cn/news/100465 §3.3-§3.4 and www.trdm.cn/news/555962 §6.2) for parity checks.
  *   topk_idx [T, k] int32   chosen experts, slot 0 = largest logit
  *   topk_w   [T, k] fp32    renormalised softmax weights
  *   counts   [E]    int32   rows per expert
@@ -205,7 +217,9 @@ colibri_status colibri_sync_status(colibri_ctx* ctx, void* stream);
  * Per-stage timing (www.0539edu.com/news/4774449 §3.3: enable_profiling reports the time of
  * each stage).  Between colibri_profile_begin and colibri_profile_end every forward on this
  * context records CUDA events on its own stream at the stage boundaries, without
- * synchronising.  colibri_profile_end synchronises those events and writes, per stage, the
+ * synchronising.  A forward that would replay a CUDA graph still does: a second graph of the
+ * same call carries event-record nodes at the stage boundaries (no programmatic dependent
+ * launch across them), so what is timed is the replayed launch sequence.  colibri_profile_end synchronises those events and writes, per stage, the
  * total milliseconds over the recorded calls:
  *   stage_ms[0] Gate (router logits, softmax, top-k)
  *   stage_ms[1] Scatter (histogram, prefix sum, permutation)
@@ -218,6 +232,15 @@ colibri_status colibri_sync_status(colibri_ctx* ctx, void* stream);
 #define COLIBRI_NUM_STAGES 5
 colibri_status colibri_profile_begin(colibri_ctx* ctx, int32_t max_calls);
 colibri_status colibri_profile_end(colibri_ctx* ctx, float* stage_ms, int32_t* ncalls);
+
+/*
+ * colibri_profile_calls -- after colibri_profile_end, the per-call stage times of the recorded
+ * calls (same stage order, same passage as above): call_stage_ms [n][COLIBRI_NUM_STAGES] host
+ * fp32 milliseconds, caller-owned, for the first n = min(max_calls, recorded calls) calls.
+ * The events stay valid until the next colibri_profile_begin.  Blocking (synchronises those
+ * events).  Errors: INVALID_ARG (NULL ctx or buffer, profiling still active), CUDA.
+ */
+colibri_status colibri_profile_calls(colibri_ctx* ctx, float* call_stage_ms, int32_t max_calls);
 
 /*
  * colibri_route_noalloc -- the Gate and Scatter stages alone (router logits, fp32 softmax,
@@ -236,15 +259,26 @@ colibri_status colibri_profile_end(colibri_ctx* ctx, float* stage_ms, int32_t* n
  * ceil(T / 256) * E <= 32768 (the size of the built-in scratch array); larger sizes are
  * rejected with COLIBRI_ERR_INVALID_ARG before anything is launched.  T == 0 launches nothing.
  * The scratch is one file-scope device array (about 257 KB, held by every GPU that loads the
- * library until exit).  The first call on each device looks up its address and should come
- * before any stream capture.  All calls share the array: calls that overlap on the GPU race.
- * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED, CUDA; reason via colibri_last_error(NULL).
+ * library until exit).  Each call looks up its device address on the current device and sets the
+ * router kernels' shared-memory limit there; the first call on each device loads the kernels and
+ * should come before any stream capture.  All calls share the array: calls that overlap on the GPU race.
+ * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED, CUDA; reason via colibri_last_error(NULL).  A
+ * device-side wait that gives up is reported by colibri_route_noalloc_check.
  */
 colibri_status colibri_route_noalloc(const void* x, int32_t act_dtype, int32_t T, int32_t d_model,
                                      const void* router_w, const float* router_b,
                                      int32_t num_experts, int32_t top_k, int32_t* topk_idx,
                                      float* topk_w, int32_t* counts, int32_t* offsets,
                                      int32_t* src_row, int32_t* dst_row, void* Xp, void* stream);
+
+/*
+ * colibri_route_noalloc_check -- synchronise `stream` and report whether a bounded device wait
+ * of the last colibri_route_noalloc call on the current device gave up (COLIBRI_ERR_TIMEOUT; its
+ * outputs are then undefined).  No counterpart on the pages (see colibri_route_noalloc).  The
+ * word lives in the same scratch array and is cleared by the next colibri_route_noalloc call.
+ * Blocking; allocates nothing.  Errors: TIMEOUT, CUDA.
+ */
+colibri_status colibri_route_noalloc_check(void* stream);
 
 /*
  * Failure-detection self test (no counterpart on the pages; it exercises the error reporting of
@@ -257,14 +291,16 @@ colibri_status colibri_route_noalloc(const void* x, int32_t act_dtype, int32_t T
  */
 colibri_status colibri_selftest_wait_timeout(colibri_ctx* ctx, int32_t timeout_us, void* stream);
 
-/* One-line description of a status code (static storage). */
+/* One-line description of a status code (static storage).  No counterpart on the pages; the
+ * codes are those of colibri_status above. */
 const char* colibri_status_string(colibri_status status);
 
 /* One-line reason for the last failure on this context, or on any context if ctx is NULL
  * (www.mhpq.cn/news/563172 §4.3 colibri_get_error).  Valid until the next call. */
 const char* colibri_last_error(const colibri_ctx* ctx);
 
-/* Release the workspace and the context.  Blocking (synchronises the device's work that
+/* colibri_free -- release the workspace and the context (www.hotelren.com/news/4731937 §2.3,
+ * §4.3: the free step of init / infer / free).  Blocking (synchronises the device's work that
  * uses the workspace).  NULL is ignored. */
 void colibri_free(colibri_ctx* ctx);
 

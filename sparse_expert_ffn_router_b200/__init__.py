@@ -16,7 +16,7 @@ from typing import Optional
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libcolibri.so")
 
-COLIBRI_F32, COLIBRI_BF16, COLIBRI_I8 = 0, 1, 2
+COLIBRI_F32, COLIBRI_BF16, COLIBRI_I8, COLIBRI_I4 = 0, 1, 2, 3
 COLIBRI_ROUTER_CLAMP, COLIBRI_ROUTER_RAW_WEIGHTS = 1, 2
 COLIBRI_SCALE_PER_CHANNEL, COLIBRI_SCALE_PER_MATRIX = 0, 1
 
@@ -40,7 +40,9 @@ EXPORTS = (
     "colibri_sync_status",
     "colibri_profile_begin",
     "colibri_profile_end",
+    "colibri_profile_calls",
     "colibri_route_noalloc",
+    "colibri_route_noalloc_check",
     "colibri_selftest_wait_timeout",
     "colibri_status_string",
     "colibri_last_error",
@@ -99,8 +101,12 @@ def load() -> ctypes.CDLL:
     lib.colibri_profile_begin.restype = ctypes.c_int
     lib.colibri_profile_end.argtypes = [vp, vp, vp]
     lib.colibri_profile_end.restype = ctypes.c_int
+    lib.colibri_profile_calls.argtypes = [vp, vp, i32]
+    lib.colibri_profile_calls.restype = ctypes.c_int
     lib.colibri_route_noalloc.argtypes = [vp, i32, i32, i32, vp, vp, i32, i32] + [vp] * 8
     lib.colibri_route_noalloc.restype = ctypes.c_int
+    lib.colibri_route_noalloc_check.argtypes = [vp]
+    lib.colibri_route_noalloc_check.restype = ctypes.c_int
     lib.colibri_selftest_wait_timeout.argtypes = [vp, i32, vp]
     lib.colibri_selftest_wait_timeout.restype = ctypes.c_int
     lib.colibri_status_string.argtypes = [ctypes.c_int]
@@ -205,6 +211,14 @@ def colibri_profile_end(ctx: int):
     return dict(zip(STAGE_NAMES, [float(v) for v in ms])), int(n.value)
 
 
+def colibri_profile_calls(ctx: int, ncalls: int):
+    """Per-call stage milliseconds of the last profiling region: a list of dicts."""
+    buf = (ctypes.c_float * (NUM_STAGES * max(ncalls, 1)))()
+    _check(load().colibri_profile_calls(ctx, buf, ncalls), "colibri_profile_calls", ctx)
+    return [dict(zip(STAGE_NAMES, [float(buf[c * NUM_STAGES + i]) for i in range(NUM_STAGES)]))
+            for c in range(ncalls)]
+
+
 def colibri_route_noalloc(x, act_dtype: int, T: int, d_model: int, router_w, router_b, num_experts: int,
                           top_k: int, topk_idx, topk_w, counts, offsets, src_row, dst_row, Xp, stream=None) -> None:
     """Gate + Scatter without a context or any device allocation (see include/colibri.h)."""
@@ -213,6 +227,11 @@ def colibri_route_noalloc(x, act_dtype: int, T: int, d_model: int, router_w, rou
                                         _addr(offsets), _addr(src_row), _addr(dst_row), _addr(Xp),
                                         _stream(stream)),
            "colibri_route_noalloc")
+
+
+def colibri_route_noalloc_check(stream=None) -> None:
+    """Raises ColibriError(TIMEOUT) if a device wait of the last colibri_route_noalloc gave up."""
+    _check(load().colibri_route_noalloc_check(_stream(stream)), "colibri_route_noalloc_check")
 
 
 def colibri_free(ctx: int) -> None:

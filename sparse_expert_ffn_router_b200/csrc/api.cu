@@ -82,17 +82,14 @@ int pick_dec_split(int f) {
 }
 
 // Tile shape of the bf16 expert GEMMs: 0 = one CTA, 128 rows x 256 columns; 1 = pairs of CTAs
-// (cta_group::2), 256 x 256; 2 = swapped operands, 128 channels x 16..256 rows.  Pair tiles when
-// experts average >= 512 rows (the halved L2 traffic outweighs the larger last tile of each
-// expert), else one-CTA tiles.  The swapped tiles pad fewer rows but measured slower on every
-// workload, so they are only used on request.
-// COLIBRI_GEMM_CTA=1, 2 or s forces a mode (all are exact; this only selects the tiling).
-enum GemmMode { kGemmOne = 0, kGemmPair = 1, kGemmSwap = 2 };
+// (cta_group::2), 256 x 256.  Pair tiles when experts average >= 512 rows (the halved L2 traffic
+// outweighs the larger last tile of each expert), else one-CTA tiles.
+// COLIBRI_GEMM_CTA=1 or 2 forces a mode (both are exact; this only selects the tiling).
+enum GemmMode { kGemmOne = 0, kGemmPair = 1 };
 int gemm_mode(int avg_rows_per_expert) {
   const char* v = getenv("COLIBRI_GEMM_CTA");
   if (v && v[0] == '1') return kGemmOne;
   if (v && v[0] == '2') return kGemmPair;
-  if (v && v[0] == 's') return kGemmSwap;
   return avg_rows_per_expert >= 512 ? kGemmPair : kGemmOne;
 }
 
@@ -167,16 +164,20 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
     return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "max_tokens * top_k too large");
   const bool f32 = D.act_dtype == COLIBRI_F32 && D.weight_dtype == COLIBRI_F32;
   const bool bf16 = D.act_dtype == COLIBRI_BF16 && D.weight_dtype == COLIBRI_BF16;
-  const bool i8 = D.act_dtype == COLIBRI_BF16 && D.weight_dtype == COLIBRI_I8;
-  if (D.act_dtype < 0 || D.act_dtype > 2 || D.weight_dtype < 0 || D.weight_dtype > 2)
+  const bool w8 = D.act_dtype == COLIBRI_BF16 && D.weight_dtype == COLIBRI_I8;
+  const bool w4 = D.act_dtype == COLIBRI_BF16 && D.weight_dtype == COLIBRI_I4;
+  const bool i8 = w8 || w4;  // the weight-streaming path (int8 tensor cores over activation planes)
+  if (D.act_dtype < 0 || D.act_dtype > 2 || D.weight_dtype < 0 || D.weight_dtype > 3)
     return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "unknown dtype code (act=%d, weight=%d)", D.act_dtype, D.weight_dtype);
   if (!f32 && !bf16 && !i8)
     return fail(nullptr, COLIBRI_ERR_UNSUPPORTED, "dtype pair (act=%d, weight=%d) not supported", D.act_dtype, D.weight_dtype);
   if (i8 && D.shared_d_ff > 0)
-    return fail(nullptr, COLIBRI_ERR_UNSUPPORTED, "shared expert with int8 weights is not supported");
+    return fail(nullptr, COLIBRI_ERR_UNSUPPORTED, "shared expert with int8 / int4 weights is not supported");
   if (i8 && D.d_ff > kDecMaxFF)
-    return fail(nullptr, COLIBRI_ERR_UNSUPPORTED, "int8 weights support d_ff <= %d", kDecMaxFF);
-  if (!i8 && D.weight_scale_mode != COLIBRI_SCALE_PER_CHANNEL)
+    return fail(nullptr, COLIBRI_ERR_UNSUPPORTED, "int8 / int4 weights support d_ff <= %d", kDecMaxFF);
+  if (w4 && (D.d_model % 128 != 0 || D.d_ff % 128 != 0))
+    return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "int4 weights need d_model and d_ff multiples of 128 (the scale group)");
+  if (!w8 && D.weight_scale_mode != COLIBRI_SCALE_PER_CHANNEL)
     return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "weight_scale_mode applies to int8 weights only");
   if (f32 && ((int64_t)D.max_tokens * D.top_k / kSimtBM + D.num_experts > 65535 ||
               ((int64_t)D.max_tokens + kSimtBM - 1) / kSimtBM > 65535))
@@ -199,7 +200,9 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   if (!ctx) return fail(nullptr, COLIBRI_ERR_OOM, "host allocation failed");
   ctx->desc = D;
   ctx->sm_count = prop.multiProcessorCount;
-  ctx->expert_stride = ((int64_t)3 * D.d_model * D.d_ff + 127) / 128 * 128;
+  // int4: 256 elements = 128 bytes, so every expert still starts on a 128-byte boundary
+  const int64_t stride_unit = D.weight_dtype == COLIBRI_I4 ? 256 : 128;
+  ctx->expert_stride = ((int64_t)3 * D.d_model * D.d_ff + stride_unit - 1) / stride_unit * stride_unit;
   ctx->profile = env_flag("COLIBRI_PROFILE");
   ctx->dec_split = i8 ? pick_dec_split(D.d_ff) : 1;
 
@@ -230,6 +233,11 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   const size_t o_rtick = c.take(rsplit ? (size_t)((M + 127) / 128) * 4 : 0);
   const size_t o_err = c.take(4);
   const size_t o_gbar = c.take(i8 ? kFusedBarCount * 4 : 0);
+  const size_t flow_bytes = (size_t)(kFlowUnitCtrs + kFlowTileCtrs) * 4;
+  const size_t o_flow = c.take(i8 ? flow_bytes : 0);
+  const int64_t flow_rows = std::min<int64_t>(M, kFlowMaxT) * D.top_k;
+  const size_t o_fhh = c.take(i8 ? flow_rows * f : 0), o_fhl = c.take(i8 ? flow_rows * f : 0);
+  const size_t o_fhs = c.take(i8 ? (size_t)kDecSplitMax * flow_rows * 4 : 0);
   ctx->ws_bytes = c.off;
 
   DeviceGuard guard(D.device_id);
@@ -263,11 +271,17 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   w.plane_scale = reinterpret_cast<float*>(b + o_psc);
   w.err = reinterpret_cast<uint32_t*>(b + o_err);
   w.grid_bar = i8 ? reinterpret_cast<int32_t*>(b + o_gbar) : nullptr;
+  w.flow_ctr = i8 ? reinterpret_cast<int32_t*>(b + o_flow) : nullptr;
+  w.flow_hhi = i8 ? reinterpret_cast<int8_t*>(b + o_fhh) : nullptr;
+  w.flow_hlo = i8 ? reinterpret_cast<int8_t*>(b + o_fhl) : nullptr;
+  w.flow_hscale = i8 ? reinterpret_cast<float*>(b + o_fhs) : nullptr;
+  w.flow_rows = i8 ? (int)flow_rows : 0;
   w.router_part = rsplit ? reinterpret_cast<float*>(b + o_rpart) : nullptr;
   w.router_ticket = rsplit ? reinterpret_cast<int32_t*>(b + o_rtick) : nullptr;
   if (cudaMemset(w.err, 0, 4) != cudaSuccess ||
       (rsplit && cudaMemset(w.router_ticket, 0, (size_t)((M + 127) / 128) * 4) != cudaSuccess) ||
-      (i8 && cudaMemset(w.grid_bar, 0, kFusedBarCount * 4) != cudaSuccess)) {
+      (i8 && cudaMemset(w.grid_bar, 0, kFusedBarCount * 4) != cudaSuccess) ||
+      (i8 && cudaMemset(w.flow_ctr, 0, flow_bytes) != cudaSuccess)) {
     cudaFree(ctx->ws_base);
     delete ctx;
     return fail(nullptr, COLIBRI_ERR_CUDA, "cudaMemset failed");
@@ -275,15 +289,22 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   if (ctx->profile) {
     for (auto& e : ctx->ev) cudaEventCreate(&e);
   }
+  for (auto& e : ctx->cap_ev) {
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      cudaGetLastError();
+      e = nullptr;
+    }
+  }
   ctx->use_graphs = !(getenv("COLIBRI_GRAPHS") && strcmp(getenv("COLIBRI_GRAPHS"), "0") == 0);
   // Programmatic dependent launch measured slower on the small-batch decode chain and neutral on
   // prefill, so it is opt-in (COLIBRI_PDL=1).
   ctx->use_pdl = env_flag("COLIBRI_PDL");
   ctx->dec_fused = !(getenv("COLIBRI_DEC_FUSED") && strcmp(getenv("COLIBRI_DEC_FUSED"), "0") == 0);
   ctx->dec_route = !(getenv("COLIBRI_DEC_ROUTE") && strcmp(getenv("COLIBRI_DEC_ROUTE"), "0") == 0);
+  // the dataflow plan of the fused int8 launch is opt-in (COLIBRI_DEC_FLOW=1) until it measures faster
+  ctx->dec_flow = env_flag("COLIBRI_DEC_FLOW");
   cudaError_t ce = configure_router_kernels();
   if (ce == cudaSuccess) ce = configure_tc_kernels();
-  if (ce == cudaSuccess) ce = configure_tcs_kernels();
   if (ce == cudaSuccess) ce = configure_dec_kernels();
   if (ce != cudaSuccess) {
     cudaGetLastError();
@@ -304,7 +325,12 @@ void colibri_free(colibri_ctx* ctx) {
       if (e) cudaEventDestroy(e);
     for (auto& e : ctx->prof_ev)
       if (e) cudaEventDestroy(e);
-    for (auto& g : ctx->graphs) cudaGraphExecDestroy(g.exec);
+    for (auto& e : ctx->cap_ev)
+      if (e) cudaEventDestroy(e);
+    for (auto& g : ctx->graphs) {
+      cudaGraphExecDestroy(g.exec);
+      if (g.graph) cudaGraphDestroy(g.graph);
+    }
   }
   delete ctx;
 }
@@ -326,10 +352,12 @@ colibri_status check_launch(colibri_ctx* ctx, cudaError_t e, const char* what) {
 
 // The launch sequence of one forward (stream-ordered, no host synchronisation unless
 // COLIBRI_PROFILE printing is on).
+// stage_ev: NULL, or 6 events recorded at the stage boundaries (as event-record nodes when
+// `ev_nodes` is set: the forward is then being captured into a graph for timed replays).
 colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int32_t T, const void* router_w,
                                const float* router_b, const int32_t* user_idx, const float* user_w,
                                const void* expert_w, const float* expert_scales, const void* shared_w, void* y,
-                               PtrKind yk, cudaStream_t s, int gemm) {
+                               PtrKind yk, cudaStream_t s, int gemm, cudaEvent_t* stage_ev, bool ev_nodes) {
   const colibri_desc& D = ctx->desc;
   const bool routed_by_caller = user_idx != nullptr;
   Workspace& w = ctx->ws;
@@ -341,7 +369,7 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
   void* yd = y;
   // Kernels after the first may overlap their predecessor's tail (not while stage events are
   // recorded between them: the events would then not bound the stages).
-  LaunchScope launch_scope(ctx->use_pdl && !ctx->profile && !ctx->prof_on);
+  LaunchScope launch_scope(ctx->use_pdl && !ctx->profile && stage_ev == nullptr);
   if (xk == kPtrHost) {
     COLIBRI_TRY(cudaMemcpyAsync(w.x_stage, x, (size_t)T * row_bytes, cudaMemcpyHostToDevice, s), "copy x to device");
     launch_chain_break();
@@ -349,12 +377,12 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
   }
   if (yk == kPtrHost) yd = w.y_stage;
   // stage boundary events: COLIBRI_PROFILE printing and/or colibri_profile_begin recording
-  const bool rec = ctx->prof_on && ctx->prof_n < ctx->prof_max;
-  cudaEvent_t* rec_ev = rec ? &ctx->prof_ev[(size_t)ctx->prof_n * 6] : nullptr;
-  if (rec) ctx->prof_n++;
   auto mark = [&](int i) {
     if (ctx->profile) cudaEventRecord(ctx->ev[i], s);
-    if (rec_ev) cudaEventRecord(rec_ev[i], s);
+    if (stage_ev) {
+      if (ev_nodes) cudaEventRecordWithFlags(stage_ev[i], s, cudaEventRecordExternal);
+      else cudaEventRecord(stage_ev[i], s);
+    }
   };
   mark(0);
 
@@ -364,6 +392,7 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
   // against 0.0874 ms per step, T=8: 0.198 against 0.204 ms).
   const bool route_in_dec =
       D.weight_dtype == COLIBRI_I8 && ctx->dec_fused && ctx->dec_route && T <= kFusedRouteMaxT;
+  const bool quant = D.weight_dtype == COLIBRI_I8 || D.weight_dtype == COLIBRI_I4;
 
   // ---- Gate
   if (routed_by_caller) {
@@ -381,7 +410,7 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
   const int nblk = (T + kCountBlock - 1) / kCountBlock;
   const int bm = D.weight_dtype == COLIBRI_F32 ? kSimtBM : (gemm == kGemmPair ? kTcPairBM : kTcBM);
   const RowPlanes xplanes{w.plane_hi, w.plane_lo, w.plane_scale};
-  const RowPlanes* planes = D.weight_dtype == COLIBRI_I8 ? &xplanes : nullptr;
+  const RowPlanes* planes = quant ? &xplanes : nullptr;
   if (route_in_dec) {
     // grouping and the x planes are phase 0 of the fused expert launch
   } else if (T <= kFusedRouteMaxT) {
@@ -436,15 +465,13 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
     a.err = w.err;
     a.sm_count = ctx->sm_count;
     a.pair = gemm == kGemmPair;
-    if (gemm == kGemmSwap) COLIBRI_TRY(launch_tcs_gateup(a, s), "tcs_gateup");
-    else COLIBRI_TRY(launch_tc_gateup(a, s), "tc_gateup");
+    COLIBRI_TRY(launch_tc_gateup(a, s), "tc_gateup");
     mark(3);
     a.A = w.H;
     a.out = w.Yp;
     a.A_sh = w.Hs;
     a.out_sh = w.Ys;
-    if (gemm == kGemmSwap) COLIBRI_TRY(launch_tcs_down(a, s), "tcs_down");
-    else COLIBRI_TRY(launch_tc_down(a, s), "tc_down");
+    COLIBRI_TRY(launch_tc_down(a, s), "tc_down");
   } else {
     // K splits of the down projection: enough work items to cover every SM a few times
     nsplit = 1;
@@ -461,7 +488,16 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
              touched * tiles * gsplit < 8 * ctx->sm_count)
         gsplit <<= 1;
     }
-    if (ctx->dec_fused) {
+    if (D.weight_dtype == COLIBRI_I4) {
+      // int4: the stream kernels that widen the packed tiles, then H planes, then down
+      COLIBRI_TRY(launch_dec4_gateup(w.plane_hi, w.plane_lo, w.plane_scale, (const uint8_t*)expert_w, expert_scales,
+                                     stride, d, f, E, w.offsets, gsplit, (float*)w.H, R, T, w.err, s), "dec4_gateup");
+      mark(3);
+      COLIBRI_TRY(launch_dec_finish_h((const float*)w.H, gsplit, R, f, nsplit, w.plane_hi, w.plane_lo,
+                                      w.plane_scale, s), "dec_finish_h");
+      COLIBRI_TRY(launch_dec4_down(w.plane_hi, w.plane_lo, w.plane_scale, (const uint8_t*)expert_w, expert_scales,
+                                   stride, d, f, E, w.offsets, nsplit, R, w.Ypart, T, w.err, s), "dec4_down");
+    } else if (ctx->dec_fused) {
       // one cooperative launch for gate/up, H, down and the combine (stages 3-5 are empty)
       DecFusedArgs fa;
       fa.planes_hi = w.plane_hi;
@@ -486,6 +522,13 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
       fa.y = (__nv_bfloat16*)yd;
       fa.bar = w.grid_bar;
       fa.err = w.err;
+      fa.flow = ctx->dec_flow;
+      fa.unit_ctr = w.flow_ctr;
+      fa.tile_ctr = w.flow_ctr + kFlowUnitCtrs;
+      fa.hplanes_hi = w.flow_hhi;
+      fa.hplanes_lo = w.flow_hlo;
+      fa.hplanes_scale = w.flow_hscale;
+      fa.flow_rows = w.flow_rows;
       if (route_in_dec) {
         fa.route_in_kernel = routed_by_caller ? 2 : 1;
         fa.x = (const __nv_bfloat16*)xd;
@@ -514,7 +557,7 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
   // ---- Gather
   if (D.weight_dtype == COLIBRI_I8 && ctx->dec_fused) {
     // done inside the fused kernel
-  } else if (D.weight_dtype == COLIBRI_I8) {
+  } else if (quant) {
     COLIBRI_TRY(launch_combine_split(w.Ypart, nsplit, R, w.dst_row, w.topk_w, T, k, d, yd, act, s),
                 "combine_split");
   } else {
@@ -553,9 +596,9 @@ colibri_status forward_impl(colibri_ctx* ctx, const void* x, int32_t T, const vo
   } else if (!router_w) {
     return fail(ctx, COLIBRI_ERR_INVALID_ARG, "router_w is NULL");
   }
-  const bool i8 = D.weight_dtype == COLIBRI_I8;
-  if (i8 != (expert_scales != nullptr))
-    return fail(ctx, COLIBRI_ERR_INVALID_ARG, "expert_scales must be given exactly when weights are int8");
+  const bool quant = D.weight_dtype == COLIBRI_I8 || D.weight_dtype == COLIBRI_I4;
+  if (quant != (expert_scales != nullptr))
+    return fail(ctx, COLIBRI_ERR_INVALID_ARG, "expert_scales must be given exactly when weights are int8 or int4");
   if ((D.shared_d_ff > 0) != (shared_w != nullptr))
     return fail(ctx, COLIBRI_ERR_INVALID_ARG, "shared_w must be given exactly when shared_d_ff > 0");
   const void* ptrs[] = {x, router_w, router_b, expert_w, expert_scales, shared_w, y, user_idx, user_w};
@@ -577,10 +620,18 @@ colibri_status forward_impl(colibri_ctx* ctx, const void* x, int32_t T, const vo
   // bf16 weights: the tiling of the expert GEMMs (see gemm_mode)
   const int gemm = D.weight_dtype == COLIBRI_BF16 ? gemm_mode(T * D.top_k / D.num_experts) : kGemmOne;
 
+  // Stage events of colibri_profile_begin: the events of this call, if it is still recorded.
+  const bool prof_rec = ctx->prof_on && ctx->prof_n < ctx->prof_max;
+  cudaEvent_t* call_ev = prof_rec ? &ctx->prof_ev[(size_t)ctx->prof_n * 6] : nullptr;
+  if (prof_rec) ctx->prof_n++;
+
   // Replay a captured CUDA graph of this exact call when possible: device x and y, a stream
-  // other than the legacy default stream that is not itself being captured, and no profiling.
+  // other than the legacy default stream that is not itself being captured, and no COLIBRI_PROFILE
+  // printing.  While stage events are recorded a second graph of the same call is used whose
+  // event-record nodes sit at the stage boundaries; before each replay they are pointed at that
+  // call's events, so the recorded stages are those of the replayed graph.
   const bool graphable = ctx->use_graphs && reinterpret_cast<uintptr_t>(s) > 2 && xk == kPtrDevice &&
-                         yk == kPtrDevice && !ctx->profile && !ctx->prof_on;
+                         yk == kPtrDevice && !ctx->profile && (!prof_rec || ctx->cap_ev[0] != nullptr);
   if (graphable) {
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) {
@@ -591,17 +642,22 @@ colibri_status forward_impl(colibri_ctx* ctx, const void* x, int32_t T, const vo
       const uintptr_t key[14] = {(uintptr_t)x,        (uintptr_t)T,        (uintptr_t)router_w, (uintptr_t)router_b,
                                  (uintptr_t)user_idx, (uintptr_t)user_w,   (uintptr_t)expert_w, (uintptr_t)expert_scales,
                                  (uintptr_t)shared_w, (uintptr_t)y,        (uintptr_t)s,        (uintptr_t)gemm,
-                                 0, 0};
-      for (auto& g : ctx->graphs) {
-        if (memcmp(g.key, key, sizeof(key)) == 0) {
-          g.last_use = ++ctx->graph_clock;
-          COLIBRI_TRY(cudaGraphLaunch(g.exec, s), "graph launch");
-          return COLIBRI_OK;
-        }
-      }
+                                 (uintptr_t)prof_rec, 0};
+      // points the stage-event nodes of a timed graph at this call's events, then launches it
+      auto replay = [&](colibri_ctx::GraphEntry& g) -> colibri_status {
+        if (prof_rec)
+          for (int i = 0; i < 6; ++i)
+            COLIBRI_TRY(cudaGraphExecEventRecordNodeSetEvent(g.exec, g.ev_node[i], call_ev[i]), "set stage event");
+        g.last_use = ++ctx->graph_clock;
+        COLIBRI_TRY(cudaGraphLaunch(g.exec, s), "graph launch");
+        return COLIBRI_OK;
+      };
+      for (auto& g : ctx->graphs)
+        if (memcmp(g.key, key, sizeof(key)) == 0) return replay(g);
       COLIBRI_TRY(cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal), "begin capture");
       const colibri_status st = enqueue_forward(ctx, x, xk, T, router_w, router_b, user_idx, user_w, expert_w,
-                                                expert_scales, shared_w, y, yk, s, gemm);
+                                                expert_scales, shared_w, y, yk, s, gemm,
+                                                prof_rec ? ctx->cap_ev : nullptr, prof_rec);
       cudaGraph_t graph = nullptr;
       const cudaError_t ce = cudaStreamEndCapture(s, &graph);
       if (st != COLIBRI_OK) {
@@ -610,28 +666,51 @@ colibri_status forward_impl(colibri_ctx* ctx, const void* x, int32_t T, const vo
         return st;
       }
       if (ce != cudaSuccess) return check_launch(ctx, ce, "end capture");
+      colibri_ctx::GraphEntry ge;
+      memcpy(ge.key, key, sizeof(key));
+      if (prof_rec) {
+        // find the event-record node of each stage boundary by the event it was captured with
+        size_t n = 0;
+        cudaError_t ne = cudaGraphGetNodes(graph, nullptr, &n);
+        std::vector<cudaGraphNode_t> nodes(n);
+        if (ne == cudaSuccess && n) ne = cudaGraphGetNodes(graph, nodes.data(), &n);
+        for (size_t j = 0; ne == cudaSuccess && j < n; ++j) {
+          cudaGraphNodeType t;
+          ne = cudaGraphNodeGetType(nodes[j], &t);
+          if (ne != cudaSuccess || t != cudaGraphNodeTypeEventRecord) continue;
+          cudaEvent_t ev = nullptr;
+          ne = cudaGraphEventRecordNodeGetEvent(nodes[j], &ev);
+          for (int i = 0; ne == cudaSuccess && i < 6; ++i)
+            if (ev == ctx->cap_ev[i]) ge.ev_node[i] = nodes[j];
+        }
+        bool found = ne == cudaSuccess;
+        for (int i = 0; i < 6; ++i) found = found && ge.ev_node[i] != nullptr;
+        if (!found) {
+          cudaGraphDestroy(graph);
+          cudaGetLastError();
+          return fail(ctx, COLIBRI_ERR_CUDA, "stage-event nodes not found in the captured forward");
+        }
+      }
       cudaGraphExec_t exec = nullptr;
       const cudaError_t ie = cudaGraphInstantiate(&exec, graph, 0);
-      cudaGraphDestroy(graph);
+      if (ie != cudaSuccess || !prof_rec) cudaGraphDestroy(graph);
       if (ie != cudaSuccess) return check_launch(ctx, ie, "graph instantiate");
       if (ctx->graphs.size() >= kMaxGraphs) {
         size_t lru = 0;
         for (size_t i = 1; i < ctx->graphs.size(); ++i)
           if (ctx->graphs[i].last_use < ctx->graphs[lru].last_use) lru = i;
         cudaGraphExecDestroy(ctx->graphs[lru].exec);
+        if (ctx->graphs[lru].graph) cudaGraphDestroy(ctx->graphs[lru].graph);
         ctx->graphs.erase(ctx->graphs.begin() + lru);
       }
-      colibri_ctx::GraphEntry ge;
-      memcpy(ge.key, key, sizeof(key));
       ge.exec = exec;
-      ge.last_use = ++ctx->graph_clock;
+      ge.graph = prof_rec ? graph : nullptr;
       ctx->graphs.push_back(ge);
-      COLIBRI_TRY(cudaGraphLaunch(exec, s), "graph launch");
-      return COLIBRI_OK;
+      return replay(ctx->graphs.back());
     }
   }
   return enqueue_forward(ctx, x, xk, T, router_w, router_b, user_idx, user_w, expert_w, expert_scales, shared_w, y,
-                         yk, s, gemm);
+                         yk, s, gemm, call_ev, false);
 }
 
 }  // namespace
@@ -688,6 +767,9 @@ colibri_status colibri_sync_status(colibri_ctx* ctx, void* stream) {
     // a wait that gave up may leave the fused kernel's grid-barrier counters out of step
     if (ctx->ws.grid_bar)
       COLIBRI_TRY(cudaMemset(ctx->ws.grid_bar, 0, kFusedBarCount * 4), "reset grid-barrier counters");
+    if (ctx->ws.flow_ctr)
+      COLIBRI_TRY(cudaMemset(ctx->ws.flow_ctr, 0, (size_t)(kFlowUnitCtrs + kFlowTileCtrs) * 4),
+                  "reset completion counters");
     return fail(ctx, COLIBRI_ERR_TIMEOUT, "device error word 0x%x (a bounded wait gave up)", err);
   }
   return COLIBRI_OK;
@@ -731,6 +813,24 @@ colibri_status colibri_profile_end(colibri_ctx* ctx, float* stage_ms, int32_t* n
   if (stage_ms)
     for (int i = 0; i < COLIBRI_NUM_STAGES; ++i) stage_ms[i] = (float)tot[i];
   if (ncalls) *ncalls = ctx->prof_n;
+  return COLIBRI_OK;
+}
+
+colibri_status colibri_profile_calls(colibri_ctx* ctx, float* call_stage_ms, int32_t max_calls) {
+  if (!ctx) return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "ctx is NULL");
+  if (ctx->prof_on) return fail(ctx, COLIBRI_ERR_INVALID_ARG, "colibri_profile_end was not called");
+  if (!call_stage_ms || max_calls < 0) return fail(ctx, COLIBRI_ERR_INVALID_ARG, "bad output buffer");
+  DeviceGuard guard(ctx->desc.device_id);
+  const int n = std::min(max_calls, ctx->prof_n);
+  for (int c = 0; c < n; ++c) {
+    cudaEvent_t* ev = &ctx->prof_ev[(size_t)c * 6];
+    COLIBRI_TRY(cudaEventSynchronize(ev[5]), "event synchronize");
+    for (int i = 0; i < COLIBRI_NUM_STAGES; ++i) {
+      float ms = 0.f;
+      COLIBRI_TRY(cudaEventElapsedTime(&ms, ev[i], ev[i + 1]), "event elapsed time");
+      call_stage_ms[(size_t)c * COLIBRI_NUM_STAGES + i] = ms;
+    }
+  }
   return COLIBRI_OK;
 }
 

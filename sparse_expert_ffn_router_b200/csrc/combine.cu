@@ -38,44 +38,95 @@ __device__ __forceinline__ void store8(float* p, const float (&v)[8]) {
   reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
 
-// One thread per (token, 8 consecutive outputs): the k slot loads of a thread are independent,
-// and a warp covers 512 contiguous bytes of each row it reads or writes.
-template <typename Tout, typename Typ>
+// One warp per token row: the routing state of the token is loaded once (one broadcast load per
+// slot), then each lane sums 8 consecutive outputs at a time, U = 8 / KK such groups per step
+// with all U x KK slot loads of the step (16 bytes each for bf16) issued before any is used, so
+// a lane keeps 8 loads in flight and a warp covers 512 contiguous bytes of each row it reads or
+// writes.  KK is the top-k (1, 2, 4 or 8; other k run with KK = 8 and the unused slots skipped).
+template <typename Typ>
+struct Raw8;  // 8 consecutive Yp values as loaded
+template <>
+struct Raw8<__nv_bfloat16> {
+  uint4 q;
+  __device__ void load(const __nv_bfloat16* p) { q = __ldg(reinterpret_cast<const uint4*>(p)); }
+  __device__ float get(int i) const {
+    const uint32_t wv = i < 2 ? q.x : (i < 4 ? q.y : (i < 6 ? q.z : q.w));
+    return __uint_as_float((i & 1) ? (wv & 0xffff0000u) : (wv << 16));
+  }
+};
+template <>
+struct Raw8<float> {
+  float4 a, b;
+  __device__ void load(const float* p) {
+    a = __ldg(reinterpret_cast<const float4*>(p));
+    b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  }
+  __device__ float get(int i) const {
+    return i == 0 ? a.x : i == 1 ? a.y : i == 2 ? a.z : i == 3 ? a.w : i == 4 ? b.x : i == 5 ? b.y : i == 6 ? b.z : b.w;
+  }
+};
+
+template <typename Tout, typename Typ, int KK>
 __global__ void __launch_bounds__(256) combine_kernel(const Typ* __restrict__ Yp,
                                                       const int32_t* __restrict__ dst_row,
                                                       const float* __restrict__ w, int T, int k,
                                                       int d, const Typ* __restrict__ Ys,
                                                       Tout* __restrict__ y) {
+  constexpr int U = 8 / KK;
   pdl_trigger();
   pdl_wait();
+  const int lane = threadIdx.x & 31;
   const int chunks = d >> 3;
-  for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < (long long)T * chunks;
-       q += (long long)gridDim.x * blockDim.x) {
-    const int t = (int)(q / chunks), c = (int)(q - (long long)t * chunks) * 8;
-    int rows[kMaxTopK];
-    float ws[kMaxTopK];
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long t = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
+    int rows[KK];
+    float ws[KK];
 #pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
-      rows[j] = j < k ? dst_row[(size_t)t * k + j] : 0;
-      ws[j] = j < k ? w[(size_t)t * k + j] : 0.f;
+    for (int j = 0; j < KK; ++j) {
+      rows[j] = j < k ? __ldg(dst_row + (size_t)t * k + j) : 0;
+      ws[j] = j < k ? __ldg(w + (size_t)t * k + j) : 0.f;
     }
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int c0 = lane; c0 < chunks; c0 += 32 * U) {
+      Raw8<Typ> v[U][KK];
 #pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
-      if (j < k) {
-        float v[8];
-        load8(Yp + (size_t)rows[j] * d + c, v);
+      for (int u = 0; u < U; ++u) {
+        const int c = (c0 + 32 * u) * 8;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = fmaf(ws[j], v[i], acc[i]);
+        for (int j = 0; j < KK; ++j)
+          if (j < k && c < d) v[u][j].load(Yp + (size_t)rows[j] * d + c);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c = (c0 + 32 * u) * 8;
+        if (c >= d) continue;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < KK; ++j)
+          if (j < k)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = fmaf(ws[j], v[u][j].get(i), acc[i]);
+        if (Ys) {
+          float vs[8];
+          load8(Ys + (size_t)t * d + c, vs);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] += vs[i];
+        }
+        store8(y + (size_t)t * d + c, acc);
       }
     }
-    if (Ys) {
-      float v[8];
-      load8(Ys + (size_t)t * d + c, v);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] += v[i];
-    }
-    store8(y + (size_t)t * d + c, acc);
+  }
+}
+
+template <typename Tout, typename Typ>
+cudaError_t launch_combine_k(const Typ* yp, const int32_t* dst_row, const float* w, int T, int k, int d, const Typ* ys,
+                             Tout* y, dim3 grid, cudaStream_t s) {
+  const dim3 block(256);
+  switch (k) {
+    case 1: return launch_kernel(combine_kernel<Tout, Typ, 1>, grid, block, 0, s, 1, yp, dst_row, w, T, k, d, ys, y);
+    case 2: return launch_kernel(combine_kernel<Tout, Typ, 2>, grid, block, 0, s, 1, yp, dst_row, w, T, k, d, ys, y);
+    case 3:
+    case 4: return launch_kernel(combine_kernel<Tout, Typ, 4>, grid, block, 0, s, 1, yp, dst_row, w, T, k, d, ys, y);
+    default: return launch_kernel(combine_kernel<Tout, Typ, 8>, grid, block, 0, s, 1, yp, dst_row, w, T, k, d, ys, y);
   }
 }
 
@@ -140,32 +191,26 @@ __global__ void __launch_bounds__(256) combine_split_kernel(const float* __restr
   }
 }
 
-int grid_for_rows(int T, int d) {
-  const long long threads = (long long)T * (d / 8);
-  return (int)std::min<long long>((threads + 255) / 256, 16384);
-}
+// one warp per token, up to 16 CTAs of 8 warps per SM of a 148-SM part
+int grid_for_rows(int T) { return (int)std::min<long long>(((long long)T + 7) / 8, 148 * 16); }
 
 }  // namespace
 
 cudaError_t launch_combine(const void* Yp, int yp_dtype, const int32_t* dst_row, const float* w,
                            int T, int k, int d, const void* Ys, void* y, int act, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  const dim3 grid(grid_for_rows(T, d)), block(256);
+  if (k < 1 || k > kMaxTopK) return cudaErrorInvalidValue;
+  const dim3 grid(grid_for_rows(T));
   if (yp_dtype == COLIBRI_BF16) {
     const __nv_bfloat16* yp = (const __nv_bfloat16*)Yp;
     const __nv_bfloat16* ys = (const __nv_bfloat16*)Ys;
-    if (act == COLIBRI_BF16)
-      return launch_kernel(combine_kernel<__nv_bfloat16, __nv_bfloat16>, grid, block, 0, s, 1, yp, dst_row, w, T, k,
-                           d, ys, (__nv_bfloat16*)y);
-    return launch_kernel(combine_kernel<float, __nv_bfloat16>, grid, block, 0, s, 1, yp, dst_row, w, T, k, d, ys,
-                         (float*)y);
+    if (act == COLIBRI_BF16) return launch_combine_k(yp, dst_row, w, T, k, d, ys, (__nv_bfloat16*)y, grid, s);
+    return launch_combine_k(yp, dst_row, w, T, k, d, ys, (float*)y, grid, s);
   }
   const float* yp = (const float*)Yp;
   const float* ys = (const float*)Ys;
-  if (act == COLIBRI_BF16)
-    return launch_kernel(combine_kernel<__nv_bfloat16, float>, grid, block, 0, s, 1, yp, dst_row, w, T, k, d, ys,
-                         (__nv_bfloat16*)y);
-  return launch_kernel(combine_kernel<float, float>, grid, block, 0, s, 1, yp, dst_row, w, T, k, d, ys, (float*)y);
+  if (act == COLIBRI_BF16) return launch_combine_k(yp, dst_row, w, T, k, d, ys, (__nv_bfloat16*)y, grid, s);
+  return launch_combine_k(yp, dst_row, w, T, k, d, ys, (float*)y, grid, s);
 }
 
 cudaError_t launch_combine_split(const float* Ypart, int nsplit, int rows, const int32_t* dst_row,

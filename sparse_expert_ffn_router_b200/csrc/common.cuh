@@ -78,6 +78,11 @@ struct Workspace {
   float* router_part = nullptr;    // [8, M, E] K-split partial logits
   int32_t* router_ticket = nullptr;  // [ceil(M/128)] arrival counters (zero between calls)
   int32_t* grid_bar = nullptr;       // [4] grid-barrier counters of the fused int8 kernel (zero between calls)
+  int32_t* flow_ctr = nullptr;       // [kFlowUnitCtrs + kFlowTileCtrs] dataflow int8 kernel (zero between calls)
+  int8_t* flow_hhi = nullptr;        // [flow_rows, f] H planes of the dataflow int8 kernel
+  int8_t* flow_hlo = nullptr;
+  float* flow_hscale = nullptr;      // [kDecSplitMax, flow_rows]
+  int flow_rows = 0;                 // min(max_tokens, kFlowMaxT) * k
   int8_t* plane_hi = nullptr;  // [M*k, max(d, f)] int8 activation planes, int8 path
   int8_t* plane_lo = nullptr;
   float* plane_scale = nullptr;  // [M*k]
@@ -109,13 +114,19 @@ struct colibri_ctx {
     uintptr_t key[14];
     cudaGraphExec_t exec;
     uint64_t last_use;
+    // graphs captured while colibri_profile_begin is active also hold one event-record node per
+    // stage boundary; the graph is kept so that each replay can point them at that call's events
+    cudaGraph_t graph = nullptr;
+    cudaGraphNode_t ev_node[6] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
   };
+  cudaEvent_t cap_ev[6] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};  // events the nodes are captured with
   std::vector<GraphEntry> graphs;
   uint64_t graph_clock = 0;
   bool use_graphs = true;
   bool use_pdl = false;  // programmatic dependent launch between the kernels of a forward (opt-in)
   bool dec_fused = true;  // int8 weights: the one-launch expert stage (COLIBRI_DEC_FUSED=0: four launches)
   bool dec_route = true;  // int8, T <= 64: routing inside that launch too (COLIBRI_DEC_ROUTE=0: not)
+  bool dec_flow = false;  // int8, T <= 64: completion counters instead of grid barriers (COLIBRI_DEC_FLOW=1)
 };
 
 namespace colibri {
@@ -255,9 +266,11 @@ struct TcGemmArgs {
   int sm_count;
   bool pair;            // clusters of two CTAs with 256-row pair tiles (cta_group::2)
 };
-// Tensor map with a 128-byte inner box, 128-byte swizzle, zero fill out of bounds
+// Tensor map, zero fill out of bounds; 128-byte swizzle (with a 128-byte inner box) unless told
+// otherwise
 bool make_tmap(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int rank, const uint64_t* dims,
-               const uint64_t* strides_bytes, const uint32_t* box);
+               const uint64_t* strides_bytes, const uint32_t* box,
+               CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B);
 // bf16 tensor map: 64-element (128-byte) inner box, 128-byte swizzle, zero fill out of bounds
 bool make_bf16_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                     const uint64_t* strides_bytes, const uint32_t* box);
@@ -265,12 +278,6 @@ cudaError_t configure_tc_kernels();      // once per device, before any launch
 cudaError_t configure_router_kernels();  // once per device, before any launch
 cudaError_t launch_tc_gateup(const TcGemmArgs& a, cudaStream_t s);
 cudaError_t launch_tc_down(const TcGemmArgs& a, cudaStream_t s);
-// The same grouped GEMMs with weights on the M side and token rows on the N side (tiles of
-// 128 channels x 16..256 rows), see gemm_tcs.cu.  Reads A/rows/offsets/E/W/wstride/out, the
-// shared-expert fields, d/f/fs, err and sm_count of TcGemmArgs.
-cudaError_t configure_tcs_kernels();     // once per device, before any launch
-cudaError_t launch_tcs_gateup(const TcGemmArgs& a, cudaStream_t s);
-cudaError_t launch_tcs_down(const TcGemmArgs& a, cudaStream_t s);
 
 // int8 weight-streaming decode path, see decode_i8.cu (the x planes come from the scatter)
 // max_rows_per_expert: an upper bound (T) that picks the token chunk (8, 16 or 32 rows).
@@ -290,6 +297,15 @@ cudaError_t launch_dec_down(const int8_t* Hhi, const int8_t* Hlo, const float* h
                             const float* scales, int scale_mode, int64_t wstride, int d, int f, int E,
                             const int32_t* offsets, int nsplit, int R, float* Ypart, int max_rows_per_expert,
                             uint32_t* err, cudaStream_t s);
+// Group-wise int4 weights (two per byte along K, group scales [K / 128][out] per matrix, per
+// expert W1 | W3 | W2): the same outputs as launch_dec_gateup / launch_dec_down.  wstride counts
+// int4 elements (a multiple of 256); d and f must be multiples of 128.
+cudaError_t launch_dec4_gateup(const int8_t* Xhi, const int8_t* Xlo, const float* xscale, const uint8_t* W,
+                               const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
+                               int nsplit, float* GU, int R, int max_rows_per_expert, uint32_t* err, cudaStream_t s);
+cudaError_t launch_dec4_down(const int8_t* Hhi, const int8_t* Hlo, const float* hscale, const uint8_t* W,
+                             const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
+                             int nsplit, int R, float* Ypart, int max_rows_per_expert, uint32_t* err, cudaStream_t s);
 // The whole int8 expert stage (gate/up stream, H planes, down stream, combine) in one
 // cooperative launch with grid barriers; the x planes must already be in planes_hi/lo/scale.
 struct DecFusedArgs {
@@ -322,8 +338,22 @@ struct DecFusedArgs {
   int32_t* counts = nullptr;                // [E]
   int32_t* offsets_out = nullptr;           // [E+1]
   int32_t* src_row = nullptr;               // [T*k]
+  // dataflow plan (dec_flow_kernel, T <= kFlowMaxT): completion counters instead of grid barriers
+  bool flow = false;
+  int32_t* unit_ctr = nullptr;              // [kFlowUnitCtrs], zero between launches
+  int32_t* tile_ctr = nullptr;              // [kFlowTileCtrs], zero between launches
+  // the H planes have buffers of their own in this plan: an H unit is written while gate/up
+  // items of other units may still read the x planes of the same rows
+  int8_t* hplanes_hi = nullptr;             // [flow_rows, f]
+  int8_t* hplanes_lo = nullptr;
+  float* hplanes_scale = nullptr;           // [dsplit, flow_rows]
+  int flow_rows = 0;                        // rows those buffers hold (R <= flow_rows)
 };
 constexpr int kFusedBarCount = 8;
+constexpr int kFlowMaxT = 64;
+// (token chunks of all experts) x (down splits) for T <= 64 tokens: chunks <= R / 8 + E
+constexpr int kFlowUnitCtrs = (kFlowMaxT * kMaxTopK / 8 + kMaxExperts) * kDecSplitMax;
+constexpr int kFlowTileCtrs = 65536 / 128;  // 128-column output tiles of d_model
 cudaError_t launch_dec_fused(const DecFusedArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------------------------------

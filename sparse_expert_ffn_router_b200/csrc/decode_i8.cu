@@ -143,13 +143,50 @@ struct alignas(64) DecStreamParams {
 
 struct DecItem {
   int e, mat, tile, split, chunk, row0, ntok;
+  int gchunk;  // chunk number over all touched experts
 };
+
+// Shared-memory control block of the stream kernels (after the ring).
+struct DsCtl {
+  uint64_t full[kDsMaxStages];
+  uint64_t empty[kDsMaxStages];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem;
+  int abort;
+  int issued;    // copies issued / stages consumed, for the error path
+  int consumed;
+  int flag;      // result of a grid-wide wait, broadcast to the epilogue warps
+  int eflag;     // flow kernel: this CTA completed a unit / an output tile (epilogue warps)
+  int hpass;     // fused kernel: 1 once the epilogue warps passed the H barrier, -1 if it failed
+  int first;     // this CTA's first work item (items first, first + gridDim.x, ...)
+  int ntouched;
+  int32_t off[kMaxExperts + 1];     // row offsets of the experts' groups
+  int32_t touched[kMaxExperts];
+  int32_t pre[2][kMaxExperts + 1];  // item prefix over the touched experts: [0] gate/up, [1] down
+  int32_t cpre[kMaxExperts + 1];    // token-chunk prefix over the touched experts (chunk numbers)
+  int32_t defer_row[kDsMaxStages];  // fused kernel: down stages whose plane copies wait for H
+  int32_t defer_kx[kDsMaxStages][kDsMaxKbs];
+  int32_t defer_nk[kDsMaxStages];
+  int32_t defer_s[kDsMaxStages];
+  int32_t defer_unit[kDsMaxStages];  // flow kernel: the H unit whose planes a held stage waits for
+  int32_t defer_n[kDsMaxStages];     // and the stage's number (ring position) among all issued
+  int32_t defer_fresh[kDsMaxStages]; // 1: the first held stage of its item (counts as the item's use)
+  float red[4];                     // fused kernel: per-warp maxima of the H pass
+};
+constexpr size_t kDsCtlBytes = 8192;
+static_assert(sizeof(DsCtl) <= kDsCtlBytes, "stream-kernel control block");
+
 
 // Items of one touched expert: (matrix: W1 and W3 for gate/up, W2 for down) x 128-row tiles x
 // K splits x token chunks, tile fastest.
-template <bool kGateUp>
-__device__ __forceinline__ bool dec_item(const DecStreamParams& p, const int32_t* touched, const int32_t* item_prefix,
-                                         int ntouched, const int32_t* off, int L, DecItem& it) {
+template <bool kGateUp, typename Ctl>
+__device__ __forceinline__ bool dec_item(const DecStreamParams& p, const Ctl& c, int pre_idx, int L, DecItem& it) {
+  const int32_t* item_prefix = c.pre[pre_idx];
+  const int32_t* touched = c.touched;
+  const int32_t* off = c.off;
+  const int ntouched = c.ntouched;
   if (L >= item_prefix[ntouched]) return false;
   int lo = 0, hi = ntouched - 1;  // largest ti with item_prefix[ti] <= L
   while (lo < hi) {
@@ -174,6 +211,7 @@ __device__ __forceinline__ bool dec_item(const DecStreamParams& p, const int32_t
   const int base = off[e], cnt = off[e + 1] - base;
   it.row0 = base + it.chunk * p.nt8;
   it.ntok = min(p.nt8, cnt - it.chunk * p.nt8);
+  it.gchunk = c.cpre[lo] + it.chunk;
   return true;
 }
 
@@ -190,34 +228,8 @@ __device__ __forceinline__ bool ds_wait(uint64_t* bar, uint32_t parity, volatile
   }
 }
 
-// Shared-memory control block of the stream kernels (after the ring).
-struct DsCtl {
-  uint64_t full[kDsMaxStages];
-  uint64_t empty[kDsMaxStages];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
-  uint64_t drain;
-  uint32_t tmem;
-  int abort;
-  int issued;    // copies issued / stages consumed, for the error path
-  int consumed;
-  int flag;      // result of a grid-wide wait, broadcast to the epilogue warps
-  int hpass;     // fused kernel: 1 once the epilogue warps passed the H barrier, -1 if it failed
-  int first;     // this CTA's first work item (items first, first + gridDim.x, ...)
-  int ntouched;
-  int32_t off[kMaxExperts + 1];     // row offsets of the experts' groups
-  int32_t touched[kMaxExperts];
-  int32_t pre[2][kMaxExperts + 1];  // item prefix over the touched experts: [0] gate/up, [1] down
-  int32_t defer_row[kDsMaxStages];  // fused kernel: down stages whose plane copies wait for H
-  int32_t defer_kx[kDsMaxStages][kDsMaxKbs];
-  int32_t defer_nk[kDsMaxStages];
-  int32_t defer_s[kDsMaxStages];
-  float red[4];                     // fused kernel: per-warp maxima of the H pass
-};
-constexpr size_t kDsCtlBytes = 8192;
-static_assert(sizeof(DsCtl) <= kDsCtlBytes, "stream-kernel control block");
-
-__device__ __forceinline__ void ds_abort(DsCtl& c, uint32_t* err) {
+template <typename Ctl>
+__device__ __forceinline__ void ds_abort(Ctl& c, uint32_t* err) {
   *(volatile int*)&c.abort = 1;
   atomicOr(err, kErrWaitTimeout);
 }
@@ -263,7 +275,7 @@ __device__ bool ds_produce(const DecStreamParams& p, uint8_t* smem, DsCtl& c, in
     }
   };
   DecItem it;
-  for (int L = c.first; dec_item<kGateUp>(p, c.touched, c.pre[pre_idx], c.ntouched, c.off, L, it); L += gridDim.x) {
+  for (int L = c.first; dec_item<kGateUp>(p, c, pre_idx, L, it); L += gridDim.x) {
     // The item's K blocks start at a rotated block (item index mod block count): items in flight
     // at the same time then read different column offsets of their weight rows, which spreads
     // the requests over the DRAM channels instead of hitting the same address bits everywhere.
@@ -325,7 +337,7 @@ __device__ bool ds_mma(const DecStreamParams& p, uint8_t* smem, DsCtl& c, int S,
   const uint32_t idesc = idesc_s8_s32(128, N);
   const uint32_t plane_bytes = (uint32_t)(2 * p.nt8 * 128);
   DecItem it;
-  for (int L = c.first; dec_item<kGateUp>(p, c.touched, c.pre[pre_idx], c.ntouched, c.off, L, it);
+  for (int L = c.first; dec_item<kGateUp>(p, c, pre_idx, L, it);
        L += gridDim.x, ++iter) {
     const int a = iter & 1;
     const uint32_t aph = (uint32_t)(iter >> 1) & 1u;
@@ -358,14 +370,22 @@ __device__ bool ds_mma(const DecStreamParams& p, uint8_t* smem, DsCtl& c, int S,
   return true;
 }
 
-// Epilogue (warps 2..5): every item of one phase; writes the scaled fp32 partial sums.
-template <bool kGateUp>
+struct NoItemHook {
+  __device__ bool operator()(const DecItem&, bool ok) const { return ok; }
+};
+
+// Epilogue (warps 2..5): every item of one phase; writes the scaled fp32 partial sums.  `after`
+// runs in all four warps once an item's sums are written and its accumulator is released, and
+// also when a warp's wait for the accumulator gave up (ok = false, with the CTA's abort flag set
+// first), so that a hook that synchronises the four warps is reached by all of them for the same
+// item; it returns false to stop the phase.
+template <bool kGateUp, typename After = NoItemHook>
 __device__ bool ds_epilogue(const DecStreamParams& p, DsCtl& c, int pre_idx, int& iter, uint32_t tmem, int warp,
-                            int lane) {
+                            int lane, After after = After()) {
   const int q = warp & 3;
   const int N = 2 * p.nt8;
   DecItem it;
-  for (int L = c.first; dec_item<kGateUp>(p, c.touched, c.pre[pre_idx], c.ntouched, c.off, L, it);
+  for (int L = c.first; dec_item<kGateUp>(p, c, pre_idx, L, it);
        L += gridDim.x, ++iter) {
     const int a = iter & 1;
     const uint32_t aph = (uint32_t)(iter >> 1) & 1u;
@@ -377,7 +397,12 @@ __device__ bool ds_epilogue(const DecStreamParams& p, DsCtl& c, int pre_idx, int
                                          : p.wscale + (size_t)it.e * (2 * p.f + p.d) + (size_t)m * p.f + o;
     const float sc = vo ? __ldg(sp) : 0.f;
     const bool got = ds_wait(&c.tfull[a], aph, &c.abort);
-    if (!__all_sync(0xffffffffu, got)) return false;
+    if (!__all_sync(0xffffffffu, got)) {
+      if (lane == 0) *(volatile int*)&c.abort = 1;
+      __syncwarp();
+      after(it, false);
+      return false;
+    }
     tc_fence_after();
     const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * N);
     // columns [0, nt8) hold the hi plane, [nt8, 2 nt8) the lo plane of the same tokens
@@ -418,6 +443,7 @@ __device__ bool ds_epilogue(const DecStreamParams& p, DsCtl& c, int pre_idx, int
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&c.tempty[a]);
+    if (!after(it, true)) return false;
   }
   return true;
 }
@@ -461,7 +487,8 @@ __device__ __forceinline__ void ds_init(const DecStreamParams* const* phases, in
 
 // The experts' row offsets (from global memory, or already in c.off when `offsets` is NULL),
 // the touched experts and the prefix of their work items per phase.
-__device__ __forceinline__ void ds_items(const DecStreamParams* const* phases, int nphases, DsCtl& c,
+template <typename Ctl>
+__device__ __forceinline__ void ds_items(const DecStreamParams* const* phases, int nphases, Ctl& c,
                                          const int32_t* offsets) {
   const int E = phases[0]->E;
   if (offsets)
@@ -470,10 +497,13 @@ __device__ __forceinline__ void ds_items(const DecStreamParams* const* phases, i
   if (threadIdx.x == 0) {
     int n = 0;
     int acc[2] = {0, 0};
+    int chunks = 0;
     for (int e = 0; e < E; ++e) {
       const int cnt = c.off[e + 1] - c.off[e];
       if (cnt <= 0) continue;
       c.touched[n] = e;
+      c.cpre[n] = chunks;
+      chunks += (cnt + phases[0]->nt8 - 1) / phases[0]->nt8;
       for (int i = 0; i < nphases; ++i) {
         const DecStreamParams& p = *phases[i];
         const bool gateup = p.GU != nullptr;
@@ -483,6 +513,7 @@ __device__ __forceinline__ void ds_items(const DecStreamParams* const* phases, i
       ++n;
     }
     for (int i = 0; i < nphases; ++i) c.pre[i][n] = acc[i];
+    c.cpre[n] = chunks;
     c.ntouched = n;
   }
   __syncthreads();
@@ -541,6 +572,341 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_stream_kernel(const __grid_
   ds_teardown(c, S);
 }
 
+// ------------------------------------------------------------------------- int4 stream kernel
+// Group-wise int4 weights (www.mhpq.cn/news/563172 §4.2: INT4 packed in INT32, groups of 128
+// inputs; www.trdm.cn/news/555962 §6.1: two 4-bit weights per byte, split apart at compute time):
+//
+//   W[o][i] = s[i / 128][o] * q[o][i],  q in [-8, 7] two's complement, element 2j in the low
+//   nibble of byte j;  y[o] = sum_g s[g][o] * (sum_{i in g} q[o][i] x[i])
+//
+// The stream is the int8 one with two changes.  The packed tiles (128 rows x 64 bytes = one
+// 128-wide K block) arrive unswizzled; converter warps widen them to int8, values unchanged, in
+// the 128-byte swizzled layout of the MMA's A operand, so the MMA is the same exact kind::i8
+// product against the activation planes.  And since every K block is one scale group, each K
+// block accumulates into an accumulator of its own (a ring of kD4Bufs in TMEM) that the epilogue
+// reads at once, scales by its group scale and adds into fp32 registers.
+//
+// Shared memory: kD4Slots widened A tiles (16 KB each), then the TMA ring whose stages hold the
+// packed tiles and the plane tiles of kbs K blocks (so that the bytes in flight are packed ones).
+// Warps: 0 TMA producer, 1 MMA issuer, 2-5 epilogue, 6-9 converters (one per SM sub-partition).
+constexpr int kD4Threads = 320;
+constexpr int kD4Bufs = 8;
+constexpr int kD4Slots = 4;
+constexpr int kD4RawBytes = 128 * 64;  // packed tile: 128 rows x 128 int4
+constexpr size_t kD4SlotBytes = (size_t)kD4Slots * 128 * 128;
+
+struct D4Ctl {
+  uint64_t raw[kDsMaxStages];    // packed tiles landed (TMA bytes)
+  uint64_t full[kDsMaxStages];   // plane tiles landed (TMA bytes)
+  uint64_t empty[kDsMaxStages];  // stage free again (MMA commit)
+  uint64_t afull[kD4Slots];      // widened A tile written (four converter warps)
+  uint64_t aempty[kD4Slots];     // widened A tile read (MMA commit)
+  uint64_t tfull[kD4Bufs];       // one K block's accumulator complete (MMA commit)
+  uint64_t tempty[kD4Bufs];      // that accumulator read (four epilogue warps)
+  uint64_t drain;
+  uint32_t tmem;
+  int abort;
+  int issued;    // stages issued / consumed, for the error path
+  int consumed;
+  int first;
+  int ntouched;
+  int32_t off[kMaxExperts + 1];
+  int32_t touched[kMaxExperts];
+  int32_t pre[2][kMaxExperts + 1];
+  int32_t cpre[kMaxExperts + 1];
+};
+static_assert(sizeof(D4Ctl) <= kDsCtlBytes, "int4 stream control block");
+
+// One stage: plane tiles of its kbs K blocks, then their packed weight tiles.
+__device__ __forceinline__ uint32_t d4_plane_bytes(const DecStreamParams& p) { return (uint32_t)(2 * p.nt8) * 128u; }
+__device__ __forceinline__ uint8_t* d4_raw(const DecStreamParams& p, uint8_t* stage, int j) {
+  return stage + (size_t)p.kbs * d4_plane_bytes(p) + (size_t)j * kD4RawBytes;
+}
+
+// Widen one packed word (8 int4, element 2j in the low nibble of byte j) to 8 int8 in order.
+__device__ __forceinline__ uint2 widen_int4x8(uint32_t w) {
+  // nibbles biased by 8 (q + 8 in [0, 15]), even elements in lo, odd elements in hi
+  const uint32_t lo = (w & 0x0F0F0F0Fu) ^ 0x08080808u;
+  const uint32_t hi = ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+  uint32_t a = __byte_perm(lo, hi, 0x5140);  // elements 0..3
+  uint32_t b = __byte_perm(lo, hi, 0x7362);  // elements 4..7
+  // per byte: (u + 0x78) ^ 0x80 = u - 8 (mod 256), no carry between bytes since u + 0x78 <= 0x87
+  a = (a + 0x78787878u) ^ 0x80808080u;
+  b = (b + 0x78787878u) ^ 0x80808080u;
+  return make_uint2(a, b);
+}
+
+// The K blocks of an item, in the rotated order every role walks them.
+struct D4Walk {
+  int kbeg, nkb;
+  __device__ D4Walk(const DecStreamParams& p, const DecItem& it) {
+    kbeg = it.split * p.kspan;
+    const int kend = min(p.K, kbeg + p.kspan);
+    nkb = (kend - kbeg + 127) / 128;
+  }
+};
+
+template <bool kGateUp>
+__device__ bool d4_produce(const DecStreamParams& p, uint8_t* ring, D4Ctl& c, int S) {
+  const uint32_t pb = d4_plane_bytes(p);
+  const uint64_t policy = l2_evict_first_policy();
+  DsRing r;
+  DecItem it;
+  for (int L = c.first; dec_item<kGateUp>(p, c, 0, L, it); L += gridDim.x) {
+    const D4Walk w(p, it);
+    int kb = L % w.nkb;
+    for (int i = 0; i < w.nkb; i += p.kbs) {
+      const int nk = min(p.kbs, w.nkb - i);
+      if (!ds_wait(&c.empty[r.s], r.ph ^ 1u, &c.abort)) return false;
+      uint8_t* st = ring + (size_t)r.s * p.stage_bytes;
+      mbar_arrive_expect_tx(&c.raw[r.s], (uint32_t)nk * kD4RawBytes);
+      mbar_arrive_expect_tx(&c.full[r.s], (uint32_t)nk * pb);
+      for (int j = 0; j < nk; ++j, kb = (kb + 1 == w.nkb) ? 0 : kb + 1) {
+        const int kx = w.kbeg + kb * 128;  // K element; the packed tile starts at byte kx / 2
+        uint8_t* rw = d4_raw(p, st, j);
+        if (kGateUp) tma_load_4d_hint(rw, &p.mapW, &c.raw[r.s], kx / 2, it.tile * 128, it.mat, it.e, policy);
+        else tma_load_3d_hint(rw, &p.mapW, &c.raw[r.s], kx / 2, it.tile * 128, it.e, policy);
+        uint8_t* pl = st + (size_t)j * pb;
+        tma_load_2d(pl, &p.mapHi, &c.full[r.s], kx, it.row0);
+        tma_load_2d(pl + p.nt8 * 128, &p.mapLo, &c.full[r.s], kx, it.row0);
+      }
+      c.issued = r.n + 1;
+      r.advance(S);
+    }
+  }
+  return true;
+}
+
+// Converter warps (warp cw = 0..3 of them): every K block, packed tile -> widened A tile in the
+// next slot.  Each warp waits for itself (warp-uniform decisions, no barrier between the warps)
+// and arrives on the slot's barrier once its share is written.
+template <bool kGateUp>
+__device__ bool d4_convert(const DecStreamParams& p, uint8_t* slots, uint8_t* ring, D4Ctl& c, int S, int cw, int lane) {
+  DsRing r;
+  uint32_t ka = 0;  // K blocks converted (slot ring position)
+  DecItem it;
+  for (int L = c.first; dec_item<kGateUp>(p, c, 0, L, it); L += gridDim.x) {
+    const D4Walk w(p, it);
+    for (int i = 0; i < w.nkb; i += p.kbs) {
+      const int nk = min(p.kbs, w.nkb - i);
+      if (!__all_sync(0xffffffffu, ds_wait(&c.raw[r.s], r.ph, &c.abort))) return false;
+      uint8_t* st = ring + (size_t)r.s * p.stage_bytes;
+      for (int j = 0; j < nk; ++j, ++ka) {
+        const uint32_t a = ka % kD4Slots, aph = (ka / kD4Slots) & 1u;
+        if (!__all_sync(0xffffffffu, ds_wait(&c.aempty[a], aph ^ 1u, &c.abort))) return false;
+        const uint8_t* rw = d4_raw(p, st, j);
+        uint8_t* at = slots + (size_t)a * 128 * 128;
+        // this warp's 32 rows; a task is (row, 16-byte output chunk), so one instruction of the
+        // warp reads 256 contiguous packed bytes (4 rows) and writes 4 whole swizzled rows
+#pragma unroll
+        for (int t8 = 0; t8 < 8; ++t8) {
+          const int row = cw * 32 + t8 * 4 + (lane >> 3), ch = lane & 7;
+          const uint2 v = *reinterpret_cast<const uint2*>(rw + row * 64 + ch * 8);
+          const uint2 e0 = widen_int4x8(v.x), e1 = widen_int4x8(v.y);
+          *reinterpret_cast<uint4*>(at + row * 128 + ((ch ^ (row & 7)) << 4)) = make_uint4(e0.x, e0.y, e1.x, e1.y);
+        }
+        // the tensor core reads the tile through the async proxy
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c.afull[a]);
+      }
+      r.advance(S);
+    }
+  }
+  return true;
+}
+
+template <bool kGateUp>
+__device__ bool d4_mma(const DecStreamParams& p, uint8_t* slots, uint8_t* ring, D4Ctl& c, int S, uint32_t tmem) {
+  const int N = 2 * p.nt8;
+  const uint32_t idesc = idesc_s8_s32(128, N);
+  const uint32_t pb = d4_plane_bytes(p);
+  DsRing r;
+  uint32_t kc = 0;  // K blocks issued (slot and accumulator ring position)
+  DecItem it;
+  for (int L = c.first; dec_item<kGateUp>(p, c, 0, L, it); L += gridDim.x) {
+    const D4Walk w(p, it);
+    for (int i = 0; i < w.nkb; i += p.kbs) {
+      const int nk = min(p.kbs, w.nkb - i);
+      if (!ds_wait(&c.full[r.s], r.ph, &c.abort)) return false;
+      const uint32_t st = smem_u32(ring + (size_t)r.s * p.stage_bytes);
+      for (int j = 0; j < nk; ++j, ++kc) {
+        const uint32_t a = kc % kD4Slots, aph = (kc / kD4Slots) & 1u;
+        const uint32_t b = kc % kD4Bufs, bph = (kc / kD4Bufs) & 1u;
+        if (!ds_wait(&c.afull[a], aph, &c.abort) || !ds_wait(&c.tempty[b], bph ^ 1u, &c.abort)) return false;
+        tc_fence_after();
+        const uint32_t at = smem_u32(slots + (size_t)a * 128 * 128);
+        const uint32_t dbase = tmem + b * (uint32_t)N;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_i8(dbase, smem_desc_sw128(at + kk * 32), smem_desc_sw128(st + j * pb + kk * 32), idesc, kk ? 1u : 0u);
+        tc_commit(&c.aempty[a]);
+        tc_commit(&c.tfull[b]);
+      }
+      tc_commit(&c.empty[r.s]);
+      c.consumed = r.n + 1;
+      r.advance(S);
+    }
+  }
+  return true;
+}
+
+// Epilogue: per K block, the accumulator scaled by that block's group scale is added into fp32
+// registers (one per token of the chunk); per item the sums times the plane scale are written.
+template <bool kGateUp>
+__device__ bool d4_epilogue(const DecStreamParams& p, D4Ctl& c, uint32_t tmem, int warp, int lane) {
+  const int q = warp & 3;
+  const int N = 2 * p.nt8;
+  uint32_t kc = 0;
+  DecItem it;
+  for (int L = c.first; dec_item<kGateUp>(p, c, 0, L, it); L += gridDim.x) {
+    const D4Walk w(p, it);
+    const int kb0 = L % w.nkb;
+    const int o = it.tile * 128 + q * 32 + lane;
+    const bool vo = o < p.out_rows;
+    // group scales of this matrix: [K / 128][out_rows], matrices W1 | W3 | W2 of each expert
+    const int m = kGateUp ? it.mat : 2;
+    const float* sg = p.wscale + (size_t)it.e * (3 * (size_t)p.d * p.f / 128) +
+                      (size_t)m * ((size_t)p.d * p.f / 128) + (vo ? o : 0);
+    auto group_scale = [&](int i) {  // scale of the i-th K block of the item's walk
+      const int g = w.kbeg / 128 + (kb0 + i) % w.nkb;
+      return (vo && i < w.nkb) ? __ldg(sg + (size_t)g * p.out_rows) : 0.f;
+    };
+    float acc[32];
+#pragma unroll
+    for (int t = 0; t < 32; ++t) acc[t] = 0.f;
+    float sc[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) sc[u] = group_scale(u);
+    for (int i0 = 0; i0 < w.nkb; i0 += 8) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u;
+        if (i >= w.nkb) break;
+        const uint32_t b = kc % kD4Bufs, bph = (kc / kD4Bufs) & 1u;
+        ++kc;
+        if (!__all_sync(0xffffffffu, ds_wait(&c.tfull[b], bph, &c.abort))) return false;
+        tc_fence_after();
+        const float s = sc[u];
+        sc[u] = group_scale(i + 8);  // the scale 8 blocks ahead, loaded while these are in use
+        const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + b * (uint32_t)N;
+        // columns [0, nt8) hold the hi plane, [nt8, 2 nt8) the lo plane of the same tokens
+        if (p.nt8 == 8) {
+          float v[16];
+          tmem_ld16(tb, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int t = 0; t < 8; ++t)
+            acc[t] = fmaf(s, (float)__float_as_int(v[t]) + (float)__float_as_int(v[8 + t]) * (1.0f / 254.0f), acc[t]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; j += 16) {
+            if (j >= p.nt8) break;
+            float vh[16], vl[16];
+            tmem_ld16(tb + j, vh);
+            tmem_ld16(tb + p.nt8 + j, vl);
+            tmem_ld_wait();
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+              acc[j + t] = fmaf(s, (float)__float_as_int(vh[t]) + (float)__float_as_int(vl[t]) * (1.0f / 254.0f),
+                                acc[j + t]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c.tempty[b]);
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+      if (t >= it.ntok || !vo) continue;
+      const int row = it.row0 + t;
+      const float v = __ldcg(p.rscale + (size_t)it.split * p.rscale_split_stride + row) * acc[t];
+      if (kGateUp) p.GU[(((size_t)it.split * 2 + it.mat) * p.R + row) * p.f + o] = v;
+      else p.Ypart[((size_t)it.split * p.R + row) * p.d + o] = v;
+    }
+  }
+  return true;
+}
+
+template <bool kGateUp>
+__global__ void __launch_bounds__(kD4Threads, 1) dec_stream4_kernel(const __grid_constant__ DecStreamParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {
+    pdl_wait();
+    if (threadIdx.x == 0) atomicOr(p.err, kErrWaitTimeout);
+    return;
+  }
+  const int S = p.stages;
+  uint8_t* slots = smem;
+  uint8_t* ring = smem + kD4SlotBytes;
+  D4Ctl& c = *reinterpret_cast<D4Ctl*>(ring + (size_t)S * p.stage_bytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t tmem_cols = p.nt8 == 8 ? 128u : (p.nt8 == 16 ? 256u : 512u);  // kD4Bufs x 2 nt8
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&c.raw[s], 1);
+      mbar_init(&c.full[s], 1);
+      mbar_init(&c.empty[s], 1);
+    }
+    for (int a = 0; a < kD4Slots; ++a) {
+      mbar_init(&c.afull[a], 4);
+      mbar_init(&c.aempty[a], 1);
+    }
+    for (int b = 0; b < kD4Bufs; ++b) {
+      mbar_init(&c.tfull[b], 1);
+      mbar_init(&c.tempty[b], 4);
+    }
+    mbar_init(&c.drain, 1);
+    c.abort = 0;
+    c.issued = 0;
+    c.consumed = 0;
+    c.first = blockIdx.x;
+    mbar_fence_init();
+    tma_prefetch_desc(&p.mapW);
+    tma_prefetch_desc(&p.mapHi);
+    tma_prefetch_desc(&p.mapLo);
+  }
+  pdl_wait();
+  if (warp == 1) {
+    tmem_alloc(&c.tmem, tmem_cols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  const DecStreamParams* phases[1] = {&p};
+  ds_items(phases, 1, c, p.offsets);  // starts and ends with a CTA barrier
+  const uint32_t tmem = c.tmem;
+  if (warp == 0) {
+    if (lane == 0 && !d4_produce<kGateUp>(p, ring, c, S)) ds_abort(c, p.err);
+    pdl_trigger();
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      if (!d4_mma<kGateUp>(p, slots, ring, c, S, tmem)) ds_abort(c, p.err);
+      tc_commit(&c.drain);
+      mbar_wait_bounded(&c.drain, 0);
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    if (!d4_epilogue<kGateUp>(p, c, tmem, warp, lane) && lane == 0) ds_abort(c, p.err);
+  } else {
+    if (!d4_convert<kGateUp>(p, slots, ring, c, S, warp - 6, lane) && lane == 0) ds_abort(c, p.err);
+  }
+  // error path: copies issued but never consumed land before the CTA exits; then TMEM is freed
+  __syncthreads();
+  if (threadIdx.x == 0 && c.abort) {
+    for (int i = c.consumed; i < c.issued; ++i) {
+      if (!mbar_wait_bounded(&c.raw[i % S], (uint32_t)(i / S) & 1u)) break;
+      if (!mbar_wait_bounded(&c.full[i % S], (uint32_t)(i / S) & 1u)) break;
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, tmem_cols);
+  }
+}
+
 // ------------------------------------------------------------------------- fused decode kernel
 // The whole int8 expert stage in one cooperative launch (all CTAs resident, one per SM):
 //   phase 1  gate/up weight stream -> GU partials                 (as dec_stream_kernel<true>)
@@ -576,7 +942,12 @@ struct alignas(64) DecFusedParams {
   int32_t* counts;          // [E]
   int32_t* offsets;         // [E+1]
   int32_t* src_row;         // [T*k]
+  int8_t* xhi;              // [R, d] x planes written by the routing phase (the buffers p.gu reads)
+  int8_t* xlo;
   float* xscale;            // [R] scales of the x planes (the buffer p.gu.rscale reads)
+  // dec_flow_kernel: completion counters, zero between launches (each launch returns them to 0)
+  int32_t* unit_ctr;        // [chunks x dsplit] H units: gate/up arrivals, then kUnitReady + uses
+  int32_t* tile_ctr;        // [ceil(d / 128)] output tiles: down arrivals
 };
 // up to this many tokens every CTA of the fused kernel routes all of them itself
 constexpr int kRedundantT = 1;
@@ -835,8 +1206,8 @@ __device__ void fused_route(const DecFusedParams& p, uint8_t* smem, DsCtl& c) {
 #pragma unroll
       for (int j = 0; j < kMaxTopK; ++j) {
         if (j < k) {
-          reinterpret_cast<uint2*>(p.hhi + (size_t)rows[j] * d)[v] = make_uint2(hw[0], hw[1]);
-          reinterpret_cast<uint2*>(p.hlo + (size_t)rows[j] * d)[v] = make_uint2(lw[0], lw[1]);
+          reinterpret_cast<uint2*>(p.xhi + (size_t)rows[j] * d)[v] = make_uint2(hw[0], hw[1]);
+          reinterpret_cast<uint2*>(p.xlo + (size_t)rows[j] * d)[v] = make_uint2(lw[0], lw[1]);
         }
       }
     }
@@ -844,6 +1215,101 @@ __device__ void fused_route(const DecFusedParams& p, uint8_t* smem, DsCtl& c) {
   // the planes are read next by TMA copies of other CTAs; the caller arrives on the planes
   // barrier after its next CTA barrier
   fence_proxy_async_global();
+}
+
+// H for one (row r, down split sp) unit, by the 128 epilogue threads of a CTA (tid 0..127): h =
+// silu(g) * u over the columns of split sp, from the gate/up partials summed in split order, rounded
+// to bf16, then split into int8 planes with one scale for the unit.  The caller makes the planes
+// visible to the async proxy and publishes them.
+__device__ void h_row_planes(const DecFusedParams& p, DsCtl& c, int r, int sp, int tid, int lane) {
+  float* red = c.red;
+  const int R = p.gu.R, f = p.gu.f, gs = p.gu.nsplit, ds = p.dn.nsplit;
+  const size_t plane = (size_t)R * f;
+  const int span = f / ds, k0 = sp * span;
+  const float* g0 = p.gu.GU + (size_t)r * f + k0;
+  // h for 4 consecutive columns: all gsplit partials are loaded before they are summed (in
+  // split order), so one pass is one memory round trip per step
+  auto hvals = [&](int j, float (&hv)[4]) {
+    float4 gv[kDecGateSplitMax], uv[kDecGateSplitMax];
+#pragma unroll
+    for (int s2 = 0; s2 < kDecGateSplitMax; ++s2) {
+      if (s2 < gs) {
+        gv[s2] = __ldcg(reinterpret_cast<const float4*>(g0 + (size_t)(2 * s2) * plane + j));
+        uv[s2] = __ldcg(reinterpret_cast<const float4*>(g0 + (size_t)(2 * s2 + 1) * plane + j));
+      }
+    }
+    float4 g = gv[0], uu = uv[0];
+#pragma unroll
+    for (int s2 = 1; s2 < kDecGateSplitMax; ++s2) {
+      if (s2 < gs) {
+        g.x += gv[s2].x; g.y += gv[s2].y; g.z += gv[s2].z; g.w += gv[s2].w;
+        uu.x += uv[s2].x; uu.y += uv[s2].y; uu.z += uv[s2].z; uu.w += uv[s2].w;
+      }
+    }
+    hv[0] = __bfloat162float(__float2bfloat16_rn(silu_mul(g.x, uu.x)));
+    hv[1] = __bfloat162float(__float2bfloat16_rn(silu_mul(g.y, uu.y)));
+    hv[2] = __bfloat162float(__float2bfloat16_rn(silu_mul(g.z, uu.z)));
+    hv[3] = __bfloat162float(__float2bfloat16_rn(silu_mul(g.w, uu.w)));
+  };
+  // A short unit (at most kHKeep steps per thread, e.g. one token's 896-column unit) keeps its
+  // h values in registers between the max and the split; a longer one makes two passes over
+  // the partials (holding every step measured slower: the kernel's register count doubled).
+  constexpr int kHKeep = 2;
+  const bool keep = span <= 128 * 4 * kHKeep;
+  float hk[kHKeep][4];
+  float mx = 0.f;
+  if (keep) {
+#pragma unroll
+    for (int it = 0; it < kHKeep; ++it) {
+      const int j = tid * 4 + it * 128 * 4;
+      if (j < span) {
+        hvals(j, hk[it]);
+        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(hk[it][0]), fabsf(hk[it][1])), fmaxf(fabsf(hk[it][2]), fabsf(hk[it][3]))));
+      }
+      asm volatile("" ::: "memory");  // one step's partials in registers at a time
+    }
+  } else {
+    for (int j = tid * 4; j < span; j += 128 * 4) {
+      float hv[4];
+      hvals(j, hv);
+      mx = fmaxf(mx, fmaxf(fmaxf(fabsf(hv[0]), fabsf(hv[1])), fmaxf(fabsf(hv[2]), fabsf(hv[3]))));
+    }
+  }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  if (lane == 0) red[tid >> 5] = mx;
+  epi_sync();
+  mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  epi_sync();  // red[] is rewritten by the next unit
+  const float a = plane_scale(mx), inv_a = __frcp_rn(a);  // correctly rounded 1 / a
+  if (tid == 0) p.hscale[(size_t)sp * R + r] = a;
+  int8_t* hrow = p.hhi + (size_t)r * f + k0;
+  int8_t* lrow = p.hlo + (size_t)r * f + k0;
+  auto put = [&](int j, const float (&hv)[4]) {
+    uint32_t hw = 0u, lw = 0u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      int qh, ql;
+      split_planes(hv[i], a, inv_a, qh, ql);
+      hw |= ((uint32_t)qh & 0xffu) << (8 * i);
+      lw |= ((uint32_t)ql & 0xffu) << (8 * i);
+    }
+    *reinterpret_cast<uint32_t*>(hrow + j) = hw;
+    *reinterpret_cast<uint32_t*>(lrow + j) = lw;
+  };
+  if (keep) {
+#pragma unroll
+    for (int it = 0; it < kHKeep; ++it) {
+      const int j = tid * 4 + it * 128 * 4;
+      if (j < span) put(j, hk[it]);
+    }
+  } else {
+    for (int j = tid * 4; j < span; j += 128 * 4) {  // the same values again, now split
+      float hv[4];
+      hvals(j, hv);
+      put(j, hv);
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_constant__ DecFusedParams p) {
@@ -942,96 +1408,10 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_c
     ok = grid_barrier(kBarGU);
     if (ok) {
       // phase 2: H planes, one (row, down split) unit per round
-      float* red = c.red;
-      const int R = p.gu.R, f = p.gu.f, gs = p.gu.nsplit, ds = p.dn.nsplit;
-      const size_t plane = (size_t)R * f;
-      const int span = f / ds;
+      const int R = p.gu.R, ds = p.dn.nsplit;
       for (int u = blockIdx.x; u < R * ds; u += G) {
-        const int r = u / ds, sp = u - r * ds, k0 = sp * span;
-        const float* g0 = p.gu.GU + (size_t)r * f + k0;
-        // h for 4 consecutive columns: all gsplit partials are loaded before they are summed (in
-        // split order), so one pass is one memory round trip per step
-        auto hvals = [&](int j, float (&hv)[4]) {
-          float4 gv[kDecGateSplitMax], uv[kDecGateSplitMax];
-#pragma unroll
-          for (int s2 = 0; s2 < kDecGateSplitMax; ++s2) {
-            if (s2 < gs) {
-              gv[s2] = __ldcg(reinterpret_cast<const float4*>(g0 + (size_t)(2 * s2) * plane + j));
-              uv[s2] = __ldcg(reinterpret_cast<const float4*>(g0 + (size_t)(2 * s2 + 1) * plane + j));
-            }
-          }
-          float4 g = gv[0], uu = uv[0];
-#pragma unroll
-          for (int s2 = 1; s2 < kDecGateSplitMax; ++s2) {
-            if (s2 < gs) {
-              g.x += gv[s2].x; g.y += gv[s2].y; g.z += gv[s2].z; g.w += gv[s2].w;
-              uu.x += uv[s2].x; uu.y += uv[s2].y; uu.z += uv[s2].z; uu.w += uv[s2].w;
-            }
-          }
-          hv[0] = __bfloat162float(__float2bfloat16_rn(silu_mul(g.x, uu.x)));
-          hv[1] = __bfloat162float(__float2bfloat16_rn(silu_mul(g.y, uu.y)));
-          hv[2] = __bfloat162float(__float2bfloat16_rn(silu_mul(g.z, uu.z)));
-          hv[3] = __bfloat162float(__float2bfloat16_rn(silu_mul(g.w, uu.w)));
-        };
-        // A short unit (at most kHKeep steps per thread, e.g. one token's 896-column unit) keeps its
-        // h values in registers between the max and the split; a longer one makes two passes over
-        // the partials (holding every step measured slower: the kernel's register count doubled).
-        constexpr int kHKeep = 2;
-        const bool keep = span <= 128 * 4 * kHKeep;
-        float hk[kHKeep][4];
-        float mx = 0.f;
-        if (keep) {
-#pragma unroll
-          for (int it = 0; it < kHKeep; ++it) {
-            const int j = tid * 4 + it * 128 * 4;
-            if (j < span) {
-              hvals(j, hk[it]);
-              mx = fmaxf(mx, fmaxf(fmaxf(fabsf(hk[it][0]), fabsf(hk[it][1])), fmaxf(fabsf(hk[it][2]), fabsf(hk[it][3]))));
-            }
-            asm volatile("" ::: "memory");  // one step's partials in registers at a time
-          }
-        } else {
-          for (int j = tid * 4; j < span; j += 128 * 4) {
-            float hv[4];
-            hvals(j, hv);
-            mx = fmaxf(mx, fmaxf(fmaxf(fabsf(hv[0]), fabsf(hv[1])), fmaxf(fabsf(hv[2]), fabsf(hv[3]))));
-          }
-        }
-#pragma unroll
-        for (int off = 16; off; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        if (lane == 0) red[tid >> 5] = mx;
-        epi_sync();
-        mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-        epi_sync();  // red[] is rewritten by the next unit
-        const float a = plane_scale(mx), inv_a = __frcp_rn(a);  // correctly rounded 1 / a
-        if (tid == 0) p.hscale[(size_t)sp * R + r] = a;
-        int8_t* hrow = p.hhi + (size_t)r * f + k0;
-        int8_t* lrow = p.hlo + (size_t)r * f + k0;
-        auto put = [&](int j, const float (&hv)[4]) {
-          uint32_t hw = 0u, lw = 0u;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            int qh, ql;
-            split_planes(hv[i], a, inv_a, qh, ql);
-            hw |= ((uint32_t)qh & 0xffu) << (8 * i);
-            lw |= ((uint32_t)ql & 0xffu) << (8 * i);
-          }
-          *reinterpret_cast<uint32_t*>(hrow + j) = hw;
-          *reinterpret_cast<uint32_t*>(lrow + j) = lw;
-        };
-        if (keep) {
-#pragma unroll
-          for (int it = 0; it < kHKeep; ++it) {
-            const int j = tid * 4 + it * 128 * 4;
-            if (j < span) put(j, hk[it]);
-          }
-        } else {
-          for (int j = tid * 4; j < span; j += 128 * 4) {  // the same values again, now split
-            float hv[4];
-            hvals(j, hv);
-            put(j, hv);
-          }
-        }
+        const int r = u / ds, sp = u - r * ds;
+        h_row_planes(p, c, r, sp, tid, lane);
       }
       fence_proxy_async_global();  // the planes are read next by TMA copies of other CTAs
     }
@@ -1085,6 +1465,289 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_c
   else __syncthreads();
 }
 
+// ------------------------------------------------------------------------- dataflow decode kernel
+// The same stage as dec_fused_kernel for up to 64 tokens, with the three grid barriers replaced by
+// completion counters, so that no CTA waits for the slowest one between phases:
+//   * An H unit is (token chunk of one expert, down split): the H columns of that split for the
+//     chunk's rows.  Every gate/up item adds one arrival to the unit its output tile falls in; the
+//     CTA whose arrival completes the count computes the unit (the rows' H planes and scales) in
+//     its epilogue warps and marks the unit ready.
+//   * A down item's weight copies go out at once; the copies of its H planes wait for its unit
+//     (held in the ring, in order, while other copies proceed), so a CTA moves on to its down
+//     items as soon as its gate/up items are done.
+//   * Every down item adds one arrival to its 128-column output tile; the CTA that completes the
+//     tile sums the tile's partials in fixed order (splits, then slots) and writes y.
+// The counters return to zero by the end of every launch: the CTA that completes a tile resets
+// it; an H unit counts its gate/up arrivals, is set to kUnitReady, counts one use per down item,
+// and the last use resets it.  Sums and orders are those of dec_fused_kernel, so results are
+// bit-identical to it.
+constexpr int32_t kUnitReady = 1 << 24;
+
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int32_t* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ int atom_add_relaxed_gpu(int32_t* p, int v) {
+  int old;
+  asm volatile("atom.relaxed.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ void st_release_gpu(int32_t* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st_relaxed_gpu(int32_t* p, int v) {
+  asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Counts of the flow kernel, the same in every CTA.
+struct FlowCounts {
+  int tpu;     // gate/up output tiles per H unit
+  int need_g;  // gate/up arrivals that complete an H unit
+  int need_c;  // down items that use an H unit
+  int need_y;  // down arrivals that complete an output tile
+};
+__device__ __forceinline__ FlowCounts flow_counts(const DecFusedParams& p, const DsCtl& c) {
+  FlowCounts n;
+  const int span = p.gu.f / p.dn.nsplit;
+  n.tpu = (span + 127) / 128;
+  n.need_g = n.tpu * 2 * p.gu.nsplit;
+  n.need_c = (p.dn.d + 127) / 128;
+  n.need_y = c.cpre[c.ntouched] * p.dn.nsplit;
+  return n;
+}
+
+// Producer of the down phase: weight copies at once; the H-plane copies of a stage once its unit
+// is ready.  Stages whose unit is not ready yet are held in order (at most a ring-full): the
+// MMA consumes stages in order, so the oldest stage in flight is released (waiting for its unit)
+// before the producer waits for its ring slot.  The first stage of each item uses the unit once.
+__device__ bool flow_produce_down(const DecFusedParams& fp, uint8_t* smem, DsCtl& c, int S, DsRing& r) {
+  const DecStreamParams& p = fp.dn;
+  const FlowCounts nc = flow_counts(fp, c);
+  const uint32_t blk_bytes = 128u * 128u + (uint32_t)(2 * p.nt8) * 128u;
+  const uint64_t policy = l2_evict_first_policy();
+  int qh = 0, qn = 0;  // held stages: a queue of up to S entries in c.defer_*
+  auto ready = [&](int u) { return ld_acquire(fp.unit_ctr + u) >= kUnitReady; };
+  auto use = [&](int u) {  // after the unit was seen ready: make its planes visible to TMA, count the use
+    fence_proxy_async_global();
+    if (atom_add_relaxed_gpu(fp.unit_ctr + u, 1) == kUnitReady + nc.need_c - 1) st_relaxed_gpu(fp.unit_ctr + u, 0);
+  };
+  auto release_head = [&]() {
+    uint8_t* st = smem + (size_t)c.defer_s[qh] * p.stage_bytes;
+    for (int j = 0; j < c.defer_nk[qh]; ++j)
+      ds_load_planes(p, st, &c.full[c.defer_s[qh]], j, c.defer_kx[qh][j], c.defer_row[qh]);
+    qh = qh + 1 == S ? 0 : qh + 1;
+    --qn;
+  };
+  auto wait_unit = [&](int u) -> bool {
+    const unsigned long long t0 = global_ns();
+    while (!ready(u)) {
+      if (*(volatile int*)&c.abort || global_ns() - t0 > kWaitTimeoutNs) return false;
+      __nanosleep(32);
+    }
+    return true;
+  };
+  bool ok = true;
+  DecItem it;
+  for (int L = c.first; ok && dec_item<false>(p, c, 1, L, it); L += gridDim.x) {
+    const int u = it.gchunk * p.nsplit + it.split;
+    const int kbeg = it.split * p.kspan, kend = min(p.K, kbeg + p.kspan);
+    const int nkb = (kend - kbeg + 127) / 128;
+    int kb = L % nkb;
+    for (int i = 0; i < nkb; i += p.kbs) {
+      const bool fresh = i == 0;
+      // release held stages whose units are ready (in order; a later stage of an item whose first
+      // stage was released needs no check)
+      while (qn > 0 && (!c.defer_fresh[qh] || ready(c.defer_unit[qh]))) {
+        if (c.defer_fresh[qh]) use(c.defer_unit[qh]);
+        release_head();
+      }
+      // the stage in the slot about to be reused must have its planes on the way
+      while (ok && qn > 0 && c.defer_n[qh] <= r.n - S) {
+        if (c.defer_fresh[qh]) {
+          ok = wait_unit(c.defer_unit[qh]);
+          if (ok) use(c.defer_unit[qh]);
+        }
+        release_head();  // issued even when the wait gave up, so that every issued stage completes
+      }
+      if (!ok || !ds_wait(&c.empty[r.s], r.ph ^ 1u, &c.abort)) {
+        ok = false;
+        break;
+      }
+      const int nk = min(p.kbs, nkb - i);
+      uint8_t* st = smem + (size_t)r.s * p.stage_bytes;
+      mbar_arrive_expect_tx(&c.full[r.s], (uint32_t)nk * blk_bytes);
+      int kxs[kDsMaxKbs];
+      for (int j = 0; j < nk; ++j, kb = (kb + 1 == nkb) ? 0 : kb + 1) {
+        kxs[j] = kbeg + kb * 128;
+        uint8_t* sw = st + (size_t)j * 128 * 128;
+        if (p.evict_first) tma_load_3d_hint(sw, &p.mapW, &c.full[r.s], kxs[j], it.tile * 128, it.e, policy);
+        else tma_load_3d(sw, &p.mapW, &c.full[r.s], kxs[j], it.tile * 128, it.e);
+      }
+      // with nothing held, a later stage of an item goes out at once (its first stage was
+      // released, so the unit is ready), and a first stage if its unit is ready
+      const bool now = qn == 0 && (!fresh || ready(u));
+      if (now) {
+        if (fresh) use(u);
+        for (int j = 0; j < nk; ++j) ds_load_planes(p, st, &c.full[r.s], j, kxs[j], it.row0);
+      } else {
+        const int t = qh + qn < S ? qh + qn : qh + qn - S;
+        c.defer_s[t] = r.s;
+        c.defer_nk[t] = nk;
+        for (int j = 0; j < nk; ++j) c.defer_kx[t][j] = kxs[j];
+        c.defer_row[t] = it.row0;
+        c.defer_unit[t] = u;
+        c.defer_n[t] = r.n;
+        c.defer_fresh[t] = fresh ? 1 : 0;
+        ++qn;
+      }
+      c.issued = r.n + 1;
+      r.advance(S);
+    }
+  }
+  // the rest of the held stages (their copies are issued even after a failed wait)
+  while (qn > 0) {
+    if (c.defer_fresh[qh] && ok) {
+      ok = wait_unit(c.defer_unit[qh]);
+      if (ok) use(c.defer_unit[qh]);
+    }
+    release_head();
+  }
+  return ok;
+}
+
+// The combine of one 128-column output tile for every token, by the 128 epilogue threads:
+// y[t][o] = sum_j w[t][j] * (sum over splits of Ypart[split][dst_row[t][j]][o]), in the order of
+// dec_fused_kernel's combine.
+__device__ void flow_combine_tile(const DecFusedParams& p, int dt, int tid) {
+  const int d = p.dn.d, ns = p.dn.nsplit, k = p.k;
+  const int o = dt * 128 + tid;
+  if (o >= d) return;
+  const size_t ss = (size_t)p.dn.R * d;
+  for (int t = 0; t < p.T; ++t) {
+    float acc = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const int rr = __ldcg(p.dst_row + (size_t)t * k + j);
+      const float wj = __ldcg(p.topk_w + (size_t)t * k + j);
+      const float* base = p.dn.Ypart + (size_t)rr * d + o;
+      float part = 0.f;
+      int sp = 0;
+      for (; sp + 8 <= ns; sp += 8) {
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = __ldcg(base + (size_t)(sp + i) * ss);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) part += v[i];
+      }
+      for (; sp < ns; ++sp) part += __ldcg(base + (size_t)sp * ss);
+      acc = fmaf(wj, part, acc);
+    }
+    p.y[(size_t)t * d + o] = __float2bfloat16_rn(acc);
+  }
+}
+
+__global__ void __launch_bounds__(kDsThreads, 1) dec_flow_kernel(const __grid_constant__ DecFusedParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int S = p.gu.stages;
+  DsCtl& c = *reinterpret_cast<DsCtl*>(smem + (size_t)S * p.gu.stage_bytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = gridDim.x;
+  const bool aligned = (smem_u32(smem) & 1023u) == 0;  // the 128-byte swizzle needs 1024-byte stages
+  const DecStreamParams* phases[2] = {&p.gu, &p.dn};
+  uint32_t planes_old = 0;  // thread 0: the planes barrier count before its arrival
+  if (aligned) {
+    ds_init(phases, 2, c, S);
+    if (p.route_in_kernel) {
+      fused_route(p, smem, c);
+      if (threadIdx.x == 0) c.first = (int)((blockIdx.x + gridDim.x - (unsigned)min(p.T, (int)gridDim.x)) % gridDim.x);
+      ds_items(phases, 2, c, nullptr);
+      if (threadIdx.x == 0) planes_old = bar_arrive(&p.bar[kBarPlanes], G);
+    } else {
+      ds_items(phases, 2, c, p.gu.offsets);
+    }
+  }
+  const uint32_t tmem = aligned ? c.tmem : 0u;
+  if (!aligned) {
+    if (threadIdx.x == 0) {  // report, and arrive at the barriers the others wait on
+      atomicOr(p.gu.err, kErrWaitTimeout);
+      if (p.route_in_kernel == 1 && p.T > kRedundantT) bar_arrive(&p.bar[kBarRouter], G);
+      if (p.route_in_kernel) bar_arrive(&p.bar[kBarPlanes], G);
+    }
+  } else if (warp == 0) {
+    if (lane == 0) {
+      DsRing r;
+      bool ok = ds_produce<true>(p.gu, smem, c, S, 0, r, p.route_in_kernel != 0, [&] {
+        if (!grid_wait(&p.bar[kBarPlanes], bar_base(planes_old, G), G, &c.abort)) return false;
+        fence_proxy_async_global();
+        return true;
+      });
+      if (ok) ok = flow_produce_down(p, smem, c, S, r);
+      if (!ok) ds_abort(c, p.gu.err);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      DsRing r;
+      int iter = 0;
+      bool ok = ds_mma<true>(p.gu, smem, c, S, 0, r, iter, tmem);
+      if (ok) ok = ds_mma<false>(p.dn, smem, c, S, 1, r, iter, tmem);
+      if (!ok) ds_abort(c, p.gu.err);
+      tc_commit(&c.drain);
+      mbar_wait_bounded(&c.drain, 0);
+    }
+    __syncwarp();
+  } else {
+    const int tid = threadIdx.x - 64;  // 0..127
+    const FlowCounts nc = flow_counts(p, c);
+    int iter = 0;
+    // after a gate/up item: arrive on its H unit; the completing CTA computes the unit
+    // Both hooks decide in thread 0 and broadcast through shared memory, so the four warps take
+    // the same path (and pass the same named barriers): -1 once the CTA has aborted (a warp whose
+    // wait gave up sets the flag before its first barrier here), 1 if this CTA completed the
+    // counter, else 0.
+    // After a gate/up item: arrive on its H unit; the completing CTA computes the unit.
+    auto gu_done = [&](const DecItem& it, bool) -> bool {
+      const int sp = it.tile / nc.tpu;
+      const int u = it.gchunk * p.dn.nsplit + sp;
+      epi_sync();  // the four warps' partials of this item are written
+      if (tid == 0)
+        c.eflag = *(volatile int*)&c.abort ? -1 : (atom_add_acq_rel_gpu(p.unit_ctr + u, 1) == nc.need_g - 1 ? 1 : 0);
+      epi_sync();
+      const int v = *(volatile int*)&c.eflag;
+      if (v == 1) {
+        for (int r = it.row0; r < it.row0 + it.ntok; ++r) h_row_planes(p, c, r, sp, tid, lane);
+        fence_proxy_async_global();  // the planes are read next by TMA copies of other CTAs
+        epi_sync();
+        if (tid == 0) st_release_gpu(p.unit_ctr + u, kUnitReady);
+      }
+      return v >= 0;
+    };
+    // After a down item: arrive on its output tile; the completing CTA writes the tile of y.
+    auto dn_done = [&](const DecItem& it, bool) -> bool {
+      epi_sync();
+      if (tid == 0) {
+        c.eflag = *(volatile int*)&c.abort ? -1
+                                           : (atom_add_acq_rel_gpu(p.tile_ctr + it.tile, 1) == nc.need_y - 1 ? 1 : 0);
+        // the routing state the combine reads was written before every CTA's planes-barrier
+        // arrival: acquire the completed barrier directly
+        if (c.eflag == 1 && p.route_in_kernel) (void)ld_acquire(&p.bar[kBarPlanes]);
+      }
+      epi_sync();
+      const int v = *(volatile int*)&c.eflag;
+      if (v == 1) {
+        flow_combine_tile(p, it.tile, tid);
+        if (tid == 0) st_relaxed_gpu(p.tile_ctr + it.tile, 0);
+      }
+      return v >= 0;
+    };
+    bool ok = ds_epilogue<true>(p.gu, c, 0, iter, tmem, warp, lane, gu_done);
+    if (ok) ok = ds_epilogue<false>(p.dn, c, 1, iter, tmem, warp, lane, dn_done);
+    if (!__all_sync(0xffffffffu, ok) && lane == 0) ds_abort(c, p.gu.err);
+  }
+  if (aligned) ds_teardown(c, S);
+  else __syncthreads();
+}
+
 // K blocks per ring stage: COLIBRI_DEC_KB (1..4), default 2.
 int dec_kbs() {
   const char* v = getenv("COLIBRI_DEC_KB");
@@ -1131,6 +1794,11 @@ cudaError_t configure_dec_kernels() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(dec_stream_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(dec_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(dec_flow_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(dec_stream4_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(dec_stream4_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(dec_finish_h_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFinishMaxSmem);
   return e;
@@ -1206,6 +1874,79 @@ cudaError_t launch_dec_gateup(const int8_t* Xhi, const int8_t* Xlo, const float*
   return launch_stream<true>(p, s);
 }
 
+namespace {
+
+// Stream parameters of the int4 kernels: the packed weights are copied unswizzled, 64 bytes
+// (128 K elements) of 128 rows per tile; the stage holds kbs such tiles and their plane tiles.
+bool dec4_params(DecStreamParams& p, bool gateup, const int8_t* hi, const int8_t* lo, const float* rscale,
+                 int rscale_split_stride, const uint8_t* W, const float* scales, int64_t wstride, int d, int f, int E,
+                 const int32_t* offsets, int nsplit, float* out, int R, int max_rows_per_expert, uint32_t* err) {
+  memset(&p, 0, sizeof(p));
+  if (d % 128 || f % 128 || wstride % 256) return false;
+  if (gateup) {
+    const uint64_t dims[4] = {(uint64_t)d / 2, (uint64_t)f, 2, (uint64_t)E};
+    const uint64_t st[3] = {(uint64_t)d / 2, (uint64_t)f * d / 2, (uint64_t)wstride / 2};
+    const uint32_t box[4] = {64, 128, 1, 1};
+    if (!make_tmap(&p.mapW, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, 4, dims, st, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return false;
+  } else {
+    const uint64_t dims[3] = {(uint64_t)f / 2, (uint64_t)d, (uint64_t)E};
+    const uint64_t st[2] = {(uint64_t)f / 2, (uint64_t)wstride / 2};
+    const uint32_t box[3] = {64, 128, 1};
+    if (!make_tmap(&p.mapW, CU_TENSOR_MAP_DATA_TYPE_UINT8, W + (size_t)f * d, 3, dims, st, box,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+      return false;
+  }
+  p.wscale = scales;
+  p.rscale = rscale;
+  p.rscale_split_stride = rscale_split_stride;
+  p.offsets = offsets;
+  p.E = E;
+  p.d = d;
+  p.f = f;
+  p.out_rows = gateup ? f : d;
+  p.K = gateup ? d : f;
+  p.nsplit = nsplit;
+  p.kspan = p.K / nsplit;
+  p.nt8 = dec_nt8(max_rows_per_expert);
+  p.R = R;
+  if (gateup) p.GU = out;
+  else p.Ypart = out;
+  p.err = err;
+  if (!plane_maps(p, hi, lo, p.K)) return false;
+  p.stage_bytes = (uint32_t)((p.kbs * (2 * p.nt8 * 128 + kD4RawBytes) + 1023) / 1024 * 1024);
+  p.stages = (int)std::min<size_t>(kDsMaxStages, (kDsRingBytes - kD4SlotBytes) / p.stage_bytes);
+  return p.stages >= 2;
+}
+
+template <bool kGateUp>
+cudaError_t launch_stream4(const DecStreamParams& p, cudaStream_t s) {
+  const size_t smem = kD4SlotBytes + (size_t)p.stages * p.stage_bytes + kDsCtlBytes;
+  return launch_kernel(dec_stream4_kernel<kGateUp>, dim3(sm_count_current()), dim3(kD4Threads), smem, s, 1, p);
+}
+
+}  // namespace
+
+cudaError_t launch_dec4_gateup(const int8_t* Xhi, const int8_t* Xlo, const float* xscale, const uint8_t* W,
+                               const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
+                               int nsplit, float* GU, int R, int max_rows_per_expert, uint32_t* err, cudaStream_t s) {
+  DecStreamParams p;
+  if (!dec4_params(p, true, Xhi, Xlo, xscale, 0, W, scales, wstride, d, f, E, offsets, nsplit, GU, R,
+                   max_rows_per_expert, err))
+    return cudaErrorInvalidValue;
+  return launch_stream4<true>(p, s);
+}
+
+cudaError_t launch_dec4_down(const int8_t* Hhi, const int8_t* Hlo, const float* hscale, const uint8_t* W,
+                             const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
+                             int nsplit, int R, float* Ypart, int max_rows_per_expert, uint32_t* err, cudaStream_t s) {
+  DecStreamParams p;
+  if (!dec4_params(p, false, Hhi, Hlo, hscale, R, W, scales, wstride, d, f, E, offsets, nsplit, Ypart, R,
+                   max_rows_per_expert, err))
+    return cudaErrorInvalidValue;
+  return launch_stream4<false>(p, s);
+}
+
 cudaError_t launch_dec_finish_h(const float* GU, int gsplit, int R, int f, int dsplit, int8_t* hi, int8_t* lo,
                                 float* scale, cudaStream_t s) {
   if (R <= 0) return cudaSuccess;
@@ -1233,16 +1974,22 @@ cudaError_t launch_dec_fused(const DecFusedArgs& a, cudaStream_t s) {
   DecFusedParams p;
   memset(&p, 0, sizeof(p));
   const int R = a.T * a.k;
+  // the dataflow plan writes H into planes of its own (the x planes may still be read meanwhile)
+  const bool flow = a.flow && a.unit_ctr && a.tile_ctr && a.hplanes_hi && a.hplanes_lo && a.hplanes_scale &&
+                    a.T <= kFlowMaxT && R <= a.flow_rows && a.dsplit <= kDecSplitMax &&
+                    (int64_t)(R / dec_nt8(a.T) + a.E) * a.dsplit <= kFlowUnitCtrs && (a.d + 127) / 128 <= kFlowTileCtrs;
+  int8_t* hhi = flow ? a.hplanes_hi : a.planes_hi;
+  int8_t* hlo = flow ? a.hplanes_lo : a.planes_lo;
+  float* hsc = flow ? a.hplanes_scale : a.planes_scale;
   if (!dec_gateup_params(p.gu, a.planes_hi, a.planes_lo, a.planes_scale, a.W, a.scales, a.scale_mode, a.wstride, a.d,
                          a.f, a.E,
                          a.offsets, a.gsplit, a.GU, R, a.T, a.err) ||
-      !dec_down_params(p.dn, a.planes_hi, a.planes_lo, a.planes_scale, a.W, a.scales, a.scale_mode, a.wstride, a.d,
-                       a.f, a.E,
-                       a.offsets, a.dsplit, R, a.Ypart, a.T, a.err))
+      !dec_down_params(p.dn, hhi, hlo, hsc, a.W, a.scales, a.scale_mode, a.wstride, a.d, a.f, a.E, a.offsets, a.dsplit,
+                       R, a.Ypart, a.T, a.err))
     return cudaErrorInvalidValue;
-  p.hhi = a.planes_hi;
-  p.hlo = a.planes_lo;
-  p.hscale = a.planes_scale;
+  p.hhi = hhi;
+  p.hlo = hlo;
+  p.hscale = hsc;
   p.dst_row = a.dst_row;
   p.topk_w = a.topk_w;
   p.T = a.T;
@@ -1258,7 +2005,11 @@ cudaError_t launch_dec_fused(const DecFusedArgs& a, cudaStream_t s) {
   p.counts = a.counts;
   p.offsets = a.offsets_out;
   p.src_row = a.src_row;
+  p.xhi = a.planes_hi;
+  p.xlo = a.planes_lo;
   p.xscale = a.planes_scale;
+  p.unit_ctr = a.unit_ctr;
+  p.tile_ctr = a.tile_ctr;
   if (a.route_in_kernel && (a.T > 64 || !a.x || !a.topk_idx || !a.counts || !a.offsets_out || !a.src_row ||
                             (a.route_in_kernel == 1 && !a.router_w)))
     return cudaErrorInvalidValue;
@@ -1274,7 +2025,7 @@ cudaError_t launch_dec_fused(const DecFusedArgs& a, cudaStream_t s) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   launch_chain_break();  // an ordinary launch: the next one must not overlap it
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, dec_fused_kernel, p);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, flow ? dec_flow_kernel : dec_fused_kernel, p);
   launch_chain_break();
   return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -748,7 +748,7 @@ bool make_bf16_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t
 }
 
 bool make_tmap(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int rank, const uint64_t* dims,
-               const uint64_t* strides_bytes, const uint32_t* box) {
+               const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swizzle) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return false;
   cuuint64_t gd[5], gs[4];
@@ -760,7 +760,7 @@ bool make_tmap(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, in
   }
   for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
   const CUresult r = enc(map, dtype, (cuuint32_t)rank, const_cast<void*>(base),
-                         gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }

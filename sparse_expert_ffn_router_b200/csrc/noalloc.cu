@@ -11,13 +11,15 @@
 //
 // The scratch array is a static __device__ object: every GPU that loads this library holds its
 // 257 KB until the process exits.  Host code may not use its name as an address (on the host the
-// name is only a stand-in), so the first call on each device looks up the device address with
-// cudaGetSymbolAddress, with that device current, and caches it; that first call should come
-// before any stream capture.  Every call shares the array and it keeps the last call's contents:
-// every entry a call reads is written by that call first, so nothing needs clearing.  Calls that
-// overlap on the GPU (two streams, or two host threads) race on the array.
-#include <mutex>
-
+// name is only a stand-in), so every call looks up the device address with cudaGetSymbolAddress,
+// with the caller's device current, and raises the router kernels' shared-memory limit there
+// (both cheap once the module is loaded, and both stay right if the context is torn down and
+// re-created).  The first call on each device loads the module and should come before any stream
+// capture.  Every call shares the array and it keeps the last call's contents: every entry a call
+// reads is written by that call first, and the error word the tensor-core router sets when a
+// bounded wait gives up is cleared at the start of each call (a stream-ordered memset, not an
+// allocation); colibri_route_noalloc_check reads it.  Calls that overlap on the GPU (two streams,
+// or two host threads) race on the array.
 #include "common.cuh"
 
 namespace colibri {
@@ -29,33 +31,33 @@ using namespace colibri;
 namespace {
 
 constexpr int kNoAllocMaxBlockExperts = 32768;  // ceil(T / 256) * num_experts
-constexpr size_t kScratchInts = 2 * (size_t)kNoAllocMaxBlockExperts + (kMaxExperts + 1);
+// block counts | block bases | m-tile prefix [E+1] | device error word
+constexpr size_t kErrWordOffset = 2 * (size_t)kNoAllocMaxBlockExperts + (kMaxExperts + 1);
+constexpr size_t kScratchInts = kErrWordOffset + 1;
 
 static __device__ __align__(256) int32_t g_route_scratch[kScratchInts];
 
-constexpr int kMaxDevices = 128;
-std::mutex g_scratch_mu;
-int32_t* g_scratch_addr[kMaxDevices] = {};
 
 colibri_status nf_fail(colibri_status st, const char* msg) {
   record_error(msg);
   return st;
 }
 
-// Device address of g_route_scratch on the current device (looked up once per device).
-colibri_status scratch_address(int dev, int32_t** out) {
-  if (dev < 0 || dev >= kMaxDevices) return nf_fail(COLIBRI_ERR_UNSUPPORTED, "device index too large");
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
-    if (e != cudaSuccess || !p) {
-      cudaGetLastError();
-      return nf_fail(COLIBRI_ERR_CUDA, "cudaGetSymbolAddress of the routing scratch array failed");
-    }
-    g_scratch_addr[dev] = static_cast<int32_t*>(p);
+// Device address of g_route_scratch on the current device, after setting the router kernels'
+// shared-memory limits there (both cheap once the module is loaded; done on every call so that
+// they stay right if the caller tears the context down and re-creates it).
+colibri_status scratch_address(int32_t** out) {
+  if (configure_router_kernels() != cudaSuccess) {
+    cudaGetLastError();
+    return nf_fail(COLIBRI_ERR_CUDA, "router kernel configuration failed");
   }
-  *out = g_scratch_addr[dev];
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
+  if (e != cudaSuccess || !p) {
+    cudaGetLastError();
+    return nf_fail(COLIBRI_ERR_CUDA, "cudaGetSymbolAddress of the routing scratch array failed");
+  }
+  *out = static_cast<int32_t*>(p);
   return COLIBRI_OK;
 }
 
@@ -107,14 +109,17 @@ extern "C" colibri_status colibri_route_noalloc(const void* x, int32_t act_dtype
     if (p && !is_device_ptr(p, dev))
       return nf_fail(COLIBRI_ERR_INVALID_ARG, "every buffer must be device memory of the current device");
   int32_t* scratch = nullptr;
-  const colibri_status st = scratch_address(dev, &scratch);
+  const colibri_status st = scratch_address(&scratch);
   if (st != COLIBRI_OK) return st;
   int32_t* blk_counts = scratch;
   int32_t* blk_base = scratch + kNoAllocMaxBlockExperts;
   int32_t* mt_prefix = scratch + 2 * kNoAllocMaxBlockExperts;
+  uint32_t* err = reinterpret_cast<uint32_t*>(scratch + kErrWordOffset);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_router_topk(x, act_dtype, T, d_model, router_w, router_b, num_experts, top_k, 0,
-                                     topk_idx, topk_w, nullptr, nullptr, nullptr, s);
+  cudaError_t e = cudaMemsetAsync(err, 0, sizeof(uint32_t), s);
+  if (e == cudaSuccess)
+    e = launch_router_topk(x, act_dtype, T, d_model, router_w, router_b, num_experts, top_k, 0, topk_idx, topk_w,
+                           err, nullptr, nullptr, s);
   if (e == cudaSuccess) e = launch_route_count(topk_idx, T, top_k, num_experts, blk_counts, dst_row, s);
   if (e == cudaSuccess)
     e = launch_route_scan(blk_counts, (int)nblk, num_experts, kTcBM, blk_base, counts, offsets, mt_prefix, s);
@@ -122,5 +127,23 @@ extern "C" colibri_status colibri_route_noalloc(const void* x, int32_t act_dtype
     e = launch_route_scatter(x, act_dtype, T, d_model, top_k, num_experts, topk_idx, blk_base, offsets, dst_row,
                              src_row, Xp, nullptr, s);
   if (e != cudaSuccess) return nf_fail(COLIBRI_ERR_CUDA, cudaGetErrorString(e));
+  return COLIBRI_OK;
+}
+
+extern "C" colibri_status colibri_route_noalloc_check(void* stream) {
+  int32_t* scratch = nullptr;
+  const colibri_status st = scratch_address(&scratch);
+  if (st != COLIBRI_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return nf_fail(COLIBRI_ERR_CUDA, "stream synchronize failed");
+  }
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, scratch + kErrWordOffset, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return nf_fail(COLIBRI_ERR_CUDA, "reading the error word failed");
+  }
+  if (word) return nf_fail(COLIBRI_ERR_TIMEOUT, "a bounded device wait of colibri_route_noalloc gave up");
   return COLIBRI_OK;
 }

@@ -159,6 +159,7 @@ struct alignas(64) RouterTcParams {
   float* part;       // [ksplit, E, T] partial logits (ksplit > 1; token-contiguous, so stores coalesce)
   int32_t* ticket;   // [tiles] arrival counters, zero between calls (ksplit > 1)
   int stages;  // ring depth: as many stages as fit in kRtRingBytes (small expert counts go deeper)
+  int kbs;     // consecutive 64-wide K blocks per stage (1 or 2): each x row is read kbs x 128 bytes at a time
   uint32_t stage_bytes, tmem_cols;
   int32_t* idx;
   float* w;
@@ -220,18 +221,20 @@ __global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant
   const int kspan = p.d / p.ksplit;               // a multiple of 64
   const int kb0 = blockIdx.y * (kspan / 64);
   const int nkb = kspan / 64;
-
-  const uint32_t bytes = kRtABytes + (uint32_t)p.N * 128u;
-  // The CTAs of a launch start their K walk at different blocks (rotated by the tile index), so
+  // A stage holds kbs consecutive K blocks: x tiles first, then the Wr tiles.
+  const int kbs = p.kbs, nst = nkb / kbs;
+  const uint32_t wtile = (uint32_t)p.N * 128u;
+  const uint32_t bytes = (uint32_t)kbs * (kRtABytes + wtile);
+  // The CTAs of a launch start their K walk at different stages (rotated by the tile index), so
   // the x rows read at one time do not all sit at the same column offset, which would put every
   // request on the same DRAM channels.  (This fixes, per tile, the order of the fp32 sum.)
-  const int kb_rot = blockIdx.x % nkb;
+  const int st_rot = blockIdx.x % nst;
   if (warp == 0) {
     if (lane == 0) {
       // ----------------------------------------------------------- TMA producer
       bool ok = true;
-      for (int i = 0; i < nkb; ++i) {
-        const int kb = (kb_rot + i) % nkb;
+      for (int i = 0; i < nst; ++i) {
+        const int kb = ((st_rot + i) % nst) * kbs;
         const int s = i % S;
         const uint32_t ph = (uint32_t)(i / S) & 1u;
         if (!rt_wait(&empty[s], ph ^ 1u, abort_flag)) {
@@ -240,8 +243,10 @@ __global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant
         }
         uint8_t* sa = smem + (size_t)s * p.stage_bytes;
         mbar_arrive_expect_tx(&full[s], bytes);
-        tma_load_2d(sa, &p.mapX, &full[s], (kb0 + kb) * 64, row0);
-        tma_load_2d(sa + kRtABytes, &p.mapW, &full[s], (kb0 + kb) * 64, 0);
+        for (int j = 0; j < kbs; ++j) {
+          tma_load_2d(sa + (size_t)j * kRtABytes, &p.mapX, &full[s], (kb0 + kb + j) * 64, row0);
+          tma_load_2d(sa + (size_t)kbs * kRtABytes + (size_t)j * wtile, &p.mapW, &full[s], (kb0 + kb + j) * 64, 0);
+        }
         *issued_s = i + 1;
       }
       if (!ok) {
@@ -256,7 +261,7 @@ __global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant
       // ----------------------------------------------------------- MMA issuer
       const uint32_t idesc = idesc_bf16_f32(128, p.N);
       bool ok = true;
-      for (int i = 0; i < nkb; ++i) {
+      for (int i = 0; i < nst; ++i) {
         const int s = i % S;
         const uint32_t ph = (uint32_t)(i / S) & 1u;
         if (!rt_wait(&full[s], ph, abort_flag)) {
@@ -265,10 +270,13 @@ __global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant
         }
         tc_fence_after();
         const uint32_t sa = smem_u32(smem + (size_t)s * p.stage_bytes);
+        for (int j = 0; j < kbs; ++j) {
+          const uint32_t xa = sa + (uint32_t)j * kRtABytes, wa = sa + (uint32_t)kbs * kRtABytes + (uint32_t)j * wtile;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          tc_mma_f16(tmem, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sa + kRtABytes + kk * 32), idesc,
-                     (i | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk)
+            tc_mma_f16(tmem, smem_desc_sw128(xa + kk * 32), smem_desc_sw128(wa + kk * 32), idesc,
+                       (i | j | kk) != 0 ? 1u : 0u);
+        }
         tc_commit(&empty[s]);  // frees the stage once these MMAs have read it
         *consumed_s = i + 1;
       }
@@ -406,7 +414,10 @@ cudaError_t launch_router_tc(const void* x, int T, int d, const void* wr, const 
   p.E = E;
   p.k = k;
   p.rflags = rflags;
-  p.stage_bytes = (uint32_t)((kRtABytes + p.N * 128 + 1023) / 1024 * 1024);
+  // two consecutive K blocks per stage when the slice has an even number of them (256 contiguous
+  // bytes of each x row per copy pair instead of 128)
+  p.kbs = ((d / ksplit) / 64) % 2 == 0 ? 2 : 1;
+  p.stage_bytes = (uint32_t)((p.kbs * (kRtABytes + p.N * 128) + 1023) / 1024 * 1024);
   p.stages = (int)std::min<size_t>(kRtMaxStages, kRtRingBytes / p.stage_bytes);
   p.tmem_cols = 32;
   while ((int)p.tmem_cols < p.N) p.tmem_cols <<= 1;

@@ -18,12 +18,12 @@ import oracle
 import sparse_expert_ffn_router_b200 as colibri
 
 NEAR_TIE = 1e-4
-TOL = {inputgen.F32: 1e-4, inputgen.BF16: 2e-2, inputgen.I8: 5e-2}
+TOL = {inputgen.F32: 1e-4, inputgen.BF16: 2e-2, inputgen.I8: 5e-2, inputgen.I4: 5e-2}
 
 
 def tolerance(wl) -> float:
-    if wl.wdt == inputgen.I8:
-        return TOL[inputgen.I8]
+    if wl.wdt in (inputgen.I8, inputgen.I4):  # quantised-weight configs
+        return TOL[wl.wdt]
     return TOL[wl.act]
 
 
