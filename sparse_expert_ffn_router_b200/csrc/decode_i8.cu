@@ -697,12 +697,19 @@ __device__ bool d4_convert(const DecStreamParams& p, uint8_t* slots, uint8_t* ri
         const uint8_t* rw = d4_raw(p, st, j);
         uint8_t* at = slots + (size_t)a * 128 * 128;
         // this warp's 32 rows; a task is (row, 16-byte output chunk), so one instruction of the
-        // warp reads 256 contiguous packed bytes (4 rows) and writes 4 whole swizzled rows
+        // warp reads 256 contiguous packed bytes (4 rows) and writes 4 whole swizzled rows.  All
+        // eight packed loads are issued before the first store (a store may not be passed by a
+        // later load the compiler cannot prove disjoint from it).
+        uint2 v[8];
 #pragma unroll
         for (int t8 = 0; t8 < 8; ++t8) {
           const int row = cw * 32 + t8 * 4 + (lane >> 3), ch = lane & 7;
-          const uint2 v = *reinterpret_cast<const uint2*>(rw + row * 64 + ch * 8);
-          const uint2 e0 = widen_int4x8(v.x), e1 = widen_int4x8(v.y);
+          v[t8] = *reinterpret_cast<const uint2*>(rw + row * 64 + ch * 8);
+        }
+#pragma unroll
+        for (int t8 = 0; t8 < 8; ++t8) {
+          const int row = cw * 32 + t8 * 4 + (lane >> 3), ch = lane & 7;
+          const uint2 e0 = widen_int4x8(v[t8].x), e1 = widen_int4x8(v[t8].y);
           *reinterpret_cast<uint4*>(at + row * 128 + ((ch ^ (row & 7)) << 4)) = make_uint4(e0.x, e0.y, e1.x, e1.y);
         }
         // the tensor core reads the tile through the async proxy
@@ -753,6 +760,32 @@ __device__ bool d4_mma(const DecStreamParams& p, uint8_t* slots, uint8_t* ring, 
 
 // Epilogue: per K block, the accumulator scaled by that block's group scale is added into fp32
 // registers (one per token of the chunk); per item the sums times the plane scale are written.
+// K blocks are taken two at a time (both accumulators waited for, read, then released), so the
+// fixed latencies of the wait and the TMEM load are paid once per pair.
+__device__ __forceinline__ void d4_accumulate(float (&acc)[32], int nt8, uint32_t tb, float s) {
+  // columns [0, nt8) of the accumulator hold the hi plane, [nt8, 2 nt8) the lo plane
+  if (nt8 == 8) {
+    float v[16];
+    tmem_ld16(tb, v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+      acc[t] = fmaf(s, (float)__float_as_int(v[t]) + (float)__float_as_int(v[8 + t]) * (1.0f / 254.0f), acc[t]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; j += 16) {
+      if (j >= nt8) break;
+      float vh[16], vl[16];
+      tmem_ld16(tb + j, vh);
+      tmem_ld16(tb + nt8 + j, vl);
+      tmem_ld_wait();
+#pragma unroll
+      for (int t = 0; t < 16; ++t)
+        acc[j + t] = fmaf(s, (float)__float_as_int(vh[t]) + (float)__float_as_int(vl[t]) * (1.0f / 254.0f), acc[j + t]);
+    }
+  }
+}
+
 template <bool kGateUp>
 __device__ bool d4_epilogue(const DecStreamParams& p, D4Ctl& c, uint32_t tmem, int warp, int lane) {
   const int q = warp & 3;
@@ -775,46 +808,33 @@ __device__ bool d4_epilogue(const DecStreamParams& p, D4Ctl& c, uint32_t tmem, i
     float acc[32];
 #pragma unroll
     for (int t = 0; t < 32; ++t) acc[t] = 0.f;
-    float sc[8];
+    float sc[8];  // the scales of K blocks i .. i + 7, loaded 8 blocks ahead
 #pragma unroll
     for (int u = 0; u < 8; ++u) sc[u] = group_scale(u);
     for (int i0 = 0; i0 < w.nkb; i0 += 8) {
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < 8; u += 2) {
         const int i = i0 + u;
         if (i >= w.nkb) break;
-        const uint32_t b = kc % kD4Bufs, bph = (kc / kD4Bufs) & 1u;
-        ++kc;
-        if (!__all_sync(0xffffffffu, ds_wait(&c.tfull[b], bph, &c.abort))) return false;
+        const bool two = i + 1 < w.nkb;
+        const uint32_t b0 = kc % kD4Bufs, ph0 = (kc / kD4Bufs) & 1u;
+        const uint32_t b1 = (kc + 1) % kD4Bufs, ph1 = ((kc + 1) / kD4Bufs) & 1u;
+        const bool got = ds_wait(&c.tfull[b0], ph0, &c.abort) && (!two || ds_wait(&c.tfull[b1], ph1, &c.abort));
+        if (!__all_sync(0xffffffffu, got)) return false;
         tc_fence_after();
-        const float s = sc[u];
-        sc[u] = group_scale(i + 8);  // the scale 8 blocks ahead, loaded while these are in use
-        const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + b * (uint32_t)N;
-        // columns [0, nt8) hold the hi plane, [nt8, 2 nt8) the lo plane of the same tokens
-        if (p.nt8 == 8) {
-          float v[16];
-          tmem_ld16(tb, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int t = 0; t < 8; ++t)
-            acc[t] = fmaf(s, (float)__float_as_int(v[t]) + (float)__float_as_int(v[8 + t]) * (1.0f / 254.0f), acc[t]);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; j += 16) {
-            if (j >= p.nt8) break;
-            float vh[16], vl[16];
-            tmem_ld16(tb + j, vh);
-            tmem_ld16(tb + p.nt8 + j, vl);
-            tmem_ld_wait();
-#pragma unroll
-            for (int t = 0; t < 16; ++t)
-              acc[j + t] = fmaf(s, (float)__float_as_int(vh[t]) + (float)__float_as_int(vl[t]) * (1.0f / 254.0f),
-                                acc[j + t]);
-          }
-        }
+        const float s0 = sc[u], s1 = sc[u + 1];
+        sc[u] = group_scale(i + 8);
+        sc[u + 1] = group_scale(i + 9);
+        const uint32_t lanes = (uint32_t)(q * 32) << 16;
+        d4_accumulate(acc, p.nt8, tmem + lanes + b0 * (uint32_t)N, s0);
+        if (two) d4_accumulate(acc, p.nt8, tmem + lanes + b1 * (uint32_t)N, s1);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&c.tempty[b]);
+        if (lane == 0) {
+          mbar_arrive(&c.tempty[b0]);
+          if (two) mbar_arrive(&c.tempty[b1]);
+        }
+        kc += two ? 2 : 1;
       }
     }
 #pragma unroll
