@@ -43,6 +43,8 @@ constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
 
 struct alignas(64) TcParams {
   CUtensorMap mapA;     // routed A rows
+  CUtensorMap mapA16;   // the same rows, boxes of 16 and 64 rows (light tiles copy only what
+  CUtensorMap mapA64;   // their MMAs read)
   CUtensorMap mapB;     // routed weights
   CUtensorMap mapA_sh;  // shared-expert A rows
   CUtensorMap mapB_sh;  // shared-expert weights
@@ -231,6 +233,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ffn_kernel(const __grid_con
     m.consumed = 0;
     mbar_fence_init();
     tma_prefetch_desc(&p.mapA);
+    tma_prefetch_desc(&p.mapA16);
+    tma_prefetch_desc(&p.mapA64);
     tma_prefetch_desc(&p.mapB);
     if (p.mt_sh > 0) {
       tma_prefetch_desc(&p.mapA_sh);
@@ -274,9 +278,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ffn_kernel(const __grid_con
           }
           uint8_t* sA = stage_base + (size_t)s * STAGE_BYTES;
           uint8_t* sB = sA + A_BYTES;
-          mbar_arrive_expect_tx(&m.full[s], STAGE_BYTES);
           const int kx = kb * BK;
-          tma_load_2d(sA, mA, &m.full[s], kx, t.row0);
+          // a light tile's MMAs read only its first 16 * ceil(rows / 16) rows of A: copy 16 or 64
+          const int arows = t.row_end - t.row0;
+          const uint32_t a_bytes = t.sh || arows > kLightRows ? (uint32_t)A_BYTES : (arows <= 16 ? 16u : 64u) * BK * 2;
+          mbar_arrive_expect_tx(&m.full[s], a_bytes + (uint32_t)B_BYTES);
+          tma_load_2d(sA, a_bytes == (uint32_t)A_BYTES ? mA : (arows <= 16 ? &p.mapA16 : &p.mapA64), &m.full[s], kx,
+                      t.row0);
           // the weight tile of a group with a single (light) m-tile is read by this tile alone:
           // evict it first from L2
           const bool stream = t.mtiles == 1 && t.row_end - t.row0 <= kLightRows && !t.sh;
@@ -783,9 +791,13 @@ cudaError_t launch_tc(const TcGemmArgs& a, cudaStream_t s) {
   const uint64_t S = (uint64_t)a.wstride * 2;  // bytes between experts
   bool ok = true;
   if (kGateUp) {
-    // A: grouped rows Xp [rows, d]
+    // A: grouped rows Xp [rows, d] (and the light tiles' 16- and 64-row boxes)
     { uint64_t dims[2] = {d, (uint64_t)a.rows}, st[1] = {d * 2}; uint32_t box[2] = {BK, BM};
-      ok &= make_map(&p.mapA, a.A, 2, dims, st, box); }
+      ok &= make_map(&p.mapA, a.A, 2, dims, st, box);
+      box[1] = 16;
+      ok &= make_map(&p.mapA16, a.A, 2, dims, st, box);
+      box[1] = 64;
+      ok &= make_map(&p.mapA64, a.A, 2, dims, st, box); }
     // B: W1|W3 of every expert as [d, f, 2, E]
     { uint64_t dims[4] = {d, f, 2, (uint64_t)a.E}, st[3] = {d * 2, f * d * 2, S};
       uint32_t box[4] = {BK, BN / 2, 1, 1};
@@ -803,9 +815,13 @@ cudaError_t launch_tc(const TcGemmArgs& a, cudaStream_t s) {
     p.n_out = (int)f;
     p.n_out_sh = (int)fs;
   } else {
-    // A: H [rows, f]
+    // A: H [rows, f] (and the light tiles' 16- and 64-row boxes)
     { uint64_t dims[2] = {f, (uint64_t)a.rows}, st[1] = {f * 2}; uint32_t box[2] = {BK, BM};
-      ok &= make_map(&p.mapA, a.A, 2, dims, st, box); }
+      ok &= make_map(&p.mapA, a.A, 2, dims, st, box);
+      box[1] = 16;
+      ok &= make_map(&p.mapA16, a.A, 2, dims, st, box);
+      box[1] = 64;
+      ok &= make_map(&p.mapA64, a.A, 2, dims, st, box); }
     // B: W2 of every expert as [f, d, E], starting 2*f*d elements into the expert
     { uint64_t dims[3] = {f, d, (uint64_t)a.E}, st[2] = {f * 2, S}; uint32_t box[3] = {BK, b_rows_down, 1};
       ok &= make_map(&p.mapB, (const __nv_bfloat16*)a.W + 2 * f * d, 3, dims, st, box); }
