@@ -206,6 +206,23 @@ colibri_status colibri_get_routing(colibri_ctx* ctx, int32_t* topk_idx, float* t
                                    int32_t* dst_row, void* stream);
 
 /*
+ * colibri_combine -- the Gather stage alone (www.pptc.cn/news/100465 §2.1 k-way aggregation;
+ * www.hotelren.com/news/4731937 §2.3 combine_kernel): y[t] = sum_{j<k} topk_w[t][j] *
+ * Yp[dst_row[t][j]], summed in slot order in fp32 and rounded once to act_dtype.  For callers
+ * whose expert outputs come from elsewhere, e.g. the expert-parallel layer, where the grouped
+ * rows were computed on the GPUs that own the experts and sent back.
+ *   Yp       [rows, d_model] act_dtype, the expert outputs of the grouped rows.
+ *   dst_row  [T, k] int32, grouped row of each (token, slot); topk_w [T, k] fp32.
+ *   y        [T, d_model] act_dtype, fully overwritten.
+ * All buffers caller-owned device memory of the current device, 16-byte aligned; d_model a
+ * multiple of 8; 1 <= k <= 8.  No context, no allocation; enqueued on `stream`.  T == 0 launches
+ * nothing.  Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED, CUDA (reason via colibri_last_error(NULL)).
+ */
+colibri_status colibri_combine(const void* Yp, int32_t act_dtype, const int32_t* dst_row,
+                               const float* topk_w, int32_t T, int32_t top_k, int32_t d_model,
+                               void* y, void* stream);
+
+/*
  * colibri_sync_status -- synchronise `stream`, then read and clear the context's device
  * error word.  Returns COLIBRI_ERR_TIMEOUT if a kernel's bounded wait gave up since the last
  * check (its output is then undefined), COLIBRI_ERR_CUDA if the stream reports an error,

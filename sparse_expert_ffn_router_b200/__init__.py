@@ -37,6 +37,7 @@ EXPORTS = (
     "colibri_moe_forward",
     "colibri_moe_forward_routed",
     "colibri_get_routing",
+    "colibri_combine",
     "colibri_sync_status",
     "colibri_profile_begin",
     "colibri_profile_end",
@@ -95,6 +96,8 @@ def load() -> ctypes.CDLL:
     lib.colibri_moe_forward_routed.restype = ctypes.c_int
     lib.colibri_get_routing.argtypes = [vp] * 8
     lib.colibri_get_routing.restype = ctypes.c_int
+    lib.colibri_combine.argtypes = [vp, i32, vp, vp, i32, i32, i32, vp, vp]
+    lib.colibri_combine.restype = ctypes.c_int
     lib.colibri_sync_status.argtypes = [vp, vp]
     lib.colibri_sync_status.restype = ctypes.c_int
     lib.colibri_profile_begin.argtypes = [vp, i32]
@@ -184,6 +187,12 @@ def colibri_get_routing(ctx: int, topk_idx=None, topk_w=None, counts=None, offse
     _check(load().colibri_get_routing(ctx, _addr(topk_idx), _addr(topk_w), _addr(counts), _addr(offsets),
                                       _addr(src_row), _addr(dst_row), _stream(stream)),
            "colibri_get_routing", ctx)
+
+
+def colibri_combine(Yp, act_dtype: int, dst_row, topk_w, T: int, top_k: int, d_model: int, y, stream=None) -> None:
+    """Gather stage alone: y[t] = sum_j topk_w[t][j] * Yp[dst_row[t][j]] (see include/colibri.h)."""
+    _check(load().colibri_combine(_addr(Yp), act_dtype, _addr(dst_row), _addr(topk_w), T, top_k, d_model, _addr(y),
+                                  _stream(stream)), "colibri_combine")
 
 
 def colibri_sync_status(ctx: int, stream=None) -> None:

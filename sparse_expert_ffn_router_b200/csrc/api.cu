@@ -755,6 +755,34 @@ colibri_status colibri_get_routing(colibri_ctx* ctx, int32_t* topk_idx, float* t
   return COLIBRI_OK;
 }
 
+colibri_status colibri_combine(const void* Yp, int32_t act_dtype, const int32_t* dst_row, const float* topk_w,
+                               int32_t T, int32_t top_k, int32_t d_model, void* y, void* stream) {
+  if (act_dtype != COLIBRI_F32 && act_dtype != COLIBRI_BF16)
+    return fail(nullptr, COLIBRI_ERR_UNSUPPORTED, "act_dtype must be COLIBRI_F32 or COLIBRI_BF16");
+  if (T < 0 || top_k < 1 || top_k > kMaxTopK || d_model < 8 || d_model % 8 != 0)
+    return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "T >= 0, 1 <= top_k <= 8 and d_model a positive multiple of 8");
+  if (T == 0) return COLIBRI_OK;
+  if (!Yp || !dst_row || !topk_w || !y) return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "NULL buffer");
+  const void* ptrs[] = {Yp, dst_row, topk_w, y};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return fail(nullptr, COLIBRI_ERR_ALIGNMENT, "every buffer must be 16-byte aligned");
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(nullptr, COLIBRI_ERR_CUDA, "cudaGetDevice failed");
+  }
+  for (const void* p : ptrs)
+    if (classify(p, dev) != kPtrDevice)
+      return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "every buffer must be device memory of the current device");
+  const cudaError_t e = launch_combine(Yp, act_dtype, dst_row, topk_w, T, top_k, d_model, nullptr, y, act_dtype,
+                                       reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(nullptr, COLIBRI_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
+  }
+  return COLIBRI_OK;
+}
+
 colibri_status colibri_sync_status(colibri_ctx* ctx, void* stream) {
   if (!ctx) return fail(nullptr, COLIBRI_ERR_INVALID_ARG, "ctx is NULL");
   DeviceGuard guard(ctx->desc.device_id);
