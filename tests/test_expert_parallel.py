@@ -33,7 +33,7 @@ def _problem():
     sys.path.insert(0, ROOT)
     import inputgen
 
-    wl = inputgen.custom("ep", T=40, d=64, E=8, k=2, f=96)
+    wl = inputgen.custom("ep", T=40, d=64, E=8, k=2, f=128)
     return inputgen.make_problem(wl, seed=12)
 
 
