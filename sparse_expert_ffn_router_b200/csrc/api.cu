@@ -232,6 +232,7 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   const size_t o_rpart = c.take(rsplit ? (size_t)kRouterMaxSplit * M * E * 4 : 0);
   const size_t o_rtick = c.take(rsplit ? (size_t)((M + 127) / 128) * 4 : 0);
   const size_t o_err = c.take(4);
+  const size_t o_tsched = c.take(4 * 4);
   const size_t o_gbar = c.take(i8 ? kFusedBarCount * 4 : 0);
   const size_t flow_bytes = (size_t)(kFlowUnitCtrs + kFlowTileCtrs) * 4;
   const size_t o_flow = c.take(i8 ? flow_bytes : 0);
@@ -270,6 +271,7 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   w.plane_lo = reinterpret_cast<int8_t*>(b + o_plo);
   w.plane_scale = reinterpret_cast<float*>(b + o_psc);
   w.err = reinterpret_cast<uint32_t*>(b + o_err);
+  w.tile_sched = reinterpret_cast<uint32_t*>(b + o_tsched);
   w.grid_bar = i8 ? reinterpret_cast<int32_t*>(b + o_gbar) : nullptr;
   w.flow_ctr = i8 ? reinterpret_cast<int32_t*>(b + o_flow) : nullptr;
   w.flow_hhi = i8 ? reinterpret_cast<int8_t*>(b + o_fhh) : nullptr;
@@ -278,7 +280,7 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   w.flow_rows = i8 ? (int)flow_rows : 0;
   w.router_part = rsplit ? reinterpret_cast<float*>(b + o_rpart) : nullptr;
   w.router_ticket = rsplit ? reinterpret_cast<int32_t*>(b + o_rtick) : nullptr;
-  if (cudaMemset(w.err, 0, 4) != cudaSuccess ||
+  if (cudaMemset(w.err, 0, 4) != cudaSuccess || cudaMemset(w.tile_sched, 0, 4 * 4) != cudaSuccess ||
       (rsplit && cudaMemset(w.router_ticket, 0, (size_t)((M + 127) / 128) * 4) != cudaSuccess) ||
       (i8 && cudaMemset(w.grid_bar, 0, kFusedBarCount * 4) != cudaSuccess) ||
       (i8 && cudaMemset(w.flow_ctr, 0, flow_bytes) != cudaSuccess)) {
@@ -296,6 +298,8 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
     }
   }
   ctx->use_graphs = !(getenv("COLIBRI_GRAPHS") && strcmp(getenv("COLIBRI_GRAPHS"), "0") == 0);
+  // COLIBRI_TILE_SCHED=static: the bf16 GEMMs walk their tiles round-robin instead of claiming them
+  ctx->tile_static = getenv("COLIBRI_TILE_SCHED") && strcmp(getenv("COLIBRI_TILE_SCHED"), "static") == 0;
   // Programmatic dependent launch measured slower on the small-batch decode chain and neutral on
   // prefill, so it is opt-in (COLIBRI_PDL=1).
   ctx->use_pdl = env_flag("COLIBRI_PDL");
@@ -465,8 +469,10 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
     a.err = w.err;
     a.sm_count = ctx->sm_count;
     a.pair = gemm == kGemmPair;
+    a.sched = ctx->tile_static ? nullptr : w.tile_sched;
     COLIBRI_TRY(launch_tc_gateup(a, s), "tc_gateup");
     mark(3);
+    a.sched = ctx->tile_static ? nullptr : w.tile_sched + 2;
     a.A = w.H;
     a.out = w.Yp;
     a.A_sh = w.Hs;
@@ -798,6 +804,7 @@ colibri_status colibri_sync_status(colibri_ctx* ctx, void* stream) {
     if (ctx->ws.flow_ctr)
       COLIBRI_TRY(cudaMemset(ctx->ws.flow_ctr, 0, (size_t)(kFlowUnitCtrs + kFlowTileCtrs) * 4),
                   "reset completion counters");
+    COLIBRI_TRY(cudaMemset(ctx->ws.tile_sched, 0, 4 * 4), "reset tile counters");
     return fail(ctx, COLIBRI_ERR_TIMEOUT, "device error word 0x%x (a bounded wait gave up)", err);
   }
   return COLIBRI_OK;

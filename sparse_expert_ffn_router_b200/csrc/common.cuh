@@ -87,6 +87,7 @@ struct Workspace {
   int8_t* plane_lo = nullptr;
   float* plane_scale = nullptr;  // [M*k]
   uint32_t* err = nullptr;
+  uint32_t* tile_sched = nullptr;  // [4] tile counters of the bf16 GEMMs (gate/up, down; zero between calls)
 };
 
 }  // namespace colibri
@@ -123,6 +124,7 @@ struct colibri_ctx {
   std::vector<GraphEntry> graphs;
   uint64_t graph_clock = 0;
   bool use_graphs = true;
+  bool tile_static = false;  // bf16 GEMMs: static round-robin tiles instead of the claimed schedule
   bool use_pdl = false;  // programmatic dependent launch between the kernels of a forward (opt-in)
   bool dec_fused = true;  // int8 weights: the one-launch expert stage (COLIBRI_DEC_FUSED=0: four launches)
   bool dec_route = true;  // int8, T <= 64: routing inside that launch too (COLIBRI_DEC_ROUTE=0: not)
@@ -263,6 +265,8 @@ struct TcGemmArgs {
   int fs;               // shared d_ff (0 = none)
   int mt_bound;         // upper bound on routed m-tiles
   uint32_t* err;
+  uint32_t* sched;      // [2] tile counter and finished-CTA counter (zero between launches), or
+                        // nullptr for the static round-robin schedule
   int sm_count;
   bool pair;            // clusters of two CTAs with 256-row pair tiles (cta_group::2)
 };
@@ -528,6 +532,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same wait with cluster-scope acquire: for a barrier whose arrivals (and the shared data
+// they publish) come from the other CTA of a cluster.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete; give up after kWaitTimeoutNs.
 // Returns false on timeout (the caller records the error and leaves its loop).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
@@ -683,6 +701,10 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
 }
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// 32-bit store into the shared memory of a CTA of the cluster (address from mapa_shared).
+__device__ __forceinline__ void st_shared_cluster_u32(uint32_t cluster_addr, int32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");

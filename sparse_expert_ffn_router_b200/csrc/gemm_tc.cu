@@ -21,10 +21,15 @@
 //               stage with tcgen05.commit; commits the finished accumulator to the epilogue.
 //   warps 2-5   epilogue: tcgen05.ld 32 lanes x 16 columns, SwiGLU or convert, bf16 stores;
 //               releases the accumulator so the next tile's MMAs overlap this epilogue.
-// Tiles are walked round-robin over a schedule built on the device from the per-expert row
-// offsets: expert-major, then n-tile, then m-tile fastest, so the CTAs running at one time
-// share the same weight tile through L2 and each weight byte leaves HBM about once; tiles of
-// experts with a single m-tile (weight streaming) are interleaved with the others.
+// Tiles are numbered by a schedule built on the device from the per-expert row offsets:
+// expert-major, then n-tile, then m-tile fastest, so the CTAs running at one time share the same
+// weight tile through L2 and each weight byte leaves HBM about once; tiles of experts with a
+// single m-tile (weight streaming) are interleaved with the others.  A CTA takes its first tile
+// by its index and every later one from a global counter (claimed a few stages before its
+// current tile's copies are all issued), so the tiles in flight always form one window of
+// consecutive numbers however the CTAs' speeds differ, and a faster CTA simply takes more tiles.
+// The producer hands each tile number to the MMA and epilogue roles through a small ring in
+// shared memory; the last CTA to finish zeroes the counter for the next launch.
 // Every wait is bounded (kWaitTimeoutNs); a wait that gives up sets the error word, makes the
 // other roles leave their loops, drains outstanding copies and MMAs and frees TMEM.
 #include "common.cuh"
@@ -50,6 +55,7 @@ struct alignas(64) TcParams {
   CUtensorMap mapB_sh;  // shared-expert weights
   const int32_t* offsets;
   const int32_t* mt_prefix;
+  uint32_t* sched;      // [2] tile counter, finished CTAs; nullptr: static round-robin
   int E;
   int n_tiles, n_tiles_sh;
   int mt_sh, rows_sh;
@@ -60,11 +66,17 @@ struct alignas(64) TcParams {
   uint32_t* err;
 };
 
+// Tile numbers in flight between the producer and the other roles (a sentinel -1 ends the loop).
+constexpr int kTQ = 4;
+
 struct SmemMisc {
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
+  uint64_t tq_full[kTQ];
+  uint64_t tq_empty[kTQ];
+  int32_t tq[kTQ];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -183,17 +195,37 @@ __device__ __forceinline__ Tile decode_tile(const TcParams& p, const Misc& m, in
   return t;
 }
 
-// Bounded wait that also gives up as soon as another role has aborted.
+// Bounded wait that also gives up as soon as another role has aborted (kCluster: acquire at
+// cluster scope, for barriers the other CTA of a pair arrives on).
+template <bool kCluster = false>
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  if (mbar_try_wait(bar, parity)) return true;
+  auto try_wait = [&]() { return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  if (try_wait()) return true;
   const unsigned long long t0 = global_ns();
   uint32_t n = 0;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (try_wait()) return true;
     if ((++n & 255u) == 0) {
       if (*abort_flag) return false;
       if (global_ns() - t0 > kWaitTimeoutNs) return false;
     }
+  }
+}
+
+// The tile after the current one: from the global counter (offset by the tiles the CTAs took by
+// their index), or the static round-robin successor.
+__device__ __forceinline__ int claim_next(uint32_t* sched, int L, int nworkers) {
+  return sched ? (int)atomicAdd(sched, 1u) + nworkers : L + nworkers;
+}
+
+// Called once by every CTA of the launch on its way out, after its last claim: the last one to
+// finish zeroes the counters for the next launch (launches of one forward are stream-ordered).
+__device__ __forceinline__ void sched_finish(uint32_t* sched) {
+  if (!sched) return;
+  __threadfence();
+  if (atomicAdd(sched + 1, 1u) == gridDim.x - 1) {
+    atomicExch(sched, 0u);
+    atomicExch(sched + 1, 0u);
   }
 }
 
@@ -226,6 +258,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ffn_kernel(const __grid_con
     for (int a = 0; a < 2; ++a) {
       mbar_init(&m.tfull[a], 1);
       mbar_init(&m.tempty[a], EPI_THREADS);
+    }
+    for (int i = 0; i < kTQ; ++i) {
+      mbar_init(&m.tq_full[i], 1);
+      mbar_init(&m.tq_empty[i], 1 + EPI_THREADS / 32);  // the MMA thread and the 4 epilogue warps
     }
     mbar_init(&m.drain, 1);
     m.abort = 0;
@@ -265,13 +301,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ffn_kernel(const __grid_con
       int s = 0;
       uint32_t ph = 0;
       int issued = 0;
+      int q = 0;
+      uint32_t qph = 0;
       const uint64_t evict_first = l2_evict_first_policy();
-      for (int L = blockIdx.x; L < total; L += gridDim.x) {
+      int L = blockIdx.x;
+      while (true) {
+        // publish the tile number (or the end) to the MMA and epilogue roles
+        if (!wait_or_abort(&m.tq_empty[q], qph ^ 1u, abort_flag)) {
+          raise_abort(m, p.err);
+          break;
+        }
+        const int Lq = L < total ? L : -1;
+        *(volatile int32_t*)&m.tq[q] = Lq;
+        mbar_arrive(&m.tq_full[q]);
+        if (++q == kTQ) {
+          q = 0;
+          qph ^= 1u;
+        }
+        if (Lq < 0) break;
         const Tile t = decode_tile(p, m, L, routed_total, kGateUp);
         const CUtensorMap* mA = t.sh ? &p.mapA_sh : &p.mapA;
         const CUtensorMap* mB = t.sh ? &p.mapB_sh : &p.mapB;
+        const int claim_kb = t.num_kb > STAGES ? t.num_kb - STAGES : 0;
+        int next = L;
         bool ok = true;
         for (int kb = 0; kb < t.num_kb; ++kb) {
+          if (kb == claim_kb) next = claim_next(p.sched, L, (int)gridDim.x);
           if (!wait_or_abort(&m.empty[s], ph ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -300,8 +355,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ffn_kernel(const __grid_con
               tma_load_4d(sB + B_BYTES / 2, mB, &m.full[s], kx, t.n0, 1, t.e);
             }
           } else {
+            // down projection: the W2 blocks of an expert with many m-tiles are evicted from L2
+            // first (its m-tiles read each block within a short window), so that its H rows stay
+            // for the n-tiles that start a tile later (measured: 1.15x -> 1.10x the algorithmic
+            // bytes at T=2048 with two experts of ~2000 rows; not used for two m-tiles, where it
+            // raised the traffic)
             if (t.sh) tma_load_2d(sB, mB, &m.full[s], kx, t.n0);
-            else if (stream) tma_load_3d_hint(sB, mB, &m.full[s], kx, t.n0, t.e, evict_first);
+            else if (stream || t.mtiles > 2) tma_load_3d_hint(sB, mB, &m.full[s], kx, t.n0, t.e, evict_first);
             else tma_load_3d(sB, mB, &m.full[s], kx, t.n0, t.e);
           }
           ++issued;
@@ -314,6 +374,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ffn_kernel(const __grid_con
           raise_abort(m, p.err);
           break;
         }
+        L = next;
       }
       m.issued = issued;
     }
@@ -325,8 +386,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ffn_kernel(const __grid_con
       int s = 0;
       uint32_t ph = 0;
       int it = 0, consumed = 0;
+      int q = 0;
+      uint32_t qph = 0;
       bool ok = true;
-      for (int L = blockIdx.x; L < total && ok; L += gridDim.x, ++it) {
+      for (;; ++it) {
+        if (!wait_or_abort(&m.tq_full[q], qph, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const int L = *(volatile int32_t*)&m.tq[q];
+        mbar_arrive(&m.tq_empty[q]);
+        if (++q == kTQ) {
+          q = 0;
+          qph ^= 1u;
+        }
+        if (L < 0) break;
         const Tile t = decode_tile(p, m, L, routed_total, kGateUp);
         const int a = it & 1;
         const uint32_t aph = (uint32_t)(it >> 1) & 1u;
@@ -384,8 +458,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ffn_kernel(const __grid_con
   } else {
     // ------------------------------------------------------------- epilogue (warps 2..5)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
-    int it = 0;
-    for (int L = blockIdx.x; L < total; L += gridDim.x, ++it) {
+    int tq = 0;
+    uint32_t tqph = 0;
+    for (int it = 0;; ++it) {
+      const bool gq = wait_or_abort(&m.tq_full[tq], tqph, abort_flag);
+      if (!__all_sync(0xffffffffu, gq)) {
+        if (lane == 0) raise_abort(m, p.err);
+        break;
+      }
+      const int L = *(volatile int32_t*)&m.tq[tq];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&m.tq_empty[tq]);
+      if (++tq == kTQ) {
+        tq = 0;
+        tqph ^= 1u;
+      }
+      if (L < 0) break;
       const Tile t = decode_tile(p, m, L, routed_total, kGateUp);
       const int a = it & 1;
       const uint32_t aph = (uint32_t)(it >> 1) & 1u;
@@ -476,6 +564,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ffn_kernel(const __grid_con
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
   }
+  if (threadIdx.x == 0) sched_finish(p.sched);
 }
 
 // ------------------------------------------------------------------------- pair kernel
@@ -497,6 +586,9 @@ struct SmemMisc2 {
   uint64_t empty[STAGES2];   // per CTA: freed by the leader's multicast commit
   uint64_t tfull[2];         // per CTA: accumulator ready (multicast commit)
   uint64_t tempty[2];        // used in the leader: 8 epilogue-warp arrivals (4 local, 4 peer)
+  uint64_t tq_full[kTQ];     // per CTA: tile number published by the leader's producer
+  uint64_t tq_empty[kTQ];    // used in the leader: MMA thread, peer producer, 8 epilogue warps
+  int32_t tq[kTQ];           // per CTA: the leader writes both CTAs' copies
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -516,7 +608,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
   // starts 1024-byte aligned (both CTAs of a pair take this branch together).
   if (smem_u32(smem_raw) & 1023u) {
     pdl_wait();
-    if (threadIdx.x == 0) atomicOr(p.err, kErrWaitTimeout);
+    if (threadIdx.x == 0) {
+      atomicOr(p.err, kErrWaitTimeout);
+      sched_finish(p.sched);
+    }
     return;
   }
   uint8_t* smem = smem_raw;
@@ -535,6 +630,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
     for (int a = 0; a < 2; ++a) {
       mbar_init(&m.tfull[a], 1);
       mbar_init(&m.tempty[a], 8);
+    }
+    for (int i = 0; i < kTQ; ++i) {
+      mbar_init(&m.tq_full[i], 1);
+      mbar_init(&m.tq_empty[i], 2 + 8);
     }
     mbar_init(&m.drain, 1);
     m.abort = 0;
@@ -570,13 +669,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
-      for (int L = pair; L < total; L += npairs) {
+      int q = 0;
+      uint32_t qph = 0;
+      int L = pair;
+      while (true) {
+        // the leader claims tiles and publishes each number to both CTAs; the peer reads its copy
+        int Lq;
+        if (rank == 0) {
+          if (!wait_or_abort<true>(&m.tq_empty[q], qph ^ 1u, abort_flag)) {
+            raise_abort(m, p.err);
+            break;
+          }
+          Lq = L < total ? L : -1;
+          *(volatile int32_t*)&m.tq[q] = Lq;
+          st_shared_cluster_u32(mapa_shared(smem_u32(&m.tq[q]), 1), Lq);
+          mbar_arrive(&m.tq_full[q]);
+          mbar_arrive_cluster(mapa_shared(smem_u32(&m.tq_full[q]), 1));
+        } else {
+          if (!wait_or_abort<true>(&m.tq_full[q], qph, abort_flag)) {
+            raise_abort(m, p.err);
+            break;
+          }
+          Lq = *(volatile int32_t*)&m.tq[q];
+          mbar_arrive_cluster(mapa_shared(smem_u32(&m.tq_empty[q]), 0));
+        }
+        if (++q == kTQ) {
+          q = 0;
+          qph ^= 1u;
+        }
+        if (Lq < 0) break;
+        L = Lq;
         const Tile t = decode_tile(p, m, L, routed_total, kGateUp, BM2);
         const CUtensorMap* mA = t.sh ? &p.mapA_sh : &p.mapA;
         const CUtensorMap* mB = t.sh ? &p.mapB_sh : &p.mapB;
         const int arow = t.row0 + 128 * (int)rank;
+        const int claim_kb = t.num_kb > STAGES2 ? t.num_kb - STAGES2 : 0;
+        int next = L;
         bool ok = true;
         for (int kb = 0; kb < t.num_kb; ++kb) {
+          if (rank == 0 && kb == claim_kb) next = claim_next(p.sched, L, npairs);
           if (!wait_or_abort(&m.empty[s], ph ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -603,6 +734,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
           raise_abort(m, p.err);
           break;
         }
+        L = next;
       }
     }
     pdl_trigger();  // every copy of this CTA is issued: let the next kernel be scheduled
@@ -613,8 +745,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
       int s = 0;
       uint32_t ph = 0;
       int it = 0;
+      int q = 0;
+      uint32_t qph = 0;
       bool ok = true;
-      for (int L = pair; L < total && ok; L += npairs, ++it) {
+      for (;; ++it) {
+        if (!wait_or_abort(&m.tq_full[q], qph, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const int L = *(volatile int32_t*)&m.tq[q];
+        mbar_arrive(&m.tq_empty[q]);
+        if (++q == kTQ) {
+          q = 0;
+          qph ^= 1u;
+        }
+        if (L < 0) break;
         const Tile t = decode_tile(p, m, L, routed_total, kGateUp, BM2);
         const int a = it & 1;
         const uint32_t aph = (uint32_t)(it >> 1) & 1u;
@@ -657,8 +802,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
     const int q = warp & 3;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&m.tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&m.tempty[1]), 0);
-    int it = 0;
-    for (int L = pair; L < total; L += npairs, ++it) {
+    int tq = 0;
+    uint32_t tqph = 0;
+    for (int it = 0;; ++it) {
+      const bool gq = wait_or_abort<true>(&m.tq_full[tq], tqph, abort_flag);
+      if (!__all_sync(0xffffffffu, gq)) {
+        if (lane == 0) raise_abort(m, p.err);
+        break;
+      }
+      const int L = *(volatile int32_t*)&m.tq[tq];
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&m.tq_empty[tq]), 0));
+      if (++tq == kTQ) {
+        tq = 0;
+        tqph ^= 1u;
+      }
+      if (L < 0) break;
       const Tile t = decode_tile(p, m, L, routed_total, kGateUp, BM2);
       const int a = it & 1;
       const uint32_t aph = (uint32_t)(it >> 1) & 1u;
@@ -724,6 +883,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
+  if (threadIdx.x == 0) sched_finish(p.sched);
 }
 
 // ------------------------------------------------------------------------- host side
@@ -841,6 +1001,7 @@ cudaError_t launch_tc(const TcGemmArgs& a, cudaStream_t s) {
   if (!ok) return cudaErrorInvalidValue;
   p.offsets = a.offsets;
   p.mt_prefix = a.mt_prefix;
+  p.sched = a.sched;
   p.E = a.E;
   p.mt_sh = a.fs > 0 ? (a.rows_sh + bm - 1) / bm : 0;
   p.rows_sh = a.rows_sh;

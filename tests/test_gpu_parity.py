@@ -77,6 +77,28 @@ def test_small_parity_each_tile_mode(name, mode, monkeypatch):
     H.parity(inputgen.make_problem(wl, seed=5))
 
 
+@pytest.mark.parametrize("mode", ["1", "2"])
+@pytest.mark.parametrize("name", ["bf16_ragged", "bf16_shared", "bf16_empty", "bf16_maxE"])
+def test_claimed_tile_schedule_matches_static_bit_for_bit(name, mode, monkeypatch):
+    # The bf16 GEMMs claim their tiles from a counter that the last CTA of each launch zeroes for
+    # the next one; COLIBRI_TILE_SCHED=static walks them round-robin.  Which CTA computes a tile
+    # changes nothing in it, so repeated calls on one context (the counter reset each time) must
+    # equal the static schedule bit for bit and match the oracle.
+    monkeypatch.setenv("COLIBRI_GEMM_CTA", mode)
+    wl = SMALL[name]
+    p = inputgen.make_problem(wl, seed=17)
+    t = H.to_device(p)
+    outs = {}
+    for sched in ("static", "claimed"):
+        monkeypatch.setenv("COLIBRI_TILE_SCHED", sched)
+        layer = H.make_layer(wl)
+        outs[sched] = [H.run_gpu(p, layer=layer, dev_inputs=t)["y"] for _ in range(3)]
+        layer.close()
+    for y in outs["claimed"] + outs["static"][1:]:
+        assert torch.equal(y, outs["static"][0])
+    H.parity(p)
+
+
 I8_SMALL = [n for n, w in SMALL.items() if w.wdt == I8]
 
 
