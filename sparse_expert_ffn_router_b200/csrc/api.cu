@@ -228,9 +228,6 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   const size_t plane_w = (size_t)std::max<int64_t>(d, f);
   const size_t o_phi = c.take(i8 ? R * plane_w : 0), o_plo = c.take(i8 ? R * plane_w : 0);
   const size_t o_psc = c.take(i8 ? part_rows * 4 : 0);  // per (down K split, row) scales of the H planes
-  const bool rsplit = D.act_dtype == COLIBRI_BF16 && M >= kRouterSplitMinT;
-  const size_t o_rpart = c.take(rsplit ? (size_t)kRouterMaxSplit * M * E * 4 : 0);
-  const size_t o_rtick = c.take(rsplit ? (size_t)((M + 127) / 128) * 4 : 0);
   const size_t o_err = c.take(4);
   const size_t o_tsched = c.take(4 * 4);
   const size_t o_gbar = c.take(i8 ? kFusedBarCount * 4 : 0);
@@ -278,10 +275,7 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   w.flow_hlo = i8 ? reinterpret_cast<int8_t*>(b + o_fhl) : nullptr;
   w.flow_hscale = i8 ? reinterpret_cast<float*>(b + o_fhs) : nullptr;
   w.flow_rows = i8 ? (int)flow_rows : 0;
-  w.router_part = rsplit ? reinterpret_cast<float*>(b + o_rpart) : nullptr;
-  w.router_ticket = rsplit ? reinterpret_cast<int32_t*>(b + o_rtick) : nullptr;
   if (cudaMemset(w.err, 0, 4) != cudaSuccess || cudaMemset(w.tile_sched, 0, 4 * 4) != cudaSuccess ||
-      (rsplit && cudaMemset(w.router_ticket, 0, (size_t)((M + 127) / 128) * 4) != cudaSuccess) ||
       (i8 && cudaMemset(w.grid_bar, 0, kFusedBarCount * 4) != cudaSuccess) ||
       (i8 && cudaMemset(w.flow_ctr, 0, flow_bytes) != cudaSuccess)) {
     cudaFree(ctx->ws_base);
@@ -404,8 +398,7 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
     COLIBRI_TRY(cudaMemcpyAsync(w.topk_w, user_w, (size_t)R * 4, cudaMemcpyDeviceToDevice, s), "copy topk_w");
     launch_chain_break();
   } else if (!route_in_dec) {
-    COLIBRI_TRY(launch_router_topk(xd, act, T, d, router_w, router_b, E, k, D.router_flags, w.topk_idx, w.topk_w, w.err,
-                                   w.router_part, w.router_ticket, s),
+    COLIBRI_TRY(launch_router_topk(xd, act, T, d, router_w, router_b, E, k, D.router_flags, w.topk_idx, w.topk_w, w.err, s),
                 "router_topk");
   }
   mark(1);

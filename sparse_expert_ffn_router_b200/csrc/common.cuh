@@ -75,8 +75,6 @@ struct Workspace {
   void* Hs = nullptr;   // [M, fs]
   void* Ys = nullptr;   // [M, d]
   float* Ypart = nullptr;  // [split, M*k, d] f32, int8 path
-  float* router_part = nullptr;    // [8, M, E] K-split partial logits
-  int32_t* router_ticket = nullptr;  // [ceil(M/128)] arrival counters (zero between calls)
   int32_t* grid_bar = nullptr;       // [4] grid-barrier counters of the fused int8 kernel (zero between calls)
   int32_t* flow_ctr = nullptr;       // [kFlowUnitCtrs + kFlowTileCtrs] dataflow int8 kernel (zero between calls)
   int8_t* flow_hhi = nullptr;        // [flow_rows, f] H planes of the dataflow int8 kernel
@@ -195,15 +193,12 @@ __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.lau
 // Kernel launchers (each returns cudaGetLastError() of its launch)
 // ---------------------------------------------------------------------------------------
 // err: the context's device error word for bounded waits that give up (may be NULL).
-// part/ticket: [8, T, E] partial logits and [ceil(T/128)] zeroed counters for the K-split
-// router used when T >= kRouterSplitMinT (NULL: no split).
 constexpr int kRouterSmallT = 64;       // T up to which one CTA per token computes the logits
-constexpr int kRouterSplitMinT = 2048;  // T from which the tensor-core router splits K
-constexpr int kRouterMaxSplit = 8;
+constexpr int kRouterMaxSplit = 4;      // K slices per token tile of the tensor-core router (a cluster)
+constexpr int kRouterCtaBudget = 160;   // CTAs the tensor-core router aims to stay within
 int router_ksplit(int T, int d);
 cudaError_t launch_router_topk(const void* x, int act, int T, int d, const void* wr, const float* b,
-                               int E, int k, int rflags, int32_t* idx, float* w, uint32_t* err, float* part,
-                               int32_t* ticket, cudaStream_t s);
+                               int E, int k, int rflags, int32_t* idx, float* w, uint32_t* err, cudaStream_t s);
 cudaError_t launch_route_count(const int32_t* idx, int T, int k, int E, int32_t* blk_counts,
                                int32_t* local_rank, cudaStream_t s);
 cudaError_t launch_route_scan(const int32_t* blk_counts, int nblk, int E, int bm, int32_t* blk_base,
@@ -705,6 +700,9 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
 // 32-bit store into the shared memory of a CTA of the cluster (address from mapa_shared).
 __device__ __forceinline__ void st_shared_cluster_u32(uint32_t cluster_addr, int32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st_shared_cluster_f32(uint32_t cluster_addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cluster_addr), "f"(v) : "memory");
 }
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");

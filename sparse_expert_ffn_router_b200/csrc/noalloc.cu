@@ -119,7 +119,7 @@ extern "C" colibri_status colibri_route_noalloc(const void* x, int32_t act_dtype
   cudaError_t e = cudaMemsetAsync(err, 0, sizeof(uint32_t), s);
   if (e == cudaSuccess)
     e = launch_router_topk(x, act_dtype, T, d_model, router_w, router_b, num_experts, top_k, 0, topk_idx, topk_w,
-                           err, nullptr, nullptr, s);
+                           err, s);
   if (e == cudaSuccess) e = launch_route_count(topk_idx, T, top_k, num_experts, blk_counts, dst_row, s);
   if (e == cudaSuccess)
     e = launch_route_scan(blk_counts, (int)nblk, num_experts, kTcBM, blk_base, counts, offsets, mt_prefix, s);

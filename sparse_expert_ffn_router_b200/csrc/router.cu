@@ -155,9 +155,7 @@ struct alignas(64) RouterTcParams {
   const float* b;
   int T, d, E, k, N;
   int rflags;        // kRouterClamp | kRouterRaw
-  int ksplit;        // CTAs per 128-token tile, each over d / ksplit (gridDim.y)
-  float* part;       // [ksplit, E, T] partial logits (ksplit > 1; token-contiguous, so stores coalesce)
-  int32_t* ticket;   // [tiles] arrival counters, zero between calls (ksplit > 1)
+  int ksplit;        // CTAs per 128-token tile (one cluster, gridDim.x), each over d / ksplit
   int stages;  // ring depth: as many stages as fit in kRtRingBytes (small expert counts go deeper)
   int kbs;     // consecutive 64-wide K blocks per stage (1 or 2): each x row is read kbs x 128 bytes at a time
   uint32_t stage_bytes, tmem_cols;
@@ -179,7 +177,27 @@ __device__ __forceinline__ bool rt_wait(uint64_t* bar, uint32_t parity, volatile
   }
 }
 
-__global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant__ RouterTcParams p) {
+// Insert (v, e) into a list of the k best kept in (logit descending, expert ascending) order.
+template <int KK>
+__device__ __forceinline__ void rt_insert_ordered(float (&bv)[KK], int (&bi)[KK], int k, float v, int e) {
+#pragma unroll
+  for (int j = 0; j < KK; ++j) {
+    if (j < k && (v > bv[j] || (v == bv[j] && e < bi[j]))) {
+      const float tv = bv[j];
+      const int ti = bi[j];
+      bv[j] = v;
+      bi[j] = e;
+      v = tv;
+      e = ti;
+    }
+  }
+}
+
+constexpr int kRtThreads = 256;
+
+// KK: the top-k list length the kernel is compiled for (k <= KK)
+template <int KK>
+__global__ void __launch_bounds__(kRtThreads, 1) router_tc_kernel(const __grid_constant__ RouterTcParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {  // the 128-byte swizzle needs 1024-byte aligned tiles
     pdl_wait();
@@ -217,9 +235,10 @@ __global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const int row0 = blockIdx.x * 128;
+  const int split = blockIdx.x, tile = blockIdx.y;  // the K slices of a tile form one cluster
+  const int row0 = tile * 128;
   const int kspan = p.d / p.ksplit;               // a multiple of 64
-  const int kb0 = blockIdx.y * (kspan / 64);
+  const int kb0 = split * (kspan / 64);
   const int nkb = kspan / 64;
   // A stage holds kbs consecutive K blocks: x tiles first, then the Wr tiles.
   const int kbs = p.kbs, nst = nkb / kbs;
@@ -228,7 +247,7 @@ __global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant
   // The CTAs of a launch start their K walk at different stages (rotated by the tile index), so
   // the x rows read at one time do not all sit at the same column offset, which would put every
   // request on the same DRAM channels.  (This fixes, per tile, the order of the fp32 sum.)
-  const int st_rot = blockIdx.x % nst;
+  const int st_rot = tile % nst;
   if (warp == 0) {
     if (lane == 0) {
       // ----------------------------------------------------------- TMA producer
@@ -288,88 +307,147 @@ __global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant
     }
     __syncwarp();
   }
-  // ------------------------------------------------------------- epilogue: one token per thread
+  // ------------------------------------------------------------- epilogue
   const bool got = rt_wait(done, 0, abort_flag) && !*abort_flag;
   const bool warp_ok = __all_sync(0xffffffffu, got);
   tc_fence_after();
-  float bv[kMaxTopK];
-  int bi[kMaxTopK];
+  const int q = warp & 3, half = warp >> 2;
+  const int nchunks = p.N / 16, nc0 = (nchunks + 1) / 2;
+  const int cbeg = half ? nc0 : 0, cend = half ? nchunks : nc0;
+  const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
+  __shared__ float merge_v[kRtThreads][KK];  // per-thread selections, merged per token
+  __shared__ int merge_i[kRtThreads][KK];
+  // Selection: order by (logit descending, expert ascending).  The experts a thread sees are
+  // spread over kChains chains; each chain sees its experts in ascending order and keeps its k
+  // best by insertion with a strict ">" (an equal logit never displaces the lower index seen
+  // first), so every chain holds its exact top k; chains and threads are then merged comparing
+  // (logit, index), which gives the exact top k of all experts.  Independent chains keep one
+  // thread's compare-and-insert work from being one long dependent sequence.
+  constexpr int kChains = 4;
+  float bv[kChains][KK];
+  int bi[kChains][KK];
+  float thr[kChains];
 #pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j) {
-    bv[j] = -INFINITY;
-    bi[j] = 0x7fffffff;
-  }
-  __shared__ int last_cta;
-  const int t = row0 + threadIdx.x;
-  const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16);
-  bool select = warp_ok;
-  if (p.ksplit > 1) {
-    // write this K slice's logits, then the last CTA of the tile sums the slices in order
-    if (warp_ok) {
-      for (int c0 = 0; c0 < p.N; c0 += 16) {
-        float v[16];
-        tmem_ld16(tbase + c0, v);
-        tmem_ld_wait();
-        if (t < p.T)
+  for (int g = 0; g < kChains; ++g) {
+    thr[g] = -INFINITY;
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (c0 + i < p.E) p.part[((size_t)blockIdx.y * p.E + c0 + i) * p.T + t] = v[i];
-      }
+    for (int j = 0; j < KK; ++j) {
+      bv[g][j] = -INFINITY;
+      bi[g][j] = 0x7fffffff;
     }
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) last_cta = (atomicAdd(&p.ticket[blockIdx.x], 1) == p.ksplit - 1);
-    __syncthreads();
-    select = __all_sync(0xffffffffu, warp_ok) && last_cta;
-    if (last_cta && threadIdx.x == 0) p.ticket[blockIdx.x] = 0;  // ready for the next call
-    __threadfence();
   }
-  if (select) {
-    for (int c0 = 0; c0 < p.N; c0 += 16) {
-      float v[16];
-      if (p.ksplit == 1) {
-        tmem_ld16(tbase + c0, v);
-        tmem_ld_wait();
-      } else {
-        // the 16 experts' partials of one split are loaded together, then added in split order
+  auto offer = [&](int g, int e, float l) {
+    float cv = router_clamp(l + (p.b ? p.b[e] : 0.f), p.rflags);
+    if (cv > thr[g]) {
+      int ci = e;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = 0.f;
-        for (int sp = 0; sp < p.ksplit; ++sp) {
-          float pv[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pv[i] = (t < p.T && c0 + i < p.E) ? __ldcg(&p.part[((size_t)sp * p.E + c0 + i) * p.T + t]) : 0.f;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] += pv[i];
+      for (int j = 0; j < KK; ++j) {
+        if (j < p.k && cv > bv[g][j]) {
+          const float tv = bv[g][j];
+          const int ti = bi[g][j];
+          bv[g][j] = cv;
+          bi[g][j] = ci;
+          cv = tv;
+          ci = ti;
         }
       }
+      thr[g] = bv[g][0];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int e = c0 + i;
-        if (e < p.E) {
-          float cv = router_clamp(v[i] + (p.b ? p.b[e] : 0.f), p.rflags);
-          int ci = e;
+      for (int j = 1; j < KK; ++j) thr[g] = j < p.k ? bv[g][j] : thr[g];
+    }
+  };
+  int tl, part, nparts;  // token within the tile this thread selects for, its share of the experts
+  if (p.ksplit == 1) {
+    // two threads per token: warp w reads TMEM lane quarter w & 3 (tokens 32 (w & 3) + lane)
+    // and the 16-column chunks of expert half w >> 2
+    tl = q * 32 + lane;
+    part = half;
+    nparts = 2;
+    if (warp_ok) {
+      for (int c = cbeg; c < cend; ++c) {
+        float v[16];
+        tmem_ld16(tbase + c * 16, v);
+        tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < kMaxTopK; ++j) {
-            if (j < p.k && cv > bv[j]) {
-              const float tv = bv[j];
-              const int ti = bi[j];
-              bv[j] = cv;
-              bi[j] = ci;
-              cv = tv;
-              ci = ti;
-            }
+        for (int i = 0; i < 16; ++i)
+          if (c * 16 + i < p.E) offer(i % kChains, c * 16 + i, v[i]);
+      }
+    }
+  } else {
+    // The ksplit CTAs of the tile form a cluster; CTA r selects for the tokens
+    // [r tpc, (r + 1) tpc), tpc = 128 / ksplit.  Every CTA pushes its slice of each token's logits
+    // into the shared memory (the idle ring) of the CTA that owns the token, as
+    // stage[slice][expert][token - owner tpc]; after one cluster barrier each CTA adds the slices
+    // of its tokens in K order from its own shared memory.
+    const int tpc = 128 / p.ksplit;
+    float* stage = reinterpret_cast<float*>(smem);
+    const int tq = q * 32 + lane;  // this thread's TMEM row
+    const uint32_t dst = mapa_shared(smem_u32(stage), (uint32_t)(tq / tpc)) +
+                         (uint32_t)(split * p.N * tpc + tq % tpc) * 4u;
+    if (warp_ok) {
+      for (int c = cbeg; c < cend; ++c) {
+        float v[16];
+        tmem_ld16(tbase + c * 16, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) st_shared_cluster_f32(dst + (uint32_t)((c * 16 + i) * tpc) * 4u, v[i]);
+      }
+    }
+    cluster_sync_all();  // every slice has arrived (release / acquire at cluster scope)
+    nparts = min(kRtThreads / tpc, (p.E + 7) / 8);  // at least 8 experts per thread
+    tl = split * tpc + threadIdx.x % tpc;
+    part = threadIdx.x / tpc;
+    if (part < nparts) {
+      const float* mine = stage + threadIdx.x % tpc;
+      for (int e0 = part; e0 < p.E; e0 += nparts * kChains) {
+        float v[kChains];
+#pragma unroll
+        for (int g = 0; g < kChains; ++g) v[g] = 0.f;
+        for (int sp = 0; sp < p.ksplit; ++sp) {
+#pragma unroll
+          for (int g = 0; g < kChains; ++g) {
+            const int e = e0 + g * nparts;
+            v[g] += e < p.E ? mine[(sp * p.N + e) * tpc] : 0.f;
           }
         }
+#pragma unroll
+        for (int g = 0; g < kChains; ++g)
+          if (e0 + g * nparts < p.E) offer(g, e0 + g * nparts, v[g]);
       }
     }
-    if (t < p.T) {
-      float wv[kMaxTopK];
-      topk_weights(bv, p.k, p.rflags, wv);
+  }
+  const bool select = __syncthreads_and(warp_ok) != 0;
+  if (select) {
 #pragma unroll
-      for (int j = 0; j < kMaxTopK; ++j)
+    for (int g = 1; g < kChains; ++g)
+#pragma unroll
+      for (int j = 0; j < KK; ++j)
+        if (j < p.k) rt_insert_ordered<KK>(bv[0], bi[0], p.k, bv[g][j], bi[g][j]);
+#pragma unroll
+    for (int j = 0; j < KK; ++j) {
+      merge_v[threadIdx.x][j] = bv[0][j];
+      merge_i[threadIdx.x][j] = bi[0][j];
+    }
+  }
+  __syncthreads();
+  const int t = row0 + tl;
+  if (select && part == 0) {
+    const int stride = p.ksplit == 1 ? 128 : 128 / p.ksplit;  // threads of one token: tid + m * stride
+    for (int m = 1; m < nparts; ++m) {
+      const int o = threadIdx.x + m * stride;
+#pragma unroll
+      for (int j = 0; j < KK; ++j)
+        if (j < p.k) rt_insert_ordered<KK>(bv[0], bi[0], p.k, merge_v[o][j], merge_i[o][j]);
+    }
+    if (t < p.T) {
+      float sv[kMaxTopK], wv[kMaxTopK];
+#pragma unroll
+      for (int j = 0; j < kMaxTopK; ++j) sv[j] = j < KK ? bv[0][j < KK ? j : 0] : -INFINITY;
+      topk_weights(sv, p.k, p.rflags, wv);
+#pragma unroll
+      for (int j = 0; j < KK; ++j)
         if (j < p.k) {
-          p.idx[(size_t)t * p.k + j] = bi[j];
+          p.idx[(size_t)t * p.k + j] = bi[0][j];
           p.w[(size_t)t * p.k + j] = wv[j];
         }
     }
@@ -390,14 +468,10 @@ __global__ void __launch_bounds__(128, 1) router_tc_kernel(const __grid_constant
 constexpr size_t kRtMaxSmem = kRtRingBytes + 1024;
 
 cudaError_t launch_router_tc(const void* x, int T, int d, const void* wr, const float* b, int E, int k,
-                             int rflags, int32_t* idx, float* w, uint32_t* err, int ksplit, float* part,
-                             int32_t* ticket, cudaStream_t s) {
+                             int rflags, int32_t* idx, float* w, uint32_t* err, int ksplit, cudaStream_t s) {
   RouterTcParams p;
   memset(&p, 0, sizeof(p));
   p.N = (E + 15) / 16 * 16;
-  p.ksplit = ksplit;
-  p.part = part;
-  p.ticket = ticket;
   {
     const uint64_t dims[2] = {(uint64_t)d, (uint64_t)T}, st[1] = {(uint64_t)d * 2};
     const uint32_t box[2] = {64, 128};
@@ -416,16 +490,26 @@ cudaError_t launch_router_tc(const void* x, int T, int d, const void* wr, const 
   p.rflags = rflags;
   // two consecutive K blocks per stage when the slice has an even number of them (256 contiguous
   // bytes of each x row per copy pair instead of 128)
-  p.kbs = ((d / ksplit) / 64) % 2 == 0 ? 2 : 1;
-  p.stage_bytes = (uint32_t)((p.kbs * (kRtABytes + p.N * 128) + 1023) / 1024 * 1024);
-  p.stages = (int)std::min<size_t>(kRtMaxStages, kRtRingBytes / p.stage_bytes);
+  auto ring = [&](int ks) {
+    p.ksplit = ks;
+    p.kbs = ((d / ks) / 64) % 2 == 0 ? 2 : 1;
+    p.stage_bytes = (uint32_t)((p.kbs * (kRtABytes + p.N * 128) + 1023) / 1024 * 1024);
+    p.stages = (int)std::min<size_t>(kRtMaxStages, kRtRingBytes / p.stage_bytes);
+  };
+  ring(ksplit);
+  // a split tile stages its [N][128] fp32 logits in the ring
+  if (ksplit > 1 && (size_t)p.N * 128 * 4 > (size_t)p.stages * p.stage_bytes) ring(1);
   p.tmem_cols = 32;
   while ((int)p.tmem_cols < p.N) p.tmem_cols <<= 1;
   p.idx = idx;
   p.w = w;
   p.err = err;
   const size_t smem = (size_t)p.stages * p.stage_bytes + 1024;
-  return launch_kernel(router_tc_kernel, dim3((T + 127) / 128, ksplit), dim3(128), smem, s, 1, p);
+  const dim3 grid(p.ksplit, (T + 127) / 128);
+  const unsigned cl = (unsigned)p.ksplit;
+  if (k <= 2) return launch_kernel(router_tc_kernel<2>, grid, dim3(kRtThreads), smem, s, cl, p);
+  if (k <= 4) return launch_kernel(router_tc_kernel<4>, grid, dim3(kRtThreads), smem, s, cl, p);
+  return launch_kernel(router_tc_kernel<8>, grid, dim3(kRtThreads), smem, s, cl, p);
 }
 
 }  // namespace
@@ -439,21 +523,25 @@ cudaError_t configure_router_kernels() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(router_topk_simt_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, simt);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRtMaxSmem);
+    e = cudaFuncSetAttribute(router_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRtMaxSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(router_tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRtMaxSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(router_tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRtMaxSmem);
   return e;
 }
 
+// K slices per 128-token tile: the most (up to 8, dividing the 64-wide K blocks) that keep the
+// launch within about one CTA per SM.
 int router_ksplit(int T, int d) {
-  if (T < kRouterSplitMinT) return 1;
   const int tiles = (T + 127) / 128;
   int ks = 1;
-  while (ks < 8 && tiles * ks * 2 <= 160 && (d / 64) % (2 * ks) == 0) ks <<= 1;
+  while (ks < kRouterMaxSplit && tiles * ks * 2 <= kRouterCtaBudget && (d / 64) % (2 * ks) == 0) ks <<= 1;
   return ks;
 }
 
 cudaError_t launch_router_topk(const void* x, int act, int T, int d, const void* wr, const float* b,
-                               int E, int k, int rflags, int32_t* idx, float* w, uint32_t* err, float* part,
-                               int32_t* ticket, cudaStream_t s) {
+                               int E, int k, int rflags, int32_t* idx, float* w, uint32_t* err, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
   if (T <= kRouterSmallT) {
     if (act == COLIBRI_BF16)
@@ -463,8 +551,7 @@ cudaError_t launch_router_topk(const void* x, int act, int T, int d, const void*
                          (const float*)wr, b, E, k, rflags, idx, w);
   }
   if (act == COLIBRI_BF16) {
-    const int ks = (part && ticket) ? router_ksplit(T, d) : 1;
-    return launch_router_tc(x, T, d, wr, b, E, k, rflags, idx, w, err, ks, part, ticket, s);
+    return launch_router_tc(x, T, d, wr, b, E, k, rflags, idx, w, err, router_ksplit(T, d), s);
   }
   const size_t smem =
       sizeof(float) * ((size_t)kRouterTT * (kRouterDK + 1) + (size_t)E * (kRouterDK + 1) +
