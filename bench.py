@@ -40,11 +40,13 @@ METRIC = "MoE-layer tokens/sec (prefill & decode) and % of roofline on 1 B200"
 DEFAULT_WORKLOAD = "mixtral_prefill_bf16"
 # T up to which the Scatter stage is one fused launch (histogram, prefix sum and scatter)
 FUSED_ROUTE_MAX_T = 64
+# T up to which int4 weights take the CUDA-core GEMV kernels (d and f multiples of 1024)
+GEMV4_MAX_T = 4
 
 
 def kernels_per_step(wl):
     """Kernels one forward launches, following the library's launch sequence."""
-    if wl.wdt == 3:  # int4: router, Scatter, gate/up stream, H planes, down stream, combine
+    if wl.wdt == 3:  # int4: router, Scatter, gate/up (stream or GEMV), H planes, down, combine
         return 1 + (1 if wl.T <= FUSED_ROUTE_MAX_T else 3) + 4
     fused_int8 = wl.wdt == 2 and os.environ.get("COLIBRI_DEC_FUSED", "1") != "0"
     if fused_int8 and wl.T <= FUSED_ROUTE_MAX_T and os.environ.get("COLIBRI_DEC_ROUTE", "1") != "0":
@@ -462,7 +464,12 @@ def roofline(wl, wk, stage_ms, pk):
         wbytes = wk["w13_bytes"] + wk["w2_bytes"] + wk["scale_bytes"]
         ms = stage_ms["expert_gateup"] + stage_ms["expert_down"] + stage_ms["gather"]
         achieved = wbytes / (ms / 1e3) / 1e9
-        roof = {"kernel": ("dec_stream4_kernel<gate/up> + dec_finish_h_kernel + dec_stream4_kernel<down> + "
+        gemv = (wl.T <= GEMV4_MAX_T and wl.d % 1024 == 0 and wl.f % 1024 == 0
+                and os.environ.get("COLIBRI_I4_GEMV", "1") != "0")
+        roof = {"kernel": ("gemv4_kernel<gate/up> + dec_finish_h_kernel + gemv4_kernel<down> + combine_split_kernel "
+                           "(dp4a on the CUDA cores, packed int4 weights read straight into registers, group "
+                           "scales per 32-element chunk)") if gemv else
+                          ("dec_stream4_kernel<gate/up> + dec_finish_h_kernel + dec_stream4_kernel<down> + "
                            "combine_split_kernel (packed int4 tiles widened to int8 in shared memory, tcgen05 "
                            "kind::i8, group scales per K block)"),
                 "bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",

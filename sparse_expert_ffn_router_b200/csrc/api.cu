@@ -294,6 +294,8 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   ctx->use_graphs = !(getenv("COLIBRI_GRAPHS") && strcmp(getenv("COLIBRI_GRAPHS"), "0") == 0);
   // COLIBRI_TILE_SCHED=static: the bf16 GEMMs walk their tiles round-robin instead of claiming them
   ctx->tile_static = getenv("COLIBRI_TILE_SCHED") && strcmp(getenv("COLIBRI_TILE_SCHED"), "static") == 0;
+  // COLIBRI_I4_GEMV=0: int4 weights always take the tensor-core stream kernels
+  ctx->i4_gemv = !(getenv("COLIBRI_I4_GEMV") && strcmp(getenv("COLIBRI_I4_GEMV"), "0") == 0);
   // Programmatic dependent launch measured slower on the small-batch decode chain and neutral on
   // prefill, so it is opt-in (COLIBRI_PDL=1).
   ctx->use_pdl = env_flag("COLIBRI_PDL");
@@ -487,7 +489,17 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
              touched * tiles * gsplit < 8 * ctx->sm_count)
         gsplit <<= 1;
     }
-    if (D.weight_dtype == COLIBRI_I4) {
+    if (D.weight_dtype == COLIBRI_I4 && ctx->i4_gemv && T <= kGemv4MaxT && gemv4_supported(d, f)) {
+      // int4 at decode sizes: dp4a GEMV for gate/up, H planes, dp4a GEMV for down
+      nsplit = gemv4_down_split(f, ctx->dec_split);
+      COLIBRI_TRY(launch_gemv4_gateup(w.plane_hi, w.plane_lo, w.plane_scale, (const uint8_t*)expert_w, expert_scales,
+                                      stride, d, f, E, w.offsets, (float*)w.H, R, T, s), "gemv4_gateup");
+      mark(3);
+      COLIBRI_TRY(launch_dec_finish_h((const float*)w.H, 1, R, f, nsplit, w.plane_hi, w.plane_lo, w.plane_scale, s),
+                  "dec_finish_h");
+      COLIBRI_TRY(launch_gemv4_down(w.plane_hi, w.plane_lo, w.plane_scale, (const uint8_t*)expert_w, expert_scales,
+                                    stride, d, f, E, w.offsets, nsplit, R, w.Ypart, T, s), "gemv4_down");
+    } else if (D.weight_dtype == COLIBRI_I4) {
       // int4: the stream kernels that widen the packed tiles, then H planes, then down
       COLIBRI_TRY(launch_dec4_gateup(w.plane_hi, w.plane_lo, w.plane_scale, (const uint8_t*)expert_w, expert_scales,
                                      stride, d, f, E, w.offsets, gsplit, (float*)w.H, R, T, w.err, s), "dec4_gateup");

@@ -53,6 +53,11 @@ SMALL = {
     "i4_T1": inputgen.custom("i4_T1", T=1, d=256, E=8, k=2, f=256, act=BF16, wdt=I4),
     "i4_many": inputgen.custom("i4_many", T=80, d=128, E=2, k=1, f=256, act=BF16, wdt=I4),
     "i4_wide_d": inputgen.custom("i4_wide_d", T=9, d=512, E=4, k=2, f=128, act=BF16, wdt=I4),
+    # d and f multiples of 1024 at T <= 4: the CUDA-core GEMV plan (one row per expert; a few;
+    # up to 4 rows of one expert, taken two at a time; a down projection split in two)
+    "i4_gemv_T1": inputgen.custom("i4_gemv_T1", T=1, d=1024, E=8, k=2, f=2048, act=BF16, wdt=I4),
+    "i4_gemv_T3": inputgen.custom("i4_gemv_T3", T=3, d=1024, E=4, k=2, f=1024, act=BF16, wdt=I4),
+    "i4_gemv_T4": inputgen.custom("i4_gemv_T4", T=4, d=2048, E=2, k=1, f=1024, act=BF16, wdt=I4),
 }
 
 
@@ -97,6 +102,15 @@ def test_claimed_tile_schedule_matches_static_bit_for_bit(name, mode, monkeypatc
     for y in outs["claimed"] + outs["static"][1:]:
         assert torch.equal(y, outs["static"][0])
     H.parity(p)
+
+
+@pytest.mark.parametrize("gemv", ["0", "1"])
+@pytest.mark.parametrize("name", ["i4_gemv_T1", "i4_gemv_T3", "i4_gemv_T4"])
+def test_int4_both_plans(name, gemv, monkeypatch):
+    # int4 weights at T <= 4 with d and f multiples of 1024 take the CUDA-core GEMV kernels by
+    # default; COLIBRI_I4_GEMV=0 keeps the tensor-core stream kernels.  Both meet the oracle.
+    monkeypatch.setenv("COLIBRI_I4_GEMV", gemv)
+    H.parity(inputgen.make_problem(SMALL[name], seed=27))
 
 
 I8_SMALL = [n for n, w in SMALL.items() if w.wdt == I8]
@@ -537,6 +551,14 @@ def test_full_size_workload(name, n_sample):
     # the near-tie protocol's count, reported in pytest's warnings summary (kept even with -q)
     warnings.warn(NearTieReport(f"{name}: {res['near_ties']} near-tie tokens of {wl.T}; "
                                 f"max abs err / max|ref| = {res['rel_err']:.3e}"))
+
+
+@pytest.mark.parametrize("name", ["decode_int4_T1"])
+def test_full_size_int4_stream_plan(name, monkeypatch):
+    # the tensor-core stream kernels at the full decode sizes (the default there is the GEMV plan)
+    monkeypatch.setenv("COLIBRI_I4_GEMV", "0")
+    wl = inputgen.WORKLOADS[name]
+    H.parity(inputgen.make_problem(wl, seed=0), tokens=H.sample_tokens(wl.T, 8))
 
 
 class NearTieReport(UserWarning):
