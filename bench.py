@@ -40,8 +40,9 @@ METRIC = "MoE-layer tokens/sec (prefill & decode) and % of roofline on 1 B200"
 DEFAULT_WORKLOAD = "mixtral_prefill_bf16"
 # T up to which the Scatter stage is one fused launch (histogram, prefix sum and scatter)
 FUSED_ROUTE_MAX_T = 64
-# T up to which int4 weights take the CUDA-core GEMV kernels (d and f multiples of 1024)
-GEMV4_MAX_T = 4
+# T up to which int4 weights take the GEMV kernels (d and f multiples of 1024): dp4a up to 2 tokens,
+# warp-level MMA beyond
+GEMV4_MAX_T = 16
 
 
 def kernels_per_step(wl):
@@ -466,9 +467,10 @@ def roofline(wl, wk, stage_ms, pk):
         achieved = wbytes / (ms / 1e3) / 1e9
         gemv = (wl.T <= GEMV4_MAX_T and wl.d % 1024 == 0 and wl.f % 1024 == 0
                 and os.environ.get("COLIBRI_I4_GEMV", "1") != "0")
-        roof = {"kernel": ("gemv4_kernel<gate/up> + dec_finish_h_kernel + gemv4_kernel<down> + combine_split_kernel "
-                           "(dp4a on the CUDA cores, packed int4 weights read straight into registers, group "
-                           "scales per 32-element chunk)") if gemv else
+        gk = "gemv4_kernel" if wl.T <= 2 else "gemv4m_kernel"
+        how = ("dp4a on the CUDA cores" if wl.T <= 2 else "mma.sync m16n8k32 s8, up to 8 tokens per instruction")
+        roof = {"kernel": (f"{gk}<gate/up> + dec_finish_h_kernel + {gk}<down> + combine_split_kernel "
+                           f"({how}, packed int4 weights read straight into registers, group scales)") if gemv else
                           ("dec_stream4_kernel<gate/up> + dec_finish_h_kernel + dec_stream4_kernel<down> + "
                            "combine_split_kernel (packed int4 tiles widened to int8 in shared memory, tcgen05 "
                            "kind::i8, group scales per K block)"),

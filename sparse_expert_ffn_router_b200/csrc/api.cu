@@ -492,11 +492,12 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
     if (D.weight_dtype == COLIBRI_I4 && ctx->i4_gemv && T <= kGemv4MaxT && gemv4_supported(d, f)) {
       // int4 at decode sizes: dp4a GEMV for gate/up, H planes, dp4a GEMV for down
       nsplit = gemv4_down_split(f, ctx->dec_split);
+      const int g4split = gemv4_gateup_split(d, T);
       COLIBRI_TRY(launch_gemv4_gateup(w.plane_hi, w.plane_lo, w.plane_scale, (const uint8_t*)expert_w, expert_scales,
-                                      stride, d, f, E, w.offsets, (float*)w.H, R, T, s), "gemv4_gateup");
+                                      stride, d, f, E, w.offsets, g4split, (float*)w.H, R, T, s), "gemv4_gateup");
       mark(3);
-      COLIBRI_TRY(launch_dec_finish_h((const float*)w.H, 1, R, f, nsplit, w.plane_hi, w.plane_lo, w.plane_scale, s),
-                  "dec_finish_h");
+      COLIBRI_TRY(launch_dec_finish_h((const float*)w.H, g4split, R, f, nsplit, w.plane_hi, w.plane_lo,
+                                      w.plane_scale, s), "dec_finish_h");
       COLIBRI_TRY(launch_gemv4_down(w.plane_hi, w.plane_lo, w.plane_scale, (const uint8_t*)expert_w, expert_scales,
                                     stride, d, f, E, w.offsets, nsplit, R, w.Ypart, T, s), "gemv4_down");
     } else if (D.weight_dtype == COLIBRI_I4) {

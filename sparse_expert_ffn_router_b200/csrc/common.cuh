@@ -123,7 +123,7 @@ struct colibri_ctx {
   uint64_t graph_clock = 0;
   bool use_graphs = true;
   bool tile_static = false;  // bf16 GEMMs: static round-robin tiles instead of the claimed schedule
-  bool i4_gemv = true;       // int4 weights, T <= kGemv4MaxT: CUDA-core GEMV instead of the stream kernels
+  bool i4_gemv = true;       // int4 weights, T <= kGemv4MaxT: GEMV kernels instead of the stream kernels
   bool use_pdl = false;  // programmatic dependent launch between the kernels of a forward (opt-in)
   bool dec_fused = true;  // int8 weights: the one-launch expert stage (COLIBRI_DEC_FUSED=0: four launches)
   bool dec_route = true;  // int8, T <= 64: routing inside that launch too (COLIBRI_DEC_ROUTE=0: not)
@@ -306,15 +306,16 @@ cudaError_t launch_dec4_gateup(const int8_t* Xhi, const int8_t* Xlo, const float
 cudaError_t launch_dec4_down(const int8_t* Hhi, const int8_t* Hlo, const float* hscale, const uint8_t* W,
                              const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
                              int nsplit, int R, float* Ypart, int max_rows_per_expert, uint32_t* err, cudaStream_t s);
-// Group-wise int4 weights at decode sizes: dp4a GEMV on the CUDA cores over the same planes and
-// outputs as the two stream kernels above (gate/up without K split; down with nsplit splits of
-// f / nsplit, a multiple of 1024).  Needs d and f multiples of 1024.
-constexpr int kGemv4MaxT = 4;  // tokens up to which the int4 path uses the GEMV kernels
+// Group-wise int4 weights at decode sizes: GEMV kernels over the same planes and outputs as the
+// two stream kernels above (gate/up with gsplit K splits, down with nsplit, each split a multiple
+// of 1024 wide).  Needs d and f multiples of 1024.
+constexpr int kGemv4MaxT = 16;  // tokens up to which the int4 path uses the GEMV kernels
 bool gemv4_supported(int d, int f);
 int gemv4_down_split(int f, int max_split);
+int gemv4_gateup_split(int d, int T);
 cudaError_t launch_gemv4_gateup(const int8_t* Xhi, const int8_t* Xlo, const float* xscale, const uint8_t* W,
                                 const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
-                                float* GU, int R, int max_rows_per_expert, cudaStream_t s);
+                                int gsplit, float* GU, int R, int max_rows_per_expert, cudaStream_t s);
 cudaError_t launch_gemv4_down(const int8_t* Hhi, const int8_t* Hlo, const float* hscale, const uint8_t* W,
                               const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
                               int nsplit, int R, float* Ypart, int max_rows_per_expert, cudaStream_t s);

@@ -1,6 +1,6 @@
 // Expert Compute stage for group-wise int4 weights at decode sizes, on the CUDA cores.
 //
-// With at most 4 tokens each packed weight byte meets only a row or two of activations, so the work
+// With a few tokens each packed weight byte meets only a few rows of activations, so the work
 // is a stream over the touched experts' weights and the tensor-core path (which first widens each
 // packed tile to int8 in shared memory) spends more time on that hand-off than on the stream.
 // Here the dot products run as dp4a on the same int8 activation planes the tensor-core path uses
@@ -22,8 +22,11 @@
 //
 // Work: one warp per task = (touched expert, matrix, 8 consecutive output rows, K split), for all
 // of the expert's rows; tasks are enumerated over the touched experts only, consecutive warps on
-// consecutive rows of one matrix, so the activation chunks they share stay in L1.
+// consecutive rows of one matrix, so the activation chunks they share stay in L1 (the weight
+// stream bypasses it).  This dp4a kernel serves one or two rows per expert; from three rows on the
+// warp-level MMA kernel below takes over (up to 8 rows per instruction).
 #include <algorithm>
+#include <cstdlib>
 
 #include "common.cuh"
 
@@ -48,6 +51,16 @@ struct Gemv4Params {
   float* out;              // GU [2][R][f] or Ypart [nsplit][R][d]
   bool gateup;
 };
+
+// 16 bytes of the weight stream: read once, so kept out of L1 (the activation planes, re-read by
+// every warp of the expert, stay there)
+__device__ __forceinline__ uint4 ld_stream16(const void* ptr) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(ptr));
+  return v;
+}
 
 __device__ __forceinline__ float exact_i2f(int v) {  // |v| < 2^22: the float of v without I2F
   return __int_as_float(v + 0x4B400000) - 12582912.0f;
@@ -121,7 +134,7 @@ __global__ void __launch_bounds__(kG4Threads, 1) gemv4_kernel(const __grid_const
       auto load_w = [&](uint4 (&dst)[kG4Rows], int n) {
         const uint8_t* src = wbase + (size_t)(lane + 32 * n) * 16;
 #pragma unroll
-        for (int r = 0; r < kG4Rows; ++r) dst[r] = __ldg(reinterpret_cast<const uint4*>(src + (size_t)r * row_bytes));
+        for (int r = 0; r < kG4Rows; ++r) dst[r] = ld_stream16(src + (size_t)r * row_bytes);
       };
       if (nsteps > 0) load_w(wcur, 0);
       for (int n = 0; n < nsteps; ++n) {
@@ -189,10 +202,171 @@ __global__ void __launch_bounds__(kG4Threads, 1) gemv4_kernel(const __grid_const
         if (t < nr && lane == t) {
           const int row = row0 + t;
           const float a = __ldcg(p.rscale + (size_t)sp * p.rscale_split_stride + row);
-          float* dst = p.gateup ? p.out + ((size_t)m * p.R + row) * p.f + o0
+          float* dst = p.gateup ? p.out + (((size_t)sp * 2 + m) * p.R + row) * p.f + o0
                                 : p.out + ((size_t)sp * p.R + row) * p.d + o0;
           reinterpret_cast<float4*>(dst)[0] = make_float4(a * acc[0][t], a * acc[1][t], a * acc[2][t], a * acc[3][t]);
           reinterpret_cast<float4*>(dst)[1] = make_float4(a * acc[4][t], a * acc[5][t], a * acc[6][t], a * acc[7][t]);
+        }
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------- warp-level MMA plan
+// The same contraction on the tensor cores through the warp-level mma.sync.m16n8k32 (s8 x s8 ->
+// s32), the weights unpacked in registers (no shared-memory staging): up to 8 tokens share each
+// instruction, so the work per weight byte no longer grows with the token count.  A warp task is
+// (touched expert, matrix, 32 output rows, K split) for all of the expert's rows, 8 at a time.
+// Lane (g = lane / 4, t = lane % 4) reads, per K group (128 elements), the 16 packed bytes
+// [32 t, 32 t + 32) of rows g, g + 8, g + 16, g + 24; MMA kk (0..3) of the group takes from every
+// lane the 8 elements 32 t + 8 kk + [0, 8) of its rows — even elements (16 q, as above) in the
+// A register of columns 4 t.., odd ones in that of columns 16 + 4 t.. — and the activation bytes
+// of token g at the same K positions, permuted the same way, as B.  The contraction order over K
+// is thereby permuted identically in A and B, which leaves the exact int32 group sums unchanged.
+// Per group and plane the MMA accumulators (rows g, g + 8 of each 16-row half, tokens 2 t, 2 t + 1)
+// are scaled by the group scale and added into fp32 registers.
+constexpr int kG4mThreads = 384;
+constexpr int kG4mRows = 32;
+constexpr int kG4mAhead = 2;  // K groups of weight loads in flight per warp beyond the current one
+
+__device__ __forceinline__ void mma_s8_16x8x32(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__global__ void __launch_bounds__(kG4mThreads, 1) gemv4m_kernel(const __grid_constant__ Gemv4Params p) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ int32_t off_s[kMaxExperts + 1];
+  __shared__ int32_t touched[kMaxExperts];
+  __shared__ int32_t n_touched;
+  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) off_s[i] = p.offsets[i];
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    int base = 0;
+    for (int e0 = 0; e0 < p.E; e0 += 32) {
+      const int e = e0 + (int)threadIdx.x;
+      const bool has = e < p.E && off_s[e + 1] > off_s[e];
+      const unsigned m = __ballot_sync(0xffffffffu, has);
+      if (has) touched[base + __popc(m & ((1u << threadIdx.x) - 1u))] = e;
+      base += __popc(m);
+    }
+    if (threadIdx.x == 0) n_touched = base;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int ntiles = p.out_rows / kG4mRows;
+  const int per_e = p.mats * p.nsplit * ntiles;
+  const int tasks = n_touched * per_e;
+  const int ngr = p.kspan / 128;
+  const size_t mat_bytes = (size_t)p.d * p.f / 2;
+  const size_t scales_per_mat = (size_t)p.d * p.f / 128;
+  const size_t row_bytes = (size_t)p.K / 2;
+
+  for (int task = blockIdx.x * (kG4mThreads / 32) + (threadIdx.x >> 5); task < tasks;
+       task += gridDim.x * (kG4mThreads / 32)) {
+    const int te = task / per_e;
+    int rest = task - te * per_e;
+    const int ot = rest % ntiles;
+    rest /= ntiles;
+    const int sp = rest % p.nsplit;
+    const int m = rest / p.nsplit;
+    const int e = touched[te];
+    const int r_beg = off_s[e], r_end = off_s[e + 1];
+    const int o0 = ot * kG4mRows;
+    const int kbeg = sp * p.kspan;
+    // this lane's packed bytes: rows o0 + g + 8 j, bytes [16 t, 16 t + 16) of every 64-byte group
+    const uint8_t* wbase = p.W + (size_t)e * (size_t)(p.wstride / 2) +
+                           (p.gateup ? (size_t)m * mat_bytes : 2 * mat_bytes) + (size_t)(o0 + g) * row_bytes +
+                           kbeg / 2 + 16 * t;
+    const float* sbase = p.wscale + (size_t)e * 3 * scales_per_mat + (size_t)(p.gateup ? m : 2) * scales_per_mat +
+                         (size_t)(kbeg / 128) * p.out_rows + o0 + g;
+
+    for (int row0 = r_beg; row0 < r_end; row0 += 8) {
+      const int nr = min(8, r_end - row0);
+      const bool has_tok = g < nr;  // this lane supplies B for token g
+      const int8_t* hp = p.hi + (size_t)(row0 + (has_tok ? g : 0)) * p.K + kbeg + 32 * t;
+      const int8_t* lp = p.lo + (size_t)(row0 + (has_tok ? g : 0)) * p.K + kbeg + 32 * t;
+      float acc[4][2];  // rows g + 8 j, tokens 2 t, 2 t + 1
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[j][0] = acc[j][1] = 0.f;
+      uint4 wq[kG4mAhead + 1][4];
+      auto load_w = [&](uint4 (&dst)[4], int gi) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          dst[j] = ld_stream16(wbase + (size_t)(8 * j) * row_bytes + (size_t)gi * 64);
+      };
+#pragma unroll
+      for (int a = 0; a < kG4mAhead; ++a)
+        if (a < ngr) load_w(wq[a], a);
+      for (int gi = 0; gi < ngr; ++gi) {
+        // rotate the prefetch window (register arrays indexed by constants only)
+        if (gi + kG4mAhead < ngr) load_w(wq[kG4mAhead], gi + kG4mAhead);
+        uint4 w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) w[j] = wq[0][j];
+#pragma unroll
+        for (int a = 0; a < kG4mAhead; ++a)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) wq[a][j] = wq[a + 1][j];
+        // activation bytes of token g at K 128 gi + 32 t + [0, 32), both planes
+        uint4 h0 = make_uint4(0, 0, 0, 0), h1 = h0, l0 = h0, l1 = h0;
+        if (has_tok) {
+          h0 = __ldg(reinterpret_cast<const uint4*>(hp + 128 * gi));
+          h1 = __ldg(reinterpret_cast<const uint4*>(hp + 128 * gi + 16));
+          l0 = __ldg(reinterpret_cast<const uint4*>(lp + 128 * gi));
+          l1 = __ldg(reinterpret_cast<const uint4*>(lp + 128 * gi + 16));
+        }
+        const uint32_t hw[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+        const uint32_t lw[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+        int dh[2][4], dl[2][4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dh[h][i] = dl[h][i] = 0;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          // B: token g's 8 bytes at 32 t + 8 kk, even ones then odd ones
+          const uint32_t bhe = __byte_perm(hw[2 * kk], hw[2 * kk + 1], 0x6420);
+          const uint32_t bho = __byte_perm(hw[2 * kk], hw[2 * kk + 1], 0x7531);
+          const uint32_t ble = __byte_perm(lw[2 * kk], lw[2 * kk + 1], 0x6420);
+          const uint32_t blo = __byte_perm(lw[2 * kk], lw[2 * kk + 1], 0x7531);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {  // 16-row halves: rows g + 16 h and g + 8 + 16 h
+            const uint32_t wa = (kk == 0 ? w[2 * h].x : kk == 1 ? w[2 * h].y : kk == 2 ? w[2 * h].z : w[2 * h].w);
+            const uint32_t wb = (kk == 0 ? w[2 * h + 1].x : kk == 1 ? w[2 * h + 1].y : kk == 2 ? w[2 * h + 1].z
+                                                                                          : w[2 * h + 1].w);
+            const uint32_t a[4] = {(wa << 4) & 0xF0F0F0F0u, (wb << 4) & 0xF0F0F0F0u, wa & 0xF0F0F0F0u,
+                                   wb & 0xF0F0F0F0u};
+            mma_s8_16x8x32(dh[h], a, bhe, bho);
+            mma_s8_16x8x32(dl[h], a, ble, blo);
+          }
+        }
+        // the group's exact sums (x 16) times its scales / 16
+        const float* sg = sbase + (size_t)gi * p.out_rows;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float s0 = __ldg(sg + 16 * h) * 0.0625f, s1 = __ldg(sg + 16 * h + 8) * 0.0625f;
+          acc[2 * h][0] = fmaf(s0, exact_i2f(dh[h][0]) + exact_i2f(dl[h][0]) * (1.0f / 254.0f), acc[2 * h][0]);
+          acc[2 * h][1] = fmaf(s0, exact_i2f(dh[h][1]) + exact_i2f(dl[h][1]) * (1.0f / 254.0f), acc[2 * h][1]);
+          acc[2 * h + 1][0] = fmaf(s1, exact_i2f(dh[h][2]) + exact_i2f(dl[h][2]) * (1.0f / 254.0f), acc[2 * h + 1][0]);
+          acc[2 * h + 1][1] = fmaf(s1, exact_i2f(dh[h][3]) + exact_i2f(dl[h][3]) * (1.0f / 254.0f), acc[2 * h + 1][1]);
+        }
+      }
+      // lane (g, t) holds rows o0 + g + 8 j for tokens 2 t and 2 t + 1
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int tok = 2 * t + c;
+        if (tok < nr) {
+          const int row = row0 + tok;
+          const float a = __ldcg(p.rscale + (size_t)sp * p.rscale_split_stride + row);
+          float* dst = p.gateup ? p.out + (((size_t)sp * 2 + m) * p.R + row) * p.f + o0 + g
+                                : p.out + ((size_t)sp * p.R + row) * p.d + o0 + g;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) dst[8 * j] = a * acc[j][c];
         }
       }
     }
@@ -212,6 +386,12 @@ int sm_count_here() {
 
 cudaError_t launch_gemv4(const Gemv4Params& p, int max_rows_per_expert, cudaStream_t s) {
   const int grid = sm_count_here();
+  // up to 2 rows per expert the dp4a kernel, beyond that the warp-MMA one (measured on B200:
+  // 4096 x 14336 layer, T = 1: 87 against 123 us per call; T = 8: 380 against 242 us);
+  // COLIBRI_I4_GEMV_MMA=0 / 1 forces one of them
+  const char* force = getenv("COLIBRI_I4_GEMV_MMA");
+  const bool mma_plan = force ? atoi(force) != 0 : max_rows_per_expert > 2;
+  if (mma_plan) return launch_kernel(gemv4m_kernel, dim3(grid), dim3(kG4mThreads), 0, s, 1, p);
   if (max_rows_per_expert <= 1) return launch_kernel(gemv4_kernel<1>, dim3(grid), dim3(kG4Threads), 0, s, 1, p);
   return launch_kernel(gemv4_kernel<2>, dim3(grid), dim3(kG4Threads), 0, s, 1, p);
 }
@@ -219,6 +399,10 @@ cudaError_t launch_gemv4(const Gemv4Params& p, int max_rows_per_expert, cudaStre
 }  // namespace
 
 bool gemv4_supported(int d, int f) { return d % 1024 == 0 && f % 1024 == 0; }
+
+// a second K split of the gate/up projection doubles its tasks when only one or two experts are
+// touched (fewer tasks than warps otherwise leave SMs idle at the end)
+int gemv4_gateup_split(int d, int T) { return T <= 2 && (d / 1024) % 2 == 0 ? 2 : 1; }
 
 int gemv4_down_split(int f, int max_split) {
   int ns = 1;
@@ -228,8 +412,8 @@ int gemv4_down_split(int f, int max_split) {
 
 cudaError_t launch_gemv4_gateup(const int8_t* Xhi, const int8_t* Xlo, const float* xscale, const uint8_t* W,
                                 const float* scales, int64_t wstride, int d, int f, int E, const int32_t* offsets,
-                                float* GU, int R, int max_rows_per_expert, cudaStream_t s) {
-  if (!gemv4_supported(d, f)) return cudaErrorInvalidValue;
+                                int gsplit, float* GU, int R, int max_rows_per_expert, cudaStream_t s) {
+  if (!gemv4_supported(d, f) || gsplit < 1 || (d / gsplit) % 1024 != 0) return cudaErrorInvalidValue;
   Gemv4Params p{};
   p.W = W;
   p.wscale = scales;
@@ -246,8 +430,8 @@ cudaError_t launch_gemv4_gateup(const int8_t* Xhi, const int8_t* Xlo, const floa
   p.K = d;
   p.out_rows = f;
   p.mats = 2;
-  p.nsplit = 1;
-  p.kspan = d;
+  p.nsplit = gsplit;
+  p.kspan = d / gsplit;
   p.out = GU;
   p.gateup = true;
   return launch_gemv4(p, max_rows_per_expert, s);

@@ -53,11 +53,12 @@ SMALL = {
     "i4_T1": inputgen.custom("i4_T1", T=1, d=256, E=8, k=2, f=256, act=BF16, wdt=I4),
     "i4_many": inputgen.custom("i4_many", T=80, d=128, E=2, k=1, f=256, act=BF16, wdt=I4),
     "i4_wide_d": inputgen.custom("i4_wide_d", T=9, d=512, E=4, k=2, f=128, act=BF16, wdt=I4),
-    # d and f multiples of 1024 at T <= 4: the CUDA-core GEMV plan (one row per expert; a few;
-    # up to 4 rows of one expert, taken two at a time; a down projection split in two)
+    # d and f multiples of 1024 at T <= 16: the GEMV plans (one row per expert; a few; up to 4
+    # rows of one expert; 12 rows of one expert, more than one MMA's 8; a down projection split in two)
     "i4_gemv_T1": inputgen.custom("i4_gemv_T1", T=1, d=1024, E=8, k=2, f=2048, act=BF16, wdt=I4),
     "i4_gemv_T3": inputgen.custom("i4_gemv_T3", T=3, d=1024, E=4, k=2, f=1024, act=BF16, wdt=I4),
     "i4_gemv_T4": inputgen.custom("i4_gemv_T4", T=4, d=2048, E=2, k=1, f=1024, act=BF16, wdt=I4),
+    "i4_gemv_T12": inputgen.custom("i4_gemv_T12", T=12, d=1024, E=1, k=1, f=1024, act=BF16, wdt=I4),
 }
 
 
@@ -104,12 +105,15 @@ def test_claimed_tile_schedule_matches_static_bit_for_bit(name, mode, monkeypatc
     H.parity(p)
 
 
-@pytest.mark.parametrize("gemv", ["0", "1"])
-@pytest.mark.parametrize("name", ["i4_gemv_T1", "i4_gemv_T3", "i4_gemv_T4"])
-def test_int4_both_plans(name, gemv, monkeypatch):
-    # int4 weights at T <= 4 with d and f multiples of 1024 take the CUDA-core GEMV kernels by
-    # default; COLIBRI_I4_GEMV=0 keeps the tensor-core stream kernels.  Both meet the oracle.
-    monkeypatch.setenv("COLIBRI_I4_GEMV", gemv)
+@pytest.mark.parametrize("plan", [("0", None), ("1", "0"), ("1", "1")])
+@pytest.mark.parametrize("name", ["i4_gemv_T1", "i4_gemv_T3", "i4_gemv_T4", "i4_gemv_T12"])
+def test_int4_each_plan(name, plan, monkeypatch):
+    # int4 weights at T <= 16 with d and f multiples of 1024 take a GEMV kernel by default (dp4a
+    # up to 2 rows per expert, warp-level MMA beyond); COLIBRI_I4_GEMV=0 keeps the tensor-core
+    # stream kernels, COLIBRI_I4_GEMV_MMA=0 / 1 forces either GEMV.  All meet the oracle.
+    monkeypatch.setenv("COLIBRI_I4_GEMV", plan[0])
+    if plan[1] is not None:
+        monkeypatch.setenv("COLIBRI_I4_GEMV_MMA", plan[1])
     H.parity(inputgen.make_problem(SMALL[name], seed=27))
 
 
