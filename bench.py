@@ -69,9 +69,9 @@ def kernels_per_step(wl):
 # same kernel on the same workload (profiles/); None where no capture of the current kernel
 # exists.  Keyed by (workload, dominant-kernel tag).
 NCU_TRAFFIC = {
-    ("mixtral_prefill_bf16", "tc2_ffn"): 3.1173e9 + 0.2305e9,      # tc2_ffn_traffic_mixtral_prefill_bf16.md
-    ("fine_grained_shared_bf16", "tc_ffn"): 1.00698e9 + 74.0e6,   # launches_fine_grained_shared_bf16.md
-    ("skewed_bf16", "tc_ffn"): 2.286978e9 + 0.060185e9,           # tc_ffn_traffic_skewed_bf16.md
+    ("mixtral_prefill_bf16", "tc2_ffn"): 1.9466e9 + 0.2246e9,      # launches_mixtral_prefill_bf16.md
+    ("fine_grained_shared_bf16", "tc_ffn"): 1.0004e9 + 0.0707e9,  # launches_fine_grained_shared_bf16.md
+    ("skewed_bf16", "tc_ffn"): 2.2694e9 + 0.0581e9,               # tc_ffn_traffic_skewed_bf16.md
 }
 
 # fp32 FMA peak: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (the unit counts and clock of the part)
