@@ -32,6 +32,8 @@
 // shared memory; the last CTA to finish zeroes the counter for the next launch.
 // Every wait is bounded (kWaitTimeoutNs); a wait that gives up sets the error word, makes the
 // other roles leave their loops, drains outstanding copies and MMAs and frees TMEM.
+#include <cstdlib>
+
 #include "common.cuh"
 
 namespace colibri {
@@ -48,8 +50,11 @@ constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
 
 struct alignas(64) TcParams {
   CUtensorMap mapA;     // routed A rows
-  CUtensorMap mapA16;   // the same rows, boxes of 16 and 64 rows (light tiles copy only what
-  CUtensorMap mapA64;   // their MMAs read)
+  CUtensorMap mapA16;   // the same rows, boxes of 16, 32 and 64 rows (light tiles copy only what
+  CUtensorMap mapA32;   // their MMAs read)
+  CUtensorMap mapA64;
+  CUtensorMap mapB16;   // gate/up weights viewed as [d, 16 rows, W1|W3, f / 16, E]: one box holds 4 x
+                        // (16 W1 rows, the same 16 W3 rows) (pair light tiles)
   CUtensorMap mapB;     // routed weights
   CUtensorMap mapA_sh;  // shared-expert A rows
   CUtensorMap mapB_sh;  // shared-expert weights
@@ -59,6 +64,7 @@ struct alignas(64) TcParams {
   int E;
   int n_tiles, n_tiles_sh;
   int mt_sh, rows_sh;
+  int pair_light_rows;  // pair kernel: m-tiles with at most this many rows are swapped tails (<= 64)
   int num_kb, num_kb_sh;
   int n_out, n_out_sh;  // output row widths (elements)
   __nv_bfloat16* out;
@@ -577,6 +583,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc_ffn_kernel(const __grid_con
 // barrier.  Per 128x256x64 unit of work a CTA moves 32 KB from L2 instead of 48 KB.
 constexpr int BM2 = 256;
 constexpr int STAGES2 = kTcPairStages;
+// A pair m-tile with at most kPairLightRows rows (an expert's short last tile) is computed with
+// the operands swapped, like the one-CTA light tiles: the weights are the M = 256 side (128 rows
+// per CTA) and the tile's rows the N side (N = rows rounded up to 16, N / 2 rows per CTA), so the
+// tail costs a fraction of a 256 x 256 tile and still reads its weight blocks from L2 in the same
+// launch as the expert's other m-tiles.  For gate/up each CTA's 128 weight rows are 4 x (16 W1
+// rows, the same 16 W3 rows), so that gate and up of one output column meet in one warp.
+constexpr int kPairLightRows = 64;
+constexpr int kPairLightBoxRows = 32;  // token rows copied per CTA (at least N / 2)
 constexpr int HALF_BYTES = 128 * BK * 2;          // 16 KB
 constexpr int STAGE2_BYTES = 2 * HALF_BYTES;      // A half + B half
 constexpr uint32_t IDESC2 = idesc_bf16_f32(BM2, BN);
@@ -640,6 +654,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
     mbar_fence_init();
     tma_prefetch_desc(&p.mapA);
     tma_prefetch_desc(&p.mapB);
+    tma_prefetch_desc(&p.mapA32);
+    if (kGateUp) tma_prefetch_desc(&p.mapB16);
     if (p.mt_sh > 0) {
       tma_prefetch_desc(&p.mapA_sh);
       tma_prefetch_desc(&p.mapB_sh);
@@ -703,6 +719,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
         const CUtensorMap* mA = t.sh ? &p.mapA_sh : &p.mapA;
         const CUtensorMap* mB = t.sh ? &p.mapB_sh : &p.mapB;
         const int arow = t.row0 + 128 * (int)rank;
+        const bool light = !t.sh && t.row_end - t.row0 <= p.pair_light_rows;
+        const int nh = (t.row_end - t.row0 + 15) / 16 * 8;  // light: token rows (N / 2) per CTA
         const int claim_kb = t.num_kb > STAGES2 ? t.num_kb - STAGES2 : 0;
         int next = L;
         bool ok = true;
@@ -714,16 +732,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
           }
           uint8_t* sA = stage_base + (size_t)s * STAGE2_BYTES;
           uint8_t* sB = sA + HALF_BYTES;
-          if (rank == 0) mbar_arrive_expect_tx(&m.full[s], 2 * STAGE2_BYTES);
           const uint32_t bar = mapa_shared(smem_u32(&m.full[s]), 0);
           const int kx = kb * BK;
-          tma2_load_2d(sA, mA, bar, kx, arow);
-          if (kGateUp) {
-            if (t.sh) tma2_load_3d(sB, mB, bar, kx, t.n0, (int)rank);
-            else tma2_load_4d(sB, mB, bar, kx, t.n0, (int)rank, t.e);
+          if (light) {
+            // swapped tail: weights into the A slot, the tile's token rows into the B slot
+            if (rank == 0) mbar_arrive_expect_tx(&m.full[s], 2 * (HALF_BYTES + kPairLightBoxRows * BK * 2));
+            if (kGateUp) {
+              tma2_load_5d(sA, &p.mapB16, bar, kx, 0, 0, (t.n0 + 64 * (int)rank) / 16, t.e);
+            } else {
+              tma2_load_3d(sA, mB, bar, kx, t.n0 + 128 * (int)rank, t.e);
+            }
+            tma2_load_2d(sB, &p.mapA32, bar, kx, t.row0 + (int)rank * nh);
           } else {
-            if (t.sh) tma2_load_2d(sB, mB, bar, kx, t.n0 + 128 * (int)rank);
-            else tma2_load_3d(sB, mB, bar, kx, t.n0 + 128 * (int)rank, t.e);
+            if (rank == 0) mbar_arrive_expect_tx(&m.full[s], 2 * STAGE2_BYTES);
+            tma2_load_2d(sA, mA, bar, kx, arow);
+            if (kGateUp) {
+              if (t.sh) tma2_load_3d(sB, mB, bar, kx, t.n0, (int)rank);
+              else tma2_load_4d(sB, mB, bar, kx, t.n0, (int)rank, t.e);
+            } else {
+              if (t.sh) tma2_load_2d(sB, mB, bar, kx, t.n0 + 128 * (int)rank);
+              else tma2_load_3d(sB, mB, bar, kx, t.n0 + 128 * (int)rank, t.e);
+            }
           }
           if (++s == STAGES2) {
             s = 0;
@@ -769,6 +798,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(a * BN);
+        const int trows = t.row_end - t.row0;
+        // light tail: M = 256 weight rows, N = the tile's rows rounded up to 16
+        const uint32_t idesc = (!t.sh && trows <= p.pair_light_rows) ? idesc_bf16_f32(BM2, (trows + 15) / 16 * 16) : IDESC2;
         for (int kb = 0; kb < t.num_kb; ++kb) {
           if (!wait_or_abort(&m.full[s], ph, abort_flag)) {
             ok = false;
@@ -781,7 +813,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = smem_desc_sw128(sA + kk * 32);
             const uint64_t bd = smem_desc_sw128(sB + kk * 32);
-            tc_mma_f16_pair(d_tmem, ad, bd, IDESC2, (kb | kk) != 0 ? 1u : 0u);
+            tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
           tc_commit_pair_mc(&m.empty[s], 0x3);
           if (++s == STAGES2) {
@@ -832,7 +864,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * BN);
       __nv_bfloat16* out = t.sh ? p.out_sh : p.out;
       const int n_out = t.sh ? p.n_out_sh : p.n_out;
-      if (kGateUp) {
+      const int trows = t.row_end - t.row0;
+      if (!t.sh && trows <= p.pair_light_rows) {
+        // swapped tail: TMEM lane = weight row of this CTA, column c = the tile's row t.row0 + c
+        if (kGateUp) {
+          // lanes 0-15 of warp q: gate of output column n0 + 64 rank + 16 q + lane; lanes 16-31: up
+          const int oc = t.n0 + 64 * (int)rank + 16 * q + (lane & 15);
+          for (int c = 0; c < trows; c += 16) {
+            float v[16];
+            tmem_ld16(tb + c, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float up = __shfl_down_sync(0xffffffffu, v[i], 16);
+              if (lane < 16 && c + i < trows && oc < n_out)
+                out[(size_t)(t.row0 + c + i) * n_out + oc] = __float2bfloat16_rn(silu_mul(v[i], up));
+            }
+          }
+        } else {
+          const int oc = t.n0 + 128 * (int)rank + q * 32 + lane;
+          for (int c = 0; c < trows; c += 16) {
+            float v[16];
+            tmem_ld16(tb + c, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (c + i < trows && oc < n_out) out[(size_t)(t.row0 + c + i) * n_out + oc] = __float2bfloat16_rn(v[i]);
+          }
+        }
+      } else if (kGateUp) {
 #pragma unroll 1
         for (int c = 0; c < BN / 2; c += 16) {
           float g[16], u[16];
@@ -956,12 +1016,17 @@ cudaError_t launch_tc(const TcGemmArgs& a, cudaStream_t s) {
       ok &= make_map(&p.mapA, a.A, 2, dims, st, box);
       box[1] = 16;
       ok &= make_map(&p.mapA16, a.A, 2, dims, st, box);
+      box[1] = kPairLightBoxRows;
+      ok &= make_map(&p.mapA32, a.A, 2, dims, st, box);
       box[1] = 64;
       ok &= make_map(&p.mapA64, a.A, 2, dims, st, box); }
-    // B: W1|W3 of every expert as [d, f, 2, E]
+    // B: W1|W3 of every expert as [d, f, 2, E] (and in 16-row boxes)
     { uint64_t dims[4] = {d, f, 2, (uint64_t)a.E}, st[3] = {d * 2, f * d * 2, S};
       uint32_t box[4] = {BK, BN / 2, 1, 1};
       ok &= make_map(&p.mapB, a.W, 4, dims, st, box); }
+    { uint64_t dims[5] = {d, 16, 2, f / 16, (uint64_t)a.E}, st[4] = {d * 2, f * d * 2, 16 * d * 2, S};
+      uint32_t box[5] = {BK, 16, 2, 4, 1};
+      ok &= f % 16 == 0 && make_map(&p.mapB16, a.W, 5, dims, st, box); }
     if (a.fs > 0) {
       { uint64_t dims[2] = {d, (uint64_t)a.rows_sh}, st[1] = {d * 2}; uint32_t box[2] = {BK, BM};
         ok &= make_map(&p.mapA_sh, a.A_sh, 2, dims, st, box); }
@@ -980,6 +1045,8 @@ cudaError_t launch_tc(const TcGemmArgs& a, cudaStream_t s) {
       ok &= make_map(&p.mapA, a.A, 2, dims, st, box);
       box[1] = 16;
       ok &= make_map(&p.mapA16, a.A, 2, dims, st, box);
+      box[1] = kPairLightBoxRows;
+      ok &= make_map(&p.mapA32, a.A, 2, dims, st, box);
       box[1] = 64;
       ok &= make_map(&p.mapA64, a.A, 2, dims, st, box); }
     // B: W2 of every expert as [f, d, E], starting 2*f*d elements into the expert
@@ -1005,6 +1072,11 @@ cudaError_t launch_tc(const TcGemmArgs& a, cudaStream_t s) {
   p.E = a.E;
   p.mt_sh = a.fs > 0 ? (a.rows_sh + bm - 1) / bm : 0;
   p.rows_sh = a.rows_sh;
+  {
+    // COLIBRI_PAIR_LIGHT=0 computes every pair m-tile as a full 256 x 256 tile
+    const char* v = getenv("COLIBRI_PAIR_LIGHT");
+    p.pair_light_rows = v && atoi(v) == 0 ? 0 : kPairLightRows;
+  }
   p.out = (__nv_bfloat16*)a.out;
   p.out_sh = (__nv_bfloat16*)a.out_sh;
   p.err = a.err;

@@ -404,9 +404,13 @@ bool gemv4_supported(int d, int f) { return d % 1024 == 0 && f % 1024 == 0; }
 // touched (fewer tasks than warps otherwise leave SMs idle at the end)
 int gemv4_gateup_split(int d, int T) { return T <= 2 && (d / 1024) % 2 == 0 ? 2 : 1; }
 
+// K splits of the down projection: the largest divisor of f / 1024 up to 8 (f = 14336: 7 splits of
+// 2048), so that the H-plane kernel (one CTA per row and split) and the down GEMV both get enough
+// CTAs and tasks for a single token
 int gemv4_down_split(int f, int max_split) {
   int ns = 1;
-  while (ns * 2 <= max_split && (f / 1024) % (ns * 2) == 0 && ns < 2) ns *= 2;
+  for (int c = 2; c <= 8 && c <= max_split; ++c)
+    if ((f / 1024) % c == 0) ns = c;
   return ns;
 }
 
