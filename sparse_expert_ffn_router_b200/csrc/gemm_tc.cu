@@ -589,8 +589,7 @@ constexpr int STAGES2 = kTcPairStages;
 // tail costs a fraction of a 256 x 256 tile and still reads its weight blocks from L2 in the same
 // launch as the expert's other m-tiles.  For gate/up each CTA's 128 weight rows are 4 x (16 W1
 // rows, the same 16 W3 rows), so that gate and up of one output column meet in one warp.
-constexpr int kPairLightRows = 64;
-constexpr int kPairLightBoxRows = 32;  // token rows copied per CTA (at least N / 2)
+constexpr int kPairLightRows = 128;  // N <= 128: at most 64 token rows per CTA (a 32- or 64-row box)
 constexpr int HALF_BYTES = 128 * BK * 2;          // 16 KB
 constexpr int STAGE2_BYTES = 2 * HALF_BYTES;      // A half + B half
 constexpr uint32_t IDESC2 = idesc_bf16_f32(BM2, BN);
@@ -655,6 +654,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
     tma_prefetch_desc(&p.mapA);
     tma_prefetch_desc(&p.mapB);
     tma_prefetch_desc(&p.mapA32);
+    tma_prefetch_desc(&p.mapA64);
     if (kGateUp) tma_prefetch_desc(&p.mapB16);
     if (p.mt_sh > 0) {
       tma_prefetch_desc(&p.mapA_sh);
@@ -736,13 +736,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
           const int kx = kb * BK;
           if (light) {
             // swapped tail: weights into the A slot, the tile's token rows into the B slot
-            if (rank == 0) mbar_arrive_expect_tx(&m.full[s], 2 * (HALF_BYTES + kPairLightBoxRows * BK * 2));
+            const int box_rows = nh <= 32 ? 32 : 64;
+            if (rank == 0) mbar_arrive_expect_tx(&m.full[s], 2 * (HALF_BYTES + box_rows * BK * 2));
             if (kGateUp) {
               tma2_load_5d(sA, &p.mapB16, bar, kx, 0, 0, (t.n0 + 64 * (int)rank) / 16, t.e);
             } else {
               tma2_load_3d(sA, mB, bar, kx, t.n0 + 128 * (int)rank, t.e);
             }
-            tma2_load_2d(sB, &p.mapA32, bar, kx, t.row0 + (int)rank * nh);
+            tma2_load_2d(sB, nh <= 32 ? &p.mapA32 : &p.mapA64, bar, kx, t.row0 + (int)rank * nh);
           } else {
             if (rank == 0) mbar_arrive_expect_tx(&m.full[s], 2 * STAGE2_BYTES);
             tma2_load_2d(sA, mA, bar, kx, arow);
@@ -1016,7 +1017,7 @@ cudaError_t launch_tc(const TcGemmArgs& a, cudaStream_t s) {
       ok &= make_map(&p.mapA, a.A, 2, dims, st, box);
       box[1] = 16;
       ok &= make_map(&p.mapA16, a.A, 2, dims, st, box);
-      box[1] = kPairLightBoxRows;
+      box[1] = 32;
       ok &= make_map(&p.mapA32, a.A, 2, dims, st, box);
       box[1] = 64;
       ok &= make_map(&p.mapA64, a.A, 2, dims, st, box); }
@@ -1045,7 +1046,7 @@ cudaError_t launch_tc(const TcGemmArgs& a, cudaStream_t s) {
       ok &= make_map(&p.mapA, a.A, 2, dims, st, box);
       box[1] = 16;
       ok &= make_map(&p.mapA16, a.A, 2, dims, st, box);
-      box[1] = kPairLightBoxRows;
+      box[1] = 32;
       ok &= make_map(&p.mapA32, a.A, 2, dims, st, box);
       box[1] = 64;
       ok &= make_map(&p.mapA64, a.A, 2, dims, st, box); }
