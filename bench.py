@@ -70,8 +70,8 @@ def kernels_per_step(wl):
 # exists.  Keyed by (workload, dominant-kernel tag).
 NCU_TRAFFIC = {
     ("mixtral_prefill_bf16", "tc2_ffn"): 1.9466e9 + 0.2246e9,      # launches_mixtral_prefill_bf16.md
-    ("fine_grained_shared_bf16", "tc_ffn"): 1.0004e9 + 0.0707e9,  # launches_fine_grained_shared_bf16.md
-    ("skewed_bf16", "tc_ffn"): 2.2694e9 + 0.0581e9,               # tc_ffn_traffic_skewed_bf16.md
+    ("fine_grained_shared_bf16", "tc2_ffn"): 1.0012e9 + 0.0707e9,  # launches_fine_grained_shared_bf16.md
+    ("skewed_bf16", "tc2_ffn"): 2.2216e9 + 0.0584e9,               # tc_ffn_traffic_skewed_bf16.md
 }
 
 # fp32 FMA peak: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz (the unit counts and clock of the part)
@@ -492,9 +492,7 @@ def roofline(wl, wk, stage_ms, pk):
     elif wl.wdt == 1:
         ms = stage_ms["expert_gateup"]
         achieved = wk["flops_gateup"] / (ms / 1e3) / 1e12
-        mode = os.environ.get("COLIBRI_GEMM_CTA", "")[:1]
-        if mode not in ("1", "2"):
-            mode = "2" if wl.T * wl.k // wl.E >= 512 else "1"
+        mode = "1" if os.environ.get("COLIBRI_GEMM_CTA", "")[:1] == "1" else "2"
         name = {"1": "tc_ffn_kernel<gate/up> (tcgen05, 128x256 tiles)",
                 "2": "tc2_ffn_kernel<gate/up> (tcgen05, 2-CTA 256x256 pair tiles)"}[mode]
         roof = {"kernel": name, "bound": "tensor", "achieved": achieved, "peak": pk["bf16"], "unit": "TFLOP/s",

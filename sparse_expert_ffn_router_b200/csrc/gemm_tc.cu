@@ -688,6 +688,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
       int q = 0;
       uint32_t qph = 0;
       int L = pair;
+      const uint64_t evict_first = l2_evict_first_policy();
       while (true) {
         // the leader claims tiles and publishes each number to both CTAs; the peer reads its copy
         int Lq;
@@ -738,10 +739,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
             // swapped tail: weights into the A slot, the tile's token rows into the B slot
             const int box_rows = nh <= 32 ? 32 : 64;
             if (rank == 0) mbar_arrive_expect_tx(&m.full[s], 2 * (HALF_BYTES + box_rows * BK * 2));
+            // an expert with this single m-tile streams its weights: evict them from L2 first
             if (kGateUp) {
-              tma2_load_5d(sA, &p.mapB16, bar, kx, 0, 0, (t.n0 + 64 * (int)rank) / 16, t.e);
+              if (t.mtiles == 1)
+                tma2_load_5d_hint(sA, &p.mapB16, bar, kx, 0, 0, (t.n0 + 64 * (int)rank) / 16, t.e, evict_first);
+              else
+                tma2_load_5d(sA, &p.mapB16, bar, kx, 0, 0, (t.n0 + 64 * (int)rank) / 16, t.e);
             } else {
-              tma2_load_3d(sA, mB, bar, kx, t.n0 + 128 * (int)rank, t.e);
+              if (t.mtiles == 1) tma2_load_3d_hint(sA, mB, bar, kx, t.n0 + 128 * (int)rank, t.e, evict_first);
+              else tma2_load_3d(sA, mB, bar, kx, t.n0 + 128 * (int)rank, t.e);
             }
             tma2_load_2d(sB, nh <= 32 ? &p.mapA32 : &p.mapA64, bar, kx, t.row0 + (int)rank * nh);
           } else {
