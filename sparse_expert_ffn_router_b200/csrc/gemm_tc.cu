@@ -611,7 +611,13 @@ struct SmemMisc2 {
   int32_t lt[kMaxExperts + 1];
 };
 
-constexpr size_t SMEM2_BYTES = (size_t)STAGES2 * STAGE2_BYTES + sizeof(SmemMisc2);
+// Light tails of at most 32 rows ("dense" light tiles) put the weights of two K blocks in a stage
+// (A and B slots) and their 16-row token boxes in a ring of their own, so that the stream of
+// weights has twice the bytes in flight
+constexpr int kDenseLightRows = 32;
+constexpr int TOK_BYTES = 16 * BK * 2;  // one 16-row token box
+constexpr size_t TOK2_RING = (size_t)STAGES2 * 2 * TOK_BYTES;
+constexpr size_t SMEM2_BYTES = (size_t)STAGES2 * STAGE2_BYTES + TOK2_RING + sizeof(SmemMisc2);
 static_assert(SMEM2_BYTES <= 232448, "pair-tile stages exceed the shared memory of one CTA");
 
 template <bool kGateUp>
@@ -629,7 +635,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
   }
   uint8_t* smem = smem_raw;
   uint8_t* stage_base = smem;
-  SmemMisc2& m = *reinterpret_cast<SmemMisc2*>(smem + (size_t)STAGES2 * STAGE2_BYTES);
+  uint8_t* tok_base = smem + (size_t)STAGES2 * STAGE2_BYTES;  // [STAGES2][2] token boxes (dense light tiles)
+  SmemMisc2& m = *reinterpret_cast<SmemMisc2*>(smem + (size_t)STAGES2 * STAGE2_BYTES + TOK2_RING);
   volatile int* abort_flag = &m.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -654,6 +661,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
     tma_prefetch_desc(&p.mapA);
     tma_prefetch_desc(&p.mapB);
     tma_prefetch_desc(&p.mapA32);
+    tma_prefetch_desc(&p.mapA16);
     tma_prefetch_desc(&p.mapA64);
     if (kGateUp) tma_prefetch_desc(&p.mapB16);
     if (p.mt_sh > 0) {
@@ -721,12 +729,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
         const CUtensorMap* mB = t.sh ? &p.mapB_sh : &p.mapB;
         const int arow = t.row0 + 128 * (int)rank;
         const bool light = !t.sh && t.row_end - t.row0 <= p.pair_light_rows;
+        const bool dense = light && t.row_end - t.row0 <= kDenseLightRows;
         const int nh = (t.row_end - t.row0 + 15) / 16 * 8;  // light: token rows (N / 2) per CTA
-        const int claim_kb = t.num_kb > STAGES2 ? t.num_kb - STAGES2 : 0;
+        const int nsteps = dense ? (t.num_kb + 1) / 2 : t.num_kb;  // ring stages of the tile
+        const int claim_step = nsteps > STAGES2 ? nsteps - STAGES2 : 0;
         int next = L;
         bool ok = true;
-        for (int kb = 0; kb < t.num_kb; ++kb) {
-          if (rank == 0 && kb == claim_kb) next = claim_next(p.sched, L, npairs);
+        for (int step = 0; step < nsteps; ++step) {
+          if (rank == 0 && step == claim_step) next = claim_next(p.sched, L, npairs);
           if (!wait_or_abort(&m.empty[s], ph ^ 1u, abort_flag)) {
             ok = false;
             break;
@@ -734,8 +744,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
           uint8_t* sA = stage_base + (size_t)s * STAGE2_BYTES;
           uint8_t* sB = sA + HALF_BYTES;
           const uint32_t bar = mapa_shared(smem_u32(&m.full[s]), 0);
+          const int kb = dense ? 2 * step : step;
           const int kx = kb * BK;
-          if (light) {
+          if (dense) {
+            // two K blocks of weights (A and B slots), their token boxes in the token ring
+            const int nk = min(2, t.num_kb - kb);
+            if (rank == 0) mbar_arrive_expect_tx(&m.full[s], (uint32_t)(2 * nk * (HALF_BYTES + TOK_BYTES)));
+            for (int j = 0; j < nk; ++j) {
+              uint8_t* wdst = sA + (size_t)j * HALF_BYTES;
+              const int kxj = kx + j * BK;
+              if (kGateUp) {
+                if (t.mtiles == 1)
+                  tma2_load_5d_hint(wdst, &p.mapB16, bar, kxj, 0, 0, (t.n0 + 64 * (int)rank) / 16, t.e, evict_first);
+                else
+                  tma2_load_5d(wdst, &p.mapB16, bar, kxj, 0, 0, (t.n0 + 64 * (int)rank) / 16, t.e);
+              } else {
+                if (t.mtiles == 1) tma2_load_3d_hint(wdst, mB, bar, kxj, t.n0 + 128 * (int)rank, t.e, evict_first);
+                else tma2_load_3d(wdst, mB, bar, kxj, t.n0 + 128 * (int)rank, t.e);
+              }
+              tma2_load_2d(tok_base + (size_t)(2 * s + j) * TOK_BYTES, &p.mapA16, bar, kxj, t.row0 + (int)rank * nh);
+            }
+          } else if (light) {
             // swapped tail: weights into the A slot, the tile's token rows into the B slot
             const int box_rows = nh <= 32 ? 32 : 64;
             if (rank == 0) mbar_arrive_expect_tx(&m.full[s], 2 * (HALF_BYTES + box_rows * BK * 2));
@@ -807,8 +836,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
         const uint32_t d_tmem = tmem_base + (uint32_t)(a * BN);
         const int trows = t.row_end - t.row0;
         // light tail: M = 256 weight rows, N = the tile's rows rounded up to 16
-        const uint32_t idesc = (!t.sh && trows <= p.pair_light_rows) ? idesc_bf16_f32(BM2, (trows + 15) / 16 * 16) : IDESC2;
-        for (int kb = 0; kb < t.num_kb; ++kb) {
+        const bool light = !t.sh && trows <= p.pair_light_rows;
+        const bool dense = light && trows <= kDenseLightRows;
+        const uint32_t idesc = light ? idesc_bf16_f32(BM2, (trows + 15) / 16 * 16) : IDESC2;
+        const int nsteps = dense ? (t.num_kb + 1) / 2 : t.num_kb;
+        for (int step = 0; step < nsteps; ++step) {
           if (!wait_or_abort(&m.full[s], ph, abort_flag)) {
             ok = false;
             break;
@@ -816,11 +848,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) tc2_ffn_kernel(const __grid_co
           tc_fence_after();
           const uint32_t sA = smem_u32(stage_base + (size_t)s * STAGE2_BYTES);
           const uint32_t sB = sA + HALF_BYTES;
+          if (dense) {
+            const int nk = min(2, t.num_kb - 2 * step);
+            for (int j = 0; j < nk; ++j) {
+              const uint32_t wa = sA + (uint32_t)(j * HALF_BYTES);
+              const uint32_t tb = smem_u32(tok_base + (size_t)(2 * s + j) * TOK_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(sA + kk * 32);
-            const uint64_t bd = smem_desc_sw128(sB + kk * 32);
-            tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+              for (int kk = 0; kk < BK / 16; ++kk)
+                tc_mma_f16_pair(d_tmem, smem_desc_sw128(wa + kk * 32), smem_desc_sw128(tb + kk * 32), idesc,
+                                (step | j | kk) != 0 ? 1u : 0u);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t ad = smem_desc_sw128(sA + kk * 32);
+              const uint64_t bd = smem_desc_sw128(sB + kk * 32);
+              tc_mma_f16_pair(d_tmem, ad, bd, idesc, (step | kk) != 0 ? 1u : 0u);
+            }
           }
           tc_commit_pair_mc(&m.empty[s], 0x3);
           if (++s == STAGES2) {
