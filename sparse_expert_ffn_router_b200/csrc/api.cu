@@ -307,6 +307,7 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   cudaError_t ce = configure_router_kernels();
   if (ce == cudaSuccess) ce = configure_tc_kernels();
   if (ce == cudaSuccess) ce = configure_dec_kernels();
+  if (ce == cudaSuccess) ce = configure_simt_kernels();
   if (ce != cudaSuccess) {
     cudaGetLastError();
     cudaFree(ctx->ws_base);

@@ -38,9 +38,8 @@ constexpr int kTcPairStages = COLIBRI_TC2_STAGES;  // 32 KB stages, pair tiles
 constexpr int kTcPairBM = 256;  // rows of a pair tile (two CTAs, cta_group::2)
 
 // SIMT fp32 grouped GEMM tile
-constexpr int kSimtBM = 64;
+constexpr int kSimtBM = 32;
 constexpr int kSimtBN = 64;
-constexpr int kSimtBK = 16;
 
 // int8 weight-streaming decode path
 constexpr int kDecSplitMax = 16;     // K splits of the down projection
@@ -282,6 +281,7 @@ cudaError_t launch_tc_down(const TcGemmArgs& a, cudaStream_t s);
 // int8 weight-streaming decode path, see decode_i8.cu (the x planes come from the scatter)
 // max_rows_per_expert: an upper bound (T) that picks the token chunk (8, 16 or 32 rows).
 cudaError_t configure_dec_kernels();  // once per device, before any launch
+cudaError_t configure_simt_kernels();  // once per device, before any launch
 // gate/up: W1 . x and W3 . x (scaled) as fp32 K-split partials GU [nsplit, 2, R, f]
 // scale_mode: COLIBRI_SCALE_PER_CHANNEL (scales per expert [f | f | d]) or
 // COLIBRI_SCALE_PER_MATRIX (scales [E][3]: W1, W3, W2)

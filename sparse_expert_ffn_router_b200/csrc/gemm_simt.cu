@@ -6,15 +6,35 @@
 //   gate/up:  H[r][n] = silu(sum_i A[r][i] W1_e[n][i]) * (sum_i A[r][i] W3_e[n][i])
 //   down:     Y[r][n] = sum_i H[r][i] W2_e[n][i]
 //
-// 64 x 64 output tiles, K staged 16 at a time through shared memory, 4 x 4 register tile per
-// thread.  Tiles are laid out on a (n-tile, m-tile) grid; m-tiles map to (expert, rows) through
-// the device-side m-tile prefix, so no host synchronisation is needed.
+// 32 x 64 output tiles (an expert of a small layer has few rows: a 64-row tile spent most of its
+// multiply-adds on padding).  K advances 32 at a time through a 4-stage shared-memory ring filled by
+// cp.async (16-byte copies, rows past a group's end or past N zero-filled), so three K slices are
+// in flight while one is multiplied: the tiles of a small layer are bound by the memory round
+// trip, which a load-then-compute loop paid once per slice.  Thread (ty, tx) of 16 x 16 owns the
+// outputs (ty + 16 i, tx + 16 j), i < 2, j < 4, each accumulated with one fmaf per K in ascending K
+// order.  Tiles are laid out on a (n-tile, m-tile) grid; m-tiles map to (expert, rows) through the
+// device-side m-tile prefix, so no host synchronisation is needed.
 #include "common.cuh"
 
 namespace colibri {
 namespace {
 
-constexpr int BM = kSimtBM, BN = kSimtBN, BK = kSimtBK;
+constexpr int BM = kSimtBM, BN = kSimtBN;
+constexpr int MI = BM / 16;  // rows per thread
+static_assert(BM % 16 == 0 && BN == 64, "16 x 16 threads: BM / 16 rows x 4 columns each");
+constexpr int SK = 32;       // K per stage (d_model and d_ff are multiples of 64)
+constexpr int SS = 4;        // stages
+constexpr int SP = SK + 4;   // floats per staged row: 16-byte aligned rows, and the 8 lanes of one
+                             // 128-bit shared load hit distinct banks
+constexpr size_t simt_smem_bytes(bool gateup) { return (size_t)SS * (BM + BN + (gateup ? BN : 0)) * SP * 4; }
+
+__device__ __forceinline__ void cp_async16(float* dst, const float* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __device__ __forceinline__ bool simt_tile_rows(const SimtGroups& g, int mt, int& grp, int& row0,
                                                int& row_end) {
@@ -45,9 +65,10 @@ __global__ void __launch_bounds__(256) simt_ffn_kernel(const float* __restrict__
                                                        float* __restrict__ out, int ldo, int N) {
   pdl_trigger();
   pdl_wait();
-  __shared__ __align__(16) float As[BK][BM + 4];
-  __shared__ __align__(16) float Bs[BK][BN + 4];
-  __shared__ __align__(16) float Cs[kGateUp ? BK : 1][BN + 4];
+  extern __shared__ __align__(16) float sm[];
+  float (*As)[BM][SP] = reinterpret_cast<float (*)[BM][SP]>(sm);                      // [SS][BM][SP]
+  float (*Bs)[BN][SP] = reinterpret_cast<float (*)[BN][SP]>(sm + SS * BM * SP);        // [SS][BN][SP]
+  float (*Cs)[BN][SP] = reinterpret_cast<float (*)[BN][SP]>(sm + SS * (BM + BN) * SP);  // gate/up: W3
   int grp, row0, row_end;
   if (!simt_tile_rows(groups, blockIdx.y, grp, row0, row_end)) return;
   const int n0 = blockIdx.x * BN;
@@ -56,53 +77,74 @@ __global__ void __launch_bounds__(256) simt_ffn_kernel(const float* __restrict__
   const float* B1 = kGateUp ? base : base + 2 * (int64_t)f * d;
   const float* B3 = base + (int64_t)f * d;
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-  const int lr = tid >> 2, lk = (tid & 3) * 4;
-  float acc1[4][4] = {}, acc3[4][4] = {};
-  for (int k0 = 0; k0 < K; k0 += BK) {
-    {
-      const int r = row0 + lr;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r < row_end) v = *reinterpret_cast<const float4*>(A + (size_t)r * lda + k0 + lk);
-      As[lk + 0][lr] = v.x; As[lk + 1][lr] = v.y; As[lk + 2][lr] = v.z; As[lk + 3][lr] = v.w;
-      const int n = n0 + lr;
-      float4 b = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (n < N) b = *reinterpret_cast<const float4*>(B1 + (size_t)n * K + k0 + lk);
-      Bs[lk + 0][lr] = b.x; Bs[lk + 1][lr] = b.y; Bs[lk + 2][lr] = b.z; Bs[lk + 3][lr] = b.w;
-      if (kGateUp) {
-        float4 c = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (n < N) c = *reinterpret_cast<const float4*>(B3 + (size_t)n * K + k0 + lk);
-        Cs[lk + 0][lr] = c.x; Cs[lk + 1][lr] = c.y; Cs[lk + 2][lr] = c.z; Cs[lk + 3][lr] = c.w;
-      }
+  const int nk = K / SK;
+  // copies of K slice kt into ring slot `slot`: 64 rows x 8 chunks of 16 bytes per operand
+  auto issue = [&](int kt, int slot) {
+    const int k0 = kt * SK;
+#pragma unroll
+    for (int q = tid; q < BM * (SK / 4); q += 256) {
+      const int rr = q >> 3, c4 = (q & 7) * 4;
+      const int r = row0 + rr;
+      const bool vr = r < row_end;
+      cp_async16(&As[slot][rr][c4], A + (size_t)(vr ? r : row0) * lda + k0 + c4, vr);
     }
-    __syncthreads();
 #pragma unroll
-    for (int kk = 0; kk < BK; ++kk) {
-      const float4 a = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
-      const float4 b = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
-      const float av[4] = {a.x, a.y, a.z, a.w};
-      const float bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc1[i][j] = fmaf(av[i], bv[j], acc1[i][j]);
-      if (kGateUp) {
-        const float4 c = *reinterpret_cast<const float4*>(&Cs[kk][tx * 4]);
-        const float cv[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) acc3[i][j] = fmaf(av[i], cv[j], acc3[i][j]);
-      }
+    for (int q = tid; q < BN * (SK / 4); q += 256) {
+      const int rr = q >> 3, c4 = (q & 7) * 4;
+      const int n = n0 + rr;
+      const bool vn = n < N;
+      cp_async16(&Bs[slot][rr][c4], B1 + (size_t)(vn ? n : n0) * K + k0 + c4, vn);
+      if (kGateUp) cp_async16(&Cs[slot][rr][c4], B3 + (size_t)(vn ? n : n0) * K + k0 + c4, vn);
     }
-    __syncthreads();
+  };
+#pragma unroll
+  for (int st = 0; st < SS - 1; ++st) {
+    if (st < nk) issue(st, st);
+    cp_async_commit();
   }
+  float acc1[MI][4] = {}, acc3[MI][4] = {};
+  for (int kt = 0; kt < nk; ++kt) {
+    cp_async_wait<SS - 2>();  // this thread's copies of slice kt have landed
+    __syncthreads();          // everyone's have, and every thread is done with slice kt - 1
+    if (kt + SS - 1 < nk) issue(kt + SS - 1, (kt + SS - 1) % SS);
+    cp_async_commit();
+    const int slot = kt % SS;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = row0 + ty * 4 + i;
+    for (int k4 = 0; k4 < SK; k4 += 4) {
+      float4 a[MI], b[4], c[4];
+#pragma unroll
+      for (int i = 0; i < MI; ++i) a[i] = *reinterpret_cast<const float4*>(&As[slot][ty + 16 * i][k4]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        b[j] = *reinterpret_cast<const float4*>(&Bs[slot][tx + 16 * j][k4]);
+        if (kGateUp) c[j] = *reinterpret_cast<const float4*>(&Cs[slot][tx + 16 * j][k4]);
+      }
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+        for (int i = 0; i < MI; ++i) {
+          const float av = kk == 0 ? a[i].x : kk == 1 ? a[i].y : kk == 2 ? a[i].z : a[i].w;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float bv = kk == 0 ? b[j].x : kk == 1 ? b[j].y : kk == 2 ? b[j].z : b[j].w;
+            acc1[i][j] = fmaf(av, bv, acc1[i][j]);
+            if (kGateUp) {
+              const float cv = kk == 0 ? c[j].x : kk == 1 ? c[j].y : kk == 2 ? c[j].z : c[j].w;
+              acc3[i][j] = fmaf(av, cv, acc3[i][j]);
+            }
+          }
+        }
+      }
+    }
+  }
+  cp_async_wait<0>();
+#pragma unroll
+  for (int i = 0; i < MI; ++i) {
+    const int r = row0 + ty + 16 * i;
     if (r >= row_end) continue;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int n = n0 + tx * 4 + j;
+      const int n = n0 + tx + 16 * j;
       if (n >= N) continue;
       float v = acc1[i][j];
       if (kGateUp) v = v / (1.0f + expf(-v)) * acc3[i][j];
@@ -117,14 +159,26 @@ cudaError_t launch_simt_gateup(const float* A, int lda, const float* W, int64_t 
                                int f, SimtGroups g, int mt_bound, float* H, cudaStream_t s) {
   if (mt_bound <= 0) return cudaSuccess;
   const dim3 grid((f + BN - 1) / BN, mt_bound);
-  return launch_kernel(simt_ffn_kernel<true>, grid, dim3(256), 0, s, 1, A, lda, d, W, wstride, d, f, g, H, f, f);
+  return launch_kernel(simt_ffn_kernel<true>, grid, dim3(256), simt_smem_bytes(true), s, 1, A, lda, d, W, wstride, d,
+                       f, g, H, f, f);
 }
 
 cudaError_t launch_simt_down(const float* H, int f, const float* W, int64_t wstride, int d,
                              SimtGroups g, int mt_bound, float* Y, cudaStream_t s) {
   if (mt_bound <= 0) return cudaSuccess;
   const dim3 grid((d + BN - 1) / BN, mt_bound);
-  return launch_kernel(simt_ffn_kernel<false>, grid, dim3(256), 0, s, 1, H, f, f, W, wstride, d, f, g, Y, d, d);
+  return launch_kernel(simt_ffn_kernel<false>, grid, dim3(256), simt_smem_bytes(false), s, 1, H, f, f, W, wstride, d,
+                       f, g, Y, d, d);
+}
+
+// Done once per device at context creation (nothing in the launch path is a non-stream call).
+cudaError_t configure_simt_kernels() {
+  cudaError_t e = cudaFuncSetAttribute(simt_ffn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)simt_smem_bytes(true));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(simt_ffn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)simt_smem_bytes(false));
+  return e;
 }
 
 }  // namespace colibri
