@@ -39,7 +39,7 @@ constexpr int kTcPairBM = 256;  // rows of a pair tile (two CTAs, cta_group::2)
 
 // SIMT fp32 grouped GEMM tile
 constexpr int kSimtBM = 32;
-constexpr int kSimtBN = 64;
+constexpr int kSimtBN = 32;
 
 // int8 weight-streaming decode path
 constexpr int kDecSplitMax = 16;     // K splits of the down projection

@@ -6,12 +6,13 @@
 //   gate/up:  H[r][n] = silu(sum_i A[r][i] W1_e[n][i]) * (sum_i A[r][i] W3_e[n][i])
 //   down:     Y[r][n] = sum_i H[r][i] W2_e[n][i]
 //
-// 32 x 64 output tiles (an expert of a small layer has few rows: a 64-row tile spent most of its
-// multiply-adds on padding).  K advances 32 at a time through a 4-stage shared-memory ring filled by
+// 32 x 32 output tiles: an expert of a small layer has few rows (a 64-row tile spent most of its
+// multiply-adds on padding), and narrow tiles give such a layer enough CTAs to keep the memory
+// system busy.  K advances 32 at a time through a 4-stage shared-memory ring filled by
 // cp.async (16-byte copies, rows past a group's end or past N zero-filled), so three K slices are
 // in flight while one is multiplied: the tiles of a small layer are bound by the memory round
 // trip, which a load-then-compute loop paid once per slice.  Thread (ty, tx) of 16 x 16 owns the
-// outputs (ty + 16 i, tx + 16 j), i < 2, j < 4, each accumulated with one fmaf per K in ascending K
+// outputs (ty + 16 i, tx + 16 j), i, j < 2, each accumulated with one fmaf per K in ascending K
 // order.  Tiles are laid out on a (n-tile, m-tile) grid; m-tiles map to (expert, rows) through the
 // device-side m-tile prefix, so no host synchronisation is needed.
 #include "common.cuh"
@@ -21,7 +22,8 @@ namespace {
 
 constexpr int BM = kSimtBM, BN = kSimtBN;
 constexpr int MI = BM / 16;  // rows per thread
-static_assert(BM % 16 == 0 && BN == 64, "16 x 16 threads: BM / 16 rows x 4 columns each");
+constexpr int NJ = BN / 16;  // columns per thread
+static_assert(BM % 16 == 0 && BN % 16 == 0, "16 x 16 threads: BM / 16 rows x BN / 16 columns each");
 constexpr int SK = 32;       // K per stage (d_model and d_ff are multiples of 64)
 constexpr int SS = 4;        // stages
 constexpr int SP = SK + 4;   // floats per staged row: 16-byte aligned rows, and the 8 lanes of one
@@ -102,7 +104,7 @@ __global__ void __launch_bounds__(256) simt_ffn_kernel(const float* __restrict__
     if (st < nk) issue(st, st);
     cp_async_commit();
   }
-  float acc1[MI][4] = {}, acc3[MI][4] = {};
+  float acc1[MI][NJ] = {}, acc3[MI][NJ] = {};
   for (int kt = 0; kt < nk; ++kt) {
     cp_async_wait<SS - 2>();  // this thread's copies of slice kt have landed
     __syncthreads();          // everyone's have, and every thread is done with slice kt - 1
@@ -111,11 +113,11 @@ __global__ void __launch_bounds__(256) simt_ffn_kernel(const float* __restrict__
     const int slot = kt % SS;
 #pragma unroll
     for (int k4 = 0; k4 < SK; k4 += 4) {
-      float4 a[MI], b[4], c[4];
+      float4 a[MI], b[NJ], c[NJ];
 #pragma unroll
       for (int i = 0; i < MI; ++i) a[i] = *reinterpret_cast<const float4*>(&As[slot][ty + 16 * i][k4]);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < NJ; ++j) {
         b[j] = *reinterpret_cast<const float4*>(&Bs[slot][tx + 16 * j][k4]);
         if (kGateUp) c[j] = *reinterpret_cast<const float4*>(&Cs[slot][tx + 16 * j][k4]);
       }
@@ -125,7 +127,7 @@ __global__ void __launch_bounds__(256) simt_ffn_kernel(const float* __restrict__
         for (int i = 0; i < MI; ++i) {
           const float av = kk == 0 ? a[i].x : kk == 1 ? a[i].y : kk == 2 ? a[i].z : a[i].w;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
+          for (int j = 0; j < NJ; ++j) {
             const float bv = kk == 0 ? b[j].x : kk == 1 ? b[j].y : kk == 2 ? b[j].z : b[j].w;
             acc1[i][j] = fmaf(av, bv, acc1[i][j]);
             if (kGateUp) {
@@ -143,7 +145,7 @@ __global__ void __launch_bounds__(256) simt_ffn_kernel(const float* __restrict__
     const int r = row0 + ty + 16 * i;
     if (r >= row_end) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < NJ; ++j) {
       const int n = n0 + tx + 16 * j;
       if (n >= N) continue;
       float v = acc1[i][j];
