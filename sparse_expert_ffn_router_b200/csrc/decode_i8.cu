@@ -762,8 +762,9 @@ __device__ bool d4_mma(const DecStreamParams& p, uint8_t* slots, uint8_t* ring, 
 // registers (one per token of the chunk); per item the sums times the plane scale are written.
 // K blocks are taken two at a time (both accumulators waited for, read, then released), so the
 // fixed latencies of the wait and the TMEM load are paid once per pair.
-__device__ __forceinline__ void d4_accumulate(float (&acc)[32], int nt8, uint32_t tb, float s) {
-  // columns [0, nt8) of the accumulator hold the hi plane, [nt8, 2 nt8) the lo plane
+__device__ __forceinline__ void d4_accumulate(float (&acc)[32], int nt8, int ntok, uint32_t tb, float s) {
+  // columns [0, nt8) of the accumulator hold the hi plane, [nt8, 2 nt8) the lo plane; only the
+  // 16-column groups that hold one of the item's ntok tokens are read
   if (nt8 == 8) {
     float v[16];
     tmem_ld16(tb, v);
@@ -774,7 +775,7 @@ __device__ __forceinline__ void d4_accumulate(float (&acc)[32], int nt8, uint32_
   } else {
 #pragma unroll
     for (int j = 0; j < 32; j += 16) {
-      if (j >= nt8) break;
+      if (j >= nt8 || j >= ntok) break;
       float vh[16], vl[16];
       tmem_ld16(tb + j, vh);
       tmem_ld16(tb + nt8 + j, vl);
@@ -826,8 +827,8 @@ __device__ bool d4_epilogue(const DecStreamParams& p, D4Ctl& c, uint32_t tmem, i
         sc[u] = group_scale(i + 8);
         sc[u + 1] = group_scale(i + 9);
         const uint32_t lanes = (uint32_t)(q * 32) << 16;
-        d4_accumulate(acc, p.nt8, tmem + lanes + b0 * (uint32_t)N, s0);
-        if (two) d4_accumulate(acc, p.nt8, tmem + lanes + b1 * (uint32_t)N, s1);
+        d4_accumulate(acc, p.nt8, it.ntok, tmem + lanes + b0 * (uint32_t)N, s0);
+        if (two) d4_accumulate(acc, p.nt8, it.ntok, tmem + lanes + b1 * (uint32_t)N, s1);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
