@@ -6,13 +6,13 @@
 //   gate/up:  H[r][n] = silu(sum_i A[r][i] W1_e[n][i]) * (sum_i A[r][i] W3_e[n][i])
 //   down:     Y[r][n] = sum_i H[r][i] W2_e[n][i]
 //
-// 32 x 32 output tiles: an expert of a small layer has few rows (a 64-row tile spent most of its
-// multiply-adds on padding), and narrow tiles give such a layer enough CTAs to keep the memory
-// system busy.  K advances 32 at a time through a 4-stage shared-memory ring filled by
+// 32 x 32 output tiles (down: 32 x 16): an expert of a small layer has few rows (a 64-row tile
+// spent most of its multiply-adds on padding), and narrow tiles give such a layer enough CTAs to
+// keep the memory system busy.  K advances 32 at a time through a 4-stage shared-memory ring filled by
 // cp.async (16-byte copies, rows past a group's end or past N zero-filled), so three K slices are
 // in flight while one is multiplied: the tiles of a small layer are bound by the memory round
 // trip, which a load-then-compute loop paid once per slice.  Thread (ty, tx) of 16 x 16 owns the
-// outputs (ty + 16 i, tx + 16 j), i, j < 2, each accumulated with one fmaf per K in ascending K
+// outputs (ty + 16 i, tx + 16 j), i < 2, j < 2 (down: j < 1), each accumulated with one fmaf per K in ascending K
 // order.  Tiles are laid out on a (n-tile, m-tile) grid; m-tiles map to (expert, rows) through the
 // device-side m-tile prefix, so no host synchronisation is needed.
 #include "common.cuh"
@@ -20,15 +20,19 @@
 namespace colibri {
 namespace {
 
-constexpr int BM = kSimtBM, BN = kSimtBN;
+constexpr int BM = kSimtBM;
 constexpr int MI = BM / 16;  // rows per thread
-constexpr int NJ = BN / 16;  // columns per thread
-static_assert(BM % 16 == 0 && BN % 16 == 0, "16 x 16 threads: BM / 16 rows x BN / 16 columns each");
+static_assert(BM % 16 == 0, "16 x 16 threads: BM / 16 rows each");
+// Tile width: gate/up 32 columns; down 16 (its N = d_model is the smaller side of a small layer, and
+// narrower tiles give it as many CTAs as gate/up has)
+template <bool kGateUp>
+constexpr int simt_bn() { return kGateUp ? kSimtBN : kSimtBN / 2; }
 constexpr int SK = 32;       // K per stage (d_model and d_ff are multiples of 64)
 constexpr int SS = 4;        // stages
 constexpr int SP = SK + 4;   // floats per staged row: 16-byte aligned rows, and the 8 lanes of one
                              // 128-bit shared load hit distinct banks
-constexpr size_t simt_smem_bytes(bool gateup) { return (size_t)SS * (BM + BN + (gateup ? BN : 0)) * SP * 4; }
+template <bool kGateUp>
+constexpr size_t simt_smem_bytes() { return (size_t)SS * (BM + simt_bn<kGateUp>() * (kGateUp ? 2 : 1)) * SP * 4; }
 
 __device__ __forceinline__ void cp_async16(float* dst, const float* src, bool valid) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 16 : 0)
@@ -65,6 +69,9 @@ __global__ void __launch_bounds__(256) simt_ffn_kernel(const float* __restrict__
                                                        int64_t wstride, int d, int f,
                                                        SimtGroups groups,
                                                        float* __restrict__ out, int ldo, int N) {
+  constexpr int BN = simt_bn<kGateUp>();
+  constexpr int NJ = BN / 16;  // columns per thread
+  static_assert(BN % 16 == 0, "16 x 16 threads: BN / 16 columns each");
   pdl_trigger();
   pdl_wait();
   extern __shared__ __align__(16) float sm[];
@@ -160,26 +167,28 @@ __global__ void __launch_bounds__(256) simt_ffn_kernel(const float* __restrict__
 cudaError_t launch_simt_gateup(const float* A, int lda, const float* W, int64_t wstride, int d,
                                int f, SimtGroups g, int mt_bound, float* H, cudaStream_t s) {
   if (mt_bound <= 0) return cudaSuccess;
+  constexpr int BN = simt_bn<true>();
   const dim3 grid((f + BN - 1) / BN, mt_bound);
-  return launch_kernel(simt_ffn_kernel<true>, grid, dim3(256), simt_smem_bytes(true), s, 1, A, lda, d, W, wstride, d,
+  return launch_kernel(simt_ffn_kernel<true>, grid, dim3(256), simt_smem_bytes<true>(), s, 1, A, lda, d, W, wstride, d,
                        f, g, H, f, f);
 }
 
 cudaError_t launch_simt_down(const float* H, int f, const float* W, int64_t wstride, int d,
                              SimtGroups g, int mt_bound, float* Y, cudaStream_t s) {
   if (mt_bound <= 0) return cudaSuccess;
+  constexpr int BN = simt_bn<false>();
   const dim3 grid((d + BN - 1) / BN, mt_bound);
-  return launch_kernel(simt_ffn_kernel<false>, grid, dim3(256), simt_smem_bytes(false), s, 1, H, f, f, W, wstride, d,
+  return launch_kernel(simt_ffn_kernel<false>, grid, dim3(256), simt_smem_bytes<false>(), s, 1, H, f, f, W, wstride, d,
                        f, g, Y, d, d);
 }
 
 // Done once per device at context creation (nothing in the launch path is a non-stream call).
 cudaError_t configure_simt_kernels() {
   cudaError_t e = cudaFuncSetAttribute(simt_ffn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)simt_smem_bytes(true));
+                                       (int)simt_smem_bytes<true>());
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(simt_ffn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)simt_smem_bytes(false));
+                             (int)simt_smem_bytes<false>());
   return e;
 }
 
