@@ -232,11 +232,6 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   const size_t o_err = c.take(4);
   const size_t o_tsched = c.take(4 * 4);
   const size_t o_gbar = c.take(i8 ? kFusedBarCount * 4 : 0);
-  const size_t flow_bytes = (size_t)(kFlowUnitCtrs + kFlowTileCtrs) * 4;
-  const size_t o_flow = c.take(i8 ? flow_bytes : 0);
-  const int64_t flow_rows = std::min<int64_t>(M, kFlowMaxT) * D.top_k;
-  const size_t o_fhh = c.take(i8 ? flow_rows * f : 0), o_fhl = c.take(i8 ? flow_rows * f : 0);
-  const size_t o_fhs = c.take(i8 ? (size_t)kDecSplitMax * flow_rows * 4 : 0);
   ctx->ws_bytes = c.off;
 
   DeviceGuard guard(D.device_id);
@@ -271,14 +266,8 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   w.err = reinterpret_cast<uint32_t*>(b + o_err);
   w.tile_sched = reinterpret_cast<uint32_t*>(b + o_tsched);
   w.grid_bar = i8 ? reinterpret_cast<int32_t*>(b + o_gbar) : nullptr;
-  w.flow_ctr = i8 ? reinterpret_cast<int32_t*>(b + o_flow) : nullptr;
-  w.flow_hhi = i8 ? reinterpret_cast<int8_t*>(b + o_fhh) : nullptr;
-  w.flow_hlo = i8 ? reinterpret_cast<int8_t*>(b + o_fhl) : nullptr;
-  w.flow_hscale = i8 ? reinterpret_cast<float*>(b + o_fhs) : nullptr;
-  w.flow_rows = i8 ? (int)flow_rows : 0;
   if (cudaMemset(w.err, 0, 4) != cudaSuccess || cudaMemset(w.tile_sched, 0, 4 * 4) != cudaSuccess ||
-      (i8 && cudaMemset(w.grid_bar, 0, kFusedBarCount * 4) != cudaSuccess) ||
-      (i8 && cudaMemset(w.flow_ctr, 0, flow_bytes) != cudaSuccess)) {
+      (i8 && cudaMemset(w.grid_bar, 0, kFusedBarCount * 4) != cudaSuccess)) {
     cudaFree(ctx->ws_base);
     delete ctx;
     return fail(nullptr, COLIBRI_ERR_CUDA, "cudaMemset failed");
@@ -302,8 +291,6 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   ctx->use_pdl = env_flag("COLIBRI_PDL");
   ctx->dec_fused = !(getenv("COLIBRI_DEC_FUSED") && strcmp(getenv("COLIBRI_DEC_FUSED"), "0") == 0);
   ctx->dec_route = !(getenv("COLIBRI_DEC_ROUTE") && strcmp(getenv("COLIBRI_DEC_ROUTE"), "0") == 0);
-  // the dataflow plan of the fused int8 launch is opt-in (COLIBRI_DEC_FLOW=1) until it measures faster
-  ctx->dec_flow = env_flag("COLIBRI_DEC_FLOW");
   cudaError_t ce = configure_router_kernels();
   if (ce == cudaSuccess) ce = configure_tc_kernels();
   if (ce == cudaSuccess) ce = configure_dec_kernels();
@@ -536,13 +523,6 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
       fa.y = (__nv_bfloat16*)yd;
       fa.bar = w.grid_bar;
       fa.err = w.err;
-      fa.flow = ctx->dec_flow;
-      fa.unit_ctr = w.flow_ctr;
-      fa.tile_ctr = w.flow_ctr + kFlowUnitCtrs;
-      fa.hplanes_hi = w.flow_hhi;
-      fa.hplanes_lo = w.flow_hlo;
-      fa.hplanes_scale = w.flow_hscale;
-      fa.flow_rows = w.flow_rows;
       if (route_in_dec) {
         fa.route_in_kernel = routed_by_caller ? 2 : 1;
         fa.x = (const __nv_bfloat16*)xd;
@@ -809,9 +789,6 @@ colibri_status colibri_sync_status(colibri_ctx* ctx, void* stream) {
     // a wait that gave up may leave the fused kernel's grid-barrier counters out of step
     if (ctx->ws.grid_bar)
       COLIBRI_TRY(cudaMemset(ctx->ws.grid_bar, 0, kFusedBarCount * 4), "reset grid-barrier counters");
-    if (ctx->ws.flow_ctr)
-      COLIBRI_TRY(cudaMemset(ctx->ws.flow_ctr, 0, (size_t)(kFlowUnitCtrs + kFlowTileCtrs) * 4),
-                  "reset completion counters");
     COLIBRI_TRY(cudaMemset(ctx->ws.tile_sched, 0, 4 * 4), "reset tile counters");
     return fail(ctx, COLIBRI_ERR_TIMEOUT, "device error word 0x%x (a bounded wait gave up)", err);
   }

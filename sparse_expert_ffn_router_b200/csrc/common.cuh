@@ -75,11 +75,6 @@ struct Workspace {
   void* Ys = nullptr;   // [M, d]
   float* Ypart = nullptr;  // [split, M*k, d] f32, int8 path
   int32_t* grid_bar = nullptr;       // [4] grid-barrier counters of the fused int8 kernel (zero between calls)
-  int32_t* flow_ctr = nullptr;       // [kFlowUnitCtrs + kFlowTileCtrs] dataflow int8 kernel (zero between calls)
-  int8_t* flow_hhi = nullptr;        // [flow_rows, f] H planes of the dataflow int8 kernel
-  int8_t* flow_hlo = nullptr;
-  float* flow_hscale = nullptr;      // [kDecSplitMax, flow_rows]
-  int flow_rows = 0;                 // min(max_tokens, kFlowMaxT) * k
   int8_t* plane_hi = nullptr;  // [M*k, max(d, f)] int8 activation planes, int8 path
   int8_t* plane_lo = nullptr;
   float* plane_scale = nullptr;  // [M*k]
@@ -126,7 +121,6 @@ struct colibri_ctx {
   bool use_pdl = false;  // programmatic dependent launch between the kernels of a forward (opt-in)
   bool dec_fused = true;  // int8 weights: the one-launch expert stage (COLIBRI_DEC_FUSED=0: four launches)
   bool dec_route = true;  // int8, T <= 64: routing inside that launch too (COLIBRI_DEC_ROUTE=0: not)
-  bool dec_flow = false;  // int8, T <= 64: completion counters instead of grid barriers (COLIBRI_DEC_FLOW=1)
 };
 
 namespace colibri {
@@ -351,22 +345,8 @@ struct DecFusedArgs {
   int32_t* counts = nullptr;                // [E]
   int32_t* offsets_out = nullptr;           // [E+1]
   int32_t* src_row = nullptr;               // [T*k]
-  // dataflow plan (dec_flow_kernel, T <= kFlowMaxT): completion counters instead of grid barriers
-  bool flow = false;
-  int32_t* unit_ctr = nullptr;              // [kFlowUnitCtrs], zero between launches
-  int32_t* tile_ctr = nullptr;              // [kFlowTileCtrs], zero between launches
-  // the H planes have buffers of their own in this plan: an H unit is written while gate/up
-  // items of other units may still read the x planes of the same rows
-  int8_t* hplanes_hi = nullptr;             // [flow_rows, f]
-  int8_t* hplanes_lo = nullptr;
-  float* hplanes_scale = nullptr;           // [dsplit, flow_rows]
-  int flow_rows = 0;                        // rows those buffers hold (R <= flow_rows)
 };
 constexpr int kFusedBarCount = 8;
-constexpr int kFlowMaxT = 64;
-// (token chunks of all experts) x (down splits) for T <= 64 tokens: chunks <= R / 8 + E
-constexpr int kFlowUnitCtrs = (kFlowMaxT * kMaxTopK / 8 + kMaxExperts) * kDecSplitMax;
-constexpr int kFlowTileCtrs = 65536 / 128;  // 128-column output tiles of d_model
 cudaError_t launch_dec_fused(const DecFusedArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------------------------------

@@ -158,7 +158,6 @@ struct DsCtl {
   int issued;    // copies issued / stages consumed, for the error path
   int consumed;
   int flag;      // result of a grid-wide wait, broadcast to the epilogue warps
-  int eflag;     // flow kernel: this CTA completed a unit / an output tile (epilogue warps)
   int hpass;     // fused kernel: 1 once the epilogue warps passed the H barrier, -1 if it failed
   int first;     // this CTA's first work item (items first, first + gridDim.x, ...)
   int ntouched;
@@ -170,9 +169,6 @@ struct DsCtl {
   int32_t defer_kx[kDsMaxStages][kDsMaxKbs];
   int32_t defer_nk[kDsMaxStages];
   int32_t defer_s[kDsMaxStages];
-  int32_t defer_unit[kDsMaxStages];  // flow kernel: the H unit whose planes a held stage waits for
-  int32_t defer_n[kDsMaxStages];     // and the stage's number (ring position) among all issued
-  int32_t defer_fresh[kDsMaxStages]; // 1: the first held stage of its item (counts as the item's use)
   float red[4];                     // fused kernel: per-warp maxima of the H pass
 };
 constexpr size_t kDsCtlBytes = 8192;
@@ -966,9 +962,6 @@ struct alignas(64) DecFusedParams {
   int8_t* xhi;              // [R, d] x planes written by the routing phase (the buffers p.gu reads)
   int8_t* xlo;
   float* xscale;            // [R] scales of the x planes (the buffer p.gu.rscale reads)
-  // dec_flow_kernel: completion counters, zero between launches (each launch returns them to 0)
-  int32_t* unit_ctr;        // [chunks x dsplit] H units: gate/up arrivals, then kUnitReady + uses
-  int32_t* tile_ctr;        // [ceil(d / 128)] output tiles: down arrivals
 };
 // up to this many tokens every CTA of the fused kernel routes all of them itself
 constexpr int kRedundantT = 1;
@@ -1486,289 +1479,6 @@ __global__ void __launch_bounds__(kDsThreads, 1) dec_fused_kernel(const __grid_c
   else __syncthreads();
 }
 
-// ------------------------------------------------------------------------- dataflow decode kernel
-// The same stage as dec_fused_kernel for up to 64 tokens, with the three grid barriers replaced by
-// completion counters, so that no CTA waits for the slowest one between phases:
-//   * An H unit is (token chunk of one expert, down split): the H columns of that split for the
-//     chunk's rows.  Every gate/up item adds one arrival to the unit its output tile falls in; the
-//     CTA whose arrival completes the count computes the unit (the rows' H planes and scales) in
-//     its epilogue warps and marks the unit ready.
-//   * A down item's weight copies go out at once; the copies of its H planes wait for its unit
-//     (held in the ring, in order, while other copies proceed), so a CTA moves on to its down
-//     items as soon as its gate/up items are done.
-//   * Every down item adds one arrival to its 128-column output tile; the CTA that completes the
-//     tile sums the tile's partials in fixed order (splits, then slots) and writes y.
-// The counters return to zero by the end of every launch: the CTA that completes a tile resets
-// it; an H unit counts its gate/up arrivals, is set to kUnitReady, counts one use per down item,
-// and the last use resets it.  Sums and orders are those of dec_fused_kernel, so results are
-// bit-identical to it.
-constexpr int32_t kUnitReady = 1 << 24;
-
-__device__ __forceinline__ int atom_add_acq_rel_gpu(int32_t* p, int v) {
-  int old;
-  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
-__device__ __forceinline__ int atom_add_relaxed_gpu(int32_t* p, int v) {
-  int old;
-  asm volatile("atom.relaxed.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
-__device__ __forceinline__ void st_release_gpu(int32_t* p, int v) {
-  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ void st_relaxed_gpu(int32_t* p, int v) {
-  asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Counts of the flow kernel, the same in every CTA.
-struct FlowCounts {
-  int tpu;     // gate/up output tiles per H unit
-  int need_g;  // gate/up arrivals that complete an H unit
-  int need_c;  // down items that use an H unit
-  int need_y;  // down arrivals that complete an output tile
-};
-__device__ __forceinline__ FlowCounts flow_counts(const DecFusedParams& p, const DsCtl& c) {
-  FlowCounts n;
-  const int span = p.gu.f / p.dn.nsplit;
-  n.tpu = (span + 127) / 128;
-  n.need_g = n.tpu * 2 * p.gu.nsplit;
-  n.need_c = (p.dn.d + 127) / 128;
-  n.need_y = c.cpre[c.ntouched] * p.dn.nsplit;
-  return n;
-}
-
-// Producer of the down phase: weight copies at once; the H-plane copies of a stage once its unit
-// is ready.  Stages whose unit is not ready yet are held in order (at most a ring-full): the
-// MMA consumes stages in order, so the oldest stage in flight is released (waiting for its unit)
-// before the producer waits for its ring slot.  The first stage of each item uses the unit once.
-__device__ bool flow_produce_down(const DecFusedParams& fp, uint8_t* smem, DsCtl& c, int S, DsRing& r) {
-  const DecStreamParams& p = fp.dn;
-  const FlowCounts nc = flow_counts(fp, c);
-  const uint32_t blk_bytes = 128u * 128u + (uint32_t)(2 * p.nt8) * 128u;
-  const uint64_t policy = l2_evict_first_policy();
-  int qh = 0, qn = 0;  // held stages: a queue of up to S entries in c.defer_*
-  auto ready = [&](int u) { return ld_acquire(fp.unit_ctr + u) >= kUnitReady; };
-  auto use = [&](int u) {  // after the unit was seen ready: make its planes visible to TMA, count the use
-    fence_proxy_async_global();
-    if (atom_add_relaxed_gpu(fp.unit_ctr + u, 1) == kUnitReady + nc.need_c - 1) st_relaxed_gpu(fp.unit_ctr + u, 0);
-  };
-  auto release_head = [&]() {
-    uint8_t* st = smem + (size_t)c.defer_s[qh] * p.stage_bytes;
-    for (int j = 0; j < c.defer_nk[qh]; ++j)
-      ds_load_planes(p, st, &c.full[c.defer_s[qh]], j, c.defer_kx[qh][j], c.defer_row[qh]);
-    qh = qh + 1 == S ? 0 : qh + 1;
-    --qn;
-  };
-  auto wait_unit = [&](int u) -> bool {
-    const unsigned long long t0 = global_ns();
-    while (!ready(u)) {
-      if (*(volatile int*)&c.abort || global_ns() - t0 > kWaitTimeoutNs) return false;
-      __nanosleep(32);
-    }
-    return true;
-  };
-  bool ok = true;
-  DecItem it;
-  for (int L = c.first; ok && dec_item<false>(p, c, 1, L, it); L += gridDim.x) {
-    const int u = it.gchunk * p.nsplit + it.split;
-    const int kbeg = it.split * p.kspan, kend = min(p.K, kbeg + p.kspan);
-    const int nkb = (kend - kbeg + 127) / 128;
-    int kb = L % nkb;
-    for (int i = 0; i < nkb; i += p.kbs) {
-      const bool fresh = i == 0;
-      // release held stages whose units are ready (in order; a later stage of an item whose first
-      // stage was released needs no check)
-      while (qn > 0 && (!c.defer_fresh[qh] || ready(c.defer_unit[qh]))) {
-        if (c.defer_fresh[qh]) use(c.defer_unit[qh]);
-        release_head();
-      }
-      // the stage in the slot about to be reused must have its planes on the way
-      while (ok && qn > 0 && c.defer_n[qh] <= r.n - S) {
-        if (c.defer_fresh[qh]) {
-          ok = wait_unit(c.defer_unit[qh]);
-          if (ok) use(c.defer_unit[qh]);
-        }
-        release_head();  // issued even when the wait gave up, so that every issued stage completes
-      }
-      if (!ok || !ds_wait(&c.empty[r.s], r.ph ^ 1u, &c.abort)) {
-        ok = false;
-        break;
-      }
-      const int nk = min(p.kbs, nkb - i);
-      uint8_t* st = smem + (size_t)r.s * p.stage_bytes;
-      mbar_arrive_expect_tx(&c.full[r.s], (uint32_t)nk * blk_bytes);
-      int kxs[kDsMaxKbs];
-      for (int j = 0; j < nk; ++j, kb = (kb + 1 == nkb) ? 0 : kb + 1) {
-        kxs[j] = kbeg + kb * 128;
-        uint8_t* sw = st + (size_t)j * 128 * 128;
-        if (p.evict_first) tma_load_3d_hint(sw, &p.mapW, &c.full[r.s], kxs[j], it.tile * 128, it.e, policy);
-        else tma_load_3d(sw, &p.mapW, &c.full[r.s], kxs[j], it.tile * 128, it.e);
-      }
-      // with nothing held, a later stage of an item goes out at once (its first stage was
-      // released, so the unit is ready), and a first stage if its unit is ready
-      const bool now = qn == 0 && (!fresh || ready(u));
-      if (now) {
-        if (fresh) use(u);
-        for (int j = 0; j < nk; ++j) ds_load_planes(p, st, &c.full[r.s], j, kxs[j], it.row0);
-      } else {
-        const int t = qh + qn < S ? qh + qn : qh + qn - S;
-        c.defer_s[t] = r.s;
-        c.defer_nk[t] = nk;
-        for (int j = 0; j < nk; ++j) c.defer_kx[t][j] = kxs[j];
-        c.defer_row[t] = it.row0;
-        c.defer_unit[t] = u;
-        c.defer_n[t] = r.n;
-        c.defer_fresh[t] = fresh ? 1 : 0;
-        ++qn;
-      }
-      c.issued = r.n + 1;
-      r.advance(S);
-    }
-  }
-  // the rest of the held stages (their copies are issued even after a failed wait)
-  while (qn > 0) {
-    if (c.defer_fresh[qh] && ok) {
-      ok = wait_unit(c.defer_unit[qh]);
-      if (ok) use(c.defer_unit[qh]);
-    }
-    release_head();
-  }
-  return ok;
-}
-
-// The combine of one 128-column output tile for every token, by the 128 epilogue threads:
-// y[t][o] = sum_j w[t][j] * (sum over splits of Ypart[split][dst_row[t][j]][o]), in the order of
-// dec_fused_kernel's combine.
-__device__ void flow_combine_tile(const DecFusedParams& p, int dt, int tid) {
-  const int d = p.dn.d, ns = p.dn.nsplit, k = p.k;
-  const int o = dt * 128 + tid;
-  if (o >= d) return;
-  const size_t ss = (size_t)p.dn.R * d;
-  for (int t = 0; t < p.T; ++t) {
-    float acc = 0.f;
-    for (int j = 0; j < k; ++j) {
-      const int rr = __ldcg(p.dst_row + (size_t)t * k + j);
-      const float wj = __ldcg(p.topk_w + (size_t)t * k + j);
-      const float* base = p.dn.Ypart + (size_t)rr * d + o;
-      float part = 0.f;
-      int sp = 0;
-      for (; sp + 8 <= ns; sp += 8) {
-        float v[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = __ldcg(base + (size_t)(sp + i) * ss);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) part += v[i];
-      }
-      for (; sp < ns; ++sp) part += __ldcg(base + (size_t)sp * ss);
-      acc = fmaf(wj, part, acc);
-    }
-    p.y[(size_t)t * d + o] = __float2bfloat16_rn(acc);
-  }
-}
-
-__global__ void __launch_bounds__(kDsThreads, 1) dec_flow_kernel(const __grid_constant__ DecFusedParams p) {
-  extern __shared__ __align__(1024) uint8_t smem[];
-  const int S = p.gu.stages;
-  DsCtl& c = *reinterpret_cast<DsCtl*>(smem + (size_t)S * p.gu.stage_bytes);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int G = gridDim.x;
-  const bool aligned = (smem_u32(smem) & 1023u) == 0;  // the 128-byte swizzle needs 1024-byte stages
-  const DecStreamParams* phases[2] = {&p.gu, &p.dn};
-  uint32_t planes_old = 0;  // thread 0: the planes barrier count before its arrival
-  if (aligned) {
-    ds_init(phases, 2, c, S);
-    if (p.route_in_kernel) {
-      fused_route(p, smem, c);
-      if (threadIdx.x == 0) c.first = (int)((blockIdx.x + gridDim.x - (unsigned)min(p.T, (int)gridDim.x)) % gridDim.x);
-      ds_items(phases, 2, c, nullptr);
-      if (threadIdx.x == 0) planes_old = bar_arrive(&p.bar[kBarPlanes], G);
-    } else {
-      ds_items(phases, 2, c, p.gu.offsets);
-    }
-  }
-  const uint32_t tmem = aligned ? c.tmem : 0u;
-  if (!aligned) {
-    if (threadIdx.x == 0) {  // report, and arrive at the barriers the others wait on
-      atomicOr(p.gu.err, kErrWaitTimeout);
-      if (p.route_in_kernel == 1 && p.T > kRedundantT) bar_arrive(&p.bar[kBarRouter], G);
-      if (p.route_in_kernel) bar_arrive(&p.bar[kBarPlanes], G);
-    }
-  } else if (warp == 0) {
-    if (lane == 0) {
-      DsRing r;
-      bool ok = ds_produce<true>(p.gu, smem, c, S, 0, r, p.route_in_kernel != 0, [&] {
-        if (!grid_wait(&p.bar[kBarPlanes], bar_base(planes_old, G), G, &c.abort)) return false;
-        fence_proxy_async_global();
-        return true;
-      });
-      if (ok) ok = flow_produce_down(p, smem, c, S, r);
-      if (!ok) ds_abort(c, p.gu.err);
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    if (lane == 0) {
-      DsRing r;
-      int iter = 0;
-      bool ok = ds_mma<true>(p.gu, smem, c, S, 0, r, iter, tmem);
-      if (ok) ok = ds_mma<false>(p.dn, smem, c, S, 1, r, iter, tmem);
-      if (!ok) ds_abort(c, p.gu.err);
-      tc_commit(&c.drain);
-      mbar_wait_bounded(&c.drain, 0);
-    }
-    __syncwarp();
-  } else {
-    const int tid = threadIdx.x - 64;  // 0..127
-    const FlowCounts nc = flow_counts(p, c);
-    int iter = 0;
-    // after a gate/up item: arrive on its H unit; the completing CTA computes the unit
-    // Both hooks decide in thread 0 and broadcast through shared memory, so the four warps take
-    // the same path (and pass the same named barriers): -1 once the CTA has aborted (a warp whose
-    // wait gave up sets the flag before its first barrier here), 1 if this CTA completed the
-    // counter, else 0.
-    // After a gate/up item: arrive on its H unit; the completing CTA computes the unit.
-    auto gu_done = [&](const DecItem& it, bool) -> bool {
-      const int sp = it.tile / nc.tpu;
-      const int u = it.gchunk * p.dn.nsplit + sp;
-      epi_sync();  // the four warps' partials of this item are written
-      if (tid == 0)
-        c.eflag = *(volatile int*)&c.abort ? -1 : (atom_add_acq_rel_gpu(p.unit_ctr + u, 1) == nc.need_g - 1 ? 1 : 0);
-      epi_sync();
-      const int v = *(volatile int*)&c.eflag;
-      if (v == 1) {
-        for (int r = it.row0; r < it.row0 + it.ntok; ++r) h_row_planes(p, c, r, sp, tid, lane);
-        fence_proxy_async_global();  // the planes are read next by TMA copies of other CTAs
-        epi_sync();
-        if (tid == 0) st_release_gpu(p.unit_ctr + u, kUnitReady);
-      }
-      return v >= 0;
-    };
-    // After a down item: arrive on its output tile; the completing CTA writes the tile of y.
-    auto dn_done = [&](const DecItem& it, bool) -> bool {
-      epi_sync();
-      if (tid == 0) {
-        c.eflag = *(volatile int*)&c.abort ? -1
-                                           : (atom_add_acq_rel_gpu(p.tile_ctr + it.tile, 1) == nc.need_y - 1 ? 1 : 0);
-        // the routing state the combine reads was written before every CTA's planes-barrier
-        // arrival: acquire the completed barrier directly
-        if (c.eflag == 1 && p.route_in_kernel) (void)ld_acquire(&p.bar[kBarPlanes]);
-      }
-      epi_sync();
-      const int v = *(volatile int*)&c.eflag;
-      if (v == 1) {
-        flow_combine_tile(p, it.tile, tid);
-        if (tid == 0) st_relaxed_gpu(p.tile_ctr + it.tile, 0);
-      }
-      return v >= 0;
-    };
-    bool ok = ds_epilogue<true>(p.gu, c, 0, iter, tmem, warp, lane, gu_done);
-    if (ok) ok = ds_epilogue<false>(p.dn, c, 1, iter, tmem, warp, lane, dn_done);
-    if (!__all_sync(0xffffffffu, ok) && lane == 0) ds_abort(c, p.gu.err);
-  }
-  if (aligned) ds_teardown(c, S);
-  else __syncthreads();
-}
-
 // K blocks per ring stage: COLIBRI_DEC_KB (1..4), default 2.
 int dec_kbs() {
   const char* v = getenv("COLIBRI_DEC_KB");
@@ -1815,7 +1525,6 @@ cudaError_t configure_dec_kernels() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(dec_stream_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(dec_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(dec_flow_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(dec_stream4_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess)
@@ -1995,13 +1704,10 @@ cudaError_t launch_dec_fused(const DecFusedArgs& a, cudaStream_t s) {
   DecFusedParams p;
   memset(&p, 0, sizeof(p));
   const int R = a.T * a.k;
-  // the dataflow plan writes H into planes of its own (the x planes may still be read meanwhile)
-  const bool flow = a.flow && a.unit_ctr && a.tile_ctr && a.hplanes_hi && a.hplanes_lo && a.hplanes_scale &&
-                    a.T <= kFlowMaxT && R <= a.flow_rows && a.dsplit <= kDecSplitMax &&
-                    (int64_t)(R / dec_nt8(a.T) + a.E) * a.dsplit <= kFlowUnitCtrs && (a.d + 127) / 128 <= kFlowTileCtrs;
-  int8_t* hhi = flow ? a.hplanes_hi : a.planes_hi;
-  int8_t* hlo = flow ? a.hplanes_lo : a.planes_lo;
-  float* hsc = flow ? a.hplanes_scale : a.planes_scale;
+  // H is split into planes in place of the x planes (the gate/up phase has finished reading them)
+  int8_t* hhi = a.planes_hi;
+  int8_t* hlo = a.planes_lo;
+  float* hsc = a.planes_scale;
   if (!dec_gateup_params(p.gu, a.planes_hi, a.planes_lo, a.planes_scale, a.W, a.scales, a.scale_mode, a.wstride, a.d,
                          a.f, a.E,
                          a.offsets, a.gsplit, a.GU, R, a.T, a.err) ||
@@ -2029,8 +1735,6 @@ cudaError_t launch_dec_fused(const DecFusedArgs& a, cudaStream_t s) {
   p.xhi = a.planes_hi;
   p.xlo = a.planes_lo;
   p.xscale = a.planes_scale;
-  p.unit_ctr = a.unit_ctr;
-  p.tile_ctr = a.tile_ctr;
   if (a.route_in_kernel && (a.T > 64 || !a.x || !a.topk_idx || !a.counts || !a.offsets_out || !a.src_row ||
                             (a.route_in_kernel == 1 && !a.router_w)))
     return cudaErrorInvalidValue;
@@ -2046,7 +1750,7 @@ cudaError_t launch_dec_fused(const DecFusedArgs& a, cudaStream_t s) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   launch_chain_break();  // an ordinary launch: the next one must not overlap it
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, flow ? dec_flow_kernel : dec_fused_kernel, p);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, dec_fused_kernel, p);
   launch_chain_break();
   return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -120,17 +120,14 @@ def test_int4_each_plan(name, plan, monkeypatch):
 I8_SMALL = [n for n, w in SMALL.items() if w.wdt == I8]
 
 
-@pytest.mark.parametrize("fused,route,flow", [("0", "0", "0"), ("1", "0", "0"), ("1", "1", "0"), ("1", "0", "1"),
-                                             ("1", "1", "1")])
+@pytest.mark.parametrize("fused,route", [("0", "0"), ("1", "0"), ("1", "1")])
 @pytest.mark.parametrize("name", I8_SMALL)
-def test_int8_each_launch_plan(name, fused, route, flow, monkeypatch):
+def test_int8_each_launch_plan(name, fused, route, monkeypatch):
     # fused "1": gate/up, H planes, down and combine in one cooperative launch (the default);
     # "0": the same stages as four launches.  route "1" (the default): for T <= 64 the router,
-    # top-k and grouping run inside that launch too.  flow "1" (opt-in, T <= 64): the launch's
-    # phases are linked by completion counters instead of grid barriers.
+    # top-k and grouping run inside that launch too.
     monkeypatch.setenv("COLIBRI_DEC_FUSED", fused)
     monkeypatch.setenv("COLIBRI_DEC_ROUTE", route)
-    monkeypatch.setenv("COLIBRI_DEC_FLOW", flow)
     wl = SMALL[name]
     p = inputgen.make_problem(wl, seed=9)
     layer = H.make_layer(wl)
@@ -142,18 +139,16 @@ def test_int8_each_launch_plan(name, fused, route, flow, monkeypatch):
 
 @pytest.mark.parametrize("name", ["i8_small", "i8_many", "i8_maxE", "i8_T1", "decode_int8_T1", "decode_int8_T8",
                                   "decode_int8_T32", "decode_int8_T8_outlier"])
-def test_int8_flow_matches_barrier_plan_bit_for_bit(name, monkeypatch):
-    # the counters change when each unit of work may start, never a sum or its order (the full
-    # decode sizes have H units much wider than their x rows, and many units per token chunk)
+def test_int8_fused_launch_is_deterministic(name, monkeypatch):
+    # every sum of the fused launch has a fixed order (split order for the gate/up and down
+    # partials, slot order in the combine) and the grid barriers only decide when a phase starts,
+    # so repeated calls, each with a fresh context, give the same bits
     if name.endswith("_outlier"):
         p = _outlier_problem(name[: -len("_outlier")], 23, "x")
     else:
         wl = VARIANT.get(name) or inputgen.WORKLOADS.get(name) or SMALL[name]
         p = inputgen.make_problem(wl, seed=23)
-    outs = []
-    for flow in ("0", "1", "1"):
-        monkeypatch.setenv("COLIBRI_DEC_FLOW", flow)
-        outs.append(H.run_gpu(p))
+    outs = [H.run_gpu(p) for _ in range(3)]
     for o in outs[1:]:
         for k in ("y", "idx", "w", "counts", "offsets", "src_row", "dst_row"):
             assert torch.equal(o[k], outs[0][k]), k
