@@ -137,7 +137,10 @@ int64_t colibri_expert_stride(const colibri_ctx* ctx);
  * colibri_moe_forward -- y = MoE(x) for T tokens.  (www.pptc.cn/news/100465 §4.1.)
  *
  *   x            [T, d_model] row-major, act_dtype.  Device memory, or host memory (pinned or
- *                pageable): host x is copied into the workspace on `stream` first.
+ *                pageable): host x is copied into one of two workspace staging buffers, on a
+ *                copy stream of the context, which `stream` then waits for.  That copy may start
+ *                before work enqueued earlier on `stream` has finished (it overlaps the previous
+ *                call's compute), so host x must hold its data when the call is made.
  *   T            0 <= T <= max_tokens.  T == 0 returns COLIBRI_OK and launches nothing.
  *   router_w     [E, d_model] row-major, act_dtype, device.
  *   router_b     [E] fp32 device, or NULL for no bias.
@@ -155,8 +158,10 @@ int64_t colibri_expert_stride(const colibri_ctx* ctx);
  *   shared_w     device, W1s[f_s][d] | W3s[f_s][d] | W2s[d][f_s] in weight_dtype, when
  *                shared_d_ff > 0; must be NULL otherwise.
  *   y            [T, d_model] act_dtype, device or host; fully overwritten.  Host y is written
- *                by a device-to-host copy enqueued on `stream`; it is valid once the stream
- *                has been synchronised.
+ *                by a device-to-host copy on a copy stream of the context that `stream` waits
+ *                for; it is valid once `stream` has been synchronised.  (With
+ *                COLIBRI_STAGED=0, or while `stream` is being captured into a graph, both copies
+ *                run on `stream` itself, through one staging pair.)
  *   stream       cudaStream_t.
  * Every device pointer must be 16-byte aligned.  Errors: INVALID_ARG, ALIGNMENT, CUDA.
  * A device-side wait that gives up is reported later by colibri_sync_status().

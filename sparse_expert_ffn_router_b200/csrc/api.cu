@@ -215,6 +215,7 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   ctx->nblk_max = nblk;
   Carver c;
   const size_t o_xs = c.take(M * d * as), o_ys = c.take(M * d * as);
+  const size_t o_xs2 = c.take(M * d * as), o_ys2 = c.take(M * d * as);  // second pair (staged calls alternate)
   const size_t o_idx = c.take(R * 4), o_w = c.take(R * 4), o_dst = c.take(R * 4), o_src = c.take(R * 4);
   const size_t o_bc = c.take((size_t)nblk * E * 4), o_bb = c.take((size_t)nblk * E * 4);
   const size_t o_cnt = c.take(E * 4), o_off = c.take((E + 1) * 4), o_mt = c.take((E + 1) * 4);
@@ -245,6 +246,8 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
   Workspace& w = ctx->ws;
   w.x_stage = b + o_xs;
   w.y_stage = b + o_ys;
+  w.x_stage2 = b + o_xs2;
+  w.y_stage2 = b + o_ys2;
   w.topk_idx = reinterpret_cast<int32_t*>(b + o_idx);
   w.topk_w = reinterpret_cast<float*>(b + o_w);
   w.dst_row = reinterpret_cast<int32_t*>(b + o_dst);
@@ -280,6 +283,15 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
       cudaGetLastError();
       e = nullptr;
     }
+  }
+  // copy streams and events of staged (host x / y) calls; without them such calls copy on the
+  // caller's stream
+  {
+    bool ok = cudaStreamCreateWithFlags(&ctx->cs_in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&ctx->cs_out, cudaStreamNonBlocking) == cudaSuccess;
+    for (auto& e : ctx->st_ev) ok = ok && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) cudaGetLastError();
+    ctx->staged = ok && !(getenv("COLIBRI_STAGED") && strcmp(getenv("COLIBRI_STAGED"), "0") == 0);
   }
   ctx->use_graphs = !(getenv("COLIBRI_GRAPHS") && strcmp(getenv("COLIBRI_GRAPHS"), "0") == 0);
   // COLIBRI_TILE_SCHED=static: the bf16 GEMMs walk their tiles round-robin instead of claiming them
@@ -320,6 +332,10 @@ void colibri_free(colibri_ctx* ctx) {
       cudaGraphExecDestroy(g.exec);
       if (g.graph) cudaGraphDestroy(g.graph);
     }
+    for (auto& e : ctx->st_ev)
+      if (e) cudaEventDestroy(e);
+    if (ctx->cs_in) cudaStreamDestroy(ctx->cs_in);
+    if (ctx->cs_out) cudaStreamDestroy(ctx->cs_out);
   }
   delete ctx;
 }
@@ -574,6 +590,64 @@ colibri_status enqueue_forward(colibri_ctx* ctx, const void* x, PtrKind xk, int3
   return COLIBRI_OK;
 }
 
+colibri_status forward_device(colibri_ctx* ctx, const void* x, PtrKind xk, int32_t T, const void* router_w,
+                              const float* router_b, const int32_t* user_idx, const float* user_w,
+                              const void* expert_w, const float* expert_scales, const void* shared_w, void* y,
+                              PtrKind yk, cudaStream_t s);
+
+bool stream_capturing(cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    return true;
+  }
+  return cs != cudaStreamCaptureStatusNone;
+}
+
+// Host x and/or y: the call alternates between two device staging pairs, and its copies run on
+// the context's two copy streams, ordered by events:
+//   cs_in:  waits until the forward two calls back has read this pair's x buffer, copies x in;
+//   stream: waits for that copy, runs the forward on device pointers (a replayed graph);
+//   cs_out: waits for the forward, copies y out; stream then waits for that copy.
+// So the next call's input copy overlaps this call's compute, host y is valid once `stream` has
+// been synchronised (as for the single-stream path), and every later use of a staging buffer on
+// `stream` comes after the copies that read it.
+colibri_status forward_staged(colibri_ctx* ctx, const void* x, PtrKind xk, int32_t T, const void* router_w,
+                              const float* router_b, const int32_t* user_idx, const float* user_w,
+                              const void* expert_w, const float* expert_scales, const void* shared_w, void* y,
+                              PtrKind yk, cudaStream_t s) {
+  const colibri_desc& D = ctx->desc;
+  Workspace& w = ctx->ws;
+  const size_t bytes = (size_t)T * D.d_model * (D.act_dtype == COLIBRI_F32 ? 4 : 2);
+  const int b = ctx->stage_next;
+  ctx->stage_next ^= 1;
+  cudaEvent_t* ev = ctx->st_ev + 4 * b;  // x buffer free, x copied in, forward done, y copied out
+  void* xs = b ? w.x_stage2 : w.x_stage;
+  void* ys = b ? w.y_stage2 : w.y_stage;
+  const void* xd = x;
+  void* yd = y;
+  if (xk == kPtrHost) {
+    COLIBRI_TRY(cudaStreamWaitEvent(ctx->cs_in, ev[0], 0), "staged: wait for the x buffer");
+    COLIBRI_TRY(cudaMemcpyAsync(xs, x, bytes, cudaMemcpyHostToDevice, ctx->cs_in), "staged: copy x to device");
+    COLIBRI_TRY(cudaEventRecord(ev[1], ctx->cs_in), "staged: record x copy");
+    COLIBRI_TRY(cudaStreamWaitEvent(s, ev[1], 0), "staged: wait for the x copy");
+    xd = xs;
+  }
+  if (yk == kPtrHost) yd = ys;
+  const colibri_status st = forward_device(ctx, xd, kPtrDevice, T, router_w, router_b, user_idx, user_w, expert_w,
+                                           expert_scales, shared_w, yd, kPtrDevice, s);
+  if (st != COLIBRI_OK) return st;
+  if (xk == kPtrHost) COLIBRI_TRY(cudaEventRecord(ev[0], s), "staged: record x buffer free");
+  if (yk == kPtrHost) {
+    COLIBRI_TRY(cudaEventRecord(ev[2], s), "staged: record forward done");
+    COLIBRI_TRY(cudaStreamWaitEvent(ctx->cs_out, ev[2], 0), "staged: wait for the forward");
+    COLIBRI_TRY(cudaMemcpyAsync(y, ys, bytes, cudaMemcpyDeviceToHost, ctx->cs_out), "staged: copy y to host");
+    COLIBRI_TRY(cudaEventRecord(ev[3], ctx->cs_out), "staged: record y copy");
+    COLIBRI_TRY(cudaStreamWaitEvent(s, ev[3], 0), "staged: wait for the y copy");
+  }
+  return COLIBRI_OK;
+}
+
 // Shared body of both forward entry points.  topk_idx/topk_w non-NULL = caller routing.
 colibri_status forward_impl(colibri_ctx* ctx, const void* x, int32_t T, const void* router_w,
                             const float* router_b, const int32_t* user_idx, const float* user_w,
@@ -611,6 +685,19 @@ colibri_status forward_impl(colibri_ctx* ctx, const void* x, int32_t T, const vo
   const PtrKind xk = classify(x, dev), yk = classify(y, dev);
   if (xk == kPtrBad || yk == kPtrBad)
     return fail(ctx, COLIBRI_ERR_INVALID_ARG, "x or y is device memory of another device");
+  if ((xk == kPtrHost || yk == kPtrHost) && ctx->staged && !ctx->profile && !stream_capturing(s))
+    return forward_staged(ctx, x, xk, T, router_w, router_b, user_idx, user_w, expert_w, expert_scales, shared_w, y,
+                          yk, s);
+  return forward_device(ctx, x, xk, T, router_w, router_b, user_idx, user_w, expert_w, expert_scales, shared_w, y,
+                        yk, s);
+}
+
+// The forward once x and y are classified: a replayed graph when possible, else the launches.
+colibri_status forward_device(colibri_ctx* ctx, const void* x, PtrKind xk, int32_t T, const void* router_w,
+                              const float* router_b, const int32_t* user_idx, const float* user_w,
+                              const void* expert_w, const float* expert_scales, const void* shared_w, void* y,
+                              PtrKind yk, cudaStream_t s) {
+  const colibri_desc& D = ctx->desc;
   // bf16 weights: the tiling of the expert GEMMs (see gemm_mode)
   const int gemm = D.weight_dtype == COLIBRI_BF16 ? gemm_mode(T * D.top_k / D.num_experts) : kGemmOne;
 

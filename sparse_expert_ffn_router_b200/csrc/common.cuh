@@ -59,6 +59,8 @@ constexpr unsigned long long kWaitTimeoutNs = 4000000000ull;
 struct Workspace {
   void* x_stage = nullptr;  // [M, d] act, for host x
   void* y_stage = nullptr;  // [M, d] act, for host y
+  void* x_stage2 = nullptr;  // the second pair: staged calls alternate between the two
+  void* y_stage2 = nullptr;
   int32_t* topk_idx = nullptr;  // [M, k]
   float* topk_w = nullptr;      // [M, k]
   int32_t* dst_row = nullptr;   // [M, k]
@@ -121,6 +123,12 @@ struct colibri_ctx {
   bool use_pdl = false;  // programmatic dependent launch between the kernels of a forward (opt-in)
   bool dec_fused = true;  // int8 weights: the one-launch expert stage (COLIBRI_DEC_FUSED=0: four launches)
   bool dec_route = true;  // int8, T <= 64: routing inside that launch too (COLIBRI_DEC_ROUTE=0: not)
+  // staged calls (host x or y): copy streams, events [2 staging pairs][x free, x in, forward done,
+  // y out], and the pair the next call takes (COLIBRI_STAGED=0: copies on the caller's stream)
+  bool staged = true;
+  cudaStream_t cs_in = nullptr, cs_out = nullptr;
+  cudaEvent_t st_ev[8] = {nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+  int stage_next = 0;
 };
 
 namespace colibri {

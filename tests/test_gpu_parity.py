@@ -197,6 +197,35 @@ def test_T_above_max_tokens_is_rejected():
     layer.close()
 
 
+@pytest.mark.parametrize("kinds", [("host", "host"), ("host", "dev"), ("dev", "host")])
+def test_staged_host_calls_back_to_back(kinds):
+    # Host x / y go through two alternating device staging pairs, copied on the context's own
+    # streams: six calls with different inputs, enqueued without any synchronisation in between
+    # on a non-default stream, must each give the device run's bits once the stream is synchronised
+    wl = SMALL["bf16_shared"]
+    layer = H.make_layer(wl)
+    stream = torch.cuda.Stream()
+    probs = [inputgen.make_problem(wl, seed=40 + i) for i in range(3)]
+    t = H.to_device(probs[0])
+    refs = []
+    for pr in probs:
+        y_ref = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device="cuda")
+        layer.forward(pr.x.cuda(), t["router_w"], t["router_b"], t["expert_w"], y_ref, shared_w=t["shared_w"])
+        refs.append(y_ref)
+    torch.cuda.synchronize()
+    xs = [pr.x.pin_memory() if kinds[0] == "host" else pr.x.cuda() for pr in probs]
+    ys = [torch.empty(wl.T, wl.d, dtype=torch.bfloat16).pin_memory() if kinds[1] == "host"
+          else torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device="cuda") for _ in range(6)]
+    for i in range(6):
+        layer.forward(xs[i % 3], t["router_w"], t["router_b"], t["expert_w"], ys[i], shared_w=t["shared_w"],
+                      stream=stream)
+    stream.synchronize()
+    layer.sync_status()
+    for i in range(6):
+        assert torch.equal(ys[i].cpu(), refs[i % 3].cpu()), i
+    layer.close()
+
+
 def test_misaligned_and_host_weight_pointers_are_rejected():
     wl = SMALL["bf16_T1"]
     layer = H.make_layer(wl)
