@@ -97,7 +97,6 @@ __global__ void __launch_bounds__(kG4Threads, 1) gemv4_kernel(const __grid_const
   const int ngroups = p.out_rows / kG4Rows;
   const int per_e = p.mats * p.nsplit * ngroups;
   const int tasks = n_touched * per_e;
-  const int ngr = p.kspan / 128;  // K groups of a split: lane l takes l, l + 32, ...
   const size_t mat_bytes = (size_t)p.d * p.f / 2;
   const size_t scales_per_mat = (size_t)p.d * p.f / 128;
   const size_t row_bytes = (size_t)p.K / 2;
