@@ -284,15 +284,6 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
       e = nullptr;
     }
   }
-  // copy streams and events of staged (host x / y) calls; without them such calls copy on the
-  // caller's stream
-  {
-    bool ok = cudaStreamCreateWithFlags(&ctx->cs_in, cudaStreamNonBlocking) == cudaSuccess &&
-              cudaStreamCreateWithFlags(&ctx->cs_out, cudaStreamNonBlocking) == cudaSuccess;
-    for (auto& e : ctx->st_ev) ok = ok && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
-    if (!ok) cudaGetLastError();
-    ctx->staged = ok && !(getenv("COLIBRI_STAGED") && strcmp(getenv("COLIBRI_STAGED"), "0") == 0);
-  }
   ctx->use_graphs = !(getenv("COLIBRI_GRAPHS") && strcmp(getenv("COLIBRI_GRAPHS"), "0") == 0);
   // COLIBRI_TILE_SCHED=static: the bf16 GEMMs walk their tiles round-robin instead of claiming them
   ctx->tile_static = getenv("COLIBRI_TILE_SCHED") && strcmp(getenv("COLIBRI_TILE_SCHED"), "static") == 0;
@@ -312,6 +303,15 @@ colibri_status colibri_init(const colibri_desc* desc, colibri_ctx** out) {
     cudaFree(ctx->ws_base);
     delete ctx;
     return fail(nullptr, COLIBRI_ERR_CUDA, "kernel configuration failed: %s", cudaGetErrorString(ce));
+  }
+  // copy streams and events of staged (host x / y) calls; without them such calls copy on the
+  // caller's stream
+  {
+    bool ok = cudaStreamCreateWithFlags(&ctx->cs_in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&ctx->cs_out, cudaStreamNonBlocking) == cudaSuccess;
+    for (auto& e : ctx->st_ev) ok = ok && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) cudaGetLastError();
+    ctx->staged = ok && !(getenv("COLIBRI_STAGED") && strcmp(getenv("COLIBRI_STAGED"), "0") == 0);
   }
   *out = ctx;
   return COLIBRI_OK;
